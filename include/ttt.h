@@ -1,0 +1,217 @@
+/*
+ * ttt.h - C ABI of the B200 (sm_100a) library for the chunked TTT-KVB fast-weight layer
+ * and its rewrite as chunked linear attention.
+ *
+ * The layer (per batch element and head, row vectors; "Test-Time Training with KV Binding
+ * Is Secretly Linear Attention", section 前置知识 / LaCT, and "Test-Time Training Done
+ * Right" notes, section 2.1):
+ *     phi(x) = silu(x W0) * (x W2),   f(x) = phi(x) W1,
+ *     W0, W2 in R^{h x m}, W1 in R^{m x h}, m = r h,
+ *     chunk loss  L_c = - sum_{i in chunk c} eta_i <f(k_i), v_i>.
+ * Each chunk takes one gradient step (step size 1, eta inside the loss) from the
+ * chunk-start weights; the chunk's queries then read f(q) with the updated weights
+ * (TTT_ORDER_UPDATE_APPLY) or with the chunk-start weights (TTT_ORDER_APPLY_UPDATE,
+ * "Test-Time Training Done Right" notes, section 2.3).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers are DEVICE pointers unless stated otherwise. Tensors are dense, row-major,
+ * contiguous:
+ *     q, k, v, out : [B, H, N, h]  element type ttt_desc.dtype (fp32 or bf16)
+ *     eta          : [B, H, N]     fp32 per-token learning rate
+ *     alpha        : [B, H, C]     fp32 per-chunk momentum factor, C = ceil(N / chunk)
+ *     W0, W2       : [H, h, m]     fp32 (or [H, m, h] when w_in_layout = 1)
+ *     W1           : [H, m, h]     fp32 (or [H, h, m] when w1_layout = 1)
+ * Initial weights are per head and broadcast over the batch; every (batch, head) starts
+ * from them (fast weights are reset per sequence). The last chunk may be shorter than
+ * `chunk`. q == k (same pointer) is allowed: the query and key features are then
+ * computed once.
+ *
+ * Ownership: the caller owns every buffer. The library allocates no device memory; the
+ * scratch it needs lives in the caller's workspace (size from ttt_workspace_bytes). Work
+ * is enqueued on the caller's stream and returns before it completes.
+ *
+ * Errors: arguments are checked on the host before anything is enqueued; a failed check
+ * returns a status and enqueues nothing (no exceptions cross the ABI). A bounded wait
+ * that runs out inside a kernel, or a device-side check that fails, is recorded in a
+ * per-device error word; ttt_last_device_status() synchronises the stream, reads and
+ * clears it. ttt_last_error_message() gives a human-readable detail of the calling
+ * thread's last failure.
+ *
+ * Precision: in TTT_DTYPE_BF16 mode the dense contractions take bf16 operands (q, k, v,
+ * the fp32 weights rounded to bf16, the features rounded to bf16) and accumulate in
+ * fp32 on the tensor cores; states, weights, momentum and all elementwise math stay
+ * fp32. In TTT_DTYPE_FP32 mode every step is fp32 on the CUDA cores.
+ */
+#ifndef TTT_B200_TTT_H_
+#define TTT_B200_TTT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t. NULL selects the legacy default stream. */
+typedef struct CUstream_st* ttt_stream_t;
+
+typedef enum ttt_status {
+  TTT_OK = 0,
+  TTT_ERR_INVALID_ARG = 1,  /* a size, flag or pointer is invalid (see the message) */
+  TTT_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+  TTT_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or smaller than required */
+  TTT_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  TTT_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out */
+  TTT_ERR_DEVICE = 6        /* a device-side bounds/alignment check failed */
+} ttt_status;
+
+enum { TTT_DTYPE_FP32 = 0, TTT_DTYPE_BF16 = 1 };
+enum { TTT_ORDER_UPDATE_APPLY = 0, TTT_ORDER_APPLY_UPDATE = 1 };
+enum { TTT_UPDATE_W0 = 1, TTT_UPDATE_W1 = 2, TTT_UPDATE_W2 = 4, TTT_UPDATE_ALL = 7 };
+enum { TTT_PATH_PARALLEL = 0, TTT_PATH_RECURRENT = 1 };
+
+/* Problem description. All fields are read; unused ones must be 0 unless noted. */
+typedef struct ttt_desc {
+  int32_t B;            /* batch size, >= 0 */
+  int32_t H;            /* heads, >= 0 */
+  int32_t N;            /* tokens per sequence, >= 0 */
+  int32_t h;            /* head (input/output) width, >= 1 */
+  int32_t m;            /* hidden width of the SwiGLU map, >= 1 */
+  int32_t chunk;        /* tokens per update chunk, >= 1 */
+  int32_t dtype;        /* TTT_DTYPE_FP32 or TTT_DTYPE_BF16 (q, k, v and out) */
+  int32_t order;        /* TTT_ORDER_UPDATE_APPLY or TTT_ORDER_APPLY_UPDATE */
+  int32_t sign;         /* +1 gradient descent, -1 gradient ascent */
+  int32_t update_mask;  /* recurrent: which of W0/W1/W2 are fast (TTT_UPDATE_*) */
+  int32_t renorm;       /* recurrent: 1 = per-column weight renormalisation */
+  int32_t momentum;     /* recurrent: 1 = momentum M <- alpha_c M + g (needs alpha) */
+  int32_t ns_steps;     /* recurrent: Newton-Schulz steps on each update, 0..8 */
+  int32_t w_in_layout;  /* 0: W0, W2 are [H,h,m]; 1: they are [H,m,h] (e.g. gate/up) */
+  int32_t w1_layout;    /* 0: W1 and S_final are [.,m,h]; 1: [.,h,m] (e.g. down proj) */
+} ttt_desc;
+
+/*
+ * Workspace size in bytes for `path` (TTT_PATH_PARALLEL or TTT_PATH_RECURRENT), or 0
+ * when the description is invalid for that path. Host-only; touches no device.
+ */
+size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path);
+
+/*
+ * Parallel last-layer-only form ("Test-Time Training with KV Binding Is Secretly Linear
+ * Attention", sections 方法步骤详情 (Theorem 5.2 and simplification steps 1-2) and
+ * 前置知识 / 前缀扫描; "NVIDIA团队揭秘", section 四): W0, W2 frozen, no renormalisation,
+ * so the features are static and the W1 updates are associative:
+ *     Delta S_c = sign * phi(K_c)^T diag(eta_c) V_c,
+ *     S_c = W1 + sum_{c' <= c} Delta S_c'   (update_apply; c' < c for apply_update),
+ *     O_c = phi(Q_c) S_c.
+ * With q == k, W0 = Wg^T, W2 = Wu^T, W1 = W_down^T, v = the target values and
+ * apply_update this is the In-Place TTT chunk update ("In-Place Test-Time Training",
+ * sections 3.1 and 3.4).
+ *
+ *   desc       problem; update_mask, renorm, momentum, ns_steps must be 0
+ *   q, k, v    [B,H,N,h] dtype
+ *   eta        [B,H,N] fp32
+ *   W0, W2     per-head input-side weights (layout per w_in_layout), fp32
+ *   W1         per-head initial state (layout per w1_layout), fp32
+ *   out        [B,H,N,h] dtype, written
+ *   S_final    nullable; [B,H,m,h] (or [B,H,h,m]) fp32 state after the last chunk
+ *   workspace  >= ttt_workspace_bytes(desc, TTT_PATH_PARALLEL) bytes, 256-byte aligned
+ */
+ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* k,
+                               const void* v, const float* eta, const float* W0,
+                               const float* W2, const float* W1, void* out,
+                               float* S_final, void* workspace, size_t workspace_bytes,
+                               ttt_stream_t stream);
+
+/*
+ * Recurrent LaCT form ("Test-Time Training Done Right" notes, sections 2.1-2.3; "Test-Time
+ * Training with KV Binding Is Secretly Linear Attention", 前置知识 / LaCT): per chunk, at
+ * the chunk-start weights, the gradients
+ *     G = -diag(eta) V,  dW1 = phi^T G,  D = G W1^T,
+ *     dW2 = K^T (D * silu(K W0)),  dW0 = K^T (D * (K W2) * silu'(K W0));
+ * then for every fast matrix X (update_mask): optional momentum M_X <- alpha_c M_X + g_X
+ * (M = 0 at the start), optional Newton-Schulz orthogonalisation of the update
+ * (X = U / (||U||_F + 1e-7) in the orientation with rows <= cols, then ns_steps times
+ * X <- 3.4445 X + (-4.7750 A + 2.0315 A^2) X with A = X X^T), the step
+ * X <- X - sign * u, and optional renormalisation of each column (output unit) over the
+ * input dimension to the column norm the matrix had at the start of the call.
+ *
+ *   desc       problem; w_in_layout and w1_layout must be 0
+ *   alpha      [B,H,C] fp32, required when desc->momentum, else ignored (may be NULL)
+ *   W0, W2, W1 per-head initial weights [H,h,m], [H,h,m], [H,m,h] fp32
+ *   out        [B,H,N,h] dtype, written
+ *   W0_out, W2_out  nullable; [B,H,h,m] fp32 weights after the last chunk
+ *   W1_out     nullable; [B,H,m,h] fp32
+ *   M_io       nullable; [B,H,(h*m + m*h + h*m)] fp32 momentum (W0 part [h,m], then W1
+ *              part [m,h], then W2 part [h,m]); read as the initial momentum and
+ *              overwritten with the final one. NULL means "start from 0, discard".
+ *   workspace  >= ttt_workspace_bytes(desc, TTT_PATH_RECURRENT) bytes, 256-byte aligned
+ */
+ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const void* k,
+                                  const void* v, const float* eta, const float* alpha,
+                                  const float* W0, const float* W2, const float* W1,
+                                  void* out, float* W0_out, float* W2_out, float* W1_out,
+                                  float* M_io, void* workspace, size_t workspace_bytes,
+                                  ttt_stream_t stream);
+
+/*
+ * LM-aligned value target ("In-Place Test-Time Training", section 3.2, eq. 3):
+ *     Vbar = Conv1D(X0) W_target,  (Conv1D(X0))_t = sum_{j=0..3} conv_w[j] * X0[t-j]
+ * (causal, depthwise, zero before the first token).
+ *
+ *   X0        [N,d] bf16 token embeddings
+ *   conv_w    [4,d] fp32 taps (tap j multiplies X0[t-j])
+ *   W_target  [d,d] bf16
+ *   vbar      [N,d] bf16, written
+ *   workspace >= ttt_lm_target_workspace_bytes(N, d) bytes, 256-byte aligned
+ */
+size_t ttt_lm_target_workspace_bytes(int32_t N, int32_t d);
+ttt_status ttt_lm_target(int32_t N, int32_t d, const void* X0, const float* conv_w,
+                         const void* W_target, void* vbar, void* workspace,
+                         size_t workspace_bytes, ttt_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the current
+ * device: TTT_OK, TTT_ERR_TIMEOUT (a bounded wait ran out) or TTT_ERR_DEVICE; or
+ * TTT_ERR_CUDA when the synchronisation itself failed.
+ */
+ttt_status ttt_last_device_status(ttt_stream_t stream);
+
+/*
+ * Diagnostic for the failure path: launches one block that waits on a barrier nobody
+ * arrives at, giving up after `timeout_ns` nanoseconds (1e5 .. 1e10). The wait records
+ * TTT_ERR_TIMEOUT in the device error word and the kernel returns normally, so the
+ * context stays usable. No paper counterpart: it exercises the library's own bounded
+ * waits.
+ */
+ttt_status ttt_debug_wait_timeout(int64_t timeout_ns, ttt_stream_t stream);
+
+/*
+ * Kernel tracing (no paper counterpart; the library's own profiling hook). After
+ * ttt_trace_enable(capacity), every kernel the library enqueues, on the current device, is
+ * bracketed by two CUDA events recorded on the stream it is launched on, until
+ * `capacity` kernels have been recorded. The events are created here (host-side CUDA
+ * objects, no device memory). ttt_trace_count() gives the number recorded;
+ * ttt_trace_get(i, ...) waits for record i to complete and returns a static kernel name
+ * and its duration in milliseconds. ttt_trace_disable() stops recording and releases the
+ * events. Tracing is process-wide and not meant for concurrent callers.
+ */
+ttt_status ttt_trace_enable(int32_t capacity);
+ttt_status ttt_trace_disable(void);
+int32_t ttt_trace_count(void);
+ttt_status ttt_trace_get(int32_t index, const char** kernel_name, float* milliseconds);
+
+/* Static, never NULL. */
+const char* ttt_status_str(ttt_status status);
+
+/* Detail of the calling thread's last non-OK status ("" if none). Static storage. */
+const char* ttt_last_error_message(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t ttt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_B200_TTT_H_ */

@@ -1,0 +1,59 @@
+// Batched GEMM problem shared by the host orchestration and the two GEMM engines
+// (tcgen05/TMA tensor-core engine for bf16 operands, CUDA-core engine for fp32).
+//
+//   C[z](i, j) = alpha * sum_k A[z](i, k) * B[z](j, k) + beta * Cin[z](i, j)
+//
+// for i < M, j < N, z = (z0, z1) in [0, Z0) x [0, Z1). Operand X in {A, B} with row index
+// r (i for A, j for B) and reduction index k sits at
+//   X.ptr + z0 * X.s0 + z1 * X.s1 + (mn_major ? k * X.ld + r : r * X.ld + k)   (elements).
+// A batch stride of 0 broadcasts the operand over that batch index.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace ttt {
+
+struct GemmOperand {
+  const void* ptr = nullptr;
+  int dtype = DT_F32;
+  bool mn_major = false;  // false: k contiguous ("K-major"); true: the row index contiguous
+  long long ld = 0, s0 = 0, s1 = 0;
+};
+
+struct GemmOut {
+  void* ptr = nullptr;
+  int dtype = DT_F32;
+  long long ld = 0, s0 = 0, s1 = 0;
+};
+
+struct GemmCin {
+  const float* ptr = nullptr;  // fp32 addend, may alias C.ptr (same layout)
+  long long ld = 0, s0 = 0, s1 = 0;
+};
+
+struct GemmProblem {
+  int M = 0, N = 0, K = 0, Z0 = 1, Z1 = 1;
+  GemmOperand A, B;
+  GemmOut C;
+  float alpha = 1.0f;
+  float beta = 0.0f;
+  GemmCin Cin;
+};
+
+// CUDA-core engine: any strides, fp32 or bf16 operands, fp32 accumulation.
+ttt_status gemm_simt(const GemmProblem& p, cudaStream_t stream);
+
+// Tensor-core engine (tcgen05.mma kind::f16, TMEM accumulators, TMA operand loads).
+// Requires bf16 A and B with 16-byte aligned bases and strides; see umma_supported.
+bool umma_supported(const GemmProblem& p);
+ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,
+                     unsigned long long wait_ns);
+
+// Error-word access (ttt_api.cu).
+unsigned* device_error_word();
+unsigned long long wait_limit_ns();
+void set_error_message(const char* fmt, ...);
+
+}  // namespace ttt

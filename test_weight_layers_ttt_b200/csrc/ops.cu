@@ -1,0 +1,431 @@
+// Non-GEMM kernels of the TTT layer: weight preparation, the SwiGLU feature map and its
+// gradient pieces, the chunk prefix scan over fp32 states, the recurrent update operators
+// (momentum, Newton-Schulz set-up, step, per-column renormalisation), the causal Conv1D of
+// the In-Place target, and the bounded-wait diagnostic.
+#include "ops.h"
+#include "umma.cuh"
+
+namespace ttt {
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+template <typename OT>
+__device__ __forceinline__ void st(void* base, long long i, float v) {
+  static_cast<OT*>(base)[i] = from_f32<OT>(v);
+}
+
+__device__ __forceinline__ float eta_of(const EtaMap& em, long long r) {
+  const long long z = r / em.T, t = r - z * em.T;
+  return em.eta[z * em.eta_ld + em.eta_off + t];
+}
+
+// ------------------------------------------------------------------ weight preparation
+template <typename OT>
+__global__ void prep_wk_kernel(const float* W0, const float* W2, OT* Wk, int n_entries,
+                               int src_heads, int h, int m, int layout) {
+  const long long per = 2LL * m * h;
+  TTT_GRID_LOOP(idx, per * n_entries) {
+    const long long e = idx / per, rem = idx - e * per;
+    const int j = (int)(rem / h), i = (int)(rem - (long long)j * h);
+    const float* src = (j < m ? W0 : W2) + (e % src_heads) * (long long)h * m;
+    const int jj = j < m ? j : j - m;
+    const float v = layout == 0 ? src[(long long)i * m + jj] : src[(long long)jj * h + i];
+    Wk[idx] = from_f32<OT>(v);
+  }
+}
+
+// ------------------------------------------------------------------ features
+template <typename OT>
+__global__ void swiglu_kernel(const float* AB, long long rows, int m, EtaMap em, OT* phi_eta,
+                              OT* phi_plain) {
+  TTT_GRID_LOOP(idx, rows * m) {
+    const long long r = idx / m;
+    const int j = (int)(idx - r * m);
+    const float a = AB[r * 2 * m + j], b = AB[r * 2 * m + m + j];
+    const float p = siluf_(a) * b;
+    if (phi_plain) phi_plain[idx] = from_f32<OT>(p);
+    if (phi_eta) phi_eta[idx] = from_f32<OT>(p * eta_of(em, r));
+  }
+}
+
+template <typename OT>
+__global__ void grad_prep_kernel(const float* AB, const float* Dv, long long rows, int m,
+                                 EtaMap em, OT* P, OT* E2, OT* E0) {
+  TTT_GRID_LOOP(idx, rows * m) {
+    const long long r = idx / m;
+    const int j = (int)(idx - r * m);
+    const float a = AB[r * 2 * m + j], b = AB[r * 2 * m + m + j];
+    const float eta = eta_of(em, r);
+    const float sa = siluf_(a);
+    P[idx] = from_f32<OT>(sa * b * eta);
+    if (E2 || E0) {
+      const float d = -eta * Dv[idx];
+      if (E2) E2[idx] = from_f32<OT>(d * sa);
+      if (E0) E0[idx] = from_f32<OT>(d * b * silu_primef_(a));
+    }
+  }
+}
+
+// ------------------------------------------------------------------ chunk prefix scan
+// One thread per state element; the chunk axis (tens of chunks) is walked sequentially so
+// every delta is read once and every chunk state written once.
+template <typename OT>
+__global__ void chunk_scan_kernel(const float* dS, const float* W1, OT* Sc, float* S_final,
+                                  int BH, int H, int C, int m, int h, int order, int layout) {
+  const long long per = (long long)m * h;
+  TTT_GRID_LOOP(idx, per * BH) {
+    const long long bh = idx / per, e = idx - bh * per;
+    const int k = (int)(e / h), j = (int)(e - (long long)k * h);
+    const long long w_off = (bh % H) * per + (layout == 0 ? e : (long long)j * m + k);
+    float s = W1[w_off];
+    const float* d = dS + bh * C * per + e;
+    OT* out = Sc + bh * C * per + e;
+    for (int c = 0; c < C; ++c) {
+      const float dv = d[(long long)c * per];
+      if (order == 1) {
+        out[(long long)c * per] = from_f32<OT>(s);
+        s += dv;
+      } else {
+        s += dv;
+        out[(long long)c * per] = from_f32<OT>(s);
+      }
+    }
+    if (S_final) S_final[bh * per + (layout == 0 ? e : (long long)j * m + k)] = s;
+  }
+}
+
+// ------------------------------------------------------------------ recurrent state
+// Part p of a (b, head) state: p = 0 W0 [h, m], p = 1 W1 [m, h], p = 2 W2 [h, m].
+__device__ __forceinline__ void part_dims(int p, int h, int m, int& R, int& Cc) {
+  if (p == 1) { R = m; Cc = h; } else { R = h; Cc = m; }
+}
+
+template <typename OT>
+__global__ void rec_init_kernel(const float* W0, const float* W2, const float* W1, int BH, int H,
+                                int h, int m, float* W_all, OT* W1o, const float* M_in,
+                                float* M_all, int momentum) {
+  const long long hm = (long long)h * m, per = 3 * hm;
+  TTT_GRID_LOOP(idx, per * BH) {
+    const long long bh = idx / per, e = idx - bh * per;
+    const int p = (int)(e / hm);
+    const long long o = e - p * hm;
+    const long long hd = bh % H;
+    const float v = p == 0 ? W0[hd * hm + o] : p == 1 ? W1[hd * hm + o] : W2[hd * hm + o];
+    W_all[idx] = v;
+    if (p == 1) W1o[bh * hm + o] = from_f32<OT>(v);
+    if (momentum) M_all[idx] = M_in ? M_in[idx] : 0.0f;
+  }
+}
+
+// Column norms (over the input dimension) of the initial weights, per head:
+// tnorm[head] = [ W0 columns (m) | W1 columns (h) | W2 columns (m) ].
+__global__ void col_norms_kernel(const float* W0, const float* W2, const float* W1, int H, int h,
+                                 int m, float* tnorm) {
+  const int per = 2 * m + h;
+  TTT_GRID_LOOP(idx, (long long)per * H) {
+    const int hd = (int)(idx / per), c = (int)(idx - (long long)hd * per);
+    const long long hm = (long long)h * m;
+    double ss = 0.0;
+    if (c < m) {
+      for (int r = 0; r < h; ++r) { const float w = W0[hd * hm + (long long)r * m + c]; ss += (double)w * w; }
+    } else if (c < m + h) {
+      const int cc = c - m;
+      for (int r = 0; r < m; ++r) { const float w = W1[hd * hm + (long long)r * h + cc]; ss += (double)w * w; }
+    } else {
+      const int cc = c - m - h;
+      for (int r = 0; r < h; ++r) { const float w = W2[hd * hm + (long long)r * m + cc]; ss += (double)w * w; }
+    }
+    tnorm[idx] = (float)sqrt(ss);
+  }
+}
+
+__global__ void rec_reduce_kernel(const float* partials, int splits, float* U, float* M_all,
+                                  const float* alpha, int C, int c, int BH, int h, int m,
+                                  int mask) {
+  const long long hm = (long long)h * m, per = 3 * hm, total = per * BH;
+  TTT_GRID_LOOP(idx, total) {
+    const long long bh = idx / per;
+    const int p = (int)((idx - bh * per) / hm);
+    if (!(mask & (1 << p))) continue;
+    float g = 0.0f;
+    for (int s = 0; s < splits; ++s) g += partials[(long long)s * total + idx];
+    if (M_all) {
+      const float mv = alpha[bh * C + c] * M_all[idx] + g;
+      M_all[idx] = mv;
+      g = mv;
+    }
+    U[idx] = g;
+  }
+}
+
+// One block per (part, bh): Frobenius norm, then the normalised update in the orientation
+// with rows <= cols.
+__global__ void ns_normalize_kernel(const float* U, float* X, int h, int m, int mask, float eps) {
+  const int p = blockIdx.x, bh = blockIdx.y;
+  if (!(mask & (1 << p))) return;
+  int R, Cc;
+  part_dims(p, h, m, R, Cc);
+  const long long hm = (long long)h * m;
+  const float* u = U + (long long)bh * 3 * hm + p * hm;
+  float* x = X + ((long long)bh * 3 + p) * hm;
+  __shared__ float red[32];
+  float ss = 0.0f;
+  for (long long e = threadIdx.x; e < hm; e += blockDim.x) ss += u[e] * u[e];
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float scale = 1.0f / (sqrtf(red[0]) + eps);
+  const bool tr = R > Cc;
+  for (long long e = threadIdx.x; e < hm; e += blockDim.x) {
+    const int i = (int)(e / Cc), j = (int)(e - (long long)i * Cc);
+    x[tr ? (long long)j * R + i : e] = u[e] * scale;
+  }
+}
+
+__global__ void ns_writeback_kernel(const float* X, float* U, int h, int m, int mask) {
+  const int p = blockIdx.x, bh = blockIdx.y;
+  if (!(mask & (1 << p))) return;
+  int R, Cc;
+  part_dims(p, h, m, R, Cc);
+  const long long hm = (long long)h * m;
+  float* u = U + (long long)bh * 3 * hm + p * hm;
+  const float* x = X + ((long long)bh * 3 + p) * hm;
+  const bool tr = R > Cc;
+  for (long long e = threadIdx.x; e < hm; e += blockDim.x) {
+    const int i = (int)(e / Cc), j = (int)(e - (long long)i * Cc);
+    u[e] = x[tr ? (long long)j * R + i : e];
+  }
+}
+
+// grid (ceil(max cols / 32), 3, BH), block (32, 8): one column per threadIdx.x.
+template <typename OT>
+__global__ void rec_step_kernel(float* W_all, const float* U, const float* tnorm, int H, int h,
+                                int m, int mask, int sign, int renorm, OT* Wk, OT* W1o) {
+  const int p = blockIdx.y, bh = blockIdx.z;
+  if (!(mask & (1 << p))) return;
+  int R, Cc;
+  part_dims(p, h, m, R, Cc);
+  const int c = blockIdx.x * 32 + threadIdx.x;
+  const bool live = c < Cc;
+  const long long hm = (long long)h * m;
+  float* w = W_all + (long long)bh * 3 * hm + p * hm;
+  const float* u = U + (long long)bh * 3 * hm + p * hm;
+  const float sg = (float)sign;
+  __shared__ float red[8][33];
+  float ss = 0.0f;
+  if (live)
+    for (int r = threadIdx.y; r < R; r += 8) {
+      const float v = w[(long long)r * Cc + c] - sg * u[(long long)r * Cc + c];
+      ss += v * v;
+    }
+  red[threadIdx.y][threadIdx.x] = ss;
+  __syncthreads();
+  float scale = 1.0f;
+  if (renorm) {
+    float tot = 0.0f;
+    for (int y = 0; y < 8; ++y) tot += red[y][threadIdx.x];
+    const float* tn = tnorm + (long long)(bh % H) * (2 * m + h) + (p == 0 ? 0 : p == 1 ? m : m + h);
+    if (live) scale = tn[c] / sqrtf(tot);
+  }
+  if (!live) return;
+  for (int r = threadIdx.y; r < R; r += 8) {
+    const long long o = (long long)r * Cc + c;
+    const float v = (w[o] - sg * u[o]) * scale;
+    w[o] = v;
+    if (p == 1) {
+      W1o[(long long)bh * hm + o] = from_f32<OT>(v);
+    } else {
+      // Wk[bh] = [W0^T ; W2^T], [2m, h]: row (p==2 ? m : 0) + c, column r.
+      Wk[(long long)bh * 2 * hm + ((long long)(p == 2 ? m : 0) + c) * h + r] = from_f32<OT>(v);
+    }
+  }
+}
+
+__global__ void rec_finish_kernel(const float* W_all, int BH, int h, int m, float* W0_out,
+                                  float* W2_out, float* W1_out, const float* M_all,
+                                  float* M_out) {
+  const long long hm = (long long)h * m, per = 3 * hm;
+  TTT_GRID_LOOP(idx, per * BH) {
+    const long long bh = idx / per, e = idx - bh * per;
+    const int p = (int)(e / hm);
+    const long long o = bh * hm + (e - p * hm);
+    const float v = W_all[idx];
+    if (p == 0 && W0_out) W0_out[o] = v;
+    if (p == 1 && W1_out) W1_out[o] = v;
+    if (p == 2 && W2_out) W2_out[o] = v;
+    if (M_out && M_all) M_out[idx] = M_all[idx];
+  }
+}
+
+// ------------------------------------------------------------------ In-Place target conv
+__global__ void conv4_kernel(const bf16* X0, const float* w, bf16* Xc, int N, int d) {
+  TTT_GRID_LOOP(idx, (long long)N * d) {
+    const long long t = idx / d;
+    const int i = (int)(idx - t * d);
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (t - j >= 0) acc += w[j * d + i] * __bfloat162float(X0[(t - j) * d + i]);
+    Xc[idx] = __float2bfloat16_rn(acc);
+  }
+}
+
+// ------------------------------------------------------------------ diagnostics
+__global__ void wait_timeout_kernel(unsigned* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    umma::mbar_init(umma::smem_u32(&bar), 1);
+    umma::mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nobody arrives on `bar`: the wait must run out and report it.
+    umma::mbar_wait(umma::smem_u32(&bar), 0, &abort_flag, err, limit_ns);
+  }
+  __syncthreads();
+}
+
+__global__ void fill_kernel(float* p, long long n, float v) {
+  TTT_GRID_LOOP(i, n) p[i] = v;
+}
+
+template <typename F>
+cudaError_t by_ot(int ot, F&& f) {
+  if (ot == DT_BF16) return f(bf16{});
+  return f(float{});
+}
+
+}  // namespace
+
+cudaError_t prep_wk(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
+                    int src_heads, int h, int m, int src_layout, cudaStream_t s) {
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    const long long n = 2LL * m * h * n_entries;
+    prep_wk_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(W0, W2, static_cast<OT*>(Wk), n_entries,
+                                                        src_heads, h, m, src_layout);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t swiglu(int ot, const float* AB, long long rows, int m, EtaMap em, void* phi_eta,
+                   void* phi_plain, cudaStream_t s) {
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    swiglu_kernel<OT><<<grid_for(rows * m, 256), 256, 0, s>>>(
+        AB, rows, m, em, static_cast<OT*>(phi_eta), static_cast<OT*>(phi_plain));
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t grad_prep(int ot, const float* AB, const float* Dv, long long rows, int m,
+                      EtaMap em, void* P, void* E2, void* E0, cudaStream_t s) {
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    grad_prep_kernel<OT><<<grid_for(rows * m, 256), 256, 0, s>>>(
+        AB, Dv, rows, m, em, static_cast<OT*>(P), static_cast<OT*>(E2), static_cast<OT*>(E0));
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t chunk_scan(int ot, const float* dS, const float* W1, void* Sc, float* S_final, int BH,
+                       int H, int C, int m, int h, int order, int layout, cudaStream_t s) {
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    const long long n = (long long)m * h * BH;
+    chunk_scan_kernel<OT><<<grid_for(n, 256, 148 * 64), 256, 0, s>>>(
+        dS, W1, static_cast<OT*>(Sc), S_final, BH, H, C, m, h, order, layout);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t rec_init(int ot, const float* W0, const float* W2, const float* W1, int BH, int H,
+                     int h, int m, float* W_all, void* W1o, const float* M_in, float* M_all,
+                     int momentum, cudaStream_t s) {
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    const long long n = 3LL * h * m * BH;
+    rec_init_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(W0, W2, W1, BH, H, h, m, W_all,
+                                                         static_cast<OT*>(W1o), M_in, M_all,
+                                                         momentum);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t col_norms(const float* W0, const float* W2, const float* W1, int H, int h, int m,
+                      float* tnorm, cudaStream_t s) {
+  col_norms_kernel<<<grid_for((long long)(2 * m + h) * H, 128), 128, 0, s>>>(W0, W2, W1, H, h, m,
+                                                                             tnorm);
+  return cudaGetLastError();
+}
+
+cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all,
+                       const float* alpha, int C, int c, int BH, int h, int m, int mask,
+                       cudaStream_t s) {
+  const long long n = 3LL * h * m * BH;
+  rec_reduce_kernel<<<grid_for(n, 256), 256, 0, s>>>(partials, splits, U, M_all, alpha, C, c, BH,
+                                                     h, m, mask);
+  return cudaGetLastError();
+}
+
+cudaError_t ns_normalize(const float* U, float* X, int BH, int h, int m, int mask, float eps,
+                         cudaStream_t s) {
+  ns_normalize_kernel<<<dim3(3, BH), 256, 0, s>>>(U, X, h, m, mask, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t ns_writeback(const float* X, float* U, int BH, int h, int m, int mask,
+                         cudaStream_t s) {
+  ns_writeback_kernel<<<dim3(3, BH), 256, 0, s>>>(X, U, h, m, mask);
+  return cudaGetLastError();
+}
+
+cudaError_t rec_step(float* W_all, const float* U, const float* tnorm, int BH, int H, int h,
+                     int m, int mask, int sign, int renorm, void* Wk, void* W1o, int ot,
+                     cudaStream_t s) {
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    const int maxc = h > m ? h : m;
+    dim3 grid((maxc + 31) / 32, 3, BH);
+    rec_step_kernel<OT><<<grid, dim3(32, 8), 0, s>>>(W_all, U, tnorm, H, h, m, mask, sign,
+                                                     renorm, static_cast<OT*>(Wk),
+                                                     static_cast<OT*>(W1o));
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t rec_finish(const float* W_all, int BH, int h, int m, float* W0_out, float* W2_out,
+                       float* W1_out, const float* M_all, float* M_out, cudaStream_t s) {
+  const long long n = 3LL * h * m * BH;
+  rec_finish_kernel<<<grid_for(n, 256), 256, 0, s>>>(W_all, BH, h, m, W0_out, W2_out, W1_out,
+                                                     M_all, M_out);
+  return cudaGetLastError();
+}
+
+cudaError_t conv4_causal(const void* X0, const float* conv_w, void* Xc, int N, int d,
+                         cudaStream_t s) {
+  conv4_kernel<<<grid_for((long long)N * d, 256), 256, 0, s>>>(
+      static_cast<const bf16*>(X0), conv_w, static_cast<bf16*>(Xc), N, d);
+  return cudaGetLastError();
+}
+
+cudaError_t wait_timeout_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t s) {
+  wait_timeout_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
+cudaError_t fill_f32(float* p, long long n, float v, cudaStream_t s) {
+  fill_kernel<<<grid_for(n, 256), 256, 0, s>>>(p, n, v);
+  return cudaGetLastError();
+}
+
+}  // namespace ttt

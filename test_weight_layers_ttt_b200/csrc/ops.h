@@ -1,0 +1,78 @@
+// Launch wrappers of the non-GEMM kernels of the TTT layer (ops.cu). All of them enqueue
+// on `s` and return the launch status. OT is the operand element type of the dense
+// contractions (bf16 in bf16 mode, fp32 in fp32 mode), passed as a DType tag.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace ttt {
+
+// Row index r of a [Z * T, width] activation maps to eta[(r / T) * eta_ld + eta_off + r % T].
+struct EtaMap {
+  const float* eta;
+  long long T, eta_ld, eta_off;
+};
+
+// Fast-weight input-side operand Wk[e] = [W0^T ; W2^T] ([2m, h], K-major) for n_entries
+// entries; entry e reads source head e % src_heads. Source layout 0: [h, m]; 1: [m, h].
+cudaError_t prep_wk(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
+                    int src_heads, int h, int m, int src_layout, cudaStream_t s);
+
+// phi = silu(A) * B from AB rows [A | B] (fp32, width 2m); writes phi * eta to phi_eta and,
+// when non-null, the unscaled phi to phi_plain (both OT, width m).
+cudaError_t swiglu(int ot, const float* AB, long long rows, int m, EtaMap em, void* phi_eta,
+                   void* phi_plain, cudaStream_t s);
+
+// Per-token pieces of the recurrent gradients from AB = [K W0 | K W2] and Dv = V W1^T:
+//   d = -eta * Dv, P = silu(A) * B * eta, E2 = d * silu(A), E0 = d * B * silu'(A).
+// E2/E0 are skipped when null.
+cudaError_t grad_prep(int ot, const float* AB, const float* Dv, long long rows, int m,
+                      EtaMap em, void* P, void* E2, void* E0, cudaStream_t s);
+
+// Chunk prefix sums: S starts at W1[bh % H] (layout 0 [m,h] / 1 [h,m]); for each chunk c
+// the state read by chunk c is written to Sc[bh, c] (OT, [m,h]): inclusive of dS[bh, c]
+// (order 0) or exclusive (order 1). The state after the last chunk goes to S_final
+// (fp32, W1's layout) when non-null.
+cudaError_t chunk_scan(int ot, const float* dS, const float* W1, void* Sc, float* S_final, int BH,
+                       int H, int C, int m, int h, int order, int layout, cudaStream_t s);
+
+// Recurrent-state helpers. Per (b, head) the fp32 state W_all holds [W0 (h*m) | W1 (m*h) |
+// W2 (h*m)]; momentum and the update buffer U use the same part layout.
+cudaError_t rec_init(int ot, const float* W0, const float* W2, const float* W1, int BH, int H,
+                     int h, int m, float* W_all, void* W1o, const float* M_in, float* M_all,
+                     int momentum, cudaStream_t s);
+// Column norms over the input dimension of the initial weights, per head:
+// tnorm[head] = [W0 columns (m) | W1 columns (h) | W2 columns (m)].
+cudaError_t col_norms(const float* W0, const float* W2, const float* W1, int H, int h, int m,
+                      float* tnorm, cudaStream_t s);
+// U = sum over `splits` partial gradients [split][BH][3hm]; with momentum
+// M <- alpha[bh, c] * M + U and U <- M. Only parts in `mask` are touched.
+cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all,
+                       const float* alpha, int C, int c, int BH, int h, int m, int mask,
+                       cudaStream_t s);
+// Newton-Schulz set-up / tear-down: X = U / (||U||_F + eps) in the wide orientation
+// ([rmin, rmax]) for every (bh, part in mask); and U <- X back in U's own orientation.
+cudaError_t ns_normalize(const float* U, float* X, int BH, int h, int m, int mask, float eps,
+                         cudaStream_t s);
+cudaError_t ns_writeback(const float* X, float* U, int BH, int h, int m, int mask,
+                         cudaStream_t s);
+// W <- W - sign * U, optional per-column renormalisation to tnorm, refresh OT copies.
+cudaError_t rec_step(float* W_all, const float* U, const float* tnorm, int BH, int H, int h,
+                     int m, int mask, int sign, int renorm, void* Wk, void* W1o, int ot,
+                     cudaStream_t s);
+// Final weights [B,H,...] (nullable outputs) and momentum copy-out.
+cudaError_t rec_finish(const float* W_all, int BH, int h, int m, float* W0_out, float* W2_out,
+                       float* W1_out, const float* M_all, float* M_out, cudaStream_t s);
+
+// Causal depthwise 4-tap convolution: Xc[t, i] = sum_j conv_w[j, i] * X0[t - j, i] (bf16).
+cudaError_t conv4_causal(const void* X0, const float* conv_w, void* Xc, int N, int d,
+                         cudaStream_t s);
+
+// Block that waits on an mbarrier nobody arrives at, bounded by `limit_ns`.
+cudaError_t wait_timeout_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t s);
+
+cudaError_t fill_f32(float* p, long long n, float v, cudaStream_t s);
+
+}  // namespace ttt

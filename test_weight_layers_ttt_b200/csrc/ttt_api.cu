@@ -1,0 +1,668 @@
+// C ABI of the TTT layer library (include/ttt.h): argument checks, workspace planning and
+// the enqueue order of the kernels for the parallel form, the recurrent form and the
+// In-Place target. Every contraction goes through run_gemm(), which picks the tcgen05
+// tensor-core engine for bf16 operands and the CUDA-core engine otherwise.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "gemm.h"
+#include "ops.h"
+
+namespace ttt {
+
+// Per-device error word written by bounded waits and device-side checks.
+static __device__ unsigned g_dev_err_word;
+
+static thread_local char g_msg[512] = "";
+
+void set_error_message(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+}
+
+unsigned* device_error_word() {
+  static std::mutex mu;
+  static unsigned* addr[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_err_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned*>(p);
+  }
+  return addr[dev];
+}
+
+unsigned long long wait_limit_ns() {
+  const char* s = getenv("TTT_WAIT_LIMIT_NS");
+  if (s && *s) {
+    const unsigned long long v = strtoull(s, nullptr, 10);
+    if (v >= 100000ull) return v;
+  }
+  return kDefaultWaitNs;
+}
+
+namespace {
+
+// ------------------------------------------------------------------ kernel tracing
+struct TraceState {
+  std::mutex mu;
+  bool on = false;
+  int dev = -1;
+  int n = 0;
+  int cap = 0;
+  std::vector<cudaEvent_t> ev;  // 2 per record
+  std::vector<const char*> names;
+};
+TraceState g_trace;
+
+// Brackets one kernel launch with two events on its stream while tracing is enabled.
+struct TraceScope {
+  int idx = -1;
+  cudaStream_t s;
+  TraceScope(const char* name, cudaStream_t st) : s(st) {
+    if (!g_trace.on) return;
+    std::lock_guard<std::mutex> lk(g_trace.mu);
+    int d = -1;
+    if (!g_trace.on || cudaGetDevice(&d) != cudaSuccess || d != g_trace.dev ||
+        g_trace.n >= g_trace.cap)
+      return;
+    idx = g_trace.n++;
+    g_trace.names[idx] = name;
+    cudaEventRecord(g_trace.ev[2 * idx], s);
+  }
+  ~TraceScope() {
+    if (idx >= 0) cudaEventRecord(g_trace.ev[2 * idx + 1], s);
+  }
+};
+
+bool force_simt() {
+  const char* s = getenv("TTT_GEMM_ENGINE");
+  return s && strcmp(s, "simt") == 0;
+}
+
+ttt_status run_gemm(const char* name, const GemmProblem& p, cudaStream_t s) {
+  if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
+  TraceScope ts(name, s);
+  if (p.K > 0 && !force_simt() && umma_supported(p))
+    return gemm_umma(p, s, device_error_word(), wait_limit_ns());
+  return gemm_simt(p, s);
+}
+
+ttt_status run_simt(const char* name, const GemmProblem& p, cudaStream_t s) {
+  if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
+  TraceScope ts(name, s);
+  return gemm_simt(p, s);
+}
+
+#define TTT_TRY(expr)                        \
+  do {                                       \
+    ttt_status st__ = (expr);                \
+    if (st__ != TTT_OK) return st__;         \
+  } while (0)
+
+#define TTT_CUDA(expr)                                                                    \
+  do {                                                                                    \
+    cudaError_t e__ = (expr);                                                             \
+    if (e__ != cudaSuccess) {                                                             \
+      set_error_message("%s failed: %s", #expr, cudaGetErrorString(e__));                 \
+      return TTT_ERR_CUDA;                                                                \
+    }                                                                                     \
+  } while (0)
+
+// One traced kernel launch of ops.h.
+#define TTT_OP(name, expr)         \
+  do {                             \
+    TraceScope ts__((name), s);    \
+    TTT_CUDA(expr);                \
+  } while (0)
+
+ttt_status fail(ttt_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Bump allocator over the caller's workspace (or a size counter when base is null).
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  void* take(size_t bytes) {
+    off = (off + 255) & ~static_cast<size_t>(255);
+    void* p = base ? base + off : nullptr;
+    off += bytes;
+    return p;
+  }
+  template <typename T> T* take_n(long long n) { return static_cast<T*>(take(sizeof(T) * (size_t)n)); }
+};
+
+ttt_status check_desc(const ttt_desc* d, int path) {
+  if (!d) return fail(TTT_ERR_INVALID_ARG, "desc is NULL");
+  if (d->B < 0 || d->H < 0 || d->N < 0) return fail(TTT_ERR_INVALID_ARG, "B, H, N must be >= 0");
+  if (d->h < 1 || d->m < 1 || d->chunk < 1)
+    return fail(TTT_ERR_INVALID_ARG, "h, m and chunk must be >= 1");
+  if (d->dtype != TTT_DTYPE_FP32 && d->dtype != TTT_DTYPE_BF16)
+    return fail(TTT_ERR_INVALID_ARG, "dtype must be TTT_DTYPE_FP32 or TTT_DTYPE_BF16");
+  if (d->order != TTT_ORDER_UPDATE_APPLY && d->order != TTT_ORDER_APPLY_UPDATE)
+    return fail(TTT_ERR_INVALID_ARG, "order must be UPDATE_APPLY or APPLY_UPDATE");
+  if (d->sign != 1 && d->sign != -1) return fail(TTT_ERR_INVALID_ARG, "sign must be +1 or -1");
+  if (d->w_in_layout != 0 && d->w_in_layout != 1)
+    return fail(TTT_ERR_INVALID_ARG, "w_in_layout must be 0 or 1");
+  if (d->w1_layout != 0 && d->w1_layout != 1)
+    return fail(TTT_ERR_INVALID_ARG, "w1_layout must be 0 or 1");
+  if (path == TTT_PATH_PARALLEL) {
+    if (d->update_mask != 0 || d->renorm != 0 || d->momentum != 0 || d->ns_steps != 0)
+      return fail(TTT_ERR_INVALID_ARG,
+                  "parallel form: update_mask, renorm, momentum and ns_steps must be 0");
+  } else if (path == TTT_PATH_RECURRENT) {
+    if (d->update_mask < 1 || d->update_mask > 7)
+      return fail(TTT_ERR_INVALID_ARG, "update_mask must be in 1..7");
+    if ((d->renorm != 0 && d->renorm != 1) || (d->momentum != 0 && d->momentum != 1))
+      return fail(TTT_ERR_INVALID_ARG, "renorm and momentum must be 0 or 1");
+    if (d->ns_steps < 0 || d->ns_steps > 8) return fail(TTT_ERR_INVALID_ARG, "ns_steps must be in 0..8");
+    if (d->w_in_layout != 0 || d->w1_layout != 0)
+      return fail(TTT_ERR_UNSUPPORTED, "recurrent form: only the default weight layouts");
+  } else {
+    return fail(TTT_ERR_INVALID_ARG, "path must be TTT_PATH_PARALLEL or TTT_PATH_RECURRENT");
+  }
+  if (d->dtype == TTT_DTYPE_BF16 && (d->h % 8 != 0 || d->m % 8 != 0))
+    return fail(TTT_ERR_UNSUPPORTED, "bf16 mode needs h and m to be multiples of 8");
+  const long long BH = (long long)d->B * d->H;
+  if (BH > 65535) return fail(TTT_ERR_UNSUPPORTED, "B*H must be <= 65535");
+  if ((long long)d->N > (1LL << 22)) return fail(TTT_ERR_UNSUPPORTED, "N must be <= 4194304");
+  const long long C = (d->N + d->chunk - 1) / d->chunk;
+  if (BH * C > 65535 && path == TTT_PATH_PARALLEL)
+    return fail(TTT_ERR_UNSUPPORTED, "B*H*ceil(N/chunk) must be <= 65535");
+  if ((long long)d->h * d->m > (1LL << 31))
+    return fail(TTT_ERR_UNSUPPORTED, "h*m must be <= 2^31");
+  return TTT_OK;
+}
+
+// ------------------------------------------------------------------ parallel form
+struct ParBufs {
+  void* Wk;
+  float* AB;
+  void* phiA;
+  void* phiB;
+  float* dS;
+  void* Sc;
+};
+
+size_t plan_parallel(const ttt_desc& d, void* base, ParBufs& b) {
+  Carve cv(base);
+  const size_t os = d.dtype == TTT_DTYPE_BF16 ? 2 : 4;
+  const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
+  const long long rows = BH * d.N, hm = (long long)d.h * d.m;
+  b.Wk = cv.take(os * 2 * hm * d.H);
+  b.AB = cv.take_n<float>(rows * 2 * d.m);
+  b.phiA = cv.take(os * rows * d.m);
+  b.phiB = cv.take(os * rows * d.m);
+  b.dS = cv.take_n<float>(BH * C * hm);
+  b.Sc = cv.take(os * BH * C * hm);
+  return cv.off;
+}
+
+// A = X (tokens x h rows of sequence (b, head)), B = Wk[head]: AB = X [W0 | W2].
+GemmProblem features_problem(const ttt_desc& d, const void* X, const void* Wk, float* AB) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long N = d.N, h = d.h, m = d.m;
+  GemmProblem p;
+  p.M = d.N; p.N = 2 * d.m; p.K = d.h; p.Z0 = d.H; p.Z1 = d.B;
+  p.A = {X, ot, false, h, N * h, (long long)d.H * N * h};
+  p.B = {Wk, ot, false, h, 2 * m * h, 0};
+  p.C = {AB, DT_F32, 2 * m, N * 2 * m, (long long)d.H * N * 2 * m};
+  return p;
+}
+
+ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
+                         const float* eta, const float* W0, const float* W2, const float* W1,
+                         void* out, float* S_final, const ParBufs& b, cudaStream_t s) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, L = d.chunk;
+  const long long C = (N + L - 1) / L, Cf = N / L, tail = N - Cf * L, hm = h * m;
+  const bool shared_qk = (q == k);
+
+  TTT_OP("prep_weights", prep_wk(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
+  // phi(K) eta (and phi(Q) when q == k)
+  TTT_TRY(run_gemm("gemm_features_k", features_problem(d, k, b.Wk, b.AB), s));
+  EtaMap em{eta, N, N, 0};
+  TTT_OP("swiglu_k", swiglu(ot, b.AB, BH * N, d.m, em, b.phiA, shared_qk ? b.phiB : nullptr, s));
+  // Delta S_c = sign * phi(K_c)^T diag(eta) V_c  (per (b, head) and chunk)
+  for (int part = 0; part < 2; ++part) {
+    const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);
+    if (nz1 == 0) continue;
+    const long long t0 = part == 0 ? 0 : Cf * L;
+    GemmProblem p;
+    p.M = d.m; p.N = d.h; p.K = (int)(part == 0 ? L : tail); p.Z0 = (int)BH; p.Z1 = (int)nz1;
+    p.A = {static_cast<const char*>(b.phiA) + t0 * m * dtype_size(ot), ot, true, m, N * m, L * m};
+    p.B = {static_cast<const char*>(v) + t0 * h * dtype_size(ot), ot, true, h, N * h, L * h};
+    p.C = {b.dS + (part == 0 ? 0 : Cf * hm), DT_F32, h, C * hm, hm};
+    p.alpha = (float)d.sign;
+    TTT_TRY(run_gemm("gemm_state_delta", p, s));
+  }
+  // States read by each chunk, and the final state.
+  TTT_OP("chunk_scan", chunk_scan(ot, b.dS, W1, b.Sc, S_final, (int)BH, d.H, (int)C, d.m, d.h,
+                                  d.order, d.w1_layout, s));
+  if (!shared_qk) {
+    TTT_TRY(run_gemm("gemm_features_q", features_problem(d, q, b.Wk, b.AB), s));
+    TTT_OP("swiglu_q", swiglu(ot, b.AB, BH * N, d.m, em, nullptr, b.phiB, s));
+  }
+  // O_c = phi(Q_c) S_c
+  for (int part = 0; part < 2; ++part) {
+    const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);
+    if (nz1 == 0) continue;
+    const long long t0 = part == 0 ? 0 : Cf * L;
+    GemmProblem p;
+    p.M = (int)(part == 0 ? L : tail); p.N = d.h; p.K = d.m; p.Z0 = (int)BH; p.Z1 = (int)nz1;
+    p.A = {static_cast<const char*>(b.phiB) + t0 * m * dtype_size(ot), ot, false, m, N * m, L * m};
+    p.B = {static_cast<const char*>(b.Sc) + (part == 0 ? 0 : Cf * hm) * dtype_size(ot), ot, true,
+           h, C * hm, hm};
+    p.C = {static_cast<char*>(out) + t0 * h * dtype_size(ot), ot, h, N * h, L * h};
+    TTT_TRY(run_gemm("gemm_output", p, s));
+  }
+  return TTT_OK;
+}
+
+// ------------------------------------------------------------------ recurrent form
+struct RecBufs {
+  float* W_all;
+  float* M_all;
+  float* U;
+  float* tnorm;
+  void* Wk;
+  void* W1o;
+  float* AB;
+  float* Dv;
+  void* P;
+  void* E2;
+  void* E0;
+  float* partials;
+  void* phiQ;
+  float* X;
+  float* X2;
+  float* Ag;
+  float* Pm;
+  int splits;
+};
+
+// Token splits of the gradient reductions: a divisor of the chunk length L such that the
+// split length stays a multiple of 64 and the three gradient GEMMs give the GPU enough CTAs.
+int choose_splits(const ttt_desc& d, long long L) {
+  const long long BH = (long long)d.B * d.H;
+  const long long tiles = BH * ((d.m + 127) / 128) * ((d.h + 255) / 256);
+  long long best = 1;
+  for (long long sp = 2; sp <= 64; sp *= 2) {
+    if (L % sp != 0 || (L / sp) % 64 != 0 || L / sp < 128) break;
+    if (tiles * (sp / 2) >= 2 * 148) break;
+    best = sp;
+  }
+  return (int)best;
+}
+
+size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
+  Carve cv(base);
+  const size_t os = d.dtype == TTT_DTYPE_BF16 ? 2 : 4;
+  const long long BH = (long long)d.B * d.H, hm = (long long)d.h * d.m, L = d.chunk;
+  const long long rows = BH * L;
+  b.splits = choose_splits(d, L);
+  b.W_all = cv.take_n<float>(BH * 3 * hm);
+  b.M_all = d.momentum ? cv.take_n<float>(BH * 3 * hm) : nullptr;
+  b.U = cv.take_n<float>(BH * 3 * hm);
+  b.tnorm = cv.take_n<float>((long long)d.H * (2 * d.m + d.h));
+  b.Wk = cv.take(os * BH * 2 * hm);
+  b.W1o = cv.take(os * BH * hm);
+  b.AB = cv.take_n<float>(rows * 2 * d.m);
+  b.Dv = cv.take_n<float>(rows * d.m);
+  b.P = cv.take(os * rows * d.m);
+  b.E2 = cv.take(os * rows * d.m);
+  b.E0 = cv.take(os * rows * d.m);
+  b.partials = cv.take_n<float>((long long)b.splits * BH * 3 * hm);
+  b.phiQ = cv.take(os * rows * d.m);
+  if (d.ns_steps > 0) {
+    const long long r = d.h < d.m ? d.h : d.m;
+    b.X = cv.take_n<float>(BH * 3 * hm);
+    b.X2 = cv.take_n<float>(BH * 3 * hm);
+    b.Ag = cv.take_n<float>(BH * 3 * r * r);
+    b.Pm = cv.take_n<float>(BH * 3 * r * r);
+  } else {
+    b.X = b.X2 = b.Ag = b.Pm = nullptr;
+  }
+  return cv.off;
+}
+
+ttt_status rec_apply(const ttt_desc& d, const void* q, void* out, long long t0, long long Lc,
+                     const RecBufs& b, cudaStream_t s) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const size_t es = dtype_size(ot);
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m;
+  GemmProblem p;
+  p.M = (int)Lc; p.N = 2 * d.m; p.K = d.h; p.Z0 = (int)BH; p.Z1 = 1;
+  p.A = {static_cast<const char*>(q) + t0 * h * es, ot, false, h, N * h, 0};
+  p.B = {b.Wk, ot, false, h, 2 * m * h, 0};
+  p.C = {b.AB, DT_F32, 2 * m, Lc * 2 * m, 0};
+  TTT_TRY(run_gemm("gemm_features_q", p, s));
+  EtaMap em{nullptr, Lc, N, t0};
+  TTT_OP("swiglu_q", swiglu(ot, b.AB, BH * Lc, d.m, em, nullptr, b.phiQ, s));
+  GemmProblem o;
+  o.M = (int)Lc; o.N = d.h; o.K = d.m; o.Z0 = (int)BH; o.Z1 = 1;
+  o.A = {b.phiQ, ot, false, m, Lc * m, 0};
+  o.B = {b.W1o, ot, true, h, m * h, 0};
+  o.C = {static_cast<char*>(out) + t0 * h * es, ot, h, N * h, 0};
+  return run_gemm("gemm_output", o, s);
+}
+
+ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const float* eta,
+                      const float* alpha, int c, long long t0, long long Lc, const RecBufs& b,
+                      cudaStream_t s) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const size_t es = dtype_size(ot);
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, hm = h * m;
+  const int mask = d.update_mask;
+  const bool need_in = (mask & (TTT_UPDATE_W0 | TTT_UPDATE_W2)) != 0;
+  const long long C = (N + d.chunk - 1) / d.chunk;
+  // [A | B] = K_c [W0 | W2]
+  GemmProblem p;
+  p.M = (int)Lc; p.N = 2 * d.m; p.K = d.h; p.Z0 = (int)BH; p.Z1 = 1;
+  p.A = {static_cast<const char*>(k) + t0 * h * es, ot, false, h, N * h, 0};
+  p.B = {b.Wk, ot, false, h, 2 * m * h, 0};
+  p.C = {b.AB, DT_F32, 2 * m, Lc * 2 * m, 0};
+  TTT_TRY(run_gemm("gemm_features_k", p, s));
+  if (need_in) {  // Dv = V_c W1^T
+    GemmProblem g;
+    g.M = (int)Lc; g.N = d.m; g.K = d.h; g.Z0 = (int)BH; g.Z1 = 1;
+    g.A = {static_cast<const char*>(v) + t0 * h * es, ot, false, h, N * h, 0};
+    g.B = {b.W1o, ot, false, h, m * h, 0};
+    g.C = {b.Dv, DT_F32, m, Lc * m, 0};
+    TTT_TRY(run_gemm("gemm_v_w1t", g, s));
+  }
+  EtaMap em{eta, Lc, N, t0};
+  TTT_OP("grad_prep", grad_prep(ot, b.AB, b.Dv, BH * Lc, d.m, em, b.P,
+                                 (mask & TTT_UPDATE_W2) ? b.E2 : nullptr,
+                                 (mask & TTT_UPDATE_W0) ? b.E0 : nullptr, s));
+  // Split-K gradient reductions over the chunk's tokens.
+  const int sp = (Lc == d.chunk) ? b.splits : 1;
+  const long long Ks = Lc / sp;
+  const long long tot = BH * 3 * hm;
+  if (mask & TTT_UPDATE_W1) {  // dW1 = -(phi eta)^T V
+    GemmProblem g;
+    g.M = d.m; g.N = d.h; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
+    g.A = {b.P, ot, true, m, Lc * m, Ks * m};
+    g.B = {static_cast<const char*>(v) + t0 * h * es, ot, true, h, N * h, Ks * h};
+    g.C = {b.partials + hm, DT_F32, h, 3 * hm, tot};
+    g.alpha = -1.0f;
+    TTT_TRY(run_gemm("gemm_grad_w1", g, s));
+  }
+  for (int pidx = 0; pidx <= 2; pidx += 2) {  // dW0 = K^T E0, dW2 = K^T E2
+    if (!(mask & (pidx == 0 ? TTT_UPDATE_W0 : TTT_UPDATE_W2))) continue;
+    GemmProblem g;
+    g.M = d.h; g.N = d.m; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
+    g.A = {static_cast<const char*>(k) + t0 * h * es, ot, true, h, N * h, Ks * h};
+    g.B = {pidx == 0 ? b.E0 : b.E2, ot, true, m, Lc * m, Ks * m};
+    g.C = {b.partials + pidx * hm, DT_F32, m, 3 * hm, tot};
+    TTT_TRY(run_gemm(pidx == 0 ? "gemm_grad_w0" : "gemm_grad_w2", g, s));
+  }
+  TTT_OP("reduce_momentum", rec_reduce(b.partials, sp, b.U, d.momentum ? b.M_all : nullptr,
+                                      alpha, (int)C, c, (int)BH, d.h, d.m, mask, s));
+  if (d.ns_steps > 0) {
+    const float a3 = 3.4445f, b3 = -4.7750f, c3 = 2.0315f;
+    const long long r = h < m ? h : m, cc = h < m ? m : h;
+    TTT_OP("ns_normalize", ns_normalize(b.U, b.X, (int)BH, d.h, d.m, mask, 1e-7f, s));
+    float* X = b.X;
+    float* X2 = b.X2;
+    for (int it = 0; it < d.ns_steps; ++it) {
+      GemmProblem g1;  // A = X X^T
+      g1.M = (int)r; g1.N = (int)r; g1.K = (int)cc; g1.Z0 = (int)(3 * BH);
+      g1.A = {X, DT_F32, false, cc, r * cc, 0};
+      g1.B = {X, DT_F32, false, cc, r * cc, 0};
+      g1.C = {b.Ag, DT_F32, r, r * r, 0};
+      TTT_TRY(run_simt("ns_gram", g1, s));
+      GemmProblem g2;  // P = c A A + b A
+      g2.M = (int)r; g2.N = (int)r; g2.K = (int)r; g2.Z0 = (int)(3 * BH);
+      g2.A = {b.Ag, DT_F32, false, r, r * r, 0};
+      g2.B = {b.Ag, DT_F32, true, r, r * r, 0};
+      g2.C = {b.Pm, DT_F32, r, r * r, 0};
+      g2.alpha = c3; g2.beta = b3; g2.Cin = {b.Ag, r, r * r, 0};
+      TTT_TRY(run_simt("ns_poly", g2, s));
+      GemmProblem g3;  // X' = P X + a X
+      g3.M = (int)r; g3.N = (int)cc; g3.K = (int)r; g3.Z0 = (int)(3 * BH);
+      g3.A = {b.Pm, DT_F32, false, r, r * r, 0};
+      g3.B = {X, DT_F32, true, cc, r * cc, 0};
+      g3.C = {X2, DT_F32, cc, r * cc, 0};
+      g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, cc, r * cc, 0};
+      TTT_TRY(run_simt("ns_apply", g3, s));
+      float* t = X; X = X2; X2 = t;
+    }
+    TTT_OP("ns_writeback", ns_writeback(X, b.U, (int)BH, d.h, d.m, mask, s));
+  }
+  TTT_OP("step_renorm", rec_step(b.W_all, b.U, b.tnorm, (int)BH, d.H, d.h, d.m, mask, d.sign,
+                                  d.renorm, b.Wk, b.W1o, ot, s));
+  return TTT_OK;
+}
+
+ttt_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return TTT_OK;
+  if (!ws) return fail(TTT_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+  if (reinterpret_cast<uintptr_t>(ws) & 255)
+    return fail(TTT_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (have < need)
+    return fail(TTT_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", have, need);
+  return TTT_OK;
+}
+
+}  // namespace
+}  // namespace ttt
+
+using namespace ttt;
+
+extern "C" {
+
+size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path) {
+  if (check_desc(desc, path) != TTT_OK) return 0;
+  if (path == TTT_PATH_PARALLEL) {
+    ParBufs b;
+    return plan_parallel(*desc, nullptr, b);
+  }
+  RecBufs b;
+  return plan_recurrent(*desc, nullptr, b);
+}
+
+ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* k, const void* v,
+                               const float* eta, const float* W0, const float* W2,
+                               const float* W1, void* out, float* S_final, void* workspace,
+                               size_t workspace_bytes, ttt_stream_t stream) {
+  TTT_TRY(check_desc(desc, TTT_PATH_PARALLEL));
+  const ttt_desc& d = *desc;
+  const long long BH = (long long)d.B * d.H;
+  if (BH == 0) return TTT_OK;
+  if (!W0 || !W2 || !W1) return fail(TTT_ERR_INVALID_ARG, "W0, W2 and W1 must not be NULL");
+  if (d.N > 0) {
+    if (!q || !k || !v || !eta || !out)
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v, eta and out must not be NULL");
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(out) || !al16(W0) || !al16(W2) || !al16(W1))
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v, out and the weights must be 16-byte aligned");
+  }
+  ParBufs b;
+  const size_t need = plan_parallel(d, nullptr, b);
+  TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  plan_parallel(d, workspace, b);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d.N == 0) {
+    if (S_final)
+      TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, W1, b.Sc, S_final, (int)BH, d.H, 0, d.m, d.h,
+                                      d.order, d.w1_layout, s));
+    return TTT_OK;
+  }
+  return parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s);
+}
+
+ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const void* k,
+                                  const void* v, const float* eta, const float* alpha,
+                                  const float* W0, const float* W2, const float* W1, void* out,
+                                  float* W0_out, float* W2_out, float* W1_out, float* M_io,
+                                  void* workspace, size_t workspace_bytes, ttt_stream_t stream) {
+  TTT_TRY(check_desc(desc, TTT_PATH_RECURRENT));
+  const ttt_desc& d = *desc;
+  const long long BH = (long long)d.B * d.H;
+  if (BH == 0) return TTT_OK;
+  if (!W0 || !W2 || !W1) return fail(TTT_ERR_INVALID_ARG, "W0, W2 and W1 must not be NULL");
+  if (d.momentum && !alpha && d.N > 0)
+    return fail(TTT_ERR_INVALID_ARG, "momentum needs alpha [B,H,C]");
+  if (d.N > 0) {
+    if (!q || !k || !v || !eta || !out)
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v, eta and out must not be NULL");
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(out) || !al16(W0) || !al16(W2) || !al16(W1))
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v, out and the weights must be 16-byte aligned");
+  }
+  RecBufs b;
+  const size_t need = plan_recurrent(d, nullptr, b);
+  TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  plan_recurrent(d, workspace, b);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1o,
+                              d.momentum ? M_io : nullptr, b.M_all, d.momentum, s));
+  TTT_OP("prep_weights", prep_wk(ot, W0, W2, b.Wk, (int)BH, d.H, d.h, d.m, 0, s));
+  if (d.renorm) TTT_OP("col_norms", col_norms(W0, W2, W1, d.H, d.h, d.m, b.tnorm, s));
+  const long long N = d.N, L = d.chunk;
+  int c = 0;
+  for (long long t0 = 0; t0 < N; t0 += L, ++c) {
+    const long long Lc = (t0 + L <= N) ? L : N - t0;
+    if (d.order == TTT_ORDER_APPLY_UPDATE) TTT_TRY(rec_apply(d, q, out, t0, Lc, b, s));
+    TTT_TRY(rec_update(d, k, v, eta, alpha, c, t0, Lc, b, s));
+    if (d.order == TTT_ORDER_UPDATE_APPLY) TTT_TRY(rec_apply(d, q, out, t0, Lc, b, s));
+  }
+  if (W0_out || W2_out || W1_out || (d.momentum && M_io))
+    TTT_OP("rec_finish", rec_finish(b.W_all, (int)BH, d.h, d.m, W0_out, W2_out, W1_out, b.M_all,
+                                    d.momentum ? M_io : nullptr, s));
+  return TTT_OK;
+}
+
+size_t ttt_lm_target_workspace_bytes(int32_t N, int32_t d) {
+  if (N < 0 || d < 1) return 0;
+  Carve cv(nullptr);
+  cv.take(2 * (size_t)N * d);
+  return cv.off;
+}
+
+ttt_status ttt_lm_target(int32_t N, int32_t d, const void* X0, const float* conv_w,
+                         const void* W_target, void* vbar, void* workspace,
+                         size_t workspace_bytes, ttt_stream_t stream) {
+  if (N < 0 || d < 1) return fail(TTT_ERR_INVALID_ARG, "N must be >= 0 and d >= 1");
+  if (d % 8 != 0) return fail(TTT_ERR_UNSUPPORTED, "d must be a multiple of 8");
+  if (N > (1 << 22)) return fail(TTT_ERR_UNSUPPORTED, "N must be <= 4194304");
+  if (N == 0) return TTT_OK;
+  if (!X0 || !conv_w || !W_target || !vbar)
+    return fail(TTT_ERR_INVALID_ARG, "X0, conv_w, W_target and vbar must not be NULL");
+  if (!al16(X0) || !al16(W_target) || !al16(vbar))
+    return fail(TTT_ERR_INVALID_ARG, "X0, W_target and vbar must be 16-byte aligned");
+  const size_t need = ttt_lm_target_workspace_bytes(N, d);
+  TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TTT_OP("conv4_causal", conv4_causal(X0, conv_w, workspace, N, d, s));
+  GemmProblem p;
+  p.M = N; p.N = d; p.K = d;
+  p.A = {workspace, DT_BF16, false, d, 0, 0};
+  p.B = {W_target, DT_BF16, true, d, 0, 0};
+  p.C = {vbar, DT_BF16, d, 0, 0};
+  return run_gemm("gemm_lm_target", p, s);
+}
+
+ttt_status ttt_last_device_status(ttt_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(TTT_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  unsigned w = 0;
+  e = cudaMemcpyFromSymbol(&w, g_dev_err_word, sizeof(w));
+  if (e != cudaSuccess) return fail(TTT_ERR_CUDA, "read error word: %s", cudaGetErrorString(e));
+  if (w) {
+    const unsigned z = 0;
+    cudaMemcpyToSymbol(g_dev_err_word, &z, sizeof(z));
+    if (w & DEVERR_TIMEOUT) return fail(TTT_ERR_TIMEOUT, "a bounded device wait ran out");
+    return fail(TTT_ERR_DEVICE, "device-side check failed (word 0x%x)", w);
+  }
+  return TTT_OK;
+}
+
+ttt_status ttt_debug_wait_timeout(int64_t timeout_ns, ttt_stream_t stream) {
+  if (timeout_ns < 100000 || timeout_ns > 10000000000LL)
+    return fail(TTT_ERR_INVALID_ARG, "timeout_ns must be in [1e5, 1e10]");
+  unsigned* w = device_error_word();
+  if (!w) return fail(TTT_ERR_CUDA, "no device error word");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TTT_OP("wait_timeout_probe", wait_timeout_probe(w, (unsigned long long)timeout_ns, s));
+  return TTT_OK;
+}
+
+ttt_status ttt_trace_enable(int32_t capacity) {
+  if (capacity < 1 || capacity > (1 << 20))
+    return fail(TTT_ERR_INVALID_ARG, "trace capacity must be in 1..2^20");
+  ttt_trace_disable();
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(TTT_ERR_CUDA, "cudaGetDevice failed");
+  g_trace.ev.assign(2 * (size_t)capacity, nullptr);
+  for (auto& e : g_trace.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) return fail(TTT_ERR_CUDA, "cudaEventCreate failed");
+  g_trace.names.assign(capacity, "");
+  g_trace.cap = capacity;
+  g_trace.n = 0;
+  g_trace.dev = dev;
+  g_trace.on = true;
+  return TTT_OK;
+}
+
+ttt_status ttt_trace_disable(void) {
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  g_trace.on = false;
+  for (auto& e : g_trace.ev)
+    if (e) cudaEventDestroy(e);
+  g_trace.ev.clear();
+  g_trace.names.clear();
+  g_trace.n = g_trace.cap = 0;
+  return TTT_OK;
+}
+
+int32_t ttt_trace_count(void) { return g_trace.n; }
+
+ttt_status ttt_trace_get(int32_t index, const char** kernel_name, float* milliseconds) {
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  if (index < 0 || index >= g_trace.n) return fail(TTT_ERR_INVALID_ARG, "trace index out of range");
+  cudaEvent_t a = g_trace.ev[2 * (size_t)index], b = g_trace.ev[2 * (size_t)index + 1];
+  if (cudaEventSynchronize(b) != cudaSuccess) return fail(TTT_ERR_CUDA, "cudaEventSynchronize failed");
+  float ms = 0.0f;
+  if (cudaEventElapsedTime(&ms, a, b) != cudaSuccess)
+    return fail(TTT_ERR_CUDA, "cudaEventElapsedTime failed");
+  if (kernel_name) *kernel_name = g_trace.names[index];
+  if (milliseconds) *milliseconds = ms;
+  return TTT_OK;
+}
+
+const char* ttt_status_str(ttt_status status) {
+  switch (status) {
+    case TTT_OK: return "TTT_OK";
+    case TTT_ERR_INVALID_ARG: return "TTT_ERR_INVALID_ARG";
+    case TTT_ERR_UNSUPPORTED: return "TTT_ERR_UNSUPPORTED";
+    case TTT_ERR_WORKSPACE: return "TTT_ERR_WORKSPACE";
+    case TTT_ERR_CUDA: return "TTT_ERR_CUDA";
+    case TTT_ERR_TIMEOUT: return "TTT_ERR_TIMEOUT";
+    case TTT_ERR_DEVICE: return "TTT_ERR_DEVICE";
+  }
+  return "TTT_ERR_UNKNOWN";
+}
+
+const char* ttt_last_error_message(void) { return g_msg; }
+
+int32_t ttt_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports every symbol
+include/ttt.h declares, sizes workspaces, and rejects bad arguments before enqueueing
+anything (so none of these calls reaches the CUDA driver)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from test_weight_layers_ttt_b200 import abi
+from test_weight_layers_ttt_b200 import build as tbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ttt.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    tbuild.build()
+    return abi.lib()
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(ttt_[a-z0-9_]+)\s*\(", src))
+
+
+def test_every_declared_symbol_is_exported():
+    declared = header_functions()
+    assert declared == set(abi.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", tbuild.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ttt_[a-z0-9_]+)$", out, flags=re.M))
+    assert declared <= exported, declared - exported
+    for name in declared:
+        assert getattr(abi.lib(), name) is not None
+
+
+def test_status_strings_and_version():
+    for st, name in [(0, "TTT_OK"), (1, "TTT_ERR_INVALID_ARG"), (2, "TTT_ERR_UNSUPPORTED"),
+                     (3, "TTT_ERR_WORKSPACE"), (4, "TTT_ERR_CUDA"), (5, "TTT_ERR_TIMEOUT"),
+                     (6, "TTT_ERR_DEVICE")]:
+        assert abi.ttt_status_str(st) == name
+    assert abi.ttt_status_str(99) == "TTT_ERR_UNKNOWN"
+    assert abi.ttt_version() == 100
+    assert ctypes.sizeof(abi.ttt_desc) == 15 * 4
+
+
+def lm_desc(**kw):
+    base = dict(B=2, H=4, N=32768, h=256, m=512, chunk=2048, dtype=abi.TTT_DTYPE_BF16)
+    base.update(kw)
+    return abi.ttt_desc(**base)
+
+
+def test_workspace_sizes():
+    par = abi.ttt_workspace_bytes(lm_desc(), abi.TTT_PATH_PARALLEL)
+    # Wk + [A|B] fp32 + two feature buffers + fp32 deltas + bf16 chunk states
+    BH, N, h, m, C = 8, 32768, 256, 512, 16
+    expect = 2 * 2 * m * h * 4 + BH * N * 2 * m * 4 + 2 * (2 * BH * N * m) + BH * C * m * h * 6
+    assert expect <= par <= expect + 6 * 256
+    assert abi.ttt_workspace_bytes(lm_desc(N=65536), 0) > par
+    rec = abi.ttt_workspace_bytes(lm_desc(update_mask=7, renorm=1), abi.TTT_PATH_RECURRENT)
+    assert rec > 0
+    with_ns = abi.ttt_workspace_bytes(lm_desc(update_mask=7, ns_steps=5, momentum=1), 1)
+    assert with_ns > rec
+    # invalid descriptions size to 0
+    assert abi.ttt_workspace_bytes(lm_desc(sign=0), 0) == 0
+    assert abi.ttt_workspace_bytes(lm_desc(update_mask=7), 0) == 0      # parallel takes no mask
+    assert abi.ttt_workspace_bytes(lm_desc(), 1) == 0                   # recurrent needs a mask
+    assert abi.ttt_workspace_bytes(lm_desc(), 7) == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("sign", 0, abi.TTT_ERR_INVALID_ARG),
+    ("dtype", 5, abi.TTT_ERR_INVALID_ARG),
+    ("order", 2, abi.TTT_ERR_INVALID_ARG),
+    ("h", 0, abi.TTT_ERR_INVALID_ARG),
+    ("chunk", 0, abi.TTT_ERR_INVALID_ARG),
+    ("N", -1, abi.TTT_ERR_INVALID_ARG),
+    ("renorm", 1, abi.TTT_ERR_INVALID_ARG),
+    ("w_in_layout", 2, abi.TTT_ERR_INVALID_ARG),
+    ("h", 100, abi.TTT_ERR_UNSUPPORTED),   # bf16 needs multiples of 8
+])
+def test_parallel_rejects_bad_desc(field, value, status):
+    d = lm_desc(**{field: value})
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_la_parallel_fwd(d, 256, 256, 256, 256, 256, 256, 256, 256, None, 256, 1 << 40,
+                                stream=0)
+    assert ei.value.status == status
+
+
+def test_parallel_rejects_pointers_and_workspace():
+    d = lm_desc()
+    need = abi.ttt_workspace_bytes(d, 0)
+    with pytest.raises(abi.TTTError) as ei:   # NULL q
+        abi.ttt_la_parallel_fwd(d, None, 256, 256, 256, 256, 256, 256, 256, None, 256, need,
+                                stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    with pytest.raises(abi.TTTError) as ei:   # misaligned k
+        abi.ttt_la_parallel_fwd(d, 256, 258, 256, 256, 256, 256, 256, 256, None, 256, need,
+                                stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    with pytest.raises(abi.TTTError) as ei:   # workspace too small
+        abi.ttt_la_parallel_fwd(d, 256, 256, 256, 256, 256, 256, 256, 256, None, 256, need - 1,
+                                stream=0)
+    assert ei.value.status == abi.TTT_ERR_WORKSPACE
+    with pytest.raises(abi.TTTError) as ei:   # misaligned workspace
+        abi.ttt_la_parallel_fwd(d, 256, 256, 256, 256, 256, 256, 256, 256, None, 272, need,
+                                stream=0)
+    assert ei.value.status == abi.TTT_ERR_WORKSPACE
+    assert "256-byte" in abi.ttt_last_error_message()
+
+
+def test_recurrent_rejects_bad_args():
+    d = lm_desc(update_mask=7, momentum=1)
+    need = abi.ttt_workspace_bytes(d, 1)
+    with pytest.raises(abi.TTTError) as ei:   # momentum without alpha
+        abi.ttt_lact_recurrent_fwd(d, 256, 256, 256, 256, None, 256, 256, 256, 256, None, None,
+                                   None, None, 256, need, stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    d2 = lm_desc(update_mask=7, w1_layout=1)
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_lact_recurrent_fwd(d2, 256, 256, 256, 256, None, 256, 256, 256, 256, None, None,
+                                   None, None, 256, 1 << 40, stream=0)
+    assert ei.value.status == abi.TTT_ERR_UNSUPPORTED
+    for bad in (dict(update_mask=8), dict(update_mask=7, ns_steps=9)):
+        with pytest.raises(abi.TTTError):
+            abi.ttt_lact_recurrent_fwd(lm_desc(**bad), 256, 256, 256, 256, None, 256, 256, 256,
+                                       256, None, None, None, None, 256, 1 << 40, stream=0)
+
+
+def test_empty_batch_is_a_no_op():
+    # B * H == 0 returns before touching the device.
+    abi.ttt_la_parallel_fwd(lm_desc(B=0), None, None, None, None, None, None, None, None, None,
+                            None, 0, stream=0)
+    abi.ttt_lact_recurrent_fwd(lm_desc(H=0, update_mask=7), None, None, None, None, None, None,
+                               None, None, None, None, None, None, None, None, 0, stream=0)
+
+
+def test_lm_target_host_checks():
+    assert abi.ttt_lm_target_workspace_bytes(32768, 4096) >= 2 * 32768 * 4096
+    assert abi.ttt_lm_target_workspace_bytes(-1, 8) == 0
+    abi.ttt_lm_target(0, 64, None, None, None, None, None, 0, stream=0)   # empty: no-op
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_lm_target(16, 12, 256, 256, 256, 256, 256, 1 << 20, stream=0)
+    assert ei.value.status == abi.TTT_ERR_UNSUPPORTED
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_debug_wait_timeout(10, stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG

@@ -1,0 +1,246 @@
+"""GPU parity of the C-ABI path against the fp64 oracle on small seeded inputs.
+
+Sizes are chosen so that the oracle finishes in seconds while the GPU kernels still run
+several tiles with ragged edges (m and N not multiples of the 128-row tiles, a short last
+chunk, N < chunk). Tolerance: max|err| / max|ref| <= 1e-4 (fp32 mode) / 2e-2 (bf16 mode).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import ttt_oracle as O
+from test_weight_layers_ttt_b200 import abi, layer
+from ttt_inputs import WORKLOADS, make_layer_inputs, make_inplace_inputs
+
+from gpu_helpers import TOL, dev, host, rel, torch_dtype
+
+pytestmark = pytest.mark.gpu
+
+ORD = {"update_apply": O.UPDATE_APPLY, "apply_update": O.APPLY_UPDATE}
+
+
+def layer_inputs(kind, dtype, B, H, N, h, m, chunk, seed, momentum=False):
+    base = WORKLOADS["tiny" if kind == "tiny" else "lm"]
+    wl = base.scaled(B=B, H=H, N=N, h=h, m=m, chunk=chunk, dtype=dtype, momentum=momentum)
+    return wl, make_layer_inputs(wl, seed=seed)
+
+
+def gpu_args(inp, dtype):
+    td = torch_dtype(dtype)
+    return (dev(inp["q"], td), dev(inp["k"], td), dev(inp["v"], td), dev(inp["eta"]),
+            dev(inp["W0"]), dev(inp["W2"]), dev(inp["W1"]))
+
+
+# ----------------------------------------------------------------------------- parallel
+PAR_CASES = [
+    # kind, dtype, B, H, N, h, m, chunk
+    ("tiny", "fp32", 1, 1, 256, 16, 16, 64),
+    ("tiny", "fp32", 2, 2, 203, 12, 20, 50),
+    ("lm", "bf16", 2, 3, 1000, 64, 200, 256),
+    ("lm", "bf16", 1, 2, 640, 128, 512, 128),
+    ("lm", "bf16", 1, 1, 300, 256, 256, 512),
+]
+
+
+@pytest.mark.parametrize("case", PAR_CASES, ids=lambda c: "-".join(map(str, c)))
+@pytest.mark.parametrize("order", ["update_apply", "apply_update"])
+def test_parallel_matches_oracle(case, order):
+    kind, dtype, B, H, N, h, m, chunk = case
+    wl, inp = layer_inputs(kind, dtype, B, H, N, h, m, chunk, seed=1000 + N)
+    ref, Sref = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
+                                      inp["W2"], inp["W1"], chunk, order=ORD[order])
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, dtype)
+    out, S = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk, order=order)
+    abi.ttt_last_device_status()
+    tol = TOL[dtype]
+    assert rel(host(out), ref) <= tol
+    assert rel(host(S), Sref) <= tol
+    # the state-driven part alone: start from a zero state
+    Z = np.zeros_like(inp["W1"])
+    ref0, Sref0 = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
+                                        inp["W2"], Z, chunk, order=ORD[order])
+    out0, S0 = layer.la_parallel_fwd(q, k, v, eta, W0, W2, dev(Z), chunk, order=order)
+    assert rel(host(out0), ref0) <= tol
+    assert rel(host(S0), Sref0) <= tol
+
+
+def test_parallel_ascent_equals_descent_with_negated_values():
+    wl, inp = layer_inputs("lm", "bf16", 1, 2, 512, 64, 128, 128, seed=7)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    a, Sa = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, 128, sign=-1)
+    d, Sd = layer.la_parallel_fwd(q, k, (-v).contiguous(), eta, W0, W2, W1, 128, sign=1)
+    assert torch.equal(a, d) and torch.equal(Sa, Sd)
+
+
+def test_parallel_edge_sizes():
+    wl, inp = layer_inputs("lm", "bf16", 1, 2, 64, 64, 128, 128, seed=11)   # N < chunk
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    out, S = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, 128)
+    ref, Sref = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
+                                      inp["W2"], inp["W1"], 128)
+    assert rel(host(out), ref) <= TOL["bf16"] and rel(host(S), Sref) <= TOL["bf16"]
+    # N = 0: no output rows, the final state is the initial one (per (b, head))
+    e = torch.empty((1, 2, 0, 64), dtype=torch.bfloat16, device="cuda")
+    eta0 = torch.empty((1, 2, 0), dtype=torch.float32, device="cuda")
+    _, S0 = layer.la_parallel_fwd(e, e, e, eta0, W0, W2, W1, 128)
+    assert torch.equal(S0[0], W1)
+    # chunk = 1 (per-token) in fp32 mode
+    wl, inp = layer_inputs("tiny", "fp32", 1, 1, 40, 8, 12, 1, seed=12)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "fp32")
+    out, S = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, 1)
+    ref, Sref = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
+                                      inp["W2"], inp["W1"], 1)
+    assert rel(host(out), ref) <= TOL["fp32"] and rel(host(S), Sref) <= TOL["fp32"]
+    abi.ttt_last_device_status()
+
+
+def test_parallel_rejects_misaligned_pointer_on_device():
+    wl, inp = layer_inputs("lm", "bf16", 1, 1, 128, 64, 128, 64, seed=13)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    desc = layer.parallel_desc(q, W1, 64)
+    ws = layer.workspace(abi.ttt_workspace_bytes(desc, 0), "cuda")
+    out = torch.empty_like(q)
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_la_parallel_fwd(desc, q.data_ptr() + 2, k, v, eta, W0, W2, W1, out, None, ws)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- recurrent
+REC_CASES = [
+    # kind, dtype, B, H, N, h, m, chunk, opts
+    ("tiny", "fp32", 1, 1, 256, 16, 16, 64, dict()),
+    ("tiny", "fp32", 1, 2, 150, 16, 24, 40, dict(renorm=True, momentum=True, ns_steps=5)),
+    ("lm", "bf16", 1, 2, 768, 64, 128, 256, dict(renorm=True)),
+    ("lm", "bf16", 2, 1, 600, 128, 256, 256, dict(renorm=True, momentum=True, ns_steps=5)),
+    ("lm", "bf16", 1, 2, 512, 64, 192, 128, dict(update_mask=abi.TTT_UPDATE_W1)),
+    ("lm", "bf16", 1, 1, 512, 128, 64, 256, dict(update_mask=5, ns_steps=5)),
+]
+
+
+@pytest.mark.parametrize("case", REC_CASES, ids=lambda c: "-".join(map(str, c[:8])))
+@pytest.mark.parametrize("order", ["update_apply", "apply_update"])
+def test_recurrent_matches_oracle(case, order):
+    kind, dtype, B, H, N, h, m, chunk, opts = case
+    momentum = opts.get("momentum", False)
+    wl, inp = layer_inputs(kind, dtype, B, H, N, h, m, chunk, seed=2000 + N, momentum=momentum)
+    mask = opts.get("update_mask", 7)
+    upd = tuple(n for bit, n in ((1, "W0"), (2, "W1"), (4, "W2")) if mask & bit)
+    ref, Wref, Mref = O.lact_recurrent_batched(
+        inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"], inp["W2"], inp["W1"], chunk,
+        order=ORD[order], update=upd, renorm=opts.get("renorm", False),
+        alpha=inp["alpha"] if momentum else None, ns_steps=opts.get("ns_steps", 0))
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, dtype)
+    alpha = dev(inp["alpha"]) if momentum else None
+    out, Wf, M = layer.lact_recurrent_fwd(q, k, v, eta, W0, W2, W1, chunk, order=order,
+                                          update_mask=mask, renorm=opts.get("renorm", False),
+                                          alpha=alpha, ns_steps=opts.get("ns_steps", 0),
+                                          return_momentum=momentum)
+    abi.ttt_last_device_status()
+    tol = TOL[dtype]
+    assert rel(host(out), ref) <= tol
+    for got, name in zip(Wf, ("W0", "W2", "W1")):
+        assert rel(host(got), Wref[name]) <= tol, name
+        # the change of each fast matrix, relative to the oracle's change
+        init = inp[name][None].repeat(B, axis=0)
+        if name in upd:
+            assert rel(host(got) - init, Wref[name] - init) <= 5 * tol, name
+        else:
+            assert np.array_equal(host(got), np.broadcast_to(init, host(got).shape))
+    if momentum:
+        hm = h * m
+        Mh = host(M)
+        for pidx, name in enumerate(("W0", "W1", "W2")):
+            if name in upd:
+                assert rel(Mh[..., pidx * hm:(pidx + 1) * hm].reshape(Mref[name].shape),
+                           Mref[name]) <= 5 * tol, name
+
+
+def test_recurrent_ascent_equals_descent_with_negated_values():
+    wl, inp = layer_inputs("lm", "bf16", 1, 2, 512, 64, 128, 128, seed=21, momentum=True)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    alpha = dev(inp["alpha"])
+    kw = dict(renorm=True, alpha=alpha, ns_steps=5)
+    a, Wa, _ = layer.lact_recurrent_fwd(q, k, v, eta, W0, W2, W1, 128, sign=-1, **kw)
+    d, Wd, _ = layer.lact_recurrent_fwd(q, k, (-v).contiguous(), eta, W0, W2, W1, 128, sign=1,
+                                        **kw)
+    assert torch.equal(a, d)
+    for x, y in zip(Wa, Wd):
+        assert torch.equal(x, y)
+
+
+def test_recurrent_resume_equals_full_run():
+    wl, inp = layer_inputs("lm", "bf16", 1, 2, 1024, 64, 128, 256, seed=22, momentum=True)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    alpha = dev(inp["alpha"])
+    kw = dict(renorm=True, ns_steps=5, return_momentum=True)
+    full, Wf, Mf = layer.lact_recurrent_fwd(q, k, v, eta, W0, W2, W1, 256, alpha=alpha, **kw)
+    h1 = slice(0, 512)
+    h2 = slice(512, 1024)
+    a, Wa, Ma = layer.lact_recurrent_fwd(q[:, :, h1].contiguous(), k[:, :, h1].contiguous(),
+                                         v[:, :, h1].contiguous(), eta[:, :, h1].contiguous(),
+                                         W0, W2, W1, 256, alpha=alpha[:, :, :2].contiguous(), **kw)
+    # resume from the carried state (one batch element: the per-(b, head) weights are the
+    # per-head weights of the next call)
+    b, Wb, Mb = layer.lact_recurrent_fwd(q[:, :, h2].contiguous(), k[:, :, h2].contiguous(),
+                                         v[:, :, h2].contiguous(), eta[:, :, h2].contiguous(),
+                                         Wa[0][0].contiguous(), Wa[1][0].contiguous(),
+                                         Wa[2][0].contiguous(), 256,
+                                         alpha=alpha[:, :, 2:].contiguous(), M_init=Ma, **kw)
+    # renorm targets are the column norms at the start of each call, equal up to rounding
+    assert rel(host(torch.cat([a, b], dim=2)), host(full)) <= TOL["bf16"]
+    for x, y in zip(Wb, Wf):
+        assert rel(host(x), host(y)) <= TOL["bf16"]
+
+
+# ----------------------------------------------------------------------------- In-Place form
+def test_inplace_shaped_update_matches_oracle():
+    """q = k = H, W0 = Wg^T, W2 = Wu^T given as [m,h]; W1 = W_down^T given as [h,m];
+    apply then update with constant eta (In-Place TTT, sections 3.1 and 3.4)."""
+    wl = WORKLOADS["inplace"].scaled(N=640, h=256, m=384, chunk=128)
+    inp = make_inplace_inputs(wl, seed=31)
+    Vbar = O.lm_target(inp["X0"], inp["conv_w"], inp["W_target"])
+    ref, Wref = O.inplace_sequential(inp["Hs"], inp["Wg"], inp["Wu"], inp["W_down"], Vbar,
+                                     wl.chunk, 1e-3)
+    Hs = dev(inp["Hs"], torch.bfloat16)[None, None]
+    vb = layer.lm_target(dev(inp["X0"], torch.bfloat16), dev(inp["conv_w"]),
+                         dev(inp["W_target"], torch.bfloat16))
+    assert rel(host(vb), Vbar) <= TOL["bf16"]
+    eta = torch.full((1, 1, wl.N), 1e-3, dtype=torch.float32, device="cuda")
+    out, S = layer.la_parallel_fwd(Hs, Hs, vb[None, None].contiguous(), eta,
+                                   dev(inp["Wg"])[None], dev(inp["Wu"])[None],
+                                   dev(inp["W_down"])[None], wl.chunk, order="apply_update",
+                                   w_in_layout=1, w1_layout=1)
+    abi.ttt_last_device_status()
+    assert rel(host(out[0, 0]), ref) <= TOL["bf16"]
+    assert rel(host(S[0, 0]), Wref) <= TOL["bf16"]
+    assert rel(host(S[0, 0]) - inp["W_down"], Wref - inp["W_down"]) <= TOL["bf16"]
+
+
+def test_lm_target_matches_oracle():
+    rng = np.random.Generator(np.random.PCG64(41))
+    N, d = 300, 64
+    from ttt_inputs import bf16_round
+    X0 = bf16_round(rng.standard_normal((N, d), dtype=np.float32))
+    cw = rng.standard_normal((4, d), dtype=np.float32)
+    Wt = bf16_round((rng.standard_normal((d, d)) / 8).astype(np.float32))
+    got = layer.lm_target(dev(X0, torch.bfloat16), dev(cw), dev(Wt, torch.bfloat16))
+    assert rel(host(got), O.lm_target(X0, cw, Wt)) <= TOL["bf16"]
+    shift = np.zeros((4, d), np.float32)
+    shift[1] = 1.0
+    got = layer.lm_target(dev(X0, torch.bfloat16), dev(shift),
+                          dev(np.eye(d, dtype=np.float32), torch.bfloat16))
+    assert np.array_equal(host(got)[1:], X0[:-1]) and not host(got)[0].any()
+
+
+# ----------------------------------------------------------------------------- failure path
+def test_bounded_wait_reports_timeout_and_context_survives():
+    abi.ttt_debug_wait_timeout(2_000_000)   # 2 ms: the barrier is never completed
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_last_device_status()
+    assert ei.value.status == abi.TTT_ERR_TIMEOUT
+    abi.ttt_last_device_status()            # the word was cleared
+    wl, inp = layer_inputs("tiny", "fp32", 1, 1, 64, 16, 16, 32, seed=51)
+    out, _ = layer.la_parallel_fwd(*gpu_args(inp, "fp32"), 32)
+    ref, _ = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
+                                   inp["W2"], inp["W1"], 32)
+    assert rel(host(out), ref) <= TOL["fp32"]
