@@ -1,0 +1,522 @@
+#!/usr/bin/env python
+"""Benchmark of the chunked TTT-KVB layer on B200: TTT-layer tokens/s of the parallel and
+the recurrent form, and the fraction of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload lm] [--impl reference]
+
+A step is one pass of the layer over one batch of the workload with inputs resident in
+HBM. The headline ``value`` is the parallel form's tokens/s summed over all ranks; the
+recurrent form is timed the same way and reported under ``forms``. With N > 1 (launched
+by torchrun) every rank runs its own replica of the workload (independent (batch, head)
+problems, no collective on the data path): weak scaling, time = max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload
+(the pages ship no runnable implementation); only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "TTT-layer tokens/sec at 1 B200 (parallel vs recurrent) and % of roofline"
+L2_BYTES = 126 * 2 ** 20
+
+
+# ----------------------------------------------------------------------------- cost model
+def state_size(d: int, n_heads: int, r: int) -> int:
+    """Fast-weight elements of one LaCT layer: three matrices of h x rh per head,
+    n_heads heads, h = d / n_heads  ->  3 r d^2 / n_heads."""
+    return 3 * r * d * d // n_heads
+
+
+def layer_flops(wl, form: str) -> float:
+    """Algorithmic FLOPs of one pass of the layer over the workload (matmuls only)."""
+    T = wl.B * wl.H * wl.N
+    hm = wl.h * wl.m
+    if form == "parallel":
+        feats = 4 * hm * T if wl.kind == "inplace" else 8 * hm * T   # q == k: once
+        return float(feats + 2 * hm * T + 2 * hm * T)
+    flops = 18.0 * hm * T   # 9 matmuls: K features (2), D, 3 gradients, Q features (2), out
+    if wl.ns_steps:
+        r, c = min(wl.h, wl.m), max(wl.h, wl.m)
+        per = wl.ns_steps * (2 * r * r * c + 2 * r ** 3 + 2 * r * r * c)
+        flops += 3.0 * per * wl.B * wl.H * wl.C
+    return flops
+
+
+def layer_bytes(wl, form: str) -> float:
+    """Algorithmic HBM bytes: each input read once, each output written once, weights."""
+    es = 2 if wl.dtype == "bf16" else 4
+    T = wl.B * wl.H * wl.N
+    hm = wl.h * wl.m
+    n_in = 1 if wl.kind == "inplace" else 2          # q and k (aliased for in-place)
+    act = (n_in + 1) * T * wl.h * es + T * wl.h * es + T * 4      # q,k,v in, O out, eta
+    weights = 3 * hm * 4 * wl.H
+    state_out = hm * 4 * wl.B * wl.H
+    return float(act + weights + state_out)
+
+
+def kernel_work(name: str, wl, calls: int):
+    """(bound, algorithmic work per launch) of a traced kernel; work in FLOP or bytes."""
+    base = name.split("@")[0]
+    BH, N, h, m = wl.B * wl.H, wl.N, wl.h, wl.m
+    rows_par = BH * N
+    C = wl.C
+    es = 2 if wl.dtype == "bf16" else 4
+    if wl_form(name) == "recurrent":
+        rows = BH * wl.chunk
+        table = {
+            "gemm_features_k": ("tensor", 4.0 * h * m * rows),
+            "gemm_features_q": ("tensor", 4.0 * h * m * rows),
+            "gemm_v_w1t": ("tensor", 2.0 * h * m * rows),
+            "gemm_grad_w1": ("tensor", 2.0 * h * m * rows),
+            "gemm_grad_w0": ("tensor", 2.0 * h * m * rows),
+            "gemm_grad_w2": ("tensor", 2.0 * h * m * rows),
+            "gemm_output": ("tensor", 2.0 * h * m * rows),
+        }
+        return table.get(base, (None, None))
+    table = {
+        "gemm_features_k": ("tensor", 4.0 * h * m * rows_par),
+        "gemm_features_q": ("tensor", 4.0 * h * m * rows_par),
+        "gemm_state_delta": ("tensor", 2.0 * h * m * rows_par),
+        "gemm_output": ("tensor", 2.0 * h * m * rows_par),
+        "chunk_scan": ("hbm", BH * C * h * m * (4.0 + es) + 2 * 4.0 * BH * h * m),
+        "swiglu_k": ("hbm", rows_par * m * (8.0 + es * (1 if wl.kind != "inplace" else 2))),
+        "swiglu_q": ("hbm", rows_par * m * (8.0 + es)),
+    }
+    return table.get(base, (None, None))
+
+
+_FORM_OF_TRACE = {}
+
+
+def wl_form(name):
+    return _FORM_OF_TRACE.get(name, "parallel")
+
+
+# ----------------------------------------------------------------------------- environment
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained",
+                                                     p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id(local, torch):
+    """nvidia-smi selector of the torch device: its UUID when torch exposes it."""
+    try:
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        if u:
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    return str(local)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = [d for d in threadpool_info() if d.get("user_api") == "blas"]
+        if info:
+            return int(max(d.get("num_threads", 1) for d in info))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- ranks
+def dist_setup(ngpus: int, backend: str):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, local, world
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput: units every rank processed divided by the slowest rank's time."""
+    return units_per_rank * world / seconds
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def _gpu_inputs(wl, seed, torch):
+    from ttt_inputs import make_layer_inputs
+    x = make_layer_inputs(wl, seed=seed)
+    td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+    def dev(a, dt=torch.float32):
+        return torch.from_numpy(a).cuda().to(dt).contiguous()
+
+    g = {n: dev(x[n], td) for n in ("q", "k", "v")}
+    g.update({n: dev(x[n]) for n in ("eta", "W0", "W2", "W1")})
+    g["alpha"] = dev(x["alpha"]) if x["alpha"] is not None else None
+    return x, g
+
+
+def _timed(fn, steps, warmup, world, torch, trace_capacity=0):
+    from test_weight_layers_ttt_b200 import abi
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    if trace_capacity:
+        abi.ttt_trace_enable(trace_capacity)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    barrier(world)
+    torch.cuda.synchronize()
+    trace = []
+    if trace_capacity:
+        n = abi.ttt_trace_count()
+        trace = [abi.ttt_trace_get(i) for i in range(n)]
+        abi.ttt_trace_disable()
+    return ms, trace
+
+
+def _kernel_table(trace, steps):
+    tot = sum(ms for _, ms in trace) or 1.0
+    table = {}
+    for name, ms in trace:
+        e = table.setdefault(name, {"launches": 0, "ms_total": 0.0})
+        e["launches"] += 1
+        e["ms_total"] += ms
+    for e in table.values():
+        e["share"] = e["ms_total"] / tot
+        e["ms_avg"] = e["ms_total"] / e["launches"]
+    return dict(sorted(table.items(), key=lambda kv: -kv[1]["ms_total"]))
+
+
+def _roofline(table, wl, peaks, form):
+    """Roofline of the dominant kernel (largest share) with a known algorithmic work."""
+    for name, e in table.items():
+        _FORM_OF_TRACE[name] = form
+        bound, work = kernel_work(name, wl, e["launches"])
+        if bound is None:
+            continue
+        secs = e["ms_avg"] / 1e3
+        if bound == "tensor":
+            achieved = work / secs / 1e12
+            peak = peaks["bf16_tflops"]
+            unit = "TFLOP/s"
+        else:
+            achieved = work / secs / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        return {"kernel": name, "bound": "tensor" if bound == "tensor" else "hbm",
+                "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "work_per_launch": work, "share": round(e["share"], 4),
+                "peak_source": peaks["source"] + " (burst)"}
+    return None
+
+
+def run_gpu(args, rank, local, world):
+    import torch
+
+    from test_weight_layers_ttt_b200 import abi, layer
+    from ttt_inputs import WORKLOADS
+
+    torch.cuda.set_device(local)
+    wl = WORKLOADS[args.workload]
+    peaks = load_peaks()
+    x, g = _gpu_inputs(wl, wl.seed + rank, torch)
+    tokens = wl.B * wl.N
+    result = {"forms": {}}
+
+    # ---- parallel form (headline)
+    forms = [f for f in ("parallel", "recurrent") if f in wl.paths]
+    for form in forms:
+        if form == "parallel":
+            desc = layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order)
+            ws = layer.workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_PARALLEL), "cuda")
+            out = torch.empty_like(g["q"])
+            S = torch.empty((wl.B, wl.H, wl.m, wl.h), dtype=torch.float32, device="cuda")
+
+            def step():
+                abi.ttt_la_parallel_fwd(desc, g["q"], g["k"], g["v"], g["eta"], g["W0"],
+                                        g["W2"], g["W1"], out, S, ws)
+        else:
+            desc = layer.recurrent_desc(g["q"], g["W1"], wl.chunk, wl.order, 1, 7, wl.renorm,
+                                        wl.momentum, wl.ns_steps)
+            ws = layer.workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_RECURRENT), "cuda")
+            out = torch.empty_like(g["q"])
+
+            def step():
+                abi.ttt_lact_recurrent_fwd(desc, g["q"], g["k"], g["v"], g["eta"], g["alpha"],
+                                           g["W0"], g["W2"], g["W1"], out, None, None, None,
+                                           None, ws)
+        steps = args.steps if form == "parallel" else max(3, args.steps // 2)
+        with ClockSampler(gpu_id(local, torch)) as clk:
+            ms, trace = _timed(step, steps, args.warmup, world, torch, trace_capacity=16384)
+        abi.ttt_last_device_status()
+        ms_max = max_over_ranks(ms, world, "cuda")
+        per_step = ms_max / steps
+        table = _kernel_table(trace, steps)
+        flops, nbytes = layer_flops(wl, form), layer_bytes(wl, form)
+        t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+        result["forms"][form] = {
+            "tokens_per_s": job_throughput(tokens, world, per_step / 1e3),
+            "ms_per_step": per_step, "steps": steps,
+            "flop_per_step": flops, "bytes_per_step": nbytes,
+            "roofline_frac": t_roof / (per_step / 1e3),
+            "roofline_frac_sustained": max(
+                flops / (peaks["bf16_tflops_sustained"] * 1e12),
+                nbytes / (peaks["hbm_gbs"] * 1e9)) / (per_step / 1e3),
+            "gpu_launches": len(trace),
+            "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv)
+                            for kk, vv in v.items()} for k, v in table.items()},
+            "roofline": _roofline(table, wl, peaks, form),
+            "clocks": clk.summary(),
+        }
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region
+    e2e = None
+    if "parallel" in forms:
+        hq = {n: g[n].cpu().pin_memory() for n in ("q", "k", "v", "eta")}
+        dq = {n: torch.empty_like(g[n]) for n in ("q", "k", "v", "eta")}
+        hout = torch.empty(g["q"].shape, dtype=g["q"].dtype).pin_memory()
+        dout = torch.empty_like(g["q"])
+        ws = layer.workspace(abi.ttt_workspace_bytes(
+            layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order), 0), "cuda")
+
+        def e2e_step():
+            for n in dq:
+                dq[n].copy_(hq[n], non_blocking=True)
+            layer.la_parallel_fwd(dq["q"], dq["k"], dq["v"], dq["eta"], g["W0"], g["W2"],
+                                  g["W1"], wl.chunk, order=wl.order, return_state=False,
+                                  out=dout, ws=ws)
+            hout.copy_(dout, non_blocking=True)
+
+        steps = max(3, args.steps // 2)
+        ms, _ = _timed(e2e_step, steps, args.warmup, world, torch)
+        ms = max_over_ranks(ms, world, "cuda")
+        h2d = sum(t.numel() * t.element_size() for t in hq.values())
+        d2h = hout.numel() * hout.element_size()
+        e2e = {"value": job_throughput(tokens, world, ms / steps / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ms / steps}
+    result["e2e"] = e2e
+    return wl, peaks, result, x
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_time(wl, x, n: int, form: str = "parallel") -> float:
+    """Seconds the fp64 oracle takes for the first ``n`` tokens of (b=0, head=0)."""
+    from oracle import ttt_oracle as O
+    q, k, v, eta = (x[name][0, 0, :n].astype("float64") for name in ("q", "k", "v", "eta"))
+    W0, W2, W1 = x["W0"][0], x["W2"][0], x["W1"][0]
+    t0 = time.perf_counter()
+    if form == "parallel":
+        O.la_parallel(q, k, v, eta, W0, W2, W1, wl.chunk, order=wl.order)
+    else:
+        alpha = x["alpha"][0, 0] if x.get("alpha") is not None else None
+        O.lact_recurrent(q, k, v, eta, W0, W2, W1, wl.chunk, order=wl.order, renorm=wl.renorm,
+                         alpha=alpha, ns_steps=wl.ns_steps)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(wl, x, target_s: float, form: str = "parallel"):
+    """Time the fp64 oracle on (b=0, head=0) with as many leading whole chunks as fit about
+    ``target_s`` seconds; returns (tokens, seconds, description)."""
+    n = min(wl.N, wl.chunk)
+    t = oracle_time(wl, x, n, form)
+    if t < target_s / 2 and n < wl.N:
+        n2 = min(wl.N, max(wl.chunk, int(n * target_s / max(t, 1e-3)) // wl.chunk * wl.chunk))
+        if n2 > n:
+            n, t = n2, oracle_time(wl, x, n2, form)
+    desc = (f"{form} form, fp64 oracle, one (batch, head) of the '{wl.name}' workload, "
+            f"first {n} of {wl.N} tokens")
+    return n, t, desc
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle as it stands, on bounded samples."""
+    from ttt_inputs import WORKLOADS, make_layer_inputs
+    wl = WORKLOADS[args.workload]
+    x = make_layer_inputs(wl.scaled(B=1, H=1), seed=wl.seed)
+    form = "parallel" if "parallel" in wl.paths else "recurrent"
+    n, t, desc = oracle_sample(wl, x, 2.0, form)
+    times = []
+    for i in range(args.warmup + args.steps):
+        ti = oracle_time(wl, x, n, form)
+        if i >= args.warmup:
+            times.append(ti)
+    secs = sum(times)
+    value = n * len(times) / secs
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / len(times) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, form),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def workload_config(wl, form):
+    return {"workload": wl.name, "form": form, "B": wl.B, "H": wl.H, "N": wl.N, "h": wl.h,
+            "m": wl.m, "chunk": wl.chunk, "order": wl.order, "renorm": wl.renorm,
+            "momentum": wl.momentum, "ns_steps": wl.ns_steps, "parallelism": "replicas",
+            "l2": "no flush: the per-step inputs exceed the 126 MB L2"}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="lm")
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target seconds of the CPU oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+
+    import torch
+    rank, local, world = dist_setup(args.gpus, "nccl" if torch.cuda.is_available() else "gloo")
+    from test_weight_layers_ttt_b200 import build as tbuild
+    if not os.path.exists(tbuild.LIB_PATH):
+        tbuild.build()
+    wl, peaks, res, x = run_gpu(args, rank, local, world)
+    if rank == 0:
+        form = "parallel" if "parallel" in res["forms"] else "recurrent"
+        head = res["forms"][form]
+        line = {
+            "metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s",
+            "n_gpus": world, "steps": head["steps"], "warmup": args.warmup,
+            "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": workload_config(wl, form),
+            "roofline": head["roofline"],
+            "step_roofline_frac": head["roofline_frac"],
+            "gpu_launches": sum(f["gpu_launches"] for f in res["forms"].values()),
+            "clocks": head["clocks"],
+            "e2e": res["e2e"],
+            "forms": res["forms"],
+        }
+        if "parallel" in res["forms"] and "recurrent" in res["forms"]:
+            line["parallel_over_recurrent"] = (res["forms"]["parallel"]["tokens_per_s"] /
+                                               res["forms"]["recurrent"]["tokens_per_s"])
+        if world == 1 and not args.no_cpu_baseline:
+            n, secs, desc = oracle_sample(wl, x, args.cpu_seconds, form)
+            line["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s",
+                                    "cores": blas_threads(), "kind": "oracle", "sample": desc}
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,75 @@
+"""Host-side logic of bench.py: the cost model against numbers the pages print, and the
+multi-rank timing reduction (max over ranks, whole-job throughput) with 2 gloo ranks."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+from ttt_inputs import WORKLOADS
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "state_size.txt")
+
+
+def test_state_size_matches_pages():
+    rows = [l.split() for l in open(GOLDEN) if l.strip() and not l.startswith("#")]
+    assert rows
+    for d, nh, r, layers, expect in rows:
+        assert bench.state_size(int(d), int(nh), int(r)) * int(layers) == int(expect)
+    assert abs(bench.state_size(768, 1, 2) * 24 / 1e6 - 84.9) < 0.05
+    assert bench.state_size(768, 4, 1) == 0.75 * 768 ** 2
+
+
+@pytest.mark.parametrize("name", ["lm", "nvs", "tiny"])
+def test_recurrent_flops_are_six_n_s(name):
+    wl = WORKLOADS[name].scaled(ns_steps=0)
+    n = wl.B * wl.N                                  # tokens through the layer
+    S = bench.state_size(wl.H * wl.h, wl.H, wl.m // wl.h)
+    assert bench.layer_flops(wl, "recurrent") == 6 * n * S
+
+
+def test_parallel_flops_and_bytes():
+    wl = WORKLOADS["lm"]
+    T = wl.B * wl.H * wl.N
+    assert bench.layer_flops(wl, "parallel") == 12 * wl.h * wl.m * T
+    ip = WORKLOADS["inplace"]
+    assert bench.layer_flops(ip, "parallel") == 8 * ip.h * ip.m * ip.N   # features once
+    # q, k, v in and O out (bf16), eta, weights, final state
+    expect = 4 * T * wl.h * 2 + 4 * T + 3 * wl.h * wl.m * 4 * wl.H + wl.h * wl.m * 4 * wl.B * wl.H
+    assert bench.layer_bytes(wl, "parallel") == expect
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, local, w = bench.dist_setup(world, "gloo")
+    ms = 10.0 + 5.0 * r                        # rank 1 is the slow one
+    slowest = bench.max_over_ranks(ms, w)
+    value = bench.job_throughput(65536, w, slowest / 1e3)
+    bench.barrier(w)
+    import torch.distributed as dist
+    dist.destroy_process_group()
+    q.put((r, w, slowest, value))
+
+
+def test_max_over_ranks_with_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r, w, slowest, value in res:
+        assert w == 2 and slowest == 15.0
+        assert value == pytest.approx(2 * 65536 / 0.015)
