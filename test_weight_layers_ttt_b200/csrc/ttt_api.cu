@@ -6,7 +6,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <string>
 #include <vector>
 
 #include "gemm.h"
@@ -88,17 +90,28 @@ bool force_simt() {
   return s && strcmp(s, "simt") == 0;
 }
 
+// "<name>@<engine>" with stable storage, for trace records.
+const char* engine_name(const char* name, const char* engine) {
+  static std::mutex mu;
+  static std::map<std::string, std::string> names;
+  std::lock_guard<std::mutex> lk(mu);
+  std::string key = std::string(name) + "@" + engine;
+  auto it = names.find(key);
+  if (it == names.end()) it = names.emplace(key, key).first;
+  return it->second.c_str();
+}
+
 ttt_status run_gemm(const char* name, const GemmProblem& p, cudaStream_t s) {
   if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
-  TraceScope ts(name, s);
-  if (p.K > 0 && !force_simt() && umma_supported(p))
-    return gemm_umma(p, s, device_error_word(), wait_limit_ns());
+  const bool tc = p.K > 0 && !force_simt() && umma_supported(p);
+  TraceScope ts(g_trace.on ? engine_name(name, tc ? "tcgen05" : "simt") : name, s);
+  if (tc) return gemm_umma(p, s, device_error_word(), wait_limit_ns());
   return gemm_simt(p, s);
 }
 
 ttt_status run_simt(const char* name, const GemmProblem& p, cudaStream_t s) {
   if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
-  TraceScope ts(name, s);
+  TraceScope ts(g_trace.on ? engine_name(name, "simt") : name, s);
   return gemm_simt(p, s);
 }
 
