@@ -124,6 +124,32 @@ ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* 
                                ttt_stream_t stream);
 
 /*
+ * Parallel form for callers that cannot allocate device memory. No paper counterpart:
+ * same arguments and results as ttt_la_parallel_fwd, minus the workspace. Some callers
+ * have no way to obtain device memory of their own: a plug-in hosted by a runtime that
+ * owns every device allocation and hands out none, or a real-time loop that must not call
+ * cudaMalloc after start-up because an allocation can synchronise the device and stall
+ * other streams. For them the scratch lives in one array built into the library,
+ * TTT_STATIC_SCRATCH_BYTES (64 MiB) per device, reserved on every GPU that loads the
+ * library until the process exits.
+ *
+ * - Problems whose workspace (ttt_workspace_bytes(desc, TTT_PATH_PARALLEL)) exceeds
+ *   TTT_STATIC_SCRATCH_BYTES are rejected with TTT_ERR_WORKSPACE; nothing is enqueued.
+ * - The first call on a device looks up that device's copy of the array (with that device
+ *   current); make that first call before any stream capture begins.
+ * - Every call on a device uses the same array. Calls whose work overlaps on the GPU
+ *   (different streams, or different host threads, without ordering between them) race on
+ *   it and give wrong results: order them. No state is carried from one call to the next;
+ *   every scratch byte a call reads it has written earlier in the same call.
+ * - Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library routine.
+ */
+#define TTT_STATIC_SCRATCH_BYTES (64ull << 20)
+ttt_status ttt_la_parallel_fwd_noalloc(const ttt_desc* desc, const void* q, const void* k,
+                                       const void* v, const float* eta, const float* W0,
+                                       const float* W2, const float* W1, void* out,
+                                       float* S_final, ttt_stream_t stream);
+
+/*
  * Recurrent LaCT form ("Test-Time Training Done Right" notes, sections 2.1-2.3; "Test-Time
  * Training with KV Binding Is Secretly Linear Attention", 前置知识 / LaCT): per chunk, at
  * the chunk-start weights, the gradients

@@ -34,10 +34,12 @@ TTT_UPDATE_W2 = 4
 TTT_UPDATE_ALL = 7
 TTT_PATH_PARALLEL = 0
 TTT_PATH_RECURRENT = 1
+TTT_STATIC_SCRATCH_BYTES = 64 << 20
 
 # Every symbol include/ttt.h declares.
 EXPORTED = (
-    "ttt_workspace_bytes", "ttt_la_parallel_fwd", "ttt_lact_recurrent_fwd",
+    "ttt_workspace_bytes", "ttt_la_parallel_fwd", "ttt_la_parallel_fwd_noalloc",
+    "ttt_lact_recurrent_fwd",
     "ttt_lm_target_workspace_bytes", "ttt_lm_target", "ttt_last_device_status",
     "ttt_debug_wait_timeout", "ttt_trace_enable", "ttt_trace_disable", "ttt_trace_count",
     "ttt_trace_get", "ttt_status_str", "ttt_last_error_message", "ttt_version",
@@ -80,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_workspace_bytes.restype = S
         L.ttt_la_parallel_fwd.argtypes = [D] + [P] * 10 + [S, P]
         L.ttt_la_parallel_fwd.restype = I32
+        L.ttt_la_parallel_fwd_noalloc.argtypes = [D] + [P] * 10
+        L.ttt_la_parallel_fwd_noalloc.restype = I32
         L.ttt_lact_recurrent_fwd.argtypes = [D] + [P] * 14 + [S, P]
         L.ttt_lact_recurrent_fwd.restype = I32
         L.ttt_lm_target_workspace_bytes.argtypes = [I32, I32]
@@ -158,6 +162,14 @@ def ttt_la_parallel_fwd(desc, q, k, v, eta, W0, W2, W1, out, S_final, workspace,
     _check(lib().ttt_la_parallel_fwd(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W0), _ptr(W2), _ptr(W1),
         _ptr(out), _ptr(S_final), _ptr(workspace), wb, _stream(stream)))
+
+
+def ttt_la_parallel_fwd_noalloc(desc, q, k, v, eta, W0, W2, W1, out, S_final, stream=None):
+    """Parallel form using the library's built-in scratch instead of a caller workspace,
+    for callers that cannot allocate device memory (see include/ttt.h)."""
+    _check(lib().ttt_la_parallel_fwd_noalloc(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W0), _ptr(W2), _ptr(W1),
+        _ptr(out), _ptr(S_final), _stream(stream)))
 
 
 def ttt_lact_recurrent_fwd(desc, q, k, v, eta, alpha, W0, W2, W1, out, W0_out, W2_out, W1_out,

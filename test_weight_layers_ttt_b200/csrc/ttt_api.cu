@@ -562,6 +562,58 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   return TTT_OK;
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------ built-in scratch
+// Scratch of ttt_la_parallel_fwd_noalloc: one array per device, part of the library's
+// device image, so the entry point never allocates. Its address is looked up once per
+// device with that device current.
+namespace ttt {
+namespace {
+static __device__ __align__(256) unsigned char g_static_scratch[TTT_STATIC_SCRATCH_BYTES];
+
+ttt_status static_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(TTT_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 128) return fail(TTT_ERR_UNSUPPORTED, "device index %d >= 128", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(TTT_ERR_CUDA, "cudaGetSymbolAddress(built-in scratch): %s",
+                  cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return TTT_OK;
+}
+}  // namespace
+}  // namespace ttt
+
+extern "C" {
+
+ttt_status ttt_la_parallel_fwd_noalloc(const ttt_desc* desc, const void* q, const void* k,
+                                       const void* v, const float* eta, const float* W0,
+                                       const float* W2, const float* W1, void* out,
+                                       float* S_final, ttt_stream_t stream) {
+  TTT_TRY(check_desc(desc, TTT_PATH_PARALLEL));
+  ParBufs b;
+  const size_t need = plan_parallel(*desc, nullptr, b);
+  if (need > TTT_STATIC_SCRATCH_BYTES)
+    return fail(TTT_ERR_WORKSPACE,
+                "problem needs %zu bytes of scratch; the built-in scratch holds %llu bytes "
+                "(use ttt_la_parallel_fwd with a caller workspace)",
+                need, (unsigned long long)TTT_STATIC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  TTT_TRY(static_scratch(&scratch));
+  return ttt_la_parallel_fwd(desc, q, k, v, eta, W0, W2, W1, out, S_final, scratch,
+                             (size_t)TTT_STATIC_SCRATCH_BYTES, stream);
+}
+
 size_t ttt_lm_target_workspace_bytes(int32_t N, int32_t d) {
   if (N < 0 || d < 1) return 0;
   Carve cv(nullptr);
