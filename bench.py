@@ -314,7 +314,7 @@ def run_gpu(args, rank, local, world):
     from ttt_inputs import WORKLOADS
 
     torch.cuda.set_device(local)
-    wl = WORKLOADS[args.workload]
+    wl = workload_from_args(args)
     peaks = load_peaks()
     x, g = _gpu_inputs(wl, wl.seed + rank, torch)
     tokens = wl.B * wl.N
@@ -426,10 +426,22 @@ def oracle_sample(wl, x, target_s: float, form: str = "parallel"):
     return n, t, desc
 
 
+def workload_from_args(args):
+    from ttt_inputs import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if args.override:
+        kw = {}
+        for item in args.override.split(","):
+            key, val = item.split("=")
+            kw[key.strip()] = type(getattr(wl, key.strip()))(val)
+        wl = wl.scaled(**kw)
+    return wl
+
+
 def run_reference(args):
     """Reference arm: the fp64 CPU oracle as it stands, on bounded samples."""
-    from ttt_inputs import WORKLOADS, make_layer_inputs
-    wl = WORKLOADS[args.workload]
+    from ttt_inputs import make_layer_inputs
+    wl = workload_from_args(args)
     x = make_layer_inputs(wl.scaled(B=1, H=1), seed=wl.seed)
     form = "parallel" if "parallel" in wl.paths else "recurrent"
     n, t, desc = oracle_sample(wl, x, 2.0, form)
@@ -456,10 +468,16 @@ def run_reference(args):
 
 
 def workload_config(wl, form):
-    return {"workload": wl.name, "form": form, "B": wl.B, "H": wl.H, "N": wl.N, "h": wl.h,
+    return {"workload": wl.name if wl == WORKLOADS_REF().get(wl.name) else wl.name + "*",
+            "form": form, "B": wl.B, "H": wl.H, "N": wl.N, "h": wl.h,
             "m": wl.m, "chunk": wl.chunk, "order": wl.order, "renorm": wl.renorm,
             "momentum": wl.momentum, "ns_steps": wl.ns_steps, "parallelism": "replicas",
             "l2": "no flush: the per-step inputs exceed the 126 MB L2"}
+
+
+def WORKLOADS_REF():
+    from ttt_inputs import WORKLOADS
+    return WORKLOADS
 
 
 # ----------------------------------------------------------------------------- main
@@ -473,6 +491,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target seconds of the CPU oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--override", default="",
+                    help="comma-separated workload field overrides for profiling, e.g. B=1,H=4")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

@@ -51,6 +51,25 @@ bool umma_supported(const GemmProblem& p);
 ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,
                      unsigned long long wait_ns);
 
+// Feature GEMM with the SwiGLU applied in the epilogue. gemm.B holds the input-side
+// weights as 128-row blocks [W0^T rows j..j+127 ; W2^T rows j..j+127] (256 rows per block,
+// zero rows past m), so gemm.N = 2 * ceil(m / 128) * 128 and every 256-wide output tile
+// carries matching A and B columns. The epilogue writes phi = silu(A) * B times
+// rowscale[z0*rs0 + z1*rs1 + row] (or 1 when rowscale is null) to gemm.C (bf16, row stride
+// gemm.C.ld, phi columns < n_valid) and, when out2 is set, the unscaled phi to out2.
+struct SwigluGemm {
+  GemmProblem gemm;
+  void* out2 = nullptr;
+  long long ld2 = 0, s20 = 0, s21 = 0;
+  const float* rowscale = nullptr;
+  long long rs0 = 0, rs1 = 0;
+  int n_valid = 0;
+};
+bool umma_swiglu_supported(const SwigluGemm& g);
+ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream);
+ttt_status gemm_umma_swiglu(const SwigluGemm& g, cudaStream_t stream, unsigned* dev_err,
+                            unsigned long long wait_ns);
+
 // Error-word access (ttt_api.cu).
 unsigned* device_error_word();
 unsigned long long wait_limit_ns();

@@ -93,7 +93,129 @@ void launch_simt(const SimtArgs& a, dim3 grid, cudaStream_t s) {
   simt_gemm_kernel<TA, TB, TC><<<grid, THREADS, 0, s>>>(a);
 }
 
+// SwiGLU-epilogue feature GEMM on CUDA cores. B holds 128-row blocks [W0^T ; W2^T]; output
+// column j (< n_valid) pairs B rows blk*256 + w (A part) and blk*256 + 128 + w (B part),
+// blk = j / 128, w = j % 128. Writes phi * rowscale to C and phi to C2 (when set).
+struct SimtSwiglu {
+  SimtArgs g;
+  void* C2; long long ld2, c2s0, c2s1;
+  const float* rs; long long rs0, rs1;
+};
+
+template <typename TA, typename TB, typename TC>
+__global__ void __launch_bounds__(THREADS) simt_swiglu_kernel(const SimtSwiglu sw) {
+  const SimtArgs& a = sw.g;
+  __shared__ float As[TK][TM + 1];
+  __shared__ float Ba[TK][TN + 1];
+  __shared__ float Bb[TK][TN + 1];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int i0 = blockIdx.y * TM, j0 = blockIdx.x * TN;
+  const int z0 = blockIdx.z % a.Z0, z1 = blockIdx.z / a.Z0;
+  const TA* A = static_cast<const TA*>(a.A) + z0 * a.as0 + z1 * a.as1;
+  const TB* B = static_cast<const TB*>(a.B) + z0 * a.bs0 + z1 * a.bs1;
+  float acc_a[4][4], acc_b[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc_a[r][c] = acc_b[r][c] = 0.0f;
+  for (int k0 = 0; k0 < a.K; k0 += TK) {
+    for (int e = tid; e < TM * TK; e += THREADS) {
+      int ii, kk;
+      if (a.a_mn) { ii = e % TM; kk = e / TM; } else { kk = e % TK; ii = e / TK; }
+      const int gi = i0 + ii, gk = k0 + kk;
+      float val = 0.0f;
+      if (gi < a.M && gk < a.K)
+        val = to_f32(A[a.a_mn ? (long long)gk * a.lda + gi : (long long)gi * a.lda + gk]);
+      As[kk][ii] = val;
+    }
+    for (int e = tid; e < TN * TK; e += THREADS) {
+      const int kk = e % TK, jj = e / TK;
+      const int gj = j0 + jj, gk = k0 + kk;
+      float va = 0.0f, vb = 0.0f;
+      if (gj < a.N && gk < a.K) {
+        const long long ra = (long long)(gj / 128) * 256 + (gj % 128);
+        va = to_f32(B[ra * a.ldb + gk]);
+        vb = to_f32(B[(ra + 128) * a.ldb + gk]);
+      }
+      Ba[kk][jj] = va;
+      Bb[kk][jj] = vb;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < TK; ++kk) {
+      float af[4], ba[4], bb[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) af[r] = As[kk][ty + 16 * r];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        ba[c] = Ba[kk][tx + 16 * c];
+        bb[c] = Bb[kk][tx + 16 * c];
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc_a[r][c] = fmaf(af[r], ba[c], acc_a[r][c]);
+          acc_b[r][c] = fmaf(af[r], bb[c], acc_b[r][c]);
+        }
+    }
+    __syncthreads();
+  }
+  TC* C = static_cast<TC*>(a.C) + z0 * a.cs0 + z1 * a.cs1;
+  TC* C2 = sw.C2 ? static_cast<TC*>(sw.C2) + z0 * sw.c2s0 + z1 * sw.c2s1 : nullptr;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int gi = i0 + ty + 16 * r;
+    if (gi >= a.M) continue;
+    const float rsv = sw.rs ? sw.rs[z0 * sw.rs0 + z1 * sw.rs1 + gi] : 1.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int gj = j0 + tx + 16 * c;
+      if (gj >= a.N) continue;
+      const float p = siluf_(acc_a[r][c]) * acc_b[r][c];
+      C[(long long)gi * a.ldc + gj] = from_f32<TC>(p * rsv);
+      if (C2) C2[(long long)gi * sw.ld2 + gj] = from_f32<TC>(p);
+    }
+  }
+}
+
 }  // namespace
+
+ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream) {
+  const GemmProblem& p = g.gemm;
+  if (p.M <= 0 || g.n_valid <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
+  const long long gy = (p.M + TM - 1) / TM, gz = (long long)p.Z0 * p.Z1;
+  if (gy > 65535 || gz > 65535 || p.B.mn_major) {
+    set_error_message("gemm_simt_swiglu: unsupported problem (M=%d, Z=%lld)", p.M, gz);
+    return TTT_ERR_UNSUPPORTED;
+  }
+  SimtSwiglu sw;
+  SimtArgs& a = sw.g;
+  a.M = p.M; a.N = g.n_valid; a.K = p.K; a.Z0 = p.Z0;
+  a.A = p.A.ptr; a.lda = p.A.ld; a.as0 = p.A.s0; a.as1 = p.A.s1; a.a_mn = p.A.mn_major;
+  a.B = p.B.ptr; a.ldb = p.B.ld; a.bs0 = p.B.s0; a.bs1 = p.B.s1; a.b_mn = 0;
+  a.C = p.C.ptr; a.ldc = p.C.ld; a.cs0 = p.C.s0; a.cs1 = p.C.s1;
+  a.Cin = nullptr; a.ldi = a.is0 = a.is1 = 0;
+  a.alpha = 1.0f; a.beta = 0.0f;
+  sw.C2 = g.out2; sw.ld2 = g.ld2; sw.c2s0 = g.s20; sw.c2s1 = g.s21;
+  sw.rs = g.rowscale; sw.rs0 = g.rs0; sw.rs1 = g.rs1;
+  dim3 grid((g.n_valid + TN - 1) / TN, (unsigned)gy, (unsigned)gz);
+  using bf = __nv_bfloat16;
+  const int key = (p.A.dtype << 2) | (p.B.dtype << 1) | p.C.dtype;
+  switch (key) {
+    case 0: simt_swiglu_kernel<float, float, float><<<grid, THREADS, 0, stream>>>(sw); break;
+    case 7: simt_swiglu_kernel<bf, bf, bf><<<grid, THREADS, 0, stream>>>(sw); break;
+    default:
+      set_error_message("gemm_simt_swiglu: operands and output must share one element type");
+      return TTT_ERR_UNSUPPORTED;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error_message("gemm_simt_swiglu launch: %s", cudaGetErrorString(e));
+    return TTT_ERR_CUDA;
+  }
+  return TTT_OK;
+}
 
 ttt_status gemm_simt(const GemmProblem& p, cudaStream_t stream) {
   if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;

@@ -1,11 +1,19 @@
 // Tensor-core batched GEMM engine for sm_100a: bf16 operands staged in shared memory by
-// TMA (128-byte swizzle, no multicast), tcgen05.mma kind::f16 with the fp32 accumulator
-// in tensor memory, and a CUDA-core epilogue that reads TMEM with tcgen05.ld.
+// TMA (128-byte swizzle, no multicast), tcgen05.mma kind::f16 with fp32 accumulators in
+// tensor memory, and CUDA-core epilogues that read TMEM with tcgen05.ld.
 //
-// One CTA computes one 128 x BN output tile. Warp roles (192 threads):
+// Persistent CTAs walk the 128 x BN output tiles of all batch entries round-robin. Two
+// TMEM accumulators alternate, so the epilogue of one tile overlaps the MMAs of the next.
+// Warp roles (320 threads):
 //   warp 0 (one lane)  TMA producer over a STAGES-deep shared-memory ring
 //   warp 1             TMEM allocation; one lane issues the MMAs and the commits
-//   warps 2..5         epilogue, warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31
+//   warps 2..9         epilogue; warp w reads TMEM lanes 32*(w%4) .. +31, and warps 2-5 /
+//                      6-9 take the first / second half of the tile's columns
+// Epilogue modes:
+//   STORE   C = alpha * acc + beta * Cin (fp32 or bf16 C)
+//   SWIGLU  the tile's columns are [A block | B block] of the fused SwiGLU input weights;
+//           writes phi = silu(a) * b times a per-row factor (bf16), and optionally the
+//           unscaled phi to a second output.
 // Every mbarrier wait is bounded; a timeout records DEVERR_TIMEOUT in the device error
 // word, raises a CTA-wide abort flag, and the CTA drains its in-flight copies and MMAs
 // (again with bounded waits) and frees its TMEM before returning.
@@ -25,15 +33,21 @@ using namespace umma;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int EPI_WARPS = 4;
+constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 
+enum EpiMode : int { EPI_STORE = 0, EPI_SWIGLU = 1 };
+
 struct UArgs {
-  int M, N, K, Z0;
+  int M, N, K, Z0, Z1;
   int a_b0, a_b1, b_b0, b_b1;  // 1 = operand uses that batch coordinate
   void* C; long long ldc, cs0, cs1;
   const float* Cin; long long ldi, is0, is1;
   float alpha, beta;
+  // SWIGLU: phi columns < n_valid are written; row factor rs[z0*rs0 + z1*rs1 + row]
+  void* C2; long long ld2, c2s0, c2s1;
+  const float* rs; long long rs0, rs1;
+  int n_valid;
   unsigned* err;
   unsigned long long wait_ns;
 };
@@ -47,61 +61,85 @@ struct Smem {
   static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
 };
 
-template <typename TC>
-__device__ __forceinline__ void store_row32(TC* dst, const float* v, int n_valid, bool vec_ok);
-
-template <>
-__device__ __forceinline__ void store_row32<float>(float* dst, const float* v, int n_valid,
-                                                   bool vec_ok) {
-  if (vec_ok && n_valid == 32) {
+__device__ __forceinline__ void store_vals(float* dst, const float* v, int n, bool vec) {
+  if (vec && n == 32) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4)
       *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
   } else {
-    for (int j = 0; j < n_valid; ++j) dst[j] = v[j];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < n) dst[j] = v[j];
   }
 }
 
-template <>
-__device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, const float* v,
-                                                           int n_valid, bool vec_ok) {
-  if (vec_ok && n_valid == 32) {
+// silu(a) = a * sigmoid(a) with sigmoid(a) = (1 + tanh(a / 2)) / 2: one MUFU tanh.approx
+// (relative error about 2^-11, below the bf16 rounding of the result).
+__device__ __forceinline__ float silu_fast(float a) {
+  const float h = 0.5f * a;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+__device__ __forceinline__ void store_vals(__nv_bfloat16* dst, const float* v, int n, bool vec) {
+  if (vec && n == 32) {
 #pragma unroll
     for (int j = 0; j < 32; j += 8) {
       uint4 pk;
-      __nv_bfloat162 t0 = __floats2bfloat162_rn(v[j], v[j + 1]);
-      __nv_bfloat162 t1 = __floats2bfloat162_rn(v[j + 2], v[j + 3]);
-      __nv_bfloat162 t2 = __floats2bfloat162_rn(v[j + 4], v[j + 5]);
-      __nv_bfloat162 t3 = __floats2bfloat162_rn(v[j + 6], v[j + 7]);
-      pk.x = *reinterpret_cast<uint32_t*>(&t0);
-      pk.y = *reinterpret_cast<uint32_t*>(&t1);
-      pk.z = *reinterpret_cast<uint32_t*>(&t2);
-      pk.w = *reinterpret_cast<uint32_t*>(&t3);
+      pk.x = pack_bf16x2(v[j], v[j + 1]);
+      pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
+      pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
+      pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
       *reinterpret_cast<uint4*>(dst + j) = pk;
     }
   } else {
-    for (int j = 0; j < n_valid; ++j) dst[j] = __float2bfloat16_rn(v[j]);
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < n) dst[j] = __float2bfloat16_rn(v[j]);
   }
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, typename TC>
+struct TileCoord {
+  int tm, tn, z0, z1;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int t, int tiles_n, int tiles_mn, int Z0) {
+  TileCoord c;
+  const int z = t / tiles_mn, rem = t - z * tiles_mn;
+  c.tm = rem / tiles_n;
+  c.tn = rem - c.tm * tiles_n;
+  c.z0 = z % Z0;
+  c.z1 = z / Z0;
+  return c;
+}
+
+template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC>
 __global__ void __launch_bounds__(THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, const UArgs args) {
   using L = Smem<BN, STAGES>;
+  constexpr uint32_t ACC_COLS = 2 * BN;  // two accumulators
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
+  uint64_t* acc_full = empty + STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile_n = blockIdx.x, tile_m = blockIdx.y;
-  const int z0 = blockIdx.z % args.Z0, z1 = blockIdx.z / args.Z0;
   const int KB = (args.K + BK - 1) / BK;
+  const int tiles_n = (args.N + BN - 1) / BN;
+  const int tiles_mn = tiles_n * ((args.M + BM - 1) / BM);
+  const int total = tiles_mn * args.Z0 * args.Z1;
   const uint32_t smem_base = smem_u32(smem);
 
   if (threadIdx.x == 0) {
@@ -109,14 +147,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    mbar_init(smem_u32(tfull), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), EPI_WARPS * 32);
+    }
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), BN);
+    tmem_alloc(smem_u32(tmem_slot), ACC_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -124,92 +165,184 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  int issued = 0;        // producer: k-blocks whose loads were issued
-  bool mma_any = false;  // MMA lane: at least one MMA issued
+  uint32_t issued = 0;   // producer: k-blocks whose loads were issued (all tiles)
+  int mma_tiles = 0;     // MMA lane: tiles whose MMAs were issued
   if (warp == 0) {
     if (lane == 0) {
-      const int ac2 = args.a_b0 ? z0 : 0, ac3 = args.a_b1 ? z1 : 0;
-      const int bc2 = args.b_b0 ? z0 : 0, bc3 = args.b_b1 ? z1 : 0;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        if (kb >= STAGES &&
-            !mbar_wait(smem_u32(&empty[s]), ((kb / STAGES) & 1) ^ 1, abort_flag, args.err,
-                       args.wait_ns))
-          break;
-        const uint32_t fb = smem_u32(&full[s]);
-        mbar_arrive_expect_tx(fb, L::STAGE);
-        const uint32_t sA = smem_base + s * L::STAGE;
-        const uint32_t sB = sA + L::A_BYTES;
-        if (A_MN) {
-          tma_load_4d(sA, &tmA, fb, tile_m * BM, kb * BK, ac2, ac3);
-          tma_load_4d(sA + 8192, &tmA, fb, tile_m * BM + 64, kb * BK, ac2, ac3);
-        } else {
-          tma_load_4d(sA, &tmA, fb, kb * BK, tile_m * BM, ac2, ac3);
-        }
-        if (B_MN) {
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+        const TileCoord tc = decode_tile(t, tiles_n, tiles_mn, args.Z0);
+        const int ac2 = args.a_b0 ? tc.z0 : 0, ac3 = args.a_b1 ? tc.z1 : 0;
+        const int bc2 = args.b_b0 ? tc.z0 : 0, bc3 = args.b_b1 ? tc.z1 : 0;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES &&
+              !mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, abort_flag, args.err,
+                         args.wait_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_arrive_expect_tx(fb, L::STAGE);
+          const uint32_t sA = smem_base + s * L::STAGE;
+          const uint32_t sB = sA + L::A_BYTES;
+          if (A_MN) {
+            tma_load_4d(sA, &tmA, fb, tc.tm * BM, kb * BK, ac2, ac3);
+            tma_load_4d(sA + 8192, &tmA, fb, tc.tm * BM + 64, kb * BK, ac2, ac3);
+          } else {
+            tma_load_4d(sA, &tmA, fb, kb * BK, tc.tm * BM, ac2, ac3);
+          }
+          if (B_MN) {
 #pragma unroll
-          for (int t = 0; t < BN / 64; ++t)
-            tma_load_4d(sB + t * 8192, &tmB, fb, tile_n * BN + 64 * t, kb * BK, bc2, bc3);
-        } else {
-          tma_load_4d(sB, &tmB, fb, kb * BK, tile_n * BN, bc2, bc3);
+            for (int q = 0; q < BN / 64; ++q)
+              tma_load_4d(sB + q * 8192, &tmB, fb, tc.tn * BN + 64 * q, kb * BK, bc2, bc3);
+          } else {
+            tma_load_4d(sB, &tmB, fb, kb * BK, tc.tn * BN, bc2, bc3);
+          }
+          issued = it + 1;
         }
-        issued = kb + 1;
+        if (!ok) break;
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t IDESC = make_idesc_bf16(BM, BN, A_MN, B_MN);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(smem_u32(&full[s]), (kb / STAGES) & 1, abort_flag, args.err, args.wait_ns))
+      uint32_t it = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        if (lt >= 2 && !mbar_wait(smem_u32(&acc_empty[buf]), ((lt >> 1) & 1) ^ 1, abort_flag,
+                                  args.err, args.wait_ns)) {
+          ok = false;
           break;
-        tc_fence_after();
-        const uint32_t sA = smem_base + s * L::STAGE;
-        const uint32_t sB = sA + L::A_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = A_MN ? make_sw128_desc(sA + kk * 2048, 8192, 1024)
-                                   : make_sw128_desc(sA + kk * 32, 16, 1024);
-          const uint64_t bd = B_MN ? make_sw128_desc(sB + kk * 2048, 8192, 1024)
-                                   : make_sw128_desc(sB + kk * 32, 16, 1024);
-          mma_f16(tmem, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_any = true;
-        mma_commit(smem_u32(&empty[s]));
+        tc_fence_after();
+        const uint32_t dt = tmem + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag, args.err,
+                         args.wait_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_base + s * L::STAGE;
+          const uint32_t sB = sA + L::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? make_sw128_desc(sA + kk * 2048, 8192, 1024)
+                                     : make_sw128_desc(sA + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? make_sw128_desc(sB + kk * 2048, 8192, 1024)
+                                     : make_sw128_desc(sB + kk * 32, 16, 1024);
+            mma_f16(dt, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&empty[s]));
+        }
+        // Arrives once the tile's MMAs are done (also on the abort path, so the teardown
+        // can wait for in-flight MMAs before freeing TMEM).
+        mma_commit(smem_u32(&acc_full[buf]));
+        mma_tiles = lt + 1;
       }
-      // Arrives once every MMA above is done (also on the abort path, so that the
-      // teardown can wait for in-flight MMAs before freeing TMEM).
-      mma_commit(smem_u32(tfull));
     }
   } else {
-    // Epilogue: TMEM -> registers -> alpha * acc + beta * Cin -> global.
-    const bool ok = mbar_wait(smem_u32(tfull), 0, abort_flag, args.err, args.wait_ns);
-    tc_fence_after();
+    const int ew = warp - 2;
     const int quarter = warp & 3;
-    const int row = tile_m * BM + quarter * 32 + lane;
-    TC* crow = static_cast<TC*>(args.C) + z0 * args.cs0 + z1 * args.cs1 + (long long)row * args.ldc;
-    const float* irow = args.Cin ? args.Cin + z0 * args.is0 + z1 * args.is1 +
-                                       (long long)row * args.ldi
-                                 : nullptr;
-    const bool vec_ok =
-        ((reinterpret_cast<uintptr_t>(crow) & 15) == 0) && ((args.ldc * sizeof(TC)) % 16 == 0);
-    if (ok) {
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, r);
-        tmem_ld_wait();
-        const int col0 = tile_n * BN + c0;
-        int nv = args.N - col0;
-        nv = nv > 32 ? 32 : nv;
-        if (row < args.M && nv > 0) {
-          float v[32];
+    const int part = ew >> 2;  // 0: first half of the tile's columns, 1: second half
+    int lt = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      if (!mbar_wait(smem_u32(&acc_full[buf]), (lt >> 1) & 1, abort_flag, args.err,
+                     args.wait_ns))
+        break;
+      tc_fence_after();
+      const TileCoord tc = decode_tile(t, tiles_n, tiles_mn, args.Z0);
+      const int row = tc.tm * BM + quarter * 32 + lane;
+      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
+      if (MODE == EPI_STORE) {
+        constexpr int HALF = BN / 2;
+        uint32_t r[HALF];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = args.alpha * __uint_as_float(r[j]);
-          if (irow) {
-            for (int j = 0; j < nv; ++j) v[j] += args.beta * irow[col0 + j];
+        for (int c0 = 0; c0 < HALF; c0 += 32)
+          tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0),
+                    *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
+        tmem_ld_wait();
+        float v[HALF];
+#pragma unroll
+        for (int j = 0; j < HALF; ++j) v[j] = __uint_as_float(r[j]);
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[buf]));
+        if (row < args.M) {
+          TC* crow = static_cast<TC*>(args.C) + tc.z0 * args.cs0 + tc.z1 * args.cs1 +
+                     (long long)row * args.ldc;
+          const float* irow = args.Cin ? args.Cin + tc.z0 * args.is0 + tc.z1 * args.is1 +
+                                             (long long)row * args.ldi
+                                       : nullptr;
+          const bool vec = ((reinterpret_cast<uintptr_t>(crow) & 15) == 0) &&
+                           ((args.ldc * (long long)sizeof(TC)) % 16 == 0);
+#pragma unroll
+          for (int c0 = 0; c0 < HALF; c0 += 32) {
+            const int col0 = tc.tn * BN + part * HALF + c0;
+            const int nv = min(32, args.N - col0);
+            if (nv <= 0) break;
+            float w[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) w[j] = args.alpha * v[c0 + j];
+            if (irow) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nv) w[j] += args.beta * irow[col0 + j];
+            }
+            store_vals(crow + col0, w, nv, vec);
           }
-          store_row32<TC>(crow + col0, v, nv, vec_ok);
+        }
+      } else {
+        // SWIGLU: phi column p of this tile uses accumulator columns p (A) and BN/2 + p (B).
+        constexpr int PH = BN / 2;       // phi columns per tile
+        constexpr int QW = PH / 2;       // phi columns per epilogue half
+        uint32_t ra[QW], rb[QW];
+#pragma unroll
+        for (int c0 = 0; c0 < QW; c0 += 32) {
+          tmem_ld32(lane_addr + (uint32_t)(part * QW + c0),
+                    *reinterpret_cast<uint32_t(*)[32]>(&ra[c0]));
+          tmem_ld32(lane_addr + (uint32_t)(PH + part * QW + c0),
+                    *reinterpret_cast<uint32_t(*)[32]>(&rb[c0]));
+        }
+        tmem_ld_wait();
+        float a[QW], b[QW];
+#pragma unroll
+        for (int j = 0; j < QW; ++j) {
+          a[j] = __uint_as_float(ra[j]);
+          b[j] = __uint_as_float(rb[j]);
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[buf]));
+        if (row < args.M) {
+          const float rsv = args.rs ? args.rs[tc.z0 * args.rs0 + tc.z1 * args.rs1 + row] : 1.0f;
+          const long long cbase = (long long)row * args.ldc + tc.z0 * args.cs0 + tc.z1 * args.cs1;
+          TC* c1 = static_cast<TC*>(args.C) + cbase;
+          TC* c2 = args.C2 ? static_cast<TC*>(args.C2) + tc.z0 * args.c2s0 + tc.z1 * args.c2s1 +
+                                 (long long)row * args.ld2
+                           : nullptr;
+          const bool vec = ((reinterpret_cast<uintptr_t>(c1) & 15) == 0) &&
+                           ((args.ldc * (long long)sizeof(TC)) % 16 == 0) &&
+                           (!c2 || (((reinterpret_cast<uintptr_t>(c2) & 15) == 0) &&
+                                    ((args.ld2 * (long long)sizeof(TC)) % 16 == 0)));
+#pragma unroll
+          for (int c0 = 0; c0 < QW; c0 += 32) {
+            const int col0 = tc.tn * PH + part * QW + c0;
+            const int nv = min(32, args.n_valid - col0);
+            if (nv <= 0) break;
+            float p[32], pe[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              p[j] = silu_fast(a[c0 + j]) * b[c0 + j];
+              pe[j] = p[j] * rsv;
+            }
+            store_vals(c1 + col0, pe, nv, vec);
+            if (c2) store_vals(c2 + col0, p, nv, vec);
+          }
         }
       }
     }
@@ -220,17 +353,21 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (*abort_flag) {
     // Drain: the producer waits for its loads still in flight; warp 1 for its MMAs.
     if (warp == 0 && lane == 0) {
-      for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
-        mbar_wait(smem_u32(&full[kb % STAGES]), (kb / STAGES) & 1, abort_flag, nullptr,
+      const uint32_t lo = issued > (uint32_t)STAGES ? issued - STAGES : 0;
+      for (uint32_t it = lo; it < issued; ++it)
+        mbar_wait(smem_u32(&full[it % STAGES]), (it / STAGES) & 1, abort_flag, nullptr,
                   args.wait_ns, true);
     }
-    if (warp == 1 && lane == 0 && mma_any)
-      mbar_wait(smem_u32(tfull), 0, abort_flag, nullptr, args.wait_ns, true);
+    if (warp == 1 && lane == 0 && mma_tiles > 0) {
+      const int lt = mma_tiles - 1;
+      mbar_wait(smem_u32(&acc_full[lt & 1]), (lt >> 1) & 1, abort_flag, nullptr, args.wait_ns,
+                true);
+    }
     __syncthreads();
   }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, ACC_COLS);
   }
 }
 
@@ -247,6 +384,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   return fn;
+}
+
+int sm_count() {
+  static int cache[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
 }
 
 // 4-D map {inner, outer, z0, z1} over one operand; box {64, box_outer, 1, 1}.
@@ -278,7 +428,7 @@ bool make_map(CUtensorMap* map, const GemmOperand& op, int rows, int K, int Z0, 
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, typename TC>
+template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC>
 ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, p.A, p.M, p.K, p.Z0, p.Z1, BM) ||
@@ -286,15 +436,18 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
     set_error_message("gemm_umma: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", p.M, p.N, p.K);
     return TTT_ERR_CUDA;
   }
-  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, TC>;
+  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC>;
   constexpr int SMEM = Smem<BN, STAGES>::TOTAL;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
       cudaSuccess) {
     set_error_message("gemm_umma: cannot set %d bytes of dynamic shared memory", SMEM);
     return TTT_ERR_CUDA;
   }
-  dim3 grid((p.N + BN - 1) / BN, (p.M + BM - 1) / BM, p.Z0 * p.Z1);
-  kern<<<grid, THREADS, SMEM, s>>>(ma, mb, a);
+  const long long tiles = (long long)((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM) * p.Z0 * p.Z1;
+  const int per_sm = (SMEM <= 110 * 1024) ? 2 : 1;
+  long long grid = (long long)sm_count() * per_sm;
+  if (tiles < grid) grid = tiles;
+  kern<<<(unsigned)grid, THREADS, SMEM, s>>>(ma, mb, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error_message("gemm_umma launch: %s", cudaGetErrorString(e));
@@ -303,22 +456,22 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   return TTT_OK;
 }
 
-template <int BN, int STAGES, typename TC>
+template <int BN, int STAGES, int MODE, typename TC>
 ttt_status dispatch_major(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   const int key = (p.A.mn_major ? 2 : 0) | (p.B.mn_major ? 1 : 0);
   switch (key) {
-    case 0: return launch_umma<BN, false, false, STAGES, TC>(p, a, s);
-    case 1: return launch_umma<BN, false, true, STAGES, TC>(p, a, s);
-    case 2: return launch_umma<BN, true, false, STAGES, TC>(p, a, s);
-    default: return launch_umma<BN, true, true, STAGES, TC>(p, a, s);
+    case 0: return launch_umma<BN, false, false, STAGES, MODE, TC>(p, a, s);
+    case 1: return launch_umma<BN, false, true, STAGES, MODE, TC>(p, a, s);
+    case 2: return launch_umma<BN, true, false, STAGES, MODE, TC>(p, a, s);
+    default: return launch_umma<BN, true, true, STAGES, MODE, TC>(p, a, s);
   }
 }
 
 template <typename TC>
 ttt_status dispatch_bn(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  if (p.N > 128) return dispatch_major<256, 4, TC>(p, a, s);
-  if (p.N > 64) return dispatch_major<128, 3, TC>(p, a, s);
-  return dispatch_major<64, 4, TC>(p, a, s);
+  if (p.N > 128) return dispatch_major<256, 4, EPI_STORE, TC>(p, a, s);
+  if (p.N > 64) return dispatch_major<128, 3, EPI_STORE, TC>(p, a, s);
+  return dispatch_major<64, 4, EPI_STORE, TC>(p, a, s);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -328,12 +481,25 @@ bool operand_ok(const GemmOperand& o) {
          (o.s0 % 8) == 0 && (o.s1 % 8) == 0 && o.s0 >= 0 && o.s1 >= 0;
 }
 
+UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait_ns) {
+  UArgs a{};
+  a.M = p.M; a.N = p.N; a.K = p.K; a.Z0 = p.Z0; a.Z1 = p.Z1;
+  a.a_b0 = p.A.s0 != 0; a.a_b1 = p.A.s1 != 0; a.b_b0 = p.B.s0 != 0; a.b_b1 = p.B.s1 != 0;
+  a.C = p.C.ptr; a.ldc = p.C.ld; a.cs0 = p.C.s0; a.cs1 = p.C.s1;
+  a.Cin = p.beta != 0.0f ? p.Cin.ptr : nullptr;
+  a.ldi = p.Cin.ld; a.is0 = p.Cin.s0; a.is1 = p.Cin.s1;
+  a.alpha = p.alpha; a.beta = p.beta;
+  a.err = dev_err;
+  a.wait_ns = wait_ns;
+  return a;
+}
+
 }  // namespace
 
 bool umma_supported(const GemmProblem& p) {
   if (!operand_ok(p.A) || !operand_ok(p.B)) return false;
   if (p.K <= 0 || p.M <= 0 || p.N <= 0) return false;
-  if ((long long)p.Z0 * p.Z1 > 65535 || (p.M + BM - 1) / BM > 65535) return false;
+  if ((long long)p.Z0 * p.Z1 * ((p.M + BM - 1) / BM) * ((p.N + 63) / 64) > (1LL << 31)) return false;
   if (p.beta != 0.0f && !p.Cin.ptr) return false;
   return encode_fn() != nullptr;
 }
@@ -345,17 +511,30 @@ ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_er
     set_error_message("gemm_umma: unsupported operand layout");
     return TTT_ERR_UNSUPPORTED;
   }
-  UArgs a;
-  a.M = p.M; a.N = p.N; a.K = p.K; a.Z0 = p.Z0;
-  a.a_b0 = p.A.s0 != 0; a.a_b1 = p.A.s1 != 0; a.b_b0 = p.B.s0 != 0; a.b_b1 = p.B.s1 != 0;
-  a.C = p.C.ptr; a.ldc = p.C.ld; a.cs0 = p.C.s0; a.cs1 = p.C.s1;
-  a.Cin = p.beta != 0.0f ? p.Cin.ptr : nullptr;
-  a.ldi = p.Cin.ld; a.is0 = p.Cin.s0; a.is1 = p.Cin.s1;
-  a.alpha = p.alpha; a.beta = p.beta;
-  a.err = dev_err;
-  a.wait_ns = wait_ns;
+  const UArgs a = base_args(p, dev_err, wait_ns);
   if (p.C.dtype == DT_BF16) return dispatch_bn<__nv_bfloat16>(p, a, stream);
   return dispatch_bn<float>(p, a, stream);
+}
+
+bool umma_swiglu_supported(const SwigluGemm& g) {
+  const GemmProblem& p = g.gemm;
+  return umma_supported(p) && p.C.dtype == DT_BF16 && p.N % 256 == 0 && p.beta == 0.0f &&
+         (!g.out2 || aligned16(g.out2));
+}
+
+ttt_status gemm_umma_swiglu(const SwigluGemm& g, cudaStream_t stream, unsigned* dev_err,
+                            unsigned long long wait_ns) {
+  const GemmProblem& p = g.gemm;
+  if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
+  if (!umma_swiglu_supported(g)) {
+    set_error_message("gemm_umma_swiglu: unsupported problem");
+    return TTT_ERR_UNSUPPORTED;
+  }
+  UArgs a = base_args(p, dev_err, wait_ns);
+  a.C2 = g.out2; a.ld2 = g.ld2; a.c2s0 = g.s20; a.c2s1 = g.s21;
+  a.rs = g.rowscale; a.rs0 = g.rs0; a.rs1 = g.rs1;
+  a.n_valid = g.n_valid;
+  return dispatch_major<256, 4, EPI_SWIGLU, __nv_bfloat16>(p, a, stream);
 }
 
 }  // namespace ttt

@@ -35,6 +35,25 @@ __global__ void prep_wk_kernel(const float* W0, const float* W2, OT* Wk, int n_e
   }
 }
 
+template <typename OT>
+__global__ void prep_wk_blocked_kernel(const float* W0, const float* W2, OT* Wk, int n_entries,
+                                       int src_heads, int h, int m, int layout) {
+  const int mpad = (m + 127) / 128 * 128;
+  const long long per = 2LL * mpad * h;
+  TTT_GRID_LOOP(idx, per * n_entries) {
+    const long long e = idx / per, rem = idx - e * per;
+    const int r = (int)(rem / h), i = (int)(rem - (long long)r * h);
+    const int blk = r >> 8, w = r & 255;
+    const int j = blk * 128 + (w & 127);
+    float v = 0.0f;
+    if (j < m) {
+      const float* src = (w < 128 ? W0 : W2) + (e % src_heads) * (long long)h * m;
+      v = layout == 0 ? src[(long long)i * m + j] : src[(long long)j * h + i];
+    }
+    Wk[idx] = from_f32<OT>(v);
+  }
+}
+
 // ------------------------------------------------------------------ features
 template <typename OT>
 __global__ void swiglu_kernel(const float* AB, long long rows, int m, EtaMap em, OT* phi_eta,
@@ -71,8 +90,9 @@ __global__ void grad_prep_kernel(const float* AB, const float* Dv, long long row
 // One thread per state element; the chunk axis (tens of chunks) is walked sequentially so
 // every delta is read once and every chunk state written once.
 template <typename OT>
-__global__ void chunk_scan_kernel(const float* dS, const float* W1, OT* Sc, float* S_final,
-                                  int BH, int H, int C, int m, int h, int order, int layout) {
+__global__ void chunk_scan_kernel(const float* __restrict__ dS, const float* __restrict__ W1,
+                                  OT* __restrict__ Sc, float* __restrict__ S_final, int BH,
+                                  int H, int C, int m, int h, int order, int layout) {
   const long long per = (long long)m * h;
   TTT_GRID_LOOP(idx, per * BH) {
     const long long bh = idx / per, e = idx - bh * per;
@@ -81,8 +101,26 @@ __global__ void chunk_scan_kernel(const float* dS, const float* W1, OT* Sc, floa
     float s = W1[w_off];
     const float* d = dS + bh * C * per + e;
     OT* out = Sc + bh * C * per + e;
-    for (int c = 0; c < C; ++c) {
-      const float dv = d[(long long)c * per];
+    int c = 0;
+    // Four chunks per step with the loads issued first, so each thread keeps four
+    // independent loads in flight.
+    for (; c + 4 <= C; c += 4) {
+      float dv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) dv[u] = __ldcs(d + (long long)(c + u) * per);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (order == 1) {
+          out[(long long)(c + u) * per] = from_f32<OT>(s);
+          s += dv[u];
+        } else {
+          s += dv[u];
+          out[(long long)(c + u) * per] = from_f32<OT>(s);
+        }
+      }
+    }
+    for (; c < C; ++c) {
+      const float dv = __ldcs(d + (long long)c * per);
       if (order == 1) {
         out[(long long)c * per] = from_f32<OT>(s);
         s += dv;
@@ -313,6 +351,18 @@ cudaError_t prep_wk(int ot, const float* W0, const float* W2, void* Wk, int n_en
     const long long n = 2LL * m * h * n_entries;
     prep_wk_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(W0, W2, static_cast<OT*>(Wk), n_entries,
                                                         src_heads, h, m, src_layout);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
+                            int src_heads, int h, int m, int src_layout, cudaStream_t s) {
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    const long long mpad = (m + 127) / 128 * 128;
+    const long long n = 2LL * mpad * h * n_entries;
+    prep_wk_blocked_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(
+        W0, W2, static_cast<OT*>(Wk), n_entries, src_heads, h, m, src_layout);
     return cudaGetLastError();
   });
 }

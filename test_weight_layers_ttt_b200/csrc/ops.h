@@ -19,6 +19,10 @@ struct EtaMap {
 // entries; entry e reads source head e % src_heads. Source layout 0: [h, m]; 1: [m, h].
 cudaError_t prep_wk(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
                     int src_heads, int h, int m, int src_layout, cudaStream_t s);
+// Same weights as 128-row blocks [W0^T rows j..j+127 ; W2^T rows j..j+127] per entry
+// ([2 * ceil(m/128) * 128, h], zero rows past m): the B operand of the SwiGLU-epilogue GEMM.
+cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
+                            int src_heads, int h, int m, int src_layout, cudaStream_t s);
 
 // phi = silu(A) * B from AB rows [A | B] (fp32, width 2m); writes phi * eta to phi_eta and,
 // when non-null, the unscaled phi to phi_plain (both OT, width m).

@@ -205,21 +205,21 @@ ttt_status check_desc(const ttt_desc* d, int path) {
 
 // ------------------------------------------------------------------ parallel form
 struct ParBufs {
-  void* Wk;
-  float* AB;
-  void* phiA;
-  void* phiB;
-  float* dS;
-  void* Sc;
+  void* Wk;    // [H, 2*mpad, h] blocked [W0^T ; W2^T] operand
+  void* phiA;  // phi(K) * eta  [BH, N, m]
+  void* phiB;  // phi(Q)        [BH, N, m]
+  float* dS;   // [BH, C, m, h]
+  void* Sc;    // [BH, C, m, h] state read by each chunk
 };
+
+long long padded_m(int m) { return (m + 127LL) / 128 * 128; }
 
 size_t plan_parallel(const ttt_desc& d, void* base, ParBufs& b) {
   Carve cv(base);
   const size_t os = d.dtype == TTT_DTYPE_BF16 ? 2 : 4;
   const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
   const long long rows = BH * d.N, hm = (long long)d.h * d.m;
-  b.Wk = cv.take(os * 2 * hm * d.H);
-  b.AB = cv.take_n<float>(rows * 2 * d.m);
+  b.Wk = cv.take(os * 2 * padded_m(d.m) * d.h * d.H);
   b.phiA = cv.take(os * rows * d.m);
   b.phiB = cv.take(os * rows * d.m);
   b.dS = cv.take_n<float>(BH * C * hm);
@@ -227,16 +227,33 @@ size_t plan_parallel(const ttt_desc& d, void* base, ParBufs& b) {
   return cv.off;
 }
 
-// A = X (tokens x h rows of sequence (b, head)), B = Wk[head]: AB = X [W0 | W2].
-GemmProblem features_problem(const ttt_desc& d, const void* X, const void* Wk, float* AB) {
+// phi(X) for every token of every (b, head): X [B,H,N,h] against the blocked weights of
+// its head; writes phi * eta to `scaled` (when eta is set, else phi) and phi to `plain`.
+SwigluGemm features_problem(const ttt_desc& d, const void* X, const void* Wk, void* scaled,
+                            void* plain, const float* eta) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
-  const long long N = d.N, h = d.h, m = d.m;
-  GemmProblem p;
-  p.M = d.N; p.N = 2 * d.m; p.K = d.h; p.Z0 = d.H; p.Z1 = d.B;
-  p.A = {X, ot, false, h, N * h, (long long)d.H * N * h};
-  p.B = {Wk, ot, false, h, 2 * m * h, 0};
-  p.C = {AB, DT_F32, 2 * m, N * 2 * m, (long long)d.H * N * 2 * m};
-  return p;
+  const long long N = d.N, h = d.h, m = d.m, H = d.H, mp = padded_m(d.m);
+  SwigluGemm g;
+  GemmProblem& p = g.gemm;
+  p.M = d.N; p.N = (int)(2 * mp); p.K = d.h; p.Z0 = d.H; p.Z1 = d.B;
+  p.A = {X, ot, false, h, N * h, H * N * h};
+  p.B = {Wk, ot, false, h, 2 * mp * h, 0};
+  p.C = {scaled, ot, m, N * m, H * N * m};
+  g.out2 = plain;
+  g.ld2 = m; g.s20 = N * m; g.s21 = H * N * m;
+  g.rowscale = eta;
+  g.rs0 = N; g.rs1 = H * N;
+  g.n_valid = d.m;
+  return g;
+}
+
+ttt_status run_swiglu(const char* name, const SwigluGemm& g, cudaStream_t s) {
+  const GemmProblem& p = g.gemm;
+  if (p.M <= 0 || g.n_valid <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
+  const bool tc = !force_simt() && umma_swiglu_supported(g);
+  TraceScope ts(g_trace.on ? engine_name(name, tc ? "tcgen05" : "simt") : name, s);
+  if (tc) return gemm_umma_swiglu(g, s, device_error_word(), wait_limit_ns());
+  return gemm_simt_swiglu(g, s);
 }
 
 ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
@@ -247,11 +264,12 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
   const long long C = (N + L - 1) / L, Cf = N / L, tail = N - Cf * L, hm = h * m;
   const bool shared_qk = (q == k);
 
-  TTT_OP("prep_weights", prep_wk(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
+  TTT_OP("prep_weights",
+         prep_wk_blocked(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
   // phi(K) eta (and phi(Q) when q == k)
-  TTT_TRY(run_gemm("gemm_features_k", features_problem(d, k, b.Wk, b.AB), s));
-  EtaMap em{eta, N, N, 0};
-  TTT_OP("swiglu_k", swiglu(ot, b.AB, BH * N, d.m, em, b.phiA, shared_qk ? b.phiB : nullptr, s));
+  TTT_TRY(run_swiglu("gemm_features_k",
+                     features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
+                     s));
   // Delta S_c = sign * phi(K_c)^T diag(eta) V_c  (per (b, head) and chunk)
   for (int part = 0; part < 2; ++part) {
     const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);
@@ -268,10 +286,9 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
   // States read by each chunk, and the final state.
   TTT_OP("chunk_scan", chunk_scan(ot, b.dS, W1, b.Sc, S_final, (int)BH, d.H, (int)C, d.m, d.h,
                                   d.order, d.w1_layout, s));
-  if (!shared_qk) {
-    TTT_TRY(run_gemm("gemm_features_q", features_problem(d, q, b.Wk, b.AB), s));
-    TTT_OP("swiglu_q", swiglu(ot, b.AB, BH * N, d.m, em, nullptr, b.phiB, s));
-  }
+  if (!shared_qk)
+    TTT_TRY(run_swiglu("gemm_features_q",
+                       features_problem(d, q, b.Wk, b.phiB, nullptr, nullptr), s));
   // O_c = phi(Q_c) S_c
   for (int part = 0; part < 2; ++part) {
     const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);

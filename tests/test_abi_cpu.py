@@ -56,9 +56,9 @@ def lm_desc(**kw):
 
 def test_workspace_sizes():
     par = abi.ttt_workspace_bytes(lm_desc(), abi.TTT_PATH_PARALLEL)
-    # Wk + [A|B] fp32 + two feature buffers + fp32 deltas + bf16 chunk states
+    # blocked bf16 weights + two bf16 feature buffers + fp32 deltas + bf16 chunk states
     BH, N, h, m, C = 8, 32768, 256, 512, 16
-    expect = 2 * 2 * m * h * 4 + BH * N * 2 * m * 4 + 2 * (2 * BH * N * m) + BH * C * m * h * 6
+    expect = 2 * 2 * m * h * 4 + 2 * (2 * BH * N * m) + BH * C * m * h * 6
     assert expect <= par <= expect + 6 * 256
     assert abi.ttt_workspace_bytes(lm_desc(N=65536), 0) > par
     rec = abi.ttt_workspace_bytes(lm_desc(update_mask=7, renorm=1), abi.TTT_PATH_RECURRENT)
