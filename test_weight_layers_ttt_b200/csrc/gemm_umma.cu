@@ -21,6 +21,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "gemm.h"
@@ -52,13 +53,22 @@ struct UArgs {
   unsigned long long wait_ns;
 };
 
-template <int BN, int STAGES>
+// Shared-memory layout. Streaming mode: a ring of STAGES (A tile + B tile) stages.
+// B-resident mode (BRES): the CTA's whole B tile for K <= 256 (up to four 64-wide k-blocks)
+// stays in shared memory and the ring carries only A tiles.
+// SWIGLU mode adds a 32 KB staging tile (128 rows x 128 bf16 phi columns, as two
+// 128-byte-swizzled 64-column boxes) written by the epilogue and stored with TMA.
+template <int BN, int STAGES, bool BRES, int MODE>
 struct Smem {
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int BAR_OFF = STAGES * STAGE;
-  static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
+  static constexpr int B_BYTES = BN * BK * 2;             // one k-block of B
+  static constexpr int B_RES = BRES ? 4 * B_BYTES : 0;    // resident B, at most 4 k-blocks
+  static constexpr int STAGE = BRES ? A_BYTES : A_BYTES + B_BYTES;
+  static constexpr int OUT_BYTES = MODE == 1 ? BM * 128 * 2 : 0;
+  static constexpr int OUT_OFF = B_RES;
+  static constexpr int RING_OFF = OUT_OFF + OUT_BYTES;
+  static constexpr int BAR_OFF = RING_OFF + STAGES * STAGE;
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;      // + barriers + alignment slack
 };
 
 __device__ __forceinline__ void store_vals(float* dst, const float* v, int n, bool vec) {
@@ -119,11 +129,57 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int tiles_n, int tiles_m
   return c;
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC>
+// The sequence of tiles one CTA processes; every warp role walks the same sequence.
+// Streaming mode: tiles blockIdx.x, blockIdx.x + gridDim.x, ... of the (z, tm, tn) order
+// (n fastest, so the CTAs working at the same time share A tiles in L2).
+// B-resident mode: CTA c keeps n-tile c % tiles_n and walks a contiguous range of the
+// flattened (z, tm) row tiles, shared with the other n-tile CTAs of its group, so a
+// group reads each A tile from HBM once and each CTA reloads B only when z changes.
+struct TileWalker {
+  int tiles_n, tiles_m, Z0, total, count;
+  int bres, nt, r0;
+  __device__ TileWalker(int M, int N, int Z0_, int Z1, int BN, bool b_res) {
+    tiles_n = (N + BN - 1) / BN;
+    tiles_m = (M + BM - 1) / BM;
+    Z0 = Z0_;
+    total = tiles_n * tiles_m * Z0_ * Z1;
+    bres = b_res;
+    if (!b_res) {
+      count = blockIdx.x < (unsigned)total ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+      nt = r0 = 0;
+    } else {
+      const int groups = gridDim.x / tiles_n, g = blockIdx.x / tiles_n;
+      const int rows = tiles_m * Z0_ * Z1;
+      nt = blockIdx.x % tiles_n;
+      if (g >= groups) {
+        count = 0;
+        r0 = 0;
+      } else {
+        const long long lo = (long long)rows * g / groups, hi = (long long)rows * (g + 1) / groups;
+        r0 = (int)lo;
+        count = (int)(hi - lo);
+      }
+    }
+  }
+  __device__ TileCoord at(int i) const {
+    if (!bres) return decode_tile(blockIdx.x + i * gridDim.x, tiles_n, tiles_n * tiles_m, Z0);
+    const int r = r0 + i, z = r / tiles_m;
+    TileCoord c;
+    c.tm = r - z * tiles_m;
+    c.tn = nt;
+    c.z0 = z % Z0;
+    c.z1 = z / Z0;
+    return c;
+  }
+};
+
+template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES>
 __global__ void __launch_bounds__(THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                     const __grid_constant__ CUtensorMap tmB, const UArgs args) {
-  using L = Smem<BN, STAGES>;
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC,
+                     const __grid_constant__ CUtensorMap tmC2, const UArgs args) {
+  using L = Smem<BN, STAGES, BRES, MODE>;
   constexpr uint32_t ACC_COLS = 2 * BN;  // two accumulators
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -132,15 +188,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* b_full = acc_empty + 2;     // resident B loaded
+  uint64_t* b_empty = b_full + 1;       // resident B no longer read by MMAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = (args.K + BK - 1) / BK;
-  const int tiles_n = (args.N + BN - 1) / BN;
-  const int tiles_mn = tiles_n * ((args.M + BM - 1) / BM);
-  const int total = tiles_mn * args.Z0 * args.Z1;
+  const TileWalker walk(args.M, args.N, args.Z0, args.Z1, BN, BRES);
   const uint32_t smem_base = smem_u32(smem);
+  const uint32_t ring_base = smem_base + L::RING_OFF;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -151,6 +208,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(smem_u32(&acc_full[b]), 1);
       mbar_init(smem_u32(&acc_empty[b]), EPI_WARPS * 32);
     }
+    mbar_init(smem_u32(b_full), 1);
+    mbar_init(smem_u32(b_empty), 1);
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
@@ -166,14 +225,36 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   uint32_t issued = 0;   // producer: k-blocks whose loads were issued (all tiles)
+  int b_loads = 0;       // producer: resident-B loads issued
   int mma_tiles = 0;     // MMA lane: tiles whose MMAs were issued
   if (warp == 0) {
     if (lane == 0) {
       uint32_t it = 0;
-      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-        const TileCoord tc = decode_tile(t, tiles_n, tiles_mn, args.Z0);
+      int bkey = -1;
+      for (int i = 0; i < walk.count && !*abort_flag; ++i) {
+        const TileCoord tc = walk.at(i);
         const int ac2 = args.a_b0 ? tc.z0 : 0, ac3 = args.a_b1 ? tc.z1 : 0;
         const int bc2 = args.b_b0 ? tc.z0 : 0, bc3 = args.b_b1 ? tc.z1 : 0;
+        if (BRES && (bc2 * 65536 + bc3) != bkey) {
+          // (Re)load the CTA's B tile once the MMAs have stopped reading the previous one.
+          if (b_loads > 0 && !mbar_wait(smem_u32(b_empty), (b_loads - 1) & 1, abort_flag,
+                                        args.err, args.wait_ns))
+            break;
+          const uint32_t bb = smem_u32(b_full);
+          mbar_arrive_expect_tx(bb, KB * L::B_BYTES);
+          for (int kb = 0; kb < KB; ++kb) {
+            const uint32_t sB = smem_base + kb * L::B_BYTES;
+            if (B_MN) {
+#pragma unroll
+              for (int q = 0; q < BN / 64; ++q)
+                tma_load_4d(sB + q * 8192, &tmB, bb, tc.tn * BN + 64 * q, kb * BK, bc2, bc3);
+            } else {
+              tma_load_4d(sB, &tmB, bb, kb * BK, tc.tn * BN, bc2, bc3);
+            }
+          }
+          ++b_loads;
+          bkey = bc2 * 65536 + bc3;
+        }
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
@@ -185,20 +266,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           const uint32_t fb = smem_u32(&full[s]);
           mbar_arrive_expect_tx(fb, L::STAGE);
-          const uint32_t sA = smem_base + s * L::STAGE;
-          const uint32_t sB = sA + L::A_BYTES;
+          const uint32_t sA = ring_base + s * L::STAGE;
           if (A_MN) {
             tma_load_4d(sA, &tmA, fb, tc.tm * BM, kb * BK, ac2, ac3);
             tma_load_4d(sA + 8192, &tmA, fb, tc.tm * BM + 64, kb * BK, ac2, ac3);
           } else {
             tma_load_4d(sA, &tmA, fb, kb * BK, tc.tm * BM, ac2, ac3);
           }
-          if (B_MN) {
+          if (!BRES) {
+            const uint32_t sB = sA + L::A_BYTES;
+            if (B_MN) {
 #pragma unroll
-            for (int q = 0; q < BN / 64; ++q)
-              tma_load_4d(sB + q * 8192, &tmB, fb, tc.tn * BN + 64 * q, kb * BK, bc2, bc3);
-          } else {
-            tma_load_4d(sB, &tmB, fb, kb * BK, tc.tn * BN, bc2, bc3);
+              for (int q = 0; q < BN / 64; ++q)
+                tma_load_4d(sB + q * 8192, &tmB, fb, tc.tn * BN + 64 * q, kb * BK, bc2, bc3);
+            } else {
+              tma_load_4d(sB, &tmB, fb, kb * BK, tc.tn * BN, bc2, bc3);
+            }
           }
           issued = it + 1;
         }
@@ -209,14 +292,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC = make_idesc_bf16(BM, BN, A_MN, B_MN);
       uint32_t it = 0;
-      int lt = 0;
+      int bkey = -1, b_uses = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+      for (int lt = 0; lt < walk.count && ok; ++lt) {
+        const TileCoord tc = walk.at(lt);
         const int buf = lt & 1;
         if (lt >= 2 && !mbar_wait(smem_u32(&acc_empty[buf]), ((lt >> 1) & 1) ^ 1, abort_flag,
                                   args.err, args.wait_ns)) {
           ok = false;
           break;
+        }
+        if (BRES) {
+          const int key = (args.b_b0 ? tc.z0 : 0) * 65536 + (args.b_b1 ? tc.z1 : 0);
+          if (key != bkey) {
+            if (b_uses > 0) mma_commit(smem_u32(b_empty));  // old B free once MMAs finish
+            if (!mbar_wait(smem_u32(b_full), b_uses & 1, abort_flag, args.err, args.wait_ns)) {
+              ok = false;
+              break;
+            }
+            ++b_uses;
+            bkey = key;
+          }
         }
         tc_fence_after();
         const uint32_t dt = tmem + (uint32_t)(buf * BN);
@@ -228,8 +324,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sA = smem_base + s * L::STAGE;
-          const uint32_t sB = sA + L::A_BYTES;
+          const uint32_t sA = ring_base + s * L::STAGE;
+          const uint32_t sB = BRES ? smem_base + kb * L::B_BYTES : sA + L::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = A_MN ? make_sw128_desc(sA + kk * 2048, 8192, 1024)
@@ -250,14 +346,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int ew = warp - 2;
     const int quarter = warp & 3;
     const int part = ew >> 2;  // 0: first half of the tile's columns, 1: second half
-    int lt = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
+    for (int lt = 0; lt < walk.count; ++lt) {
       const int buf = lt & 1;
-      if (!mbar_wait(smem_u32(&acc_full[buf]), (lt >> 1) & 1, abort_flag, args.err,
-                     args.wait_ns))
-        break;
+      bool ok = mbar_wait(smem_u32(&acc_full[buf]), (lt >> 1) & 1, abort_flag, args.err,
+                          args.wait_ns);
+      if (!ok) break;
       tc_fence_after();
-      const TileCoord tc = decode_tile(t, tiles_n, tiles_mn, args.Z0);
+      const TileCoord tc = walk.at(lt);
       const int row = tc.tm * BM + quarter * 32 + lane;
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
       if (MODE == EPI_STORE) {
@@ -318,34 +413,52 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&acc_empty[buf]));
-        if (row < args.M) {
-          const float rsv = args.rs ? args.rs[tc.z0 * args.rs0 + tc.z1 * args.rs1 + row] : 1.0f;
-          const long long cbase = (long long)row * args.ldc + tc.z0 * args.cs0 + tc.z1 * args.cs1;
-          TC* c1 = static_cast<TC*>(args.C) + cbase;
-          TC* c2 = args.C2 ? static_cast<TC*>(args.C2) + tc.z0 * args.c2s0 + tc.z1 * args.c2s1 +
-                                 (long long)row * args.ld2
-                           : nullptr;
-          const bool vec = ((reinterpret_cast<uintptr_t>(c1) & 15) == 0) &&
-                           ((args.ldc * (long long)sizeof(TC)) % 16 == 0) &&
-                           (!c2 || (((reinterpret_cast<uintptr_t>(c2) & 15) == 0) &&
-                                    ((args.ld2 * (long long)sizeof(TC)) % 16 == 0)));
+        const int rin = quarter * 32 + lane;  // row within the tile
+        const float rsv =
+            (args.rs && row < args.M) ? args.rs[tc.z0 * args.rs0 + tc.z1 * args.rs1 + row] : 1.0f;
+        // phi in place of b; packed outputs only where they are stored.
 #pragma unroll
-          for (int c0 = 0; c0 < QW; c0 += 32) {
-            const int col0 = tc.tn * PH + part * QW + c0;
-            const int nv = min(32, args.n_valid - col0);
-            if (nv <= 0) break;
-            float p[32], pe[32];
+        for (int j = 0; j < QW; ++j) b[j] = silu_fast(a[j]) * b[j];
+        uint32_t pk[QW / 2], pk2[QW / 2];
+        if (args.rs) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              p[j] = silu_fast(a[c0 + j]) * b[c0 + j];
-              pe[j] = p[j] * rsv;
-            }
-            store_vals(c1 + col0, pe, nv, vec);
-            if (c2) store_vals(c2 + col0, p, nv, vec);
+          for (int j = 0; j < QW; j += 2) pk[j / 2] = pack_bf16x2(b[j] * rsv, b[j + 1] * rsv);
+        } else {
+#pragma unroll
+          for (int j = 0; j < QW; j += 2) pk[j / 2] = pack_bf16x2(b[j], b[j + 1]);
+        }
+        if (args.C2) {
+#pragma unroll
+          for (int j = 0; j < QW; j += 2) pk2[j / 2] = pack_bf16x2(b[j], b[j + 1]);
+        }
+        // Each epilogue warp stages its own 32 rows x 64 phi columns (4 KB, 128-byte
+        // swizzle) and its lane 0 stores them with TMA, so the warps never wait on each
+        // other; a warp reuses its box once its previous store has read it.
+        const int ox = tc.tn * PH + part * QW;   // first phi column of this warp's box
+        const int oy = tc.tm * BM + quarter * 32;
+        const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
+        const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
+        for (int o = 0; o < (args.C2 ? 2 : 1); ++o) {
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* src = o == 0 ? &pk[4 * c] : &pk2[4 * c];
+            const uint32_t addr = box + lane * 128 + ((c ^ (lane & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(src[0]),
+                         "r"(src[1]), "r"(src[2]), "r"(src[3])
+                         : "memory");
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0 && ox < args.n_valid) {
+            tma_store_4d(o == 0 ? &tmC : &tmC2, box, ox, oy, c2, c3);
+            tma_store_commit();
           }
         }
       }
     }
+    if (MODE == EPI_SWIGLU && lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -357,6 +470,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (uint32_t it = lo; it < issued; ++it)
         mbar_wait(smem_u32(&full[it % STAGES]), (it / STAGES) & 1, abort_flag, nullptr,
                   args.wait_ns, true);
+      if (BRES && b_loads > 0)
+        mbar_wait(smem_u32(b_full), (b_loads - 1) & 1, abort_flag, nullptr, args.wait_ns, true);
     }
     if (warp == 1 && lane == 0 && mma_tiles > 0) {
       const int lt = mma_tiles - 1;
@@ -428,26 +543,57 @@ bool make_map(CUtensorMap* map, const GemmOperand& op, int rows, int K, int Z0, 
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC>
+// Map of a bf16 [rows, cols] output with two batch strides; box {64, 32}.
+bool make_out_map(CUtensorMap* map, void* ptr, int cols, int rows, long long ld, long long s0,
+                  long long s1, int Z0, int Z1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)(s0 ? Z0 : 1),
+                        (cuuint64_t)(s1 ? Z1 : 1)};
+  const cuuint64_t row_bytes = (cuuint64_t)ld * 2;
+  const cuuint64_t plane = ((row_bytes * dims[1]) + 15) & ~(cuuint64_t)15;
+  cuuint64_t strides[3] = {row_bytes, s0 ? (cuuint64_t)s0 * 2 : plane,
+                           s1 ? (cuuint64_t)s1 * 2 : plane * dims[2]};
+  cuuint32_t box[4] = {64, 32, 1, 1};  // one epilogue warp's 32 rows x 64 columns
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES>
 ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mc, mc2;
   if (!make_map(&ma, p.A, p.M, p.K, p.Z0, p.Z1, BM) ||
       !make_map(&mb, p.B, p.N, p.K, p.Z0, p.Z1, BN)) {
     set_error_message("gemm_umma: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", p.M, p.N, p.K);
     return TTT_ERR_CUDA;
   }
-  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC>;
-  constexpr int SMEM = Smem<BN, STAGES>::TOTAL;
+  memset(&mc, 0, sizeof(mc));
+  memset(&mc2, 0, sizeof(mc2));
+  if (MODE == EPI_SWIGLU) {
+    if (!make_out_map(&mc, a.C, a.n_valid, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1) ||
+        (a.C2 && !make_out_map(&mc2, a.C2, a.n_valid, p.M, a.ld2, a.c2s0, a.c2s1, p.Z0, p.Z1))) {
+      set_error_message("gemm_umma: output tensor map encoding failed");
+      return TTT_ERR_CUDA;
+    }
+  }
+  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC, BRES>;
+  constexpr int SMEM = Smem<BN, STAGES, BRES, MODE>::TOTAL;
+  static_assert(SMEM <= 232448, "shared memory budget");
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
       cudaSuccess) {
     set_error_message("gemm_umma: cannot set %d bytes of dynamic shared memory", SMEM);
     return TTT_ERR_CUDA;
   }
-  const long long tiles = (long long)((p.N + BN - 1) / BN) * ((p.M + BM - 1) / BM) * p.Z0 * p.Z1;
+  const long long tiles_n = (p.N + BN - 1) / BN;
+  const long long tiles = tiles_n * ((p.M + BM - 1) / BM) * p.Z0 * p.Z1;
   const int per_sm = (SMEM <= 110 * 1024) ? 2 : 1;
   long long grid = (long long)sm_count() * per_sm;
+  if (BRES) grid = (grid / tiles_n) * tiles_n;  // whole groups of n-tile CTAs
   if (tiles < grid) grid = tiles;
-  kern<<<(unsigned)grid, THREADS, SMEM, s>>>(ma, mb, a);
+  if (grid < 1) grid = 1;
+  kern<<<(unsigned)grid, THREADS, SMEM, s>>>(ma, mb, mc, mc2, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error_message("gemm_umma launch: %s", cudaGetErrorString(e));
@@ -456,14 +602,24 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   return TTT_OK;
 }
 
+// B-resident pays when K fits the resident buffer and the B operand is K-major.
+bool use_bres(const GemmProblem& p, int BN) {
+  return BN == 256 && p.K <= 4 * BK && !p.B.mn_major && (p.N + BN - 1) / BN <= sm_count();
+}
+
 template <int BN, int STAGES, int MODE, typename TC>
 ttt_status dispatch_major(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
+  constexpr int RES_STAGES = MODE == EPI_SWIGLU ? 4 : 6;
+  if (BN == 256 && use_bres(p, BN)) {
+    if (p.A.mn_major) return launch_umma<BN, true, false, RES_STAGES, MODE, TC, true>(p, a, s);
+    return launch_umma<BN, false, false, RES_STAGES, MODE, TC, true>(p, a, s);
+  }
   const int key = (p.A.mn_major ? 2 : 0) | (p.B.mn_major ? 1 : 0);
   switch (key) {
-    case 0: return launch_umma<BN, false, false, STAGES, MODE, TC>(p, a, s);
-    case 1: return launch_umma<BN, false, true, STAGES, MODE, TC>(p, a, s);
-    case 2: return launch_umma<BN, true, false, STAGES, MODE, TC>(p, a, s);
-    default: return launch_umma<BN, true, true, STAGES, MODE, TC>(p, a, s);
+    case 0: return launch_umma<BN, false, false, STAGES, MODE, TC, false>(p, a, s);
+    case 1: return launch_umma<BN, false, true, STAGES, MODE, TC, false>(p, a, s);
+    case 2: return launch_umma<BN, true, false, STAGES, MODE, TC, false>(p, a, s);
+    default: return launch_umma<BN, true, true, STAGES, MODE, TC, false>(p, a, s);
   }
 }
 
@@ -518,8 +674,12 @@ ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_er
 
 bool umma_swiglu_supported(const SwigluGemm& g) {
   const GemmProblem& p = g.gemm;
+  auto strides_ok = [](long long ld, long long s0, long long s1) {
+    return ld % 8 == 0 && s0 % 8 == 0 && s1 % 8 == 0 && s0 >= 0 && s1 >= 0;
+  };
   return umma_supported(p) && p.C.dtype == DT_BF16 && p.N % 256 == 0 && p.beta == 0.0f &&
-         (!g.out2 || aligned16(g.out2));
+         aligned16(p.C.ptr) && strides_ok(p.C.ld, p.C.s0, p.C.s1) &&
+         (!g.out2 || (aligned16(g.out2) && strides_ok(g.ld2, g.s20, g.s21)));
 }
 
 ttt_status gemm_umma_swiglu(const SwigluGemm& g, cudaStream_t stream, unsigned* dev_err,
