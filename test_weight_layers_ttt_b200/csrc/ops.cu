@@ -35,22 +35,38 @@ __global__ void prep_wk_kernel(const float* W0, const float* W2, OT* Wk, int n_e
   }
 }
 
+// Tiled through shared memory so both the reads of W0/W2 (either layout) and the writes
+// of the blocked operand are coalesced. grid (mpad/32, ceil(h/32), 2 * n_entries),
+// block (32, 8); blockIdx.z = 2 * entry + which (0: W0, 1: W2).
 template <typename OT>
-__global__ void prep_wk_blocked_kernel(const float* W0, const float* W2, OT* Wk, int n_entries,
-                                       int src_heads, int h, int m, int layout) {
+__global__ void prep_wk_blocked_kernel(const float* W0, const float* W2, OT* Wk, int src_heads,
+                                       int h, int m, int layout) {
+  __shared__ float tile[32][33];
   const int mpad = (m + 127) / 128 * 128;
-  const long long per = 2LL * mpad * h;
-  TTT_GRID_LOOP(idx, per * n_entries) {
-    const long long e = idx / per, rem = idx - e * per;
-    const int r = (int)(rem / h), i = (int)(rem - (long long)r * h);
-    const int blk = r >> 8, w = r & 255;
-    const int j = blk * 128 + (w & 127);
-    float v = 0.0f;
-    if (j < m) {
-      const float* src = (w < 128 ? W0 : W2) + (e % src_heads) * (long long)h * m;
-      v = layout == 0 ? src[(long long)i * m + j] : src[(long long)j * h + i];
+  const int j0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
+  const int e = blockIdx.z >> 1, which = blockIdx.z & 1;
+  const float* src = (which ? W2 : W0) + (long long)(e % src_heads) * h * m;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  // tile[jj][ii] = W(i0 + ii, j0 + jj), zero past m (padding rows) or past h
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = ty + 8 * k;
+    if (layout == 0) {  // [h, m]: consecutive tx -> consecutive j
+      const int i = i0 + r, j = j0 + tx;
+      tile[tx][r] = (i < h && j < m) ? src[(long long)i * m + j] : 0.0f;
+    } else {            // [m, h]: consecutive tx -> consecutive i
+      const int j = j0 + r, i = i0 + tx;
+      tile[r][tx] = (i < h && j < m) ? src[(long long)j * h + i] : 0.0f;
     }
-    Wk[idx] = from_f32<OT>(v);
+  }
+  __syncthreads();
+  OT* dst = Wk + (long long)e * 2 * mpad * h;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int jj = ty + 8 * k, j = j0 + jj, i = i0 + tx;
+    if (j >= mpad || i >= h) continue;
+    const long long row = (long long)(j >> 7) * 256 + (which ? 128 : 0) + (j & 127);
+    dst[row * h + i] = from_f32<OT>(tile[jj][tx]);
   }
 }
 
@@ -130,6 +146,51 @@ __global__ void chunk_scan_kernel(const float* __restrict__ dS, const float* __r
       }
     }
     if (S_final) S_final[bh * per + (layout == 0 ? e : (long long)j * m + k)] = s;
+  }
+}
+
+// Four consecutive state elements per thread (16-byte loads), for W1 in layout 0 and
+// m*h divisible by 4; the chunk loop keeps four 16-byte loads in flight.
+template <typename OT>
+__global__ void chunk_scan4_kernel(const float4* __restrict__ dS, const float4* __restrict__ W1,
+                                   OT* __restrict__ Sc, float4* __restrict__ S_final, int BH,
+                                   int H, int C, long long per4, int order) {
+  TTT_GRID_LOOP(idx, per4 * BH) {
+    const long long bh = idx / per4, e = idx - bh * per4;
+    float4 s = W1[(bh % H) * per4 + e];
+    const float4* d = dS + bh * C * per4 + e;
+    OT* out = Sc + (bh * C * per4 + e) * 4;
+    auto put = [&](int c, const float4& v) {
+      OT* o = out + (long long)c * per4 * 4;
+      if constexpr (sizeof(OT) == 2) {
+        uint2 pk;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(o) = pk;
+      } else {
+        *reinterpret_cast<float4*>(o) = v;
+      }
+    };
+    int c = 0;
+    for (; c + 4 <= C; c += 4) {
+      float4 dv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) dv[u] = __ldcs(d + (long long)(c + u) * per4);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (order == 1) put(c + u, s);
+        s.x += dv[u].x; s.y += dv[u].y; s.z += dv[u].z; s.w += dv[u].w;
+        if (order != 1) put(c + u, s);
+      }
+    }
+    for (; c < C; ++c) {
+      const float4 dv = __ldcs(d + (long long)c * per4);
+      if (order == 1) put(c, s);
+      s.x += dv.x; s.y += dv.y; s.z += dv.z; s.w += dv.w;
+      if (order != 1) put(c, s);
+    }
+    if (S_final) S_final[bh * per4 + e] = s;
   }
 }
 
@@ -359,10 +420,10 @@ cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, 
                             int src_heads, int h, int m, int src_layout, cudaStream_t s) {
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
-    const long long mpad = (m + 127) / 128 * 128;
-    const long long n = 2LL * mpad * h * n_entries;
-    prep_wk_blocked_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(
-        W0, W2, static_cast<OT*>(Wk), n_entries, src_heads, h, m, src_layout);
+    const int mpad = (m + 127) / 128 * 128;
+    dim3 grid(mpad / 32, (h + 31) / 32, 2 * n_entries);
+    prep_wk_blocked_kernel<OT><<<grid, dim3(32, 8), 0, s>>>(
+        W0, W2, static_cast<OT*>(Wk), src_heads, h, m, src_layout);
     return cudaGetLastError();
   });
 }
@@ -389,11 +450,21 @@ cudaError_t grad_prep(int ot, const float* AB, const float* Dv, long long rows, 
 
 cudaError_t chunk_scan(int ot, const float* dS, const float* W1, void* Sc, float* S_final, int BH,
                        int H, int C, int m, int h, int order, int layout, cudaStream_t s) {
+  const long long per = (long long)m * h;
+  const bool vec = layout == 0 && per % 4 == 0 &&
+                   ((reinterpret_cast<uintptr_t>(dS) | reinterpret_cast<uintptr_t>(W1) |
+                     reinterpret_cast<uintptr_t>(Sc) | reinterpret_cast<uintptr_t>(S_final)) & 15) == 0;
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
-    const long long n = (long long)m * h * BH;
-    chunk_scan_kernel<OT><<<grid_for(n, 256, 148 * 64), 256, 0, s>>>(
-        dS, W1, static_cast<OT*>(Sc), S_final, BH, H, C, m, h, order, layout);
+    if (vec) {
+      const long long n4 = per / 4 * BH;
+      chunk_scan4_kernel<OT><<<grid_for(n4, 256, 148 * 16), 256, 0, s>>>(
+          reinterpret_cast<const float4*>(dS), reinterpret_cast<const float4*>(W1),
+          static_cast<OT*>(Sc), reinterpret_cast<float4*>(S_final), BH, H, C, per / 4, order);
+    } else {
+      chunk_scan_kernel<OT><<<grid_for(per * BH, 256, 148 * 64), 256, 0, s>>>(
+          dS, W1, static_cast<OT*>(Sc), S_final, BH, H, C, m, h, order, layout);
+    }
     return cudaGetLastError();
   });
 }
