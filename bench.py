@@ -66,42 +66,34 @@ def layer_bytes(wl, form: str) -> float:
     return float(act + weights + state_out)
 
 
-def kernel_work(name: str, wl, calls: int):
-    """(bound, algorithmic work per launch) of a traced kernel; work in FLOP or bytes."""
+def kernel_work(name: str, wl, form: str):
+    """(bound, algorithmic work of one whole step) of a traced kernel: FLOP for tensor
+    kernels, HBM bytes for memory-bound ones. Per-launch work = this / launches per step."""
     base = name.split("@")[0]
-    BH, N, h, m = wl.B * wl.H, wl.N, wl.h, wl.m
-    rows_par = BH * N
-    C = wl.C
+    BH, h, m = wl.B * wl.H, wl.h, wl.m
+    T = BH * wl.N
     es = 2 if wl.dtype == "bf16" else 4
-    if wl_form(name) == "recurrent":
-        rows = BH * wl.chunk
+    if form == "recurrent":
         table = {
-            "gemm_features_k": ("tensor", 4.0 * h * m * rows),
-            "gemm_features_q": ("tensor", 4.0 * h * m * rows),
-            "gemm_v_w1t": ("tensor", 2.0 * h * m * rows),
-            "gemm_grad_w1": ("tensor", 2.0 * h * m * rows),
-            "gemm_grad_w0": ("tensor", 2.0 * h * m * rows),
-            "gemm_grad_w2": ("tensor", 2.0 * h * m * rows),
-            "gemm_output": ("tensor", 2.0 * h * m * rows),
+            "gemm_features_k": ("tensor", 4.0 * h * m * T),
+            "gemm_features_q": ("tensor", 4.0 * h * m * T),
+            "gemm_v_w1t": ("tensor", 2.0 * h * m * T),
+            "gemm_grad_w1": ("tensor", 2.0 * h * m * T),
+            "gemm_grad_w0": ("tensor", 2.0 * h * m * T),
+            "gemm_grad_w2": ("tensor", 2.0 * h * m * T),
+            "gemm_output": ("tensor", 2.0 * h * m * T),
         }
         return table.get(base, (None, None))
     table = {
-        "gemm_features_k": ("tensor", 4.0 * h * m * rows_par),
-        "gemm_features_q": ("tensor", 4.0 * h * m * rows_par),
-        "gemm_state_delta": ("tensor", 2.0 * h * m * rows_par),
-        "gemm_output": ("tensor", 2.0 * h * m * rows_par),
-        "chunk_scan": ("hbm", BH * C * h * m * (4.0 + es) + 2 * 4.0 * BH * h * m),
-        "swiglu_k": ("hbm", rows_par * m * (8.0 + es * (1 if wl.kind != "inplace" else 2))),
-        "swiglu_q": ("hbm", rows_par * m * (8.0 + es)),
+        "gemm_features_k": ("tensor", 4.0 * h * m * T),
+        "gemm_features_q": ("tensor", 4.0 * h * m * T),
+        "gemm_state_delta": ("tensor", 2.0 * h * m * T),
+        "gemm_output": ("tensor", 2.0 * h * m * T),
+        "chunk_scan": ("hbm", BH * wl.C * h * m * (4.0 + es) + 2 * 4.0 * BH * h * m),
+        "swiglu_k": ("hbm", T * m * (8.0 + es * (1 if wl.kind != "inplace" else 2))),
+        "swiglu_q": ("hbm", T * m * (8.0 + es)),
     }
     return table.get(base, (None, None))
-
-
-_FORM_OF_TRACE = {}
-
-
-def wl_form(name):
-    return _FORM_OF_TRACE.get(name, "parallel")
 
 
 # ----------------------------------------------------------------------------- environment
@@ -283,13 +275,13 @@ def _kernel_table(trace, steps):
     return dict(sorted(table.items(), key=lambda kv: -kv[1]["ms_total"]))
 
 
-def _roofline(table, wl, peaks, form):
+def _roofline(table, wl, peaks, form, steps):
     """Roofline of the dominant kernel (largest share) with a known algorithmic work."""
     for name, e in table.items():
-        _FORM_OF_TRACE[name] = form
-        bound, work = kernel_work(name, wl, e["launches"])
+        bound, step_work = kernel_work(name, wl, form)
         if bound is None:
             continue
+        work = step_work / (e["launches"] / steps)
         secs = e["ms_avg"] / 1e3
         if bound == "tensor":
             achieved = work / secs / 1e12
@@ -362,7 +354,7 @@ def run_gpu(args, rank, local, world):
             "gpu_launches": len(trace),
             "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv)
                             for kk, vv in v.items()} for k, v in table.items()},
-            "roofline": _roofline(table, wl, peaks, form),
+            "roofline": _roofline(table, wl, peaks, form, steps),
             "clocks": clk.summary(),
         }
 

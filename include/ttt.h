@@ -162,7 +162,7 @@ ttt_status ttt_la_parallel_fwd_noalloc(const ttt_desc* desc, const void* q, cons
  * X <- X - sign * u, and optional renormalisation of each column (output unit) over the
  * input dimension to the column norm the matrix had at the start of the call.
  *
- *   desc       problem; w_in_layout and w1_layout must be 0
+ *   desc       problem; w_in_layout and w1_layout must be 0; h, m <= 1536
  *   alpha      [B,H,C] fp32, required when desc->momentum, else ignored (may be NULL)
  *   W0, W2, W1 per-head initial weights [H,h,m], [H,h,m], [H,m,h] fp32
  *   out        [B,H,N,h] dtype, written

@@ -57,6 +57,11 @@ ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_er
 // carries matching A and B columns. The epilogue writes phi = silu(A) * B times
 // rowscale[z0*rs0 + z1*rs1 + row] (or 1 when rowscale is null) to gemm.C (bf16, row stride
 // gemm.C.ld, phi columns < n_valid) and, when out2 is set, the unscaled phi to out2.
+//
+// Gradient variant (grad = 1, recurrent form): with eta = rowscale and d = -eta * Dv, Dv =
+// V W1^T given in `dv` (bf16 [rows, n_valid] with its own strides), the epilogue writes
+// P = phi * eta to gemm.C, E2 = d * silu(A) to out2 (when set) and E0 = d * B * silu'(A)
+// to out3 (when set).
 struct SwigluGemm {
   GemmProblem gemm;
   void* out2 = nullptr;
@@ -64,6 +69,11 @@ struct SwigluGemm {
   const float* rowscale = nullptr;
   long long rs0 = 0, rs1 = 0;
   int n_valid = 0;
+  int grad = 0;
+  void* out3 = nullptr;
+  long long ld3 = 0, s30 = 0, s31 = 0;
+  const void* dv = nullptr;
+  long long ldd = 0, ds0 = 0, ds1 = 0;
 };
 bool umma_swiglu_supported(const SwigluGemm& g);
 ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream);

@@ -100,6 +100,10 @@ struct SimtSwiglu {
   SimtArgs g;
   void* C2; long long ld2, c2s0, c2s1;
   const float* rs; long long rs0, rs1;
+  // gradient variant (see SwigluGemm): C = phi * eta, C2 = d silu(A), C3 = d B silu'(A)
+  int grad;
+  void* C3;
+  const void* dv; long long ldd, ds0, ds1;
 };
 
 template <typename TA, typename TB, typename TC>
@@ -163,6 +167,8 @@ __global__ void __launch_bounds__(THREADS) simt_swiglu_kernel(const SimtSwiglu s
   }
   TC* C = static_cast<TC*>(a.C) + z0 * a.cs0 + z1 * a.cs1;
   TC* C2 = sw.C2 ? static_cast<TC*>(sw.C2) + z0 * sw.c2s0 + z1 * sw.c2s1 : nullptr;
+  TC* C3 = sw.C3 ? static_cast<TC*>(sw.C3) + z0 * a.cs0 + z1 * a.cs1 : nullptr;
+  const TC* DV = sw.dv ? static_cast<const TC*>(sw.dv) + z0 * sw.ds0 + z1 * sw.ds1 : nullptr;
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const int gi = i0 + ty + 16 * r;
@@ -172,9 +178,17 @@ __global__ void __launch_bounds__(THREADS) simt_swiglu_kernel(const SimtSwiglu s
     for (int c = 0; c < 4; ++c) {
       const int gj = j0 + tx + 16 * c;
       if (gj >= a.N) continue;
-      const float p = siluf_(acc_a[r][c]) * acc_b[r][c];
+      const float av = acc_a[r][c], bv = acc_b[r][c];
+      const float sa = siluf_(av);
+      const float p = sa * bv;
       C[(long long)gi * a.ldc + gj] = from_f32<TC>(p * rsv);
-      if (C2) C2[(long long)gi * sw.ld2 + gj] = from_f32<TC>(p);
+      if (sw.grad) {
+        const float d = -rsv * to_f32(DV[(long long)gi * sw.ldd + gj]);
+        if (C2) C2[(long long)gi * a.ldc + gj] = from_f32<TC>(d * sa);
+        if (C3) C3[(long long)gi * a.ldc + gj] = from_f32<TC>(d * bv * silu_primef_(av));
+      } else if (C2) {
+        C2[(long long)gi * sw.ld2 + gj] = from_f32<TC>(p);
+      }
     }
   }
 }
@@ -199,6 +213,14 @@ ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream) {
   a.alpha = 1.0f; a.beta = 0.0f;
   sw.C2 = g.out2; sw.ld2 = g.ld2; sw.c2s0 = g.s20; sw.c2s1 = g.s21;
   sw.rs = g.rowscale; sw.rs0 = g.rs0; sw.rs1 = g.rs1;
+  sw.grad = g.grad;
+  sw.C3 = g.grad ? g.out3 : nullptr;
+  sw.dv = g.grad ? g.dv : nullptr;
+  sw.ldd = g.ldd; sw.ds0 = g.ds0; sw.ds1 = g.ds1;
+  if (g.grad && (!g.rowscale || !g.dv)) {
+    set_error_message("gemm_simt_swiglu: the gradient variant needs eta and Dv");
+    return TTT_ERR_INVALID_ARG;
+  }
   dim3 grid((g.n_valid + TN - 1) / TN, (unsigned)gy, (unsigned)gz);
   using bf = __nv_bfloat16;
   const int key = (p.A.dtype << 2) | (p.B.dtype << 1) | p.C.dtype;

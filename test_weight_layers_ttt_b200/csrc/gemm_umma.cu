@@ -49,6 +49,10 @@ struct UArgs {
   void* C2; long long ld2, c2s0, c2s1;
   const float* rs; long long rs0, rs1;
   int n_valid;
+  // SWIGLU gradient variant: third output and the Dv input (bf16)
+  int grad;
+  void* C3;
+  const __nv_bfloat16* dv; long long ldd, ds0, ds1;
   unsigned* err;
   unsigned long long wait_ns;
 };
@@ -173,12 +177,16 @@ struct TileWalker {
   }
 };
 
+// Tensor maps of the (up to three) TMA-stored outputs of the SWIGLU epilogue.
+struct OutMaps {
+  CUtensorMap m[3];
+};
+
 template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES>
 __global__ void __launch_bounds__(THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC,
-                     const __grid_constant__ CUtensorMap tmC2, const UArgs args) {
+                     const __grid_constant__ OutMaps om, const UArgs args) {
   using L = Smem<BN, STAGES, BRES, MODE>;
   constexpr uint32_t ACC_COLS = 2 * BN;  // two accumulators
   extern __shared__ uint8_t smem_raw[];
@@ -392,6 +400,87 @@ __global__ void __launch_bounds__(THREADS, 1)
             store_vals(crow + col0, w, nv, vec);
           }
         }
+      } else if (args.grad) {
+        // Gradient pieces of the recurrent form. Each output is produced in two 32-column
+        // halves straight from TMEM (re-read per output to keep registers low) into this
+        // warp's staging box, then stored with TMA; TMEM is released after the last read.
+        constexpr int PH = BN / 2;
+        constexpr int QW = PH / 2;
+        const bool live = row < args.M;
+        const float eta = live ? args.rs[tc.z0 * args.rs0 + tc.z1 * args.rs1 + row] : 0.0f;
+        const __nv_bfloat16* dvrow =
+            args.dv + tc.z0 * args.ds0 + tc.z1 * args.ds1 + (long long)(live ? row : 0) * args.ldd;
+        const int ox = tc.tn * PH + part * QW;
+        const int oy = tc.tm * BM + quarter * 32;
+        const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
+        const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
+        for (int o = 0; o < 3; ++o) {
+          if ((o == 1 && !args.C2) || (o == 2 && !args.C3)) continue;
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t ra[32], rb[32];
+            tmem_ld32(lane_addr + (uint32_t)(part * QW + hh * 32), ra);
+            tmem_ld32(lane_addr + (uint32_t)(PH + part * QW + hh * 32), rb);
+            tmem_ld_wait();
+            const int col0 = ox + hh * 32;
+            float dvv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dvv[j] = 0.0f;
+            if (o > 0 && live) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                if (col0 + j + 8 <= args.n_valid) {
+                  const uint4 u = *reinterpret_cast<const uint4*>(dvrow + col0 + j);
+                  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) {
+                    const float2 f = __bfloat1622float2(h2[q]);
+                    dvv[j + 2 * q] = f.x;
+                    dvv[j + 2 * q + 1] = f.y;
+                  }
+                }
+              }
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float v[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const float a = __uint_as_float(ra[j + u]), bb = __uint_as_float(rb[j + u]);
+                const float hlf = 0.5f * a;
+                float t;
+                asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hlf));
+                const float sg = fmaf(0.5f, t, 0.5f);   // sigmoid(a)
+                const float sa = a * sg;                // silu(a)
+                const float d = -eta * dvv[j + u];
+                if (o == 0) v[u] = sa * bb * eta;
+                else if (o == 1) v[u] = d * sa;
+                else v[u] = d * bb * sg * fmaf(a, 1.0f - sg, 1.0f);
+              }
+              pk[j / 2] = pack_bf16x2(v[0], v[1]);
+            }
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const int c = hh * 4 + cc;
+              const uint32_t addr = box + lane * 128 + ((c ^ (lane & 7)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                           "r"(pk[4 * cc]), "r"(pk[4 * cc + 1]), "r"(pk[4 * cc + 2]),
+                           "r"(pk[4 * cc + 3])
+                           : "memory");
+            }
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0 && ox < args.n_valid) {
+            tma_store_4d(&om.m[o], box, ox, oy, c2, c3);
+            tma_store_commit();
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[buf]));
       } else {
         // SWIGLU: phi column p of this tile uses accumulator columns p (A) and BN/2 + p (B).
         constexpr int PH = BN / 2;       // phi columns per tile
@@ -452,7 +541,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0 && ox < args.n_valid) {
-            tma_store_4d(o == 0 ? &tmC : &tmC2, box, ox, oy, c2, c3);
+            tma_store_4d(&om.m[o], box, ox, oy, c2, c3);
             tma_store_commit();
           }
         }
@@ -563,17 +652,19 @@ bool make_out_map(CUtensorMap* map, void* ptr, int cols, int rows, long long ld,
 
 template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES>
 ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  CUtensorMap ma, mb, mc, mc2;
+  CUtensorMap ma, mb;
+  OutMaps om;
   if (!make_map(&ma, p.A, p.M, p.K, p.Z0, p.Z1, BM) ||
       !make_map(&mb, p.B, p.N, p.K, p.Z0, p.Z1, BN)) {
     set_error_message("gemm_umma: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", p.M, p.N, p.K);
     return TTT_ERR_CUDA;
   }
-  memset(&mc, 0, sizeof(mc));
-  memset(&mc2, 0, sizeof(mc2));
+  memset(&om, 0, sizeof(om));
   if (MODE == EPI_SWIGLU) {
-    if (!make_out_map(&mc, a.C, a.n_valid, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1) ||
-        (a.C2 && !make_out_map(&mc2, a.C2, a.n_valid, p.M, a.ld2, a.c2s0, a.c2s1, p.Z0, p.Z1))) {
+    // out2 / out3 share gemm.C's strides except for their own row stride and base
+    if (!make_out_map(&om.m[0], a.C, a.n_valid, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1) ||
+        (a.C2 && !make_out_map(&om.m[1], a.C2, a.n_valid, p.M, a.ld2, a.c2s0, a.c2s1, p.Z0, p.Z1)) ||
+        (a.C3 && !make_out_map(&om.m[2], a.C3, a.n_valid, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1))) {
       set_error_message("gemm_umma: output tensor map encoding failed");
       return TTT_ERR_CUDA;
     }
@@ -593,7 +684,7 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   if (BRES) grid = (grid / tiles_n) * tiles_n;  // whole groups of n-tile CTAs
   if (tiles < grid) grid = tiles;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, THREADS, SMEM, s>>>(ma, mb, mc, mc2, a);
+  kern<<<(unsigned)grid, THREADS, SMEM, s>>>(ma, mb, om, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error_message("gemm_umma launch: %s", cudaGetErrorString(e));
@@ -677,8 +768,13 @@ bool umma_swiglu_supported(const SwigluGemm& g) {
   auto strides_ok = [](long long ld, long long s0, long long s1) {
     return ld % 8 == 0 && s0 % 8 == 0 && s1 % 8 == 0 && s0 >= 0 && s1 >= 0;
   };
+  const bool grad_ok =
+      !g.grad || (g.rowscale && g.dv && aligned16(g.dv) && strides_ok(g.ldd, g.ds0, g.ds1) &&
+                  (!g.out3 || (aligned16(g.out3) && g.ld3 == p.C.ld && g.s30 == p.C.s0 &&
+                               g.s31 == p.C.s1)) &&
+                  (!g.out2 || (g.ld2 == p.C.ld && g.s20 == p.C.s0 && g.s21 == p.C.s1)));
   return umma_supported(p) && p.C.dtype == DT_BF16 && p.N % 256 == 0 && p.beta == 0.0f &&
-         aligned16(p.C.ptr) && strides_ok(p.C.ld, p.C.s0, p.C.s1) &&
+         aligned16(p.C.ptr) && strides_ok(p.C.ld, p.C.s0, p.C.s1) && grad_ok &&
          (!g.out2 || (aligned16(g.out2) && strides_ok(g.ld2, g.s20, g.s21)));
 }
 
@@ -694,6 +790,11 @@ ttt_status gemm_umma_swiglu(const SwigluGemm& g, cudaStream_t stream, unsigned* 
   a.C2 = g.out2; a.ld2 = g.ld2; a.c2s0 = g.s20; a.c2s1 = g.s21;
   a.rs = g.rowscale; a.rs0 = g.rs0; a.rs1 = g.rs1;
   a.n_valid = g.n_valid;
+  a.grad = g.grad;
+  a.C3 = g.grad ? g.out3 : nullptr;
+  a.dv = static_cast<const __nv_bfloat16*>(g.dv);
+  a.ldd = g.ldd; a.ds0 = g.ds0; a.ds1 = g.ds1;
+  if (!g.grad) a.dv = nullptr;
   return dispatch_major<256, 4, EPI_SWIGLU, __nv_bfloat16>(p, a, stream);
 }
 

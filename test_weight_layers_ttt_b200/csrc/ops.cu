@@ -239,6 +239,33 @@ __global__ void col_norms_kernel(const float* W0, const float* W2, const float* 
   }
 }
 
+// Four consecutive elements per thread (requires h*m divisible by 4 and 16-byte bases).
+__global__ void rec_reduce4_kernel(const float4* __restrict__ partials, int splits,
+                                   float4* __restrict__ U, float4* __restrict__ M_all,
+                                   const float* __restrict__ alpha, int C, int c, int BH,
+                                   long long hm4, int mask) {
+  const long long per4 = 3 * hm4, total4 = per4 * BH;
+  TTT_GRID_LOOP(idx, total4) {
+    const long long bh = idx / per4;
+    const int p = (int)((idx - bh * per4) / hm4);
+    if (!(mask & (1 << p))) continue;
+    float4 g = partials[idx];
+    for (int s = 1; s < splits; ++s) {
+      const float4 q = partials[(long long)s * total4 + idx];
+      g.x += q.x; g.y += q.y; g.z += q.z; g.w += q.w;
+    }
+    if (M_all) {
+      const float a = alpha[bh * C + c];
+      float4 mv = M_all[idx];
+      mv.x = fmaf(a, mv.x, g.x); mv.y = fmaf(a, mv.y, g.y);
+      mv.z = fmaf(a, mv.z, g.z); mv.w = fmaf(a, mv.w, g.w);
+      M_all[idx] = mv;
+      g = mv;
+    }
+    U[idx] = g;
+  }
+}
+
 __global__ void rec_reduce_kernel(const float* partials, int splits, float* U, float* M_all,
                                   const float* alpha, int C, int c, int BH, int h, int m,
                                   int mask) {
@@ -303,47 +330,71 @@ __global__ void ns_writeback_kernel(const float* X, float* U, int h, int m, int 
   }
 }
 
-// grid (ceil(max cols / 32), 3, BH), block (32, 8): one column per threadIdx.x.
+// grid (ceil(max cols / 32), 3, BH), block (32, 32), dynamic shared memory 32 x (R + 1)
+// floats: one column per threadIdx.x, rows strided by 32 over threadIdx.y. Three phases,
+// each with all threads' loads independent: column sums of (W - sign U)^2; the new values
+// written to the fp32 master and W1o (coalesced along columns) and kept in shared memory;
+// for W0 / W2 the shared-memory columns written out as rows of the blocked operand Wk
+// (coalesced along the input dimension).
 template <typename OT>
-__global__ void rec_step_kernel(float* W_all, const float* U, const float* tnorm, int H, int h,
-                                int m, int mask, int sign, int renorm, OT* Wk, OT* W1o) {
+__global__ void __launch_bounds__(1024) rec_step_kernel(float* W_all, const float* U,
+                                                        const float* tnorm, int H, int h, int m,
+                                                        int mask, int sign, int renorm, OT* Wk,
+                                                        OT* W1o) {
+  extern __shared__ float colbuf[];  // [32][R + 1]
+  __shared__ float red[32][33];
   const int p = blockIdx.y, bh = blockIdx.z;
   if (!(mask & (1 << p))) return;
   int R, Cc;
   part_dims(p, h, m, R, Cc);
-  const int c = blockIdx.x * 32 + threadIdx.x;
+  const int c0 = blockIdx.x * 32;
+  if (c0 >= Cc) return;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int c = c0 + tx;
   const bool live = c < Cc;
   const long long hm = (long long)h * m;
   float* w = W_all + (long long)bh * 3 * hm + p * hm;
   const float* u = U + (long long)bh * 3 * hm + p * hm;
   const float sg = (float)sign;
-  __shared__ float red[8][33];
   float ss = 0.0f;
-  if (live)
-    for (int r = threadIdx.y; r < R; r += 8) {
+  if (live) {
+#pragma unroll 4
+    for (int r = ty; r < R; r += 32) {
       const float v = w[(long long)r * Cc + c] - sg * u[(long long)r * Cc + c];
-      ss += v * v;
+      ss = fmaf(v, v, ss);
     }
-  red[threadIdx.y][threadIdx.x] = ss;
+  }
+  red[ty][tx] = ss;
   __syncthreads();
   float scale = 1.0f;
-  if (renorm) {
+  if (renorm && live) {
     float tot = 0.0f;
-    for (int y = 0; y < 8; ++y) tot += red[y][threadIdx.x];
+#pragma unroll 8
+    for (int y = 0; y < 32; ++y) tot += red[y][tx];
     const float* tn = tnorm + (long long)(bh % H) * (2 * m + h) + (p == 0 ? 0 : p == 1 ? m : m + h);
-    if (live) scale = tn[c] / sqrtf(tot);
+    scale = tn[c] / sqrtf(tot);
   }
-  if (!live) return;
-  for (int r = threadIdx.y; r < R; r += 8) {
-    const long long o = (long long)r * Cc + c;
-    const float v = (w[o] - sg * u[o]) * scale;
-    w[o] = v;
-    if (p == 1) {
-      W1o[(long long)bh * hm + o] = from_f32<OT>(v);
-    } else {
-      // Wk[bh] = [W0^T ; W2^T], [2m, h]: row (p==2 ? m : 0) + c, column r.
-      Wk[(long long)bh * 2 * hm + ((long long)(p == 2 ? m : 0) + c) * h + r] = from_f32<OT>(v);
+  float* mycol = colbuf + (long long)tx * (R + 1);
+  if (live) {
+#pragma unroll 4
+    for (int r = ty; r < R; r += 32) {
+      const long long o = (long long)r * Cc + c;
+      const float v = (w[o] - sg * u[o]) * scale;
+      w[o] = v;
+      if (p == 1) W1o[(long long)bh * hm + o] = from_f32<OT>(v);
+      else mycol[r] = v;
     }
+  }
+  if (p == 1) return;
+  __syncthreads();
+  const int mpad = (m + 127) / 128 * 128;
+  OT* wk = Wk + (long long)bh * 2 * mpad * h;
+  // warp ty writes column c0 + ty as one Wk row, lanes along the input dimension
+  for (int cc = ty; cc < 32 && c0 + cc < Cc; cc += 32) {
+    const int col = c0 + cc;
+    const long long row = (long long)(col >> 7) * 256 + (p == 2 ? 128 : 0) + (col & 127);
+    const float* src = colbuf + (long long)cc * (R + 1);
+    for (int r = tx; r < R; r += 32) wk[row * h + r] = from_f32<OT>(src[r]);
   }
 }
 
@@ -492,9 +543,18 @@ cudaError_t col_norms(const float* W0, const float* W2, const float* W1, int H, 
 cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all,
                        const float* alpha, int C, int c, int BH, int h, int m, int mask,
                        cudaStream_t s) {
-  const long long n = 3LL * h * m * BH;
-  rec_reduce_kernel<<<grid_for(n, 256), 256, 0, s>>>(partials, splits, U, M_all, alpha, C, c, BH,
-                                                     h, m, mask);
+  const long long hm = (long long)h * m, n = 3 * hm * BH;
+  const bool vec = hm % 4 == 0 &&
+                   ((reinterpret_cast<uintptr_t>(partials) | reinterpret_cast<uintptr_t>(U) |
+                     reinterpret_cast<uintptr_t>(M_all)) & 15) == 0;
+  if (vec) {
+    rec_reduce4_kernel<<<grid_for(n / 4, 256), 256, 0, s>>>(
+        reinterpret_cast<const float4*>(partials), splits, reinterpret_cast<float4*>(U),
+        reinterpret_cast<float4*>(M_all), alpha, C, c, BH, hm / 4, mask);
+  } else {
+    rec_reduce_kernel<<<grid_for(n, 256), 256, 0, s>>>(partials, splits, U, M_all, alpha, C, c,
+                                                       BH, h, m, mask);
+  }
   return cudaGetLastError();
 }
 
@@ -516,10 +576,16 @@ cudaError_t rec_step(float* W_all, const float* U, const float* tnorm, int BH, i
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
     const int maxc = h > m ? h : m;
+    const int maxr = h > m ? h : m;
+    const size_t smem = (size_t)32 * (maxr + 1) * sizeof(float);
+    auto kern = rec_step_kernel<OT>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+      return cudaErrorInvalidValue;
     dim3 grid((maxc + 31) / 32, 3, BH);
-    rec_step_kernel<OT><<<grid, dim3(32, 8), 0, s>>>(W_all, U, tnorm, H, h, m, mask, sign,
-                                                     renorm, static_cast<OT*>(Wk),
-                                                     static_cast<OT*>(W1o));
+    kern<<<grid, dim3(32, 32), smem, s>>>(W_all, U, tnorm, H, h, m, mask, sign, renorm,
+                                          static_cast<OT*>(Wk), static_cast<OT*>(W1o));
     return cudaGetLastError();
   });
 }

@@ -62,7 +62,9 @@ cudaError_t ns_normalize(const float* U, float* X, int BH, int h, int m, int mas
                          cudaStream_t s);
 cudaError_t ns_writeback(const float* X, float* U, int BH, int h, int m, int mask,
                          cudaStream_t s);
-// W <- W - sign * U, optional per-column renormalisation to tnorm, refresh OT copies.
+// W <- W - sign * U, optional per-column renormalisation to tnorm, refresh the OT copies:
+// W1o [BH, m, h] and the blocked input-side operand Wk [BH, 2 * mpad, h] (see
+// prep_wk_blocked).
 cudaError_t rec_step(float* W_all, const float* U, const float* tnorm, int BH, int H, int h,
                      int m, int mask, int sign, int renorm, void* Wk, void* W1o, int ot,
                      cudaStream_t s);

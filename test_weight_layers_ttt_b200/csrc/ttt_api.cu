@@ -187,6 +187,8 @@ ttt_status check_desc(const ttt_desc* d, int path) {
     if (d->ns_steps < 0 || d->ns_steps > 8) return fail(TTT_ERR_INVALID_ARG, "ns_steps must be in 0..8");
     if (d->w_in_layout != 0 || d->w1_layout != 0)
       return fail(TTT_ERR_UNSUPPORTED, "recurrent form: only the default weight layouts");
+    if (d->h > 1536 || d->m > 1536)
+      return fail(TTT_ERR_UNSUPPORTED, "recurrent form: h and m must be <= 1536");
   } else {
     return fail(TTT_ERR_INVALID_ARG, "path must be TTT_PATH_PARALLEL or TTT_PATH_RECURRENT");
   }
@@ -307,19 +309,18 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
 
 // ------------------------------------------------------------------ recurrent form
 struct RecBufs {
-  float* W_all;
-  float* M_all;
-  float* U;
-  float* tnorm;
-  void* Wk;
-  void* W1o;
-  float* AB;
-  float* Dv;
-  void* P;
-  void* E2;
-  void* E0;
+  float* W_all;   // fp32 masters [BH][W0 | W1 | W2]
+  float* M_all;   // momentum, same layout
+  float* U;       // update, same layout
+  float* tnorm;   // initial column norms per head
+  void* Wk;       // [BH, 2*mpad, h] blocked [W0^T ; W2^T] operand
+  void* W1o;      // [BH, m, h] W1 operand
+  void* Dv;       // [BH, chunk, m] V W1^T
+  void* P;        // [BH, chunk, m] phi * eta
+  void* E2;       // [BH, chunk, m] d * silu(A)
+  void* E0;       // [BH, chunk, m] d * B * silu'(A)
   float* partials;
-  void* phiQ;
+  void* phiQ;     // [BH, chunk, m]
   float* X;
   float* X2;
   float* Ag;
@@ -327,15 +328,16 @@ struct RecBufs {
   int splits;
 };
 
-// Token splits of the gradient reductions: a divisor of the chunk length L such that the
-// split length stays a multiple of 64 and the three gradient GEMMs give the GPU enough CTAs.
+// Token splits of the gradient reductions: the largest power of two that divides the chunk
+// length, keeps split lengths a multiple of 64 (and >= 256), and keeps the grid of the
+// gradient GEMMs within about two CTAs per SM.
 int choose_splits(const ttt_desc& d, long long L) {
   const long long BH = (long long)d.B * d.H;
   const long long tiles = BH * ((d.m + 127) / 128) * ((d.h + 255) / 256);
   long long best = 1;
   for (long long sp = 2; sp <= 64; sp *= 2) {
-    if (L % sp != 0 || (L / sp) % 64 != 0 || L / sp < 128) break;
-    if (tiles * (sp / 2) >= 2 * 148) break;
+    if (L % sp != 0 || (L / sp) % 64 != 0 || L / sp < 256) break;
+    if (tiles * sp > 2 * 148) break;
     best = sp;
   }
   return (int)best;
@@ -351,10 +353,9 @@ size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
   b.M_all = d.momentum ? cv.take_n<float>(BH * 3 * hm) : nullptr;
   b.U = cv.take_n<float>(BH * 3 * hm);
   b.tnorm = cv.take_n<float>((long long)d.H * (2 * d.m + d.h));
-  b.Wk = cv.take(os * BH * 2 * hm);
+  b.Wk = cv.take(os * BH * 2 * padded_m(d.m) * d.h);
   b.W1o = cv.take(os * BH * hm);
-  b.AB = cv.take_n<float>(rows * 2 * d.m);
-  b.Dv = cv.take_n<float>(rows * d.m);
+  b.Dv = cv.take(os * rows * d.m);
   b.P = cv.take(os * rows * d.m);
   b.E2 = cv.take(os * rows * d.m);
   b.E0 = cv.take(os * rows * d.m);
@@ -372,22 +373,32 @@ size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
   return cv.off;
 }
 
+// Features of tokens [t0, t0 + Lc) of every (b, head) against that (b, head)'s own blocked
+// weights; rows of the outputs are chunk-local ([BH, chunk, m]).
+SwigluGemm rec_features(const ttt_desc& d, const void* X, const RecBufs& b, long long t0,
+                        long long Lc, void* out) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, mp = padded_m(d.m);
+  const long long L = d.chunk;
+  SwigluGemm g;
+  GemmProblem& p = g.gemm;
+  p.M = (int)Lc; p.N = (int)(2 * mp); p.K = d.h; p.Z0 = (int)BH; p.Z1 = 1;
+  p.A = {static_cast<const char*>(X) + t0 * h * dtype_size(ot), ot, false, h, N * h, 0};
+  p.B = {b.Wk, ot, false, h, 2 * mp * h, 0};
+  p.C = {out, ot, m, L * m, 0};
+  g.n_valid = d.m;
+  return g;
+}
+
 ttt_status rec_apply(const ttt_desc& d, const void* q, void* out, long long t0, long long Lc,
                      const RecBufs& b, cudaStream_t s) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const size_t es = dtype_size(ot);
-  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m;
-  GemmProblem p;
-  p.M = (int)Lc; p.N = 2 * d.m; p.K = d.h; p.Z0 = (int)BH; p.Z1 = 1;
-  p.A = {static_cast<const char*>(q) + t0 * h * es, ot, false, h, N * h, 0};
-  p.B = {b.Wk, ot, false, h, 2 * m * h, 0};
-  p.C = {b.AB, DT_F32, 2 * m, Lc * 2 * m, 0};
-  TTT_TRY(run_gemm("gemm_features_q", p, s));
-  EtaMap em{nullptr, Lc, N, t0};
-  TTT_OP("swiglu_q", swiglu(ot, b.AB, BH * Lc, d.m, em, nullptr, b.phiQ, s));
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, L = d.chunk;
+  TTT_TRY(run_swiglu("gemm_features_q", rec_features(d, q, b, t0, Lc, b.phiQ), s));
   GemmProblem o;
   o.M = (int)Lc; o.N = d.h; o.K = d.m; o.Z0 = (int)BH; o.Z1 = 1;
-  o.A = {b.phiQ, ot, false, m, Lc * m, 0};
+  o.A = {b.phiQ, ot, false, m, L * m, 0};
   o.B = {b.W1o, ot, true, h, m * h, 0};
   o.C = {static_cast<char*>(out) + t0 * h * es, ot, h, N * h, 0};
   return run_gemm("gemm_output", o, s);
@@ -399,28 +410,33 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const size_t es = dtype_size(ot);
   const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, hm = h * m;
+  const long long L = d.chunk;
   const int mask = d.update_mask;
   const bool need_in = (mask & (TTT_UPDATE_W0 | TTT_UPDATE_W2)) != 0;
   const long long C = (N + d.chunk - 1) / d.chunk;
-  // [A | B] = K_c [W0 | W2]
-  GemmProblem p;
-  p.M = (int)Lc; p.N = 2 * d.m; p.K = d.h; p.Z0 = (int)BH; p.Z1 = 1;
-  p.A = {static_cast<const char*>(k) + t0 * h * es, ot, false, h, N * h, 0};
-  p.B = {b.Wk, ot, false, h, 2 * m * h, 0};
-  p.C = {b.AB, DT_F32, 2 * m, Lc * 2 * m, 0};
-  TTT_TRY(run_gemm("gemm_features_k", p, s));
   if (need_in) {  // Dv = V_c W1^T
     GemmProblem g;
     g.M = (int)Lc; g.N = d.m; g.K = d.h; g.Z0 = (int)BH; g.Z1 = 1;
     g.A = {static_cast<const char*>(v) + t0 * h * es, ot, false, h, N * h, 0};
     g.B = {b.W1o, ot, false, h, m * h, 0};
-    g.C = {b.Dv, DT_F32, m, Lc * m, 0};
+    g.C = {b.Dv, ot, m, L * m, 0};
     TTT_TRY(run_gemm("gemm_v_w1t", g, s));
   }
-  EtaMap em{eta, Lc, N, t0};
-  TTT_OP("grad_prep", grad_prep(ot, b.AB, b.Dv, BH * Lc, d.m, em, b.P,
-                                 (mask & TTT_UPDATE_W2) ? b.E2 : nullptr,
-                                 (mask & TTT_UPDATE_W0) ? b.E0 : nullptr, s));
+  // [A | B] = K_c [W0 | W2] -> P = phi eta (and E2, E0 for the input-side matrices)
+  SwigluGemm f = rec_features(d, k, b, t0, Lc, b.P);
+  f.rowscale = eta + t0;
+  f.rs0 = N;
+  f.rs1 = 0;
+  if (need_in) {
+    f.grad = 1;
+    f.out2 = (mask & TTT_UPDATE_W2) ? b.E2 : nullptr;
+    f.ld2 = m; f.s20 = L * m; f.s21 = 0;
+    f.out3 = (mask & TTT_UPDATE_W0) ? b.E0 : nullptr;
+    f.ld3 = m; f.s30 = L * m; f.s31 = 0;
+    f.dv = b.Dv;
+    f.ldd = m; f.ds0 = L * m; f.ds1 = 0;
+  }
+  TTT_TRY(run_swiglu("gemm_features_k", f, s));
   // Split-K gradient reductions over the chunk's tokens.
   const int sp = (Lc == d.chunk) ? b.splits : 1;
   const long long Ks = Lc / sp;
@@ -428,7 +444,7 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
   if (mask & TTT_UPDATE_W1) {  // dW1 = -(phi eta)^T V
     GemmProblem g;
     g.M = d.m; g.N = d.h; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
-    g.A = {b.P, ot, true, m, Lc * m, Ks * m};
+    g.A = {b.P, ot, true, m, L * m, Ks * m};
     g.B = {static_cast<const char*>(v) + t0 * h * es, ot, true, h, N * h, Ks * h};
     g.C = {b.partials + hm, DT_F32, h, 3 * hm, tot};
     g.alpha = -1.0f;
@@ -439,7 +455,7 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
     GemmProblem g;
     g.M = d.h; g.N = d.m; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
     g.A = {static_cast<const char*>(k) + t0 * h * es, ot, true, h, N * h, Ks * h};
-    g.B = {pidx == 0 ? b.E0 : b.E2, ot, true, m, Lc * m, Ks * m};
+    g.B = {pidx == 0 ? b.E0 : b.E2, ot, true, m, L * m, Ks * m};
     g.C = {b.partials + pidx * hm, DT_F32, m, 3 * hm, tot};
     TTT_TRY(run_gemm(pidx == 0 ? "gemm_grad_w0" : "gemm_grad_w2", g, s));
   }
@@ -563,7 +579,7 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1o,
                               d.momentum ? M_io : nullptr, b.M_all, d.momentum, s));
-  TTT_OP("prep_weights", prep_wk(ot, W0, W2, b.Wk, (int)BH, d.H, d.h, d.m, 0, s));
+  TTT_OP("prep_weights", prep_wk_blocked(ot, W0, W2, b.Wk, (int)BH, d.H, d.h, d.m, 0, s));
   if (d.renorm) TTT_OP("col_norms", col_norms(W0, W2, W1, d.H, d.h, d.m, b.tnorm, s));
   const long long N = d.N, L = d.chunk;
   int c = 0;
