@@ -73,6 +73,13 @@ def kernel_work(name: str, wl, form: str):
     BH, h, m = wl.B * wl.H, wl.h, wl.m
     T = BH * wl.N
     es = 2 if wl.dtype == "bf16" else 4
+    if form == "lm_target":
+        # Vbar = conv4(X0) W_target: one [N,d]x[d,d] product; the conv reads X0, writes bf16
+        table = {
+            "gemm_lm_target": ("tensor", 2.0 * wl.N * h * h),
+            "conv4_causal": ("hbm", 2.0 * 2 * wl.N * h),
+        }
+        return table.get(base, (None, None))
     if form == "recurrent":
         table = {
             "gemm_features_k": ("tensor", 4.0 * h * m * T),
@@ -222,16 +229,33 @@ def barrier(world):
 
 # ----------------------------------------------------------------------------- GPU arm
 def _gpu_inputs(wl, seed, torch):
-    from ttt_inputs import make_layer_inputs
-    x = make_layer_inputs(wl, seed=seed)
-    td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    """Device inputs of the workload. For the In-Place workload q = k = H (one tensor),
+    v = the LM-aligned target computed on the GPU from X0 (see lm_target), the gate/up
+    projections and W_down in their own layouts."""
+    from ttt_inputs import make_inplace_inputs, make_layer_inputs
 
     def dev(a, dt=torch.float32):
         return torch.from_numpy(a).cuda().to(dt).contiguous()
 
+    if wl.kind == "inplace":
+        x = make_inplace_inputs(wl, seed=seed)
+        bf = torch.bfloat16
+        g = {"X0": dev(x["X0"], bf), "conv_w": dev(x["conv_w"]), "W_target": dev(x["W_target"], bf)}
+        g["q"] = dev(x["Hs"], bf)[None, None].contiguous()
+        g["k"] = g["q"]
+        g["v"] = torch.empty_like(g["q"])
+        g["eta"] = dev(x["eta"])[None, None].contiguous()
+        g["W0"], g["W2"] = dev(x["Wg"])[None].contiguous(), dev(x["Wu"])[None].contiguous()
+        g["W1"] = dev(x["W_down"])[None].contiguous()
+        g["alpha"] = None
+        g["layouts"] = (1, 1)
+        return x, g
+    x = make_layer_inputs(wl, seed=seed)
+    td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     g = {n: dev(x[n], td) for n in ("q", "k", "v")}
     g.update({n: dev(x[n]) for n in ("eta", "W0", "W2", "W1")})
     g["alpha"] = dev(x["alpha"]) if x["alpha"] is not None else None
+    g["layouts"] = (0, 0)
     return x, g
 
 
@@ -314,12 +338,23 @@ def run_gpu(args, rank, local, world):
 
     # ---- parallel form (headline)
     forms = [f for f in ("parallel", "recurrent") if f in wl.paths]
+    lin, l1 = g["layouts"]
+    if wl.kind == "inplace":
+        # the value target is part of the In-Place step; timed on its own below
+        layer.lm_target(g["X0"], g["conv_w"], g["W_target"], out=g["v"][0, 0])
+        forms = ["lm_target"] + forms
     for form in forms:
-        if form == "parallel":
-            desc = layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order)
+        if form == "lm_target":
+            tws = layer.workspace(abi.ttt_lm_target_workspace_bytes(wl.N, wl.h), "cuda")
+
+            def step():
+                abi.ttt_lm_target(wl.N, wl.h, g["X0"], g["conv_w"], g["W_target"], g["v"], tws)
+        elif form == "parallel":
+            desc = layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order, 1, lin, l1)
             ws = layer.workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_PARALLEL), "cuda")
             out = torch.empty_like(g["q"])
-            S = torch.empty((wl.B, wl.H, wl.m, wl.h), dtype=torch.float32, device="cuda")
+            S = torch.empty((wl.B, wl.H, wl.m, wl.h) if l1 == 0 else (wl.B, wl.H, wl.h, wl.m),
+                            dtype=torch.float32, device="cuda")
 
             def step():
                 abi.ttt_la_parallel_fwd(desc, g["q"], g["k"], g["v"], g["eta"], g["W0"],
@@ -341,7 +376,11 @@ def run_gpu(args, rank, local, world):
         ms_max = max_over_ranks(ms, world, "cuda")
         per_step = ms_max / steps
         table = _kernel_table(trace, steps)
-        flops, nbytes = layer_flops(wl, form), layer_bytes(wl, form)
+        if form == "lm_target":
+            flops = 2.0 * wl.N * wl.h * wl.h
+            nbytes = 2.0 * (2 * wl.N * wl.h + wl.h * wl.h) + 16.0 * wl.h
+        else:
+            flops, nbytes = layer_flops(wl, form), layer_bytes(wl, form)
         t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
         result["forms"][form] = {
             "tokens_per_s": job_throughput(tokens, world, per_step / 1e3),
@@ -360,7 +399,33 @@ def run_gpu(args, rank, local, world):
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     e2e = None
-    if "parallel" in forms:
+    if "parallel" in forms and wl.kind == "inplace":
+        hq = {n: g[n].cpu().pin_memory() for n in ("q", "X0")}
+        dq = {n: torch.empty_like(g[n]) for n in hq}
+        hout = torch.empty(g["q"].shape, dtype=g["q"].dtype).pin_memory()
+        dout = torch.empty_like(g["q"])
+        dv = torch.empty_like(g["v"])
+        ws = layer.workspace(abi.ttt_workspace_bytes(
+            layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order, 1, lin, l1), 0), "cuda")
+        tws = layer.workspace(abi.ttt_lm_target_workspace_bytes(wl.N, wl.h), "cuda")
+
+        def e2e_step():
+            for n in dq:
+                dq[n].copy_(hq[n], non_blocking=True)
+            layer.lm_target(dq["X0"], g["conv_w"], g["W_target"], out=dv[0, 0], ws=tws)
+            layer.la_parallel_fwd(dq["q"], dq["q"], dv, g["eta"], g["W0"], g["W2"], g["W1"],
+                                  wl.chunk, order=wl.order, w_in_layout=lin, w1_layout=l1,
+                                  return_state=False, out=dout, ws=ws)
+            hout.copy_(dout, non_blocking=True)
+
+        steps = max(3, args.steps // 2)
+        ms, _ = _timed(e2e_step, steps, args.warmup, world, torch)
+        ms = max_over_ranks(ms, world, "cuda")
+        e2e = {"value": job_throughput(tokens, world, ms / steps / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hq.values()),
+               "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+               "ms_per_step": ms / steps}
+    elif "parallel" in forms:
         hq = {n: g[n].cpu().pin_memory() for n in ("q", "k", "v", "eta")}
         dq = {n: torch.empty_like(g[n]) for n in ("q", "k", "v", "eta")}
         hout = torch.empty(g["q"].shape, dtype=g["q"].dtype).pin_memory()
@@ -390,8 +455,15 @@ def run_gpu(args, rank, local, world):
 
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_time(wl, x, n: int, form: str = "parallel") -> float:
-    """Seconds the fp64 oracle takes for the first ``n`` tokens of (b=0, head=0)."""
+    """Seconds the fp64 oracle takes for the first ``n`` tokens of (b=0, head=0) (for the
+    In-Place workload: the target prologue and the sequential update on n tokens)."""
     from oracle import ttt_oracle as O
+    if wl.kind == "inplace":
+        t0 = time.perf_counter()
+        vbar = O.lm_target(x["X0"][:n], x["conv_w"], x["W_target"])
+        O.inplace_sequential(x["Hs"][:n], x["Wg"], x["Wu"], x["W_down"], vbar, wl.chunk,
+                             float(x["eta"][0]))
+        return time.perf_counter() - t0
     q, k, v, eta = (x[name][0, 0, :n].astype("float64") for name in ("q", "k", "v", "eta"))
     W0, W2, W1 = x["W0"][0], x["W2"][0], x["W1"][0]
     t0 = time.perf_counter()
@@ -432,9 +504,12 @@ def workload_from_args(args):
 
 def run_reference(args):
     """Reference arm: the fp64 CPU oracle as it stands, on bounded samples."""
-    from ttt_inputs import make_layer_inputs
+    from ttt_inputs import make_inplace_inputs, make_layer_inputs
     wl = workload_from_args(args)
-    x = make_layer_inputs(wl.scaled(B=1, H=1), seed=wl.seed)
+    if wl.kind == "inplace":
+        x = make_inplace_inputs(wl, seed=wl.seed)
+    else:
+        x = make_layer_inputs(wl.scaled(B=1, H=1), seed=wl.seed)
     form = "parallel" if "parallel" in wl.paths else "recurrent"
     n, t, desc = oracle_sample(wl, x, 2.0, form)
     times = []
@@ -502,7 +577,16 @@ def main():
     wl, peaks, res, x = run_gpu(args, rank, local, world)
     if rank == 0:
         form = "parallel" if "parallel" in res["forms"] else "recurrent"
-        head = res["forms"][form]
+        head = dict(res["forms"][form])
+        if "lm_target" in res["forms"]:
+            # In-Place step = target prologue + parallel update/apply
+            pro = res["forms"]["lm_target"]
+            ms = head["ms_per_step"] + pro["ms_per_step"]
+            head["tokens_per_s"] = job_throughput(wl.B * wl.N, world, ms / 1e3)
+            head["ms_per_step"] = ms
+            head["roofline_frac"] = (res["forms"][form]["roofline_frac"] *
+                                     res["forms"][form]["ms_per_step"] +
+                                     pro["roofline_frac"] * pro["ms_per_step"]) / ms
         line = {
             "metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s",
             "n_gpus": world, "steps": head["steps"], "warmup": args.warmup,
