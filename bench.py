@@ -299,6 +299,28 @@ def _kernel_table(trace, steps):
     return dict(sorted(table.items(), key=lambda kv: -kv[1]["ms_total"]))
 
 
+def _traffic(workload: str, kernel: str):
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.txt), or None
+    when there is none or the kernel's source changed since the capture."""
+    import hashlib
+    try:
+        lines = open(os.path.join(ROOT, "profiles", "traffic.txt")).read().splitlines()
+    except OSError:
+        return None
+    for ln in lines:
+        f = ln.split()
+        if len(f) < 4 or ln.startswith("#") or f[0] != workload or f[1] != kernel:
+            continue
+        src, want = f[3].split(":")
+        path = os.path.join(ROOT, "test_weight_layers_ttt_b200", "csrc", src)
+        try:
+            have = hashlib.sha256(open(path, "rb").read()).hexdigest()[:len(want)]
+        except OSError:
+            return None
+        return float(f[2]) if have == want else None
+    return None
+
+
 def _roofline(table, wl, peaks, form, steps):
     """Roofline of the dominant kernel (largest share) with a known algorithmic work."""
     for name, e in table.items():
@@ -317,7 +339,9 @@ def _roofline(table, wl, peaks, form, steps):
             unit = "GB/s"
         return {"kernel": name, "bound": "tensor" if bound == "tensor" else "hbm",
                 "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4),
+                "traffic": (_traffic(wl.name, name)
+                            if form == "parallel" and wl == WORKLOADS_REF().get(wl.name) else None),
                 "work_per_launch": work, "share": round(e["share"], 4),
                 "peak_source": peaks["source"] + " (burst)"}
     return None
