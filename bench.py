@@ -81,7 +81,10 @@ def kernel_work(name: str, wl, form: str):
         }
         return table.get(base, (None, None))
     if form == "recurrent":
+        r, c = min(h, m), max(h, m)
+        ns = wl.ns_steps * (4.0 * r * r * c + 2.0 * r ** 3) * 3 * BH * wl.C
         table = {
+            "ns_mma": ("tensor", 3.0 * ns),   # three bf16 hi/lo terms per product
             "gemm_features_k": ("tensor", 4.0 * h * m * T),
             "gemm_features_q": ("tensor", 4.0 * h * m * T),
             "gemm_v_w1t": ("tensor", 2.0 * h * m * T),
@@ -337,7 +340,7 @@ def _roofline(table, wl, peaks, form, steps):
             achieved = work / secs / 1e9
             peak = peaks["hbm_gbs"]
             unit = "GB/s"
-        return {"kernel": name, "bound": "tensor" if bound == "tensor" else "hbm",
+        return {"kernel": name, "bound": "hbm" if bound == "hbm" else "tensor",
                 "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                 "frac": round(achieved / peak, 4),
                 "traffic": (_traffic(wl.name, name)

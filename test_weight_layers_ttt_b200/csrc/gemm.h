@@ -52,9 +52,10 @@ ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_er
                      unsigned long long wait_ns);
 
 // Feature GEMM with the SwiGLU applied in the epilogue. gemm.B holds the input-side
-// weights as 128-row blocks [W0^T rows j..j+127 ; W2^T rows j..j+127] (256 rows per block,
-// zero rows past m), so gemm.N = 2 * ceil(m / 128) * 128 and every 256-wide output tile
-// carries matching A and B columns. The epilogue writes phi = silu(A) * B times
+// weights as 128-row blocks [W0^T rows j..j+127 / 2 ; W2^T rows j..j+127] (256 rows per
+// block, zero rows past m; see prep_wk_blocked), so gemm.N = 2 * ceil(m / 128) * 128 and
+// every 256-wide output tile carries matching A/2 and B columns. With A = X W0 and
+// B = X W2, the epilogue writes phi = silu(A) * B = (A/2) (1 + tanh(A/2)) B times
 // rowscale[z0*rs0 + z1*rs1 + row] (or 1 when rowscale is null) to gemm.C (bf16, row stride
 // gemm.C.ld, phi columns < n_valid) and, when out2 is set, the unscaled phi to out2.
 //

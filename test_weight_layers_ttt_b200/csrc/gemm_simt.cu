@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(THREADS) simt_swiglu_kernel(const SimtSwiglu s
     for (int c = 0; c < 4; ++c) {
       const int gj = j0 + tx + 16 * c;
       if (gj >= a.N) continue;
-      const float av = acc_a[r][c], bv = acc_b[r][c];
+      const float av = 2.0f * acc_a[r][c], bv = acc_b[r][c];   // the operand holds W0 / 2
       const float sa = siluf_(av);
       const float p = sa * bv;
       C[(long long)gi * a.ldc + gj] = from_f32<TC>(p * rsv);

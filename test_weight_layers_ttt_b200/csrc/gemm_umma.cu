@@ -87,18 +87,53 @@ __device__ __forceinline__ void store_vals(float* dst, const float* v, int n, bo
   }
 }
 
-// silu(a) = a * sigmoid(a) with sigmoid(a) = (1 + tanh(a / 2)) / 2: one MUFU tanh.approx
-// (relative error about 2^-11, below the bf16 rounding of the result).
-__device__ __forceinline__ float silu_fast(float a) {
-  const float h = 0.5f * a;
+__device__ __forceinline__ float tanh_fast(float x) {
   float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
-  return fmaf(h, t, h);
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
+  return t;
+}
+
+// Two SwiGLU outputs from the half pre-activations h = A/2 (the operand holds W0 / 2) and
+// B: silu(A) B = A sigmoid(A) B = h (1 + tanh(h)) B, so with p = h B the result is
+// p + p tanh(h); `s` scales it (the row's eta, or 1). One MUFU tanh.approx per element
+// (relative error about 2^-11, below the bf16 rounding of the result) and the rest as
+// packed fp32x2 multiplies / fma.
+__device__ __forceinline__ void swiglu2(uint32_t h0, uint32_t h1, uint32_t b0, uint32_t b1,
+                                        float s, float& o0, float& o1) {
+  const float t0 = tanh_fast(__uint_as_float(h0)), t1 = tanh_fast(__uint_as_float(h1));
+  asm("{\n\t.reg .b64 H, B, P, T, S;\n\t"
+      "mov.b64 H, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mov.b64 T, {%6, %7};\n\tmov.b64 S, {%8, %9};\n\t"
+      "mul.rn.f32x2 P, H, B;\n\tmul.rn.f32x2 P, P, S;\n\t"
+      "fma.rn.f32x2 P, P, T, P;\n\tmov.b64 {%0, %1}, P;\n\t}"
+      : "=f"(o0), "=f"(o1)
+      : "r"(h0), "r"(h1), "r"(b0), "r"(b1), "f"(t0), "f"(t1), "f"(s), "f"(s));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
+}
+
+// 32 SwiGLU outputs of one TMEM row slice (h = A/2 and B, 32 columns each), scaled by `sc`,
+// packed to bf16 and written as 16-byte chunks c0 .. c0 + 3 of this lane's 128-byte row of
+// a 128-byte-swizzled staging box.
+__device__ __forceinline__ void swiglu_piece(const uint32_t (&ra)[32], const uint32_t (&rb)[32],
+                                             float sc, uint32_t box, int lane, int c0) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    float f0, f1;
+    swiglu2(ra[j], ra[j + 1], rb[j], rb[j + 1], sc, f0, f1);
+    pk[j / 2] = pack_bf16x2(f0, f1);
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const uint32_t addr = box + lane * 128 + (((c0 + cc) ^ (lane & 7)) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * cc]),
+                 "r"(pk[4 * cc + 1]), "r"(pk[4 * cc + 2]), "r"(pk[4 * cc + 3])
+                 : "memory");
+  }
 }
 
 __device__ __forceinline__ void store_vals(__nv_bfloat16* dst, const float* v, int n, bool vec) {
@@ -356,14 +391,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int part = ew >> 2;  // 0: first half of the tile's columns, 1: second half
     for (int lt = 0; lt < walk.count; ++lt) {
       const int buf = lt & 1;
+      const TileCoord tc = walk.at(lt);
+      const int row = tc.tm * BM + quarter * 32 + lane;
+      // the SwiGLU row scale is fetched before the wait, so its latency hides behind it
+      const float rsv = (MODE == EPI_SWIGLU && !args.grad && args.rs && row < args.M)
+                            ? args.rs[tc.z0 * args.rs0 + tc.z1 * args.rs1 + row]
+                            : 1.0f;
       bool ok = mbar_wait(smem_u32(&acc_full[buf]), (lt >> 1) & 1, abort_flag, args.err,
                           args.wait_ns);
       if (!ok) break;
       tc_fence_after();
-      const TileCoord tc = walk.at(lt);
-      const int row = tc.tm * BM + quarter * 32 + lane;
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      if (MODE == EPI_STORE) {
+      if constexpr (MODE == EPI_STORE) {
         constexpr int HALF = BN / 2;
         uint32_t r[HALF];
 #pragma unroll
@@ -449,16 +488,15 @@ __global__ void __launch_bounds__(THREADS, 1)
               float v[2];
 #pragma unroll
               for (int u = 0; u < 2; ++u) {
-                const float a = __uint_as_float(ra[j + u]), bb = __uint_as_float(rb[j + u]);
-                const float hlf = 0.5f * a;
-                float t;
-                asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hlf));
+                // accumulator half A holds a/2 (the operand carries W0 / 2)
+                const float hlf = __uint_as_float(ra[j + u]), bb = __uint_as_float(rb[j + u]);
+                const float t = tanh_fast(hlf);
                 const float sg = fmaf(0.5f, t, 0.5f);   // sigmoid(a)
-                const float sa = a * sg;                // silu(a)
+                const float sa = fmaf(hlf, t, hlf);     // silu(a) = (a/2)(1 + tanh(a/2))
                 const float d = -eta * dvv[j + u];
                 if (o == 0) v[u] = sa * bb * eta;
                 else if (o == 1) v[u] = d * sa;
-                else v[u] = d * bb * sg * fmaf(a, 1.0f - sg, 1.0f);
+                else v[u] = d * bb * sg * fmaf(2.0f * hlf, 1.0f - sg, 1.0f);   // silu'(a)
               }
               pk[j / 2] = pack_bf16x2(v[0], v[1]);
             }
@@ -482,62 +520,39 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_before();
         mbar_arrive(smem_u32(&acc_empty[buf]));
       } else {
-        // SWIGLU: phi column p of this tile uses accumulator columns p (A) and BN/2 + p (B).
+        // SWIGLU: phi column p of this tile uses accumulator columns p (A/2) and BN/2 + p (B).
+        // Each epilogue warp owns 32 rows x 64 phi columns: two 32-column pieces, the
+        // second piece's TMEM loads in flight while the first is computed. It stages them
+        // in its own 4 KB box (128-byte swizzle) and its lane 0 stores the box with TMA,
+        // so the warps never wait on each other; a warp reuses its box once its previous
+        // store has read it. With a second output (the unscaled phi) the accumulator is
+        // read twice and released after the second read.
+        static_assert(BN == 256, "the SwiGLU epilogue works on 256-column tiles");
         constexpr int PH = BN / 2;       // phi columns per tile
-        constexpr int QW = PH / 2;       // phi columns per epilogue half
-        uint32_t ra[QW], rb[QW];
-#pragma unroll
-        for (int c0 = 0; c0 < QW; c0 += 32) {
-          tmem_ld32(lane_addr + (uint32_t)(part * QW + c0),
-                    *reinterpret_cast<uint32_t(*)[32]>(&ra[c0]));
-          tmem_ld32(lane_addr + (uint32_t)(PH + part * QW + c0),
-                    *reinterpret_cast<uint32_t(*)[32]>(&rb[c0]));
-        }
-        tmem_ld_wait();
-        float a[QW], b[QW];
-#pragma unroll
-        for (int j = 0; j < QW; ++j) {
-          a[j] = __uint_as_float(ra[j]);
-          b[j] = __uint_as_float(rb[j]);
-        }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&acc_empty[buf]));
-        const int rin = quarter * 32 + lane;  // row within the tile
-        const float rsv =
-            (args.rs && row < args.M) ? args.rs[tc.z0 * args.rs0 + tc.z1 * args.rs1 + row] : 1.0f;
-        // phi in place of b; packed outputs only where they are stored.
-#pragma unroll
-        for (int j = 0; j < QW; ++j) b[j] = silu_fast(a[j]) * b[j];
-        uint32_t pk[QW / 2], pk2[QW / 2];
-        if (args.rs) {
-#pragma unroll
-          for (int j = 0; j < QW; j += 2) pk[j / 2] = pack_bf16x2(b[j] * rsv, b[j + 1] * rsv);
-        } else {
-#pragma unroll
-          for (int j = 0; j < QW; j += 2) pk[j / 2] = pack_bf16x2(b[j], b[j + 1]);
-        }
-        if (args.C2) {
-#pragma unroll
-          for (int j = 0; j < QW; j += 2) pk2[j / 2] = pack_bf16x2(b[j], b[j + 1]);
-        }
-        // Each epilogue warp stages its own 32 rows x 64 phi columns (4 KB, 128-byte
-        // swizzle) and its lane 0 stores them with TMA, so the warps never wait on each
-        // other; a warp reuses its box once its previous store has read it.
+        constexpr int QW = PH / 2;       // phi columns per epilogue warp
         const int ox = tc.tn * PH + part * QW;   // first phi column of this warp's box
         const int oy = tc.tm * BM + quarter * 32;
         const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
         const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
-        for (int o = 0; o < (args.C2 ? 2 : 1); ++o) {
+        const uint32_t ta = lane_addr + (uint32_t)(part * QW), tb = ta + (uint32_t)PH;
+        const int nout = args.C2 ? 2 : 1;
+        for (int o = 0; o < nout; ++o) {
+          const float sc = o == 0 ? rsv : 1.0f;
           if (lane == 0) tma_store_wait_read();
           __syncwarp();
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t* src = o == 0 ? &pk[4 * c] : &pk2[4 * c];
-            const uint32_t addr = box + lane * 128 + ((c ^ (lane & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(src[0]),
-                         "r"(src[1]), "r"(src[2]), "r"(src[3])
-                         : "memory");
+          uint32_t ra0[32], rb0[32], ra1[32], rb1[32];
+          tmem_ld32(ta, ra0);
+          tmem_ld32(tb, rb0);
+          tmem_ld_wait_regs(ra0, rb0);
+          tmem_ld32(ta + 32, ra1);
+          tmem_ld32(tb + 32, rb1);
+          swiglu_piece(ra0, rb0, sc, box, lane, 0);
+          tmem_ld_wait_regs(ra1, rb1);
+          if (o == nout - 1) {
+            tc_fence_before();
+            mbar_arrive(smem_u32(&acc_empty[buf]));
           }
+          swiglu_piece(ra1, rb1, sc, box, lane, 4);
           fence_async_smem();
           __syncwarp();
           if (lane == 0 && ox < args.n_valid) {

@@ -1,5 +1,5 @@
-// Non-GEMM kernels of the TTT layer: weight preparation, the SwiGLU feature map and its
-// gradient pieces, the chunk prefix scan over fp32 states, the recurrent update operators
+// Non-GEMM kernels of the TTT layer: weight preparation (the blocked input-side operand),
+// the chunk prefix scan over fp32 states, the recurrent update operators
 // (momentum, Newton-Schulz set-up, step, per-column renormalisation), the causal Conv1D of
 // the In-Place target, and the bounded-wait diagnostic.
 #include "ops.h"
@@ -10,31 +10,7 @@ namespace {
 
 using bf16 = __nv_bfloat16;
 
-template <typename OT>
-__device__ __forceinline__ void st(void* base, long long i, float v) {
-  static_cast<OT*>(base)[i] = from_f32<OT>(v);
-}
-
-__device__ __forceinline__ float eta_of(const EtaMap& em, long long r) {
-  const long long z = r / em.T, t = r - z * em.T;
-  return em.eta[z * em.eta_ld + em.eta_off + t];
-}
-
 // ------------------------------------------------------------------ weight preparation
-template <typename OT>
-__global__ void prep_wk_kernel(const float* W0, const float* W2, OT* Wk, int n_entries,
-                               int src_heads, int h, int m, int layout) {
-  const long long per = 2LL * m * h;
-  TTT_GRID_LOOP(idx, per * n_entries) {
-    const long long e = idx / per, rem = idx - e * per;
-    const int j = (int)(rem / h), i = (int)(rem - (long long)j * h);
-    const float* src = (j < m ? W0 : W2) + (e % src_heads) * (long long)h * m;
-    const int jj = j < m ? j : j - m;
-    const float v = layout == 0 ? src[(long long)i * m + jj] : src[(long long)jj * h + i];
-    Wk[idx] = from_f32<OT>(v);
-  }
-}
-
 // Tiled through shared memory so both the reads of W0/W2 (either layout) and the writes
 // of the blocked operand are coalesced. grid (mpad/32, ceil(h/32), 2 * n_entries),
 // block (32, 8); blockIdx.z = 2 * entry + which (0: W0, 1: W2).
@@ -66,39 +42,7 @@ __global__ void prep_wk_blocked_kernel(const float* W0, const float* W2, OT* Wk,
     const int jj = ty + 8 * k, j = j0 + jj, i = i0 + tx;
     if (j >= mpad || i >= h) continue;
     const long long row = (long long)(j >> 7) * 256 + (which ? 128 : 0) + (j & 127);
-    dst[row * h + i] = from_f32<OT>(tile[jj][tx]);
-  }
-}
-
-// ------------------------------------------------------------------ features
-template <typename OT>
-__global__ void swiglu_kernel(const float* AB, long long rows, int m, EtaMap em, OT* phi_eta,
-                              OT* phi_plain) {
-  TTT_GRID_LOOP(idx, rows * m) {
-    const long long r = idx / m;
-    const int j = (int)(idx - r * m);
-    const float a = AB[r * 2 * m + j], b = AB[r * 2 * m + m + j];
-    const float p = siluf_(a) * b;
-    if (phi_plain) phi_plain[idx] = from_f32<OT>(p);
-    if (phi_eta) phi_eta[idx] = from_f32<OT>(p * eta_of(em, r));
-  }
-}
-
-template <typename OT>
-__global__ void grad_prep_kernel(const float* AB, const float* Dv, long long rows, int m,
-                                 EtaMap em, OT* P, OT* E2, OT* E0) {
-  TTT_GRID_LOOP(idx, rows * m) {
-    const long long r = idx / m;
-    const int j = (int)(idx - r * m);
-    const float a = AB[r * 2 * m + j], b = AB[r * 2 * m + m + j];
-    const float eta = eta_of(em, r);
-    const float sa = siluf_(a);
-    P[idx] = from_f32<OT>(sa * b * eta);
-    if (E2 || E0) {
-      const float d = -eta * Dv[idx];
-      if (E2) E2[idx] = from_f32<OT>(d * sa);
-      if (E0) E0[idx] = from_f32<OT>(d * b * silu_primef_(a));
-    }
+    dst[row * h + i] = from_f32<OT>(which ? tile[jj][tx] : 0.5f * tile[jj][tx]);
   }
 }
 
@@ -394,7 +338,8 @@ __global__ void __launch_bounds__(1024) rec_step_kernel(float* W_all, const floa
     const int col = c0 + cc;
     const long long row = (long long)(col >> 7) * 256 + (p == 2 ? 128 : 0) + (col & 127);
     const float* src = colbuf + (long long)cc * (R + 1);
-    for (int r = tx; r < R; r += 32) wk[row * h + r] = from_f32<OT>(src[r]);
+    const float f = p == 0 ? 0.5f : 1.0f;   // the blocked operand holds W0 / 2
+    for (int r = tx; r < R; r += 32) wk[row * h + r] = from_f32<OT>(f * src[r]);
   }
 }
 
@@ -427,6 +372,75 @@ __global__ void conv4_kernel(const bf16* X0, const float* w, bf16* Xc, int N, in
   }
 }
 
+// 16-byte version: a thread owns 8 channels over a run of CONV_RUN tokens and slides a
+// window of the last three input rows through registers, so every input row is read once
+// per run (plus a three-row halo) and every load and store is a coalesced 16-byte access.
+// grid (ceil(d / 8 / 128), ceil(N / CONV_RUN)), block 128. Needs d % 8 == 0 and 16-byte
+// aligned X0 / Xc.
+constexpr int CONV_RUN = 32;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 v = __bfloat1622float2(h[q]);
+    f[2 * q] = v.x;
+    f[2 * q + 1] = v.y;
+  }
+}
+
+__global__ void __launch_bounds__(128) conv4_vec_kernel(const bf16* X0, const float* w, bf16* Xc,
+                                                        int N, int d) {
+  const int g = blockIdx.x * 128 + threadIdx.x;   // channel group
+  if (g * 8 >= d) return;
+  const int c = g * 8;
+  const long long t0 = (long long)blockIdx.y * CONV_RUN;
+  float wt[4][8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float4 a = *reinterpret_cast<const float4*>(w + (long long)j * d + c);
+    const float4 b = *reinterpret_cast<const float4*>(w + (long long)j * d + c + 4);
+    wt[j][0] = a.x; wt[j][1] = a.y; wt[j][2] = a.z; wt[j][3] = a.w;
+    wt[j][4] = b.x; wt[j][5] = b.y; wt[j][6] = b.z; wt[j][7] = b.w;
+  }
+  float win[3][8];   // win[j - 1] = X0[t - j]
+#pragma unroll
+  for (int j = 1; j <= 3; ++j) {
+    const long long t = t0 - j;
+    if (t >= 0) {
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(X0 + t * d + c), win[j - 1]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) win[j - 1][q] = 0.0f;
+    }
+  }
+  const long long t_end = min((long long)N, t0 + CONV_RUN);
+  for (long long t = t0; t < t_end; ++t) {
+    float x[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(X0 + t * d + c), x);
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 8; q += 2) {
+      float r[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int k = q + u;
+        r[u] = wt[0][k] * x[k] + wt[1][k] * win[0][k] + wt[2][k] * win[1][k] +
+               wt[3][k] * win[2][k];
+      }
+      const __nv_bfloat162 pk = __floats2bfloat162_rn(r[0], r[1]);
+      o[q / 2] = *reinterpret_cast<const uint32_t*>(&pk);
+    }
+    *reinterpret_cast<uint4*>(Xc + t * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      win[2][q] = win[1][q];
+      win[1][q] = win[0][q];
+      win[0][q] = x[q];
+    }
+  }
+}
+
 // ------------------------------------------------------------------ diagnostics
 __global__ void wait_timeout_kernel(unsigned* err, unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar;
@@ -456,17 +470,6 @@ cudaError_t by_ot(int ot, F&& f) {
 
 }  // namespace
 
-cudaError_t prep_wk(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
-                    int src_heads, int h, int m, int src_layout, cudaStream_t s) {
-  return by_ot(ot, [&](auto tag) {
-    using OT = decltype(tag);
-    const long long n = 2LL * m * h * n_entries;
-    prep_wk_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(W0, W2, static_cast<OT*>(Wk), n_entries,
-                                                        src_heads, h, m, src_layout);
-    return cudaGetLastError();
-  });
-}
-
 cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
                             int src_heads, int h, int m, int src_layout, cudaStream_t s) {
   return by_ot(ot, [&](auto tag) {
@@ -475,26 +478,6 @@ cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, 
     dim3 grid(mpad / 32, (h + 31) / 32, 2 * n_entries);
     prep_wk_blocked_kernel<OT><<<grid, dim3(32, 8), 0, s>>>(
         W0, W2, static_cast<OT*>(Wk), src_heads, h, m, src_layout);
-    return cudaGetLastError();
-  });
-}
-
-cudaError_t swiglu(int ot, const float* AB, long long rows, int m, EtaMap em, void* phi_eta,
-                   void* phi_plain, cudaStream_t s) {
-  return by_ot(ot, [&](auto tag) {
-    using OT = decltype(tag);
-    swiglu_kernel<OT><<<grid_for(rows * m, 256), 256, 0, s>>>(
-        AB, rows, m, em, static_cast<OT*>(phi_eta), static_cast<OT*>(phi_plain));
-    return cudaGetLastError();
-  });
-}
-
-cudaError_t grad_prep(int ot, const float* AB, const float* Dv, long long rows, int m,
-                      EtaMap em, void* P, void* E2, void* E0, cudaStream_t s) {
-  return by_ot(ot, [&](auto tag) {
-    using OT = decltype(tag);
-    grad_prep_kernel<OT><<<grid_for(rows * m, 256), 256, 0, s>>>(
-        AB, Dv, rows, m, em, static_cast<OT*>(P), static_cast<OT*>(E2), static_cast<OT*>(E0));
     return cudaGetLastError();
   });
 }
@@ -600,8 +583,17 @@ cudaError_t rec_finish(const float* W_all, int BH, int h, int m, float* W0_out, 
 
 cudaError_t conv4_causal(const void* X0, const float* conv_w, void* Xc, int N, int d,
                          cudaStream_t s) {
-  conv4_kernel<<<grid_for((long long)N * d, 256), 256, 0, s>>>(
-      static_cast<const bf16*>(X0), conv_w, static_cast<bf16*>(Xc), N, d);
+  const bool vec = d % 8 == 0 && ((reinterpret_cast<uintptr_t>(X0) | reinterpret_cast<uintptr_t>(Xc) |
+                                    reinterpret_cast<uintptr_t>(conv_w)) & 15) == 0 &&
+                   (N + CONV_RUN - 1) / CONV_RUN <= 65535;
+  if (vec) {
+    const dim3 grid((unsigned)((d / 8 + 127) / 128), (unsigned)((N + CONV_RUN - 1) / CONV_RUN));
+    conv4_vec_kernel<<<grid, 128, 0, s>>>(static_cast<const bf16*>(X0), conv_w,
+                                          static_cast<bf16*>(Xc), N, d);
+  } else {
+    conv4_kernel<<<grid_for((long long)N * d, 256), 256, 0, s>>>(
+        static_cast<const bf16*>(X0), conv_w, static_cast<bf16*>(Xc), N, d);
+  }
   return cudaGetLastError();
 }
 

@@ -9,31 +9,14 @@
 
 namespace ttt {
 
-// Row index r of a [Z * T, width] activation maps to eta[(r / T) * eta_ld + eta_off + r % T].
-struct EtaMap {
-  const float* eta;
-  long long T, eta_ld, eta_off;
-};
-
-// Fast-weight input-side operand Wk[e] = [W0^T ; W2^T] ([2m, h], K-major) for n_entries
-// entries; entry e reads source head e % src_heads. Source layout 0: [h, m]; 1: [m, h].
-cudaError_t prep_wk(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
-                    int src_heads, int h, int m, int src_layout, cudaStream_t s);
-// Same weights as 128-row blocks [W0^T rows j..j+127 ; W2^T rows j..j+127] per entry
-// ([2 * ceil(m/128) * 128, h], zero rows past m): the B operand of the SwiGLU-epilogue GEMM.
+// Fast-weight input-side operand of the SwiGLU-epilogue GEMM, per entry e (source head
+// e % src_heads; source layout 0: [h, m], 1: [m, h]): 128-row blocks
+// [W0^T rows j..j+127 / 2 ; W2^T rows j..j+127] ([2 * ceil(m/128) * 128, h], K-major, zero
+// rows past m). W0 enters halved (exact in binary floating point), so the GEMM's first
+// half yields a/2 = (x W0)/2, the argument silu takes through tanh:
+// silu(a) = (a/2) (1 + tanh(a/2)).
 cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
                             int src_heads, int h, int m, int src_layout, cudaStream_t s);
-
-// phi = silu(A) * B from AB rows [A | B] (fp32, width 2m); writes phi * eta to phi_eta and,
-// when non-null, the unscaled phi to phi_plain (both OT, width m).
-cudaError_t swiglu(int ot, const float* AB, long long rows, int m, EtaMap em, void* phi_eta,
-                   void* phi_plain, cudaStream_t s);
-
-// Per-token pieces of the recurrent gradients from AB = [K W0 | K W2] and Dv = V W1^T:
-//   d = -eta * Dv, P = silu(A) * B * eta, E2 = d * silu(A), E0 = d * B * silu'(A).
-// E2/E0 are skipped when null.
-cudaError_t grad_prep(int ot, const float* AB, const float* Dv, long long rows, int m,
-                      EtaMap em, void* P, void* E2, void* E0, cudaStream_t s);
 
 // Chunk prefix sums: S starts at W1[bh % H] (layout 0 [m,h] / 1 [h,m]); for each chunk c
 // the state read by chunk c is written to Sc[bh, c] (OT, [m,h]): inclusive of dS[bh, c]
@@ -62,6 +45,14 @@ cudaError_t ns_normalize(const float* U, float* X, int BH, int h, int m, int mas
                          cudaStream_t s);
 cudaError_t ns_writeback(const float* X, float* U, int BH, int h, int m, int mask,
                          cudaStream_t s);
+// The whole Newton-Schulz orthogonalisation of U's parts in `mask` on the tensor cores
+// (ns_mma.cu; operands split into bf16 hi + lo pairs, fp32 accumulation): normalise,
+// `steps` iterations X <- a X + (b A + c A A) X with A = X X^T on the rows <= cols
+// orientation, write back. Only for min(h, m) <= 128 and max(h, m) <= 256
+// (ns_mma_supported). Bounded waits report through `err`.
+bool ns_mma_supported(int h, int m);
+cudaError_t ns_mma(float* U, int BH, int h, int m, int mask, int steps, float eps, float a,
+                   float b, float c, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
 // W <- W - sign * U, optional per-column renormalisation to tnorm, refresh the OT copies:
 // W1o [BH, m, h] and the blocked input-side operand Wk [BH, 2 * mpad, h] (see
 // prep_wk_blocked).

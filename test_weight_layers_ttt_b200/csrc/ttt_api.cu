@@ -308,6 +308,12 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
 }
 
 // ------------------------------------------------------------------ recurrent form
+// bf16 mode runs Newton-Schulz on the tensor cores (split bf16 operands, close to fp32)
+// when the matrices fit one CTA; fp32 mode and larger matrices use fp32 CUDA-core products.
+bool ns_on_tensor_cores(const ttt_desc& d) {
+  return d.dtype == TTT_DTYPE_BF16 && ns_mma_supported(d.h, d.m);
+}
+
 struct RecBufs {
   float* W_all;   // fp32 masters [BH][W0 | W1 | W2]
   float* M_all;   // momentum, same layout
@@ -361,7 +367,7 @@ size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
   b.E0 = cv.take(os * rows * d.m);
   b.partials = cv.take_n<float>((long long)b.splits * BH * 3 * hm);
   b.phiQ = cv.take(os * rows * d.m);
-  if (d.ns_steps > 0) {
+  if (d.ns_steps > 0 && !ns_on_tensor_cores(d)) {
     const long long r = d.h < d.m ? d.h : d.m;
     b.X = cv.take_n<float>(BH * 3 * hm);
     b.X2 = cv.take_n<float>(BH * 3 * hm);
@@ -461,7 +467,10 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
   }
   TTT_OP("reduce_momentum", rec_reduce(b.partials, sp, b.U, d.momentum ? b.M_all : nullptr,
                                       alpha, (int)C, c, (int)BH, d.h, d.m, mask, s));
-  if (d.ns_steps > 0) {
+  if (d.ns_steps > 0 && ns_on_tensor_cores(d)) {
+    TTT_OP("ns_mma", ns_mma(b.U, (int)BH, d.h, d.m, mask, d.ns_steps, 1e-7f, 3.4445f,
+                            -4.7750f, 2.0315f, device_error_word(), wait_limit_ns(), s));
+  } else if (d.ns_steps > 0) {
     const float a3 = 3.4445f, b3 = -4.7750f, c3 = 2.0315f;
     const long long r = h < m ? h : m, cc = h < m ? m : h;
     TTT_OP("ns_normalize", ns_normalize(b.U, b.X, (int)BH, d.h, d.m, mask, 1e-7f, s));

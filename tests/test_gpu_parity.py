@@ -114,6 +114,10 @@ REC_CASES = [
     ("lm", "bf16", 2, 1, 600, 128, 256, 256, dict(renorm=True, momentum=True, ns_steps=5)),
     ("lm", "bf16", 1, 2, 512, 64, 192, 128, dict(update_mask=abi.TTT_UPDATE_W1)),
     ("lm", "bf16", 1, 1, 512, 128, 64, 256, dict(update_mask=5, ns_steps=5)),
+    # ragged matrices for the tensor-core Newton-Schulz (zero padding inside the CTA)
+    ("lm", "bf16", 1, 2, 320, 40, 200, 96, dict(renorm=True, momentum=True, ns_steps=5)),
+    # min(h, m) > 128: bf16 mode falls back to CUDA-core Newton-Schulz; 3 steps
+    ("lm", "bf16", 1, 1, 256, 256, 136, 128, dict(ns_steps=3)),
 ]
 
 
