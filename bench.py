@@ -46,6 +46,8 @@ def layer_flops(wl, form: str) -> float:
     if form == "parallel":
         feats = 4 * hm * T if wl.kind == "inplace" else 8 * hm * T   # q == k: once
         return float(feats + 2 * hm * T + 2 * hm * T)
+    if form == "linear":   # identity features: state deltas and outputs, [h, h] states
+        return 4.0 * wl.h * wl.h * T
     flops = 18.0 * hm * T   # 9 matmuls: K features (2), D, 3 gradients, Q features (2), out
     if wl.ns_steps:
         r, c = min(wl.h, wl.m), max(wl.h, wl.m)
@@ -61,6 +63,9 @@ def layer_bytes(wl, form: str) -> float:
     hm = wl.h * wl.m
     n_in = 1 if wl.kind == "inplace" else 2          # q and k (aliased for in-place)
     act = (n_in + 1) * T * wl.h * es + T * wl.h * es + T * 4      # q,k,v in, O out, eta
+    if form == "linear":
+        hh = wl.h * wl.h
+        return float(act + hh * 4 * wl.H + hh * 4 * wl.B * wl.H)
     weights = 3 * hm * 4 * wl.H
     state_out = hm * 4 * wl.B * wl.H
     return float(act + weights + state_out)
@@ -73,6 +78,15 @@ def kernel_work(name: str, wl, form: str):
     BH, h, m = wl.B * wl.H, wl.h, wl.m
     T = BH * wl.N
     es = 2 if wl.dtype == "bf16" else 4
+    if form == "linear":
+        hh = h * h
+        table = {
+            "gemm_state_delta": ("tensor", 2.0 * hh * T),
+            "gemm_output": ("tensor", 2.0 * hh * T),
+            "scale_rows": ("hbm", T * h * 2.0 * es + T * 4.0),
+            "chunk_scan": ("hbm", BH * wl.C * hh * (4.0 + es) + 2 * 4.0 * BH * hh),
+        }
+        return table.get(base, (None, None))
     if form == "lm_target":
         # Vbar = conv4(X0) W_target: one [N,d]x[d,d] product; the conv reads X0, writes bf16
         table = {
@@ -365,6 +379,8 @@ def run_gpu(args, rank, local, world):
 
     # ---- parallel form (headline)
     forms = [f for f in ("parallel", "recurrent") if f in wl.paths]
+    if wl.kind == "lm" and "parallel" in forms:
+        forms.insert(1, "linear")   # identity features (plain chunked linear attention)
     lin, l1 = g["layouts"]
     if wl.kind == "inplace":
         # the value target is part of the In-Place step; timed on its own below
@@ -376,6 +392,18 @@ def run_gpu(args, rank, local, world):
 
             def step():
                 abi.ttt_lm_target(wl.N, wl.h, g["X0"], g["conv_w"], g["W_target"], g["v"], tws)
+        elif form == "linear":
+            ldesc = abi.ttt_desc(B=wl.B, H=wl.H, N=wl.N, h=wl.h, m=wl.h, chunk=wl.chunk,
+                                 dtype=abi.TTT_DTYPE_BF16 if wl.dtype == "bf16" else 0,
+                                 order=layer.ORDERS[wl.order], sign=1)
+            lws = layer.workspace(abi.ttt_workspace_bytes(ldesc, abi.TTT_PATH_LINEAR), "cuda")
+            lS0 = torch.zeros((wl.H, wl.h, wl.h), dtype=torch.float32, device="cuda")
+            lS0[:, :, :] = g["W1"][:, :wl.h, :]
+            lout = torch.empty_like(g["q"])
+
+            def step():
+                abi.ttt_linear_attn_fwd(ldesc, g["q"], g["k"], g["v"], g["eta"], lS0, lout,
+                                        None, lws)
         elif form == "parallel":
             desc = layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order, 1, lin, l1)
             ws = layer.workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_PARALLEL), "cuda")
@@ -396,7 +424,7 @@ def run_gpu(args, rank, local, world):
                 abi.ttt_lact_recurrent_fwd(desc, g["q"], g["k"], g["v"], g["eta"], g["alpha"],
                                            g["W0"], g["W2"], g["W1"], out, None, None, None,
                                            None, ws)
-        steps = args.steps if form == "parallel" else max(3, args.steps // 2)
+        steps = args.steps if form in ("parallel", "linear") else max(3, args.steps // 2)
         with ClockSampler(gpu_id(local, torch)) as clk:
             ms, trace = _timed(step, steps, args.warmup, world, torch, trace_capacity=16384)
         abi.ttt_last_device_status()

@@ -69,7 +69,7 @@ typedef enum ttt_status {
 enum { TTT_DTYPE_FP32 = 0, TTT_DTYPE_BF16 = 1 };
 enum { TTT_ORDER_UPDATE_APPLY = 0, TTT_ORDER_APPLY_UPDATE = 1 };
 enum { TTT_UPDATE_W0 = 1, TTT_UPDATE_W1 = 2, TTT_UPDATE_W2 = 4, TTT_UPDATE_ALL = 7 };
-enum { TTT_PATH_PARALLEL = 0, TTT_PATH_RECURRENT = 1 };
+enum { TTT_PATH_PARALLEL = 0, TTT_PATH_RECURRENT = 1, TTT_PATH_LINEAR = 2 };
 
 /* Problem description. All fields are read; unused ones must be 0 unless noted. */
 typedef struct ttt_desc {
@@ -91,8 +91,9 @@ typedef struct ttt_desc {
 } ttt_desc;
 
 /*
- * Workspace size in bytes for `path` (TTT_PATH_PARALLEL or TTT_PATH_RECURRENT), or 0
- * when the description is invalid for that path. Host-only; touches no device.
+ * Workspace size in bytes for `path` (TTT_PATH_PARALLEL, TTT_PATH_RECURRENT or
+ * TTT_PATH_LINEAR), or 0 when the description is invalid for that path. Host-only;
+ * touches no device.
  */
 size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path);
 
@@ -120,6 +121,30 @@ size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path);
 ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* k,
                                const void* v, const float* eta, const float* W0,
                                const float* W2, const float* W1, void* out,
+                               float* S_final, void* workspace, size_t workspace_bytes,
+                               ttt_stream_t stream);
+
+/*
+ * Parallel form with identity features: the end of the simplification ladder ("Test-Time
+ * Training with KV Binding Is Secretly Linear Attention", section 方法步骤详情,
+ * variants 3-6: the inner MLP reduced to one linear map, phi(x) = x), i.e. chunked linear
+ * attention with a per-token step size:
+ *     Delta S_c = sign * K_c^T diag(eta_c) V_c,
+ *     S_c = S0 + sum_{c' <= c} Delta S_c'   (update_apply; c' < c for apply_update),
+ *     O_c = Q_c S_c.
+ *
+ *   desc       problem; m must equal h; w_in_layout 0; update_mask, renorm, momentum,
+ *              ns_steps must be 0
+ *   q, k, v    [B,H,N,h] dtype
+ *   eta        [B,H,N] fp32
+ *   S0         per-head initial state [H,h,h] fp32 (transposed when w1_layout = 1)
+ *   out        [B,H,N,h] dtype, written
+ *   S_final    nullable; [B,H,h,h] fp32 state after the last chunk (S0's layout)
+ *   workspace  >= ttt_workspace_bytes(desc, TTT_PATH_LINEAR) bytes, 256-byte aligned
+ * Errors, streams and aliasing as for ttt_la_parallel_fwd.
+ */
+ttt_status ttt_linear_attn_fwd(const ttt_desc* desc, const void* q, const void* k,
+                               const void* v, const float* eta, const float* S0, void* out,
                                float* S_final, void* workspace, size_t workspace_bytes,
                                ttt_stream_t stream);
 

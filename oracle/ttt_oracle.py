@@ -343,6 +343,21 @@ def la_parallel_batched(q, k, v, eta, W0, W2, W1, chunk, *, order=UPDATE_APPLY, 
     return O, S
 
 
+def linear_attention_batched(q, k, v, eta, S0, chunk, *, order=UPDATE_APPLY, sign=1):
+    """The parallel form with identity features over [B,H,...] inputs (TTT≡LA notes,
+    方法步骤详情, variants 3-6: phi(x) = x), per-head initial states S0 [H,h,h].
+    Returns O [B,H,N,h] and the final states [B,H,h,h]."""
+    B, H, N, h = q.shape
+    O = np.empty((B, H, N, h))
+    S = np.empty((B, H, h, h))
+    for b in range(B):
+        for hd in range(H):
+            O[b, hd], S[b, hd] = chunked_linear_attention(q[b, hd], k[b, hd], v[b, hd],
+                                                          eta[b, hd], S0[hd], chunk, order,
+                                                          sign)
+    return O, S
+
+
 def lact_recurrent_batched(q, k, v, eta, W0, W2, W1, chunk, *, order=UPDATE_APPLY, sign=1,
                            update=WEIGHTS, renorm=False, alpha=None, ns_steps=0):
     """lact_recurrent over [B,H,...] inputs. Returns O [B,H,N,h], final weights

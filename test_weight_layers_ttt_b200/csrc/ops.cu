@@ -46,6 +46,33 @@ __global__ void prep_wk_blocked_kernel(const float* W0, const float* W2, OT* Wk,
   }
 }
 
+// ------------------------------------------------------------------ row scaling
+template <typename OT>
+__global__ void scale_rows_kernel(const OT* X, const float* eta, OT* Xs, long long rows, int w) {
+  TTT_GRID_LOOP(idx, rows * w) {
+    const long long r = idx / w;
+    Xs[idx] = from_f32<OT>(to_f32(X[idx]) * eta[r]);
+  }
+}
+
+// 16-byte version: one thread per 8 bf16 of a row (w % 8 == 0, 16-byte aligned rows).
+__global__ void scale_rows8_kernel(const uint4* X, const float* eta, uint4* Xs, long long rows,
+                                   int w8) {
+  TTT_GRID_LOOP(idx, rows * w8) {
+    const float e = eta[idx / w8];
+    const uint4 u = X[idx];
+    const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
+    uint4 o;
+    __nv_bfloat162* ov = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(hv[q]);
+      ov[q] = __floats2bfloat162_rn(f.x * e, f.y * e);
+    }
+    Xs[idx] = o;
+  }
+}
+
 // ------------------------------------------------------------------ chunk prefix scan
 // One thread per state element; the chunk axis (tens of chunks) is walked sequentially so
 // every delta is read once and every chunk state written once.
@@ -478,6 +505,24 @@ cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, 
     dim3 grid(mpad / 32, (h + 31) / 32, 2 * n_entries);
     prep_wk_blocked_kernel<OT><<<grid, dim3(32, 8), 0, s>>>(
         W0, W2, static_cast<OT*>(Wk), src_heads, h, m, src_layout);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t scale_rows(int ot, const void* X, const float* eta, void* Xs, long long rows, int w,
+                       cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const bool vec = ot == DT_BF16 && w % 8 == 0 &&
+                   ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Xs)) & 15) == 0;
+  if (vec) {
+    scale_rows8_kernel<<<grid_for(rows * (w / 8), 256), 256, 0, s>>>(
+        static_cast<const uint4*>(X), eta, static_cast<uint4*>(Xs), rows, w / 8);
+    return cudaGetLastError();
+  }
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    scale_rows_kernel<OT><<<grid_for(rows * w, 256), 256, 0, s>>>(
+        static_cast<const OT*>(X), eta, static_cast<OT*>(Xs), rows, w);
     return cudaGetLastError();
   });
 }

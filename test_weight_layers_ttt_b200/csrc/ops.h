@@ -18,6 +18,10 @@ namespace ttt {
 cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
                             int src_heads, int h, int m, int src_layout, cudaStream_t s);
 
+// Xs[r, :] = X[r, :] * eta[r] for `rows` rows of width w (OT in and out; eta fp32).
+cudaError_t scale_rows(int ot, const void* X, const float* eta, void* Xs, long long rows, int w,
+                       cudaStream_t s);
+
 // Chunk prefix sums: S starts at W1[bh % H] (layout 0 [m,h] / 1 [h,m]); for each chunk c
 // the state read by chunk c is written to Sc[bh, c] (OT, [m,h]): inclusive of dS[bh, c]
 // (order 0) or exclusive (order 1). The state after the last chunk goes to S_final

@@ -175,10 +175,12 @@ ttt_status check_desc(const ttt_desc* d, int path) {
     return fail(TTT_ERR_INVALID_ARG, "w_in_layout must be 0 or 1");
   if (d->w1_layout != 0 && d->w1_layout != 1)
     return fail(TTT_ERR_INVALID_ARG, "w1_layout must be 0 or 1");
-  if (path == TTT_PATH_PARALLEL) {
+  if (path == TTT_PATH_PARALLEL || path == TTT_PATH_LINEAR) {
     if (d->update_mask != 0 || d->renorm != 0 || d->momentum != 0 || d->ns_steps != 0)
       return fail(TTT_ERR_INVALID_ARG,
                   "parallel form: update_mask, renorm, momentum and ns_steps must be 0");
+    if (path == TTT_PATH_LINEAR && (d->m != d->h || d->w_in_layout != 0))
+      return fail(TTT_ERR_INVALID_ARG, "identity features: m must equal h, w_in_layout 0");
   } else if (path == TTT_PATH_RECURRENT) {
     if (d->update_mask < 1 || d->update_mask > 7)
       return fail(TTT_ERR_INVALID_ARG, "update_mask must be in 1..7");
@@ -190,7 +192,8 @@ ttt_status check_desc(const ttt_desc* d, int path) {
     if (d->h > 1536 || d->m > 1536)
       return fail(TTT_ERR_UNSUPPORTED, "recurrent form: h and m must be <= 1536");
   } else {
-    return fail(TTT_ERR_INVALID_ARG, "path must be TTT_PATH_PARALLEL or TTT_PATH_RECURRENT");
+    return fail(TTT_ERR_INVALID_ARG,
+                "path must be TTT_PATH_PARALLEL, TTT_PATH_RECURRENT or TTT_PATH_LINEAR");
   }
   if (d->dtype == TTT_DTYPE_BF16 && (d->h % 8 != 0 || d->m % 8 != 0))
     return fail(TTT_ERR_UNSUPPORTED, "bf16 mode needs h and m to be multiples of 8");
@@ -198,7 +201,7 @@ ttt_status check_desc(const ttt_desc* d, int path) {
   if (BH > 65535) return fail(TTT_ERR_UNSUPPORTED, "B*H must be <= 65535");
   if ((long long)d->N > (1LL << 22)) return fail(TTT_ERR_UNSUPPORTED, "N must be <= 4194304");
   const long long C = (d->N + d->chunk - 1) / d->chunk;
-  if (BH * C > 65535 && path == TTT_PATH_PARALLEL)
+  if (BH * C > 65535 && path != TTT_PATH_RECURRENT)
     return fail(TTT_ERR_UNSUPPORTED, "B*H*ceil(N/chunk) must be <= 65535");
   if ((long long)d->h * d->m > (1LL << 31))
     return fail(TTT_ERR_UNSUPPORTED, "h*m must be <= 2^31");
@@ -258,12 +261,57 @@ ttt_status run_swiglu(const char* name, const SwigluGemm& g, cudaStream_t s) {
   return gemm_simt_swiglu(g, s);
 }
 
+// Shared by both parallel variants. X_eta: the key-side features times eta, [BH, N, m].
+// Delta S_c = sign * X_eta(K_c)^T V_c per (b, head) and chunk, then the prefix scan to the
+// state read by each chunk (Sc) and the final state.
+ttt_status state_delta_and_scan(const ttt_desc& d, const void* X_eta, const void* v,
+                                const float* W1, float* S_final, float* dS, void* Sc,
+                                cudaStream_t s) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, L = d.chunk;
+  const long long C = (N + L - 1) / L, Cf = N / L, tail = N - Cf * L, hm = h * m;
+  for (int part = 0; part < 2; ++part) {
+    const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);
+    if (nz1 == 0) continue;
+    const long long t0 = part == 0 ? 0 : Cf * L;
+    GemmProblem p;
+    p.M = d.m; p.N = d.h; p.K = (int)(part == 0 ? L : tail); p.Z0 = (int)BH; p.Z1 = (int)nz1;
+    p.A = {static_cast<const char*>(X_eta) + t0 * m * dtype_size(ot), ot, true, m, N * m, L * m};
+    p.B = {static_cast<const char*>(v) + t0 * h * dtype_size(ot), ot, true, h, N * h, L * h};
+    p.C = {dS + (part == 0 ? 0 : Cf * hm), DT_F32, h, C * hm, hm};
+    p.alpha = (float)d.sign;
+    TTT_TRY(run_gemm("gemm_state_delta", p, s));
+  }
+  TTT_OP("chunk_scan", chunk_scan(ot, dS, W1, Sc, S_final, (int)BH, d.H, (int)C, d.m, d.h,
+                                  d.order, d.w1_layout, s));
+  return TTT_OK;
+}
+
+// O_c = X_q(Q_c) S_c with X_q the query-side features [BH, N, m].
+ttt_status chunk_outputs(const ttt_desc& d, const void* X_q, const void* Sc, void* out,
+                         cudaStream_t s) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, L = d.chunk;
+  const long long C = (N + L - 1) / L, Cf = N / L, tail = N - Cf * L, hm = h * m;
+  for (int part = 0; part < 2; ++part) {
+    const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);
+    if (nz1 == 0) continue;
+    const long long t0 = part == 0 ? 0 : Cf * L;
+    GemmProblem p;
+    p.M = (int)(part == 0 ? L : tail); p.N = d.h; p.K = d.m; p.Z0 = (int)BH; p.Z1 = (int)nz1;
+    p.A = {static_cast<const char*>(X_q) + t0 * m * dtype_size(ot), ot, false, m, N * m, L * m};
+    p.B = {static_cast<const char*>(Sc) + (part == 0 ? 0 : Cf * hm) * dtype_size(ot), ot, true,
+           h, C * hm, hm};
+    p.C = {static_cast<char*>(out) + t0 * h * dtype_size(ot), ot, h, N * h, L * h};
+    TTT_TRY(run_gemm("gemm_output", p, s));
+  }
+  return TTT_OK;
+}
+
 ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
                          const float* eta, const float* W0, const float* W2, const float* W1,
                          void* out, float* S_final, const ParBufs& b, cudaStream_t s) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
-  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, L = d.chunk;
-  const long long C = (N + L - 1) / L, Cf = N / L, tail = N - Cf * L, hm = h * m;
   const bool shared_qk = (q == k);
 
   TTT_OP("prep_weights",
@@ -272,39 +320,40 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
   TTT_TRY(run_swiglu("gemm_features_k",
                      features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
                      s));
-  // Delta S_c = sign * phi(K_c)^T diag(eta) V_c  (per (b, head) and chunk)
-  for (int part = 0; part < 2; ++part) {
-    const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);
-    if (nz1 == 0) continue;
-    const long long t0 = part == 0 ? 0 : Cf * L;
-    GemmProblem p;
-    p.M = d.m; p.N = d.h; p.K = (int)(part == 0 ? L : tail); p.Z0 = (int)BH; p.Z1 = (int)nz1;
-    p.A = {static_cast<const char*>(b.phiA) + t0 * m * dtype_size(ot), ot, true, m, N * m, L * m};
-    p.B = {static_cast<const char*>(v) + t0 * h * dtype_size(ot), ot, true, h, N * h, L * h};
-    p.C = {b.dS + (part == 0 ? 0 : Cf * hm), DT_F32, h, C * hm, hm};
-    p.alpha = (float)d.sign;
-    TTT_TRY(run_gemm("gemm_state_delta", p, s));
-  }
-  // States read by each chunk, and the final state.
-  TTT_OP("chunk_scan", chunk_scan(ot, b.dS, W1, b.Sc, S_final, (int)BH, d.H, (int)C, d.m, d.h,
-                                  d.order, d.w1_layout, s));
+  TTT_TRY(state_delta_and_scan(d, b.phiA, v, W1, S_final, b.dS, b.Sc, s));
   if (!shared_qk)
     TTT_TRY(run_swiglu("gemm_features_q",
                        features_problem(d, q, b.Wk, b.phiB, nullptr, nullptr), s));
-  // O_c = phi(Q_c) S_c
-  for (int part = 0; part < 2; ++part) {
-    const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);
-    if (nz1 == 0) continue;
-    const long long t0 = part == 0 ? 0 : Cf * L;
-    GemmProblem p;
-    p.M = (int)(part == 0 ? L : tail); p.N = d.h; p.K = d.m; p.Z0 = (int)BH; p.Z1 = (int)nz1;
-    p.A = {static_cast<const char*>(b.phiB) + t0 * m * dtype_size(ot), ot, false, m, N * m, L * m};
-    p.B = {static_cast<const char*>(b.Sc) + (part == 0 ? 0 : Cf * hm) * dtype_size(ot), ot, true,
-           h, C * hm, hm};
-    p.C = {static_cast<char*>(out) + t0 * h * dtype_size(ot), ot, h, N * h, L * h};
-    TTT_TRY(run_gemm("gemm_output", p, s));
-  }
-  return TTT_OK;
+  return chunk_outputs(d, b.phiB, b.Sc, out, s);
+}
+
+// ------------------------------------------------------------------ identity features
+// Variants 3-6 of the simplification ladder: phi = identity, i.e. plain chunked linear
+// attention with per-token eta; the state is [h, h].
+struct LinBufs {
+  void* Keta;  // k * eta  [BH, N, h]
+  float* dS;   // [BH, C, h, h]
+  void* Sc;    // [BH, C, h, h]
+};
+
+size_t plan_linear(const ttt_desc& d, void* base, LinBufs& b) {
+  Carve cv(base);
+  const size_t os = d.dtype == TTT_DTYPE_BF16 ? 2 : 4;
+  const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
+  const long long hh = (long long)d.h * d.h;
+  b.Keta = cv.take(os * BH * d.N * d.h);
+  b.dS = cv.take_n<float>(BH * C * hh);
+  b.Sc = cv.take(os * BH * C * hh);
+  return cv.off;
+}
+
+ttt_status linear_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
+                       const float* eta, const float* S0, void* out, float* S_final,
+                       const LinBufs& b, cudaStream_t s) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  TTT_OP("scale_rows", scale_rows(ot, k, eta, b.Keta, (long long)d.B * d.H * d.N, d.h, s));
+  TTT_TRY(state_delta_and_scan(d, b.Keta, v, S0, S_final, b.dS, b.Sc, s));
+  return chunk_outputs(d, q, b.Sc, out, s);
 }
 
 // ------------------------------------------------------------------ recurrent form
@@ -529,6 +578,10 @@ size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path) {
     ParBufs b;
     return plan_parallel(*desc, nullptr, b);
   }
+  if (path == TTT_PATH_LINEAR) {
+    LinBufs b;
+    return plan_linear(*desc, nullptr, b);
+  }
   RecBufs b;
   return plan_recurrent(*desc, nullptr, b);
 }
@@ -560,6 +613,34 @@ ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* 
     return TTT_OK;
   }
   return parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s);
+}
+
+ttt_status ttt_linear_attn_fwd(const ttt_desc* desc, const void* q, const void* k, const void* v,
+                               const float* eta, const float* S0, void* out, float* S_final,
+                               void* workspace, size_t workspace_bytes, ttt_stream_t stream) {
+  TTT_TRY(check_desc(desc, TTT_PATH_LINEAR));
+  const ttt_desc& d = *desc;
+  const long long BH = (long long)d.B * d.H;
+  if (BH == 0) return TTT_OK;
+  if (!S0) return fail(TTT_ERR_INVALID_ARG, "S0 must not be NULL");
+  if (d.N > 0) {
+    if (!q || !k || !v || !eta || !out)
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v, eta and out must not be NULL");
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(out) || !al16(S0))
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v, out and S0 must be 16-byte aligned");
+  }
+  LinBufs b;
+  const size_t need = plan_linear(d, nullptr, b);
+  TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  plan_linear(d, workspace, b);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d.N == 0) {
+    if (S_final)
+      TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, S0, b.Sc, S_final, (int)BH, d.H, 0, d.h, d.h,
+                                      d.order, d.w1_layout, s));
+    return TTT_OK;
+  }
+  return linear_impl(d, q, k, v, eta, S0, out, S_final, b, s);
 }
 
 ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const void* k,

@@ -70,6 +70,26 @@ def la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk, *, order="update_apply", si
     return out, S
 
 
+def linear_attn_fwd(q, k, v, eta, S0, chunk, *, order="update_apply", sign=1, s_layout=0,
+                    return_state=True, out=None, ws=None, stream=None):
+    """Parallel form with identity features (plain chunked linear attention with per-token
+    eta). S0 [H,h,h] fp32. Returns (out [B,H,N,h], final state [B,H,h,h] or None)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    _need(eta, "eta", torch.float32)
+    _need(S0, "S0", torch.float32)
+    B, H, N, h = q.shape
+    desc = abi.ttt_desc(B=B, H=H, N=N, h=h, m=h, chunk=chunk, dtype=_dtype_code(q),
+                        order=ORDERS[order], sign=sign, w1_layout=s_layout)
+    if out is None:
+        out = torch.empty_like(q)
+    S = torch.empty((B, H, h, h), dtype=torch.float32, device=q.device) if return_state else None
+    if ws is None:
+        ws = workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_LINEAR), q.device)
+    abi.ttt_linear_attn_fwd(desc, q, k, v, eta, S0, out, S, ws, stream=stream)
+    return out, S
+
+
 def recurrent_desc(q, W1, chunk, order="update_apply", sign=1, update_mask=abi.TTT_UPDATE_ALL,
                    renorm=False, momentum=False, ns_steps=0):
     B, H, N, h = q.shape

@@ -113,6 +113,28 @@ def test_parallel_rejects_pointers_and_workspace():
     assert "256-byte" in abi.ttt_last_error_message()
 
 
+def test_linear_attention_workspace_and_checks():
+    d = lm_desc(m=256)   # identity features: the state is [h, h]
+    BH, N, h, C = 8, 32768, 256, 16
+    expect = 2 * BH * N * h + 4 * BH * C * h * h + 2 * BH * C * h * h
+    got = abi.ttt_workspace_bytes(d, abi.TTT_PATH_LINEAR)
+    assert expect <= got <= expect + 3 * 256
+    assert abi.ttt_workspace_bytes(lm_desc(), abi.TTT_PATH_LINEAR) == 0        # m != h
+    assert abi.ttt_workspace_bytes(lm_desc(m=256, w_in_layout=1), 2) == 0
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_linear_attn_fwd(lm_desc(), 256, 256, 256, 256, 256, 256, None, 256, 1 << 40,
+                                stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    with pytest.raises(abi.TTTError) as ei:   # NULL S0
+        abi.ttt_linear_attn_fwd(d, 256, 256, 256, 256, None, 256, None, 256, got, stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    with pytest.raises(abi.TTTError) as ei:   # workspace too small
+        abi.ttt_linear_attn_fwd(d, 256, 256, 256, 256, 256, 256, None, 256, got - 1, stream=0)
+    assert ei.value.status == abi.TTT_ERR_WORKSPACE
+    abi.ttt_linear_attn_fwd(lm_desc(B=0, m=256), None, None, None, None, None, None, None,
+                            None, 0, stream=0)
+
+
 def test_recurrent_rejects_bad_args():
     d = lm_desc(update_mask=7, momentum=1)
     need = abi.ttt_workspace_bytes(d, 1)

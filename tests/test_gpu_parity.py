@@ -135,6 +135,45 @@ def test_parallel_rejects_misaligned_pointer_on_device():
     assert ei.value.status == abi.TTT_ERR_INVALID_ARG
 
 
+# ----------------------------------------------------------------------------- identity features
+LIN_CASES = [
+    # dtype, B, H, N, h, chunk, s_layout, sign
+    ("fp32", 1, 2, 200, 24, 48, 0, 1),
+    ("bf16", 2, 2, 1000, 128, 256, 0, 1),
+    ("bf16", 1, 3, 700, 64, 128, 1, -1),
+]
+
+
+@pytest.mark.parametrize("case", LIN_CASES, ids=lambda c: "-".join(map(str, c)))
+@pytest.mark.parametrize("order", ["update_apply", "apply_update"])
+def test_linear_attention_matches_oracle(case, order):
+    """phi = identity (variants 3-6 of the simplification ladder): plain chunked linear
+    attention with per-token eta, multi-tile and ragged last chunk, both state layouts."""
+    dtype, B, H, N, h, chunk, s_layout, sign = case
+    wl, inp = layer_inputs("lm", dtype, B, H, N, h, h, chunk, seed=3000 + N)
+    S0 = inp["W1"]                        # [H, h, h]
+    ref, Sref = O.linear_attention_batched(inp["q"], inp["k"], inp["v"], inp["eta"], S0, chunk,
+                                           order=ORD[order], sign=sign)
+    td = torch_dtype(dtype)
+    q, k, v = (dev(inp[n], td) for n in ("q", "k", "v"))
+    eta = dev(inp["eta"])
+    S0_dev = dev(np.ascontiguousarray(np.swapaxes(S0, 1, 2)) if s_layout else S0)
+    out, S = layer.linear_attn_fwd(q, k, v, eta, S0_dev, chunk, order=order, sign=sign,
+                                   s_layout=s_layout)
+    abi.ttt_last_device_status()
+    Sh = host(S)
+    if s_layout:
+        Sh = np.swapaxes(Sh, 2, 3)
+    assert rel(host(out), ref) <= TOL[dtype]
+    assert rel(Sh, Sref) <= TOL[dtype]
+    # state-driven part alone (zero initial state)
+    Z = np.zeros_like(S0)
+    ref0, Sref0 = O.linear_attention_batched(inp["q"], inp["k"], inp["v"], inp["eta"], Z, chunk,
+                                             order=ORD[order], sign=sign)
+    out0, S0r = layer.linear_attn_fwd(q, k, v, eta, dev(Z), chunk, order=order, sign=sign)
+    assert rel(host(out0), ref0) <= TOL[dtype]
+
+
 # ----------------------------------------------------------------------------- recurrent
 REC_CASES = [
     # kind, dtype, B, H, N, h, m, chunk, opts
