@@ -109,6 +109,7 @@ def kernel_work(name: str, wl, form: str):
         }
         return table.get(base, (None, None))
     table = {
+        "fused_apply": ("tensor", 6.0 * h * m * T),   # phi(Q) (4hm) and phi(Q) S_c (2hm)
         "gemm_features_k": ("tensor", 4.0 * h * m * T),
         "gemm_features_q": ("tensor", 4.0 * h * m * T),
         "gemm_state_delta": ("tensor", 2.0 * h * m * T),

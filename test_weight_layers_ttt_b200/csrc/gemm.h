@@ -76,6 +76,16 @@ struct SwigluGemm {
   const void* dv = nullptr;
   long long ldd = 0, ds0 = 0, ds1 = 0;
 };
+// Query side of the parallel form fused (apply_fused.cu): out = phi(Q) S_c per 128-row tile
+// with phi kept in shared memory. q [B,H,N,h] bf16; Wk the blocked [W0/2 ; W2] operand per
+// head ([H, 2 * mpad, h], see prep_wk_blocked); Sc the bf16 chunk states [B*H, C, m, h];
+// out [B,H,N,h] bf16. Needs h = 128 or 256 and chunk % 128 == 0.
+bool fused_apply_supported(int dtype, int h, int m, int chunk, const void* q, const void* Wk,
+                           const void* Sc, const void* out);
+ttt_status fused_apply(const void* q, const void* Wk, const void* Sc, void* out, int B, int H,
+                       int N, int h, int m, int chunk, unsigned* err,
+                       unsigned long long wait_ns, cudaStream_t s);
+
 bool umma_swiglu_supported(const SwigluGemm& g);
 ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream);
 ttt_status gemm_umma_swiglu(const SwigluGemm& g, cudaStream_t stream, unsigned* dev_err,

@@ -321,6 +321,13 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
                      features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
                      s));
   TTT_TRY(state_delta_and_scan(d, b.phiA, v, W1, S_final, b.dS, b.Sc, s));
+  if (!shared_qk && !force_simt() && !getenv("TTT_NO_FUSED_APPLY") &&
+      fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
+    // phi(Q) S_c with phi kept on chip
+    TraceScope ts("fused_apply@tcgen05", s);
+    return fused_apply(q, b.Wk, b.Sc, out, d.B, d.H, d.N, d.h, d.m, d.chunk,
+                       device_error_word(), wait_limit_ns(), s);
+  }
   if (!shared_qk)
     TTT_TRY(run_swiglu("gemm_features_q",
                        features_problem(d, q, b.Wk, b.phiB, nullptr, nullptr), s));

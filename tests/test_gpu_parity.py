@@ -94,6 +94,30 @@ def test_feature_gemm_on_cta_pairs_and_single_ctas(monkeypatch):
         assert rel(a, b) <= 1e-2
 
 
+@pytest.mark.parametrize("case", [
+    # B, H, N, h, m, chunk: odd number of 128-column phi blocks and more tiles than SMs;
+    # ragged m (zero-padded phi block, state rows past m) and ragged N
+    (2, 4, 4096, 128, 384, 512),
+    (1, 2, 1000, 256, 200, 256),
+], ids=lambda c: "-".join(map(str, c)))
+def test_fused_query_side_matches_oracle_and_unfused(case, monkeypatch):
+    """phi(Q_c) S_c computed with phi kept in shared memory (h = 128 or 256, chunk a
+    multiple of 128) against the oracle and against the unfused feature + output GEMMs."""
+    B, H, N, h, m, chunk = case
+    wl, inp = layer_inputs("lm", "bf16", B, H, N, h, m, chunk, seed=90 + N)
+    ref, Sref = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
+                                      inp["W2"], inp["W1"], chunk)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    monkeypatch.delenv("TTT_NO_FUSED_APPLY", raising=False)
+    fused, Sf = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk)
+    monkeypatch.setenv("TTT_NO_FUSED_APPLY", "1")
+    plain, Sp = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk)
+    abi.ttt_last_device_status()
+    assert rel(host(fused), ref) <= TOL["bf16"] and rel(host(Sf), Sref) <= TOL["bf16"]
+    assert rel(host(fused), host(plain)) <= 1e-2
+    assert torch.equal(Sf, Sp)
+
+
 def test_parallel_ascent_equals_descent_with_negated_values():
     wl, inp = layer_inputs("lm", "bf16", 1, 2, 512, 64, 128, 128, seed=7)
     q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
