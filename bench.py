@@ -48,6 +48,9 @@ def layer_flops(wl, form: str) -> float:
         return float(feats + 2 * hm * T + 2 * hm * T)
     if form == "linear":   # identity features: state deltas and outputs, [h, h] states
         return 4.0 * wl.h * wl.h * T
+    if form == "parallel_momentum":   # parallel form + Newton-Schulz 5 on every chunk's W1 step
+        r, c = min(wl.h, wl.m), max(wl.h, wl.m)
+        return 12.0 * hm * T + 5 * (4.0 * r * r * c + 2.0 * r ** 3) * wl.B * wl.H * wl.C
     flops = 18.0 * hm * T   # 9 matmuls: K features (2), D, 3 gradients, Q features (2), out
     if wl.ns_steps:
         r, c = min(wl.h, wl.m), max(wl.h, wl.m)
@@ -382,6 +385,8 @@ def run_gpu(args, rank, local, world):
     forms = [f for f in ("parallel", "recurrent") if f in wl.paths]
     if wl.kind == "lm" and "parallel" in forms:
         forms.insert(1, "linear")   # identity features (plain chunked linear attention)
+        # W1 momentum + Newton-Schulz 5 (simplification variant 2)
+        forms.insert(2, "parallel_momentum")
     lin, l1 = g["layouts"]
     if wl.kind == "inplace":
         # the value target is part of the In-Place step; timed on its own below
@@ -405,6 +410,18 @@ def run_gpu(args, rank, local, world):
             def step():
                 abi.ttt_linear_attn_fwd(ldesc, g["q"], g["k"], g["v"], g["eta"], lS0, lout,
                                         None, lws)
+        elif form == "parallel_momentum":
+            mdesc = layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order, 1, lin, l1)
+            mdesc.momentum, mdesc.ns_steps = 1, 5
+            mws = layer.workspace(
+                abi.ttt_workspace_bytes(mdesc, abi.TTT_PATH_PARALLEL_MOMENTUM), "cuda")
+            malpha = g["alpha"] if g["alpha"] is not None else torch.full(
+                (wl.B, wl.H, wl.C), 0.9, dtype=torch.float32, device="cuda")
+            mout = torch.empty_like(g["q"])
+
+            def step():
+                abi.ttt_la_parallel_momentum_fwd(mdesc, g["q"], g["k"], g["v"], g["eta"], malpha,
+                                                 g["W0"], g["W2"], g["W1"], mout, None, mws)
         elif form == "parallel":
             desc = layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order, 1, lin, l1)
             ws = layer.workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_PARALLEL), "cuda")
@@ -425,7 +442,7 @@ def run_gpu(args, rank, local, world):
                 abi.ttt_lact_recurrent_fwd(desc, g["q"], g["k"], g["v"], g["eta"], g["alpha"],
                                            g["W0"], g["W2"], g["W1"], out, None, None, None,
                                            None, ws)
-        steps = args.steps if form in ("parallel", "linear") else max(3, args.steps // 2)
+        steps = args.steps if form in ("parallel", "linear") else max(3, args.steps // 4)
         with ClockSampler(gpu_id(local, torch)) as clk:
             ms, trace = _timed(step, steps, args.warmup, world, torch, trace_capacity=16384)
         abi.ttt_last_device_status()

@@ -69,7 +69,12 @@ typedef enum ttt_status {
 enum { TTT_DTYPE_FP32 = 0, TTT_DTYPE_BF16 = 1 };
 enum { TTT_ORDER_UPDATE_APPLY = 0, TTT_ORDER_APPLY_UPDATE = 1 };
 enum { TTT_UPDATE_W0 = 1, TTT_UPDATE_W1 = 2, TTT_UPDATE_W2 = 4, TTT_UPDATE_ALL = 7 };
-enum { TTT_PATH_PARALLEL = 0, TTT_PATH_RECURRENT = 1, TTT_PATH_LINEAR = 2 };
+enum {
+  TTT_PATH_PARALLEL = 0,
+  TTT_PATH_RECURRENT = 1,
+  TTT_PATH_LINEAR = 2,
+  TTT_PATH_PARALLEL_MOMENTUM = 3
+};
 
 /* Problem description. All fields are read; unused ones must be 0 unless noted. */
 typedef struct ttt_desc {
@@ -91,9 +96,8 @@ typedef struct ttt_desc {
 } ttt_desc;
 
 /*
- * Workspace size in bytes for `path` (TTT_PATH_PARALLEL, TTT_PATH_RECURRENT or
- * TTT_PATH_LINEAR), or 0 when the description is invalid for that path. Host-only;
- * touches no device.
+ * Workspace size in bytes for `path` (one of TTT_PATH_*), or 0 when the description is
+ * invalid for that path. Host-only; touches no device.
  */
 size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path);
 
@@ -123,6 +127,33 @@ ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* 
                                const float* W2, const float* W1, void* out,
                                float* S_final, void* workspace, size_t workspace_bytes,
                                ttt_stream_t stream);
+
+/*
+ * Parallel last-layer-only form with momentum and orthogonalisation of the W1 update
+ * ("Test-Time Training with KV Binding Is Secretly Linear Attention", section 方法步骤详情:
+ * simplification variant 2 keeps momentum and Newton-Schulz; the pages' recurrent -> parallel
+ * throughput comparison is made on it). W0, W2 frozen and no renormalisation make each
+ * chunk's W1 gradient independent of W1, so for all chunks at once
+ *     D_c = sign * phi(K_c)^T diag(eta_c) V_c,
+ *     M_c = alpha_c M_{c-1} + D_c            (momentum = 1; M_{-1} = 0; else M_c = D_c),
+ *     U_c = NS_{ns_steps}(M_c)               (ns_steps > 0; else U_c = M_c),
+ *     S_c = W1 + sum_{c' <= c} U_c'          (update_apply; c' < c for apply_update),
+ *     O_c = phi(Q_c) S_c.
+ * NS is the pages' iteration (coefficients 3.4445, -4.7750, 2.0315 on X = M / (||M||_F +
+ * 1e-7), rows <= cols orientation). This equals the recurrent form with update_mask = W1,
+ * the same momentum and ns_steps and no renormalisation.
+ *
+ *   desc       problem; update_mask and renorm must be 0; momentum 0 or 1; ns_steps 0..8;
+ *              w1_layout 0
+ *   alpha      [B,H,ceil(N/chunk)] fp32 momentum factors (needed when momentum = 1)
+ *   other arguments as for ttt_la_parallel_fwd; workspace >=
+ *   ttt_workspace_bytes(desc, TTT_PATH_PARALLEL_MOMENTUM)
+ */
+ttt_status ttt_la_parallel_momentum_fwd(const ttt_desc* desc, const void* q, const void* k,
+                                        const void* v, const float* eta, const float* alpha,
+                                        const float* W0, const float* W2, const float* W1,
+                                        void* out, float* S_final, void* workspace,
+                                        size_t workspace_bytes, ttt_stream_t stream);
 
 /*
  * Parallel form with identity features: the end of the simplification ladder ("Test-Time

@@ -35,12 +35,13 @@ TTT_UPDATE_ALL = 7
 TTT_PATH_PARALLEL = 0
 TTT_PATH_RECURRENT = 1
 TTT_PATH_LINEAR = 2
+TTT_PATH_PARALLEL_MOMENTUM = 3
 TTT_STATIC_SCRATCH_BYTES = 64 << 20
 
 # Every symbol include/ttt.h declares.
 EXPORTED = (
     "ttt_workspace_bytes", "ttt_la_parallel_fwd", "ttt_la_parallel_fwd_noalloc",
-    "ttt_linear_attn_fwd",
+    "ttt_linear_attn_fwd", "ttt_la_parallel_momentum_fwd",
     "ttt_lact_recurrent_fwd",
     "ttt_lm_target_workspace_bytes", "ttt_lm_target", "ttt_last_device_status",
     "ttt_debug_wait_timeout", "ttt_trace_enable", "ttt_trace_disable", "ttt_trace_count",
@@ -88,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_la_parallel_fwd_noalloc.restype = I32
         L.ttt_linear_attn_fwd.argtypes = [D] + [P] * 8 + [S, P]
         L.ttt_linear_attn_fwd.restype = I32
+        L.ttt_la_parallel_momentum_fwd.argtypes = [D] + [P] * 11 + [S, P]
+        L.ttt_la_parallel_momentum_fwd.restype = I32
         L.ttt_lact_recurrent_fwd.argtypes = [D] + [P] * 14 + [S, P]
         L.ttt_lact_recurrent_fwd.restype = I32
         L.ttt_lm_target_workspace_bytes.argtypes = [I32, I32]
@@ -166,6 +169,14 @@ def ttt_la_parallel_fwd(desc, q, k, v, eta, W0, W2, W1, out, S_final, workspace,
     _check(lib().ttt_la_parallel_fwd(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W0), _ptr(W2), _ptr(W1),
         _ptr(out), _ptr(S_final), _ptr(workspace), wb, _stream(stream)))
+
+
+def ttt_la_parallel_momentum_fwd(desc, q, k, v, eta, alpha, W0, W2, W1, out, S_final,
+                                 workspace, workspace_bytes=None, stream=None):
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    _check(lib().ttt_la_parallel_momentum_fwd(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(alpha), _ptr(W0),
+        _ptr(W2), _ptr(W1), _ptr(out), _ptr(S_final), _ptr(workspace), wb, _stream(stream)))
 
 
 def ttt_linear_attn_fwd(desc, q, k, v, eta, S0, out, S_final, workspace, workspace_bytes=None,

@@ -96,8 +96,8 @@ __device__ __forceinline__ void load_join8(uint32_t hbase, uint32_t lbase, uint3
 }
 
 __global__ void __launch_bounds__(NS_THREADS, 1)
-    ns_mma_kernel(float* U, int h, int m, int mask, int steps, float eps, float ca, float cb,
-                  float cc, unsigned* err, unsigned long long wait_ns) {
+    ns_mma_kernel(float* U, NsLayout Lay, int steps, float eps, float ca, float cb, float cc,
+                  unsigned* err, unsigned long long wait_ns) {
   extern __shared__ uint8_t ns_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(ns_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -106,13 +106,13 @@ __global__ void __launch_bounds__(NS_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   float* red = reinterpret_cast<float*>(tslot + 2);   // [4] warp partial sums
 
-  const int p = blockIdx.x, bh = blockIdx.y;
-  if (!(mask & (1 << p))) return;
-  const int R = p == 1 ? m : h, Cc = p == 1 ? h : m;   // U's own [R, Cc]
+  const int p = blockIdx.x, z = blockIdx.y;
+  if (!(Lay.mask & (1 << p))) return;
+  const int R = Lay.R[p], Cc = Lay.C[p];               // U's own [R, Cc]
   const bool tr = R > Cc;
   const int r = tr ? Cc : R, cols = tr ? R : Cc;       // iterate on [r, cols], r <= cols
-  const long long hm = (long long)h * m;
-  float* u = U + (long long)bh * 3 * hm + p * hm;
+  const long long hm = (long long)R * Cc;
+  float* u = U + z * Lay.zstride + p * Lay.pstride;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sb = smem_u32(smem);
   const uint32_t sXh = sb + XH_OFF, sXl = sb + XL_OFF, sGh = sb + GH_OFF, sGl = sb + GL_OFF;
@@ -289,18 +289,19 @@ __global__ void __launch_bounds__(NS_THREADS, 1)
 
 }  // namespace
 
-bool ns_mma_supported(int h, int m) {
-  const int r = h < m ? h : m, c = h < m ? m : h;
+bool ns_mma_supported(int R, int C) {
+  const int r = R < C ? R : C, c = R < C ? C : R;
   return r <= NS_ROWS && c <= NS_COLS;
 }
 
-cudaError_t ns_mma(float* U, int BH, int h, int m, int mask, int steps, float eps, float a,
-                   float b, float c, unsigned* err, unsigned long long wait_ns, cudaStream_t s) {
+cudaError_t ns_mma(float* U, int Z, const NsLayout& L, int steps, float eps, float a, float b,
+                   float c, unsigned* err, unsigned long long wait_ns, cudaStream_t s) {
+  if (Z <= 0) return cudaSuccess;
   cudaError_t e =
       cudaFuncSetAttribute(ns_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, NS_SMEM);
   if (e != cudaSuccess) return e;
-  ns_mma_kernel<<<dim3(3, BH), NS_THREADS, NS_SMEM, s>>>(U, h, m, mask, steps, eps, a, b, c,
-                                                         err, wait_ns);
+  ns_mma_kernel<<<dim3(L.parts, Z), NS_THREADS, NS_SMEM, s>>>(U, L, steps, eps, a, b, c, err,
+                                                              wait_ns);
   return cudaGetLastError();
 }
 

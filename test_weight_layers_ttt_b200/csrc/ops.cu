@@ -258,17 +258,16 @@ __global__ void rec_reduce_kernel(const float* partials, int splits, float* U, f
 
 // One block per (part, bh): Frobenius norm, then the normalised update in the orientation
 // with rows <= cols.
-__global__ void ns_normalize_kernel(const float* U, float* X, int h, int m, int mask, float eps) {
-  const int p = blockIdx.x, bh = blockIdx.y;
-  if (!(mask & (1 << p))) return;
-  int R, Cc;
-  part_dims(p, h, m, R, Cc);
-  const long long hm = (long long)h * m;
-  const float* u = U + (long long)bh * 3 * hm + p * hm;
-  float* x = X + ((long long)bh * 3 + p) * hm;
+__global__ void ns_normalize_kernel(const float* U, float* X, NsLayout L, float eps) {
+  const int p = blockIdx.x, z = blockIdx.y;
+  if (!(L.mask & (1 << p))) return;
+  const int R = L.R[p], Cc = L.C[p];
+  const long long n = (long long)R * Cc;
+  const float* u = U + z * L.zstride + p * L.pstride;
+  float* x = X + ((long long)z * L.parts + p) * n;
   __shared__ float red[32];
   float ss = 0.0f;
-  for (long long e = threadIdx.x; e < hm; e += blockDim.x) ss += u[e] * u[e];
+  for (long long e = threadIdx.x; e < n; e += blockDim.x) ss += u[e] * u[e];
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
@@ -280,24 +279,36 @@ __global__ void ns_normalize_kernel(const float* U, float* X, int h, int m, int 
   __syncthreads();
   const float scale = 1.0f / (sqrtf(red[0]) + eps);
   const bool tr = R > Cc;
-  for (long long e = threadIdx.x; e < hm; e += blockDim.x) {
+  for (long long e = threadIdx.x; e < n; e += blockDim.x) {
     const int i = (int)(e / Cc), j = (int)(e - (long long)i * Cc);
     x[tr ? (long long)j * R + i : e] = u[e] * scale;
   }
 }
 
-__global__ void ns_writeback_kernel(const float* X, float* U, int h, int m, int mask) {
-  const int p = blockIdx.x, bh = blockIdx.y;
-  if (!(mask & (1 << p))) return;
-  int R, Cc;
-  part_dims(p, h, m, R, Cc);
-  const long long hm = (long long)h * m;
-  float* u = U + (long long)bh * 3 * hm + p * hm;
-  const float* x = X + ((long long)bh * 3 + p) * hm;
+__global__ void ns_writeback_kernel(const float* X, float* U, NsLayout L) {
+  const int p = blockIdx.x, z = blockIdx.y;
+  if (!(L.mask & (1 << p))) return;
+  const int R = L.R[p], Cc = L.C[p];
+  const long long n = (long long)R * Cc;
+  float* u = U + z * L.zstride + p * L.pstride;
+  const float* x = X + ((long long)z * L.parts + p) * n;
   const bool tr = R > Cc;
-  for (long long e = threadIdx.x; e < hm; e += blockDim.x) {
+  for (long long e = threadIdx.x; e < n; e += blockDim.x) {
     const int i = (int)(e / Cc), j = (int)(e - (long long)i * Cc);
     u[e] = x[tr ? (long long)j * R + i : e];
+  }
+}
+
+// One thread per element, chunks in order (the chunk axis is short).
+__global__ void momentum_scan_kernel(float* D, const float* alpha, int BH, int C, long long n) {
+  TTT_GRID_LOOP(idx, (long long)BH * n) {
+    const long long bh = idx / n, e = idx - bh * n;
+    float* d = D + bh * C * n + e;
+    float mv = d[0];
+    for (int c = 1; c < C; ++c) {
+      mv = fmaf(alpha[bh * C + c], mv, d[(long long)c * n]);
+      d[(long long)c * n] = mv;
+    }
   }
 }
 
@@ -586,15 +597,21 @@ cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all
   return cudaGetLastError();
 }
 
-cudaError_t ns_normalize(const float* U, float* X, int BH, int h, int m, int mask, float eps,
+cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
                          cudaStream_t s) {
-  ns_normalize_kernel<<<dim3(3, BH), 256, 0, s>>>(U, X, h, m, mask, eps);
+  ns_normalize_kernel<<<dim3(L.parts, Z), 256, 0, s>>>(U, X, L, eps);
   return cudaGetLastError();
 }
 
-cudaError_t ns_writeback(const float* X, float* U, int BH, int h, int m, int mask,
-                         cudaStream_t s) {
-  ns_writeback_kernel<<<dim3(3, BH), 256, 0, s>>>(X, U, h, m, mask);
+cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cudaStream_t s) {
+  ns_writeback_kernel<<<dim3(L.parts, Z), 256, 0, s>>>(X, U, L);
+  return cudaGetLastError();
+}
+
+cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long n,
+                          cudaStream_t s) {
+  if (BH <= 0 || C <= 1 || n <= 0) return cudaSuccess;
+  momentum_scan_kernel<<<grid_for((long long)BH * n, 256), 256, 0, s>>>(D, alpha, BH, C, n);
   return cudaGetLastError();
 }
 

@@ -43,20 +43,45 @@ cudaError_t col_norms(const float* W0, const float* W2, const float* W1, int H, 
 cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all,
                        const float* alpha, int C, int c, int BH, int h, int m, int mask,
                        cudaStream_t s);
-// Newton-Schulz set-up / tear-down: X = U / (||U||_F + eps) in the wide orientation
-// ([rmin, rmax]) for every (bh, part in mask); and U <- X back in U's own orientation.
-cudaError_t ns_normalize(const float* U, float* X, int BH, int h, int m, int mask, float eps,
+// Where the matrices of a batched Newton-Schulz live: matrix (part p, entry z) starts at
+// U + z * zstride + p * pstride and is [R[p], C[p]] row-major (every part has R * C
+// elements); parts not in `mask` are skipped.
+struct NsLayout {
+  int parts, mask;
+  long long zstride, pstride;
+  int R[3], C[3];
+};
+// The recurrent state [W0 (h x m) | W1 (m x h) | W2 (h x m)] of each (b, head).
+inline NsLayout ns_layout_weights(int h, int m, int mask) {
+  const long long hm = (long long)h * m;
+  return NsLayout{3, mask, 3 * hm, hm, {h, m, h}, {m, h, m}};
+}
+// One [R, C] matrix per entry, entries R * C apart.
+inline NsLayout ns_layout_single(int R, int C) {
+  return NsLayout{1, 1, (long long)R * C, 0, {R, R, R}, {C, C, C}};
+}
+
+// Newton-Schulz set-up / tear-down for the CUDA-core path: X = U / (||U||_F + eps) in the
+// wide orientation ([min(R,C), max(R,C)]) into the scratch X (problem (z, p) at
+// (z * parts + p) * R * C), and U <- X back in U's own orientation. Z entries.
+cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
                          cudaStream_t s);
-cudaError_t ns_writeback(const float* X, float* U, int BH, int h, int m, int mask,
-                         cudaStream_t s);
-// The whole Newton-Schulz orthogonalisation of U's parts in `mask` on the tensor cores
+cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cudaStream_t s);
+
+// The whole Newton-Schulz orthogonalisation of the matrices of L on the tensor cores
 // (ns_mma.cu; operands split into bf16 hi + lo pairs, fp32 accumulation): normalise,
 // `steps` iterations X <- a X + (b A + c A A) X with A = X X^T on the rows <= cols
-// orientation, write back. Only for min(h, m) <= 128 and max(h, m) <= 256
+// orientation, write back. Only for min(R, C) <= 128 and max(R, C) <= 256 for every part
 // (ns_mma_supported). Bounded waits report through `err`.
-bool ns_mma_supported(int h, int m);
-cudaError_t ns_mma(float* U, int BH, int h, int m, int mask, int steps, float eps, float a,
-                   float b, float c, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
+bool ns_mma_supported(int R, int C);
+cudaError_t ns_mma(float* U, int Z, const NsLayout& L, int steps, float eps, float a, float b,
+                   float c, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
+
+// Momentum over chunks, in place: D[bh, c] <- alpha[bh, c] * D[bh, c - 1] + D[bh, c] for
+// c = 1 .. C-1 (D [BH, C, n] fp32, alpha [BH, C]).
+cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long n,
+                          cudaStream_t s);
+
 // W <- W - sign * U, optional per-column renormalisation to tnorm, refresh the OT copies:
 // W1o [BH, m, h] and the blocked input-side operand Wk [BH, 2 * mpad, h] (see
 // prep_wk_blocked).

@@ -175,7 +175,15 @@ ttt_status check_desc(const ttt_desc* d, int path) {
     return fail(TTT_ERR_INVALID_ARG, "w_in_layout must be 0 or 1");
   if (d->w1_layout != 0 && d->w1_layout != 1)
     return fail(TTT_ERR_INVALID_ARG, "w1_layout must be 0 or 1");
-  if (path == TTT_PATH_PARALLEL || path == TTT_PATH_LINEAR) {
+  if (path == TTT_PATH_PARALLEL_MOMENTUM) {
+    if (d->update_mask != 0 || d->renorm != 0)
+      return fail(TTT_ERR_INVALID_ARG, "parallel form: update_mask and renorm must be 0");
+    if (d->momentum != 0 && d->momentum != 1)
+      return fail(TTT_ERR_INVALID_ARG, "momentum must be 0 or 1");
+    if (d->ns_steps < 0 || d->ns_steps > 8) return fail(TTT_ERR_INVALID_ARG, "ns_steps must be in 0..8");
+    if (d->w1_layout != 0)
+      return fail(TTT_ERR_UNSUPPORTED, "parallel form with momentum: W1 layout 0 only");
+  } else if (path == TTT_PATH_PARALLEL || path == TTT_PATH_LINEAR) {
     if (d->update_mask != 0 || d->renorm != 0 || d->momentum != 0 || d->ns_steps != 0)
       return fail(TTT_ERR_INVALID_ARG,
                   "parallel form: update_mask, renorm, momentum and ns_steps must be 0");
@@ -192,8 +200,7 @@ ttt_status check_desc(const ttt_desc* d, int path) {
     if (d->h > 1536 || d->m > 1536)
       return fail(TTT_ERR_UNSUPPORTED, "recurrent form: h and m must be <= 1536");
   } else {
-    return fail(TTT_ERR_INVALID_ARG,
-                "path must be TTT_PATH_PARALLEL, TTT_PATH_RECURRENT or TTT_PATH_LINEAR");
+    return fail(TTT_ERR_INVALID_ARG, "path must be one of TTT_PATH_*");
   }
   if (d->dtype == TTT_DTYPE_BF16 && (d->h % 8 != 0 || d->m % 8 != 0))
     return fail(TTT_ERR_UNSUPPORTED, "bf16 mode needs h and m to be multiples of 8");
@@ -264,9 +271,8 @@ ttt_status run_swiglu(const char* name, const SwigluGemm& g, cudaStream_t s) {
 // Shared by both parallel variants. X_eta: the key-side features times eta, [BH, N, m].
 // Delta S_c = sign * X_eta(K_c)^T V_c per (b, head) and chunk, then the prefix scan to the
 // state read by each chunk (Sc) and the final state.
-ttt_status state_delta_and_scan(const ttt_desc& d, const void* X_eta, const void* v,
-                                const float* W1, float* S_final, float* dS, void* Sc,
-                                cudaStream_t s) {
+ttt_status state_deltas(const ttt_desc& d, const void* X_eta, const void* v, float* dS,
+                        cudaStream_t s) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, L = d.chunk;
   const long long C = (N + L - 1) / L, Cf = N / L, tail = N - Cf * L, hm = h * m;
@@ -282,9 +288,23 @@ ttt_status state_delta_and_scan(const ttt_desc& d, const void* X_eta, const void
     p.alpha = (float)d.sign;
     TTT_TRY(run_gemm("gemm_state_delta", p, s));
   }
+  return TTT_OK;
+}
+
+ttt_status chunk_states(const ttt_desc& d, const float* dS, const float* W1, float* S_final,
+                        void* Sc, cudaStream_t s) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
   TTT_OP("chunk_scan", chunk_scan(ot, dS, W1, Sc, S_final, (int)BH, d.H, (int)C, d.m, d.h,
                                   d.order, d.w1_layout, s));
   return TTT_OK;
+}
+
+ttt_status state_delta_and_scan(const ttt_desc& d, const void* X_eta, const void* v,
+                                const float* W1, float* S_final, float* dS, void* Sc,
+                                cudaStream_t s) {
+  TTT_TRY(state_deltas(d, X_eta, v, dS, s));
+  return chunk_states(d, dS, W1, S_final, Sc, s);
 }
 
 // O_c = X_q(Q_c) S_c with X_q the query-side features [BH, N, m].
@@ -363,13 +383,121 @@ ttt_status linear_impl(const ttt_desc& d, const void* q, const void* k, const vo
   return chunk_outputs(d, q, b.Sc, out, s);
 }
 
-// ------------------------------------------------------------------ recurrent form
+// ------------------------------------------------------------------ Newton-Schulz
 // bf16 mode runs Newton-Schulz on the tensor cores (split bf16 operands, close to fp32)
 // when the matrices fit one CTA; fp32 mode and larger matrices use fp32 CUDA-core products.
 bool ns_on_tensor_cores(const ttt_desc& d) {
   return d.dtype == TTT_DTYPE_BF16 && ns_mma_supported(d.h, d.m);
 }
 
+// Scratch of the CUDA-core Newton-Schulz: X, X2 [problems, r, c], Ag, Pm [problems, r, r].
+struct NsScratch {
+  float *X, *X2, *Ag, *Pm;
+};
+
+// Newton-Schulz (the pages' five-step coefficients, eps 1e-7) in place on the matrices of
+// L: tensor cores for bf16 mode when they fit one CTA, else fp32 CUDA-core products (the
+// problems of the masked-out parts are computed and not written back).
+ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const NsScratch& w,
+                  cudaStream_t s) {
+  const float a3 = 3.4445f, b3 = -4.7750f, c3 = 2.0315f;
+  const long long R = L.R[0], Cc = L.C[0];
+  if (ot == DT_BF16 && ns_mma_supported((int)R, (int)Cc)) {
+    TTT_OP("ns_mma", ns_mma(U, Z, L, steps, 1e-7f, a3, b3, c3, device_error_word(),
+                            wait_limit_ns(), s));
+    return TTT_OK;
+  }
+  const long long r = R < Cc ? R : Cc, cc = R < Cc ? Cc : R;
+  const int P = Z * L.parts;
+  TTT_OP("ns_normalize", ns_normalize(U, w.X, Z, L, 1e-7f, s));
+  float* X = w.X;
+  float* X2 = w.X2;
+  for (int it = 0; it < steps; ++it) {
+    GemmProblem g1;  // A = X X^T
+    g1.M = (int)r; g1.N = (int)r; g1.K = (int)cc; g1.Z0 = P;
+    g1.A = {X, DT_F32, false, cc, r * cc, 0};
+    g1.B = {X, DT_F32, false, cc, r * cc, 0};
+    g1.C = {w.Ag, DT_F32, r, r * r, 0};
+    TTT_TRY(run_simt("ns_gram", g1, s));
+    GemmProblem g2;  // P = c A A + b A
+    g2.M = (int)r; g2.N = (int)r; g2.K = (int)r; g2.Z0 = P;
+    g2.A = {w.Ag, DT_F32, false, r, r * r, 0};
+    g2.B = {w.Ag, DT_F32, true, r, r * r, 0};
+    g2.C = {w.Pm, DT_F32, r, r * r, 0};
+    g2.alpha = c3; g2.beta = b3; g2.Cin = {w.Ag, r, r * r, 0};
+    TTT_TRY(run_simt("ns_poly", g2, s));
+    GemmProblem g3;  // X' = P X + a X
+    g3.M = (int)r; g3.N = (int)cc; g3.K = (int)r; g3.Z0 = P;
+    g3.A = {w.Pm, DT_F32, false, r, r * r, 0};
+    g3.B = {X, DT_F32, true, cc, r * cc, 0};
+    g3.C = {X2, DT_F32, cc, r * cc, 0};
+    g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, cc, r * cc, 0};
+    TTT_TRY(run_simt("ns_apply", g3, s));
+    float* t = X; X = X2; X2 = t;
+  }
+  TTT_OP("ns_writeback", ns_writeback(X, U, Z, L, s));
+  return TTT_OK;
+}
+
+// ------------------------------------------------------------------ momentum + Newton-Schulz
+// The parallel form with W1's momentum and orthogonalisation (simplification variant 2).
+// With W0, W2 frozen the W1 gradient of chunk c, g_c = -phi(K_c)^T diag(eta_c) V_c, does not
+// depend on W1, so for all chunks at once: D_c = sign * phi(K_c)^T diag(eta_c) V_c, the
+// momentum scan M_c = alpha_c M_{c-1} + D_c, U_c = NS(M_c) (NS is odd, so the sign and the
+// minus of the gradient pass through it), and S_c = W1 + sum_{c' <= c} U_c'.
+struct MomBufs {
+  ParBufs p;
+  NsScratch ns;
+};
+
+size_t plan_momentum(const ttt_desc& d, void* base, MomBufs& b) {
+  const size_t off = (plan_parallel(d, base, b.p) + 255) & ~static_cast<size_t>(255);
+  Carve cv(base ? static_cast<char*>(base) + off : nullptr);
+  const long long Z = (long long)d.B * d.H * ((d.N + d.chunk - 1) / d.chunk);
+  const long long hm = (long long)d.h * d.m, r = d.h < d.m ? d.h : d.m;
+  if (d.ns_steps > 0 && !(d.dtype == TTT_DTYPE_BF16 && ns_mma_supported(d.m, d.h))) {
+    b.ns.X = cv.take_n<float>(Z * hm);
+    b.ns.X2 = cv.take_n<float>(Z * hm);
+    b.ns.Ag = cv.take_n<float>(Z * r * r);
+    b.ns.Pm = cv.take_n<float>(Z * r * r);
+  } else {
+    b.ns = NsScratch{nullptr, nullptr, nullptr, nullptr};
+  }
+  return off + cv.off;
+}
+
+ttt_status momentum_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
+                         const float* eta, const float* alpha, const float* W0, const float* W2,
+                         const float* W1, void* out, float* S_final, const MomBufs& mb,
+                         cudaStream_t s) {
+  const ParBufs& b = mb.p;
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
+  const bool shared_qk = (q == k);
+  TTT_OP("prep_weights",
+         prep_wk_blocked(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
+  TTT_TRY(run_swiglu("gemm_features_k",
+                     features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
+                     s));
+  TTT_TRY(state_deltas(d, b.phiA, v, b.dS, s));
+  if (d.momentum)
+    TTT_OP("momentum_scan", momentum_scan(b.dS, alpha, (int)BH, (int)C, (long long)d.h * d.m, s));
+  if (d.ns_steps > 0)
+    TTT_TRY(run_ns(ot, b.dS, (int)(BH * C), ns_layout_single(d.m, d.h), d.ns_steps, mb.ns, s));
+  TTT_TRY(chunk_states(d, b.dS, W1, S_final, b.Sc, s));
+  if (!shared_qk && !force_simt() && !getenv("TTT_NO_FUSED_APPLY") &&
+      fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
+    TraceScope ts("fused_apply@tcgen05", s);
+    return fused_apply(q, b.Wk, b.Sc, out, d.B, d.H, d.N, d.h, d.m, d.chunk,
+                       device_error_word(), wait_limit_ns(), s);
+  }
+  if (!shared_qk)
+    TTT_TRY(run_swiglu("gemm_features_q",
+                       features_problem(d, q, b.Wk, b.phiB, nullptr, nullptr), s));
+  return chunk_outputs(d, b.phiB, b.Sc, out, s);
+}
+
+// ------------------------------------------------------------------ recurrent form
 struct RecBufs {
   float* W_all;   // fp32 masters [BH][W0 | W1 | W2]
   float* M_all;   // momentum, same layout
@@ -523,40 +651,9 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
   }
   TTT_OP("reduce_momentum", rec_reduce(b.partials, sp, b.U, d.momentum ? b.M_all : nullptr,
                                       alpha, (int)C, c, (int)BH, d.h, d.m, mask, s));
-  if (d.ns_steps > 0 && ns_on_tensor_cores(d)) {
-    TTT_OP("ns_mma", ns_mma(b.U, (int)BH, d.h, d.m, mask, d.ns_steps, 1e-7f, 3.4445f,
-                            -4.7750f, 2.0315f, device_error_word(), wait_limit_ns(), s));
-  } else if (d.ns_steps > 0) {
-    const float a3 = 3.4445f, b3 = -4.7750f, c3 = 2.0315f;
-    const long long r = h < m ? h : m, cc = h < m ? m : h;
-    TTT_OP("ns_normalize", ns_normalize(b.U, b.X, (int)BH, d.h, d.m, mask, 1e-7f, s));
-    float* X = b.X;
-    float* X2 = b.X2;
-    for (int it = 0; it < d.ns_steps; ++it) {
-      GemmProblem g1;  // A = X X^T
-      g1.M = (int)r; g1.N = (int)r; g1.K = (int)cc; g1.Z0 = (int)(3 * BH);
-      g1.A = {X, DT_F32, false, cc, r * cc, 0};
-      g1.B = {X, DT_F32, false, cc, r * cc, 0};
-      g1.C = {b.Ag, DT_F32, r, r * r, 0};
-      TTT_TRY(run_simt("ns_gram", g1, s));
-      GemmProblem g2;  // P = c A A + b A
-      g2.M = (int)r; g2.N = (int)r; g2.K = (int)r; g2.Z0 = (int)(3 * BH);
-      g2.A = {b.Ag, DT_F32, false, r, r * r, 0};
-      g2.B = {b.Ag, DT_F32, true, r, r * r, 0};
-      g2.C = {b.Pm, DT_F32, r, r * r, 0};
-      g2.alpha = c3; g2.beta = b3; g2.Cin = {b.Ag, r, r * r, 0};
-      TTT_TRY(run_simt("ns_poly", g2, s));
-      GemmProblem g3;  // X' = P X + a X
-      g3.M = (int)r; g3.N = (int)cc; g3.K = (int)r; g3.Z0 = (int)(3 * BH);
-      g3.A = {b.Pm, DT_F32, false, r, r * r, 0};
-      g3.B = {X, DT_F32, true, cc, r * cc, 0};
-      g3.C = {X2, DT_F32, cc, r * cc, 0};
-      g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, cc, r * cc, 0};
-      TTT_TRY(run_simt("ns_apply", g3, s));
-      float* t = X; X = X2; X2 = t;
-    }
-    TTT_OP("ns_writeback", ns_writeback(X, b.U, (int)BH, d.h, d.m, mask, s));
-  }
+  if (d.ns_steps > 0)
+    TTT_TRY(run_ns(ot, b.U, (int)BH, ns_layout_weights(d.h, d.m, mask), d.ns_steps,
+                   NsScratch{b.X, b.X2, b.Ag, b.Pm}, s));
   TTT_OP("step_renorm", rec_step(b.W_all, b.U, b.tnorm, (int)BH, d.H, d.h, d.m, mask, d.sign,
                                   d.renorm, b.Wk, b.W1o, ot, s));
   return TTT_OK;
@@ -588,6 +685,10 @@ size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path) {
   if (path == TTT_PATH_LINEAR) {
     LinBufs b;
     return plan_linear(*desc, nullptr, b);
+  }
+  if (path == TTT_PATH_PARALLEL_MOMENTUM) {
+    MomBufs b;
+    return plan_momentum(*desc, nullptr, b);
   }
   RecBufs b;
   return plan_recurrent(*desc, nullptr, b);
@@ -648,6 +749,38 @@ ttt_status ttt_linear_attn_fwd(const ttt_desc* desc, const void* q, const void* 
     return TTT_OK;
   }
   return linear_impl(d, q, k, v, eta, S0, out, S_final, b, s);
+}
+
+ttt_status ttt_la_parallel_momentum_fwd(const ttt_desc* desc, const void* q, const void* k,
+                                        const void* v, const float* eta, const float* alpha,
+                                        const float* W0, const float* W2, const float* W1,
+                                        void* out, float* S_final, void* workspace,
+                                        size_t workspace_bytes, ttt_stream_t stream) {
+  TTT_TRY(check_desc(desc, TTT_PATH_PARALLEL_MOMENTUM));
+  const ttt_desc& d = *desc;
+  const long long BH = (long long)d.B * d.H;
+  if (BH == 0) return TTT_OK;
+  if (!W0 || !W2 || !W1) return fail(TTT_ERR_INVALID_ARG, "W0, W2 and W1 must not be NULL");
+  if (d.momentum && d.N > 0 && !alpha)
+    return fail(TTT_ERR_INVALID_ARG, "momentum needs alpha");
+  if (d.N > 0) {
+    if (!q || !k || !v || !eta || !out)
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v, eta and out must not be NULL");
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(out) || !al16(W0) || !al16(W2) || !al16(W1))
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v, out and the weights must be 16-byte aligned");
+  }
+  MomBufs b;
+  const size_t need = plan_momentum(d, nullptr, b);
+  TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  plan_momentum(d, workspace, b);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d.N == 0) {
+    if (S_final)
+      TTT_OP("chunk_scan", chunk_scan(DT_F32, b.p.dS, W1, b.p.Sc, S_final, (int)BH, d.H, 0, d.m,
+                                      d.h, d.order, d.w1_layout, s));
+    return TTT_OK;
+  }
+  return momentum_impl(d, q, k, v, eta, alpha, W0, W2, W1, out, S_final, b, s);
 }
 
 ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const void* k,

@@ -70,6 +70,29 @@ def la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk, *, order="update_apply", si
     return out, S
 
 
+def la_parallel_momentum_fwd(q, k, v, eta, W0, W2, W1, chunk, *, order="update_apply", sign=1,
+                             alpha=None, ns_steps=0, w_in_layout=0, return_state=True,
+                             out=None, ws=None, stream=None):
+    """Parallel form with W1 momentum (when ``alpha`` [B,H,C] is given) and Newton-Schulz.
+    Returns (out [B,H,N,h], final state [B,H,m,h] or None)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    _need(eta, "eta", torch.float32)
+    _need(alpha, "alpha", torch.float32)
+    desc = parallel_desc(q, W1, chunk, order, sign, w_in_layout, 0)
+    desc.momentum = int(alpha is not None)
+    desc.ns_steps = ns_steps
+    B, H, N, h = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    S = torch.empty((B, H, desc.m, h), dtype=torch.float32, device=q.device) if return_state else None
+    if ws is None:
+        ws = workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_PARALLEL_MOMENTUM), q.device)
+    abi.ttt_la_parallel_momentum_fwd(desc, q, k, v, eta, alpha, W0, W2, W1, out, S, ws,
+                                     stream=stream)
+    return out, S
+
+
 def linear_attn_fwd(q, k, v, eta, S0, chunk, *, order="update_apply", sign=1, s_layout=0,
                     return_state=True, out=None, ws=None, stream=None):
     """Parallel form with identity features (plain chunked linear attention with per-token

@@ -135,6 +135,24 @@ def test_linear_attention_workspace_and_checks():
                             None, 0, stream=0)
 
 
+def test_parallel_momentum_workspace_and_checks():
+    P = abi.TTT_PATH_PARALLEL_MOMENTUM
+    plain = abi.ttt_workspace_bytes(lm_desc(), abi.TTT_PATH_PARALLEL)
+    assert abi.ttt_workspace_bytes(lm_desc(momentum=1), P) >= plain
+    # min(h, m) = 256 > 128: the CUDA-core Newton-Schulz needs its scratch
+    assert abi.ttt_workspace_bytes(lm_desc(momentum=1, ns_steps=5), P) > plain
+    # an NVS-shaped state fits the tensor-core Newton-Schulz: no extra scratch
+    small = dict(h=128, m=256)
+    assert (abi.ttt_workspace_bytes(lm_desc(ns_steps=5, **small), P) ==
+            abi.ttt_workspace_bytes(lm_desc(**small), P))
+    for bad in (dict(renorm=1), dict(update_mask=2), dict(ns_steps=9), dict(w1_layout=1)):
+        assert abi.ttt_workspace_bytes(lm_desc(**bad), P) == 0
+    with pytest.raises(abi.TTTError) as ei:   # momentum without alpha
+        abi.ttt_la_parallel_momentum_fwd(lm_desc(momentum=1), 256, 256, 256, 256, None, 256,
+                                         256, 256, 256, None, 256, 1 << 40, stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+
+
 def test_recurrent_rejects_bad_args():
     d = lm_desc(update_mask=7, momentum=1)
     need = abi.ttt_workspace_bytes(d, 1)

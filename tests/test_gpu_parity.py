@@ -198,6 +198,48 @@ def test_linear_attention_matches_oracle(case, order):
     assert rel(host(out0), ref0) <= TOL[dtype]
 
 
+# ----------------------------------------------------------------------------- momentum + NS
+MOM_CASES = [
+    # kind, dtype, B, H, N, h, m, chunk, momentum, ns_steps
+    ("tiny", "fp32", 1, 2, 200, 16, 24, 48, True, 5),      # CUDA-core Newton-Schulz
+    ("lm", "bf16", 2, 1, 1000, 128, 256, 256, True, 5),    # tensor-core Newton-Schulz
+    ("lm", "bf16", 1, 2, 640, 64, 192, 128, False, 5),
+    ("lm", "bf16", 1, 2, 640, 64, 192, 128, True, 0),
+    ("lm", "bf16", 1, 1, 512, 256, 136, 128, True, 3),     # bf16, min(h, m) > 128: CUDA cores
+]
+
+
+@pytest.mark.parametrize("case", MOM_CASES, ids=lambda c: "-".join(map(str, c[:10])))
+@pytest.mark.parametrize("order", ["update_apply", "apply_update"])
+def test_parallel_momentum_matches_recurrent_oracle(case, order):
+    """The parallel form with W1 momentum and Newton-Schulz equals the recurrent form with
+    only W1 fast, the same momentum and steps and no renormalisation (oracle)."""
+    kind, dtype, B, H, N, h, m, chunk, momentum, ns = case
+    wl, inp = layer_inputs(kind, dtype, B, H, N, h, m, chunk, seed=4000 + N + h, momentum=True)
+    ref, Wref, _ = O.lact_recurrent_batched(
+        inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"], inp["W2"], inp["W1"], chunk,
+        order=ORD[order], update=("W1",), alpha=inp["alpha"] if momentum else None,
+        ns_steps=ns)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, dtype)
+    alpha = dev(inp["alpha"]) if momentum else None
+    out, S = layer.la_parallel_momentum_fwd(q, k, v, eta, W0, W2, W1, chunk, order=order,
+                                            alpha=alpha, ns_steps=ns)
+    abi.ttt_last_device_status()
+    tol = TOL[dtype]
+    assert rel(host(out), ref) <= tol
+    assert rel(host(S), Wref["W1"]) <= tol
+    init = inp["W1"][None].repeat(B, axis=0)
+    assert rel(host(S) - init, Wref["W1"] - init) <= 5 * tol
+
+
+def test_parallel_momentum_without_options_is_the_parallel_form():
+    wl, inp = layer_inputs("lm", "bf16", 1, 2, 512, 64, 128, 128, seed=41)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    a, Sa = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, 128)
+    b, Sb = layer.la_parallel_momentum_fwd(q, k, v, eta, W0, W2, W1, 128)
+    assert torch.equal(a, b) and torch.equal(Sa, Sb)
+
+
 # ----------------------------------------------------------------------------- recurrent
 REC_CASES = [
     # kind, dtype, B, H, N, h, m, chunk, opts
