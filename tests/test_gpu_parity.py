@@ -240,6 +240,52 @@ def test_parallel_momentum_without_options_is_the_parallel_form():
     assert torch.equal(a, b) and torch.equal(Sa, Sb)
 
 
+# ----------------------------------------------------------------------------- context parallel
+def test_sequence_shards_through_the_library_equal_one_call():
+    """The context-parallel decomposition on one device: shard totals from a zero state,
+    prefix, then each shard from W1 + prefix (what the ranks of la_parallel_fwd_cp do)."""
+    wl, inp = layer_inputs("lm", "bf16", 2, 2, 1024, 128, 256, 128, seed=61)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    full, Sfull = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, 128)
+    shards = [slice(0, 384), slice(384, 768), slice(768, 1024)]
+    prefix = torch.zeros((2, 2, 256, 128), dtype=torch.float32, device="cuda")
+    outs = []
+    for sl in shards:
+        args = [t[:, :, sl].contiguous() for t in (q, k, v, eta)]
+        _, total = layer.la_parallel_fwd(*args, W0, W2, torch.zeros_like(W1), 128)
+        o = []
+        for b in range(2):
+            ob, Sb = layer.la_parallel_fwd(*(a[b:b + 1].contiguous() for a in args), W0, W2,
+                                           (W1 + prefix[b]).contiguous(), 128)
+            o.append(ob)
+        outs.append(torch.cat(o, 0))
+        prefix = prefix + total
+    abi.ttt_last_device_status()
+    assert rel(host(torch.cat(outs, 2)), host(full)) <= 1e-2
+    assert rel(host(prefix + W1[None]), host(Sfull)) <= 1e-5
+
+
+def test_context_parallel_single_rank_nccl():
+    import datetime
+    import socket
+    import torch.distributed as dist
+    from test_weight_layers_ttt_b200.context_parallel import la_parallel_fwd_cp
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=30))
+    dist.init_process_group("nccl", rank=0, world_size=1, store=store,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        wl, inp = layer_inputs("lm", "bf16", 1, 2, 512, 128, 256, 128, seed=62)
+        q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+        out, S = la_parallel_fwd_cp(q, k, v, eta, W0, W2, W1, 128)
+        ref, Sref = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, 128)
+        assert rel(host(out), host(ref)) <= 1e-2 and rel(host(S), host(Sref)) <= 1e-5
+    finally:
+        dist.destroy_process_group()
+
+
 # ----------------------------------------------------------------------------- recurrent
 REC_CASES = [
     # kind, dtype, B, H, N, h, m, chunk, opts
