@@ -258,44 +258,123 @@ __global__ void rec_reduce_kernel(const float* partials, int splits, float* U, f
 
 // One block per (part, bh): Frobenius norm, then the normalised update in the orientation
 // with rows <= cols.
-__global__ void ns_normalize_kernel(const float* U, float* X, NsLayout L, float eps) {
+// ||U||_F of every (part, entry) problem: grid (parts, Z, NS_SLABS) blocks of 256 threads,
+// each adding its slab's sum of squares into nrm[z * parts + p] (zeroed first).
+constexpr int NS_SLABS = 16;
+
+__global__ void ns_sumsq_kernel(const float* U, NsLayout L, float* nrm) {
   const int p = blockIdx.x, z = blockIdx.y;
   if (!(L.mask & (1 << p))) return;
-  const int R = L.R[p], Cc = L.C[p];
-  const long long n = (long long)R * Cc;
+  const long long n = (long long)L.R[p] * L.C[p];
   const float* u = U + z * L.zstride + p * L.pstride;
-  float* x = X + ((long long)z * L.parts + p) * n;
-  __shared__ float red[32];
+  __shared__ float red[8];
   float ss = 0.0f;
-  for (long long e = threadIdx.x; e < n; e += blockDim.x) ss += u[e] * u[e];
+  for (long long e = blockIdx.z * 256LL + threadIdx.x; e < n; e += 256LL * NS_SLABS)
+    ss = fmaf(u[e], u[e], ss);
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (threadIdx.x == 0) red[0] = v;
-  }
-  __syncthreads();
-  const float scale = 1.0f / (sqrtf(red[0]) + eps);
-  const bool tr = R > Cc;
-  for (long long e = threadIdx.x; e < n; e += blockDim.x) {
-    const int i = (int)(e / Cc), j = (int)(e - (long long)i * Cc);
-    x[tr ? (long long)j * R + i : e] = u[e] * scale;
+  if (threadIdx.x == 0) {
+    float t = 0.0f;
+    for (int w = 0; w < 8; ++w) t += red[w];
+    atomicAdd(&nrm[(long long)z * L.parts + p], t);
   }
 }
 
-__global__ void ns_writeback_kernel(const float* X, float* U, NsLayout L) {
-  const int p = blockIdx.x, z = blockIdx.y;
+// X (wide orientation) = U * scale, or U <- X back (to_u): 32 x 32 tiles through shared
+// memory so both sides are read and written along rows. grid (tiles of the problem,
+// parts, Z), block (32, 8).
+__global__ void ns_copy_kernel(const float* U_in, float* X, float* U_out, NsLayout L,
+                               const float* nrm, float eps, int to_u) {
+  const int p = blockIdx.y, z = blockIdx.z;
   if (!(L.mask & (1 << p))) return;
   const int R = L.R[p], Cc = L.C[p];
+  const int tc = (Cc + 31) / 32, tr_ = (R + 31) / 32;
+  if ((int)blockIdx.x >= tc * tr_) return;
+  const int i0 = (blockIdx.x / tc) * 32, j0 = (blockIdx.x % tc) * 32;   // tile of U [R, Cc]
   const long long n = (long long)R * Cc;
-  float* u = U + z * L.zstride + p * L.pstride;
-  const float* x = X + ((long long)z * L.parts + p) * n;
+  const long long uoff = z * L.zstride + p * L.pstride;
+  float* x = X + ((long long)z * L.parts + p) * n;
   const bool tr = R > Cc;
-  for (long long e = threadIdx.x; e < n; e += blockDim.x) {
-    const int i = (int)(e / Cc), j = (int)(e - (long long)i * Cc);
-    u[e] = x[tr ? (long long)j * R + i : e];
+  __shared__ float t[32][33];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  if (!to_u) {
+    const float scale = 1.0f / (sqrtf(nrm[(long long)z * L.parts + p]) + eps);
+    const float* u = U_in + uoff;
+    for (int k = ty; k < 32; k += 8) {
+      const int i = i0 + k, j = j0 + tx;
+      t[k][tx] = (i < R && j < Cc) ? u[(long long)i * Cc + j] * scale : 0.0f;
+    }
+    __syncthreads();
+    for (int k = ty; k < 32; k += 8) {
+      if (!tr) {
+        const int i = i0 + k, j = j0 + tx;
+        if (i < R && j < Cc) x[(long long)i * Cc + j] = t[k][tx];
+      } else {   // x is [Cc, R]: x[j][i] = u[i][j]
+        const int j = j0 + k, i = i0 + tx;
+        if (i < R && j < Cc) x[(long long)j * R + i] = t[tx][k];
+      }
+    }
+  } else {
+    float* u = U_out + uoff;
+    for (int k = ty; k < 32; k += 8) {
+      if (!tr) {
+        const int i = i0 + k, j = j0 + tx;
+        t[k][tx] = (i < R && j < Cc) ? x[(long long)i * Cc + j] : 0.0f;
+      } else {
+        const int j = j0 + k, i = i0 + tx;
+        t[tx][k] = (i < R && j < Cc) ? x[(long long)j * R + i] : 0.0f;
+      }
+    }
+    __syncthreads();
+    for (int k = ty; k < 32; k += 8) {
+      const int i = i0 + k, j = j0 + tx;
+      if (i < R && j < Cc) u[(long long)i * Cc + j] = t[k][tx];
+    }
+  }
+}
+
+// One thread per 8 consecutive columns of a row: 16-byte loads and stores.
+__global__ void split_hilo_kernel(const float* M, long long P, int rows, int cols, uint4* hhl,
+                                  uint4* hlh, uint4* stack) {
+  const int c8 = cols / 8;
+  TTT_GRID_LOOP(idx, P * rows * c8) {
+    const long long pr = idx / c8;              // p * rows + row
+    const int q = (int)(idx - pr * c8);
+    const long long p = pr / rows;
+    const int row = (int)(pr - p * rows);
+    const float4 a = *reinterpret_cast<const float4*>(M + pr * cols + 8 * q);
+    const float4 b = *reinterpret_cast<const float4*>(M + pr * cols + 8 * q + 4);
+    const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * t], x[2 * t + 1]);
+      const float2 hf = __bfloat1622float2(h2);
+      const __nv_bfloat162 l2 = __floats2bfloat162_rn(x[2 * t] - hf.x, x[2 * t + 1] - hf.y);
+      hi[t] = *reinterpret_cast<const uint32_t*>(&h2);
+      lo[t] = *reinterpret_cast<const uint32_t*>(&l2);
+    }
+    const uint4 H = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    const uint4 Lo = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    if (hhl) {   // row pr of [rows, 3 cols]: column blocks hi | hi | lo
+      uint4* o = hhl + pr * 3 * c8 + q;
+      o[0] = H;
+      o[c8] = H;
+      o[2 * c8] = Lo;
+    }
+    if (hlh) {
+      uint4* o = hlh + pr * 3 * c8 + q;
+      o[0] = H;
+      o[c8] = Lo;
+      o[2 * c8] = H;
+    }
+    if (stack) {   // rows row, rows + row, 2 rows + row of [3 rows, cols]
+      uint4* o = stack + (p * 3 * rows + row) * c8 + q;
+      o[0] = H;
+      o[(long long)rows * c8] = Lo;
+      o[2LL * rows * c8] = H;
+    }
   }
 }
 
@@ -598,13 +677,37 @@ cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all
 }
 
 cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
-                         cudaStream_t s) {
-  ns_normalize_kernel<<<dim3(L.parts, Z), 256, 0, s>>>(U, X, L, eps);
+                         float* nrm, cudaStream_t s) {
+  if (Z <= 0) return cudaSuccess;
+  cudaError_t e = fill_f32(nrm, (long long)Z * L.parts, 0.0f, s);
+  if (e != cudaSuccess) return e;
+  ns_sumsq_kernel<<<dim3(L.parts, Z, NS_SLABS), 256, 0, s>>>(U, L, nrm);
+  int tiles = 0;
+  for (int p = 0; p < L.parts; ++p)
+    tiles = max(tiles, ((L.R[p] + 31) / 32) * ((L.C[p] + 31) / 32));
+  ns_copy_kernel<<<dim3(tiles, L.parts, Z), dim3(32, 8), 0, s>>>(U, X, nullptr, L, nrm, eps, 0);
   return cudaGetLastError();
 }
 
 cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cudaStream_t s) {
-  ns_writeback_kernel<<<dim3(L.parts, Z), 256, 0, s>>>(X, U, L);
+  if (Z <= 0) return cudaSuccess;
+  int tiles = 0;
+  for (int p = 0; p < L.parts; ++p)
+    tiles = max(tiles, ((L.R[p] + 31) / 32) * ((L.C[p] + 31) / 32));
+  ns_copy_kernel<<<dim3(tiles, L.parts, Z), dim3(32, 8), 0, s>>>(
+      nullptr, const_cast<float*>(X), U, L, nullptr, 0.0f, 1);
+  return cudaGetLastError();
+}
+
+cudaError_t split_hilo(const float* M, int P, int rows, int cols, void* hhl, void* hlh,
+                       void* stack, cudaStream_t s) {
+  if (P <= 0 || rows <= 0 || cols <= 0) return cudaSuccess;
+  if (cols % 8 != 0) return cudaErrorInvalidValue;
+  const long long n = (long long)P * rows * (cols / 8);
+  split_hilo_kernel<<<grid_for(n, 256), 256, 0, s>>>(M, P, rows, cols,
+                                                     static_cast<uint4*>(hhl),
+                                                     static_cast<uint4*>(hlh),
+                                                     static_cast<uint4*>(stack));
   return cudaGetLastError();
 }
 

@@ -63,9 +63,10 @@ inline NsLayout ns_layout_single(int R, int C) {
 
 // Newton-Schulz set-up / tear-down for the CUDA-core path: X = U / (||U||_F + eps) in the
 // wide orientation ([min(R,C), max(R,C)]) into the scratch X (problem (z, p) at
-// (z * parts + p) * R * C), and U <- X back in U's own orientation. Z entries.
+// (z * parts + p) * R * C), and U <- X back in U's own orientation. Z entries. nrm: fp32
+// scratch of Z * parts sums of squares.
 cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
-                         cudaStream_t s);
+                         float* nrm, cudaStream_t s);
 cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cudaStream_t s);
 
 // The whole Newton-Schulz orthogonalisation of the matrices of L on the tensor cores
@@ -76,6 +77,12 @@ cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cud
 bool ns_mma_supported(int R, int C);
 cudaError_t ns_mma(float* U, int Z, const NsLayout& L, int steps, float eps, float a, float b,
                    float c, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
+
+// Split fp32 matrices M [P, rows, cols] into bf16 hi = bf16(x), lo = bf16(x - hi) and
+// write the nullable outputs hhl = [hi|hi|lo] and hlh = [hi|lo|hi] ([P, rows, 3 cols],
+// concatenated along the columns) and stack = [hi;lo;hi] ([P, 3 rows, cols]). cols % 8 == 0.
+cudaError_t split_hilo(const float* M, int P, int rows, int cols, void* hhl, void* hlh,
+                       void* stack, cudaStream_t s);
 
 // Momentum over chunks, in place: D[bh, c] <- alpha[bh, c] * D[bh, c - 1] + D[bh, c] for
 // c = 1 .. C-1 (D [BH, C, n] fp32, alpha [BH, C]).

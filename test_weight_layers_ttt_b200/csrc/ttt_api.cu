@@ -384,16 +384,48 @@ ttt_status linear_impl(const ttt_desc& d, const void* q, const void* k, const vo
 }
 
 // ------------------------------------------------------------------ Newton-Schulz
-// bf16 mode runs Newton-Schulz on the tensor cores (split bf16 operands, close to fp32)
-// when the matrices fit one CTA; fp32 mode and larger matrices use fp32 CUDA-core products.
-bool ns_on_tensor_cores(const ttt_desc& d) {
-  return d.dtype == TTT_DTYPE_BF16 && ns_mma_supported(d.h, d.m);
+// bf16 mode runs Newton-Schulz on the tensor cores with split bf16 operands (close to
+// fp32): one CTA per matrix when it fits, else batched GEMMs; fp32 mode uses fp32
+// CUDA-core products.
+
+// Newton-Schulz scratch. CUDA-core path: X, X2 [problems, r, c], Ag, Pm [problems, r, r]
+// fp32. Split-bf16 GEMM path: the same fp32 buffers (Ag holds A = X X^T, Pm the polynomial)
+// plus the bf16 hi/lo operands concatenated along K (see run_ns): Xa = [Xh|Xh|Xl] and
+// Xb = [Xh|Xl|Xh] [problems, r, 3c], Xs = [Xh;Xl;Xh] [problems, 3r, c], Ga = [Ah|Ah|Al]
+// and Pa = [Ph|Ph|Pl] [problems, r, 3r], Gs = [Ah;Al;Ah] [problems, 3r, r].
+struct NsScratch {
+  float *X = nullptr, *X2 = nullptr, *Ag = nullptr, *Pm = nullptr, *nrm = nullptr;
+  void *Xa = nullptr, *Xb = nullptr, *Xs = nullptr, *Ga = nullptr, *Gs = nullptr, *Pa = nullptr;
+};
+
+enum NsPath { NS_TENSOR_CTA = 0, NS_TENSOR_GEMM = 1, NS_CUDA_CORES = 2 };
+
+NsPath ns_path(int ot, int R, int C) {
+  if (ot == DT_BF16 && ns_mma_supported(R, C)) return NS_TENSOR_CTA;
+  if (ot == DT_BF16) return NS_TENSOR_GEMM;
+  return NS_CUDA_CORES;
 }
 
-// Scratch of the CUDA-core Newton-Schulz: X, X2 [problems, r, c], Ag, Pm [problems, r, r].
-struct NsScratch {
-  float *X, *X2, *Ag, *Pm;
-};
+NsScratch plan_ns(Carve& cv, int ot, long long problems, int R, int C) {
+  NsScratch w;
+  const NsPath path = ns_path(ot, R, C);
+  if (path == NS_TENSOR_CTA) return w;
+  const long long r = R < C ? R : C, c = R < C ? C : R;
+  w.X = cv.take_n<float>(problems * r * c);
+  w.X2 = cv.take_n<float>(problems * r * c);
+  w.Ag = cv.take_n<float>(problems * r * r);
+  w.Pm = cv.take_n<float>(problems * r * r);
+  w.nrm = cv.take_n<float>(problems);
+  if (path == NS_TENSOR_GEMM) {
+    w.Xa = cv.take(2 * problems * r * 3 * c);
+    w.Xb = cv.take(2 * problems * r * 3 * c);
+    w.Xs = cv.take(2 * problems * 3 * r * c);
+    w.Ga = cv.take(2 * problems * r * 3 * r);
+    w.Gs = cv.take(2 * problems * 3 * r * r);
+    w.Pa = cv.take(2 * problems * r * 3 * r);
+  }
+  return w;
+}
 
 // Newton-Schulz (the pages' five-step coefficients, eps 1e-7) in place on the matrices of
 // L: tensor cores for bf16 mode when they fit one CTA, else fp32 CUDA-core products (the
@@ -409,7 +441,41 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
   }
   const long long r = R < Cc ? R : Cc, cc = R < Cc ? Cc : R;
   const int P = Z * L.parts;
-  TTT_OP("ns_normalize", ns_normalize(U, w.X, Z, L, 1e-7f, s));
+  TTT_OP("ns_normalize", ns_normalize(U, w.X, Z, L, 1e-7f, w.nrm, s));
+  if (ns_path(ot, (int)R, (int)Cc) == NS_TENSOR_GEMM) {
+    // Each product as one bf16 GEMM over K tripled: hi*hi + hi*lo + lo*hi of the split
+    // operands (x = hi + lo to about 2^-16), fp32 accumulation in TMEM.
+    float* X = w.X;
+    float* X2 = w.X2;
+    for (int it = 0; it < steps; ++it) {
+      TTT_OP("ns_split", split_hilo(X, P, (int)r, (int)cc, w.Xa, w.Xb, w.Xs, s));
+      GemmProblem g1;  // A = X X^T
+      g1.M = (int)r; g1.N = (int)r; g1.K = (int)(3 * cc); g1.Z0 = P;
+      g1.A = {w.Xa, DT_BF16, false, 3 * cc, 3 * r * cc, 0};
+      g1.B = {w.Xb, DT_BF16, false, 3 * cc, 3 * r * cc, 0};
+      g1.C = {w.Ag, DT_F32, r, r * r, 0};
+      TTT_TRY(run_gemm("ns_gram", g1, s));
+      TTT_OP("ns_split", split_hilo(w.Ag, P, (int)r, (int)r, w.Ga, nullptr, w.Gs, s));
+      GemmProblem g2;  // P = c A A + b A
+      g2.M = (int)r; g2.N = (int)r; g2.K = (int)(3 * r); g2.Z0 = P;
+      g2.A = {w.Ga, DT_BF16, false, 3 * r, 3 * r * r, 0};
+      g2.B = {w.Gs, DT_BF16, true, r, 3 * r * r, 0};
+      g2.C = {w.Pm, DT_F32, r, r * r, 0};
+      g2.alpha = c3; g2.beta = b3; g2.Cin = {w.Ag, r, r * r, 0};
+      TTT_TRY(run_gemm("ns_poly", g2, s));
+      TTT_OP("ns_split", split_hilo(w.Pm, P, (int)r, (int)r, w.Pa, nullptr, nullptr, s));
+      GemmProblem g3;  // X' = P X + a X
+      g3.M = (int)r; g3.N = (int)cc; g3.K = (int)(3 * r); g3.Z0 = P;
+      g3.A = {w.Pa, DT_BF16, false, 3 * r, 3 * r * r, 0};
+      g3.B = {w.Xs, DT_BF16, true, cc, 3 * r * cc, 0};
+      g3.C = {X2, DT_F32, cc, r * cc, 0};
+      g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, cc, r * cc, 0};
+      TTT_TRY(run_gemm("ns_apply", g3, s));
+      float* t = X; X = X2; X2 = t;
+    }
+    TTT_OP("ns_writeback", ns_writeback(X, U, Z, L, s));
+    return TTT_OK;
+  }
   float* X = w.X;
   float* X2 = w.X2;
   for (int it = 0; it < steps; ++it) {
@@ -454,15 +520,8 @@ size_t plan_momentum(const ttt_desc& d, void* base, MomBufs& b) {
   const size_t off = (plan_parallel(d, base, b.p) + 255) & ~static_cast<size_t>(255);
   Carve cv(base ? static_cast<char*>(base) + off : nullptr);
   const long long Z = (long long)d.B * d.H * ((d.N + d.chunk - 1) / d.chunk);
-  const long long hm = (long long)d.h * d.m, r = d.h < d.m ? d.h : d.m;
-  if (d.ns_steps > 0 && !(d.dtype == TTT_DTYPE_BF16 && ns_mma_supported(d.m, d.h))) {
-    b.ns.X = cv.take_n<float>(Z * hm);
-    b.ns.X2 = cv.take_n<float>(Z * hm);
-    b.ns.Ag = cv.take_n<float>(Z * r * r);
-    b.ns.Pm = cv.take_n<float>(Z * r * r);
-  } else {
-    b.ns = NsScratch{nullptr, nullptr, nullptr, nullptr};
-  }
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  b.ns = d.ns_steps > 0 ? plan_ns(cv, ot, Z, d.m, d.h) : NsScratch{};
   return off + cv.off;
 }
 
@@ -511,10 +570,7 @@ struct RecBufs {
   void* E0;       // [BH, chunk, m] d * B * silu'(A)
   float* partials;
   void* phiQ;     // [BH, chunk, m]
-  float* X;
-  float* X2;
-  float* Ag;
-  float* Pm;
+  NsScratch ns;   // Newton-Schulz scratch for the 3 matrices of every (b, head)
   int splits;
 };
 
@@ -551,15 +607,9 @@ size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
   b.E0 = cv.take(os * rows * d.m);
   b.partials = cv.take_n<float>((long long)b.splits * BH * 3 * hm);
   b.phiQ = cv.take(os * rows * d.m);
-  if (d.ns_steps > 0 && !ns_on_tensor_cores(d)) {
-    const long long r = d.h < d.m ? d.h : d.m;
-    b.X = cv.take_n<float>(BH * 3 * hm);
-    b.X2 = cv.take_n<float>(BH * 3 * hm);
-    b.Ag = cv.take_n<float>(BH * 3 * r * r);
-    b.Pm = cv.take_n<float>(BH * 3 * r * r);
-  } else {
-    b.X = b.X2 = b.Ag = b.Pm = nullptr;
-  }
+  b.ns = d.ns_steps > 0 ? plan_ns(cv, d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32, BH * 3,
+                                   d.h, d.m)
+                        : NsScratch{};
   return cv.off;
 }
 
@@ -653,7 +703,7 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
                                       alpha, (int)C, c, (int)BH, d.h, d.m, mask, s));
   if (d.ns_steps > 0)
     TTT_TRY(run_ns(ot, b.U, (int)BH, ns_layout_weights(d.h, d.m, mask), d.ns_steps,
-                   NsScratch{b.X, b.X2, b.Ag, b.Pm}, s));
+                   b.ns, s));
   TTT_OP("step_renorm", rec_step(b.W_all, b.U, b.tnorm, (int)BH, d.H, d.h, d.m, mask, d.sign,
                                   d.renorm, b.Wk, b.W1o, ot, s));
   return TTT_OK;
