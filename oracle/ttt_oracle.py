@@ -239,6 +239,63 @@ def la_parallel(q, k, v, eta, W0, W2, W1, chunk, *, order=UPDATE_APPLY, sign=1):
     return chunked_linear_attention(phiQ, phiK, v, eta, W1, chunk, order, sign)
 
 
+def la_parallel_backward(q, k, v, eta, W0, W2, W1, dO, chunk, *, order=UPDATE_APPLY, sign=1,
+                         dS_final=None):
+    """Gradients of the parallel form's outputs (and of its final state, when dS_final is
+    given) for one (batch, head): the chain rule through O_c = phi(Q_c) S_c, the prefix sum
+    S_c = W1 + sum ΔS_c' and ΔS_c = sign phi(K_c)^T diag(eta_c) V_c (TTT≡LA notes,
+    方法步骤详情), then through phi = silu(X W0) * (X W2). Returns dq, dk, dv, deta, dW0, dW2,
+    dW1 in the shapes of the inputs.
+
+    With R_c = dS_final + sum_{c' >= c} phi(Q_c')^T dO_c' (suffix sum), the gradient of
+    ΔS_c is G_c = R_c (update_apply: chunk c's own delta reaches its own outputs) or R_{c+1}
+    (apply_update), and dW1 = R_0."""
+    q, k, v, eta, dO = _f64(q), _f64(k), _f64(v), _f64(eta), _f64(dO)
+    W0, W2, W1 = _f64(W0), _f64(W2), _f64(W1)
+    N = len(q)
+    Aq, Bq, Ak, Bk = q @ W0, q @ W2, k @ W0, k @ W2
+    phiQ, phiK = silu(Aq) * Bq, silu(Ak) * Bk
+    sl = chunk_slices(N, chunk)
+    dS = [sign * (phiK[c].T @ (eta[c, None] * v[c])) for c in sl]
+    # the state each chunk reads
+    S, Sc = W1.copy(), []
+    for d in dS:
+        if order == APPLY_UPDATE:
+            Sc.append(S.copy())
+            S = S + d
+        else:
+            S = S + d
+            Sc.append(S.copy())
+    R = np.zeros_like(W1) if dS_final is None else _f64(dS_final).copy()
+    Rs = [None] * (len(sl) + 1)
+    Rs[len(sl)] = R.copy()
+    for ci in range(len(sl) - 1, -1, -1):
+        R = R + phiQ[sl[ci]].T @ dO[sl[ci]]
+        Rs[ci] = R.copy()
+    dphiQ = np.empty_like(phiQ)
+    dphiK = np.empty_like(phiK)
+    dv = np.empty_like(v)
+    deta = np.empty_like(eta)
+    for ci, c in enumerate(sl):
+        G = Rs[ci] if order == UPDATE_APPLY else Rs[ci + 1]
+        dphiQ[c] = dO[c] @ Sc[ci].T
+        T = phiK[c] @ G                              # [L, h]
+        dv[c] = sign * eta[c, None] * T
+        deta[c] = sign * np.sum(T * v[c], axis=1)
+        dphiK[c] = sign * eta[c, None] * (v[c] @ G.T)
+    out = {"dW1": Rs[0]}
+    dW0 = np.zeros_like(W0)
+    dW2 = np.zeros_like(W2)
+    for X, A, B, dphi, name in ((q, Aq, Bq, dphiQ, "dq"), (k, Ak, Bk, dphiK, "dk")):
+        dA = dphi * B * silu_prime(A)
+        dB = dphi * silu(A)
+        out[name] = dA @ W0.T + dB @ W2.T
+        dW0 += X.T @ dA
+        dW2 += X.T @ dB
+    out.update(dv=dv, deta=deta, dW0=dW0, dW2=dW2)
+    return out
+
+
 def la_parallel_rows(q, k, v, eta, W0, W2, W1, chunk, rows, *, order=UPDATE_APPLY, sign=1):
     """Outputs of the parallel form at the given token rows only, plus the final state.
     Every chunk state up to the last needed chunk is formed in full; only the query side

@@ -353,3 +353,56 @@ def test_lm_target_conv_brute_force_and_shift():
     ident = np.zeros((4, d))
     ident[0] = 1.0
     assert np.array_equal(O.lm_target(X0, ident, np.eye(d)), X0)
+
+
+# ----------------------------------------------------------------------------- backward
+@pytest.mark.parametrize("order", [O.UPDATE_APPLY, O.APPLY_UPDATE])
+@pytest.mark.parametrize("sign", [1, -1])
+def test_parallel_backward_matches_finite_differences(order, sign):
+    """Every gradient of the parallel form against central differences of the forward
+    oracle (fp64) on a tiny ragged problem, through a random linear functional of the
+    outputs and of the final state."""
+    rng = np.random.default_rng(17)
+    N, h, m, chunk = 11, 3, 4, 4
+    x = dict(q=rng.standard_normal((N, h)), k=rng.standard_normal((N, h)),
+             v=rng.standard_normal((N, h)), eta=rng.uniform(0.1, 0.9, N),
+             W0=rng.standard_normal((h, m)) * 0.5, W2=rng.standard_normal((h, m)) * 0.5,
+             W1=rng.standard_normal((m, h)) * 0.5)
+    dO = rng.standard_normal((N, h))
+    dSf = rng.standard_normal((m, h))
+
+    def loss(**kw):
+        a = dict(x)
+        a.update(kw)
+        O_, S_ = O.la_parallel(a["q"], a["k"], a["v"], a["eta"], a["W0"], a["W2"], a["W1"],
+                               chunk, order=order, sign=sign)
+        return float(np.sum(O_ * dO) + np.sum(S_ * dSf))
+
+    g = O.la_parallel_backward(x["q"], x["k"], x["v"], x["eta"], x["W0"], x["W2"], x["W1"], dO,
+                               chunk, order=order, sign=sign, dS_final=dSf)
+    eps = 1e-6
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("eta", "deta"), ("W0", "dW0"),
+                      ("W2", "dW2"), ("W1", "dW1")):
+        base = x[name]
+        num = np.empty_like(base)
+        for idx in np.ndindex(base.shape):
+            up, dn = base.copy(), base.copy()
+            up[idx] += eps
+            dn[idx] -= eps
+            num[idx] = (loss(**{name: up}) - loss(**{name: dn})) / (2 * eps)
+        assert np.allclose(g[key], num, rtol=1e-6, atol=1e-7), key
+
+
+def test_parallel_backward_w1_gradient_is_the_output_functional():
+    """The outputs are linear in W1 with every state containing it once: dW1 is the sum over
+    chunks of phi(Q_c)^T dO_c (plus the final-state cotangent), in both orders."""
+    rng = np.random.default_rng(3)
+    N, h, m, chunk = 9, 2, 3, 3
+    q, k, v = (rng.standard_normal((N, h)) for _ in range(3))
+    eta = np.full(N, 0.5)
+    W0, W2, W1 = rng.standard_normal((h, m)), rng.standard_normal((h, m)), rng.standard_normal((m, h))
+    dO = rng.standard_normal((N, h))
+    phiQ = O.swiglu_features(q, W0, W2)
+    for order in (O.UPDATE_APPLY, O.APPLY_UPDATE):
+        g = O.la_parallel_backward(q, k, v, eta, W0, W2, W1, dO, chunk, order=order)
+        assert np.allclose(g["dW1"], phiQ.T @ dO, rtol=1e-12, atol=1e-12)
