@@ -73,7 +73,8 @@ enum {
   TTT_PATH_PARALLEL = 0,
   TTT_PATH_RECURRENT = 1,
   TTT_PATH_LINEAR = 2,
-  TTT_PATH_PARALLEL_MOMENTUM = 3
+  TTT_PATH_PARALLEL_MOMENTUM = 3,
+  TTT_PATH_PARALLEL_BWD = 4
 };
 
 /* Problem description. All fields are read; unused ones must be 0 unless noted. */
@@ -154,6 +155,33 @@ ttt_status ttt_la_parallel_momentum_fwd(const ttt_desc* desc, const void* q, con
                                         const float* W0, const float* W2, const float* W1,
                                         void* out, float* S_final, void* workspace,
                                         size_t workspace_bytes, ttt_stream_t stream);
+
+/*
+ * Backward pass of ttt_la_parallel_fwd (training; "Test-Time Training with KV Binding Is
+ * Secretly Linear Attention", section 方法步骤详情: the parallel form is what makes the
+ * layer trainable at scale). Given the gradient dout of the outputs (and optionally
+ * dS_final of the final state), computes the gradients of every input by the chain rule
+ * through O_c = phi(Q_c) S_c, S_c = W1 + sum Delta S_c' and Delta S_c = sign phi(K_c)^T
+ * diag(eta_c) V_c. With R_c = dS_final + sum_{c' >= c} phi(Q_c')^T dO_c', the gradient of
+ * Delta S_c is R_c (update_apply) or R_{c+1} (apply_update) and dW1 = R_0. The forward
+ * quantities are recomputed, nothing is saved between the calls.
+ *
+ *   desc        as for ttt_la_parallel_fwd; default weight layouts only
+ *   q, k, v, eta, W0, W2, W1   the forward inputs (q and k distinct)
+ *   dout        [B,H,N,h] dtype
+ *   dS_final    nullable; [B,H,m,h] fp32
+ *   dq, dk, dv  [B,H,N,h] dtype, written (distinct buffers)
+ *   deta        [B,H,N] fp32, written
+ *   dW0, dW2    [H,h,m] fp32, dW1 [H,m,h] fp32, written (summed over the batch)
+ *   workspace   >= ttt_workspace_bytes(desc, TTT_PATH_PARALLEL_BWD) bytes, 256-byte aligned
+ * Errors and streams as for ttt_la_parallel_fwd.
+ */
+ttt_status ttt_la_parallel_bwd(const ttt_desc* desc, const void* q, const void* k,
+                               const void* v, const float* eta, const float* W0,
+                               const float* W2, const float* W1, const void* dout,
+                               const float* dS_final, void* dq, void* dk, void* dv,
+                               float* deta, float* dW0, float* dW2, float* dW1,
+                               void* workspace, size_t workspace_bytes, ttt_stream_t stream);
 
 /*
  * Parallel form with identity features: the end of the simplification ladder ("Test-Time

@@ -36,12 +36,13 @@ TTT_PATH_PARALLEL = 0
 TTT_PATH_RECURRENT = 1
 TTT_PATH_LINEAR = 2
 TTT_PATH_PARALLEL_MOMENTUM = 3
+TTT_PATH_PARALLEL_BWD = 4
 TTT_STATIC_SCRATCH_BYTES = 64 << 20
 
 # Every symbol include/ttt.h declares.
 EXPORTED = (
     "ttt_workspace_bytes", "ttt_la_parallel_fwd", "ttt_la_parallel_fwd_noalloc",
-    "ttt_linear_attn_fwd", "ttt_la_parallel_momentum_fwd",
+    "ttt_linear_attn_fwd", "ttt_la_parallel_momentum_fwd", "ttt_la_parallel_bwd",
     "ttt_lact_recurrent_fwd",
     "ttt_lm_target_workspace_bytes", "ttt_lm_target", "ttt_last_device_status",
     "ttt_debug_wait_timeout", "ttt_trace_enable", "ttt_trace_disable", "ttt_trace_count",
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_linear_attn_fwd.restype = I32
         L.ttt_la_parallel_momentum_fwd.argtypes = [D] + [P] * 11 + [S, P]
         L.ttt_la_parallel_momentum_fwd.restype = I32
+        L.ttt_la_parallel_bwd.argtypes = [D] + [P] * 17 + [S, P]
+        L.ttt_la_parallel_bwd.restype = I32
         L.ttt_lact_recurrent_fwd.argtypes = [D] + [P] * 14 + [S, P]
         L.ttt_lact_recurrent_fwd.restype = I32
         L.ttt_lm_target_workspace_bytes.argtypes = [I32, I32]
@@ -177,6 +180,15 @@ def ttt_la_parallel_momentum_fwd(desc, q, k, v, eta, alpha, W0, W2, W1, out, S_f
     _check(lib().ttt_la_parallel_momentum_fwd(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(alpha), _ptr(W0),
         _ptr(W2), _ptr(W1), _ptr(out), _ptr(S_final), _ptr(workspace), wb, _stream(stream)))
+
+
+def ttt_la_parallel_bwd(desc, q, k, v, eta, W0, W2, W1, dout, dS_final, dq, dk, dv, deta, dW0,
+                        dW2, dW1, workspace, workspace_bytes=None, stream=None):
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    _check(lib().ttt_la_parallel_bwd(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W0), _ptr(W2), _ptr(W1),
+        _ptr(dout), _ptr(dS_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(deta), _ptr(dW0),
+        _ptr(dW2), _ptr(dW1), _ptr(workspace), wb, _stream(stream)))
 
 
 def ttt_linear_attn_fwd(desc, q, k, v, eta, S0, out, S_final, workspace, workspace_bytes=None,

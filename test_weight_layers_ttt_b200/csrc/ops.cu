@@ -378,6 +378,57 @@ __global__ void split_hilo_kernel(const float* M, long long P, int rows, int col
   }
 }
 
+// ------------------------------------------------------------------ backward helpers
+template <typename OT>
+__global__ void suffix_scan_kernel(const float* dSc, const float* dS_final, OT* G, float* R0,
+                                   int BH, int C, long long n, int order) {
+  TTT_GRID_LOOP(idx, (long long)BH * n) {
+    const long long bh = idx / n, e = idx - bh * n;
+    float r = dS_final ? dS_final[idx] : 0.0f;
+    for (int c = C - 1; c >= 0; --c) {
+      const long long o = (bh * C + c) * n + e;
+      if (order == 1) G[o] = from_f32<OT>(r);
+      r += dSc[o];
+      if (order != 1) G[o] = from_f32<OT>(r);
+    }
+    R0[idx] = r;
+  }
+}
+
+// one warp per row
+template <typename OT>
+__global__ void row_grads_kernel(const float* T, const OT* v, const float* eta, float sgn,
+                                 OT* dv, float* deta, long long rows, int w) {
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += warps) {
+    const int lane = threadIdx.x & 31;
+    const float se = sgn * eta[r];
+    float acc = 0.0f;
+    for (int j = lane; j < w; j += 32) {
+      const float t = T[r * w + j];
+      acc = fmaf(t, to_f32(v[r * w + j]), acc);
+      dv[r * w + j] = from_f32<OT>(se * t);
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) deta[r] = sgn * acc;
+  }
+}
+
+__global__ void sum_batches_kernel(const float* X, int B, long long stride, long long n,
+                                   float* out) {
+  TTT_GRID_LOOP(i, n) {
+    float acc = 0.0f;
+    for (int b = 0; b < B; ++b) acc += X[b * stride + i];
+    out[i] = acc;
+  }
+}
+
+template <typename OT>
+__global__ void cast_kernel(const float* X, OT* out, long long n) {
+  TTT_GRID_LOOP(i, n) out[i] = from_f32<OT>(X[i]);
+}
+
 // One thread per element, chunks in order (the chunk axis is short).
 __global__ void momentum_scan_kernel(float* D, const float* alpha, int BH, int C, long long n) {
   TTT_GRID_LOOP(idx, (long long)BH * n) {
@@ -709,6 +760,45 @@ cudaError_t split_hilo(const float* M, int P, int rows, int cols, void* hhl, voi
                                                      static_cast<uint4*>(hlh),
                                                      static_cast<uint4*>(stack));
   return cudaGetLastError();
+}
+
+cudaError_t suffix_scan(int ot, const float* dSc, const float* dS_final, void* G, float* R0,
+                        int BH, int C, long long n, int order, cudaStream_t s) {
+  if (BH <= 0 || n <= 0) return cudaSuccess;
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    suffix_scan_kernel<OT><<<grid_for((long long)BH * n, 256), 256, 0, s>>>(
+        dSc, dS_final, static_cast<OT*>(G), R0, BH, C, n, order);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t row_grads(int ot, const float* T, const void* v, const float* eta, int sign,
+                      void* dv, float* deta, long long rows, int w, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    const long long blocks = (rows + 7) / 8;
+    row_grads_kernel<OT><<<(unsigned)(blocks < 148 * 32 ? blocks : 148 * 32), 256, 0, s>>>(
+        T, static_cast<const OT*>(v), eta, (float)sign, static_cast<OT*>(dv), deta, rows, w);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t sum_batches(const float* X, int B, long long stride, long long n, float* out,
+                        cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  sum_batches_kernel<<<grid_for(n, 256), 256, 0, s>>>(X, B, stride, n, out);
+  return cudaGetLastError();
+}
+
+cudaError_t cast_to(int ot, const float* X, void* out, long long n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    cast_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(X, static_cast<OT*>(out), n);
+    return cudaGetLastError();
+  });
 }
 
 cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long n,

@@ -84,6 +84,21 @@ cudaError_t ns_mma(float* U, int Z, const NsLayout& L, int steps, float eps, flo
 cudaError_t split_hilo(const float* M, int P, int rows, int cols, void* hhl, void* hlh,
                        void* stack, cudaStream_t s);
 
+// Backward of the prefix scan: R = dS_final[bh] (or 0 when null), then for c = C-1 .. 0:
+// R += dSc[bh, c] and the gradient of chunk c's delta G[bh, c] (OT) is R (order 0) or the
+// value before the addition (order 1); R0[bh] = the final R (fp32). [BH, C, n] / [BH, n].
+cudaError_t suffix_scan(int ot, const float* dSc, const float* dS_final, void* G, float* R0,
+                        int BH, int C, long long n, int order, cudaStream_t s);
+// dv[r] = sign * eta[r] * T[r] (OT) and deta[r] = sign * <T[r], v[r]> for `rows` rows of
+// width w (T fp32, v OT).
+cudaError_t row_grads(int ot, const float* T, const void* v, const float* eta, int sign,
+                      void* dv, float* deta, long long rows, int w, cudaStream_t s);
+// out[i] = sum over b of X[b * stride + i] for i < n (fp32).
+cudaError_t sum_batches(const float* X, int B, long long stride, long long n, float* out,
+                        cudaStream_t s);
+// Cast fp32 to OT (n elements).
+cudaError_t cast_to(int ot, const float* X, void* out, long long n, cudaStream_t s);
+
 // Momentum over chunks, in place: D[bh, c] <- alpha[bh, c] * D[bh, c - 1] + D[bh, c] for
 // c = 1 .. C-1 (D [BH, C, n] fp32, alpha [BH, C]).
 cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long n,

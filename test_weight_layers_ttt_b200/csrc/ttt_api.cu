@@ -175,7 +175,13 @@ ttt_status check_desc(const ttt_desc* d, int path) {
     return fail(TTT_ERR_INVALID_ARG, "w_in_layout must be 0 or 1");
   if (d->w1_layout != 0 && d->w1_layout != 1)
     return fail(TTT_ERR_INVALID_ARG, "w1_layout must be 0 or 1");
-  if (path == TTT_PATH_PARALLEL_MOMENTUM) {
+  if (path == TTT_PATH_PARALLEL_BWD) {
+    if (d->update_mask != 0 || d->renorm != 0 || d->momentum != 0 || d->ns_steps != 0)
+      return fail(TTT_ERR_INVALID_ARG,
+                  "parallel form: update_mask, renorm, momentum and ns_steps must be 0");
+    if (d->w_in_layout != 0 || d->w1_layout != 0)
+      return fail(TTT_ERR_UNSUPPORTED, "backward: default weight layouts only");
+  } else if (path == TTT_PATH_PARALLEL_MOMENTUM) {
     if (d->update_mask != 0 || d->renorm != 0)
       return fail(TTT_ERR_INVALID_ARG, "parallel form: update_mask and renorm must be 0");
     if (d->momentum != 0 && d->momentum != 1)
@@ -556,6 +562,176 @@ ttt_status momentum_impl(const ttt_desc& d, const void* q, const void* k, const 
   return chunk_outputs(d, b.phiB, b.Sc, out, s);
 }
 
+// ------------------------------------------------------------------ backward
+// Gradients of the parallel form (the oracle's la_parallel_backward, in the same order):
+// recompute phi(K) eta, phi(K), the chunk states and phi(Q); dS_c = phi(Q_c)^T dO_c; the
+// suffix scan gives each delta's gradient G_c and dW1; dphi(Q_c) = dO_c S_c^T,
+// dphi(K_c) = sign diag(eta) V_c G_c^T, T_c = phi(K_c) G_c gives dV = sign eta T and
+// deta = sign <T, v>; the SwiGLU backward runs as the feature GEMM's gradient epilogue
+// (row scale -1: dA = dphi B silu'(A), dB = dphi silu(A)); dX = dA W0^T + dB W2^T and
+// dW0 / dW2 = X^T dA / X^T dB per (b, head), summed over the batch.
+struct BwdBufs {
+  ParBufs p;        // Wk, phiA (phi eta -> dphi(K)), phiB (phi(Q) -> dphi(Q)), dS, Sc
+  void* phiK;       // phi(K) [BH, N, m], then the gradient epilogue's discarded output
+  void* G;          // [BH, C, m, h]
+  float* R0;        // [BH, m, h]
+  void* Ve;         // v * eta [BH, N, h]
+  float* T;         // [BH, N, h] fp32 (then dX partials)
+  float* neg1;      // [BH * N] = -1
+  void* dA;         // [BH, N, m]
+  void* dB;         // [BH, N, m]
+  void* W0b;        // [H, h, m] operand copies
+  void* W2b;
+  float* dW0p;      // [BH, h, m]
+  float* dW2p;
+};
+
+size_t plan_backward(const ttt_desc& d, void* base, BwdBufs& b) {
+  const size_t off = (plan_parallel(d, base, b.p) + 255) & ~static_cast<size_t>(255);
+  Carve cv(base ? static_cast<char*>(base) + off : nullptr);
+  const size_t os = d.dtype == TTT_DTYPE_BF16 ? 2 : 4;
+  const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
+  const long long T = BH * d.N, hm = (long long)d.h * d.m;
+  b.phiK = cv.take(os * T * d.m);
+  b.G = cv.take(os * BH * C * hm);
+  b.R0 = cv.take_n<float>(BH * hm);
+  b.Ve = cv.take(os * T * d.h);
+  b.T = cv.take_n<float>(T * d.h);
+  b.neg1 = cv.take_n<float>(T);
+  b.dA = cv.take(os * T * d.m);
+  b.dB = cv.take(os * T * d.m);
+  b.W0b = cv.take(os * d.H * hm);
+  b.W2b = cv.take(os * d.H * hm);
+  b.dW0p = cv.take_n<float>(BH * hm);
+  b.dW2p = cv.take_n<float>(BH * hm);
+  return off + cv.off;
+}
+
+// One operand of a per-chunk GEMM: either token rows of [B*H, N, w] sliced to the chunk,
+// or the chunk's own matrix of [B*H, C, r, w] (r * w = h * m).
+struct ChunkOp {
+  const void* ptr;
+  int dt;
+  bool mn;
+  long long w;
+  bool tokens;
+};
+
+// For every chunk of every (b, head): C_c = alpha * A_c B_c (the chunk-length dimension of
+// M, N or K given as -1).
+ttt_status chunk_gemm(const char* name, const ttt_desc& d, int M, int Nn, int K, ChunkOp A,
+                      ChunkOp B, ChunkOp Cc, float alpha, cudaStream_t s) {
+  const long long BH = (long long)d.B * d.H, N = d.N, L = d.chunk, hm = (long long)d.h * d.m;
+  const long long C = (N + L - 1) / L, Cf = N / L, tail = N - Cf * L;
+  for (int part = 0; part < 2; ++part) {
+    const long long nz1 = part == 0 ? Cf : (tail > 0 ? 1 : 0);
+    if (nz1 == 0) continue;
+    const long long t0 = part == 0 ? 0 : Cf * L, c0 = part == 0 ? 0 : Cf;
+    const int Lc = (int)(part == 0 ? L : tail);
+    auto op = [&](const ChunkOp& o) {
+      const size_t es = dtype_size(o.dt);
+      if (o.tokens)
+        return GemmOperand{static_cast<const char*>(o.ptr) + t0 * o.w * es, o.dt, o.mn, o.w,
+                           N * o.w, L * o.w};
+      return GemmOperand{static_cast<const char*>(o.ptr) + c0 * hm * es, o.dt, o.mn, o.w,
+                         C * hm, hm};
+    };
+    GemmProblem p;
+    p.M = M < 0 ? Lc : M; p.N = Nn < 0 ? Lc : Nn; p.K = K < 0 ? Lc : K;
+    p.Z0 = (int)BH; p.Z1 = (int)nz1;
+    p.A = op(A);
+    p.B = op(B);
+    const GemmOperand c = op(Cc);
+    p.C = {const_cast<void*>(c.ptr), c.dtype, c.ld, c.s0, c.s1};
+    p.alpha = alpha;
+    TTT_TRY(run_gemm(name, p, s));
+  }
+  return TTT_OK;
+}
+
+ttt_status backward_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
+                         const float* eta, const float* W0, const float* W2, const float* W1,
+                         const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
+                         float* deta, float* dW0, float* dW2, float* dW1, const BwdBufs& b,
+                         cudaStream_t s) {
+  const ParBufs& pb = b.p;
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, H = d.H;
+  const long long C = (N + d.chunk - 1) / d.chunk, T = BH * N, hm = h * m;
+  const float sg = (float)d.sign;
+  // forward recomputation
+  TTT_OP("prep_weights",
+         prep_wk_blocked(ot, W0, W2, pb.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
+  TTT_OP("cast_weights", cast_to(ot, W0, b.W0b, H * hm, s));
+  TTT_OP("cast_weights", cast_to(ot, W2, b.W2b, H * hm, s));
+  TTT_TRY(run_swiglu("gemm_features_k", features_problem(d, k, pb.Wk, pb.phiA, b.phiK, eta), s));
+  TTT_TRY(state_deltas(d, pb.phiA, v, pb.dS, s));
+  TTT_TRY(chunk_states(d, pb.dS, W1, nullptr, pb.Sc, s));
+  TTT_TRY(run_swiglu("gemm_features_q", features_problem(d, q, pb.Wk, pb.phiB, nullptr, nullptr),
+                     s));
+  // dS_c = phi(Q_c)^T dO_c, then G_c and dW1 per (b, head)
+  TTT_TRY(chunk_gemm("gemm_bwd_state", d, d.m, d.h, -1, {pb.phiB, ot, true, m, true},
+                     {dO, ot, true, h, true}, {pb.dS, DT_F32, false, h, false}, 1.0f, s));
+  TTT_OP("suffix_scan", suffix_scan(ot, pb.dS, dS_final, b.G, b.R0, (int)BH, (int)C, hm,
+                                    d.order, s));
+  // dphi(Q_c) = dO_c S_c^T (into phiB), dphi(K_c) = sign diag(eta) V_c G_c^T (into phiA)
+  TTT_TRY(chunk_gemm("gemm_bwd_dphi_q", d, -1, d.m, d.h, {dO, ot, false, h, true},
+                     {pb.Sc, ot, false, h, false}, {pb.phiB, ot, false, m, true}, 1.0f, s));
+  TTT_OP("scale_rows", scale_rows(ot, v, eta, b.Ve, T, d.h, s));
+  TTT_TRY(chunk_gemm("gemm_bwd_dphi_k", d, -1, d.m, d.h, {b.Ve, ot, false, h, true},
+                     {b.G, ot, false, h, false}, {pb.phiA, ot, false, m, true}, sg, s));
+  // T_c = phi(K_c) G_c: dV and deta
+  TTT_TRY(chunk_gemm("gemm_bwd_t", d, -1, d.h, d.m, {b.phiK, ot, false, m, true},
+                     {b.G, ot, true, h, false}, {b.T, DT_F32, false, h, true}, 1.0f, s));
+  TTT_OP("row_grads", row_grads(ot, b.T, v, eta, d.sign, dv, deta, T, d.h, s));
+  TTT_OP("fill", fill_f32(b.neg1, T, -1.0f, s));
+  // SwiGLU backward and input / weight gradients, key side then query side
+  for (int side = 0; side < 2; ++side) {
+    const void* X = side == 0 ? k : q;
+    void* dX = side == 0 ? dk : dq;
+    SwigluGemm g = features_problem(d, X, pb.Wk, b.phiK, nullptr, b.neg1);
+    g.grad = 1;
+    g.out2 = b.dB; g.ld2 = m; g.s20 = N * m; g.s21 = H * N * m;
+    g.out3 = b.dA; g.ld3 = m; g.s30 = N * m; g.s31 = H * N * m;
+    g.dv = side == 0 ? pb.phiA : pb.phiB;
+    g.ldd = m; g.ds0 = N * m; g.ds1 = H * N * m;
+    TTT_TRY(run_swiglu(side == 0 ? "gemm_bwd_swiglu_k" : "gemm_bwd_swiglu_q", g, s));
+    // dX = dA W0^T + dB W2^T
+    for (int t = 0; t < 2; ++t) {
+      GemmProblem p;
+      p.M = d.N; p.N = d.h; p.K = d.m; p.Z0 = d.H; p.Z1 = d.B;
+      p.A = {t == 0 ? b.dA : b.dB, ot, false, m, N * m, H * N * m};
+      p.B = {t == 0 ? b.W0b : b.W2b, ot, false, m, hm, 0};
+      if (t == 0) {
+        p.C = {b.T, DT_F32, h, N * h, H * N * h};
+      } else {
+        p.C = {dX, ot, h, N * h, H * N * h};
+        p.beta = 1.0f;
+        p.Cin = {b.T, h, N * h, H * N * h};
+      }
+      TTT_TRY(run_gemm("gemm_bwd_dx", p, s));
+    }
+    // dW0 / dW2 per (b, head) += X^T dA / X^T dB
+    for (int t = 0; t < 2; ++t) {
+      GemmProblem p;
+      p.M = d.h; p.N = d.m; p.K = d.N; p.Z0 = d.H; p.Z1 = d.B;
+      p.A = {X, ot, true, h, N * h, H * N * h};
+      p.B = {t == 0 ? b.dA : b.dB, ot, true, m, N * m, H * N * m};
+      float* out = t == 0 ? b.dW0p : b.dW2p;
+      p.C = {out, DT_F32, m, hm, H * hm};
+      if (side == 1) {
+        p.beta = 1.0f;
+        p.Cin = {out, m, hm, H * hm};
+      }
+      TTT_TRY(run_gemm("gemm_bwd_dw", p, s));
+    }
+  }
+  TTT_OP("sum_batches", sum_batches(b.dW0p, d.B, H * hm, H * hm, dW0, s));
+  TTT_OP("sum_batches", sum_batches(b.dW2p, d.B, H * hm, H * hm, dW2, s));
+  TTT_OP("sum_batches", sum_batches(b.R0, d.B, H * hm, H * hm, dW1, s));
+  return TTT_OK;
+}
+
 // ------------------------------------------------------------------ recurrent form
 struct RecBufs {
   float* W_all;   // fp32 masters [BH][W0 | W1 | W2]
@@ -740,6 +916,10 @@ size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path) {
     MomBufs b;
     return plan_momentum(*desc, nullptr, b);
   }
+  if (path == TTT_PATH_PARALLEL_BWD) {
+    BwdBufs b;
+    return plan_backward(*desc, nullptr, b);
+  }
   RecBufs b;
   return plan_recurrent(*desc, nullptr, b);
 }
@@ -831,6 +1011,44 @@ ttt_status ttt_la_parallel_momentum_fwd(const ttt_desc* desc, const void* q, con
     return TTT_OK;
   }
   return momentum_impl(d, q, k, v, eta, alpha, W0, W2, W1, out, S_final, b, s);
+}
+
+ttt_status ttt_la_parallel_bwd(const ttt_desc* desc, const void* q, const void* k, const void* v,
+                               const float* eta, const float* W0, const float* W2,
+                               const float* W1, const void* dout, const float* dS_final,
+                               void* dq, void* dk, void* dv, float* deta, float* dW0,
+                               float* dW2, float* dW1, void* workspace, size_t workspace_bytes,
+                               ttt_stream_t stream) {
+  TTT_TRY(check_desc(desc, TTT_PATH_PARALLEL_BWD));
+  const ttt_desc& d = *desc;
+  const long long BH = (long long)d.B * d.H;
+  if (BH == 0) return TTT_OK;
+  if (!W0 || !W2 || !W1 || !dW0 || !dW2 || !dW1)
+    return fail(TTT_ERR_INVALID_ARG, "weights and weight gradients must not be NULL");
+  if (d.N > 0) {
+    if (!q || !k || !v || !eta || !dout || !dq || !dk || !dv || !deta)
+      return fail(TTT_ERR_INVALID_ARG, "inputs, dout and input gradients must not be NULL");
+    if (q == k || dq == dk)
+      return fail(TTT_ERR_INVALID_ARG, "backward: q and k (and dq, dk) must be distinct");
+    const void* ptrs[] = {q, k, v, dout, dq, dk, dv, W0, W2, W1, eta, deta};
+    for (const void* p : ptrs)
+      if (!al16(p)) return fail(TTT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  BwdBufs b;
+  const size_t need = plan_backward(d, nullptr, b);
+  TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  plan_backward(d, workspace, b);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long hm = (long long)d.h * d.m;
+  if (d.N == 0) {   // no outputs: dW1 = sum over the batch of dS_final, the rest zero
+    TTT_OP("fill", fill_f32(dW0, d.H * hm, 0.0f, s));
+    TTT_OP("fill", fill_f32(dW2, d.H * hm, 0.0f, s));
+    if (dS_final) TTT_OP("sum_batches", sum_batches(dS_final, d.B, d.H * hm, d.H * hm, dW1, s));
+    else TTT_OP("fill", fill_f32(dW1, d.H * hm, 0.0f, s));
+    return TTT_OK;
+  }
+  return backward_impl(d, q, k, v, eta, W0, W2, W1, dout, dS_final, dq, dk, dv, deta, dW0, dW2,
+                       dW1, b, s);
 }
 
 ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const void* k,

@@ -93,6 +93,25 @@ def la_parallel_momentum_fwd(q, k, v, eta, W0, W2, W1, chunk, *, order="update_a
     return out, S
 
 
+def la_parallel_bwd(q, k, v, eta, W0, W2, W1, dout, chunk, *, order="update_apply", sign=1,
+                    dS_final=None, ws=None, stream=None):
+    """Backward of la_parallel_fwd. Returns dq, dk, dv (q's dtype), deta, dW0, dW2, dW1
+    (fp32; weight gradients per head, summed over the batch)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _need(t, n, q.dtype)
+    _need(eta, "eta", torch.float32)
+    _need(dS_final, "dS_final", torch.float32)
+    desc = parallel_desc(q, W1, chunk, order, sign)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    deta = torch.empty_like(eta)
+    dW0, dW2, dW1 = torch.empty_like(W0), torch.empty_like(W2), torch.empty_like(W1)
+    if ws is None:
+        ws = workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_PARALLEL_BWD), q.device)
+    abi.ttt_la_parallel_bwd(desc, q, k, v, eta, W0, W2, W1, dout, dS_final, dq, dk, dv, deta,
+                            dW0, dW2, dW1, ws, stream=stream)
+    return dq, dk, dv, deta, dW0, dW2, dW1
+
+
 def linear_attn_fwd(q, k, v, eta, S0, chunk, *, order="update_apply", sign=1, s_layout=0,
                     return_state=True, out=None, ws=None, stream=None):
     """Parallel form with identity features (plain chunked linear attention with per-token

@@ -153,6 +153,23 @@ def test_parallel_momentum_workspace_and_checks():
     assert ei.value.status == abi.TTT_ERR_INVALID_ARG
 
 
+def test_backward_workspace_and_checks():
+    P = abi.TTT_PATH_PARALLEL_BWD
+    assert abi.ttt_workspace_bytes(lm_desc(), P) > abi.ttt_workspace_bytes(lm_desc(), 0)
+    assert abi.ttt_workspace_bytes(lm_desc(w_in_layout=1), P) == 0
+    assert abi.ttt_workspace_bytes(lm_desc(momentum=1), P) == 0
+    d = lm_desc()
+    need = abi.ttt_workspace_bytes(d, P)
+    with pytest.raises(abi.TTTError) as ei:   # q aliased with k
+        abi.ttt_la_parallel_bwd(d, 256, 256, 256, 256, 256, 256, 256, 256, None, 512, 768, 1024,
+                                1280, 256, 256, 256, 256, need, stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    with pytest.raises(abi.TTTError) as ei:   # missing weight gradient
+        abi.ttt_la_parallel_bwd(d, 256, 512, 256, 256, 256, 256, 256, 256, None, 512, 768, 1024,
+                                1280, None, 256, 256, 256, need, stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+
+
 def test_recurrent_rejects_bad_args():
     d = lm_desc(update_mask=7, momentum=1)
     need = abi.ttt_workspace_bytes(d, 1)

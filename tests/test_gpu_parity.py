@@ -10,7 +10,7 @@ import torch
 
 from oracle import ttt_oracle as O
 from test_weight_layers_ttt_b200 import abi, layer
-from ttt_inputs import WORKLOADS, make_layer_inputs, make_inplace_inputs
+from ttt_inputs import WORKLOADS, bf16_round, make_layer_inputs, make_inplace_inputs
 
 from gpu_helpers import TOL, dev, host, rel, torch_dtype
 
@@ -157,6 +157,51 @@ def test_parallel_rejects_misaligned_pointer_on_device():
     with pytest.raises(abi.TTTError) as ei:
         abi.ttt_la_parallel_fwd(desc, q.data_ptr() + 2, k, v, eta, W0, W2, W1, out, None, ws)
     assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- backward
+BWD_CASES = [
+    # kind, dtype, B, H, N, h, m, chunk, order, sign, with dS_final
+    ("tiny", "fp32", 1, 2, 150, 16, 24, 40, "update_apply", 1, True),
+    ("lm", "bf16", 2, 2, 1000, 128, 256, 256, "update_apply", 1, True),
+    ("lm", "bf16", 1, 3, 640, 64, 192, 128, "apply_update", -1, False),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_parallel_backward_matches_oracle(case):
+    """Every gradient of the parallel form (inputs, step sizes, weights summed over the batch)
+    against the oracle's chain rule."""
+    kind, dtype, B, H, N, h, m, chunk, order, sign, with_sf = case
+    wl, inp = layer_inputs(kind, dtype, B, H, N, h, m, chunk, seed=5000 + N)
+    rng = np.random.default_rng(N)
+    dO = rng.standard_normal((B, H, N, h))
+    if dtype == "bf16":
+        dO = bf16_round(dO.astype(np.float32)).astype(np.float64)
+    dSf = rng.standard_normal((B, H, m, h)) if with_sf else None
+    ref = {key: [] for key in ("dq", "dk", "dv", "deta")}
+    wsum = {key: 0.0 for key in ("dW0", "dW2", "dW1")}
+    for b in range(B):
+        for hd in range(H):
+            g = O.la_parallel_backward(inp["q"][b, hd], inp["k"][b, hd], inp["v"][b, hd],
+                                       inp["eta"][b, hd], inp["W0"][hd], inp["W2"][hd],
+                                       inp["W1"][hd], dO[b, hd], chunk, order=ORD[order],
+                                       sign=sign, dS_final=None if dSf is None else dSf[b, hd])
+            for key in ref:
+                ref[key].append(g[key])
+            for key in wsum:
+                wsum[key] = wsum[key] + np.eye(H)[hd][:, None, None] * g[key][None]
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, dtype)
+    td = torch_dtype(dtype)
+    grads = layer.la_parallel_bwd(q, k, v, eta, W0, W2, W1, dev(dO, td), chunk, order=order,
+                                  sign=sign, dS_final=None if dSf is None else dev(dSf))
+    abi.ttt_last_device_status()
+    tol = TOL[dtype] * (1 if dtype == "fp32" else 1.5)
+    for key, got in zip(("dq", "dk", "dv", "deta"), grads[:4]):
+        want = np.stack(ref[key]).reshape(host(got).shape)
+        assert rel(host(got), want) <= tol, key
+    for key, got in zip(("dW0", "dW2", "dW1"), grads[4:]):
+        assert rel(host(got), wsum[key]) <= tol, key
 
 
 # ----------------------------------------------------------------------------- identity features
