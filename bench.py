@@ -48,6 +48,9 @@ def layer_flops(wl, form: str) -> float:
         return float(feats + 2 * hm * T + 2 * hm * T)
     if form == "linear":   # identity features: state deltas and outputs, [h, h] states
         return 4.0 * wl.h * wl.h * T
+    if form == "train":   # forward 12hm + backward: recomputed forward 10hm, 4 chunk GEMMs
+        # 8hm, SwiGLU backward GEMMs 8hm, dX 8hm, dW 8hm per token-head
+        return 54.0 * hm * T
     if form == "parallel_momentum":   # parallel form + Newton-Schulz 5 on every chunk's W1 step
         r, c = min(wl.h, wl.m), max(wl.h, wl.m)
         return 12.0 * hm * T + 5 * (4.0 * r * r * c + 2.0 * r ** 3) * wl.B * wl.H * wl.C
@@ -387,6 +390,8 @@ def run_gpu(args, rank, local, world):
         forms.insert(1, "linear")   # identity features (plain chunked linear attention)
         # W1 momentum + Newton-Schulz 5 (simplification variant 2)
         forms.insert(2, "parallel_momentum")
+        # one training step of the layer: parallel forward + backward
+        forms.insert(3, "train")
     lin, l1 = g["layouts"]
     if wl.kind == "inplace":
         # the value target is part of the In-Place step; timed on its own below
@@ -410,6 +415,20 @@ def run_gpu(args, rank, local, world):
             def step():
                 abi.ttt_linear_attn_fwd(ldesc, g["q"], g["k"], g["v"], g["eta"], lS0, lout,
                                         None, lws)
+        elif form == "train":
+            tdesc = layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order)
+            tws = layer.workspace(max(abi.ttt_workspace_bytes(tdesc, abi.TTT_PATH_PARALLEL_BWD),
+                                      abi.ttt_workspace_bytes(tdesc, abi.TTT_PATH_PARALLEL)),
+                                  "cuda")
+            tout = torch.empty_like(g["q"])
+            tdo = torch.randn_like(g["q"])
+            tgr = [torch.empty_like(g[n]) for n in ("q", "k", "v", "eta", "W0", "W2", "W1")]
+
+            def step():
+                abi.ttt_la_parallel_fwd(tdesc, g["q"], g["k"], g["v"], g["eta"], g["W0"],
+                                        g["W2"], g["W1"], tout, None, tws)
+                abi.ttt_la_parallel_bwd(tdesc, g["q"], g["k"], g["v"], g["eta"], g["W0"],
+                                        g["W2"], g["W1"], tdo, None, *tgr, tws)
         elif form == "parallel_momentum":
             mdesc = layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order, 1, lin, l1)
             mdesc.momentum, mdesc.ns_steps = 1, 5
