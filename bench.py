@@ -310,6 +310,46 @@ def _timed(fn, steps, warmup, world, torch, trace_capacity=0):
     return ms, trace
 
 
+def _timed_graph(fn, steps, warmup, world, torch):
+    """The same steps replayed from one CUDA graph capture of `fn` (the kernels and their
+    arguments are baked at capture; replays launch them without host work). Returns
+    (ms over `steps` replays) or None when `fn` cannot be captured."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()                     # one eager call on the capture stream first
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            fn()
+        torch.cuda.synchronize()
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+    for _ in range(max(1, warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        g.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    barrier(world)
+    torch.cuda.synchronize()
+    del g
+    return ms
+
+
 def _kernel_table(trace, steps):
     tot = sum(ms for _, ms in trace) or 1.0
     table = {}
@@ -462,12 +502,20 @@ def run_gpu(args, rank, local, world):
                                            g["W0"], g["W2"], g["W1"], out, None, None, None,
                                            None, ws)
         steps = args.steps if form in ("parallel", "linear") else max(3, args.steps // 4)
+        # timed region: the step replayed from a CUDA graph (eager launches when the step
+        # cannot be captured); the per-kernel table comes from a separate traced eager pass
         with ClockSampler(gpu_id(local, torch)) as clk:
-            ms, trace = _timed(step, steps, args.warmup, world, torch, trace_capacity=16384)
+            ms = _timed_graph(step, steps, args.warmup, world, torch)
+            mode = "cuda_graph"
+            if ms is None:
+                ms, _ = _timed(step, steps, args.warmup, world, torch)
+                mode = "eager"
         abi.ttt_last_device_status()
         ms_max = max_over_ranks(ms, world, "cuda")
         per_step = ms_max / steps
-        table = _kernel_table(trace, steps)
+        tsteps = min(steps, 5)
+        _, trace = _timed(step, tsteps, 1, world, torch, trace_capacity=16384)
+        table = _kernel_table(trace, tsteps)
         if form == "lm_target":
             flops = 2.0 * wl.N * wl.h * wl.h
             nbytes = 2.0 * (2 * wl.N * wl.h + wl.h * wl.h) + 16.0 * wl.h
@@ -482,10 +530,11 @@ def run_gpu(args, rank, local, world):
             "roofline_frac_sustained": max(
                 flops / (peaks["bf16_tflops_sustained"] * 1e12),
                 nbytes / (peaks["hbm_gbs"] * 1e9)) / (per_step / 1e3),
-            "gpu_launches": len(trace),
+            "gpu_launches": len(trace) * steps // tsteps,
+            "launch_mode": mode,
             "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv)
                             for kk, vv in v.items()} for k, v in table.items()},
-            "roofline": _roofline(table, wl, peaks, form, steps),
+            "roofline": _roofline(table, wl, peaks, form, tsteps),
             "clocks": clk.summary(),
         }
 
