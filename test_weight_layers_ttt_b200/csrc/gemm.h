@@ -61,8 +61,9 @@ ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_er
 //
 // Gradient variant (grad = 1, recurrent form): with eta = rowscale and d = -eta * Dv, Dv =
 // V W1^T given in `dv` (bf16 [rows, n_valid] with its own strides), the epilogue writes
-// P = phi * eta to gemm.C, E2 = d * silu(A) to out2 (when set) and E0 = d * B * silu'(A)
-// to out3 (when set).
+// P = phi * eta to gemm.C (unless skip_out1), E2 = d * silu(A) to out2 (when set) and
+// E0 = d * B * silu'(A) to out3 (when set). With rowscale = -1 and dv = dphi this is the
+// SwiGLU backward: E0 = dA, E2 = dB.
 struct SwigluGemm {
   GemmProblem gemm;
   void* out2 = nullptr;
@@ -71,6 +72,7 @@ struct SwigluGemm {
   long long rs0 = 0, rs1 = 0;
   int n_valid = 0;
   int grad = 0;
+  int skip_out1 = 0;   // gradient variant: do not write P (gemm.C)
   void* out3 = nullptr;
   long long ld3 = 0, s30 = 0, s31 = 0;
   const void* dv = nullptr;

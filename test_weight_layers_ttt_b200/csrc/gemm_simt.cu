@@ -101,7 +101,7 @@ struct SimtSwiglu {
   void* C2; long long ld2, c2s0, c2s1;
   const float* rs; long long rs0, rs1;
   // gradient variant (see SwigluGemm): C = phi * eta, C2 = d silu(A), C3 = d B silu'(A)
-  int grad;
+  int grad, skip_out1;
   void* C3;
   const void* dv; long long ldd, ds0, ds1;
 };
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(THREADS) simt_swiglu_kernel(const SimtSwiglu s
       const float av = 2.0f * acc_a[r][c], bv = acc_b[r][c];   // the operand holds W0 / 2
       const float sa = siluf_(av);
       const float p = sa * bv;
-      C[(long long)gi * a.ldc + gj] = from_f32<TC>(p * rsv);
+      if (!sw.skip_out1) C[(long long)gi * a.ldc + gj] = from_f32<TC>(p * rsv);
       if (sw.grad) {
         const float d = -rsv * to_f32(DV[(long long)gi * sw.ldd + gj]);
         if (C2) C2[(long long)gi * a.ldc + gj] = from_f32<TC>(d * sa);
@@ -214,6 +214,7 @@ ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream) {
   sw.C2 = g.out2; sw.ld2 = g.ld2; sw.c2s0 = g.s20; sw.c2s1 = g.s21;
   sw.rs = g.rowscale; sw.rs0 = g.rs0; sw.rs1 = g.rs1;
   sw.grad = g.grad;
+  sw.skip_out1 = g.grad ? g.skip_out1 : 0;
   sw.C3 = g.grad ? g.out3 : nullptr;
   sw.dv = g.grad ? g.dv : nullptr;
   sw.ldd = g.ldd; sw.ds0 = g.ds0; sw.ds1 = g.ds1;

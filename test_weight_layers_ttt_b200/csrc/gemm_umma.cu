@@ -61,6 +61,7 @@ struct UArgs {
   int n_valid;
   // SWIGLU gradient variant: third output and the Dv input (bf16)
   int grad;
+  int skip_out1;
   void* C3;
   const __nv_bfloat16* dv; long long ldd, ds0, ds1;
   unsigned* err;
@@ -496,7 +497,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
         const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
         for (int o = 0; o < 3; ++o) {
-          if ((o == 1 && !args.C2) || (o == 2 && !args.C3)) continue;
+          if ((o == 0 && args.skip_out1) || (o == 1 && !args.C2) || (o == 2 && !args.C3))
+            continue;
           if (lane == 0) tma_store_wait_read();
           __syncwarp();
 #pragma unroll
@@ -888,6 +890,7 @@ ttt_status gemm_umma_swiglu(const SwigluGemm& g, cudaStream_t stream, unsigned* 
   a.rs = g.rowscale; a.rs0 = g.rs0; a.rs1 = g.rs1;
   a.n_valid = g.n_valid;
   a.grad = g.grad;
+  a.skip_out1 = g.grad ? g.skip_out1 : 0;
   a.C3 = g.grad ? g.out3 : nullptr;
   a.dv = static_cast<const __nv_bfloat16*>(g.dv);
   a.ldd = g.ldd; a.ds0 = g.ds0; a.ds1 = g.ds1;

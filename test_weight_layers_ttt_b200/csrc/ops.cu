@@ -429,6 +429,27 @@ __global__ void cast_kernel(const float* X, OT* out, long long n) {
   TTT_GRID_LOOP(i, n) out[i] = from_f32<OT>(X[i]);
 }
 
+template <typename OT>
+__global__ void cat_cols_kernel(const float* A, const float* B, OT* out, long long rows, int w) {
+  TTT_GRID_LOOP(i, rows * 2 * w) {
+    const long long r = i / (2 * w);
+    const int c = (int)(i - r * 2 * w);
+    out[i] = from_f32<OT>(c < w ? A[r * w + c] : B[r * w + c - w]);
+  }
+}
+
+__global__ void sum_split_cols_kernel(const float* X, int nb, long long rows, int w,
+                                      float* out0, float* out1) {
+  TTT_GRID_LOOP(i, rows * 2 * w) {
+    const long long r = i / (2 * w);
+    const int c = (int)(i - r * 2 * w);
+    float acc = 0.0f;
+    for (int b = 0; b < nb; ++b) acc += X[(long long)b * rows * 2 * w + i];
+    if (c < w) out0[r * w + c] = acc;
+    else out1[r * w + c - w] = acc;
+  }
+}
+
 // One thread per element, chunks in order (the chunk axis is short).
 __global__ void momentum_scan_kernel(float* D, const float* alpha, int BH, int C, long long n) {
   TTT_GRID_LOOP(idx, (long long)BH * n) {
@@ -799,6 +820,24 @@ cudaError_t cast_to(int ot, const float* X, void* out, long long n, cudaStream_t
     cast_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(X, static_cast<OT*>(out), n);
     return cudaGetLastError();
   });
+}
+
+cudaError_t cat_cols(int ot, const float* A, const float* B, void* out, long long rows, int w,
+                     cudaStream_t s) {
+  if (rows <= 0 || w <= 0) return cudaSuccess;
+  return by_ot(ot, [&](auto tag) {
+    using OT = decltype(tag);
+    cat_cols_kernel<OT><<<grid_for(rows * 2 * w, 256), 256, 0, s>>>(A, B, static_cast<OT*>(out),
+                                                                   rows, w);
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t sum_split_cols(const float* X, int nb, long long rows, int w, float* out0,
+                           float* out1, cudaStream_t s) {
+  if (rows <= 0 || w <= 0) return cudaSuccess;
+  sum_split_cols_kernel<<<grid_for(rows * 2 * w, 256), 256, 0, s>>>(X, nb, rows, w, out0, out1);
+  return cudaGetLastError();
 }
 
 cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long n,

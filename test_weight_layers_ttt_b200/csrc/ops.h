@@ -98,6 +98,12 @@ cudaError_t sum_batches(const float* X, int B, long long stride, long long n, fl
                         cudaStream_t s);
 // Cast fp32 to OT (n elements).
 cudaError_t cast_to(int ot, const float* X, void* out, long long n, cudaStream_t s);
+// out[r] = [A[r] | B[r]] (OT) for `rows` rows of width w each (A, B fp32).
+cudaError_t cat_cols(int ot, const float* A, const float* B, void* out, long long rows, int w,
+                     cudaStream_t s);
+// X [nb, rows, 2w] fp32 summed over nb: columns < w to out0 [rows, w], the rest to out1.
+cudaError_t sum_split_cols(const float* X, int nb, long long rows, int w, float* out0,
+                           float* out1, cudaStream_t s);
 
 // Momentum over chunks, in place: D[bh, c] <- alpha[bh, c] * D[bh, c - 1] + D[bh, c] for
 // c = 1 .. C-1 (D [BH, C, n] fp32, alpha [BH, C]).

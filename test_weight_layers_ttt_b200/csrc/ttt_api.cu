@@ -572,19 +572,26 @@ ttt_status momentum_impl(const ttt_desc& d, const void* q, const void* k, const 
 // dW0 / dW2 = X^T dA / X^T dB per (b, head), summed over the batch.
 struct BwdBufs {
   ParBufs p;        // Wk, phiA (phi eta -> dphi(K)), phiB (phi(Q) -> dphi(Q)), dS, Sc
-  void* phiK;       // phi(K) [BH, N, m], then the gradient epilogue's discarded output
+  void* phiK;       // phi(K) [BH, N, m]
   void* G;          // [BH, C, m, h]
   float* R0;        // [BH, m, h]
   void* Ve;         // v * eta [BH, N, h]
   float* T;         // [BH, N, h] fp32 (then dX partials)
   float* neg1;      // [BH * N] = -1
-  void* dA;         // [BH, N, m]
-  void* dB;         // [BH, N, m]
-  void* W0b;        // [H, h, m] operand copies
-  void* W2b;
-  float* dW0p;      // [BH, h, m]
-  float* dW2p;
+  void* dAB;        // [BH, N, 2m]: dA | dB per token row
+  void* Wcat;       // [H, h, 2m]: W0 | W2 operand
+  float* dWp;       // [splits, B, H, h, 2m] split-K partials of X^T [dA | dB]
+  int splits;
 };
+
+// Token splits of the weight-gradient GEMMs (their K is the sequence): enough (b, head,
+// split) tiles to fill the SMs twice, splits of at least 512 tokens dividing N.
+int bwd_splits(const ttt_desc& d) {
+  const long long tiles = (long long)d.B * d.H * ((d.h + 127) / 128) * ((2LL * d.m + 255) / 256);
+  int sp = 1;
+  while (sp < 64 && d.N % (2 * sp) == 0 && d.N / (2 * sp) >= 512 && tiles * sp < 2 * 148) sp *= 2;
+  return sp;
+}
 
 size_t plan_backward(const ttt_desc& d, void* base, BwdBufs& b) {
   const size_t off = (plan_parallel(d, base, b.p) + 255) & ~static_cast<size_t>(255);
@@ -598,12 +605,10 @@ size_t plan_backward(const ttt_desc& d, void* base, BwdBufs& b) {
   b.Ve = cv.take(os * T * d.h);
   b.T = cv.take_n<float>(T * d.h);
   b.neg1 = cv.take_n<float>(T);
-  b.dA = cv.take(os * T * d.m);
-  b.dB = cv.take(os * T * d.m);
-  b.W0b = cv.take(os * d.H * hm);
-  b.W2b = cv.take(os * d.H * hm);
-  b.dW0p = cv.take_n<float>(BH * hm);
-  b.dW2p = cv.take_n<float>(BH * hm);
+  b.splits = bwd_splits(d);
+  b.dAB = cv.take(os * T * 2 * d.m);
+  b.Wcat = cv.take(os * d.H * 2 * hm);
+  b.dWp = cv.take_n<float>((long long)b.splits * BH * 2 * hm);
   return off + cv.off;
 }
 
@@ -662,8 +667,7 @@ ttt_status backward_impl(const ttt_desc& d, const void* q, const void* k, const 
   // forward recomputation
   TTT_OP("prep_weights",
          prep_wk_blocked(ot, W0, W2, pb.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
-  TTT_OP("cast_weights", cast_to(ot, W0, b.W0b, H * hm, s));
-  TTT_OP("cast_weights", cast_to(ot, W2, b.W2b, H * hm, s));
+  TTT_OP("cast_weights", cat_cols(ot, W0, W2, b.Wcat, H * h, m, s));
   TTT_TRY(run_swiglu("gemm_features_k", features_problem(d, k, pb.Wk, pb.phiA, b.phiK, eta), s));
   TTT_TRY(state_deltas(d, pb.phiA, v, pb.dS, s));
   TTT_TRY(chunk_states(d, pb.dS, W1, nullptr, pb.Sc, s));
@@ -686,48 +690,44 @@ ttt_status backward_impl(const ttt_desc& d, const void* q, const void* k, const 
   TTT_OP("row_grads", row_grads(ot, b.T, v, eta, d.sign, dv, deta, T, d.h, s));
   TTT_OP("fill", fill_f32(b.neg1, T, -1.0f, s));
   // SwiGLU backward and input / weight gradients, key side then query side
+  const int sp = b.splits;
+  const long long Ks = N / sp;
   for (int side = 0; side < 2; ++side) {
     const void* X = side == 0 ? k : q;
     void* dX = side == 0 ? dk : dq;
-    SwigluGemm g = features_problem(d, X, pb.Wk, b.phiK, nullptr, b.neg1);
+    // [dA | dB] per token row: the gradient epilogue writes dB (out2) at column m and dA
+    // (out3) at column 0 of the same 2m-wide rows
+    // (gemm.C names dAB for the epilogue's output layout; that output is skipped)
+    SwigluGemm g = features_problem(d, X, pb.Wk, b.dAB, nullptr, b.neg1);
+    g.gemm.C.ld = 2 * m; g.gemm.C.s0 = N * 2 * m; g.gemm.C.s1 = H * N * 2 * m;
     g.grad = 1;
-    g.out2 = b.dB; g.ld2 = m; g.s20 = N * m; g.s21 = H * N * m;
-    g.out3 = b.dA; g.ld3 = m; g.s30 = N * m; g.s31 = H * N * m;
+    g.skip_out1 = 1;
+    g.out2 = static_cast<char*>(b.dAB) + m * dtype_size(ot);
+    g.ld2 = 2 * m; g.s20 = N * 2 * m; g.s21 = H * N * 2 * m;
+    g.out3 = b.dAB; g.ld3 = 2 * m; g.s30 = N * 2 * m; g.s31 = H * N * 2 * m;
     g.dv = side == 0 ? pb.phiA : pb.phiB;
     g.ldd = m; g.ds0 = N * m; g.ds1 = H * N * m;
     TTT_TRY(run_swiglu(side == 0 ? "gemm_bwd_swiglu_k" : "gemm_bwd_swiglu_q", g, s));
-    // dX = dA W0^T + dB W2^T
-    for (int t = 0; t < 2; ++t) {
-      GemmProblem p;
-      p.M = d.N; p.N = d.h; p.K = d.m; p.Z0 = d.H; p.Z1 = d.B;
-      p.A = {t == 0 ? b.dA : b.dB, ot, false, m, N * m, H * N * m};
-      p.B = {t == 0 ? b.W0b : b.W2b, ot, false, m, hm, 0};
-      if (t == 0) {
-        p.C = {b.T, DT_F32, h, N * h, H * N * h};
-      } else {
-        p.C = {dX, ot, h, N * h, H * N * h};
-        p.beta = 1.0f;
-        p.Cin = {b.T, h, N * h, H * N * h};
-      }
-      TTT_TRY(run_gemm("gemm_bwd_dx", p, s));
+    // dX = [dA | dB] [W0 | W2]^T
+    GemmProblem p;
+    p.M = d.N; p.N = d.h; p.K = (int)(2 * m); p.Z0 = d.H; p.Z1 = d.B;
+    p.A = {b.dAB, ot, false, 2 * m, N * 2 * m, H * N * 2 * m};
+    p.B = {b.Wcat, ot, false, 2 * m, 2 * hm, 0};
+    p.C = {dX, ot, h, N * h, H * N * h};
+    TTT_TRY(run_gemm("gemm_bwd_dx", p, s));
+    // X^T [dA | dB] per (b, head) and token split, accumulated over the two sides
+    GemmProblem w;
+    w.M = d.h; w.N = (int)(2 * m); w.K = (int)Ks; w.Z0 = (int)BH; w.Z1 = sp;
+    w.A = {X, ot, true, h, N * h, Ks * h};
+    w.B = {b.dAB, ot, true, 2 * m, N * 2 * m, Ks * 2 * m};
+    w.C = {b.dWp, DT_F32, 2 * m, 2 * hm, BH * 2 * hm};
+    if (side == 1) {
+      w.beta = 1.0f;
+      w.Cin = {b.dWp, 2 * m, 2 * hm, BH * 2 * hm};
     }
-    // dW0 / dW2 per (b, head) += X^T dA / X^T dB
-    for (int t = 0; t < 2; ++t) {
-      GemmProblem p;
-      p.M = d.h; p.N = d.m; p.K = d.N; p.Z0 = d.H; p.Z1 = d.B;
-      p.A = {X, ot, true, h, N * h, H * N * h};
-      p.B = {t == 0 ? b.dA : b.dB, ot, true, m, N * m, H * N * m};
-      float* out = t == 0 ? b.dW0p : b.dW2p;
-      p.C = {out, DT_F32, m, hm, H * hm};
-      if (side == 1) {
-        p.beta = 1.0f;
-        p.Cin = {out, m, hm, H * hm};
-      }
-      TTT_TRY(run_gemm("gemm_bwd_dw", p, s));
-    }
+    TTT_TRY(run_gemm("gemm_bwd_dw", w, s));
   }
-  TTT_OP("sum_batches", sum_batches(b.dW0p, d.B, H * hm, H * hm, dW0, s));
-  TTT_OP("sum_batches", sum_batches(b.dW2p, d.B, H * hm, H * hm, dW2, s));
+  TTT_OP("sum_batches", sum_split_cols(b.dWp, sp * d.B, H * h, m, dW0, dW2, s));
   TTT_OP("sum_batches", sum_batches(b.R0, d.B, H * hm, H * hm, dW1, s));
   return TTT_OK;
 }
