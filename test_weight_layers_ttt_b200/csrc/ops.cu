@@ -378,6 +378,23 @@ __global__ void split_hilo_kernel(const float* M, long long P, int rows, int col
   }
 }
 
+// out[z] = in[z]^T for Z row-major [rows, cols] fp32 matrices: 32 x 32 tiles through shared
+// memory, both sides along rows. grid (ceil(cols/32), ceil(rows/32), Z), block (32, 8).
+__global__ void transpose_kernel(const float* in, float* out, int rows, int cols) {
+  __shared__ float t[32][33];
+  const long long z = blockIdx.z, n = (long long)rows * cols;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32, tx = threadIdx.x, ty = threadIdx.y;
+  for (int k = ty; k < 32; k += 8) {
+    const int r = r0 + k, c = c0 + tx;
+    if (r < rows && c < cols) t[k][tx] = in[z * n + (long long)r * cols + c];
+  }
+  __syncthreads();
+  for (int k = ty; k < 32; k += 8) {
+    const int c = c0 + k, r = r0 + tx;   // out [cols, rows]
+    if (r < rows && c < cols) out[z * n + (long long)c * rows + r] = t[tx][k];
+  }
+}
+
 // ------------------------------------------------------------------ backward helpers
 template <typename OT>
 __global__ void suffix_scan_kernel(const float* dSc, const float* dS_final, OT* G, float* R0,
@@ -690,8 +707,21 @@ cudaError_t scale_rows(int ot, const void* X, const float* eta, void* Xs, long l
 }
 
 cudaError_t chunk_scan(int ot, const float* dS, const float* W1, void* Sc, float* S_final, int BH,
-                       int H, int C, int m, int h, int order, int layout, cudaStream_t s) {
+                       int H, int C, int m, int h, int order, int layout, float* scratch,
+                       cudaStream_t s) {
   const long long per = (long long)m * h;
+  if (layout == 1 && scratch) {
+    // transposed W1 / S_final: transpose once on each side and scan in the [m, h] layout
+    float* W1t = scratch;
+    float* Sft = scratch + (long long)H * per;
+    transpose_kernel<<<dim3((m + 31) / 32, (h + 31) / 32, H), dim3(32, 8), 0, s>>>(W1, W1t, h, m);
+    cudaError_t e = chunk_scan(ot, dS, W1t, Sc, S_final ? Sft : nullptr, BH, H, C, m, h, order, 0,
+                               nullptr, s);
+    if (e != cudaSuccess || !S_final) return e;
+    transpose_kernel<<<dim3((h + 31) / 32, (m + 31) / 32, BH), dim3(32, 8), 0, s>>>(Sft, S_final,
+                                                                                  m, h);
+    return cudaGetLastError();
+  }
   const bool vec = layout == 0 && per % 4 == 0 &&
                    ((reinterpret_cast<uintptr_t>(dS) | reinterpret_cast<uintptr_t>(W1) |
                      reinterpret_cast<uintptr_t>(Sc) | reinterpret_cast<uintptr_t>(S_final)) & 15) == 0;

@@ -25,9 +25,11 @@ cudaError_t scale_rows(int ot, const void* X, const float* eta, void* Xs, long l
 // Chunk prefix sums: S starts at W1[bh % H] (layout 0 [m,h] / 1 [h,m]); for each chunk c
 // the state read by chunk c is written to Sc[bh, c] (OT, [m,h]): inclusive of dS[bh, c]
 // (order 0) or exclusive (order 1). The state after the last chunk goes to S_final
-// (fp32, W1's layout) when non-null.
+// (fp32, W1's layout) when non-null. With layout 1 and a scratch of (H + BH) * m * h floats,
+// W1 and S_final are transposed through it so the scan itself runs on 16-byte vectors.
 cudaError_t chunk_scan(int ot, const float* dS, const float* W1, void* Sc, float* S_final, int BH,
-                       int H, int C, int m, int h, int order, int layout, cudaStream_t s);
+                       int H, int C, int m, int h, int order, int layout, float* scratch,
+                       cudaStream_t s);
 
 // Recurrent-state helpers. Per (b, head) the fp32 state W_all holds [W0 (h*m) | W1 (m*h) |
 // W2 (h*m)]; momentum and the update buffer U use the same part layout.

@@ -228,6 +228,7 @@ struct ParBufs {
   void* phiB;  // phi(Q)        [BH, N, m]
   float* dS;   // [BH, C, m, h]
   void* Sc;    // [BH, C, m, h] state read by each chunk
+  float* scan_tmp;   // w1_layout 1: transposed W1 and final state ((H + BH) m h), else null
 };
 
 long long padded_m(int m) { return (m + 127LL) / 128 * 128; }
@@ -242,6 +243,7 @@ size_t plan_parallel(const ttt_desc& d, void* base, ParBufs& b) {
   b.phiB = cv.take(os * rows * d.m);
   b.dS = cv.take_n<float>(BH * C * hm);
   b.Sc = cv.take(os * BH * C * hm);
+  b.scan_tmp = d.w1_layout == 1 ? cv.take_n<float>((d.H + BH) * hm) : nullptr;
   return cv.off;
 }
 
@@ -298,19 +300,19 @@ ttt_status state_deltas(const ttt_desc& d, const void* X_eta, const void* v, flo
 }
 
 ttt_status chunk_states(const ttt_desc& d, const float* dS, const float* W1, float* S_final,
-                        void* Sc, cudaStream_t s) {
+                        void* Sc, float* scan_tmp, cudaStream_t s) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
   TTT_OP("chunk_scan", chunk_scan(ot, dS, W1, Sc, S_final, (int)BH, d.H, (int)C, d.m, d.h,
-                                  d.order, d.w1_layout, s));
+                                  d.order, d.w1_layout, scan_tmp, s));
   return TTT_OK;
 }
 
 ttt_status state_delta_and_scan(const ttt_desc& d, const void* X_eta, const void* v,
                                 const float* W1, float* S_final, float* dS, void* Sc,
-                                cudaStream_t s) {
+                                float* scan_tmp, cudaStream_t s) {
   TTT_TRY(state_deltas(d, X_eta, v, dS, s));
-  return chunk_states(d, dS, W1, S_final, Sc, s);
+  return chunk_states(d, dS, W1, S_final, Sc, scan_tmp, s);
 }
 
 // O_c = X_q(Q_c) S_c with X_q the query-side features [BH, N, m].
@@ -346,7 +348,7 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
   TTT_TRY(run_swiglu("gemm_features_k",
                      features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
                      s));
-  TTT_TRY(state_delta_and_scan(d, b.phiA, v, W1, S_final, b.dS, b.Sc, s));
+  TTT_TRY(state_delta_and_scan(d, b.phiA, v, W1, S_final, b.dS, b.Sc, b.scan_tmp, s));
   if (!shared_qk && !force_simt() && !getenv("TTT_NO_FUSED_APPLY") &&
       fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
     // phi(Q) S_c with phi kept on chip
@@ -367,6 +369,7 @@ struct LinBufs {
   void* Keta;  // k * eta  [BH, N, h]
   float* dS;   // [BH, C, h, h]
   void* Sc;    // [BH, C, h, h]
+  float* scan_tmp;
 };
 
 size_t plan_linear(const ttt_desc& d, void* base, LinBufs& b) {
@@ -377,6 +380,7 @@ size_t plan_linear(const ttt_desc& d, void* base, LinBufs& b) {
   b.Keta = cv.take(os * BH * d.N * d.h);
   b.dS = cv.take_n<float>(BH * C * hh);
   b.Sc = cv.take(os * BH * C * hh);
+  b.scan_tmp = d.w1_layout == 1 ? cv.take_n<float>((d.H + BH) * hh) : nullptr;
   return cv.off;
 }
 
@@ -385,7 +389,7 @@ ttt_status linear_impl(const ttt_desc& d, const void* q, const void* k, const vo
                        const LinBufs& b, cudaStream_t s) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   TTT_OP("scale_rows", scale_rows(ot, k, eta, b.Keta, (long long)d.B * d.H * d.N, d.h, s));
-  TTT_TRY(state_delta_and_scan(d, b.Keta, v, S0, S_final, b.dS, b.Sc, s));
+  TTT_TRY(state_delta_and_scan(d, b.Keta, v, S0, S_final, b.dS, b.Sc, b.scan_tmp, s));
   return chunk_outputs(d, q, b.Sc, out, s);
 }
 
@@ -549,7 +553,7 @@ ttt_status momentum_impl(const ttt_desc& d, const void* q, const void* k, const 
     TTT_OP("momentum_scan", momentum_scan(b.dS, alpha, (int)BH, (int)C, (long long)d.h * d.m, s));
   if (d.ns_steps > 0)
     TTT_TRY(run_ns(ot, b.dS, (int)(BH * C), ns_layout_single(d.m, d.h), d.ns_steps, mb.ns, s));
-  TTT_TRY(chunk_states(d, b.dS, W1, S_final, b.Sc, s));
+  TTT_TRY(chunk_states(d, b.dS, W1, S_final, b.Sc, nullptr, s));
   if (!shared_qk && !force_simt() && !getenv("TTT_NO_FUSED_APPLY") &&
       fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
     TraceScope ts("fused_apply@tcgen05", s);
@@ -670,7 +674,7 @@ ttt_status backward_impl(const ttt_desc& d, const void* q, const void* k, const 
   TTT_OP("cast_weights", cat_cols(ot, W0, W2, b.Wcat, H * h, m, s));
   TTT_TRY(run_swiglu("gemm_features_k", features_problem(d, k, pb.Wk, pb.phiA, b.phiK, eta), s));
   TTT_TRY(state_deltas(d, pb.phiA, v, pb.dS, s));
-  TTT_TRY(chunk_states(d, pb.dS, W1, nullptr, pb.Sc, s));
+  TTT_TRY(chunk_states(d, pb.dS, W1, nullptr, pb.Sc, nullptr, s));
   TTT_TRY(run_swiglu("gemm_features_q", features_problem(d, q, pb.Wk, pb.phiB, nullptr, nullptr),
                      s));
   // dS_c = phi(Q_c)^T dO_c, then G_c and dW1 per (b, head)
@@ -947,7 +951,7 @@ ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* 
   if (d.N == 0) {
     if (S_final)
       TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, W1, b.Sc, S_final, (int)BH, d.H, 0, d.m, d.h,
-                                      d.order, d.w1_layout, s));
+                                      d.order, d.w1_layout, nullptr, s));
     return TTT_OK;
   }
   return parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s);
@@ -975,7 +979,7 @@ ttt_status ttt_linear_attn_fwd(const ttt_desc* desc, const void* q, const void* 
   if (d.N == 0) {
     if (S_final)
       TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, S0, b.Sc, S_final, (int)BH, d.H, 0, d.h, d.h,
-                                      d.order, d.w1_layout, s));
+                                      d.order, d.w1_layout, nullptr, s));
     return TTT_OK;
   }
   return linear_impl(d, q, k, v, eta, S0, out, S_final, b, s);
@@ -1007,7 +1011,7 @@ ttt_status ttt_la_parallel_momentum_fwd(const ttt_desc* desc, const void* q, con
   if (d.N == 0) {
     if (S_final)
       TTT_OP("chunk_scan", chunk_scan(DT_F32, b.p.dS, W1, b.p.Sc, S_final, (int)BH, d.H, 0, d.m,
-                                      d.h, d.order, d.w1_layout, s));
+                                      d.h, d.order, d.w1_layout, nullptr, s));
     return TTT_OK;
   }
   return momentum_impl(d, q, k, v, eta, alpha, W0, W2, W1, out, S_final, b, s);
