@@ -1,5 +1,5 @@
 // Tensor-core batched GEMM engine for sm_100a: bf16 operands staged in shared memory by
-// TMA (128-byte swizzle, no multicast), tcgen05.mma kind::f16 with fp32 accumulators in
+// TMA (128-byte swizzle, one destination CTA), tcgen05.mma kind::f16 with fp32 accumulators in
 // tensor memory, and CUDA-core epilogues that read TMEM with tcgen05.ld.
 //
 // Persistent CTAs walk the 128 x BN output tiles of all batch entries round-robin. Two
@@ -14,14 +14,6 @@
 //   SWIGLU  the tile's columns are [A block | B block] of the fused SwiGLU input weights;
 //           writes phi = silu(a) * b times a per-row factor (bf16), and optionally the
 //           unscaled phi to a second output.
-// Pair mode (PAIR, B-resident problems): clusters of two CTAs on two SMs compute 256 x BN
-// tiles with tcgen05.mma.cta_group::2 (M = 256). Each CTA stages its own 128 rows of A and
-// its own half (BN / 2 rows) of the resident B, so every SM's tensor core reads half of B
-// from its own shared memory: a third less shared-memory traffic per MMA than one CTA with
-// M = 128, which is what bounds the single-CTA feature GEMM. The first CTA of the pair issues
-// the MMAs once both CTAs' stages are full (the second CTA's warp 1 forwards its own
-// "full" arrivals to the first CTA), the commits arrive on both CTAs' barriers, and each
-// CTA's epilogue drains its own 128 TMEM lanes and reports to the first CTA per warp.
 // Every mbarrier wait is bounded; a timeout records DEVERR_TIMEOUT in the device error
 // word, raises a CTA-wide abort flag, and the CTA drains its in-flight copies and MMAs
 // (again with bounded waits) and frees its TMEM before returning.
@@ -29,7 +21,6 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -73,18 +64,17 @@ struct UArgs {
 // stays in shared memory and the ring carries only A tiles.
 // SWIGLU mode adds a 32 KB staging tile (128 rows x 128 bf16 phi columns, as two
 // 128-byte-swizzled 64-column boxes) written by the epilogue and stored with TMA.
-template <int BN, int STAGES, bool BRES, int MODE, bool PAIR = false>
+template <int BN, int STAGES, bool BRES, int MODE>
 struct Smem {
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;        // this CTA's rows of the B tile
-  static constexpr int B_BYTES = B_ROWS * BK * 2;          // one k-block of B
+  static constexpr int B_BYTES = BN * BK * 2;             // one k-block of B
   static constexpr int B_RES = BRES ? 4 * B_BYTES : 0;    // resident B, at most 4 k-blocks
   static constexpr int STAGE = BRES ? A_BYTES : A_BYTES + B_BYTES;
   static constexpr int OUT_BYTES = MODE == 1 ? BM * 128 * 2 : 0;
   static constexpr int OUT_OFF = B_RES;
   static constexpr int RING_OFF = OUT_OFF + OUT_BYTES;
   static constexpr int BAR_OFF = RING_OFF + STAGES * STAGE;
-  static constexpr int TOTAL = BAR_OFF + 512 + 1024;      // + barriers + alignment slack
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;      // + barriers + alignment slack
 };
 
 __device__ __forceinline__ void store_vals(float* dst, const float* v, int n, bool vec) {
@@ -137,27 +127,22 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int tiles_n, int tiles_m
 // B-resident mode: CTA c keeps n-tile c % tiles_n and walks a contiguous range of the
 // flattened (z, tm) row tiles, shared with the other n-tile CTAs of its group, so a
 // group reads each A tile from HBM once and each CTA reloads B only when z changes.
-// Pair mode: the two CTAs of a cluster are one unit and walk the same sequence of
-// 256-row tiles (unit = blockIdx.x / 2, units = gridDim.x / 2, tile rows = 2 * BM).
 struct TileWalker {
   int tiles_n, tiles_m, Z0, total, count;
-  int bres, nt, r0, unit, units;
-  __device__ TileWalker(int M, int N, int Z0_, int Z1, int BN, bool b_res, bool pair = false) {
-    const int tm_rows = pair ? 2 * BM : BM;
-    unit = pair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    units = pair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  int bres, nt, r0;
+  __device__ TileWalker(int M, int N, int Z0_, int Z1, int BN, bool b_res) {
     tiles_n = (N + BN - 1) / BN;
-    tiles_m = (M + tm_rows - 1) / tm_rows;
+    tiles_m = (M + BM - 1) / BM;
     Z0 = Z0_;
     total = tiles_n * tiles_m * Z0_ * Z1;
     bres = b_res;
     if (!b_res) {
-      count = unit < total ? (total - 1 - unit) / units + 1 : 0;
+      count = blockIdx.x < (unsigned)total ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
       nt = r0 = 0;
     } else {
-      const int groups = units / tiles_n, g = unit / tiles_n;
+      const int groups = gridDim.x / tiles_n, g = blockIdx.x / tiles_n;
       const int rows = tiles_m * Z0_ * Z1;
-      nt = unit % tiles_n;
+      nt = blockIdx.x % tiles_n;
       if (g >= groups) {
         count = 0;
         r0 = 0;
@@ -169,7 +154,7 @@ struct TileWalker {
     }
   }
   __device__ TileCoord at(int i) const {
-    if (!bres) return decode_tile(unit + i * units, tiles_n, tiles_n * tiles_m, Z0);
+    if (!bres) return decode_tile(blockIdx.x + i * gridDim.x, tiles_n, tiles_n * tiles_m, Z0);
     const int r = r0 + i, z = r / tiles_m;
     TileCoord c;
     c.tm = r - z * tiles_m;
@@ -185,14 +170,12 @@ struct OutMaps {
   CUtensorMap m[3];
 };
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES,
-          bool PAIR = false>
+template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES>
 __global__ void __launch_bounds__(THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ OutMaps om, const UArgs args) {
-  static_assert(!PAIR || (BRES && !B_MN), "pair mode is for K-major resident B");
-  using L = Smem<BN, STAGES, BRES, MODE, PAIR>;
+  using L = Smem<BN, STAGES, BRES, MODE>;
   constexpr uint32_t ACC_COLS = 2 * BN;  // two accumulators
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -203,20 +186,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* acc_empty = acc_full + 2;    // [2]
   uint64_t* b_full = acc_empty + 2;     // resident B loaded
   uint64_t* b_empty = b_full + 1;       // resident B no longer read by MMAs
-  uint64_t* peer_full = b_empty + 1;           // [STAGES] pair mode, first CTA: second CTA's stages
-  uint64_t* peer_b_full = peer_full + STAGES;  // pair mode, first CTA: second CTA's B half
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_b_full + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = (args.K + BK - 1) / BK;
-  const TileWalker walk(args.M, args.N, args.Z0, args.Z1, BN, BRES, PAIR);
-  // pair mode: this CTA's rank, the first CTA's rank, and this CTA's first row in a tile
-  const uint32_t rank = PAIR ? cluster_rank() : 0u;
-  const uint32_t lead = rank & ~1u;
-  const bool leader = !PAIR || rank == lead;
-  constexpr int TILE_M = PAIR ? 2 * BM : BM;
-  const int row_off = PAIR ? (int)(rank - lead) * BM : 0;
+  const TileWalker walk(args.M, args.N, args.Z0, args.Z1, BN, BRES);
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t ring_base = smem_base + L::RING_OFF;
 
@@ -227,32 +202,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
-      // pair mode: one arrival per epilogue warp of both CTAs (on the first CTA's barrier)
-      mbar_init(smem_u32(&acc_empty[b]), PAIR ? 2 * EPI_WARPS : EPI_WARPS * 32);
+      mbar_init(smem_u32(&acc_empty[b]), EPI_WARPS * 32);
     }
     mbar_init(smem_u32(b_full), 1);
     mbar_init(smem_u32(b_empty), 1);
-    if (PAIR) {
-      for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&peer_full[s]), 1);
-      mbar_init(smem_u32(peer_b_full), 1);
-    }
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    if (PAIR) {
-      tmem_alloc_pair(smem_u32(tmem_slot), ACC_COLS);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(smem_u32(tmem_slot), ACC_COLS);
-      tmem_relinquish();
-    }
+    tmem_alloc(smem_u32(tmem_slot), ACC_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
-  if (PAIR) cluster_sync();   // both CTAs' barriers initialised before any remote arrive
-  else __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -281,8 +245,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               for (int q = 0; q < BN / 64; ++q)
                 tma_load_4d(sB + q * 8192, &tmB, bb, tc.tn * BN + 64 * q, kb * BK, bc2, bc3);
             } else {
-              tma_load_4d(sB, &tmB, bb, kb * BK, tc.tn * BN + (int)(rank - lead) * L::B_ROWS, bc2,
-                          bc3);
+              tma_load_4d(sB, &tmB, bb, kb * BK, tc.tn * BN, bc2, bc3);
             }
           }
           ++b_loads;
@@ -300,12 +263,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t fb = smem_u32(&full[s]);
           mbar_arrive_expect_tx(fb, L::STAGE);
           const uint32_t sA = ring_base + s * L::STAGE;
-          const int arow = tc.tm * TILE_M + row_off;
           if (A_MN) {
-            tma_load_4d(sA, &tmA, fb, arow, kb * BK, ac2, ac3);
-            tma_load_4d(sA + 8192, &tmA, fb, arow + 64, kb * BK, ac2, ac3);
+            tma_load_4d(sA, &tmA, fb, tc.tm * BM, kb * BK, ac2, ac3);
+            tma_load_4d(sA + 8192, &tmA, fb, tc.tm * BM + 64, kb * BK, ac2, ac3);
           } else {
-            tma_load_4d(sA, &tmA, fb, kb * BK, arow, ac2, ac3);
+            tma_load_4d(sA, &tmA, fb, kb * BK, tc.tm * BM, ac2, ac3);
           }
           if (!BRES) {
             const uint32_t sB = sA + L::A_BYTES;
@@ -323,16 +285,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      constexpr uint32_t IDESC = make_idesc_bf16(TILE_M, BN, A_MN, B_MN);
+    if (lane == 0) {
+      constexpr uint32_t IDESC = make_idesc_bf16(BM, BN, A_MN, B_MN);
       uint32_t it = 0;
       int bkey = -1, b_uses = 0;
       bool ok = true;
-      // Commit: this CTA's barrier, or in pair mode the same barrier of both CTAs.
-      auto commit = [&](uint64_t* bar) {
-        if (PAIR) mma_commit_pair(smem_u32(bar));
-        else mma_commit(smem_u32(bar));
-      };
       for (int lt = 0; lt < walk.count && ok; ++lt) {
         const TileCoord tc = walk.at(lt);
         const int buf = lt & 1;
@@ -344,10 +301,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (BRES) {
           const int key = (args.b_b0 ? tc.z0 : 0) * 65536 + (args.b_b1 ? tc.z1 : 0);
           if (key != bkey) {
-            if (b_uses > 0) commit(b_empty);  // old B free once MMAs finish
-            if (!mbar_wait(smem_u32(b_full), b_uses & 1, abort_flag, args.err, args.wait_ns) ||
-                (PAIR && !mbar_wait(smem_u32(peer_b_full), b_uses & 1, abort_flag, args.err,
-                                    args.wait_ns))) {
+            if (b_uses > 0) mma_commit(smem_u32(b_empty));  // old B free once MMAs finish
+            if (!mbar_wait(smem_u32(b_full), b_uses & 1, abort_flag, args.err, args.wait_ns)) {
               ok = false;
               break;
             }
@@ -360,9 +315,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag, args.err,
-                         args.wait_ns) ||
-              (PAIR && !mbar_wait(smem_u32(&peer_full[s]), (it / STAGES) & 1, abort_flag,
-                                  args.err, args.wait_ns))) {
+                         args.wait_ns)) {
             ok = false;
             break;
           }
@@ -375,68 +328,24 @@ __global__ void __launch_bounds__(THREADS, 1)
                                      : make_sw128_desc(sA + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? make_sw128_desc(sB + kk * 2048, 8192, 1024)
                                      : make_sw128_desc(sB + kk * 32, 16, 1024);
-            if (PAIR) mma_f16_pair(dt, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
-            else mma_f16(dt, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_f16(dt, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          commit(&empty[s]);
+          mma_commit(smem_u32(&empty[s]));
         }
         // Arrives once the tile's MMAs are done (also on the abort path, so the teardown
         // can wait for in-flight MMAs before freeing TMEM).
-        commit(&acc_full[buf]);
+        mma_commit(smem_u32(&acc_full[buf]));
         mma_tiles = lt + 1;
-      }
-    } else if (PAIR && lane == 0) {
-      // Second CTA of a pair: forward the completion of its own B and A stages to the
-      // first CTA, whose MMAs read them.
-      const uint32_t r_full = map_to_rank(smem_u32(peer_full), lead);
-      const uint32_t r_bfull = map_to_rank(smem_u32(peer_b_full), lead);
-      uint32_t it = 0;
-      int bkey = -1, b_uses = 0;
-      bool ok = true;
-      for (int lt = 0; lt < walk.count && ok; ++lt) {
-        const TileCoord tc = walk.at(lt);
-        if (BRES) {
-          const int key = (args.b_b0 ? tc.z0 : 0) * 65536 + (args.b_b1 ? tc.z1 : 0);
-          if (key != bkey) {
-            if (!mbar_wait(smem_u32(b_full), b_uses & 1, abort_flag, args.err, args.wait_ns)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_cluster(r_bfull);
-            ++b_uses;
-            bkey = key;
-          }
-        }
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(smem_u32(&full[s]), (it / STAGES) & 1, abort_flag, args.err,
-                         args.wait_ns)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_cluster(r_full + (uint32_t)(s * 8));
-        }
       }
     }
   } else {
     const int ew = warp - 2;
     const int quarter = warp & 3;
     const int part = ew >> 2;  // 0: first half of the tile's columns, 1: second half
-    // Accumulator buffer drained: every thread of this CTA arrives, or in pair mode one lane
-    // per warp arrives on the first CTA's barrier.
-    auto release = [&](int b) {
-      tc_fence_before();
-      if (PAIR) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&acc_empty[b]), lead));
-      } else {
-        mbar_arrive(smem_u32(&acc_empty[b]));
-      }
-    };
     for (int lt = 0; lt < walk.count; ++lt) {
       const int buf = lt & 1;
       const TileCoord tc = walk.at(lt);
-      const int row = tc.tm * TILE_M + row_off + quarter * 32 + lane;
+      const int row = tc.tm * BM + quarter * 32 + lane;
       // the SwiGLU row scale is fetched before the wait, so its latency hides behind it
       const float rsv = (MODE == EPI_SWIGLU && !args.grad && args.rs && row < args.M)
                             ? args.rs[tc.z0 * args.rs0 + tc.z1 * args.rs1 + row]
@@ -457,7 +366,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         float v[HALF];
 #pragma unroll
         for (int j = 0; j < HALF; ++j) v[j] = __uint_as_float(r[j]);
-        release(buf);
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[buf]));
         if (row < args.M) {
           TC* crow = static_cast<TC*>(args.C) + tc.z0 * args.cs0 + tc.z1 * args.cs1 +
                      (long long)row * args.ldc;
@@ -493,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const __nv_bfloat16* dvrow =
             args.dv + tc.z0 * args.ds0 + tc.z1 * args.ds1 + (long long)(live ? row : 0) * args.ldd;
         const int ox = tc.tn * PH + part * QW;
-        const int oy = tc.tm * TILE_M + row_off + quarter * 32;
+        const int oy = tc.tm * BM + quarter * 32;
         const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
         const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
         for (int o = 0; o < 3; ++o) {
@@ -561,7 +471,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_store_commit();
           }
         }
-        release(buf);
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[buf]));
       } else {
         // SWIGLU: phi column p of this tile uses accumulator columns p (A/2) and BN/2 + p (B).
         // Each epilogue warp owns 32 rows x 64 phi columns: two 32-column pieces, the
@@ -574,7 +485,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         constexpr int PH = BN / 2;       // phi columns per tile
         constexpr int QW = PH / 2;       // phi columns per epilogue warp
         const int ox = tc.tn * PH + part * QW;   // first phi column of this warp's box
-        const int oy = tc.tm * TILE_M + row_off + quarter * 32;
+        const int oy = tc.tm * BM + quarter * 32;
         const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
         const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
         const uint32_t ta = lane_addr + (uint32_t)(part * QW), tb = ta + (uint32_t)PH;
@@ -592,7 +503,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           swiglu_piece(ra0, rb0, sc, box, lane, 0);
           tmem_ld_wait_regs(ra1, rb1);
           if (o == nout - 1) {
-            release(buf);
+            tc_fence_before();
+            mbar_arrive(smem_u32(&acc_empty[buf]));
           }
           swiglu_piece(ra1, rb1, sc, box, lane, 4);
           fence_async_smem();
@@ -626,16 +538,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncthreads();
   }
-  if (PAIR) {
-    // The first CTA's MMAs read this CTA's shared memory and write its TMEM: neither is
-    // released before both CTAs got here (the first CTA has waited for its last commit).
-    tc_fence_before();
-    cluster_sync();
-  }
   if (warp == 1) {
     tc_fence_after();
-    if (PAIR) tmem_dealloc_pair(tmem, ACC_COLS);
-    else tmem_dealloc(tmem, ACC_COLS);
+    tmem_dealloc(tmem, ACC_COLS);
   }
 }
 
@@ -714,13 +619,12 @@ bool make_out_map(CUtensorMap* map, void* ptr, int cols, int rows, long long ld,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES,
-          bool PAIR = false>
+template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES>
 ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   CUtensorMap ma, mb;
   OutMaps om;
   if (!make_map(&ma, p.A, p.M, p.K, p.Z0, p.Z1, BM) ||
-      !make_map(&mb, p.B, p.N, p.K, p.Z0, p.Z1, PAIR ? BN / 2 : BN)) {
+      !make_map(&mb, p.B, p.N, p.K, p.Z0, p.Z1, BN)) {
     set_error_message("gemm_umma: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", p.M, p.N, p.K);
     return TTT_ERR_CUDA;
   }
@@ -734,42 +638,23 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
       return TTT_ERR_CUDA;
     }
   }
-  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC, BRES, PAIR>;
-  constexpr int SMEM = Smem<BN, STAGES, BRES, MODE, PAIR>::TOTAL;
+  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC, BRES>;
+  constexpr int SMEM = Smem<BN, STAGES, BRES, MODE>::TOTAL;
   static_assert(SMEM <= 232448, "shared memory budget");
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
       cudaSuccess) {
     set_error_message("gemm_umma: cannot set %d bytes of dynamic shared memory", SMEM);
     return TTT_ERR_CUDA;
   }
-  constexpr int TILE_M = PAIR ? 2 * BM : BM;
   const long long tiles_n = (p.N + BN - 1) / BN;
-  const long long tiles = tiles_n * ((p.M + TILE_M - 1) / TILE_M) * p.Z0 * p.Z1;
+  const long long tiles = tiles_n * ((p.M + BM - 1) / BM) * p.Z0 * p.Z1;
   const int per_sm = (SMEM <= 110 * 1024) ? 2 : 1;
-  // units: CTAs, or CTA pairs in pair mode
-  long long units = (long long)sm_count() * per_sm / (PAIR ? 2 : 1);
-  if (BRES) units = (units / tiles_n) * tiles_n;  // whole groups of n-tile units
-  if (tiles < units) units = tiles;
-  if (units < 1) units = 1;
-  cudaError_t e;
-  if (PAIR) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * units));
-    cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, om, a);
-  } else {
-    kern<<<(unsigned)units, THREADS, SMEM, s>>>(ma, mb, om, a);
-    e = cudaGetLastError();
-  }
+  long long grid = (long long)sm_count() * per_sm;
+  if (BRES) grid = (grid / tiles_n) * tiles_n;  // whole groups of n-tile CTAs
+  if (tiles < grid) grid = tiles;
+  if (grid < 1) grid = 1;
+  kern<<<(unsigned)grid, THREADS, SMEM, s>>>(ma, mb, om, a);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error_message("gemm_umma launch: %s", cudaGetErrorString(e));
     return TTT_ERR_CUDA;
@@ -782,24 +667,9 @@ bool use_bres(const GemmProblem& p, int BN) {
   return BN == 256 && p.K <= 4 * BK && !p.B.mn_major && (p.N + BN - 1) / BN <= sm_count();
 }
 
-// Pair mode for the SwiGLU feature GEMMs (B resident, at least one n tile per pair): opt-in
-// with TTT_PAIR=1. On B200 it measured slower than single CTAs for these shapes (the
-// tensor pipe, not shared-memory bandwidth, sets the pace), so single CTAs are the default.
-bool use_pair(const GemmProblem& p) {
-  const long long tiles_n = (p.N + 255) / 256;
-  const char* e = getenv("TTT_PAIR");
-  return tiles_n <= sm_count() / 2 && e != nullptr && e[0] == '1';
-}
-
 template <int BN, int STAGES, int MODE, typename TC>
 ttt_status dispatch_major(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   constexpr int RES_STAGES = MODE == EPI_SWIGLU ? 4 : 6;
-  constexpr int PAIR_STAGES = 8;   // 64 KB of B + 32 KB staging + 8 x 16 KB of A
-  if (MODE == EPI_SWIGLU && BN == 256 && use_bres(p, BN) && use_pair(p)) {
-    if (p.A.mn_major)
-      return launch_umma<BN, true, false, PAIR_STAGES, MODE, TC, true, true>(p, a, s);
-    return launch_umma<BN, false, false, PAIR_STAGES, MODE, TC, true, true>(p, a, s);
-  }
   if (BN == 256 && use_bres(p, BN)) {
     if (p.A.mn_major) return launch_umma<BN, true, false, RES_STAGES, MODE, TC, true>(p, a, s);
     return launch_umma<BN, false, false, RES_STAGES, MODE, TC, true>(p, a, s);

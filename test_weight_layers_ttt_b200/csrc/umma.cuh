@@ -1,7 +1,6 @@
 // Thin device wrappers over the sm_100a primitives used by the tensor-core kernels:
-// mbarriers, TMA tensor loads (no multicast), tcgen05 MMA / commit / TMEM alloc / loads for
-// one CTA or a CTA pair, and the shared-memory and instruction descriptors of
-// tcgen05.mma kind::f16.
+// mbarriers, TMA tensor loads (one destination CTA), tcgen05 MMA / commit / TMEM alloc / loads,
+// and the shared-memory and instruction descriptors of tcgen05.mma kind::f16.
 //
 // Descriptor bit layouts follow the PTX ISA description of the tcgen05 matrix and
 // instruction descriptors (same field positions as CUTLASS's cute::UMMA unions).
@@ -66,7 +65,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// ------------------------------------------------------------------ TMA (no multicast)
+// ------------------------------------------------------------------ TMA (one destination CTA)
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2, int c3) {
   asm volatile(
@@ -179,66 +178,6 @@ __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&a)[32], uint32_t (&
   tmem_ld_wait();
 #pragma unroll
   for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(a[i]), "+r"(b[i]));
-}
-
-// ------------------------------------------------------------------ CTA pairs (cta_group::2)
-// Rank of this CTA in its cluster.
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// All threads of all CTAs of the cluster (used once after set-up and once before teardown;
-// every thread of both CTAs reaches both on every path).
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-// Shared::cluster address of the object at local shared address `a` in CTA `rank`.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t a, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-  return r;
-}
-// Arrive on an mbarrier given by its shared::cluster address (possibly another CTA's).
-// Relaxed: it orders nothing by itself. Its uses only signal that an earlier, already
-// completed event happened (a TMA load this thread saw land, TMEM loads this warp waited
-// for); a release at cluster scope would wait for all of the SM's outstanding writes.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-// D[tmem of both CTAs] (+)= A[smem of both CTAs, M split] * B[smem of both, N split]^T,
-// issued by one thread of the pair's first CTA.
-__device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Arrive on the mbarrier at local offset `bar` in both CTAs of the pair once every tcgen05
-// operation issued so far by this thread completed.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
-  asm volatile(
-      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], m;\n\t}" ::"r"(bar)
-      : "memory");
 }
 
 // ------------------------------------------------------------------ descriptors

@@ -64,36 +64,6 @@ def test_parallel_matches_oracle(case, order):
     assert rel(host(S0), Sref0) <= tol
 
 
-def test_feature_gemm_on_cta_pairs_and_single_ctas(monkeypatch):
-    """With TTT_PAIR=1 the SwiGLU feature GEMMs run on CTA pairs (tcgen05.mma.cta_group::2,
-    256-row tiles), otherwise on single CTAs. Both engines match the oracle on a ragged case
-    (rows not a multiple of 256 per (b, head), two 256-column n tiles, several pairs per n
-    tile), in both forms, and agree with each other to accumulation-order rounding."""
-    wl, inp = layer_inputs("lm", "bf16", 2, 3, 1000, 64, 200, 256, seed=77, momentum=True)
-    ref, Sref = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
-                                      inp["W2"], inp["W1"], 256)
-    rref, Wref, _ = O.lact_recurrent_batched(
-        inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"], inp["W2"], inp["W1"], 256,
-        renorm=True, alpha=inp["alpha"], ns_steps=5)
-    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
-    alpha = dev(inp["alpha"])
-    got = {}
-    for pair in (True, False):
-        if pair:
-            monkeypatch.setenv("TTT_PAIR", "1")
-        else:
-            monkeypatch.delenv("TTT_PAIR", raising=False)
-        out, S = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, 256)
-        rout, Wf, _ = layer.lact_recurrent_fwd(q, k, v, eta, W0, W2, W1, 256, renorm=True,
-                                               alpha=alpha, ns_steps=5)
-        abi.ttt_last_device_status()
-        assert rel(host(out), ref) <= TOL["bf16"] and rel(host(S), Sref) <= TOL["bf16"]
-        assert rel(host(rout), rref) <= TOL["bf16"]
-        got[pair] = (host(out), host(S), host(rout))
-    for a, b in zip(got[True], got[False]):
-        assert rel(a, b) <= 1e-2
-
-
 @pytest.mark.parametrize("case", [
     # B, H, N, h, m, chunk: odd number of 128-column phi blocks and more tiles than SMs;
     # ragged m (zero-padded phi block, state rows past m) and ragged N
