@@ -190,23 +190,35 @@ __global__ void rec_init_kernel(const float* W0, const float* W2, const float* W
 
 // Column norms (over the input dimension) of the initial weights, per head:
 // tnorm[head] = [ W0 columns (m) | W1 columns (h) | W2 columns (m) ].
+// grid (ceil((2m + h) / 32), H), block (32, 8): threadIdx.x takes one of 32 consecutive
+// columns (coalesced rows), threadIdx.y every 8th row of it; the 8 partial sums (fp64) are
+// added in shared memory.
 __global__ void col_norms_kernel(const float* W0, const float* W2, const float* W1, int H, int h,
                                  int m, float* tnorm) {
-  const int per = 2 * m + h;
-  TTT_GRID_LOOP(idx, (long long)per * H) {
-    const int hd = (int)(idx / per), c = (int)(idx - (long long)hd * per);
-    const long long hm = (long long)h * m;
-    double ss = 0.0;
-    if (c < m) {
-      for (int r = 0; r < h; ++r) { const float w = W0[hd * hm + (long long)r * m + c]; ss += (double)w * w; }
-    } else if (c < m + h) {
-      const int cc = c - m;
-      for (int r = 0; r < m; ++r) { const float w = W1[hd * hm + (long long)r * h + cc]; ss += (double)w * w; }
-    } else {
-      const int cc = c - m - h;
-      for (int r = 0; r < h; ++r) { const float w = W2[hd * hm + (long long)r * m + cc]; ss += (double)w * w; }
+  __shared__ double part[8][33];
+  const int per = 2 * m + h, hd = blockIdx.y;
+  const int c = blockIdx.x * 32 + threadIdx.x, ty = threadIdx.y;
+  const long long hm = (long long)h * m;
+  double ss = 0.0;
+  if (c < per) {
+    const float* base;
+    int rows, ld;
+    if (c < m) { base = W0 + hd * hm + c; rows = h; ld = m; }
+    else if (c < m + h) { base = W1 + hd * hm + (c - m); rows = m; ld = h; }
+    else { base = W2 + hd * hm + (c - m - h); rows = h; ld = m; }
+#pragma unroll 4
+    for (int r = ty; r < rows; r += 8) {
+      const float w = base[(long long)r * ld];
+      ss += (double)w * w;
     }
-    tnorm[idx] = (float)sqrt(ss);
+  }
+  part[ty][threadIdx.x] = ss;
+  __syncthreads();
+  if (ty == 0 && c < per) {
+    double t = 0.0;
+#pragma unroll
+    for (int y = 0; y < 8; ++y) t += part[y][threadIdx.x];
+    tnorm[(long long)hd * per + c] = (float)sqrt(t);
   }
 }
 
@@ -755,8 +767,9 @@ cudaError_t rec_init(int ot, const float* W0, const float* W2, const float* W1, 
 
 cudaError_t col_norms(const float* W0, const float* W2, const float* W1, int H, int h, int m,
                       float* tnorm, cudaStream_t s) {
-  col_norms_kernel<<<grid_for((long long)(2 * m + h) * H, 128), 128, 0, s>>>(W0, W2, W1, H, h, m,
-                                                                             tnorm);
+  if (H <= 0) return cudaSuccess;
+  col_norms_kernel<<<dim3((2 * m + h + 31) / 32, H), dim3(32, 8), 0, s>>>(W0, W2, W1, H, h, m,
+                                                                          tnorm);
   return cudaGetLastError();
 }
 

@@ -742,8 +742,11 @@ struct RecBufs {
   float* M_all;   // momentum, same layout
   float* U;       // update, same layout
   float* tnorm;   // initial column norms per head
-  void* Wk;       // [BH, 2*mpad, h] blocked [W0^T ; W2^T] operand
-  void* W1o;      // [BH, m, h] W1 operand
+  // Two copies of the bf16/fp32 operands, alternating by chunk: the weights after update c
+  // are in copy (c + 1) % 2 (the initial weights in copy 0), so the apply of one chunk can
+  // read its copy while the next update writes the other.
+  void* Wk[2];    // [BH, 2*mpad, h] blocked [W0^T ; W2^T] operand
+  void* W1o[2];   // [BH, m, h] W1 operand
   void* Dv;       // [BH, chunk, m] V W1^T
   void* P;        // [BH, chunk, m] phi * eta
   void* E2;       // [BH, chunk, m] d * silu(A)
@@ -769,6 +772,32 @@ int choose_splits(const ttt_desc& d, long long L) {
   return (int)best;
 }
 
+// A second stream (and its events) per host thread and device for the recurrent form's
+// applies; created on first use. Null if creation fails: the applies then stay on the
+// caller's stream.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t gate = nullptr, applied = nullptr, joined = nullptr;
+  bool ok = false;
+};
+SideStream* side_stream() {
+  constexpr int kMaxDev = 64;
+  thread_local SideStream res[kMaxDev];
+  thread_local bool tried[kMaxDev] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  SideStream& r = res[dev];
+  if (!tried[dev]) {
+    tried[dev] = true;
+    r.ok = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking) == cudaSuccess &&
+           cudaEventCreateWithFlags(&r.gate, cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&r.applied, cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&r.joined, cudaEventDisableTiming) == cudaSuccess;
+    if (!r.ok) cudaGetLastError();
+  }
+  return r.ok ? &r : nullptr;
+}
+
 size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
   Carve cv(base);
   const size_t os = d.dtype == TTT_DTYPE_BF16 ? 2 : 4;
@@ -779,8 +808,10 @@ size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
   b.M_all = d.momentum ? cv.take_n<float>(BH * 3 * hm) : nullptr;
   b.U = cv.take_n<float>(BH * 3 * hm);
   b.tnorm = cv.take_n<float>((long long)d.H * (2 * d.m + d.h));
-  b.Wk = cv.take(os * BH * 2 * padded_m(d.m) * d.h);
-  b.W1o = cv.take(os * BH * hm);
+  for (int i = 0; i < 2; ++i) {
+    b.Wk[i] = cv.take(os * BH * 2 * padded_m(d.m) * d.h);
+    b.W1o[i] = cv.take(os * BH * hm);
+  }
   b.Dv = cv.take(os * rows * d.m);
   b.P = cv.take(os * rows * d.m);
   b.E2 = cv.take(os * rows * d.m);
@@ -795,7 +826,7 @@ size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
 
 // Features of tokens [t0, t0 + Lc) of every (b, head) against that (b, head)'s own blocked
 // weights; rows of the outputs are chunk-local ([BH, chunk, m]).
-SwigluGemm rec_features(const ttt_desc& d, const void* X, const RecBufs& b, long long t0,
+SwigluGemm rec_features(const ttt_desc& d, const void* X, const void* Wk, long long t0,
                         long long Lc, void* out) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, mp = padded_m(d.m);
@@ -804,29 +835,38 @@ SwigluGemm rec_features(const ttt_desc& d, const void* X, const RecBufs& b, long
   GemmProblem& p = g.gemm;
   p.M = (int)Lc; p.N = (int)(2 * mp); p.K = d.h; p.Z0 = (int)BH; p.Z1 = 1;
   p.A = {static_cast<const char*>(X) + t0 * h * dtype_size(ot), ot, false, h, N * h, 0};
-  p.B = {b.Wk, ot, false, h, 2 * mp * h, 0};
+  p.B = {Wk, ot, false, h, 2 * mp * h, 0};
   p.C = {out, ot, m, L * m, 0};
   g.n_valid = d.m;
   return g;
 }
 
+// Outputs of tokens [t0, t0 + Lc) with the weights in operand copy `bi`.
 ttt_status rec_apply(const ttt_desc& d, const void* q, void* out, long long t0, long long Lc,
-                     const RecBufs& b, cudaStream_t s) {
+                     const RecBufs& b, int bi, cudaStream_t s) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const size_t es = dtype_size(ot);
   const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, L = d.chunk;
-  TTT_TRY(run_swiglu("gemm_features_q", rec_features(d, q, b, t0, Lc, b.phiQ), s));
+  TTT_TRY(run_swiglu("gemm_features_q", rec_features(d, q, b.Wk[bi], t0, Lc, b.phiQ), s));
   GemmProblem o;
   o.M = (int)Lc; o.N = d.h; o.K = d.m; o.Z0 = (int)BH; o.Z1 = 1;
   o.A = {b.phiQ, ot, false, m, L * m, 0};
-  o.B = {b.W1o, ot, true, h, m * h, 0};
+  o.B = {b.W1o[bi], ot, true, h, m * h, 0};
   o.C = {static_cast<char*>(out) + t0 * h * es, ot, h, N * h, 0};
   return run_gemm("gemm_output", o, s);
 }
 
+// One gradient step on chunk c (tokens [t0, t0 + Lc)) from the weights in operand copy
+// `bin`; the updated operands are written to copy `bout`. `gate` (if not null) is recorded
+// on `s` where work on another stream may best start alongside: just before the
+// Newton-Schulz kernel when that kernel runs one CTA per matrix (it leaves most SMs idle),
+// else at the start of the update.
 ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const float* eta,
                       const float* alpha, int c, long long t0, long long Lc, const RecBufs& b,
-                      cudaStream_t s) {
+                      int bin, int bout, cudaEvent_t gate, cudaStream_t s) {
+  const int ot_ = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const bool ns_gate = d.ns_steps > 0 && ns_path(ot_, d.h, d.m) == NS_TENSOR_CTA;
+  if (gate && !ns_gate) TTT_CUDA(cudaEventRecord(gate, s));
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const size_t es = dtype_size(ot);
   const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, hm = h * m;
@@ -838,12 +878,12 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
     GemmProblem g;
     g.M = (int)Lc; g.N = d.m; g.K = d.h; g.Z0 = (int)BH; g.Z1 = 1;
     g.A = {static_cast<const char*>(v) + t0 * h * es, ot, false, h, N * h, 0};
-    g.B = {b.W1o, ot, false, h, m * h, 0};
+    g.B = {b.W1o[bin], ot, false, h, m * h, 0};
     g.C = {b.Dv, ot, m, L * m, 0};
     TTT_TRY(run_gemm("gemm_v_w1t", g, s));
   }
   // [A | B] = K_c [W0 | W2] -> P = phi eta (and E2, E0 for the input-side matrices)
-  SwigluGemm f = rec_features(d, k, b, t0, Lc, b.P);
+  SwigluGemm f = rec_features(d, k, b.Wk[bin], t0, Lc, b.P);
   f.rowscale = eta + t0;
   f.rs0 = N;
   f.rs1 = 0;
@@ -881,11 +921,13 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
   }
   TTT_OP("reduce_momentum", rec_reduce(b.partials, sp, b.U, d.momentum ? b.M_all : nullptr,
                                       alpha, (int)C, c, (int)BH, d.h, d.m, mask, s));
-  if (d.ns_steps > 0)
+  if (d.ns_steps > 0) {
+    if (gate && ns_gate) TTT_CUDA(cudaEventRecord(gate, s));
     TTT_TRY(run_ns(ot, b.U, (int)BH, ns_layout_weights(d.h, d.m, mask), d.ns_steps,
                    b.ns, s));
+  }
   TTT_OP("step_renorm", rec_step(b.W_all, b.U, b.tnorm, (int)BH, d.H, d.h, d.m, mask, d.sign,
-                                  d.renorm, b.Wk, b.W1o, ot, s));
+                                  d.renorm, b.Wk[bout], b.W1o[bout], ot, s));
   return TTT_OK;
 }
 
@@ -1079,18 +1121,64 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   plan_recurrent(d, workspace, b);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
-  TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1o,
+  TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1o[0],
                               d.momentum ? M_io : nullptr, b.M_all, d.momentum, s));
-  TTT_OP("prep_weights", prep_wk_blocked(ot, W0, W2, b.Wk, (int)BH, d.H, d.h, d.m, 0, s));
+  TTT_OP("prep_weights", prep_wk_blocked(ot, W0, W2, b.Wk[0], (int)BH, d.H, d.h, d.m, 0, s));
+  {  // both operand copies start from the initial weights (a matrix outside the update mask
+     // is never rewritten)
+    const size_t os = ot == DT_BF16 ? 2 : 4;
+    TTT_CUDA(cudaMemcpyAsync(b.Wk[1], b.Wk[0], os * BH * 2 * padded_m(d.m) * d.h,
+                             cudaMemcpyDeviceToDevice, s));
+    TTT_CUDA(cudaMemcpyAsync(b.W1o[1], b.W1o[0], os * BH * d.h * d.m, cudaMemcpyDeviceToDevice,
+                             s));
+  }
   if (d.renorm) TTT_OP("col_norms", col_norms(W0, W2, W1, d.H, d.h, d.m, b.tnorm, s));
   const long long N = d.N, L = d.chunk;
-  int c = 0;
-  for (long long t0 = 0; t0 < N; t0 += L, ++c) {
-    const long long Lc = (t0 + L <= N) ? L : N - t0;
-    if (d.order == TTT_ORDER_APPLY_UPDATE) TTT_TRY(rec_apply(d, q, out, t0, Lc, b, s));
-    TTT_TRY(rec_update(d, k, v, eta, alpha, c, t0, Lc, b, s));
-    if (d.order == TTT_ORDER_UPDATE_APPLY) TTT_TRY(rec_apply(d, q, out, t0, Lc, b, s));
+  // The apply of chunk c - 1 (update -> apply order; of chunk c in apply -> update order)
+  // and the update of chunk c read the same operand copy and write disjoint buffers, so the
+  // applies run on a second stream, each released by the gate event of update c (at its
+  // Newton-Schulz kernel, which leaves most SMs idle, or at its start); each update waits
+  // for the apply that last read the operand copy it is about to overwrite.
+  SideStream* side = side_stream();
+  const bool fork = side != nullptr && N > L;
+  const bool ua = d.order == TTT_ORDER_UPDATE_APPLY;
+  cudaStream_t sa = fork ? side->s : s;
+  auto chunks = [&]() -> ttt_status {
+    int c = 0;
+    for (long long t0 = 0; t0 < N; t0 += L, ++c) {
+      const long long Lc = (t0 + L <= N) ? L : N - t0;
+      const int bin = c & 1, bout = (c + 1) & 1;
+      // update c writes copy bout; the apply enqueued in the previous iteration read it
+      if (fork && (ua ? c >= 2 : c >= 1)) TTT_CUDA(cudaStreamWaitEvent(s, side->applied, 0));
+      TTT_TRY(rec_update(d, k, v, eta, alpha, c, t0, Lc, b, bin, bout,
+                         fork ? side->gate : nullptr, s));
+      // the apply that reads copy bin (the weights after update c - 1): of chunk c - 1 in
+      // update -> apply order, of chunk c in apply -> update order
+      if (ua && c == 0) continue;
+      const long long ta = ua ? t0 - L : t0, La = ua ? L : Lc;
+      if (fork) TTT_CUDA(cudaStreamWaitEvent(sa, side->gate, 0));
+      TTT_TRY(rec_apply(d, q, out, ta, La, b, bin, sa));
+      if (fork) TTT_CUDA(cudaEventRecord(side->applied, sa));
+    }
+    if (ua && c > 0) {   // the last chunk's apply, after the last update
+      const long long ta = (long long)(c - 1) * L;
+      if (fork) {
+        TTT_CUDA(cudaEventRecord(side->gate, s));
+        TTT_CUDA(cudaStreamWaitEvent(sa, side->gate, 0));
+      }
+      TTT_TRY(rec_apply(d, q, out, ta, N - ta, b, c & 1, sa));
+    }
+    return TTT_OK;
+  };
+  const ttt_status st = chunks();
+  // join on every path: the caller's stream is ordered after every apply
+  if (fork) {
+    const cudaError_t e1 = cudaEventRecord(side->joined, sa);
+    const cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(s, side->joined, 0) : e1;
+    if (st == TTT_OK && e2 != cudaSuccess)
+      return fail(TTT_ERR_CUDA, "joining the apply stream: %s", cudaGetErrorString(e2));
   }
+  TTT_TRY(st);
   if (W0_out || W2_out || W1_out || (d.momentum && M_io))
     TTT_OP("rec_finish", rec_finish(b.W_all, (int)BH, d.h, d.m, W0_out, W2_out, W1_out, b.M_all,
                                     d.momentum ? M_io : nullptr, s));
