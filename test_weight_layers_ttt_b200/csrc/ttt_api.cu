@@ -777,7 +777,7 @@ int choose_splits(const ttt_desc& d, long long L) {
 // caller's stream.
 struct SideStream {
   cudaStream_t s = nullptr;
-  cudaEvent_t gate = nullptr, applied = nullptr, joined = nullptr;
+  cudaEvent_t gate = nullptr, applied = nullptr, joined = nullptr, feat = nullptr, g1 = nullptr;
   bool ok = false;
 };
 SideStream* side_stream() {
@@ -792,7 +792,9 @@ SideStream* side_stream() {
     r.ok = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking) == cudaSuccess &&
            cudaEventCreateWithFlags(&r.gate, cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&r.applied, cudaEventDisableTiming) == cudaSuccess &&
-           cudaEventCreateWithFlags(&r.joined, cudaEventDisableTiming) == cudaSuccess;
+           cudaEventCreateWithFlags(&r.joined, cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&r.feat, cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&r.g1, cudaEventDisableTiming) == cudaSuccess;
     if (!r.ok) cudaGetLastError();
   }
   return r.ok ? &r : nullptr;
@@ -857,13 +859,15 @@ ttt_status rec_apply(const ttt_desc& d, const void* q, void* out, long long t0, 
 }
 
 // One gradient step on chunk c (tokens [t0, t0 + Lc)) from the weights in operand copy
-// `bin`; the updated operands are written to copy `bout`. `gate` (if not null) is recorded
-// on `s` where work on another stream may best start alongside: just before the
+// `bin`; the updated operands are written to copy `bout`. With a second stream `side`, the
+// W1 gradient runs there alongside the W0 / W2 gradients, and `side->gate` is recorded on
+// `s` where work on the second stream may best start alongside the update: just before the
 // Newton-Schulz kernel when that kernel runs one CTA per matrix (it leaves most SMs idle),
 // else at the start of the update.
 ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const float* eta,
                       const float* alpha, int c, long long t0, long long Lc, const RecBufs& b,
-                      int bin, int bout, cudaEvent_t gate, cudaStream_t s) {
+                      int bin, int bout, SideStream* side, cudaStream_t s) {
+  const cudaEvent_t gate = side ? side->gate : nullptr;
   const int ot_ = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const bool ns_gate = d.ns_steps > 0 && ns_path(ot_, d.h, d.m) == NS_TENSOR_CTA;
   if (gate && !ns_gate) TTT_CUDA(cudaEventRecord(gate, s));
@@ -901,6 +905,13 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
   const int sp = (Lc == d.chunk) ? b.splits : 1;
   const long long Ks = Lc / sp;
   const long long tot = BH * 3 * hm;
+  const bool g1_side = side && (mask & TTT_UPDATE_W1) &&
+                       (mask & (TTT_UPDATE_W0 | TTT_UPDATE_W2));
+  const cudaStream_t s1 = g1_side ? side->s : s;
+  if (g1_side) {
+    TTT_CUDA(cudaEventRecord(side->feat, s));
+    TTT_CUDA(cudaStreamWaitEvent(s1, side->feat, 0));
+  }
   if (mask & TTT_UPDATE_W1) {  // dW1 = -(phi eta)^T V
     GemmProblem g;
     g.M = d.m; g.N = d.h; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
@@ -908,8 +919,9 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
     g.B = {static_cast<const char*>(v) + t0 * h * es, ot, true, h, N * h, Ks * h};
     g.C = {b.partials + hm, DT_F32, h, 3 * hm, tot};
     g.alpha = -1.0f;
-    TTT_TRY(run_gemm("gemm_grad_w1", g, s));
+    TTT_TRY(run_gemm("gemm_grad_w1", g, s1));
   }
+  if (g1_side) TTT_CUDA(cudaEventRecord(side->g1, s1));
   for (int pidx = 0; pidx <= 2; pidx += 2) {  // dW0 = K^T E0, dW2 = K^T E2
     if (!(mask & (pidx == 0 ? TTT_UPDATE_W0 : TTT_UPDATE_W2))) continue;
     GemmProblem g;
@@ -919,6 +931,7 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
     g.C = {b.partials + pidx * hm, DT_F32, m, 3 * hm, tot};
     TTT_TRY(run_gemm(pidx == 0 ? "gemm_grad_w0" : "gemm_grad_w2", g, s));
   }
+  if (g1_side) TTT_CUDA(cudaStreamWaitEvent(s, side->g1, 0));
   TTT_OP("reduce_momentum", rec_reduce(b.partials, sp, b.U, d.momentum ? b.M_all : nullptr,
                                       alpha, (int)C, c, (int)BH, d.h, d.m, mask, s));
   if (d.ns_steps > 0) {
@@ -1150,8 +1163,8 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
       const int bin = c & 1, bout = (c + 1) & 1;
       // update c writes copy bout; the apply enqueued in the previous iteration read it
       if (fork && (ua ? c >= 2 : c >= 1)) TTT_CUDA(cudaStreamWaitEvent(s, side->applied, 0));
-      TTT_TRY(rec_update(d, k, v, eta, alpha, c, t0, Lc, b, bin, bout,
-                         fork ? side->gate : nullptr, s));
+      TTT_TRY(rec_update(d, k, v, eta, alpha, c, t0, Lc, b, bin, bout, fork ? side : nullptr,
+                         s));
       // the apply that reads copy bin (the weights after update c - 1): of chunk c - 1 in
       // update -> apply order, of chunk c in apply -> update order
       if (ua && c == 0) continue;
