@@ -391,7 +391,10 @@ def _roofline(table, wl, peaks, form, steps):
         bound, step_work = kernel_work(name, wl, form)
         if bound is None:
             continue
-        work = step_work / (e["launches"] / steps)
+        # the training step runs the forward kernels once in the forward pass and again in
+        # the backward pass (recomputed features, states): each launch does the forward
+        # form's whole per-step work
+        work = step_work if form == "train" else step_work / (e["launches"] / steps)
         secs = e["ms_avg"] / 1e3
         if bound == "tensor":
             achieved = work / secs / 1e12

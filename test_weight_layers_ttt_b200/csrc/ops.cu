@@ -494,8 +494,9 @@ __global__ void momentum_scan_kernel(float* D, const float* alpha, int BH, int C
 
 // grid (ceil(max cols / 32), 3, BH), block (32, 32), dynamic shared memory 32 x (R + 1)
 // floats: one column per threadIdx.x, rows strided by 32 over threadIdx.y. Three phases,
-// each with all threads' loads independent: column sums of (W - sign U)^2; the new values
-// written to the fp32 master and W1o (coalesced along columns) and kept in shared memory;
+// each with all threads' loads independent: W - sign U into shared memory and its column
+// sums of squares; the rescaled values written to the fp32 master and W1o (coalesced along
+// columns) and kept in shared memory;
 // for W0 / W2 the shared-memory columns written out as rows of the blocked operand Wk
 // (coalesced along the input dimension).
 template <typename OT>
@@ -518,11 +519,13 @@ __global__ void __launch_bounds__(1024) rec_step_kernel(float* W_all, const floa
   float* w = W_all + (long long)bh * 3 * hm + p * hm;
   const float* u = U + (long long)bh * 3 * hm + p * hm;
   const float sg = (float)sign;
+  float* mycol = colbuf + (long long)tx * (R + 1);
   float ss = 0.0f;
   if (live) {
 #pragma unroll 4
     for (int r = ty; r < R; r += 32) {
       const float v = w[(long long)r * Cc + c] - sg * u[(long long)r * Cc + c];
+      mycol[r] = v;
       ss = fmaf(v, v, ss);
     }
   }
@@ -536,12 +539,11 @@ __global__ void __launch_bounds__(1024) rec_step_kernel(float* W_all, const floa
     const float* tn = tnorm + (long long)(bh % H) * (2 * m + h) + (p == 0 ? 0 : p == 1 ? m : m + h);
     scale = tn[c] / sqrtf(tot);
   }
-  float* mycol = colbuf + (long long)tx * (R + 1);
-  if (live) {
+  if (live) {   // each thread rescales the values it computed itself (same rows)
 #pragma unroll 4
     for (int r = ty; r < R; r += 32) {
       const long long o = (long long)r * Cc + c;
-      const float v = (w[o] - sg * u[o]) * scale;
+      const float v = mycol[r] * scale;
       w[o] = v;
       if (p == 1) W1o[(long long)bh * hm + o] = from_f32<OT>(v);
       else mycol[r] = v;

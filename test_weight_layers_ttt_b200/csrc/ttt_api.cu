@@ -758,15 +758,17 @@ struct RecBufs {
 };
 
 // Token splits of the gradient reductions: the largest power of two that divides the chunk
-// length, keeps split lengths a multiple of 64 (and >= 256), and keeps the grid of the
-// gradient GEMMs within about two CTAs per SM.
+// length, keeps split lengths a multiple of 64 (and >= 256), and keeps the grid of each
+// gradient GEMM within one CTA per SM (every split writes a full fp32 partial that the
+// reduction reads back, so more splits than one wave costs more HBM traffic than it
+// saves in GEMM time).
 int choose_splits(const ttt_desc& d, long long L) {
   const long long BH = (long long)d.B * d.H;
   const long long tiles = BH * ((d.m + 127) / 128) * ((d.h + 255) / 256);
   long long best = 1;
   for (long long sp = 2; sp <= 64; sp *= 2) {
     if (L % sp != 0 || (L / sp) % 64 != 0 || L / sp < 256) break;
-    if (tiles * sp > 2 * 148) break;
+    if (tiles * sp > 148) break;
     best = sp;
   }
   return (int)best;
