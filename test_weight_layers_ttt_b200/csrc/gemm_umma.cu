@@ -406,6 +406,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int oy = tc.tm * BM + quarter * 32;
         const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
         const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
+        // this row's 64 dv values of the tile (both 32-column halves), loaded once for the
+        // two outputs that use them, all eight 16-byte loads in flight together
+        uint4 dvq[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int col = ox + (j >> 2) * 32 + (j & 3) * 8;
+          dvq[j] = (live && (args.C2 || args.C3) && col + 8 <= args.n_valid)
+                       ? *reinterpret_cast<const uint4*>(dvrow + col)
+                       : make_uint4(0u, 0u, 0u, 0u);
+        }
         for (int o = 0; o < 3; ++o) {
           if ((o == 0 && args.skip_out1) || (o == 1 && !args.C2) || (o == 2 && !args.C3))
             continue;
@@ -417,23 +427,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             tmem_ld32(lane_addr + (uint32_t)(part * QW + hh * 32), ra);
             tmem_ld32(lane_addr + (uint32_t)(PH + part * QW + hh * 32), rb);
             tmem_ld_wait();
-            const int col0 = ox + hh * 32;
             float dvv[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dvv[j] = 0.0f;
-            if (o > 0 && live) {
+            for (int j = 0; j < 32; j += 8) {
+              const uint4 u = dvq[hh * 4 + j / 8];
+              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                if (col0 + j + 8 <= args.n_valid) {
-                  const uint4 u = *reinterpret_cast<const uint4*>(dvrow + col0 + j);
-                  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    const float2 f = __bfloat1622float2(h2[q]);
-                    dvv[j + 2 * q] = f.x;
-                    dvv[j + 2 * q + 1] = f.y;
-                  }
-                }
+              for (int q = 0; q < 4; ++q) {
+                const float2 f = __bfloat1622float2(h2[q]);
+                dvv[j + 2 * q] = f.x;
+                dvv[j + 2 * q + 1] = f.y;
               }
             }
             uint32_t pk[16];
