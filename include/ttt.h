@@ -256,6 +256,14 @@ ttt_status ttt_la_parallel_fwd_noalloc(const ttt_desc* desc, const void* q, cons
  *              part [m,h], then W2 part [h,m]); read as the initial momentum and
  *              overwritten with the final one. NULL means "start from 0, discard".
  *   workspace  >= ttt_workspace_bytes(desc, TTT_PATH_RECURRENT) bytes, 256-byte aligned
+ *
+ * Streams: with more than one chunk, part of the work (each chunk's outputs and the W1
+ * gradient) runs on a second stream that the library creates once per host thread and
+ * device; it forks from `stream` with events and is joined back into `stream` before the
+ * call returns, on error paths too. Everything the call enqueues is therefore ordered
+ * before later work on `stream`, and the call can be captured into a CUDA graph from
+ * `stream` (the fork and join become graph dependencies). If the second stream cannot be
+ * created, all work stays on `stream`.
  */
 ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const void* k,
                                   const void* v, const float* eta, const float* alpha,
