@@ -392,6 +392,37 @@ def test_recurrent_resume_equals_full_run():
         assert rel(host(x), host(y)) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("order", ["update_apply", "apply_update"])
+def test_recurrent_graph_replay_equals_eager(order):
+    """The recurrent form forks its applies and the W1 gradient onto a second stream and
+    joins it before returning; captured into a CUDA graph from the caller's stream and
+    replayed, it gives the eager call's results bit for bit (no kernel depends on the
+    interleaving of the two streams). NS on the one-CTA path, momentum, renorm, 5 chunks."""
+    wl, inp = layer_inputs("lm", "bf16", 1, 2, 1280, 128, 256, 256, seed=23, momentum=True)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    alpha = dev(inp["alpha"])
+    kw = dict(order=order, renorm=True, alpha=alpha, ns_steps=5)
+    ref, Wr, _ = layer.lact_recurrent_fwd(q, k, v, eta, W0, W2, W1, 256, **kw)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer.lact_recurrent_fwd(q, k, v, eta, W0, W2, W1, 256, **kw)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        out, Wf, _ = layer.lact_recurrent_fwd(q, k, v, eta, W0, W2, W1, 256, **kw)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    abi.ttt_last_device_status()
+    assert torch.equal(out, ref)
+    for x, y in zip(Wf, Wr):
+        assert torch.equal(x, y)
+    del g
+
+
 # ----------------------------------------------------------------------------- In-Place form
 def test_inplace_shaped_update_matches_oracle():
     """q = k = H, W0 = Wg^T, W2 = Wu^T given as [m,h]; W1 = W_down^T given as [h,m];
