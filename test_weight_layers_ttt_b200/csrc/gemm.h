@@ -20,6 +20,12 @@ struct GemmOperand {
   int dtype = DT_F32;
   bool mn_major = false;  // false: k contiguous ("K-major"); true: the row index contiguous
   long long ld = 0, s0 = 0, s1 = 0;
+  // Split-precision operand (tensor-core engine only): the logical K = 3 * k0 is three
+  // k0-wide thirds, [hi hi lo] (hilo 1) or [hi lo hi] (hilo 2), of a matrix stored once as
+  // [hi | lo] along K (2 * k0 wide); k0 a multiple of 64. The engine reads each k-block
+  // from its third's copy, so hi*hi + hi*lo + lo*hi needs no duplicated copies.
+  int hilo = 0;
+  long long k0 = 0;
 };
 
 struct GemmOut {

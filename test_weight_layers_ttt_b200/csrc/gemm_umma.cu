@@ -43,6 +43,7 @@ enum EpiMode : int { EPI_STORE = 0, EPI_SWIGLU = 1 };
 struct UArgs {
   int M, N, K, Z0, Z1;
   int a_b0, a_b1, b_b0, b_b1;  // 1 = operand uses that batch coordinate
+  int a_hilo, a_k0, b_hilo, b_k0;  // split-precision operands (GemmOperand::hilo)
   void* C; long long ldc, cs0, cs1;
   const float* Cin; long long ldi, is0, is1;
   float alpha, beta;
@@ -110,6 +111,17 @@ __device__ __forceinline__ void store_vals(__nv_bfloat16* dst, const float* v, i
 struct TileCoord {
   int tm, tn, z0, z1;
 };
+
+// K coordinate, in the operand's buffer, of k-block kb: kb * BK, or for a split-precision
+// operand (logical K = three k0-wide thirds, stored once as [hi | lo]) the block's offset
+// inside its third plus k0 when that third is the lo copy.
+__device__ __forceinline__ int kcoord(int kb, int hilo, int k0) {
+  const int k = kb * BK;
+  if (!hilo) return k;
+  const int third = k / k0, kk = k - third * k0;
+  const bool lo = hilo == 1 ? third == 2 : third == 1;
+  return kk + (lo ? k0 : 0);
+}
 
 __device__ __forceinline__ TileCoord decode_tile(int t, int tiles_n, int tiles_mn, int Z0) {
   TileCoord c;
@@ -240,12 +252,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_arrive_expect_tx(bb, KB * L::B_BYTES);
           for (int kb = 0; kb < KB; ++kb) {
             const uint32_t sB = smem_base + kb * L::B_BYTES;
+            const int kB = kcoord(kb, args.b_hilo, args.b_k0);
             if (B_MN) {
 #pragma unroll
               for (int q = 0; q < BN / 64; ++q)
-                tma_load_4d(sB + q * 8192, &tmB, bb, tc.tn * BN + 64 * q, kb * BK, bc2, bc3);
+                tma_load_4d(sB + q * 8192, &tmB, bb, tc.tn * BN + 64 * q, kB, bc2, bc3);
             } else {
-              tma_load_4d(sB, &tmB, bb, kb * BK, tc.tn * BN, bc2, bc3);
+              tma_load_4d(sB, &tmB, bb, kB, tc.tn * BN, bc2, bc3);
             }
           }
           ++b_loads;
@@ -263,20 +276,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t fb = smem_u32(&full[s]);
           mbar_arrive_expect_tx(fb, L::STAGE);
           const uint32_t sA = ring_base + s * L::STAGE;
+          const int kA = kcoord(kb, args.a_hilo, args.a_k0);
           if (A_MN) {
-            tma_load_4d(sA, &tmA, fb, tc.tm * BM, kb * BK, ac2, ac3);
-            tma_load_4d(sA + 8192, &tmA, fb, tc.tm * BM + 64, kb * BK, ac2, ac3);
+            tma_load_4d(sA, &tmA, fb, tc.tm * BM, kA, ac2, ac3);
+            tma_load_4d(sA + 8192, &tmA, fb, tc.tm * BM + 64, kA, ac2, ac3);
           } else {
-            tma_load_4d(sA, &tmA, fb, kb * BK, tc.tm * BM, ac2, ac3);
+            tma_load_4d(sA, &tmA, fb, kA, tc.tm * BM, ac2, ac3);
           }
           if (!BRES) {
             const uint32_t sB = sA + L::A_BYTES;
+            const int kB = kcoord(kb, args.b_hilo, args.b_k0);
             if (B_MN) {
 #pragma unroll
               for (int q = 0; q < BN / 64; ++q)
-                tma_load_4d(sB + q * 8192, &tmB, fb, tc.tn * BN + 64 * q, kb * BK, bc2, bc3);
+                tma_load_4d(sB + q * 8192, &tmB, fb, tc.tn * BN + 64 * q, kB, bc2, bc3);
             } else {
-              tma_load_4d(sB, &tmB, fb, kb * BK, tc.tn * BN, bc2, bc3);
+              tma_load_4d(sB, &tmB, fb, kB, tc.tn * BN, bc2, bc3);
             }
           }
           issued = it + 1;
@@ -581,6 +596,7 @@ bool make_map(CUtensorMap* map, const GemmOperand& op, int rows, int K, int Z0, 
   auto fn = encode_fn();
   if (!fn) return false;
   const bool mn = op.mn_major;
+  if (op.hilo) K = (int)(2 * op.k0);   // the buffer holds [hi | lo] along K
   cuuint64_t dims[4];
   cuuint64_t strides[3];
   cuuint32_t box[4];
@@ -704,6 +720,7 @@ UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait
   UArgs a{};
   a.M = p.M; a.N = p.N; a.K = p.K; a.Z0 = p.Z0; a.Z1 = p.Z1;
   a.a_b0 = p.A.s0 != 0; a.a_b1 = p.A.s1 != 0; a.b_b0 = p.B.s0 != 0; a.b_b1 = p.B.s1 != 0;
+  a.a_hilo = p.A.hilo; a.a_k0 = (int)p.A.k0; a.b_hilo = p.B.hilo; a.b_k0 = (int)p.B.k0;
   a.C = p.C.ptr; a.ldc = p.C.ld; a.cs0 = p.C.s0; a.cs1 = p.C.s1;
   a.Cin = p.beta != 0.0f ? p.Cin.ptr : nullptr;
   a.ldi = p.Cin.ld; a.is0 = p.Cin.s0; a.is1 = p.Cin.s1;
@@ -718,6 +735,10 @@ UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait
 bool umma_supported(const GemmProblem& p) {
   if (!operand_ok(p.A) || !operand_ok(p.B)) return false;
   if (p.K <= 0 || p.M <= 0 || p.N <= 0) return false;
+  for (const GemmOperand* o : {&p.A, &p.B})
+    if (o->hilo && (o->hilo > 2 || o->k0 <= 0 || o->k0 % BK != 0 || p.K != 3 * o->k0 ||
+                    o->k0 > (1LL << 30)))
+      return false;
   if ((long long)p.Z0 * p.Z1 * ((p.M + BM - 1) / BM) * ((p.N + 63) / 64) > (1LL << 31)) return false;
   if (p.beta != 0.0f && !p.Cin.ptr) return false;
   return encode_fn() != nullptr;

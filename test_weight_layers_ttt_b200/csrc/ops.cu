@@ -346,46 +346,47 @@ __global__ void ns_copy_kernel(const float* U_in, float* X, float* U_out, NsLayo
   }
 }
 
-// One thread per 8 consecutive columns of a row: 16-byte loads and stores.
-__global__ void split_hilo_kernel(const float* M, long long P, int rows, int cols, uint4* hhl,
-                                  uint4* hlh, uint4* stack) {
-  const int c8 = cols / 8;
-  TTT_GRID_LOOP(idx, P * rows * c8) {
-    const long long pr = idx / c8;              // p * rows + row
-    const int q = (int)(idx - pr * c8);
-    const long long p = pr / rows;
-    const int row = (int)(pr - p * rows);
-    const float4 a = *reinterpret_cast<const float4*>(M + pr * cols + 8 * q);
-    const float4 b = *reinterpret_cast<const float4*>(M + pr * cols + 8 * q + 4);
-    const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t hi[4], lo[4];
+
+// P row-major [rows, cols] fp32 matrices -> bf16 hi = bf16(x), lo = bf16(x - hi), stored
+// once each for split-precision GEMM operands:
+//   kmaj [P][rows][2 cols_p]   row r: hi (cols) | zeros | lo (cols) | zeros   (K along a row)
+//   mmaj [P][2 rows_p][cols]   rows 0..rows-1 hi, zero rows, rows_p.. lo, zero rows (K down)
+// (either may be null). One thread per 8 columns of one row of the padded shape.
+__global__ void split_hilo2_kernel(const float* M, long long P, int rows, int cols, int rows_p,
+                                   int cols_p, uint4* kmaj, uint4* mmaj) {
+  const int c8 = cols / 8, c8p = cols_p / 8;
+  TTT_GRID_LOOP(idx, P * rows_p * c8p) {
+    const long long pr = idx / c8p;             // p * rows_p + row
+    const int q = (int)(idx - pr * c8p);
+    const long long p = pr / rows_p;
+    const int row = (int)(pr - p * rows_p);
+    uint4 H = make_uint4(0u, 0u, 0u, 0u), Lo = H;
+    if (row < rows && q < c8) {
+      const float* src = M + (p * rows + row) * cols + 8 * q;
+      const float4 a = *reinterpret_cast<const float4*>(src);
+      const float4 b = *reinterpret_cast<const float4*>(src + 4);
+      const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint32_t hi[4], lo[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * t], x[2 * t + 1]);
-      const float2 hf = __bfloat1622float2(h2);
-      const __nv_bfloat162 l2 = __floats2bfloat162_rn(x[2 * t] - hf.x, x[2 * t + 1] - hf.y);
-      hi[t] = *reinterpret_cast<const uint32_t*>(&h2);
-      lo[t] = *reinterpret_cast<const uint32_t*>(&l2);
+      for (int t = 0; t < 4; ++t) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * t], x[2 * t + 1]);
+        const float2 hf = __bfloat1622float2(h2);
+        const __nv_bfloat162 l2 = __floats2bfloat162_rn(x[2 * t] - hf.x, x[2 * t + 1] - hf.y);
+        hi[t] = *reinterpret_cast<const uint32_t*>(&h2);
+        lo[t] = *reinterpret_cast<const uint32_t*>(&l2);
+      }
+      H = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      Lo = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    const uint4 H = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    const uint4 Lo = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    if (hhl) {   // row pr of [rows, 3 cols]: column blocks hi | hi | lo
-      uint4* o = hhl + pr * 3 * c8 + q;
+    if (kmaj && row < rows) {
+      uint4* o = kmaj + (p * rows + row) * 2 * c8p + q;
       o[0] = H;
-      o[c8] = H;
-      o[2 * c8] = Lo;
+      o[c8p] = Lo;
     }
-    if (hlh) {
-      uint4* o = hlh + pr * 3 * c8 + q;
+    if (mmaj && q < c8) {
+      uint4* o = mmaj + (p * 2 * rows_p + row) * c8 + q;
       o[0] = H;
-      o[c8] = Lo;
-      o[2 * c8] = H;
-    }
-    if (stack) {   // rows row, rows + row, 2 rows + row of [3 rows, cols]
-      uint4* o = stack + (p * 3 * rows + row) * c8 + q;
-      o[0] = H;
-      o[(long long)rows * c8] = Lo;
-      o[2LL * rows * c8] = H;
+      o[(long long)rows_p * c8] = Lo;
     }
   }
 }
@@ -816,15 +817,16 @@ cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cud
   return cudaGetLastError();
 }
 
-cudaError_t split_hilo(const float* M, int P, int rows, int cols, void* hhl, void* hlh,
-                       void* stack, cudaStream_t s) {
+
+cudaError_t split_hilo2(const float* M, int P, int rows, int cols, int rows_p, int cols_p,
+                        void* kmaj, void* mmaj, cudaStream_t s) {
   if (P <= 0 || rows <= 0 || cols <= 0) return cudaSuccess;
-  if (cols % 8 != 0) return cudaErrorInvalidValue;
-  const long long n = (long long)P * rows * (cols / 8);
-  split_hilo_kernel<<<grid_for(n, 256), 256, 0, s>>>(M, P, rows, cols,
-                                                     static_cast<uint4*>(hhl),
-                                                     static_cast<uint4*>(hlh),
-                                                     static_cast<uint4*>(stack));
+  if (cols % 8 != 0 || cols_p % 8 != 0 || cols_p < cols || rows_p < rows)
+    return cudaErrorInvalidValue;
+  const long long n = (long long)P * rows_p * (cols_p / 8);
+  split_hilo2_kernel<<<grid_for(n, 256), 256, 0, s>>>(M, P, rows, cols, rows_p, cols_p,
+                                                      static_cast<uint4*>(kmaj),
+                                                      static_cast<uint4*>(mmaj));
   return cudaGetLastError();
 }
 

@@ -80,11 +80,12 @@ bool ns_mma_supported(int R, int C);
 cudaError_t ns_mma(float* U, int Z, const NsLayout& L, int steps, float eps, float a, float b,
                    float c, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
 
-// Split fp32 matrices M [P, rows, cols] into bf16 hi = bf16(x), lo = bf16(x - hi) and
-// write the nullable outputs hhl = [hi|hi|lo] and hlh = [hi|lo|hi] ([P, rows, 3 cols],
-// concatenated along the columns) and stack = [hi;lo;hi] ([P, 3 rows, cols]). cols % 8 == 0.
-cudaError_t split_hilo(const float* M, int P, int rows, int cols, void* hhl, void* hlh,
-                       void* stack, cudaStream_t s);
+// Split fp32 matrices M [P, rows, cols] (cols % 8 == 0) into bf16 hi = bf16(x) and
+// lo = bf16(x - hi), each stored once for split-precision GEMM operands (GemmOperand::hilo):
+// kmaj [P][rows][2 cols_p] = [hi | lo] along each row, mmaj [P][2 rows_p][cols] = [hi ; lo]
+// down the rows, zero padded to cols_p / rows_p (multiples of 64); either may be null.
+cudaError_t split_hilo2(const float* M, int P, int rows, int cols, int rows_p, int cols_p,
+                        void* kmaj, void* mmaj, cudaStream_t s);
 
 // Backward of the prefix scan: R = dS_final[bh] (or 0 when null), then for c = C-1 .. 0:
 // R += dSc[bh, c] and the gradient of chunk c's delta G[bh, c] (OT) is R (order 0) or the

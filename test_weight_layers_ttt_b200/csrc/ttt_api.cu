@@ -101,9 +101,14 @@ const char* engine_name(const char* name, const char* engine) {
   return it->second.c_str();
 }
 
+ttt_status fail(ttt_status st, const char* fmt, ...);
+
 ttt_status run_gemm(const char* name, const GemmProblem& p, cudaStream_t s) {
   if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
   const bool tc = p.K > 0 && !force_simt() && umma_supported(p);
+  if (!tc && (p.A.hilo || p.B.hilo))
+    return fail(TTT_ERR_UNSUPPORTED, "%s: split-precision operands need the tensor-core engine",
+                name);
   TraceScope ts(g_trace.on ? engine_name(name, tc ? "tcgen05" : "simt") : name, s);
   if (tc) return gemm_umma(p, s, device_error_word(), wait_limit_ns());
   return gemm_simt(p, s);
@@ -405,7 +410,10 @@ ttt_status linear_impl(const ttt_desc& d, const void* q, const void* k, const vo
 // and Pa = [Ph|Ph|Pl] [problems, r, 3r], Gs = [Ah;Al;Ah] [problems, 3r, r].
 struct NsScratch {
   float *X = nullptr, *X2 = nullptr, *Ag = nullptr, *Pm = nullptr, *nrm = nullptr;
-  void *Xa = nullptr, *Xb = nullptr, *Xs = nullptr, *Ga = nullptr, *Gs = nullptr, *Pa = nullptr;
+  // split-precision operands of the tensor-core GEMM path ([hi | lo] stored once; r, c
+  // padded to rp, cp, multiples of 64): X along rows [r][2cp] and down rows [2rp][c], A and
+  // P along rows [r][2rp]
+  void *Xk = nullptr, *Xm = nullptr, *Gk = nullptr, *Pk = nullptr;
 };
 
 enum NsPath { NS_TENSOR_CTA = 0, NS_TENSOR_GEMM = 1, NS_CUDA_CORES = 2 };
@@ -427,12 +435,11 @@ NsScratch plan_ns(Carve& cv, int ot, long long problems, int R, int C) {
   w.Pm = cv.take_n<float>(problems * r * r);
   w.nrm = cv.take_n<float>(problems);
   if (path == NS_TENSOR_GEMM) {
-    w.Xa = cv.take(2 * problems * r * 3 * c);
-    w.Xb = cv.take(2 * problems * r * 3 * c);
-    w.Xs = cv.take(2 * problems * 3 * r * c);
-    w.Ga = cv.take(2 * problems * r * 3 * r);
-    w.Gs = cv.take(2 * problems * 3 * r * r);
-    w.Pa = cv.take(2 * problems * r * 3 * r);
+    const long long rp = (r + 63) / 64 * 64, cp = (c + 63) / 64 * 64;
+    w.Xk = cv.take(2 * problems * r * 2 * cp);
+    w.Xm = cv.take(2 * problems * 2 * rp * c);
+    w.Gk = cv.take(2 * problems * r * 2 * rp);
+    w.Pk = cv.take(2 * problems * r * 2 * rp);
   }
   return w;
 }
@@ -454,30 +461,41 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
   TTT_OP("ns_normalize", ns_normalize(U, w.X, Z, L, 1e-7f, w.nrm, s));
   if (ns_path(ot, (int)R, (int)Cc) == NS_TENSOR_GEMM) {
     // Each product as one bf16 GEMM over K tripled: hi*hi + hi*lo + lo*hi of the split
-    // operands (x = hi + lo to about 2^-16), fp32 accumulation in TMEM.
+    // operands (x = hi + lo to about 2^-16), fp32 accumulation in TMEM. Each split matrix
+    // is stored once as [hi | lo]; the GEMM reads the thirds [hi hi lo] of the A operand
+    // and [hi lo hi] of the B operand from it (GemmOperand::hilo).
     float* X = w.X;
     float* X2 = w.X2;
+    const long long rp = (r + 63) / 64 * 64, cp = (cc + 63) / 64 * 64;
+    auto op = [](void* ptr, bool mn, long long ld, long long s0, int hilo, long long k0) {
+      GemmOperand o;
+      o.ptr = ptr; o.dtype = DT_BF16; o.mn_major = mn; o.ld = ld; o.s0 = s0; o.s1 = 0;
+      o.hilo = hilo; o.k0 = k0;
+      return o;
+    };
     for (int it = 0; it < steps; ++it) {
-      TTT_OP("ns_split", split_hilo(X, P, (int)r, (int)cc, w.Xa, w.Xb, w.Xs, s));
+      TTT_OP("ns_split", split_hilo2(X, P, (int)r, (int)cc, (int)rp, (int)cp, w.Xk, w.Xm, s));
       GemmProblem g1;  // A = X X^T
-      g1.M = (int)r; g1.N = (int)r; g1.K = (int)(3 * cc); g1.Z0 = P;
-      g1.A = {w.Xa, DT_BF16, false, 3 * cc, 3 * r * cc, 0};
-      g1.B = {w.Xb, DT_BF16, false, 3 * cc, 3 * r * cc, 0};
+      g1.M = (int)r; g1.N = (int)r; g1.K = (int)(3 * cp); g1.Z0 = P;
+      g1.A = op(w.Xk, false, 2 * cp, r * 2 * cp, 1, cp);
+      g1.B = op(w.Xk, false, 2 * cp, r * 2 * cp, 2, cp);
       g1.C = {w.Ag, DT_F32, r, r * r, 0};
       TTT_TRY(run_gemm("ns_gram", g1, s));
-      TTT_OP("ns_split", split_hilo(w.Ag, P, (int)r, (int)r, w.Ga, nullptr, w.Gs, s));
-      GemmProblem g2;  // P = c A A + b A
-      g2.M = (int)r; g2.N = (int)r; g2.K = (int)(3 * r); g2.Z0 = P;
-      g2.A = {w.Ga, DT_BF16, false, 3 * r, 3 * r * r, 0};
-      g2.B = {w.Gs, DT_BF16, true, r, 3 * r * r, 0};
+      TTT_OP("ns_split", split_hilo2(w.Ag, P, (int)r, (int)r, (int)rp, (int)rp, w.Gk, nullptr,
+                                      s));
+      GemmProblem g2;  // P = c A A + b A (A symmetric: its B operand is read K-major)
+      g2.M = (int)r; g2.N = (int)r; g2.K = (int)(3 * rp); g2.Z0 = P;
+      g2.A = op(w.Gk, false, 2 * rp, r * 2 * rp, 1, rp);
+      g2.B = op(w.Gk, false, 2 * rp, r * 2 * rp, 2, rp);
       g2.C = {w.Pm, DT_F32, r, r * r, 0};
       g2.alpha = c3; g2.beta = b3; g2.Cin = {w.Ag, r, r * r, 0};
       TTT_TRY(run_gemm("ns_poly", g2, s));
-      TTT_OP("ns_split", split_hilo(w.Pm, P, (int)r, (int)r, w.Pa, nullptr, nullptr, s));
+      TTT_OP("ns_split", split_hilo2(w.Pm, P, (int)r, (int)r, (int)rp, (int)rp, w.Pk, nullptr,
+                                      s));
       GemmProblem g3;  // X' = P X + a X
-      g3.M = (int)r; g3.N = (int)cc; g3.K = (int)(3 * r); g3.Z0 = P;
-      g3.A = {w.Pa, DT_BF16, false, 3 * r, 3 * r * r, 0};
-      g3.B = {w.Xs, DT_BF16, true, cc, 3 * r * cc, 0};
+      g3.M = (int)r; g3.N = (int)cc; g3.K = (int)(3 * rp); g3.Z0 = P;
+      g3.A = op(w.Pk, false, 2 * rp, r * 2 * rp, 1, rp);
+      g3.B = op(w.Xm, true, cc, 2 * rp * cc, 2, rp);
       g3.C = {X2, DT_F32, cc, r * cc, 0};
       g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, cc, r * cc, 0};
       TTT_TRY(run_gemm("ns_apply", g3, s));
