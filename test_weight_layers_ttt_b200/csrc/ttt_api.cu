@@ -405,9 +405,7 @@ ttt_status linear_impl(const ttt_desc& d, const void* q, const void* k, const vo
 
 // Newton-Schulz scratch. CUDA-core path: X, X2 [problems, r, c], Ag, Pm [problems, r, r]
 // fp32. Split-bf16 GEMM path: the same fp32 buffers (Ag holds A = X X^T, Pm the polynomial)
-// plus the bf16 hi/lo operands concatenated along K (see run_ns): Xa = [Xh|Xh|Xl] and
-// Xb = [Xh|Xl|Xh] [problems, r, 3c], Xs = [Xh;Xl;Xh] [problems, 3r, c], Ga = [Ah|Ah|Al]
-// and Pa = [Ph|Ph|Pl] [problems, r, 3r], Gs = [Ah;Al;Ah] [problems, 3r, r].
+// plus the bf16 hi/lo operands below (see run_ns). The one-CTA path needs none of them.
 struct NsScratch {
   float *X = nullptr, *X2 = nullptr, *Ag = nullptr, *Pm = nullptr, *nrm = nullptr;
   // split-precision operands of the tensor-core GEMM path ([hi | lo] stored once; r, c
