@@ -774,17 +774,21 @@ struct RecBufs {
 };
 
 // Token splits of the gradient reductions: the largest power of two that divides the chunk
-// length, keeps split lengths a multiple of 64 (and >= 256), and keeps the grid of each
-// gradient GEMM within one CTA per SM (every split writes a full fp32 partial that the
-// reduction reads back, so more splits than one wave costs more HBM traffic than it
-// saves in GEMM time).
+// length, keeps split lengths a multiple of 64 (and >= 256), keeps the grid of each
+// gradient GEMM within one CTA per SM, and keeps all partials within 32 MB. Every split
+// writes a full fp32 partial of the three gradients that the reduction reads back, so
+// beyond one wave, or once the partials leave L2, more splits cost more traffic than they
+// save in GEMM time (measured: 2 splits at lm, 12.6 MB per partial, beat 4 by 12 %; 8 at
+// nvs, 2.4 MB per partial, beat 4 by 3 %).
 int choose_splits(const ttt_desc& d, long long L) {
   const long long BH = (long long)d.B * d.H;
   const long long tiles = BH * ((d.m + 127) / 128) * ((d.h + 255) / 256);
+  const long long partial_bytes = BH * 3LL * d.h * d.m * 4;
   long long best = 1;
   for (long long sp = 2; sp <= 64; sp *= 2) {
     if (L % sp != 0 || (L / sp) % 64 != 0 || L / sp < 256) break;
     if (tiles * sp > 148) break;
+    if (sp * partial_bytes > (32LL << 20)) break;
     best = sp;
   }
   return (int)best;
