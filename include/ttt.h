@@ -59,7 +59,7 @@ typedef struct CUstream_st* ttt_stream_t;
 typedef enum ttt_status {
   TTT_OK = 0,
   TTT_ERR_INVALID_ARG = 1,  /* a size, flag or pointer is invalid (see the message) */
-  TTT_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+  TTT_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement */
   TTT_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or smaller than required */
   TTT_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
   TTT_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out */
