@@ -73,3 +73,36 @@ def test_max_over_ranks_with_two_gloo_ranks():
     for r, w, slowest, value in res:
         assert w == 2 and slowest == 15.0
         assert value == pytest.approx(2 * 65536 / 0.015)
+
+
+def test_roofline_per_launch_work():
+    """The dominant kernel's algorithmic work per launch is the form's per-step work over its
+    launches per step; in the training step every launch of a forward kernel (forward pass
+    and the backward's recomputation) does the forward form's whole work."""
+    wl = WORKLOADS["lm"]
+    T = wl.B * wl.H * wl.N
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0, "source": "test"}
+    table = {"no_such_kernel": {"launches": 5, "ms_avg": 1.0, "share": 0.9},
+             "gemm_features_k@tcgen05": {"launches": 10, "ms_avg": 0.1, "share": 0.1}}
+    r = bench._roofline(table, wl, peaks, "parallel", 5)          # two launches per step
+    assert r["kernel"] == "gemm_features_k@tcgen05"               # unknown work skipped
+    assert r["work_per_launch"] == 4.0 * wl.h * wl.m * T / 2
+    t = bench._roofline(table, wl, peaks, "train", 5)
+    assert t["work_per_launch"] == 4.0 * wl.h * wl.m * T
+    assert abs(t["achieved"] - 4.0 * wl.h * wl.m * T / 1e-4 / 1e12) < 0.01
+    assert abs(t["frac"] - t["achieved"] / 1000.0) < 1e-4
+    assert t["bound"] == "tensor" and t["unit"] == "TFLOP/s"
+
+
+def test_traffic_only_while_the_captured_source_is_unchanged():
+    import hashlib
+    path = os.path.join(os.path.dirname(bench.__file__), "profiles", "traffic.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    assert rows
+    for wl, kernel, value, src in (r[:4] for r in rows):
+        name, want = src.split(":")
+        f = os.path.join(os.path.dirname(bench.__file__), "test_weight_layers_ttt_b200", "csrc",
+                         name)
+        have = hashlib.sha256(open(f, "rb").read()).hexdigest()[:len(want)]
+        assert bench._traffic(wl, kernel) == (float(value) if have == want else None)
+    assert bench._traffic("lm", "no_such_kernel") is None
