@@ -13,7 +13,11 @@
 //   STORE   C = alpha * acc + beta * Cin (fp32 or bf16 C)
 //   SWIGLU  the tile's columns are [A block | B block] of the fused SwiGLU input weights;
 //           writes phi = silu(a) * b times a per-row factor (bf16), and optionally the
-//           unscaled phi to a second output.
+//           unscaled phi to a second output; the gradient variant writes the recurrent
+//           form's pieces (phi * eta, D * silu(a), D * b * silu'(a)) instead.
+// Split-precision operands (GemmOperand::hilo): the producer reads the k-blocks of a
+// K-tripled operand [hi hi lo] / [hi lo hi] from one [hi | lo] copy by remapping the K
+// coordinate; nothing else changes.
 // Every mbarrier wait is bounded; a timeout records DEVERR_TIMEOUT in the device error
 // word, raises a CTA-wide abort flag, and the CTA drains its in-flight copies and MMAs
 // (again with bounded waits) and frees its TMEM before returning.
