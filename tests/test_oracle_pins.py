@@ -248,6 +248,61 @@ def test_momentum_is_value_reweighting_closed_form(order):
     assert np.max(np.abs(g0 - g1)) < 1e-13
 
 
+def _ns5_spectral(G):
+    """Five Newton-Schulz steps written on the singular values: for G = U diag(s) V^T the
+    iteration only maps s / (||G||_F + 1e-7) through p(x) = a x + b x^3 + c x^5 five times
+    (an SVD route, independent of the oracle's matrix iteration)."""
+    a, b, c = 3.4445, -4.7750, 2.0315
+    U, s, Vt = np.linalg.svd(G, full_matrices=False)
+    x = s / (math.sqrt(float(np.sum(s * s))) + 1e-7)
+    for _ in range(5):
+        x = a * x + b * x ** 3 + c * x ** 5
+    return U @ np.diag(x) @ Vt
+
+
+@pytest.mark.parametrize("order", [O.UPDATE_APPLY, O.APPLY_UPDATE])
+def test_momentum_then_newton_schulz_order(order):
+    """Momentum before orthogonalisation ("Test-Time Training Done Right" notes, section
+    2.2: the momentum buffer accumulates raw gradients, Muon orthogonalises the buffer):
+    with W0, W2 frozen and only W1 fast, M_c = sum_{i <= c} (prod_{l=i+1}^{c} alpha_l) g_i
+    (nested loops over the raw chunk gradients g_i = -Delta S_i), U_c = NS5(M_c) by the
+    spectral route, W1_c = W1 - sum_{c' <= c} U_c'. The two plausible mistakes (NS before
+    the momentum, NS fed the raw gradient) give different weights and fail this pin."""
+    q, k, v, eta, W0, W2, W1 = _layer(21, N=24, h=4, m=6)
+    chunk, C = 4, 6
+    alpha = _rng(22).uniform(0.3, 0.95, C)
+    g = [-d for d in O.chunk_state_deltas(O.swiglu_features(k, W0, W2), v, eta, chunk)]
+    states = []
+    S = W1.copy()
+    for c in range(C):
+        M = np.zeros_like(W1)
+        for i in range(c + 1):
+            prod = 1.0
+            for l in range(i + 1, c + 1):
+                prod *= alpha[l]
+            M = M + prod * g[i]
+        S = S - _ns5_spectral(M)
+        states.append(S)
+    pq = O.swiglu_features(q, W0, W2)
+    expect = np.empty_like(q)
+    for c in range(C):
+        sl = slice(c * chunk, (c + 1) * chunk)
+        Sc = states[c] if order == O.UPDATE_APPLY else (W1 if c == 0 else states[c - 1])
+        expect[sl] = pq[sl] @ Sc
+    got, W, M = O.lact_recurrent(q, k, v, eta, W0, W2, W1, chunk, order=order, update=("W1",),
+                                 alpha=alpha, ns_steps=5)
+    assert np.max(np.abs(W["W1"] - states[-1])) < 1e-10
+    assert np.max(np.abs(got - expect)) < 1e-10
+    # the pin separates the orders: NS before momentum / NS of the raw gradient differ
+    Mw, Sw1, Sw2 = np.zeros_like(W1), W1.copy(), W1.copy()
+    for c in range(C):
+        Mw = alpha[c] * Mw + _ns5_spectral(g[c])
+        Sw1 = Sw1 - Mw
+        Sw2 = Sw2 - _ns5_spectral(g[c])
+    assert np.max(np.abs(Sw1 - states[-1])) > 1e-2
+    assert np.max(np.abs(Sw2 - states[-1])) > 1e-2
+
+
 # --------------------------------------------------------------------------- Newton-Schulz
 @pytest.mark.parametrize("shape", [(6, 9), (9, 6), (7, 7)])
 def test_newton_schulz_acts_on_singular_values(shape):
