@@ -77,20 +77,59 @@ def layer_bytes(wl, form: str) -> float:
     return float(act + weights + state_out)
 
 
+def _ns_work(wl, r, c, matrices):
+    """Step-level work of the Newton-Schulz kernels on `matrices` [r, c] matrices (r <= c):
+    tensor FLOPs of the split-precision products (three bf16 terms hi*hi + hi*lo + lo*hi per
+    fp32 product) and the HBM bytes of the fp32 set-up, splits and write-back."""
+    steps = wl.ns_steps if wl.ns_steps else 5
+    Z = float(matrices)
+    return {
+        "ns_mma": ("tensor", 3.0 * steps * (4.0 * r * r * c + 2.0 * r ** 3) * Z),
+        "ns_gram": ("tensor", 3.0 * steps * 2.0 * r * r * c * Z),
+        "ns_poly": ("tensor", 3.0 * steps * 2.0 * r ** 3 * Z),
+        "ns_apply": ("tensor", 3.0 * steps * 2.0 * r * r * c * Z),
+        # per step: X read (4rc) -> [hi|lo] along rows and down rows (8rc); A and P read
+        # (4r^2 each) -> [hi|lo] (4r^2 each)
+        "ns_split": ("hbm", steps * (12.0 * r * c + 16.0 * r * r) * Z),
+        "ns_normalize": ("hbm", 8.0 * r * c * Z),
+        "ns_writeback": ("hbm", 8.0 * r * c * Z),
+    }
+
+
+def rec_splits(wl) -> int:
+    """Token splits of the recurrent form's gradient GEMMs, as the library chooses them:
+    the largest power of two dividing the chunk with splits of at least 256 tokens (a
+    multiple of 64), one wave of tiles and at most 32 MB of fp32 partials."""
+    BH, L = wl.B * wl.H, wl.chunk
+    tiles = BH * (-(-wl.m // 128)) * (-(-wl.h // 256))
+    partial = BH * 3 * wl.h * wl.m * 4
+    best, sp = 1, 2
+    while sp <= 64:
+        if L % sp or (L // sp) % 64 or L // sp < 256 or tiles * sp > 148 or \
+                sp * partial > 32 << 20:
+            break
+        best, sp = sp, sp * 2
+    return best
+
+
 def kernel_work(name: str, wl, form: str):
     """(bound, algorithmic work of one whole step) of a traced kernel: FLOP for tensor
-    kernels, HBM bytes for memory-bound ones. Per-launch work = this / launches per step."""
+    kernels, HBM bytes for memory-bound ones. Per-launch work = this / launches per step.
+    Every kernel the library launches for a form has an entry."""
     base = name.split("@")[0]
-    BH, h, m = wl.B * wl.H, wl.h, wl.m
+    BH, h, m, H, C = wl.B * wl.H, wl.h, wl.m, wl.H, wl.C
     T = BH * wl.N
+    hm = h * m
     es = 2 if wl.dtype == "bf16" else 4
+    mpad = -(-m // 128) * 128
+    r, c = min(h, m), max(h, m)
     if form == "linear":
         hh = h * h
         table = {
             "gemm_state_delta": ("tensor", 2.0 * hh * T),
             "gemm_output": ("tensor", 2.0 * hh * T),
             "scale_rows": ("hbm", T * h * 2.0 * es + T * 4.0),
-            "chunk_scan": ("hbm", BH * wl.C * hh * (4.0 + es) + 2 * 4.0 * BH * hh),
+            "chunk_scan": ("hbm", BH * C * hh * (4.0 + es) + 2 * 4.0 * BH * hh),
         }
         return table.get(base, (None, None))
     if form == "lm_target":
@@ -101,29 +140,63 @@ def kernel_work(name: str, wl, form: str):
         }
         return table.get(base, (None, None))
     if form == "recurrent":
-        r, c = min(h, m), max(h, m)
-        ns = wl.ns_steps * (4.0 * r * r * c + 2.0 * r ** 3) * 3 * BH * wl.C
+        # per chunk: fp32 masters W (3hm), update U (3hm), momentum M (3hm) per (b, head)
+        sp = rec_splits(wl)
+        mom = 2.0 * 3 * hm * 4 if wl.momentum else 0.0
         table = {
-            "ns_mma": ("tensor", 3.0 * ns),   # three bf16 hi/lo terms per product
-            "gemm_features_k": ("tensor", 4.0 * h * m * T),
-            "gemm_features_q": ("tensor", 4.0 * h * m * T),
-            "gemm_v_w1t": ("tensor", 2.0 * h * m * T),
-            "gemm_grad_w1": ("tensor", 2.0 * h * m * T),
-            "gemm_grad_w0": ("tensor", 2.0 * h * m * T),
-            "gemm_grad_w2": ("tensor", 2.0 * h * m * T),
-            "gemm_output": ("tensor", 2.0 * h * m * T),
+            "gemm_features_k": ("tensor", 4.0 * hm * T),
+            "gemm_features_q": ("tensor", 4.0 * hm * T),
+            "gemm_v_w1t": ("tensor", 2.0 * hm * T),
+            "gemm_grad_w1": ("tensor", 2.0 * hm * T),
+            "gemm_grad_w0": ("tensor", 2.0 * hm * T),
+            "gemm_grad_w2": ("tensor", 2.0 * hm * T),
+            "gemm_output": ("tensor", 2.0 * hm * T),
+            # split-K partials in, U out (and M in / out)
+            "reduce_momentum": ("hbm", C * BH * (sp * 3 * hm * 4.0 + 3 * hm * 4.0 + mom)),
+            # W and U in, W out, bf16 operands (blocked W0/W2, W1) out
+            "step_renorm": ("hbm", C * BH * (3 * 3 * hm * 4.0 + (2 * mpad * h + hm) * es)),
+            "rec_init": ("hbm", 3 * hm * 4.0 * H + BH * (3 * hm * 4.0 + hm * es)),
+            "col_norms": ("hbm", 3 * hm * 4.0 * H),
+            "prep_weights": ("hbm", 2 * hm * 4.0 * H + BH * 2 * mpad * h * es),
+            "rec_finish": ("hbm", 2 * BH * 3 * hm * 4.0),
         }
+        table.update(_ns_work(wl, r, c, 3 * BH * C))
         return table.get(base, (None, None))
+    # parallel forms; the training step runs the forward kernels twice (forward call and
+    # the backward's recomputation)
+    feats = 1 if wl.kind == "inplace" else 2
+    fw = 2 if form == "train" else 1
+    scan = BH * C * hm * (4.0 + es) + 2 * 4.0 * BH * hm
     table = {
-        "fused_apply": ("tensor", 6.0 * h * m * T),   # phi(Q) (4hm) and phi(Q) S_c (2hm)
-        "gemm_features_k": ("tensor", 4.0 * h * m * T),
-        "gemm_features_q": ("tensor", 4.0 * h * m * T),
-        "gemm_state_delta": ("tensor", 2.0 * h * m * T),
-        "gemm_output": ("tensor", 2.0 * h * m * T),
-        "chunk_scan": ("hbm", BH * wl.C * h * m * (4.0 + es) + 2 * 4.0 * BH * h * m),
-        "swiglu_k": ("hbm", T * m * (8.0 + es * (1 if wl.kind != "inplace" else 2))),
-        "swiglu_q": ("hbm", T * m * (8.0 + es)),
+        "prep_weights": ("hbm", fw * (2 * hm * 4.0 * H + 2 * mpad * h * es * H)),
+        "gemm_features_k": ("tensor", fw * 4.0 * hm * T),
+        "gemm_state_delta": ("tensor", fw * 2.0 * hm * T),
+        "chunk_scan": ("hbm", fw * scan),
+        "fused_apply": ("tensor", 6.0 * hm * T),   # phi(Q) (4hm) and phi(Q) S_c (2hm)
+        "gemm_features_q": ("tensor", 4.0 * hm * T),
+        "gemm_output": ("tensor", 2.0 * hm * T),
+        "momentum_scan": ("hbm", 2 * 4.0 * BH * C * hm + 4.0 * BH * C),
     }
+    if form == "parallel_momentum":
+        table.update(_ns_work(wl, r, c, BH * C))
+    if form == "train":
+        table.update({
+            "cast_weights": ("hbm", 2 * hm * 4.0 * H + 2 * hm * es * H),
+            "gemm_bwd_state": ("tensor", 2.0 * hm * T),
+            "suffix_scan": ("hbm", BH * C * hm * (4.0 + es) + 4.0 * BH * hm),
+            "gemm_bwd_dphi_q": ("tensor", 2.0 * hm * T),
+            "scale_rows": ("hbm", T * h * 2.0 * es + T * 4.0),
+            "gemm_bwd_dphi_k": ("tensor", 2.0 * hm * T),
+            "gemm_bwd_t": ("tensor", 2.0 * hm * T),
+            "row_grads": ("hbm", T * h * (4.0 + 2 * es) + 8.0 * T),
+            "fill": ("hbm", 4.0 * T),
+            "gemm_bwd_swiglu_k": ("tensor", 4.0 * hm * T),
+            "gemm_bwd_swiglu_q": ("tensor", 4.0 * hm * T),
+            "gemm_bwd_dx": ("tensor", 2 * 4.0 * hm * T),     # k side and q side
+            "gemm_bwd_dw": ("tensor", 2 * 4.0 * hm * T),
+            # split partials of [dW0 | dW2] and the batch's R0 in, weight gradients out
+            "sum_batches": ("hbm", 4.0 * (2 * hm * BH * 2 + 2 * hm * H + hm * BH + hm * H)),
+        })
     return table.get(base, (None, None))
 
 
@@ -386,32 +459,34 @@ def _traffic(workload: str, kernel: str):
 
 
 def _roofline(table, wl, peaks, form, steps):
-    """Roofline of the dominant kernel (largest share) with a known algorithmic work."""
-    for name, e in table.items():
-        bound, step_work = kernel_work(name, wl, form)
-        if bound is None:
-            continue
-        # the training step runs the forward kernels once in the forward pass and again in
-        # the backward pass (recomputed features, states): each launch does the forward
-        # form's whole per-step work
-        work = step_work if form == "train" else step_work / (e["launches"] / steps)
-        secs = e["ms_avg"] / 1e3
-        if bound == "tensor":
-            achieved = work / secs / 1e12
-            peak = peaks["bf16_tflops"]
-            unit = "TFLOP/s"
-        else:
-            achieved = work / secs / 1e9
-            peak = peaks["hbm_gbs"]
-            unit = "GB/s"
-        return {"kernel": name, "bound": "hbm" if bound == "hbm" else "tensor",
-                "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-                "frac": round(achieved / peak, 4),
-                "traffic": (_traffic(wl.name, name)
-                            if form == "parallel" and wl == WORKLOADS_REF().get(wl.name) else None),
-                "work_per_launch": work, "share": round(e["share"], 4),
-                "peak_source": peaks["source"] + " (burst)"}
-    return None
+    """Roofline of the dominant kernel: the one with the largest share of the traced step.
+    Its algorithmic work per launch is the form's per-step work (kernel_work) over its
+    launches per step; a kernel without an entry is reported with null figures."""
+    if not table:
+        return None
+    name, e = next(iter(table.items()))
+    bound, step_work = kernel_work(name, wl, form)
+    if bound is None:
+        return {"kernel": name, "bound": None, "achieved": None, "peak": None, "unit": None,
+                "frac": None, "traffic": None, "work_per_launch": None,
+                "share": round(e["share"], 4), "peak_source": peaks["source"]}
+    work = step_work / (e["launches"] / steps)
+    secs = e["ms_avg"] / 1e3
+    if bound == "tensor":
+        achieved = work / secs / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    else:
+        achieved = work / secs / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    return {"kernel": name, "bound": "hbm" if bound == "hbm" else "tensor",
+            "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4),
+            "traffic": (_traffic(wl.name, name)
+                        if form == "parallel" and wl == WORKLOADS_REF().get(wl.name) else None),
+            "work_per_launch": work, "share": round(e["share"], 4),
+            "peak_source": peaks["source"] + " (burst)"}
 
 
 def run_gpu(args, rank, local, world):
@@ -599,8 +674,10 @@ def run_gpu(args, rank, local, world):
 
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_time(wl, x, n: int, form: str = "parallel") -> float:
-    """Seconds the fp64 oracle takes for the first ``n`` tokens of (b=0, head=0) (for the
-    In-Place workload: the target prologue and the sequential update on n tokens)."""
+    """Seconds the fp64 oracle takes for the first ``n`` tokens of batch element 0 through
+    all H heads of the layer, so that n / seconds counts layer tokens like the GPU arm's
+    ``value`` (for the In-Place workload: the target prologue and the sequential update on
+    n tokens)."""
     from oracle import ttt_oracle as O
     if wl.kind == "inplace":
         t0 = time.perf_counter()
@@ -608,29 +685,35 @@ def oracle_time(wl, x, n: int, form: str = "parallel") -> float:
         O.inplace_sequential(x["Hs"][:n], x["Wg"], x["Wu"], x["W_down"], vbar, wl.chunk,
                              float(x["eta"][0]))
         return time.perf_counter() - t0
-    q, k, v, eta = (x[name][0, 0, :n].astype("float64") for name in ("q", "k", "v", "eta"))
-    W0, W2, W1 = x["W0"][0], x["W2"][0], x["W1"][0]
+    heads = x["q"].shape[1]
     t0 = time.perf_counter()
-    if form == "parallel":
-        O.la_parallel(q, k, v, eta, W0, W2, W1, wl.chunk, order=wl.order)
-    else:
-        alpha = x["alpha"][0, 0] if x.get("alpha") is not None else None
-        O.lact_recurrent(q, k, v, eta, W0, W2, W1, wl.chunk, order=wl.order, renorm=wl.renorm,
-                         alpha=alpha, ns_steps=wl.ns_steps)
+    for hd in range(heads):
+        q, k, v, eta = (x[name][0, hd, :n].astype("float64") for name in ("q", "k", "v", "eta"))
+        W0, W2, W1 = x["W0"][hd], x["W2"][hd], x["W1"][hd]
+        if form == "parallel":
+            O.la_parallel(q, k, v, eta, W0, W2, W1, wl.chunk, order=wl.order)
+        else:
+            alpha = x["alpha"][0, hd] if x.get("alpha") is not None else None
+            O.lact_recurrent(q, k, v, eta, W0, W2, W1, wl.chunk, order=wl.order,
+                             renorm=wl.renorm, alpha=alpha, ns_steps=wl.ns_steps)
     return time.perf_counter() - t0
 
 
 def oracle_sample(wl, x, target_s: float, form: str = "parallel"):
-    """Time the fp64 oracle on (b=0, head=0) with as many leading whole chunks as fit about
-    ``target_s`` seconds; returns (tokens, seconds, description)."""
+    """Time the fp64 oracle on batch element 0, all heads, with as many leading whole
+    chunks as fit about ``target_s`` seconds; returns (tokens, seconds, description)."""
     n = min(wl.N, wl.chunk)
     t = oracle_time(wl, x, n, form)
     if t < target_s / 2 and n < wl.N:
         n2 = min(wl.N, max(wl.chunk, int(n * target_s / max(t, 1e-3)) // wl.chunk * wl.chunk))
         if n2 > n:
             n, t = n2, oracle_time(wl, x, n2, form)
-    desc = (f"{form} form, fp64 oracle, one (batch, head) of the '{wl.name}' workload, "
-            f"first {n} of {wl.N} tokens")
+    if wl.kind == "inplace":
+        what = "the target prologue and the sequential update"
+    else:
+        what = f"all {x['q'].shape[1]} heads of batch element 0"
+    desc = (f"{form} form, fp64 oracle, {what} of the '{wl.name}' workload, first {n} of "
+            f"{wl.N} tokens; layer tokens/s (each token through every head)")
     return n, t, desc
 
 
@@ -653,7 +736,7 @@ def run_reference(args):
     if wl.kind == "inplace":
         x = make_inplace_inputs(wl, seed=wl.seed)
     else:
-        x = make_layer_inputs(wl.scaled(B=1, H=1), seed=wl.seed)
+        x = make_layer_inputs(wl.scaled(B=1), seed=wl.seed)
     form = "parallel" if "parallel" in wl.paths else "recurrent"
     n, t, desc = oracle_sample(wl, x, 2.0, form)
     times = []
@@ -679,11 +762,16 @@ def run_reference(args):
 
 
 def workload_config(wl, form):
-    return {"workload": wl.name if wl == WORKLOADS_REF().get(wl.name) else wl.name + "*",
-            "form": form, "B": wl.B, "H": wl.H, "N": wl.N, "h": wl.h,
-            "m": wl.m, "chunk": wl.chunk, "order": wl.order, "renorm": wl.renorm,
-            "momentum": wl.momentum, "ns_steps": wl.ns_steps, "parallelism": "replicas",
-            "l2": "no flush: the per-step inputs exceed the 126 MB L2"}
+    """The workload's sizes and the options of `form` (the recurrent options only on the
+    recurrent form's line)."""
+    cfg = {"workload": wl.name if wl == WORKLOADS_REF().get(wl.name) else wl.name + "*",
+           "form": form, "B": wl.B, "H": wl.H, "N": wl.N, "h": wl.h,
+           "m": wl.m, "chunk": wl.chunk, "order": wl.order}
+    if form == "recurrent":
+        cfg.update({"renorm": wl.renorm, "momentum": wl.momentum, "ns_steps": wl.ns_steps})
+    cfg.update({"parallelism": "replicas",
+                "l2": "no flush: the per-step inputs exceed the 126 MB L2"})
+    return cfg
 
 
 def WORKLOADS_REF():

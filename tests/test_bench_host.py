@@ -76,22 +76,51 @@ def test_max_over_ranks_with_two_gloo_ranks():
 
 
 def test_roofline_per_launch_work():
-    """The dominant kernel's algorithmic work per launch is the form's per-step work over its
-    launches per step; in the training step every launch of a forward kernel (forward pass
-    and the backward's recomputation) does the forward form's whole work."""
+    """The dominant kernel (largest share) is reported; its algorithmic work per launch is
+    the form's per-step work over its launches per step. In the training step the forward
+    kernels run twice per step (forward pass and the backward's recomputation), each launch
+    doing the forward form's whole work."""
     wl = WORKLOADS["lm"]
     T = wl.B * wl.H * wl.N
     peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0, "source": "test"}
-    table = {"no_such_kernel": {"launches": 5, "ms_avg": 1.0, "share": 0.9},
-             "gemm_features_k@tcgen05": {"launches": 10, "ms_avg": 0.1, "share": 0.1}}
+    table = {"gemm_features_k@tcgen05": {"launches": 10, "ms_avg": 0.1, "share": 0.6},
+             "no_such_kernel": {"launches": 5, "ms_avg": 1.0, "share": 0.1}}
     r = bench._roofline(table, wl, peaks, "parallel", 5)          # two launches per step
-    assert r["kernel"] == "gemm_features_k@tcgen05"               # unknown work skipped
+    assert r["kernel"] == "gemm_features_k@tcgen05"
     assert r["work_per_launch"] == 4.0 * wl.h * wl.m * T / 2
     t = bench._roofline(table, wl, peaks, "train", 5)
-    assert t["work_per_launch"] == 4.0 * wl.h * wl.m * T
+    assert t["work_per_launch"] == 4.0 * wl.h * wl.m * T / 2 * 2
+    t = bench._roofline({"gemm_features_k@tcgen05": {"launches": 10, "ms_avg": 0.1,
+                                                      "share": 0.6}}, wl, peaks, "train", 5)
     assert abs(t["achieved"] - 4.0 * wl.h * wl.m * T / 1e-4 / 1e12) < 0.01
     assert abs(t["frac"] - t["achieved"] / 1000.0) < 1e-4
     assert t["bound"] == "tensor" and t["unit"] == "TFLOP/s"
+    # a dominant kernel without known work is still the one reported, with null figures
+    u = bench._roofline({"no_such_kernel": {"launches": 5, "ms_avg": 1.0, "share": 0.9}},
+                        wl, peaks, "parallel", 5)
+    assert u["kernel"] == "no_such_kernel" and u["achieved"] is None
+
+
+def test_every_traced_kernel_has_algorithmic_work():
+    """Every kernel name the library traces (the names passed to its trace scopes) has an
+    entry in the work table of each form that launches it."""
+    import re
+    src = open(os.path.join(os.path.dirname(bench.__file__), "test_weight_layers_ttt_b200",
+                            "csrc", "ttt_api.cu")).read()
+    names = set(re.findall(r'(?:TTT_OP|run_gemm|run_simt|run_swiglu|TraceScope ts)\(\s*"(\w+)',
+                           src))
+    names |= set(re.findall(r'"(gemm_\w+|fused_apply)(?:@tcgen05)?"', src))
+    assert {"gemm_features_k", "ns_mma", "step_renorm", "fused_apply"} <= names
+    forms = {"parallel": WORKLOADS["lm"], "parallel_momentum": WORKLOADS["lm"],
+             "train": WORKLOADS["lm"], "recurrent": WORKLOADS["nvs"],
+             "linear": WORKLOADS["lm"], "lm_target": WORKLOADS["inplace"]}
+    known = set()
+    for form, wl in forms.items():
+        known |= {n for n in names if bench.kernel_work(n, wl, form)[0] is not None}
+    # the failure-path probe and the debug-check kernels are not part of any timed form
+    missing = names - known - {"wait_timeout_probe", "guards_fill", "guards_check",
+                               "finite_scan"}
+    assert not missing, missing
 
 
 def test_traffic_only_while_the_captured_source_is_unchanged():
