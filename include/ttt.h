@@ -33,10 +33,12 @@
  *
  * Errors: arguments are checked on the host before anything is enqueued; a failed check
  * returns a status and enqueues nothing (no exceptions cross the ABI). A bounded wait
- * that runs out inside a kernel, or a device-side check that fails, is recorded in a
- * per-device error word; ttt_last_device_status() synchronises the stream, reads and
- * clears it. ttt_last_error_message() gives a human-readable detail of the calling
- * thread's last failure.
+ * that runs out inside a kernel, or a failed debug check (ttt_set_debug_checks), is
+ * recorded in a per-device error word; ttt_last_device_status() synchronises the stream,
+ * reads and clears it. ttt_last_error_message() gives a human-readable detail of the
+ * calling thread's last failure. In bf16 mode every contraction runs on the tensor cores;
+ * a problem the tensor-core engine cannot take is refused with TTT_ERR_UNSUPPORTED (it is
+ * never rerouted to another engine).
  *
  * Precision: in TTT_DTYPE_BF16 mode the dense contractions take bf16 operands (q, k, v,
  * the fp32 weights rounded to bf16, the features rounded to bf16) and accumulate in
@@ -63,7 +65,8 @@ typedef enum ttt_status {
   TTT_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or smaller than required */
   TTT_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
   TTT_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out */
-  TTT_ERR_DEVICE = 6        /* a device-side bounds/alignment check failed */
+  TTT_ERR_DEVICE = 6        /* a debug check failed: a workspace guard was overwritten, or
+                               an output holds NaN/Inf (see ttt_set_debug_checks) */
 } ttt_status;
 
 enum { TTT_DTYPE_FP32 = 0, TTT_DTYPE_BF16 = 1 };
@@ -290,10 +293,40 @@ ttt_status ttt_lm_target(int32_t N, int32_t d, const void* X0, const float* conv
 
 /*
  * Synchronises `stream`, then reads and clears the device error word of the current
- * device: TTT_OK, TTT_ERR_TIMEOUT (a bounded wait ran out) or TTT_ERR_DEVICE; or
- * TTT_ERR_CUDA when the synchronisation itself failed.
+ * device: TTT_OK, TTT_ERR_TIMEOUT (a bounded wait ran out) or TTT_ERR_DEVICE (a debug
+ * check failed, see ttt_set_debug_checks); or TTT_ERR_CUDA when the synchronisation itself
+ * failed.
  */
 ttt_status ttt_last_device_status(ttt_stream_t stream);
+
+/*
+ * Debug checks (no paper counterpart: the library's own stand-in for a device memory
+ * checker). `flags` is a combination of
+ *   TTT_CHECK_GUARDS  every region a call carves from its workspace gets a 256-byte guard
+ *                     in front of the first region and right after each region's end;
+ *                     ttt_workspace_bytes / ttt_lm_target_workspace_bytes grow to hold
+ *                     them. Each call fills its guards with a fixed pattern before its
+ *                     first kernel and compares them after its last one; a changed guard
+ *                     (a write outside its region) sets the device error word.
+ *   TTT_CHECK_FINITE  after its last kernel each call scans its outputs (out, final
+ *                     states / weights, momentum, gradients) for NaN or Inf.
+ * A failed check is reported by ttt_last_device_status as TTT_ERR_DEVICE, with the check
+ * named in ttt_last_error_message. The checks never stop or fault a kernel; they cost
+ * extra launches. The setting is process-wide; change it only while no call is in flight
+ * and size workspaces after changing it (a workspace sized with guards off is too small
+ * with guards on: TTT_ERR_WORKSPACE). Unknown flags: TTT_ERR_INVALID_ARG.
+ */
+enum { TTT_CHECK_GUARDS = 1, TTT_CHECK_FINITE = 2 };
+ttt_status ttt_set_debug_checks(int32_t flags);
+int32_t ttt_get_debug_checks(void);
+
+/*
+ * Compares, now (enqueued on `stream`), the guards of a workspace that a call with the
+ * same `desc` and `path` planned with TTT_CHECK_GUARDS on; a changed guard is reported by
+ * the next ttt_last_device_status. TTT_ERR_INVALID_ARG when guards are off.
+ */
+ttt_status ttt_debug_check_workspace(const ttt_desc* desc, int32_t path, void* workspace,
+                                     size_t workspace_bytes, ttt_stream_t stream);
 
 /*
  * Diagnostic for the failure path: launches one block that waits on a barrier nobody

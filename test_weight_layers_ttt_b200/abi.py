@@ -38,6 +38,8 @@ TTT_PATH_LINEAR = 2
 TTT_PATH_PARALLEL_MOMENTUM = 3
 TTT_PATH_PARALLEL_BWD = 4
 TTT_STATIC_SCRATCH_BYTES = 64 << 20
+TTT_CHECK_GUARDS = 1
+TTT_CHECK_FINITE = 2
 
 # Every symbol include/ttt.h declares.
 EXPORTED = (
@@ -45,6 +47,7 @@ EXPORTED = (
     "ttt_linear_attn_fwd", "ttt_la_parallel_momentum_fwd", "ttt_la_parallel_bwd",
     "ttt_lact_recurrent_fwd",
     "ttt_lm_target_workspace_bytes", "ttt_lm_target", "ttt_last_device_status",
+    "ttt_set_debug_checks", "ttt_get_debug_checks", "ttt_debug_check_workspace",
     "ttt_debug_wait_timeout", "ttt_trace_enable", "ttt_trace_disable", "ttt_trace_count",
     "ttt_trace_get", "ttt_status_str", "ttt_last_error_message", "ttt_version",
 )
@@ -102,6 +105,12 @@ def lib() -> ctypes.CDLL:
         L.ttt_lm_target.restype = I32
         L.ttt_last_device_status.argtypes = [P]
         L.ttt_last_device_status.restype = I32
+        L.ttt_set_debug_checks.argtypes = [I32]
+        L.ttt_set_debug_checks.restype = I32
+        L.ttt_get_debug_checks.argtypes = []
+        L.ttt_get_debug_checks.restype = I32
+        L.ttt_debug_check_workspace.argtypes = [D, I32, P, S, P]
+        L.ttt_debug_check_workspace.restype = I32
         L.ttt_debug_wait_timeout.argtypes = [I64, P]
         L.ttt_debug_wait_timeout.restype = I32
         L.ttt_trace_enable.argtypes = [I32]
@@ -229,6 +238,20 @@ def ttt_lm_target(N, d, X0, conv_w, W_target, vbar, workspace, workspace_bytes=N
 
 def ttt_last_device_status(stream=None):
     _check(lib().ttt_last_device_status(_stream(stream)))
+
+
+def ttt_set_debug_checks(flags: int):
+    _check(lib().ttt_set_debug_checks(int(flags)))
+
+
+def ttt_get_debug_checks() -> int:
+    return int(lib().ttt_get_debug_checks())
+
+
+def ttt_debug_check_workspace(desc, path, workspace, workspace_bytes=None, stream=None):
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    _check(lib().ttt_debug_check_workspace(ctypes.byref(desc), int(path), _ptr(workspace), wb,
+                                           _stream(stream)))
 
 
 def ttt_debug_wait_timeout(timeout_ns: int, stream=None):

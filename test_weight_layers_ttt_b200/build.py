@@ -21,7 +21,8 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libttt_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
-SOURCES = ["ttt_api.cu", "ops.cu", "gemm_simt.cu", "gemm_umma.cu", "ns_mma.cu", "apply_fused.cu"]
+SOURCES = ["ttt_api.cu", "ops.cu", "gemm_simt.cu", "gemm_umma.cu", "ns_mma.cu", "apply_fused.cu",
+           "checks.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
               "-I" + os.path.join(ROOT, "include")]

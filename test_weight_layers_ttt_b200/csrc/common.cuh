@@ -16,8 +16,9 @@ enum DType : int { DT_F32 = 0, DT_BF16 = 1 };
 inline size_t dtype_size(int dt) { return dt == DT_BF16 ? 2 : 4; }
 
 // Bits of the device error word (one per device, file-scope __device__ variable in
-// ttt_api.cu; kernels receive its address as an argument).
-enum : unsigned { DEVERR_TIMEOUT = 1u, DEVERR_BOUNDS = 2u };
+// ttt_api.cu; kernels receive its address as an argument): a bounded wait ran out, a
+// workspace guard word changed (debug checks), an output held NaN / Inf (debug checks).
+enum : unsigned { DEVERR_TIMEOUT = 1u, DEVERR_BOUNDS = 2u, DEVERR_NONFINITE = 4u };
 
 // Default limit of every bounded device-side wait, in nanoseconds.
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;

@@ -54,6 +54,8 @@ ttt_status gemm_simt(const GemmProblem& p, cudaStream_t stream);
 // Tensor-core engine (tcgen05.mma kind::f16, TMEM accumulators, TMA operand loads).
 // Requires bf16 A and B with 16-byte aligned bases and strides; see umma_supported.
 bool umma_supported(const GemmProblem& p);
+// Why the tensor-core engine cannot take `p` (a static string), or null when it can.
+const char* umma_unsupported_reason(const GemmProblem& p);
 ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,
                      unsigned long long wait_ns);
 
@@ -95,6 +97,7 @@ ttt_status fused_apply(const void* q, const void* Wk, const void* Sc, void* out,
                        unsigned long long wait_ns, cudaStream_t s);
 
 bool umma_swiglu_supported(const SwigluGemm& g);
+const char* umma_swiglu_unsupported_reason(const SwigluGemm& g);
 ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream);
 ttt_status gemm_umma_swiglu(const SwigluGemm& g, cudaStream_t stream, unsigned* dev_err,
                             unsigned long long wait_ns);

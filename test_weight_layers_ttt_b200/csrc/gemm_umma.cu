@@ -715,11 +715,6 @@ ttt_status dispatch_bn(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-bool operand_ok(const GemmOperand& o) {
-  return o.dtype == DT_BF16 && o.ptr && aligned16(o.ptr) && o.ld > 0 && (o.ld % 8) == 0 &&
-         (o.s0 % 8) == 0 && (o.s1 % 8) == 0 && o.s0 >= 0 && o.s1 >= 0;
-}
-
 UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait_ns) {
   UArgs a{};
   a.M = p.M; a.N = p.N; a.K = p.K; a.Z0 = p.Z0; a.Z1 = p.Z1;
@@ -736,17 +731,26 @@ UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait
 
 }  // namespace
 
-bool umma_supported(const GemmProblem& p) {
-  if (!operand_ok(p.A) || !operand_ok(p.B)) return false;
-  if (p.K <= 0 || p.M <= 0 || p.N <= 0) return false;
-  for (const GemmOperand* o : {&p.A, &p.B})
+const char* umma_unsupported_reason(const GemmProblem& p) {
+  for (const GemmOperand* o : {&p.A, &p.B}) {
+    if (o->dtype != DT_BF16) return "operands must be bf16";
+    if (!o->ptr || !aligned16(o->ptr)) return "operand base must be 16-byte aligned";
+    if (o->ld <= 0 || o->ld % 8 != 0) return "operand row stride must be a multiple of 8";
+    if (o->s0 < 0 || o->s1 < 0 || o->s0 % 8 != 0 || o->s1 % 8 != 0)
+      return "operand batch strides must be non-negative multiples of 8";
     if (o->hilo && (o->hilo > 2 || o->k0 <= 0 || o->k0 % BK != 0 || p.K != 3 * o->k0 ||
                     o->k0 > (1LL << 30)))
-      return false;
-  if ((long long)p.Z0 * p.Z1 * ((p.M + BM - 1) / BM) * ((p.N + 63) / 64) > (1LL << 31)) return false;
-  if (p.beta != 0.0f && !p.Cin.ptr) return false;
-  return encode_fn() != nullptr;
+      return "split-precision operand needs K = 3 k0 with k0 a multiple of 64";
+  }
+  if (p.K <= 0 || p.M <= 0 || p.N <= 0) return "M, N and K must be positive";
+  if ((long long)p.Z0 * p.Z1 * ((p.M + BM - 1) / BM) * ((p.N + 63) / 64) > (1LL << 31))
+    return "too many output tiles";
+  if (p.beta != 0.0f && !p.Cin.ptr) return "beta != 0 needs an addend";
+  if (encode_fn() == nullptr) return "cuTensorMapEncodeTiled is unavailable";
+  return nullptr;
 }
+
+bool umma_supported(const GemmProblem& p) { return umma_unsupported_reason(p) == nullptr; }
 
 ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,
                      unsigned long long wait_ns) {
@@ -760,19 +764,32 @@ ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_er
   return dispatch_bn<float>(p, a, stream);
 }
 
-bool umma_swiglu_supported(const SwigluGemm& g) {
+const char* umma_swiglu_unsupported_reason(const SwigluGemm& g) {
   const GemmProblem& p = g.gemm;
   auto strides_ok = [](long long ld, long long s0, long long s1) {
     return ld % 8 == 0 && s0 % 8 == 0 && s1 % 8 == 0 && s0 >= 0 && s1 >= 0;
   };
-  const bool grad_ok =
-      !g.grad || (g.rowscale && g.dv && aligned16(g.dv) && strides_ok(g.ldd, g.ds0, g.ds1) &&
-                  (!g.out3 || (aligned16(g.out3) && g.ld3 == p.C.ld && g.s30 == p.C.s0 &&
-                               g.s31 == p.C.s1)) &&
-                  (!g.out2 || (g.ld2 == p.C.ld && g.s20 == p.C.s0 && g.s21 == p.C.s1)));
-  return umma_supported(p) && p.C.dtype == DT_BF16 && p.N % 256 == 0 && p.beta == 0.0f &&
-         aligned16(p.C.ptr) && strides_ok(p.C.ld, p.C.s0, p.C.s1) && grad_ok &&
-         (!g.out2 || (aligned16(g.out2) && strides_ok(g.ld2, g.s20, g.s21)));
+  if (const char* r = umma_unsupported_reason(p)) return r;
+  if (p.C.dtype != DT_BF16) return "SwiGLU output must be bf16";
+  if (p.N % 256 != 0) return "SwiGLU GEMM width must be a multiple of 256";
+  if (p.beta != 0.0f) return "SwiGLU GEMM takes no addend";
+  if (!aligned16(p.C.ptr) || !strides_ok(p.C.ld, p.C.s0, p.C.s1))
+    return "SwiGLU output must be 16-byte aligned with strides a multiple of 8";
+  if (g.out2 && (!aligned16(g.out2) || !strides_ok(g.ld2, g.s20, g.s21)))
+    return "second SwiGLU output must be 16-byte aligned with strides a multiple of 8";
+  if (g.grad) {
+    if (!g.rowscale || !g.dv || !aligned16(g.dv) || !strides_ok(g.ldd, g.ds0, g.ds1))
+      return "gradient epilogue needs the row scale and an aligned dv";
+    if (g.out3 && (!aligned16(g.out3) || g.ld3 != p.C.ld || g.s30 != p.C.s0 || g.s31 != p.C.s1))
+      return "gradient epilogue: third output must share the first output's strides";
+    if (g.out2 && (g.ld2 != p.C.ld || g.s20 != p.C.s0 || g.s21 != p.C.s1))
+      return "gradient epilogue: second output must share the first output's strides";
+  }
+  return nullptr;
+}
+
+bool umma_swiglu_supported(const SwigluGemm& g) {
+  return umma_swiglu_unsupported_reason(g) == nullptr;
 }
 
 ttt_status gemm_umma_swiglu(const SwigluGemm& g, cudaStream_t stream, unsigned* dev_err,

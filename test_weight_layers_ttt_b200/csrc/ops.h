@@ -132,4 +132,18 @@ cudaError_t wait_timeout_probe(unsigned* err, unsigned long long limit_ns, cudaS
 
 cudaError_t fill_f32(float* p, long long n, float v, cudaStream_t s);
 
+// Debug checks (checks.cu). Guards: kGuardBytes-long words written before a call's first
+// kernel and compared after its last one (a change records DEVERR_BOUNDS); at most
+// kMaxGuards per launch. finite_scan records DEVERR_NONFINITE when any of the n elements
+// (fp32 or bf16, dt) is NaN or Inf.
+constexpr int kGuardBytes = 256;
+constexpr int kMaxGuards = 64;
+struct GuardList {
+  int n;
+  unsigned* p[kMaxGuards];
+};
+cudaError_t guards_fill(const GuardList& g, cudaStream_t s);
+cudaError_t guards_check(const GuardList& g, unsigned* err, cudaStream_t s);
+cudaError_t finite_scan(int dt, const void* x, long long n, unsigned* err, cudaStream_t s);
+
 }  // namespace ttt

@@ -1,11 +1,15 @@
 // C ABI of the TTT layer library (include/ttt.h): argument checks, workspace planning and
 // the enqueue order of the kernels for the parallel form, the recurrent form and the
-// In-Place target. Every contraction goes through run_gemm(), which picks the tcgen05
-// tensor-core engine for bf16 operands and the CUDA-core engine otherwise.
+// In-Place target. Every contraction goes through run_gemm() / run_swiglu(): bf16 mode
+// runs them on the tcgen05 tensor-core engine (a problem it cannot take is refused), fp32
+// mode on the fp32 CUDA-core engine.
+#include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <initializer_list>
 #include <map>
 #include <mutex>
 #include <string>
@@ -85,11 +89,6 @@ struct TraceScope {
   }
 };
 
-bool force_simt() {
-  const char* s = getenv("TTT_GEMM_ENGINE");
-  return s && strcmp(s, "simt") == 0;
-}
-
 // "<name>@<engine>" with stable storage, for trace records.
 const char* engine_name(const char* name, const char* engine) {
   static std::mutex mu;
@@ -103,14 +102,21 @@ const char* engine_name(const char* name, const char* engine) {
 
 ttt_status fail(ttt_status st, const char* fmt, ...);
 
+// One contraction. bf16 operands (bf16 mode) run on the tcgen05 tensor-core engine only: a
+// problem that engine cannot take is refused with TTT_ERR_UNSUPPORTED, never rerouted.
+// fp32 operands (fp32 mode) run on the fp32 CUDA-core engine.
 ttt_status run_gemm(const char* name, const GemmProblem& p, cudaStream_t s) {
   if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
-  const bool tc = p.K > 0 && !force_simt() && umma_supported(p);
-  if (!tc && (p.A.hilo || p.B.hilo))
-    return fail(TTT_ERR_UNSUPPORTED, "%s: split-precision operands need the tensor-core engine",
-                name);
-  TraceScope ts(g_trace.on ? engine_name(name, tc ? "tcgen05" : "simt") : name, s);
-  if (tc) return gemm_umma(p, s, device_error_word(), wait_limit_ns());
+  if (p.A.dtype == DT_BF16 || p.B.dtype == DT_BF16) {
+    if (const char* why = umma_unsupported_reason(p))
+      return fail(TTT_ERR_UNSUPPORTED, "%s: tensor-core engine: %s (M=%d N=%d K=%d)", name, why,
+                  p.M, p.N, p.K);
+    TraceScope ts(g_trace.on ? engine_name(name, "tcgen05") : name, s);
+    return gemm_umma(p, s, device_error_word(), wait_limit_ns());
+  }
+  if (p.A.hilo || p.B.hilo)
+    return fail(TTT_ERR_UNSUPPORTED, "%s: split-precision operands need bf16", name);
+  TraceScope ts(g_trace.on ? engine_name(name, "simt") : name, s);
   return gemm_simt(p, s);
 }
 
@@ -152,19 +158,87 @@ ttt_status fail(ttt_status st, const char* fmt, ...) {
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// Bump allocator over the caller's workspace (or a size counter when base is null).
+// ------------------------------------------------------------------ debug checks
+// Process-wide TTT_CHECK_* flags (ttt_set_debug_checks), and the guards the calling thread's
+// current call carved from its workspace.
+std::atomic<int> g_checks{0};
+thread_local std::vector<unsigned*> t_guards;
+
+// Bump allocator over the caller's workspace (or a size counter when base is null). With
+// TTT_CHECK_GUARDS on, a kGuardBytes guard sits in front of the first region and right
+// after the end of every region (16-byte aligned); the guards of a real workspace are
+// listed in t_guards.
 struct Carve {
   char* base;
   size_t off = 0;
-  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  bool guards;
+  explicit Carve(void* b)
+      : base(static_cast<char*>(b)), guards((g_checks.load() & TTT_CHECK_GUARDS) != 0) {
+    if (guards) guard();
+  }
+  void guard() {
+    off = (off + 15) & ~static_cast<size_t>(15);
+    if (base) t_guards.push_back(reinterpret_cast<unsigned*>(base + off));
+    off += kGuardBytes;
+  }
   void* take(size_t bytes) {
     off = (off + 255) & ~static_cast<size_t>(255);
     void* p = base ? base + off : nullptr;
     off += bytes;
+    if (guards) guard();
     return p;
   }
   template <typename T> T* take_n(long long n) { return static_cast<T*>(take(sizeof(T) * (size_t)n)); }
 };
+
+// Fills (check = false) or compares (check = true) every guard in t_guards.
+ttt_status run_guards(bool check, cudaStream_t s) {
+  for (size_t i0 = 0; i0 < t_guards.size(); i0 += kMaxGuards) {
+    GuardList g;
+    g.n = (int)std::min<size_t>(kMaxGuards, t_guards.size() - i0);
+    for (int i = 0; i < g.n; ++i) g.p[i] = t_guards[i0 + i];
+    TraceScope ts(check ? "guards_check" : "guards_fill", s);
+    const cudaError_t e = check ? guards_check(g, device_error_word(), s) : guards_fill(g, s);
+    if (e != cudaSuccess)
+      return fail(TTT_ERR_CUDA, "debug guards: %s", cudaGetErrorString(e));
+  }
+  return TTT_OK;
+}
+
+// One output of a call, for the non-finite scan.
+struct OutBuf {
+  const void* p;
+  long long n;
+  int dt;
+};
+
+// Start of a call's work on `s`: writes the guards of the workspace just planned.
+ttt_status checks_begin(cudaStream_t s) {
+  if (!(g_checks.load() & TTT_CHECK_GUARDS)) return TTT_OK;
+  return run_guards(false, s);
+}
+
+// End of a call's work on `s`: compares the guards and scans the outputs.
+ttt_status checks_end(cudaStream_t s, std::initializer_list<OutBuf> outs) {
+  const int f = g_checks.load();
+  if (f & TTT_CHECK_GUARDS) TTT_TRY(run_guards(true, s));
+  if (f & TTT_CHECK_FINITE)
+    for (const OutBuf& o : outs) {
+      if (!o.p || o.n <= 0) continue;
+      TraceScope ts("finite_scan", s);
+      const cudaError_t e = finite_scan(o.dt, o.p, o.n, device_error_word(), s);
+      if (e != cudaSuccess) return fail(TTT_ERR_CUDA, "finite scan: %s", cudaGetErrorString(e));
+    }
+  return TTT_OK;
+}
+
+// A call's body between checks_begin and checks_end; the end runs after a successful body.
+template <typename F>
+ttt_status with_checks(cudaStream_t s, std::initializer_list<OutBuf> outs, F&& body) {
+  TTT_TRY(checks_begin(s));
+  TTT_TRY(body());
+  return checks_end(s, outs);
+}
 
 ttt_status check_desc(const ttt_desc* d, int path) {
   if (!d) return fail(TTT_ERR_INVALID_ARG, "desc is NULL");
@@ -272,12 +346,19 @@ SwigluGemm features_problem(const ttt_desc& d, const void* X, const void* Wk, vo
   return g;
 }
 
+// Feature GEMM with the SwiGLU epilogue: tensor cores for bf16 operands (refused, never
+// rerouted, when the engine cannot take the problem), fp32 CUDA cores for fp32 operands.
 ttt_status run_swiglu(const char* name, const SwigluGemm& g, cudaStream_t s) {
   const GemmProblem& p = g.gemm;
   if (p.M <= 0 || g.n_valid <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
-  const bool tc = !force_simt() && umma_swiglu_supported(g);
-  TraceScope ts(g_trace.on ? engine_name(name, tc ? "tcgen05" : "simt") : name, s);
-  if (tc) return gemm_umma_swiglu(g, s, device_error_word(), wait_limit_ns());
+  if (p.A.dtype == DT_BF16 || p.B.dtype == DT_BF16) {
+    if (const char* why = umma_swiglu_unsupported_reason(g))
+      return fail(TTT_ERR_UNSUPPORTED, "%s: tensor-core engine: %s (M=%d N=%d K=%d)", name, why,
+                  p.M, p.N, p.K);
+    TraceScope ts(g_trace.on ? engine_name(name, "tcgen05") : name, s);
+    return gemm_umma_swiglu(g, s, device_error_word(), wait_limit_ns());
+  }
+  TraceScope ts(g_trace.on ? engine_name(name, "simt") : name, s);
   return gemm_simt_swiglu(g, s);
 }
 
@@ -354,7 +435,7 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
                      features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
                      s));
   TTT_TRY(state_delta_and_scan(d, b.phiA, v, W1, S_final, b.dS, b.Sc, b.scan_tmp, s));
-  if (!shared_qk && !force_simt() && !getenv("TTT_NO_FUSED_APPLY") &&
+  if (!shared_qk && !getenv("TTT_NO_FUSED_APPLY") &&
       fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
     // phi(Q) S_c with phi kept on chip
     TraceScope ts("fused_apply@tcgen05", s);
@@ -570,7 +651,7 @@ ttt_status momentum_impl(const ttt_desc& d, const void* q, const void* k, const 
   if (d.ns_steps > 0)
     TTT_TRY(run_ns(ot, b.dS, (int)(BH * C), ns_layout_single(d.m, d.h), d.ns_steps, mb.ns, s));
   TTT_TRY(chunk_states(d, b.dS, W1, S_final, b.Sc, nullptr, s));
-  if (!shared_qk && !force_simt() && !getenv("TTT_NO_FUSED_APPLY") &&
+  if (!shared_qk && !getenv("TTT_NO_FUSED_APPLY") &&
       fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
     TraceScope ts("fused_apply@tcgen05", s);
     return fused_apply(q, b.Wk, b.Sc, out, d.B, d.H, d.N, d.h, d.m, d.chunk,
@@ -1023,15 +1104,21 @@ ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* 
   ParBufs b;
   const size_t need = plan_parallel(d, nullptr, b);
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  t_guards.clear();
   plan_parallel(d, workspace, b);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d.N == 0) {
-    if (S_final)
-      TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, W1, b.Sc, S_final, (int)BH, d.H, 0, d.m, d.h,
-                                      d.order, d.w1_layout, nullptr, s));
-    return TTT_OK;
-  }
-  return parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s);
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long hm = (long long)d.h * d.m;
+  return with_checks(s, {{out, BH * d.N * d.h, ot}, {S_final, BH * hm, DT_F32}},
+                     [&]() -> ttt_status {
+    if (d.N == 0) {
+      if (S_final)
+        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, W1, b.Sc, S_final, (int)BH, d.H, 0, d.m,
+                                        d.h, d.order, d.w1_layout, nullptr, s));
+      return TTT_OK;
+    }
+    return parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s);
+  });
 }
 
 ttt_status ttt_linear_attn_fwd(const ttt_desc* desc, const void* q, const void* k, const void* v,
@@ -1051,15 +1138,20 @@ ttt_status ttt_linear_attn_fwd(const ttt_desc* desc, const void* q, const void* 
   LinBufs b;
   const size_t need = plan_linear(d, nullptr, b);
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  t_guards.clear();
   plan_linear(d, workspace, b);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d.N == 0) {
-    if (S_final)
-      TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, S0, b.Sc, S_final, (int)BH, d.H, 0, d.h, d.h,
-                                      d.order, d.w1_layout, nullptr, s));
-    return TTT_OK;
-  }
-  return linear_impl(d, q, k, v, eta, S0, out, S_final, b, s);
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  return with_checks(s, {{out, BH * d.N * d.h, ot}, {S_final, BH * d.h * d.h, DT_F32}},
+                     [&]() -> ttt_status {
+    if (d.N == 0) {
+      if (S_final)
+        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, S0, b.Sc, S_final, (int)BH, d.H, 0, d.h,
+                                        d.h, d.order, d.w1_layout, nullptr, s));
+      return TTT_OK;
+    }
+    return linear_impl(d, q, k, v, eta, S0, out, S_final, b, s);
+  });
 }
 
 ttt_status ttt_la_parallel_momentum_fwd(const ttt_desc* desc, const void* q, const void* k,
@@ -1083,15 +1175,21 @@ ttt_status ttt_la_parallel_momentum_fwd(const ttt_desc* desc, const void* q, con
   MomBufs b;
   const size_t need = plan_momentum(d, nullptr, b);
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  t_guards.clear();
   plan_momentum(d, workspace, b);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d.N == 0) {
-    if (S_final)
-      TTT_OP("chunk_scan", chunk_scan(DT_F32, b.p.dS, W1, b.p.Sc, S_final, (int)BH, d.H, 0, d.m,
-                                      d.h, d.order, d.w1_layout, nullptr, s));
-    return TTT_OK;
-  }
-  return momentum_impl(d, q, k, v, eta, alpha, W0, W2, W1, out, S_final, b, s);
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long hm = (long long)d.h * d.m;
+  return with_checks(s, {{out, BH * d.N * d.h, ot}, {S_final, BH * hm, DT_F32}},
+                     [&]() -> ttt_status {
+    if (d.N == 0) {
+      if (S_final)
+        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.p.dS, W1, b.p.Sc, S_final, (int)BH, d.H, 0,
+                                        d.m, d.h, d.order, d.w1_layout, nullptr, s));
+      return TTT_OK;
+    }
+    return momentum_impl(d, q, k, v, eta, alpha, W0, W2, W1, out, S_final, b, s);
+  });
 }
 
 ttt_status ttt_la_parallel_bwd(const ttt_desc* desc, const void* q, const void* k, const void* v,
@@ -1118,18 +1216,28 @@ ttt_status ttt_la_parallel_bwd(const ttt_desc* desc, const void* q, const void* 
   BwdBufs b;
   const size_t need = plan_backward(d, nullptr, b);
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  t_guards.clear();
   plan_backward(d, workspace, b);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const long long hm = (long long)d.h * d.m;
-  if (d.N == 0) {   // no outputs: dW1 = sum over the batch of dS_final, the rest zero
-    TTT_OP("fill", fill_f32(dW0, d.H * hm, 0.0f, s));
-    TTT_OP("fill", fill_f32(dW2, d.H * hm, 0.0f, s));
-    if (dS_final) TTT_OP("sum_batches", sum_batches(dS_final, d.B, d.H * hm, d.H * hm, dW1, s));
-    else TTT_OP("fill", fill_f32(dW1, d.H * hm, 0.0f, s));
-    return TTT_OK;
-  }
-  return backward_impl(d, q, k, v, eta, W0, W2, W1, dout, dS_final, dq, dk, dv, deta, dW0, dW2,
-                       dW1, b, s);
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long T = BH * d.N;
+  return with_checks(s, {{dq, T * d.h, ot}, {dk, T * d.h, ot}, {dv, T * d.h, ot},
+                         {deta, T, DT_F32}, {dW0, d.H * hm, DT_F32}, {dW2, d.H * hm, DT_F32},
+                         {dW1, d.H * hm, DT_F32}},
+                     [&]() -> ttt_status {
+    if (d.N == 0) {   // no outputs: dW1 = sum over the batch of dS_final, the rest zero
+      TTT_OP("fill", fill_f32(dW0, d.H * hm, 0.0f, s));
+      TTT_OP("fill", fill_f32(dW2, d.H * hm, 0.0f, s));
+      if (dS_final)
+        TTT_OP("sum_batches", sum_batches(dS_final, d.B, d.H * hm, d.H * hm, dW1, s));
+      else
+        TTT_OP("fill", fill_f32(dW1, d.H * hm, 0.0f, s));
+      return TTT_OK;
+    }
+    return backward_impl(d, q, k, v, eta, W0, W2, W1, dout, dS_final, dq, dk, dv, deta, dW0,
+                         dW2, dW1, b, s);
+  });
 }
 
 ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const void* k,
@@ -1153,9 +1261,11 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   RecBufs b;
   const size_t need = plan_recurrent(d, nullptr, b);
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  t_guards.clear();
   plan_recurrent(d, workspace, b);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  TTT_TRY(checks_begin(s));
   TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1o[0],
                               d.momentum ? M_io : nullptr, b.M_all, d.momentum, s));
   TTT_OP("prep_weights", prep_wk_blocked(ot, W0, W2, b.Wk[0], (int)BH, d.H, d.h, d.m, 0, s));
@@ -1217,7 +1327,10 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   if (W0_out || W2_out || W1_out || (d.momentum && M_io))
     TTT_OP("rec_finish", rec_finish(b.W_all, (int)BH, d.h, d.m, W0_out, W2_out, W1_out, b.M_all,
                                     d.momentum ? M_io : nullptr, s));
-  return TTT_OK;
+  const long long hm = (long long)d.h * d.m;
+  return checks_end(s, {{out, BH * N * d.h, ot}, {W0_out, BH * hm, DT_F32},
+                        {W2_out, BH * hm, DT_F32}, {W1_out, BH * hm, DT_F32},
+                        {d.momentum ? M_io : nullptr, BH * 3 * hm, DT_F32}});
 }
 
 }  // extern "C"
@@ -1292,14 +1405,19 @@ ttt_status ttt_lm_target(int32_t N, int32_t d, const void* X0, const float* conv
     return fail(TTT_ERR_INVALID_ARG, "X0, W_target and vbar must be 16-byte aligned");
   const size_t need = ttt_lm_target_workspace_bytes(N, d);
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  t_guards.clear();
+  Carve cv(workspace);
+  void* Xc = cv.take(2 * (size_t)N * d);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  TTT_OP("conv4_causal", conv4_causal(X0, conv_w, workspace, N, d, s));
-  GemmProblem p;
-  p.M = N; p.N = d; p.K = d;
-  p.A = {workspace, DT_BF16, false, d, 0, 0};
-  p.B = {W_target, DT_BF16, true, d, 0, 0};
-  p.C = {vbar, DT_BF16, d, 0, 0};
-  return run_gemm("gemm_lm_target", p, s);
+  return with_checks(s, {{vbar, (long long)N * d, DT_BF16}}, [&]() -> ttt_status {
+    TTT_OP("conv4_causal", conv4_causal(X0, conv_w, Xc, N, d, s));
+    GemmProblem p;
+    p.M = N; p.N = d; p.K = d;
+    p.A = {Xc, DT_BF16, false, d, 0, 0};
+    p.B = {W_target, DT_BF16, true, d, 0, 0};
+    p.C = {vbar, DT_BF16, d, 0, 0};
+    return run_gemm("gemm_lm_target", p, s);
+  });
 }
 
 ttt_status ttt_last_device_status(ttt_stream_t stream) {
@@ -1312,9 +1430,41 @@ ttt_status ttt_last_device_status(ttt_stream_t stream) {
     const unsigned z = 0;
     cudaMemcpyToSymbol(g_dev_err_word, &z, sizeof(z));
     if (w & DEVERR_TIMEOUT) return fail(TTT_ERR_TIMEOUT, "a bounded device wait ran out");
+    if (w & DEVERR_BOUNDS)
+      return fail(TTT_ERR_DEVICE, "a workspace guard was overwritten: a write went outside its "
+                  "region (word 0x%x)", w);
+    if (w & DEVERR_NONFINITE)
+      return fail(TTT_ERR_DEVICE, "an output holds NaN or Inf (word 0x%x)", w);
     return fail(TTT_ERR_DEVICE, "device-side check failed (word 0x%x)", w);
   }
   return TTT_OK;
+}
+
+ttt_status ttt_set_debug_checks(int32_t flags) {
+  if (flags & ~(TTT_CHECK_GUARDS | TTT_CHECK_FINITE))
+    return fail(TTT_ERR_INVALID_ARG, "unknown debug check flags 0x%x", (unsigned)flags);
+  g_checks.store(flags);
+  return TTT_OK;
+}
+
+int32_t ttt_get_debug_checks(void) { return g_checks.load(); }
+
+ttt_status ttt_debug_check_workspace(const ttt_desc* desc, int32_t path, void* workspace,
+                                     size_t workspace_bytes, ttt_stream_t stream) {
+  if (!(g_checks.load() & TTT_CHECK_GUARDS))
+    return fail(TTT_ERR_INVALID_ARG, "workspace guards are off (TTT_CHECK_GUARDS)");
+  TTT_TRY(check_desc(desc, path));
+  const size_t need = ttt_workspace_bytes(desc, path);
+  TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  t_guards.clear();
+  switch (path) {
+    case TTT_PATH_PARALLEL: { ParBufs b; plan_parallel(*desc, workspace, b); break; }
+    case TTT_PATH_LINEAR: { LinBufs b; plan_linear(*desc, workspace, b); break; }
+    case TTT_PATH_PARALLEL_MOMENTUM: { MomBufs b; plan_momentum(*desc, workspace, b); break; }
+    case TTT_PATH_PARALLEL_BWD: { BwdBufs b; plan_backward(*desc, workspace, b); break; }
+    default: { RecBufs b; plan_recurrent(*desc, workspace, b); break; }
+  }
+  return run_guards(true, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ttt_status ttt_debug_wait_timeout(int64_t timeout_ns, ttt_stream_t stream) {

@@ -206,3 +206,56 @@ def test_lm_target_host_checks():
     with pytest.raises(abi.TTTError) as ei:
         abi.ttt_debug_wait_timeout(10, stream=0)
     assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+
+
+def test_debug_checks_setting_and_guarded_workspace_sizes():
+    """TTT_CHECK_GUARDS adds a 256-byte guard in front of the first workspace region and
+    after each region; the setting is process-wide and unknown flags are refused (all host
+    logic: nothing reaches the driver)."""
+    assert abi.ttt_get_debug_checks() == 0
+    plain = {p: abi.ttt_workspace_bytes(lm_desc(), p)
+             for p in (abi.TTT_PATH_PARALLEL, abi.TTT_PATH_PARALLEL_BWD)}
+    rec = abi.ttt_workspace_bytes(lm_desc(update_mask=7), abi.TTT_PATH_RECURRENT)
+    assert rec > 0
+    tgt = abi.ttt_lm_target_workspace_bytes(1000, 64)
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_set_debug_checks(8)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    try:
+        abi.ttt_set_debug_checks(abi.TTT_CHECK_GUARDS | abi.TTT_CHECK_FINITE)
+        assert abi.ttt_get_debug_checks() == 3
+        par = abi.ttt_workspace_bytes(lm_desc(), abi.TTT_PATH_PARALLEL)
+        # 5 regions at lm (blocked weights, two feature buffers, deltas, chunk states):
+        # 6 guards, each region end rounded to 16 bytes and the next region to 256
+        assert plain[abi.TTT_PATH_PARALLEL] + 6 * 256 <= par <= \
+            plain[abi.TTT_PATH_PARALLEL] + 6 * 256 + 6 * 256
+        assert abi.ttt_workspace_bytes(lm_desc(), abi.TTT_PATH_PARALLEL_BWD) > \
+            plain[abi.TTT_PATH_PARALLEL_BWD]
+        assert abi.ttt_workspace_bytes(lm_desc(update_mask=7), abi.TTT_PATH_RECURRENT) > rec
+        assert abi.ttt_lm_target_workspace_bytes(1000, 64) >= tgt + 2 * 256
+        # a workspace sized with guards off is refused with guards on, before any launch
+        d = lm_desc()
+        with pytest.raises(abi.TTTError) as ei:
+            abi.ttt_la_parallel_fwd(d, 256, 512, 768, 1024, 2048, 4096, 8192, 16384, None,
+                                    1 << 20, plain[abi.TTT_PATH_PARALLEL], 0)
+        assert ei.value.status == abi.TTT_ERR_WORKSPACE
+        abi.ttt_set_debug_checks(0)
+        with pytest.raises(abi.TTTError) as ei:   # guards off: nothing to compare
+            abi.ttt_debug_check_workspace(d, abi.TTT_PATH_PARALLEL, 1 << 20, 1 << 30, 0)
+        assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    finally:
+        abi.ttt_set_debug_checks(0)
+    assert abi.ttt_workspace_bytes(lm_desc(), abi.TTT_PATH_PARALLEL) == \
+        plain[abi.TTT_PATH_PARALLEL]
+
+
+def test_bf16_mode_refuses_shapes_the_tensor_cores_cannot_take():
+    """bf16 mode has one engine: a request it cannot take is refused up front with
+    TTT_ERR_UNSUPPORTED (never rerouted to the CUDA cores)."""
+    for h, m in ((12, 64), (64, 20)):
+        d = lm_desc(B=1, H=1, N=256, h=h, m=m, chunk=64)
+        assert abi.ttt_workspace_bytes(d, abi.TTT_PATH_PARALLEL) == 0
+        with pytest.raises(abi.TTTError) as ei:
+            abi.ttt_la_parallel_fwd(d, 256, 512, 768, 1024, 2048, 4096, 8192, 16384, None,
+                                    1 << 20, 1 << 30, 0)
+        assert ei.value.status == abi.TTT_ERR_UNSUPPORTED
