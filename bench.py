@@ -164,13 +164,17 @@ def kernel_work(name: str, wl, form: str):
         return table.get(base, (None, None))
     # parallel forms; the training step runs the forward kernels twice (forward call and
     # the backward's recomputation)
-    feats = 1 if wl.kind == "inplace" else 2
     fw = 2 if form == "train" else 1
+    # the forward's key side runs as one fused kernel (phi(K) eta on chip) for bf16 with
+    # h = 128 or 256 and distinct q, k; the backward always recomputes it unfused
+    fused_key = wl.dtype == "bf16" and h in (128, 256) and wl.kind != "inplace"
+    unfused_k = fw - (1 if fused_key else 0)
     scan = BH * C * hm * (4.0 + es) + 2 * 4.0 * BH * hm
     table = {
         "prep_weights": ("hbm", fw * (2 * hm * 4.0 * H + 2 * mpad * h * es * H)),
-        "gemm_features_k": ("tensor", fw * 4.0 * hm * T),
-        "gemm_state_delta": ("tensor", fw * 2.0 * hm * T),
+        "fused_delta": ("tensor", 6.0 * hm * T),   # phi(K) (4hm) and phi(K)^T eta V (2hm)
+        "gemm_features_k": ("tensor", unfused_k * 4.0 * hm * T),
+        "gemm_state_delta": ("tensor", unfused_k * 2.0 * hm * T),
         "chunk_scan": ("hbm", fw * scan),
         "fused_apply": ("tensor", 6.0 * hm * T),   # phi(Q) (4hm) and phi(Q) S_c (2hm)
         "gemm_features_q": ("tensor", 4.0 * hm * T),

@@ -133,6 +133,34 @@ ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* 
                                ttt_stream_t stream);
 
 /*
+ * One contiguous shard of a sequence in the parallel form, for a sequence split over
+ * devices (context parallelism: "In-Place Test-Time Training", section 3.4, the chunk
+ * deltas of earlier shards enter a shard only through their sum; "Test-Time Training with
+ * KV Binding Is Secretly Linear Attention", 前置知识 / 前缀扫描). The same computation as
+ * ttt_la_parallel_fwd on the shard's tokens, except that the state the shard starts from
+ * is, for every (batch, head),
+ *     W1[head] (zero when W1 is NULL) + sum_{i < n_prior} prior[i, batch, head],
+ * and that `out` may be NULL, in which case only S_final is formed (no query-side work).
+ * A sequence over R shards: shard r calls this with W1 = NULL, out = NULL to get its total
+ * delta T_r; the totals are gathered in rank order; shard r calls it again with W1,
+ * prior = T_0 .. T_{r-1} (n_prior = r) and out: its outputs are those of the unsharded
+ * call, and the last shard's S_final is the sequence's final state.
+ *
+ *   desc       as for ttt_la_parallel_fwd; every shard but the last must hold whole chunks
+ *   W1         nullable; per-head initial state (layout per w1_layout)
+ *   prior      [n_prior, B, H, m, h] fp32 (W1's layout per entry; 16-byte aligned), or
+ *              NULL with n_prior = 0; n_prior <= 4096
+ *   out        nullable [B,H,N,h] dtype; S_final nullable, but not both NULL
+ *   workspace  >= ttt_workspace_bytes(desc, TTT_PATH_PARALLEL) bytes
+ * Errors and streams as for ttt_la_parallel_fwd.
+ */
+ttt_status ttt_la_parallel_fwd_shard(const ttt_desc* desc, const void* q, const void* k,
+                                     const void* v, const float* eta, const float* W0,
+                                     const float* W2, const float* W1, const float* prior,
+                                     int32_t n_prior, void* out, float* S_final, void* workspace,
+                                     size_t workspace_bytes, ttt_stream_t stream);
+
+/*
  * Parallel last-layer-only form with momentum and orthogonalisation of the W1 update
  * ("Test-Time Training with KV Binding Is Secretly Linear Attention", section 方法步骤详情:
  * simplification variant 2 keeps momentum and Newton-Schulz; the pages' recurrent -> parallel

@@ -22,7 +22,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libttt_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 SOURCES = ["ttt_api.cu", "ops.cu", "gemm_simt.cu", "gemm_umma.cu", "ns_mma.cu", "apply_fused.cu",
-           "checks.cu"]
+           "checks.cu", "delta_fused.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
               "-I" + os.path.join(ROOT, "include")]

@@ -96,6 +96,16 @@ ttt_status fused_apply(const void* q, const void* Wk, const void* Sc, void* out,
                        int N, int h, int m, int chunk, unsigned* err,
                        unsigned long long wait_ns, cudaStream_t s);
 
+// Key side of the parallel form fused (delta_fused.cu): dS[bh, c] = sign * phi(K_c)^T
+// diag(eta_c) V_c per (batch, head) and chunk with phi kept in shared memory. k, v
+// [B,H,N,h] bf16; eta [B,H,N] fp32; Wk the blocked [W0/2 ; W2] operand per head
+// ([H, 2 * mpad, h]); dS [B*H, C, m, h] fp32, written. Needs h = 128 or 256.
+bool fused_delta_supported(int dtype, int h, int m, const void* k, const void* v,
+                           const float* eta, const void* Wk, const float* dS);
+ttt_status fused_delta(const void* k, const void* v, const float* eta, const void* Wk, float* dS,
+                       int B, int H, int N, int h, int m, int chunk, int sign, unsigned* err,
+                       unsigned long long wait_ns, cudaStream_t s);
+
 bool umma_swiglu_supported(const SwigluGemm& g);
 const char* umma_swiglu_unsupported_reason(const SwigluGemm& g);
 ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream);

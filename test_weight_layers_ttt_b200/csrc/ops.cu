@@ -76,18 +76,22 @@ __global__ void scale_rows8_kernel(const uint4* X, const float* eta, uint4* Xs, 
 // ------------------------------------------------------------------ chunk prefix scan
 // One thread per state element; the chunk axis (tens of chunks) is walked sequentially so
 // every delta is read once and every chunk state written once.
+// Initial state of (b, head) bh: W1[bh % H] (zero when W1 is null) plus the n_prior states
+// prior[i, bh] ([n_prior, BH, ...] in W1's layout).
 template <typename OT>
 __global__ void chunk_scan_kernel(const float* __restrict__ dS, const float* __restrict__ W1,
+                                  const float* __restrict__ prior, int n_prior,
                                   OT* __restrict__ Sc, float* __restrict__ S_final, int BH,
                                   int H, int C, int m, int h, int order, int layout) {
   const long long per = (long long)m * h;
   TTT_GRID_LOOP(idx, per * BH) {
     const long long bh = idx / per, e = idx - bh * per;
     const int k = (int)(e / h), j = (int)(e - (long long)k * h);
-    const long long w_off = (bh % H) * per + (layout == 0 ? e : (long long)j * m + k);
-    float s = W1[w_off];
+    const long long le = layout == 0 ? e : (long long)j * m + k;   // e in W1's layout
+    float s = W1 ? W1[(bh % H) * per + le] : 0.0f;
+    for (int i = 0; i < n_prior; ++i) s += prior[((long long)i * BH + bh) * per + le];
     const float* d = dS + bh * C * per + e;
-    OT* out = Sc + bh * C * per + e;
+    OT* out = Sc ? Sc + bh * C * per + e : nullptr;
     int c = 0;
     // Four chunks per step with the loads issued first, so each thread keeps four
     // independent loads in flight.
@@ -98,22 +102,22 @@ __global__ void chunk_scan_kernel(const float* __restrict__ dS, const float* __r
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         if (order == 1) {
-          out[(long long)(c + u) * per] = from_f32<OT>(s);
+          if (out) out[(long long)(c + u) * per] = from_f32<OT>(s);
           s += dv[u];
         } else {
           s += dv[u];
-          out[(long long)(c + u) * per] = from_f32<OT>(s);
+          if (out) out[(long long)(c + u) * per] = from_f32<OT>(s);
         }
       }
     }
     for (; c < C; ++c) {
       const float dv = __ldcs(d + (long long)c * per);
       if (order == 1) {
-        out[(long long)c * per] = from_f32<OT>(s);
+        if (out) out[(long long)c * per] = from_f32<OT>(s);
         s += dv;
       } else {
         s += dv;
-        out[(long long)c * per] = from_f32<OT>(s);
+        if (out) out[(long long)c * per] = from_f32<OT>(s);
       }
     }
     if (S_final) S_final[bh * per + (layout == 0 ? e : (long long)j * m + k)] = s;
@@ -124,14 +128,20 @@ __global__ void chunk_scan_kernel(const float* __restrict__ dS, const float* __r
 // m*h divisible by 4; the chunk loop keeps four 16-byte loads in flight.
 template <typename OT>
 __global__ void chunk_scan4_kernel(const float4* __restrict__ dS, const float4* __restrict__ W1,
+                                   const float4* __restrict__ prior, int n_prior,
                                    OT* __restrict__ Sc, float4* __restrict__ S_final, int BH,
                                    int H, int C, long long per4, int order) {
   TTT_GRID_LOOP(idx, per4 * BH) {
     const long long bh = idx / per4, e = idx - bh * per4;
-    float4 s = W1[(bh % H) * per4 + e];
+    float4 s = W1 ? W1[(bh % H) * per4 + e] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int i = 0; i < n_prior; ++i) {
+      const float4 p = prior[((long long)i * BH + bh) * per4 + e];
+      s.x += p.x; s.y += p.y; s.z += p.z; s.w += p.w;
+    }
     const float4* d = dS + bh * C * per4 + e;
-    OT* out = Sc + (bh * C * per4 + e) * 4;
+    OT* out = Sc ? Sc + (bh * C * per4 + e) * 4 : nullptr;
     auto put = [&](int c, const float4& v) {
+      if (!out) return;
       OT* o = out + (long long)c * per4 * 4;
       if constexpr (sizeof(OT) == 2) {
         uint2 pk;
@@ -400,6 +410,27 @@ __global__ void transpose_kernel(const float* in, float* out, int rows, int cols
   for (int k = ty; k < 32; k += 8) {
     const int r = r0 + k, c = c0 + tx;
     if (r < rows && c < cols) t[k][tx] = in[z * n + (long long)r * cols + c];
+  }
+  __syncthreads();
+  for (int k = ty; k < 32; k += 8) {
+    const int c = c0 + k, r = r0 + tx;   // out [cols, rows]
+    if (r < rows && c < cols) out[z * n + (long long)c * rows + r] = t[tx][k];
+  }
+}
+
+// out[z] = sum_{i < n_in} in[i * Z + z]^T for Z matrices [rows, cols] per input (the same
+// tiling as transpose_kernel); grid (ceil(cols/32), ceil(rows/32), Z).
+__global__ void transpose_sum_kernel(const float* in, int n_in, float* out, int rows, int cols) {
+  __shared__ float t[32][33];
+  const long long z = blockIdx.z, Z = gridDim.z, n = (long long)rows * cols;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32, tx = threadIdx.x, ty = threadIdx.y;
+  for (int k = ty; k < 32; k += 8) {
+    const int r = r0 + k, c = c0 + tx;
+    if (r < rows && c < cols) {
+      float acc = 0.0f;
+      for (int i = 0; i < n_in; ++i) acc += in[((long long)i * Z + z) * n + (long long)r * cols + c];
+      t[k][tx] = acc;
+    }
   }
   __syncthreads();
   for (int k = ty; k < 32; k += 8) {
@@ -721,17 +752,24 @@ cudaError_t scale_rows(int ot, const void* X, const float* eta, void* Xs, long l
   });
 }
 
-cudaError_t chunk_scan(int ot, const float* dS, const float* W1, void* Sc, float* S_final, int BH,
-                       int H, int C, int m, int h, int order, int layout, float* scratch,
-                       cudaStream_t s) {
+cudaError_t chunk_scan(int ot, const float* dS, const float* W1, const float* prior, int n_prior,
+                       void* Sc, float* S_final, int BH, int H, int C, int m, int h, int order,
+                       int layout, float* scratch, cudaStream_t s) {
   const long long per = (long long)m * h;
   if (layout == 1 && scratch) {
-    // transposed W1 / S_final: transpose once on each side and scan in the [m, h] layout
-    float* W1t = scratch;
+    // transposed W1 / S_final: transpose once on each side and scan in the [m, h] layout;
+    // the prior states (W1's layout) are summed and transposed into the region of the
+    // transposed final state (each element is read there before the scan writes it)
+    float* W1t = W1 ? scratch : nullptr;
     float* Sft = scratch + (long long)H * per;
-    transpose_kernel<<<dim3((m + 31) / 32, (h + 31) / 32, H), dim3(32, 8), 0, s>>>(W1, W1t, h, m);
-    cudaError_t e = chunk_scan(ot, dS, W1t, Sc, S_final ? Sft : nullptr, BH, H, C, m, h, order, 0,
-                               nullptr, s);
+    if (W1)
+      transpose_kernel<<<dim3((m + 31) / 32, (h + 31) / 32, H), dim3(32, 8), 0, s>>>(W1, W1t, h,
+                                                                                    m);
+    if (n_prior > 0)
+      transpose_sum_kernel<<<dim3((m + 31) / 32, (h + 31) / 32, BH), dim3(32, 8), 0, s>>>(
+          prior, n_prior, Sft, h, m);
+    cudaError_t e = chunk_scan(ot, dS, W1t, n_prior > 0 ? Sft : nullptr, n_prior > 0 ? 1 : 0, Sc,
+                               S_final ? Sft : nullptr, BH, H, C, m, h, order, 0, nullptr, s);
     if (e != cudaSuccess || !S_final) return e;
     transpose_kernel<<<dim3((h + 31) / 32, (m + 31) / 32, BH), dim3(32, 8), 0, s>>>(Sft, S_final,
                                                                                   m, h);
@@ -739,17 +777,19 @@ cudaError_t chunk_scan(int ot, const float* dS, const float* W1, void* Sc, float
   }
   const bool vec = layout == 0 && per % 4 == 0 &&
                    ((reinterpret_cast<uintptr_t>(dS) | reinterpret_cast<uintptr_t>(W1) |
-                     reinterpret_cast<uintptr_t>(Sc) | reinterpret_cast<uintptr_t>(S_final)) & 15) == 0;
+                     reinterpret_cast<uintptr_t>(prior) | reinterpret_cast<uintptr_t>(Sc) |
+                     reinterpret_cast<uintptr_t>(S_final)) & 15) == 0;
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
     if (vec) {
       const long long n4 = per / 4 * BH;
       chunk_scan4_kernel<OT><<<grid_for(n4, 256, 148 * 16), 256, 0, s>>>(
           reinterpret_cast<const float4*>(dS), reinterpret_cast<const float4*>(W1),
-          static_cast<OT*>(Sc), reinterpret_cast<float4*>(S_final), BH, H, C, per / 4, order);
+          reinterpret_cast<const float4*>(prior), n_prior, static_cast<OT*>(Sc),
+          reinterpret_cast<float4*>(S_final), BH, H, C, per / 4, order);
     } else {
       chunk_scan_kernel<OT><<<grid_for(per * BH, 256, 148 * 64), 256, 0, s>>>(
-          dS, W1, static_cast<OT*>(Sc), S_final, BH, H, C, m, h, order, layout);
+          dS, W1, prior, n_prior, static_cast<OT*>(Sc), S_final, BH, H, C, m, h, order, layout);
     }
     return cudaGetLastError();
   });

@@ -22,14 +22,16 @@ cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, 
 cudaError_t scale_rows(int ot, const void* X, const float* eta, void* Xs, long long rows, int w,
                        cudaStream_t s);
 
-// Chunk prefix sums: S starts at W1[bh % H] (layout 0 [m,h] / 1 [h,m]); for each chunk c
-// the state read by chunk c is written to Sc[bh, c] (OT, [m,h]): inclusive of dS[bh, c]
-// (order 0) or exclusive (order 1). The state after the last chunk goes to S_final
-// (fp32, W1's layout) when non-null. With layout 1 and a scratch of (H + BH) * m * h floats,
-// W1 and S_final are transposed through it so the scan itself runs on 16-byte vectors.
-cudaError_t chunk_scan(int ot, const float* dS, const float* W1, void* Sc, float* S_final, int BH,
-                       int H, int C, int m, int h, int order, int layout, float* scratch,
-                       cudaStream_t s);
+// Chunk prefix sums: S starts at W1[bh % H] (layout 0 [m,h] / 1 [h,m]; zero when W1 is
+// null) plus the n_prior states prior[i, bh] (W1's layout, [n_prior, BH, ...]); for each
+// chunk c the state read by chunk c is written to Sc[bh, c] (OT, [m,h]; skipped when Sc is
+// null): inclusive of dS[bh, c] (order 0) or exclusive (order 1). The state after the last
+// chunk goes to S_final (fp32, W1's layout) when non-null. With layout 1 and a scratch of
+// (H + BH) * m * h floats, W1, the priors and S_final are transposed through it so the scan
+// itself runs on 16-byte vectors.
+cudaError_t chunk_scan(int ot, const float* dS, const float* W1, const float* prior, int n_prior,
+                       void* Sc, float* S_final, int BH, int H, int C, int m, int h, int order,
+                       int layout, float* scratch, cudaStream_t s);
 
 // Recurrent-state helpers. Per (b, head) the fp32 state W_all holds [W0 (h*m) | W1 (m*h) |
 // W2 (h*m)]; momentum and the update buffer U use the same part layout.

@@ -385,12 +385,15 @@ ttt_status state_deltas(const ttt_desc& d, const void* X_eta, const void* v, flo
   return TTT_OK;
 }
 
+// Prefix scan of the chunk deltas to the state read by every chunk (Sc, skipped when null)
+// and the final state, from W1 (zero when null) plus n_prior prior states.
 ttt_status chunk_states(const ttt_desc& d, const float* dS, const float* W1, float* S_final,
-                        void* Sc, float* scan_tmp, cudaStream_t s) {
+                        void* Sc, float* scan_tmp, cudaStream_t s, const float* prior = nullptr,
+                        int n_prior = 0) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
-  TTT_OP("chunk_scan", chunk_scan(ot, dS, W1, Sc, S_final, (int)BH, d.H, (int)C, d.m, d.h,
-                                  d.order, d.w1_layout, scan_tmp, s));
+  TTT_OP("chunk_scan", chunk_scan(ot, dS, W1, prior, n_prior, Sc, S_final, (int)BH, d.H, (int)C,
+                                  d.m, d.h, d.order, d.w1_layout, scan_tmp, s));
   return TTT_OK;
 }
 
@@ -422,19 +425,40 @@ ttt_status chunk_outputs(const ttt_desc& d, const void* X_q, const void* Sc, voi
   return TTT_OK;
 }
 
-ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
-                         const float* eta, const float* W0, const float* W2, const float* W1,
-                         void* out, float* S_final, const ParBufs& b, cudaStream_t s) {
+// The chunks' state deltas dS: fused (phi(K) eta kept on chip, one kernel) when the
+// problem allows it, else the feature GEMM (phi(K) eta, and phi(Q) when q == k, through
+// HBM) followed by the state-delta GEMM.
+ttt_status key_side(const ttt_desc& d, const void* k, const void* v, const float* eta,
+                    const ParBufs& b, bool shared_qk, cudaStream_t s) {
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
-  const bool shared_qk = (q == k);
-
-  TTT_OP("prep_weights",
-         prep_wk_blocked(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
-  // phi(K) eta (and phi(Q) when q == k)
+  if (!shared_qk && !getenv("TTT_NO_FUSED_DELTA") &&
+      fused_delta_supported(ot, d.h, d.m, k, v, eta, b.Wk, b.dS)) {
+    TraceScope ts("fused_delta@tcgen05", s);
+    return fused_delta(k, v, eta, b.Wk, b.dS, d.B, d.H, d.N, d.h, d.m, d.chunk, d.sign,
+                       device_error_word(), wait_limit_ns(), s);
+  }
   TTT_TRY(run_swiglu("gemm_features_k",
                      features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
                      s));
-  TTT_TRY(state_delta_and_scan(d, b.phiA, v, W1, S_final, b.dS, b.Sc, b.scan_tmp, s));
+  return state_deltas(d, b.phiA, v, b.dS, s);
+}
+
+// The parallel form; the initial state of (b, head) is W1[head] (zero when W1 is null)
+// plus the n_prior states prior[i, b, head]. With out null only the final state is formed
+// (no query side, no per-chunk states).
+ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
+                         const float* eta, const float* W0, const float* W2, const float* W1,
+                         void* out, float* S_final, const ParBufs& b, cudaStream_t s,
+                         const float* prior = nullptr, int n_prior = 0) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const bool shared_qk = (q == k) && out != nullptr;
+
+  TTT_OP("prep_weights",
+         prep_wk_blocked(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
+  TTT_TRY(key_side(d, k, v, eta, b, shared_qk, s));
+  TTT_TRY(chunk_states(d, b.dS, W1, S_final, out ? b.Sc : nullptr, b.scan_tmp, s, prior,
+                       n_prior));
+  if (!out) return TTT_OK;
   if (!shared_qk && !getenv("TTT_NO_FUSED_APPLY") &&
       fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
     // phi(Q) S_c with phi kept on chip
@@ -642,10 +666,7 @@ ttt_status momentum_impl(const ttt_desc& d, const void* q, const void* k, const 
   const bool shared_qk = (q == k);
   TTT_OP("prep_weights",
          prep_wk_blocked(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
-  TTT_TRY(run_swiglu("gemm_features_k",
-                     features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
-                     s));
-  TTT_TRY(state_deltas(d, b.phiA, v, b.dS, s));
+  TTT_TRY(key_side(d, k, v, eta, b, shared_qk, s));
   if (d.momentum)
     TTT_OP("momentum_scan", momentum_scan(b.dS, alpha, (int)BH, (int)C, (long long)d.h * d.m, s));
   if (d.ns_steps > 0)
@@ -1113,11 +1134,54 @@ ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* 
                      [&]() -> ttt_status {
     if (d.N == 0) {
       if (S_final)
-        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, W1, b.Sc, S_final, (int)BH, d.H, 0, d.m,
-                                        d.h, d.order, d.w1_layout, nullptr, s));
+        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, W1, nullptr, 0, b.Sc, S_final, (int)BH, d.H,
+                                        0, d.m, d.h, d.order, d.w1_layout, nullptr, s));
       return TTT_OK;
     }
     return parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s);
+  });
+}
+
+ttt_status ttt_la_parallel_fwd_shard(const ttt_desc* desc, const void* q, const void* k,
+                                     const void* v, const float* eta, const float* W0,
+                                     const float* W2, const float* W1, const float* prior,
+                                     int32_t n_prior, void* out, float* S_final, void* workspace,
+                                     size_t workspace_bytes, ttt_stream_t stream) {
+  TTT_TRY(check_desc(desc, TTT_PATH_PARALLEL));
+  const ttt_desc& d = *desc;
+  const long long BH = (long long)d.B * d.H;
+  if (BH == 0) return TTT_OK;
+  if (!W0 || !W2) return fail(TTT_ERR_INVALID_ARG, "W0 and W2 must not be NULL");
+  if (n_prior < 0 || n_prior > 4096) return fail(TTT_ERR_INVALID_ARG, "n_prior must be in 0..4096");
+  if (n_prior > 0 && (!prior || !al16(prior)))
+    return fail(TTT_ERR_INVALID_ARG, "prior must be a 16-byte aligned pointer when n_prior > 0");
+  if (!out && !S_final) return fail(TTT_ERR_INVALID_ARG, "out and S_final are both NULL");
+  if ((W1 && !al16(W1)) || !al16(W0) || !al16(W2))
+    return fail(TTT_ERR_INVALID_ARG, "the weights must be 16-byte aligned");
+  if (d.N > 0) {
+    if (!q || !k || !v || !eta)
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v and eta must not be NULL");
+    if (!al16(q) || !al16(k) || !al16(v) || (out && !al16(out)))
+      return fail(TTT_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+  }
+  ParBufs b;
+  const size_t need = plan_parallel(d, nullptr, b);
+  TTT_TRY(check_ws(workspace, workspace_bytes, need));
+  t_guards.clear();
+  plan_parallel(d, workspace, b);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long hm = (long long)d.h * d.m;
+  return with_checks(s, {{out, BH * d.N * d.h, ot}, {S_final, BH * hm, DT_F32}},
+                     [&]() -> ttt_status {
+    if (d.N == 0) {
+      if (S_final)
+        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, W1, prior, n_prior, nullptr, S_final,
+                                        (int)BH, d.H, 0, d.m, d.h, d.order, d.w1_layout,
+                                        b.scan_tmp, s));
+      return TTT_OK;
+    }
+    return parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s, prior, n_prior);
   });
 }
 
@@ -1146,8 +1210,8 @@ ttt_status ttt_linear_attn_fwd(const ttt_desc* desc, const void* q, const void* 
                      [&]() -> ttt_status {
     if (d.N == 0) {
       if (S_final)
-        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, S0, b.Sc, S_final, (int)BH, d.H, 0, d.h,
-                                        d.h, d.order, d.w1_layout, nullptr, s));
+        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.dS, S0, nullptr, 0, b.Sc, S_final, (int)BH, d.H,
+                                        0, d.h, d.h, d.order, d.w1_layout, nullptr, s));
       return TTT_OK;
     }
     return linear_impl(d, q, k, v, eta, S0, out, S_final, b, s);
@@ -1184,8 +1248,8 @@ ttt_status ttt_la_parallel_momentum_fwd(const ttt_desc* desc, const void* q, con
                      [&]() -> ttt_status {
     if (d.N == 0) {
       if (S_final)
-        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.p.dS, W1, b.p.Sc, S_final, (int)BH, d.H, 0,
-                                        d.m, d.h, d.order, d.w1_layout, nullptr, s));
+        TTT_OP("chunk_scan", chunk_scan(DT_F32, b.p.dS, W1, nullptr, 0, b.p.Sc, S_final, (int)BH,
+                                        d.H, 0, d.m, d.h, d.order, d.w1_layout, nullptr, s));
       return TTT_OK;
     }
     return momentum_impl(d, q, k, v, eta, alpha, W0, W2, W1, out, S_final, b, s);

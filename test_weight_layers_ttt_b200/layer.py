@@ -70,6 +70,36 @@ def la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk, *, order="update_apply", si
     return out, S
 
 
+def la_parallel_fwd_shard(q, k, v, eta, W0, W2, W1, chunk, *, prior=None, state_only=False,
+                          order="update_apply", sign=1, w_in_layout=0, w1_layout=0, m=None,
+                          out=None, ws=None, stream=None):
+    """One contiguous shard of a sequence (context parallelism): the parallel form from the
+    initial state W1 (zeros when None) plus the sum of ``prior`` [n, B, H, m, h] (W1's
+    layout per entry) along its first axis. ``state_only`` skips the outputs. Returns
+    (out or None, final state). ``m`` is needed when W1 is None."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    _need(eta, "eta", torch.float32)
+    for t, n in ((W0, "W0"), (W2, "W2"), (W1, "W1"), (prior, "prior")):
+        _need(t, n, torch.float32)
+    B, H, N, h = q.shape
+    if m is None:
+        m = W1.shape[1] if w1_layout == 0 else W1.shape[2]
+    desc = abi.ttt_desc(B=B, H=H, N=N, h=h, m=m, chunk=chunk, dtype=_dtype_code(q),
+                        order=ORDERS[order], sign=sign, w_in_layout=w_in_layout,
+                        w1_layout=w1_layout)
+    if out is None and not state_only:
+        out = torch.empty_like(q)
+    S = torch.empty((B, H, m, h) if w1_layout == 0 else (B, H, h, m), dtype=torch.float32,
+                    device=q.device)
+    if ws is None:
+        ws = workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_PARALLEL), q.device)
+    n_prior = 0 if prior is None else prior.shape[0]
+    abi.ttt_la_parallel_fwd_shard(desc, q, k, v, eta, W0, W2, W1, prior if n_prior else None,
+                                  n_prior, None if state_only else out, S, ws, stream=stream)
+    return (None if state_only else out), S
+
+
 def la_parallel_momentum_fwd(q, k, v, eta, W0, W2, W1, chunk, *, order="update_apply", sign=1,
                              alpha=None, ns_steps=0, w_in_layout=0, return_state=True,
                              out=None, ws=None, stream=None):
