@@ -514,6 +514,9 @@ def run_gpu(args, rank, local, world):
         forms.insert(2, "parallel_momentum")
         # one training step of the layer: parallel forward + backward
         forms.insert(3, "train")
+    if args.forms:
+        keep = set(args.forms.split(","))
+        forms = [f for f in forms if f in keep]
     lin, l1 = g["layouts"]
     if wl.kind == "inplace":
         # the value target is part of the In-Place step; timed on its own below
@@ -796,6 +799,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--override", default="",
                     help="comma-separated workload field overrides for profiling, e.g. B=1,H=4")
+    ap.add_argument("--forms", default="",
+                    help="comma-separated subset of the forms to time (profiling), e.g. "
+                         "parallel; the default times every form of the workload")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -812,7 +818,8 @@ def main():
         tbuild.build()
     wl, peaks, res, x = run_gpu(args, rank, local, world)
     if rank == 0:
-        form = "parallel" if "parallel" in res["forms"] else "recurrent"
+        form = next((f for f in ("parallel", "recurrent") if f in res["forms"]),
+                    next(iter(res["forms"])))
         head = dict(res["forms"][form])
         if "lm_target" in res["forms"]:
             # In-Place step = target prologue + parallel update/apply

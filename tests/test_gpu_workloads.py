@@ -193,6 +193,27 @@ def test_inplace_full_width_two_chunks(inplace):
     assert rel(host(S[0, 0]) - x["W_down"], Wref - x["W_down"]) <= TOL["bf16"]
 
 
+def test_inplace_reduced_width_all_chunks_match_the_oracle(inplace):
+    """All 32 chunks of the In-Place workload (N = 32768, chunk 1024, q = k, apply->update,
+    the exclusive scan over 32 chunk states) at reduced width d = 512, d_H = 1408 against
+    the oracle's sequential apply-then-update route."""
+    wl = WORKLOADS["inplace"].scaled(h=512, m=1408)
+    x = make_inplace_inputs(wl, seed=777)
+    vb, out, S = _inplace_gpu(x, wl.N, wl)
+    abi.ttt_last_device_status()
+    Vref = O.lm_target(x["X0"], x["conv_w"], x["W_target"])
+    assert rel(host(vb), Vref) <= TOL["bf16"]
+    ref, Wref = O.inplace_sequential(x["Hs"], x["Wg"], x["Wu"], x["W_down"], Vref, wl.chunk,
+                                     1e-3)
+    Oh = host(out[0, 0])
+    assert rel(Oh, ref) <= TOL["bf16"]
+    assert rel(host(S[0, 0]), Wref) <= TOL["bf16"]
+    assert rel(host(S[0, 0]) - x["W_down"], Wref - x["W_down"]) <= TOL["bf16"]
+    # the last chunk's outputs alone (read the state after 31 exclusive-scan steps)
+    last = slice(wl.N - wl.chunk, wl.N)
+    assert rel(Oh[last], ref[last]) <= TOL["bf16"]
+
+
 def test_inplace_full_length_resume_is_bitwise(inplace):
     wl, x = inplace
     vb, out, S = _inplace_gpu(x, wl.N, wl)
