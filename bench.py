@@ -101,7 +101,7 @@ def rec_splits(wl) -> int:
     the largest power of two dividing the chunk with splits of at least 256 tokens (a
     multiple of 64), one wave of tiles and at most 32 MB of fp32 partials."""
     BH, L = wl.B * wl.H, wl.chunk
-    tiles = BH * (-(-wl.m // 128)) * (-(-wl.h // 256))
+    tiles = BH * (-(-2 * wl.m // 128)) * (-(-wl.h // 256))   # the merged W0 / W2 gradient GEMM
     partial = BH * 3 * wl.h * wl.m * 4
     best, sp = 1, 2
     while sp <= 64:
@@ -143,6 +143,9 @@ def kernel_work(name: str, wl, form: str):
         # per chunk: fp32 masters W (3hm), update U (3hm), momentum M (3hm) per (b, head)
         sp = rec_splits(wl)
         mom = 2.0 * 3 * hm * 4 if wl.momentum else 0.0
+        # the step reads the update U after Newton-Schulz, else the split partials (and
+        # updates the momentum) itself; it reads and writes W and writes the bf16 operands
+        upd = 3 * hm * 4.0 if wl.ns_steps else sp * 3 * hm * 4.0 + mom
         table = {
             "gemm_features_k": ("tensor", 4.0 * hm * T),
             "gemm_features_q": ("tensor", 4.0 * hm * T),
@@ -150,11 +153,11 @@ def kernel_work(name: str, wl, form: str):
             "gemm_grad_w1": ("tensor", 2.0 * hm * T),
             "gemm_grad_w0": ("tensor", 2.0 * hm * T),
             "gemm_grad_w2": ("tensor", 2.0 * hm * T),
+            "gemm_grad_w02": ("tensor", 4.0 * hm * T),
             "gemm_output": ("tensor", 2.0 * hm * T),
             # split-K partials in, U out (and M in / out)
             "reduce_momentum": ("hbm", C * BH * (sp * 3 * hm * 4.0 + 3 * hm * 4.0 + mom)),
-            # W and U in, W out, bf16 operands (blocked W0/W2, W1) out
-            "step_renorm": ("hbm", C * BH * (3 * 3 * hm * 4.0 + (2 * mpad * h + hm) * es)),
+            "step_renorm": ("hbm", C * BH * (2 * 3 * hm * 4.0 + upd + (2 * mpad * h + hm) * es)),
             "rec_init": ("hbm", 3 * hm * 4.0 * H + BH * (3 * hm * 4.0 + hm * es)),
             "col_norms": ("hbm", 3 * hm * 4.0 * H),
             "prep_weights": ("hbm", 2 * hm * 4.0 * H + BH * 2 * mpad * h * es),

@@ -685,9 +685,16 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   return TTT_OK;
 }
 
-// B-resident pays when K fits the resident buffer and the B operand is K-major.
+// B-resident pays when K fits the resident buffer, the B operand is K-major, and each
+// resident B tile serves many row tiles: a CTA reloads B (128 KB, after its MMAs on the old
+// one drain) whenever the batch entry changes, so a B per batch entry with few row tiles
+// per entry (the recurrent form's per-(batch, head) weights over one chunk) streams B
+// through the ring with A instead.
 bool use_bres(const GemmProblem& p, int BN) {
-  return BN == 256 && p.K <= 4 * BK && !p.B.mn_major && (p.N + BN - 1) / BN <= sm_count();
+  const long long rows_per_b = (long long)((p.M + BM - 1) / BM) * (p.B.s0 ? 1 : p.Z0) *
+                               (p.B.s1 ? 1 : p.Z1);
+  return BN == 256 && p.K <= 4 * BK && !p.B.mn_major && (p.N + BN - 1) / BN <= sm_count() &&
+         rows_per_b >= 64;
 }
 
 template <int BN, int STAGES, int MODE, typename TC>

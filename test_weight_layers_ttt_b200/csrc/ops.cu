@@ -176,25 +176,76 @@ __global__ void chunk_scan4_kernel(const float4* __restrict__ dS, const float4* 
 }
 
 // ------------------------------------------------------------------ recurrent state
+// Offset, in units of h*m, of part p of a (b, head) block of the split-K gradient partials,
+// stored [W0^T | W2^T | W1^T] so the W0 and W2 gradients are one GEMM's contiguous output.
+__device__ __forceinline__ int partial_part(int p) { return p == 0 ? 0 : p == 1 ? 2 : 1; }
+
 // Part p of a (b, head) state: p = 0 W0 [h, m], p = 1 W1 [m, h], p = 2 W2 [h, m].
 __device__ __forceinline__ void part_dims(int p, int h, int m, int& R, int& Cc) {
   if (p == 1) { R = m; Cc = h; } else { R = h; Cc = m; }
 }
 
+// Part p of a (b, head) state in the original (input-major) layout: W0 [h, m], W1 [m, h],
+// W2 [h, m]; the recurrent state keeps each part output-major, i.e. transposed.
+// grid (tiles of the largest part, 3, BH), block (32, 8): one 32 x 32 tile of part p through
+// shared memory; both the original-layout side and the output-major side are accessed
+// along their rows. dir 0 (set-up): W_all[bh] part p = W_p[head]^T (and W1t = bf16 of the
+// W1 part, M_all = M_in^T or 0); dir 1 (tear-down): out_p[bh] = W_all[bh] part p^T (and
+// M_out = M_all^T).
 template <typename OT>
-__global__ void rec_init_kernel(const float* W0, const float* W2, const float* W1, int BH, int H,
-                                int h, int m, float* W_all, OT* W1o, const float* M_in,
-                                float* M_all, int momentum) {
-  const long long hm = (long long)h * m, per = 3 * hm;
-  TTT_GRID_LOOP(idx, per * BH) {
-    const long long bh = idx / per, e = idx - bh * per;
-    const int p = (int)(e / hm);
-    const long long o = e - p * hm;
-    const long long hd = bh % H;
-    const float v = p == 0 ? W0[hd * hm + o] : p == 1 ? W1[hd * hm + o] : W2[hd * hm + o];
-    W_all[idx] = v;
-    if (p == 1) W1o[bh * hm + o] = from_f32<OT>(v);
-    if (momentum) M_all[idx] = M_in ? M_in[idx] : 0.0f;
+__global__ void rec_transpose_kernel(int dir, const float* W0, const float* W2, const float* W1,
+                                     int H, int h, int m, float* W_all, OT* W1t,
+                                     const float* M_in, float* M_all, int momentum,
+                                     float* W0_out, float* W2_out, float* W1_out, float* M_out) {
+  __shared__ float t[2][32][33];
+  const int p = blockIdx.y, bh = blockIdx.z, head = bh % H;
+  int R, Cc;   // original layout [R, Cc]; output-major [Cc, R]
+  part_dims(p, h, m, R, Cc);
+  const int tiles_c = (Cc + 31) / 32;
+  if ((int)blockIdx.x >= tiles_c * ((R + 31) / 32)) return;
+  const int r0 = (blockIdx.x / tiles_c) * 32, c0 = (blockIdx.x % tiles_c) * 32;
+  const long long hm = (long long)h * m;
+  const long long st = (long long)bh * 3 * hm + p * hm;   // part p of W_all / M_all
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  if (dir == 0) {
+    const float* src = (p == 0 ? W0 : p == 1 ? W1 : W2) + (long long)head * hm;
+    const float* msrc = M_in ? M_in + st : nullptr;
+    for (int k = ty; k < 32; k += 8) {
+      const int r = r0 + k, c = c0 + tx;
+      if (r < R && c < Cc) {
+        t[0][k][tx] = src[(long long)r * Cc + c];
+        if (momentum) t[1][k][tx] = msrc ? msrc[(long long)r * Cc + c] : 0.0f;
+      }
+    }
+    __syncthreads();
+    for (int k = ty; k < 32; k += 8) {
+      const int c = c0 + k, r = r0 + tx;   // output-major [Cc, R]
+      if (r < R && c < Cc) {
+        const long long o = (long long)c * R + r;
+        W_all[st + o] = t[0][tx][k];
+        if (p == 1) W1t[(long long)bh * hm + o] = from_f32<OT>(t[0][tx][k]);
+        if (momentum) M_all[st + o] = t[1][tx][k];
+      }
+    }
+  } else {
+    float* dst = p == 0 ? W0_out : p == 1 ? W1_out : W2_out;
+    for (int k = ty; k < 32; k += 8) {
+      const int c = c0 + k, r = r0 + tx;
+      if (r < R && c < Cc) {
+        const long long o = (long long)c * R + r;
+        t[0][tx][k] = W_all[st + o];
+        if (M_out) t[1][tx][k] = M_all[st + o];
+      }
+    }
+    __syncthreads();
+    for (int k = ty; k < 32; k += 8) {
+      const int r = r0 + k, c = c0 + tx;
+      if (r < R && c < Cc) {
+        const long long o = (long long)r * Cc + c;
+        if (dst) dst[(long long)bh * hm + o] = t[0][k][tx];
+        if (M_out) M_out[st + o] = t[1][k][tx];
+      }
+    }
   }
 }
 
@@ -242,9 +293,10 @@ __global__ void rec_reduce4_kernel(const float4* __restrict__ partials, int spli
     const long long bh = idx / per4;
     const int p = (int)((idx - bh * per4) / hm4);
     if (!(mask & (1 << p))) continue;
-    float4 g = partials[idx];
+    const long long pi = idx + (partial_part(p) - p) * hm4;
+    float4 g = partials[pi];
     for (int s = 1; s < splits; ++s) {
-      const float4 q = partials[(long long)s * total4 + idx];
+      const float4 q = partials[(long long)s * total4 + pi];
       g.x += q.x; g.y += q.y; g.z += q.z; g.w += q.w;
     }
     if (M_all) {
@@ -267,8 +319,9 @@ __global__ void rec_reduce_kernel(const float* partials, int splits, float* U, f
     const long long bh = idx / per;
     const int p = (int)((idx - bh * per) / hm);
     if (!(mask & (1 << p))) continue;
+    const long long pi = idx + (partial_part(p) - p) * hm;
     float g = 0.0f;
-    for (int s = 0; s < splits; ++s) g += partials[(long long)s * total + idx];
+    for (int s = 0; s < splits; ++s) g += partials[(long long)s * total + pi];
     if (M_all) {
       const float mv = alpha[bh * C + c] * M_all[idx] + g;
       M_all[idx] = mv;
@@ -524,90 +577,118 @@ __global__ void momentum_scan_kernel(float* D, const float* alpha, int BH, int C
   }
 }
 
-// grid (ceil(max cols / 32), 3, BH), block (32, 32), dynamic shared memory 32 x (R + 1)
-// floats: one column per threadIdx.x, rows strided by 32 over threadIdx.y. Three phases,
-// each with all threads' loads independent: W - sign U into shared memory and its column
-// sums of squares; the rescaled values written to the fp32 master and W1o (coalesced along
-// columns) and kept in shared memory;
-// for W0 / W2 the shared-memory columns written out as rows of the blocked operand Wk
-// (coalesced along the input dimension).
-template <typename OT>
-__global__ void __launch_bounds__(1024) rec_step_kernel(float* W_all, const float* U,
-                                                        const float* tnorm, int H, int h, int m,
-                                                        int mask, int sign, int renorm, OT* Wk,
-                                                        OT* W1o) {
-  extern __shared__ float colbuf[];  // [32][R + 1]
-  __shared__ float red[32][33];
-  const int p = blockIdx.y, bh = blockIdx.z;
+// One warp per row of the output-major state (one output unit of a fast matrix, over its
+// input dimension): the update u = U (Newton-Schulz path) or the sum of the split-K partial
+// gradients with the momentum M <- alpha M + g folded in (written back); w <- w - sign u;
+// with renormalisation the row's norm is reduced across the warp and the row rescaled to
+// the initial column norm; the fp32 master and the bf16 / fp32 operand copy are written
+// (W1 rows to W1t [h, m], W0 / W2 rows to their rows of the blocked operand Wk, W0 halved).
+// Rows per (b, head): m of W0^T (length h), h of W1^T (length m), m of W2^T (length h).
+// VEC: rows in 16-byte vectors (h, m multiples of 4); NV: the most vectors (elements without
+// VEC) a lane holds, ceil(max(h, m) / 128) (/ 32).
+template <typename OT, bool VEC, int NV>
+__global__ void __launch_bounds__(256) rec_step_rows_kernel(float* W_all, const float* U, const float* partials,
+                                     int splits, float* M_all, const float* alpha, int C, int c,
+                                     const float* tnorm, int BH, int H, int h, int m, int mask,
+                                     int sign, int renorm, OT* Wk, OT* W1t) {
+  const long long rows_bh = 2LL * m + h, rows = rows_bh * BH;
+  const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= rows) return;
+  const int bh = (int)(wid / rows_bh);
+  int r = (int)(wid - (long long)bh * rows_bh), p = 0;
+  if (r >= m + h) { p = 2; r -= m + h; } else if (r >= m) { p = 1; r -= m; }
   if (!(mask & (1 << p))) return;
-  int R, Cc;
-  part_dims(p, h, m, R, Cc);
-  const int c0 = blockIdx.x * 32;
-  if (c0 >= Cc) return;
-  const int tx = threadIdx.x, ty = threadIdx.y;
-  const int c = c0 + tx;
-  const bool live = c < Cc;
+  const int len = p == 1 ? m : h;
   const long long hm = (long long)h * m;
-  float* w = W_all + (long long)bh * 3 * hm + p * hm;
-  const float* u = U + (long long)bh * 3 * hm + p * hm;
+  const long long off = (long long)bh * 3 * hm + p * hm + (long long)r * len;
+  const long long poff = off + (partial_part(p) - p) * hm;   // the row in the partials
+  const long long pstride = (long long)BH * 3 * hm;
   const float sg = (float)sign;
-  float* mycol = colbuf + (long long)tx * (R + 1);
+  const float a = (M_all && !U) ? alpha[(long long)bh * C + c] : 0.0f;
+  constexpr int MAXV = NV;
+  float v[VEC ? MAXV * 4 : MAXV];
   float ss = 0.0f;
-  if (live) {
-#pragma unroll 4
-    for (int r = ty; r < R; r += 32) {
-      const float v = w[(long long)r * Cc + c] - sg * u[(long long)r * Cc + c];
-      mycol[r] = v;
-      ss = fmaf(v, v, ss);
+  const int n = VEC ? len / 4 : len;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int q = lane + 32 * i;
+    if (q >= n) break;
+    if constexpr (VEC) {
+      const float4 w = reinterpret_cast<const float4*>(W_all + off)[q];
+      float4 u;
+      if (U) {
+        u = reinterpret_cast<const float4*>(U + off)[q];
+      } else {
+        u = reinterpret_cast<const float4*>(partials + poff)[q];
+        for (int s2 = 1; s2 < splits; ++s2) {
+          const float4 x = reinterpret_cast<const float4*>(partials + s2 * pstride + poff)[q];
+          u.x += x.x; u.y += x.y; u.z += x.z; u.w += x.w;
+        }
+        if (M_all) {
+          float4 mv = reinterpret_cast<float4*>(M_all + off)[q];
+          mv.x = fmaf(a, mv.x, u.x); mv.y = fmaf(a, mv.y, u.y);
+          mv.z = fmaf(a, mv.z, u.z); mv.w = fmaf(a, mv.w, u.w);
+          reinterpret_cast<float4*>(M_all + off)[q] = mv;
+          u = mv;
+        }
+      }
+      v[4 * i] = w.x - sg * u.x; v[4 * i + 1] = w.y - sg * u.y;
+      v[4 * i + 2] = w.z - sg * u.z; v[4 * i + 3] = w.w - sg * u.w;
+      ss = fmaf(v[4 * i], v[4 * i], ss); ss = fmaf(v[4 * i + 1], v[4 * i + 1], ss);
+      ss = fmaf(v[4 * i + 2], v[4 * i + 2], ss); ss = fmaf(v[4 * i + 3], v[4 * i + 3], ss);
+    } else {
+      float u;
+      if (U) {
+        u = U[off + q];
+      } else {
+        u = partials[poff + q];
+        for (int s2 = 1; s2 < splits; ++s2) u += partials[s2 * pstride + poff + q];
+        if (M_all) {
+          const float mv = fmaf(a, M_all[off + q], u);
+          M_all[off + q] = mv;
+          u = mv;
+        }
+      }
+      v[i] = W_all[off + q] - sg * u;
+      ss = fmaf(v[i], v[i], ss);
     }
   }
-  red[ty][tx] = ss;
-  __syncthreads();
   float scale = 1.0f;
-  if (renorm && live) {
-    float tot = 0.0f;
-#pragma unroll 8
-    for (int y = 0; y < 32; ++y) tot += red[y][tx];
+  if (renorm) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float* tn = tnorm + (long long)(bh % H) * (2 * m + h) + (p == 0 ? 0 : p == 1 ? m : m + h);
-    scale = tn[c] / sqrtf(tot);
+    scale = tn[r] / sqrtf(ss);
   }
-  if (live) {   // each thread rescales the values it computed itself (same rows)
-#pragma unroll 4
-    for (int r = ty; r < R; r += 32) {
-      const long long o = (long long)r * Cc + c;
-      const float v = mycol[r] * scale;
-      w[o] = v;
-      if (p == 1) W1o[(long long)bh * hm + o] = from_f32<OT>(v);
-      else mycol[r] = v;
-    }
-  }
-  if (p == 1) return;
-  __syncthreads();
   const int mpad = (m + 127) / 128 * 128;
-  OT* wk = Wk + (long long)bh * 2 * mpad * h;
-  // warp ty writes column c0 + ty as one Wk row, lanes along the input dimension
-  for (int cc = ty; cc < 32 && c0 + cc < Cc; cc += 32) {
-    const int col = c0 + cc;
-    const long long row = (long long)(col >> 7) * 256 + (p == 2 ? 128 : 0) + (col & 127);
-    const float* src = colbuf + (long long)cc * (R + 1);
-    const float f = p == 0 ? 0.5f : 1.0f;   // the blocked operand holds W0 / 2
-    for (int r = tx; r < R; r += 32) wk[row * h + r] = from_f32<OT>(f * src[r]);
-  }
-}
-
-__global__ void rec_finish_kernel(const float* W_all, int BH, int h, int m, float* W0_out,
-                                  float* W2_out, float* W1_out, const float* M_all,
-                                  float* M_out) {
-  const long long hm = (long long)h * m, per = 3 * hm;
-  TTT_GRID_LOOP(idx, per * BH) {
-    const long long bh = idx / per, e = idx - bh * per;
-    const int p = (int)(e / hm);
-    const long long o = bh * hm + (e - p * hm);
-    const float v = W_all[idx];
-    if (p == 0 && W0_out) W0_out[o] = v;
-    if (p == 1 && W1_out) W1_out[o] = v;
-    if (p == 2 && W2_out) W2_out[o] = v;
-    if (M_out && M_all) M_out[idx] = M_all[idx];
+  OT* orow = p == 1 ? W1t + (long long)bh * hm + (long long)r * len
+                    : Wk + ((long long)bh * 2 * mpad + (r >> 7) * 256 + (p == 2 ? 128 : 0) +
+                            (r & 127)) * h;
+  const float f = p == 0 ? 0.5f : 1.0f;   // the blocked operand holds W0 / 2
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int q = lane + 32 * i;
+    if (q >= n) break;
+    if constexpr (VEC) {
+      const float4 w = make_float4(v[4 * i] * scale, v[4 * i + 1] * scale, v[4 * i + 2] * scale,
+                                   v[4 * i + 3] * scale);
+      reinterpret_cast<float4*>(W_all + off)[q] = w;
+      if constexpr (sizeof(OT) == 2) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(f * w.x, f * w.y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(f * w.z, f * w.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(orow)[q] = pk;
+      } else {
+        reinterpret_cast<float4*>(orow)[q] = make_float4(f * w.x, f * w.y, f * w.z, f * w.w);
+      }
+    } else {
+      const float w = v[i] * scale;
+      W_all[off + q] = w;
+      orow[q] = from_f32<OT>(f * w);
+    }
   }
 }
 
@@ -796,14 +877,14 @@ cudaError_t chunk_scan(int ot, const float* dS, const float* W1, const float* pr
 }
 
 cudaError_t rec_init(int ot, const float* W0, const float* W2, const float* W1, int BH, int H,
-                     int h, int m, float* W_all, void* W1o, const float* M_in, float* M_all,
+                     int h, int m, float* W_all, void* W1t, const float* M_in, float* M_all,
                      int momentum, cudaStream_t s) {
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
-    const long long n = 3LL * h * m * BH;
-    rec_init_kernel<OT><<<grid_for(n, 256), 256, 0, s>>>(W0, W2, W1, BH, H, h, m, W_all,
-                                                         static_cast<OT*>(W1o), M_in, M_all,
-                                                         momentum);
+    const int tiles = ((h + 31) / 32) * ((m + 31) / 32);
+    rec_transpose_kernel<OT><<<dim3(tiles, 3, BH), dim3(32, 8), 0, s>>>(
+        0, W0, W2, W1, H, h, m, W_all, static_cast<OT*>(W1t), M_in, M_all, momentum, nullptr,
+        nullptr, nullptr, nullptr);
     return cudaGetLastError();
   });
 }
@@ -934,31 +1015,37 @@ cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long
   return cudaGetLastError();
 }
 
-cudaError_t rec_step(float* W_all, const float* U, const float* tnorm, int BH, int H, int h,
-                     int m, int mask, int sign, int renorm, void* Wk, void* W1o, int ot,
-                     cudaStream_t s) {
+cudaError_t rec_step(float* W_all, const float* U, const float* partials, int splits,
+                     float* M_all, const float* alpha, int C, int c, const float* tnorm, int BH,
+                     int H, int h, int m, int mask, int sign, int renorm, void* Wk, void* W1t,
+                     int ot, cudaStream_t s) {
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
-    const int maxc = h > m ? h : m;
-    const int maxr = h > m ? h : m;
-    const size_t smem = (size_t)32 * (maxr + 1) * sizeof(float);
-    auto kern = rec_step_kernel<OT>;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-      return cudaErrorInvalidValue;
-    dim3 grid((maxc + 31) / 32, 3, BH);
-    kern<<<grid, dim3(32, 32), smem, s>>>(W_all, U, tnorm, H, h, m, mask, sign, renorm,
-                                          static_cast<OT*>(Wk), static_cast<OT*>(W1o));
+    const long long rows = (2LL * m + h) * BH;
+    const unsigned grid = (unsigned)((rows * 32 + 255) / 256);
+    const bool vec = h % 4 == 0 && m % 4 == 0;
+    const int len = h > m ? h : m;
+    auto go = [&](auto kern) {
+      kern<<<grid, 256, 0, s>>>(W_all, U, partials, splits, M_all, alpha, C, c, tnorm, BH, H, h,
+                                m, mask, sign, renorm, static_cast<OT*>(Wk),
+                                static_cast<OT*>(W1t));
+    };
+    if (vec && len <= 256) go(rec_step_rows_kernel<OT, true, 2>);
+    else if (vec && len <= 512) go(rec_step_rows_kernel<OT, true, 4>);
+    else if (vec) go(rec_step_rows_kernel<OT, true, 12>);
+    else if (len <= 128) go(rec_step_rows_kernel<OT, false, 4>);
+    else go(rec_step_rows_kernel<OT, false, 48>);
     return cudaGetLastError();
   });
 }
 
-cudaError_t rec_finish(const float* W_all, int BH, int h, int m, float* W0_out, float* W2_out,
-                       float* W1_out, const float* M_all, float* M_out, cudaStream_t s) {
-  const long long n = 3LL * h * m * BH;
-  rec_finish_kernel<<<grid_for(n, 256), 256, 0, s>>>(W_all, BH, h, m, W0_out, W2_out, W1_out,
-                                                     M_all, M_out);
+cudaError_t rec_finish(const float* W_all, int BH, int H, int h, int m, float* W0_out,
+                       float* W2_out, float* W1_out, const float* M_all, float* M_out,
+                       cudaStream_t s) {
+  const int tiles = ((h + 31) / 32) * ((m + 31) / 32);
+  rec_transpose_kernel<float><<<dim3(tiles, 3, BH), dim3(32, 8), 0, s>>>(
+      1, nullptr, nullptr, nullptr, H, h, m, const_cast<float*>(W_all), nullptr, nullptr,
+      const_cast<float*>(M_all), 0, W0_out, W2_out, W1_out, M_out);
   return cudaGetLastError();
 }
 

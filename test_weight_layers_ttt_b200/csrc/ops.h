@@ -33,17 +33,23 @@ cudaError_t chunk_scan(int ot, const float* dS, const float* W1, const float* pr
                        void* Sc, float* S_final, int BH, int H, int C, int m, int h, int order,
                        int layout, float* scratch, cudaStream_t s);
 
-// Recurrent-state helpers. Per (b, head) the fp32 state W_all holds [W0 (h*m) | W1 (m*h) |
-// W2 (h*m)]; momentum and the update buffer U use the same part layout.
+// Recurrent-state helpers. Per (b, head) the fp32 state W_all holds the three fast
+// matrices output-major, i.e. transposed: [W0^T (m x h) | W1^T (h x m) | W2^T (m x h)], each
+// row one output unit over the input dimension (so the renormalisation is a row norm);
+// momentum, the update buffer U and the split-K gradient partials use the same layout.
+// rec_init transposes the per-head initial weights (original layouts W0, W2 [h, m], W1
+// [m, h]) into W_all, writes W1t = the OT copy of W1^T [BH, h, m] and, with momentum, M_all
+// = M_in^T (M_in in the original part layouts) or 0.
 cudaError_t rec_init(int ot, const float* W0, const float* W2, const float* W1, int BH, int H,
-                     int h, int m, float* W_all, void* W1o, const float* M_in, float* M_all,
+                     int h, int m, float* W_all, void* W1t, const float* M_in, float* M_all,
                      int momentum, cudaStream_t s);
 // Column norms over the input dimension of the initial weights, per head:
 // tnorm[head] = [W0 columns (m) | W1 columns (h) | W2 columns (m)].
 cudaError_t col_norms(const float* W0, const float* W2, const float* W1, int H, int h, int m,
                       float* tnorm, cudaStream_t s);
-// U = sum over `splits` partial gradients [split][BH][3hm]; with momentum
-// M <- alpha[bh, c] * M + U and U <- M. Only parts in `mask` are touched.
+// U = sum over `splits` partial gradients [split][BH][3hm] (parts ordered [W0^T | W2^T |
+// W1^T] in the partials, [W0^T | W1^T | W2^T] in U); with momentum M <- alpha[bh, c] * M + U
+// and U <- M. Only parts in `mask` are touched.
 cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all,
                        const float* alpha, int C, int c, int BH, int h, int m, int mask,
                        cudaStream_t s);
@@ -55,10 +61,11 @@ struct NsLayout {
   long long zstride, pstride;
   int R[3], C[3];
 };
-// The recurrent state [W0 (h x m) | W1 (m x h) | W2 (h x m)] of each (b, head).
+// The output-major recurrent state [W0^T (m x h) | W1^T (h x m) | W2^T (m x h)] of each
+// (b, head).
 inline NsLayout ns_layout_weights(int h, int m, int mask) {
   const long long hm = (long long)h * m;
-  return NsLayout{3, mask, 3 * hm, hm, {h, m, h}, {m, h, m}};
+  return NsLayout{3, mask, 3 * hm, hm, {m, h, m}, {h, m, h}};
 }
 // One [R, C] matrix per entry, entries R * C apart.
 inline NsLayout ns_layout_single(int R, int C) {
@@ -115,15 +122,21 @@ cudaError_t sum_split_cols(const float* X, int nb, long long rows, int w, float*
 cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long n,
                           cudaStream_t s);
 
-// W <- W - sign * U, optional per-column renormalisation to tnorm, refresh the OT copies:
-// W1o [BH, m, h] and the blocked input-side operand Wk [BH, 2 * mpad, h] (see
-// prep_wk_blocked).
-cudaError_t rec_step(float* W_all, const float* U, const float* tnorm, int BH, int H, int h,
-                     int m, int mask, int sign, int renorm, void* Wk, void* W1o, int ot,
-                     cudaStream_t s);
-// Final weights [B,H,...] (nullable outputs) and momentum copy-out.
-cudaError_t rec_finish(const float* W_all, int BH, int h, int m, float* W0_out, float* W2_out,
-                       float* W1_out, const float* M_all, float* M_out, cudaStream_t s);
+// One step on the output-major state, one warp per row: the update is U when given, else
+// the sum of the `splits` partials (parts ordered as for rec_reduce) with the momentum
+// M <- alpha[bh, c] M + g folded in;
+// W <- W - sign * u; optional renormalisation of each row (output unit) to its initial
+// norm tnorm; refresh of the OT operand copies W1t [BH, h, m] and the blocked input-side
+// operand Wk [BH, 2 * mpad, h] (see prep_wk_blocked). Only parts in `mask`.
+cudaError_t rec_step(float* W_all, const float* U, const float* partials, int splits,
+                     float* M_all, const float* alpha, int C, int c, const float* tnorm, int BH,
+                     int H, int h, int m, int mask, int sign, int renorm, void* Wk, void* W1t,
+                     int ot, cudaStream_t s);
+// Final weights [B,H,...] in the original layouts (nullable outputs) and the momentum
+// copy-out (original part layouts), transposed back from the output-major state.
+cudaError_t rec_finish(const float* W_all, int BH, int H, int h, int m, float* W0_out,
+                       float* W2_out, float* W1_out, const float* M_all, float* M_out,
+                       cudaStream_t s);
 
 // Causal depthwise 4-tap convolution: Xc[t, i] = sum_j conv_w[j, i] * X0[t - j, i] (bf16).
 cudaError_t conv4_causal(const void* X0, const float* conv_w, void* Xc, int N, int d,

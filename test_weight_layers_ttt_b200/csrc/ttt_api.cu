@@ -856,7 +856,7 @@ ttt_status backward_impl(const ttt_desc& d, const void* q, const void* k, const 
 
 // ------------------------------------------------------------------ recurrent form
 struct RecBufs {
-  float* W_all;   // fp32 masters [BH][W0 | W1 | W2]
+  float* W_all;   // fp32 masters [BH][W0^T | W1^T | W2^T], output-major (see ops.h)
   float* M_all;   // momentum, same layout
   float* U;       // update, same layout
   float* tnorm;   // initial column norms per head
@@ -864,12 +864,11 @@ struct RecBufs {
   // are in copy (c + 1) % 2 (the initial weights in copy 0), so the apply of one chunk can
   // read its copy while the next update writes the other.
   void* Wk[2];    // [BH, 2*mpad, h] blocked [W0^T ; W2^T] operand
-  void* W1o[2];   // [BH, m, h] W1 operand
+  void* W1t[2];   // [BH, h, m] W1^T operand
   void* Dv;       // [BH, chunk, m] V W1^T
-  void* P;        // [BH, chunk, m] phi * eta
-  void* E2;       // [BH, chunk, m] d * silu(A)
-  void* E0;       // [BH, chunk, m] d * B * silu'(A)
-  float* partials;
+  void* PE;       // [BH, chunk, 3m]: per token row E0 = d * B * silu'(A) | E2 = d * silu(A) |
+                  // P = phi * eta (E0 and E2 side by side: one GEMM gives both gradients)
+  float* partials;  // [splits][BH][W0^T | W2^T | W1^T] fp32
   void* phiQ;     // [BH, chunk, m]
   NsScratch ns;   // Newton-Schulz scratch for the 3 matrices of every (b, head)
   int splits;
@@ -884,7 +883,9 @@ struct RecBufs {
 // nvs, 2.4 MB per partial, beat 4 by 3 %).
 int choose_splits(const ttt_desc& d, long long L) {
   const long long BH = (long long)d.B * d.H;
-  const long long tiles = BH * ((d.m + 127) / 128) * ((d.h + 255) / 256);
+  // the W0 and W2 gradients are one GEMM of 2m output rows when both are fast
+  const bool both = (d.update_mask & TTT_UPDATE_W0) && (d.update_mask & TTT_UPDATE_W2);
+  const long long tiles = BH * (((both ? 2 : 1) * d.m + 127) / 128) * ((d.h + 255) / 256);
   const long long partial_bytes = BH * 3LL * d.h * d.m * 4;
   long long best = 1;
   for (long long sp = 2; sp <= 64; sp *= 2) {
@@ -936,12 +937,10 @@ size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
   b.tnorm = cv.take_n<float>((long long)d.H * (2 * d.m + d.h));
   for (int i = 0; i < 2; ++i) {
     b.Wk[i] = cv.take(os * BH * 2 * padded_m(d.m) * d.h);
-    b.W1o[i] = cv.take(os * BH * hm);
+    b.W1t[i] = cv.take(os * BH * hm);
   }
   b.Dv = cv.take(os * rows * d.m);
-  b.P = cv.take(os * rows * d.m);
-  b.E2 = cv.take(os * rows * d.m);
-  b.E0 = cv.take(os * rows * d.m);
+  b.PE = cv.take(os * rows * 3 * d.m);
   b.partials = cv.take_n<float>((long long)b.splits * BH * 3 * hm);
   b.phiQ = cv.take(os * rows * d.m);
   b.ns = d.ns_steps > 0 ? plan_ns(cv, d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32, BH * 3,
@@ -977,7 +976,7 @@ ttt_status rec_apply(const ttt_desc& d, const void* q, void* out, long long t0, 
   GemmProblem o;
   o.M = (int)Lc; o.N = d.h; o.K = d.m; o.Z0 = (int)BH; o.Z1 = 1;
   o.A = {b.phiQ, ot, false, m, L * m, 0};
-  o.B = {b.W1o[bi], ot, true, h, m * h, 0};
+  o.B = {b.W1t[bi], ot, false, m, m * h, 0};   // W1^T rows: K-major
   o.C = {static_cast<char*>(out) + t0 * h * es, ot, h, N * h, 0};
   return run_gemm("gemm_output", o, s);
 }
@@ -1006,21 +1005,25 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
     GemmProblem g;
     g.M = (int)Lc; g.N = d.m; g.K = d.h; g.Z0 = (int)BH; g.Z1 = 1;
     g.A = {static_cast<const char*>(v) + t0 * h * es, ot, false, h, N * h, 0};
-    g.B = {b.W1o[bin], ot, false, h, m * h, 0};
+    g.B = {b.W1t[bin], ot, true, m, m * h, 0};   // W1^T rows: MN-major
     g.C = {b.Dv, ot, m, L * m, 0};
     TTT_TRY(run_gemm("gemm_v_w1t", g, s));
   }
-  // [A | B] = K_c [W0 | W2] -> P = phi eta (and E2, E0 for the input-side matrices)
-  SwigluGemm f = rec_features(d, k, b.Wk[bin], t0, Lc, b.P);
+  // [A | B] = K_c [W0 | W2] -> P = phi eta (and E2, E0 for the input-side matrices), all
+  // three in the rows of PE
+  char* PE = static_cast<char*>(b.PE);
+  SwigluGemm f = rec_features(d, k, b.Wk[bin], t0, Lc, PE + 2 * m * es);
+  f.gemm.C.ld = 3 * m;
+  f.gemm.C.s0 = L * 3 * m;
   f.rowscale = eta + t0;
   f.rs0 = N;
   f.rs1 = 0;
   if (need_in) {
     f.grad = 1;
-    f.out2 = (mask & TTT_UPDATE_W2) ? b.E2 : nullptr;
-    f.ld2 = m; f.s20 = L * m; f.s21 = 0;
-    f.out3 = (mask & TTT_UPDATE_W0) ? b.E0 : nullptr;
-    f.ld3 = m; f.s30 = L * m; f.s31 = 0;
+    f.out2 = (mask & TTT_UPDATE_W2) ? PE + m * es : nullptr;
+    f.ld2 = 3 * m; f.s20 = L * 3 * m; f.s21 = 0;
+    f.out3 = (mask & TTT_UPDATE_W0) ? PE : nullptr;
+    f.ld3 = 3 * m; f.s30 = L * 3 * m; f.s31 = 0;
     f.dv = b.Dv;
     f.ldd = m; f.ds0 = L * m; f.ds1 = 0;
   }
@@ -1036,35 +1039,46 @@ ttt_status rec_update(const ttt_desc& d, const void* k, const void* v, const flo
     TTT_CUDA(cudaEventRecord(side->feat, s));
     TTT_CUDA(cudaStreamWaitEvent(s1, side->feat, 0));
   }
-  if (mask & TTT_UPDATE_W1) {  // dW1 = -(phi eta)^T V
+  if (mask & TTT_UPDATE_W1) {  // dW1^T = -V^T (phi eta), output-major [h, m]
     GemmProblem g;
-    g.M = d.m; g.N = d.h; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
-    g.A = {b.P, ot, true, m, L * m, Ks * m};
-    g.B = {static_cast<const char*>(v) + t0 * h * es, ot, true, h, N * h, Ks * h};
-    g.C = {b.partials + hm, DT_F32, h, 3 * hm, tot};
+    g.M = d.h; g.N = d.m; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
+    g.A = {static_cast<const char*>(v) + t0 * h * es, ot, true, h, N * h, Ks * h};
+    g.B = {PE + 2 * m * es, ot, true, 3 * m, L * 3 * m, Ks * 3 * m};
+    g.C = {b.partials + 2 * hm, DT_F32, m, 3 * hm, tot};
     g.alpha = -1.0f;
     TTT_TRY(run_gemm("gemm_grad_w1", g, s1));
   }
   if (g1_side) TTT_CUDA(cudaEventRecord(side->g1, s1));
-  for (int pidx = 0; pidx <= 2; pidx += 2) {  // dW0 = K^T E0, dW2 = K^T E2
-    if (!(mask & (pidx == 0 ? TTT_UPDATE_W0 : TTT_UPDATE_W2))) continue;
-    GemmProblem g;
-    g.M = d.h; g.N = d.m; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
-    g.A = {static_cast<const char*>(k) + t0 * h * es, ot, true, h, N * h, Ks * h};
-    g.B = {pidx == 0 ? b.E0 : b.E2, ot, true, m, L * m, Ks * m};
-    g.C = {b.partials + pidx * hm, DT_F32, m, 3 * hm, tot};
-    TTT_TRY(run_gemm(pidx == 0 ? "gemm_grad_w0" : "gemm_grad_w2", g, s));
+  {  // [dW0^T ; dW2^T] = [E0 | E2]^T K: [2m, h] in one GEMM (or one of them alone)
+    const bool g0 = (mask & TTT_UPDATE_W0) != 0, g2 = (mask & TTT_UPDATE_W2) != 0;
+    if (g0 || g2) {
+      GemmProblem g;
+      g.M = (g0 && g2) ? 2 * d.m : d.m; g.N = d.h; g.K = (int)Ks; g.Z0 = (int)BH; g.Z1 = sp;
+      g.A = {PE + (g0 ? 0 : m * es), ot, true, 3 * m, L * 3 * m, Ks * 3 * m};
+      g.B = {static_cast<const char*>(k) + t0 * h * es, ot, true, h, N * h, Ks * h};
+      g.C = {b.partials + (g0 ? 0 : hm), DT_F32, h, 3 * hm, tot};
+      TTT_TRY(run_gemm((g0 && g2) ? "gemm_grad_w02" : g0 ? "gemm_grad_w0" : "gemm_grad_w2", g,
+                       s));
+    }
   }
   if (g1_side) TTT_CUDA(cudaStreamWaitEvent(s, side->g1, 0));
-  TTT_OP("reduce_momentum", rec_reduce(b.partials, sp, b.U, d.momentum ? b.M_all : nullptr,
-                                      alpha, (int)C, c, (int)BH, d.h, d.m, mask, s));
   if (d.ns_steps > 0) {
+    // the update is orthogonalised: sum the splits (and the momentum) into U first
+    TTT_OP("reduce_momentum", rec_reduce(b.partials, sp, b.U, d.momentum ? b.M_all : nullptr,
+                                        alpha, (int)C, c, (int)BH, d.h, d.m, mask, s));
     if (gate && ns_gate) TTT_CUDA(cudaEventRecord(gate, s));
     TTT_TRY(run_ns(ot, b.U, (int)BH, ns_layout_weights(d.h, d.m, mask), d.ns_steps,
                    b.ns, s));
+    TTT_OP("step_renorm", rec_step(b.W_all, b.U, nullptr, 0, nullptr, nullptr, (int)C, c,
+                                    b.tnorm, (int)BH, d.H, d.h, d.m, mask, d.sign, d.renorm,
+                                    b.Wk[bout], b.W1t[bout], ot, s));
+  } else {
+    // the split sum and the momentum folded into the step
+    TTT_OP("step_renorm", rec_step(b.W_all, nullptr, b.partials, sp,
+                                    d.momentum ? b.M_all : nullptr, alpha, (int)C, c, b.tnorm,
+                                    (int)BH, d.H, d.h, d.m, mask, d.sign, d.renorm, b.Wk[bout],
+                                    b.W1t[bout], ot, s));
   }
-  TTT_OP("step_renorm", rec_step(b.W_all, b.U, b.tnorm, (int)BH, d.H, d.h, d.m, mask, d.sign,
-                                  d.renorm, b.Wk[bout], b.W1o[bout], ot, s));
   return TTT_OK;
 }
 
@@ -1330,7 +1344,7 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   TTT_TRY(checks_begin(s));
-  TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1o[0],
+  TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1t[0],
                               d.momentum ? M_io : nullptr, b.M_all, d.momentum, s));
   TTT_OP("prep_weights", prep_wk_blocked(ot, W0, W2, b.Wk[0], (int)BH, d.H, d.h, d.m, 0, s));
   {  // both operand copies start from the initial weights (a matrix outside the update mask
@@ -1338,7 +1352,7 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
     const size_t os = ot == DT_BF16 ? 2 : 4;
     TTT_CUDA(cudaMemcpyAsync(b.Wk[1], b.Wk[0], os * BH * 2 * padded_m(d.m) * d.h,
                              cudaMemcpyDeviceToDevice, s));
-    TTT_CUDA(cudaMemcpyAsync(b.W1o[1], b.W1o[0], os * BH * d.h * d.m, cudaMemcpyDeviceToDevice,
+    TTT_CUDA(cudaMemcpyAsync(b.W1t[1], b.W1t[0], os * BH * d.h * d.m, cudaMemcpyDeviceToDevice,
                              s));
   }
   if (d.renorm) TTT_OP("col_norms", col_norms(W0, W2, W1, d.H, d.h, d.m, b.tnorm, s));
@@ -1389,8 +1403,8 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   }
   TTT_TRY(st);
   if (W0_out || W2_out || W1_out || (d.momentum && M_io))
-    TTT_OP("rec_finish", rec_finish(b.W_all, (int)BH, d.h, d.m, W0_out, W2_out, W1_out, b.M_all,
-                                    d.momentum ? M_io : nullptr, s));
+    TTT_OP("rec_finish", rec_finish(b.W_all, (int)BH, d.H, d.h, d.m, W0_out, W2_out, W1_out,
+                                    b.M_all, d.momentum ? M_io : nullptr, s));
   const long long hm = (long long)d.h * d.m;
   return checks_end(s, {{out, BH * N * d.h, ot}, {W0_out, BH * hm, DT_F32},
                         {W2_out, BH * hm, DT_F32}, {W1_out, BH * hm, DT_F32},
