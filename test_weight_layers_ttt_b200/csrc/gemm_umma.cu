@@ -68,48 +68,25 @@ struct UArgs {
 // B-resident mode (BRES): the CTA's whole B tile for K <= 256 (up to four 64-wide k-blocks)
 // stays in shared memory and the ring carries only A tiles.
 // SWIGLU mode adds a 32 KB staging tile (128 rows x 128 bf16 phi columns, as two
-// 128-byte-swizzled 64-column boxes) written by the epilogue and stored with TMA.
-template <int BN, int STAGES, bool BRES, int MODE>
+// 128-byte-swizzled 64-column boxes) written by the epilogue and stored with TMA; STORE
+// mode uses the same 32 KB as one 32 x 32 fp32 staging block per epilogue warp, through
+// which each warp turns its row-per-lane values into row-contiguous global stores.
+template <int BN, int STAGES, bool BRES, int MODE, bool STG = true>
 struct Smem {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;             // one k-block of B
   static constexpr int B_RES = BRES ? 4 * B_BYTES : 0;    // resident B, at most 4 k-blocks
   static constexpr int STAGE = BRES ? A_BYTES : A_BYTES + B_BYTES;
-  static constexpr int OUT_BYTES = MODE == 1 ? BM * 128 * 2 : 0;
+  static constexpr int OUT_BYTES = (MODE == 1 || STG) ? BM * 128 * 2 : 0;
   static constexpr int OUT_OFF = B_RES;
   static constexpr int RING_OFF = OUT_OFF + OUT_BYTES;
   static constexpr int BAR_OFF = RING_OFF + STAGES * STAGE;
   static constexpr int TOTAL = BAR_OFF + 256 + 1024;      // + barriers + alignment slack
 };
 
-__device__ __forceinline__ void store_vals(float* dst, const float* v, int n, bool vec) {
-  if (vec && n == 32) {
-#pragma unroll
-    for (int j = 0; j < 32; j += 4)
-      *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < n) dst[j] = v[j];
-  }
-}
-
-__device__ __forceinline__ void store_vals(__nv_bfloat16* dst, const float* v, int n, bool vec) {
-  if (vec && n == 32) {
-#pragma unroll
-    for (int j = 0; j < 32; j += 8) {
-      uint4 pk;
-      pk.x = pack_bf16x2(v[j], v[j + 1]);
-      pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
-      pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
-      pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
-      *reinterpret_cast<uint4*>(dst + j) = pk;
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < n) dst[j] = __float2bfloat16_rn(v[j]);
-  }
+// Four consecutive values to 16-byte-aligned fp32 memory.
+__device__ __forceinline__ void store4(float* dst, const float (&x)[4]) {
+  *reinterpret_cast<float4*>(dst) = make_float4(x[0], x[1], x[2], x[3]);
 }
 
 struct TileCoord {
@@ -191,7 +168,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ OutMaps om, const UArgs args) {
-  using L = Smem<BN, STAGES, BRES, MODE>;
+  using L = Smem<BN, STAGES, BRES, MODE, sizeof(TC) == 4>;
   constexpr uint32_t ACC_COLS = 2 * BN;  // two accumulators
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -375,6 +352,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
       if constexpr (MODE == EPI_STORE) {
+        // alpha * acc (+ beta * Cin): each lane holds one row. fp32 C: per 32-column chunk
+        // the warp stages its 32 x 32 values in shared memory (128-byte rows, 16-byte chunks
+        // XOR-swizzled by row) and writes them back row-contiguous, eight lanes per row, so
+        // the global loads of Cin and the stores of C are coalesced. bf16 C: each lane
+        // stores its row's values directly (half the bytes; fewer instructions win there).
         constexpr int HALF = BN / 2;
         uint32_t r[HALF];
 #pragma unroll
@@ -382,34 +364,106 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0),
                     *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
         tmem_ld_wait();
-        float v[HALF];
 #pragma unroll
-        for (int j = 0; j < HALF; ++j) v[j] = __uint_as_float(r[j]);
+        for (int j = 0; j < HALF; ++j) asm volatile("" : "+r"(r[j]));
         tc_fence_before();
         mbar_arrive(smem_u32(&acc_empty[buf]));
-        if (row < args.M) {
-          TC* crow = static_cast<TC*>(args.C) + tc.z0 * args.cs0 + tc.z1 * args.cs1 +
-                     (long long)row * args.ldc;
-          const float* irow = args.Cin ? args.Cin + tc.z0 * args.is0 + tc.z1 * args.is1 +
-                                             (long long)row * args.ldi
-                                       : nullptr;
-          const bool vec = ((reinterpret_cast<uintptr_t>(crow) & 15) == 0) &&
-                           ((args.ldc * (long long)sizeof(TC)) % 16 == 0);
+        const uint32_t stg = smem_base + L::OUT_OFF + ew * 4096;
+        const int rbase = tc.tm * BM + quarter * 32;
+        TC* cbase = static_cast<TC*>(args.C) + tc.z0 * args.cs0 + tc.z1 * args.cs1;
+        const float* ibase =
+            args.Cin ? args.Cin + tc.z0 * args.is0 + tc.z1 * args.is1 : nullptr;
+        const bool vec =
+            ((reinterpret_cast<uintptr_t>(cbase) | reinterpret_cast<uintptr_t>(ibase)) & 15) ==
+                0 &&
+            (args.ldc * (long long)sizeof(TC)) % 16 == 0 && (!ibase || args.ldi % 4 == 0);
+        const int rr0 = lane >> 3, cq = (lane & 7) * 4;
+        if constexpr (sizeof(TC) == 2) {
+          if (row < args.M) {
+            TC* crow = cbase + (long long)row * args.ldc;
+            const float* irow = ibase ? ibase + (long long)row * args.ldi : nullptr;
+            const bool vrow = ((reinterpret_cast<uintptr_t>(crow) & 15) == 0) &&
+                              ((args.ldc * (long long)sizeof(TC)) % 16 == 0);
 #pragma unroll
-          for (int c0 = 0; c0 < HALF; c0 += 32) {
-            const int col0 = tc.tn * BN + part * HALF + c0;
-            const int nv = min(32, args.N - col0);
-            if (nv <= 0) break;
-            float w[32];
+            for (int c0 = 0; c0 < HALF; c0 += 32) {
+              const int col0 = tc.tn * BN + part * HALF + c0;
+              const int nv = min(32, args.N - col0);
+              if (nv <= 0) break;
+              float w[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) w[j] = args.alpha * v[c0 + j];
-            if (irow) {
+              for (int j = 0; j < 32; ++j) w[j] = args.alpha * __uint_as_float(r[c0 + j]);
+              if (irow) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < nv) w[j] += args.beta * irow[col0 + j];
+                for (int j = 0; j < 32; ++j)
+                  if (j < nv) w[j] += args.beta * irow[col0 + j];
+              }
+              if (vrow && nv == 32) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                  uint4 pk;
+                  pk.x = pack_bf16x2(w[j], w[j + 1]);
+                  pk.y = pack_bf16x2(w[j + 2], w[j + 3]);
+                  pk.z = pack_bf16x2(w[j + 4], w[j + 5]);
+                  pk.w = pack_bf16x2(w[j + 6], w[j + 7]);
+                  *reinterpret_cast<uint4*>(crow + col0 + j) = pk;
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nv) crow[col0 + j] = from_f32<TC>(w[j]);
+              }
             }
-            store_vals(crow + col0, w, nv, vec);
           }
+        } else {
+#pragma unroll
+        for (int c0 = 0; c0 < HALF; c0 += 32) {
+          const int col0 = tc.tn * BN + part * HALF + c0;
+          if (col0 >= args.N) break;
+          __syncwarp();   // the previous chunk's staged values have been read
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float x0 = args.alpha * __uint_as_float(r[c0 + 4 * q]);
+            const float x1 = args.alpha * __uint_as_float(r[c0 + 4 * q + 1]);
+            const float x2 = args.alpha * __uint_as_float(r[c0 + 4 * q + 2]);
+            const float x3 = args.alpha * __uint_as_float(r[c0 + 4 * q + 3]);
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             stg + lane * 128 + ((q ^ (lane & 7)) << 4)),
+                         "f"(x0), "f"(x1), "f"(x2), "f"(x3)
+                         : "memory");
+          }
+          __syncwarp();
+          const int col = col0 + cq;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + rr0, row_o = rbase + rr;
+            float x[4];
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3])
+                         : "r"(stg + rr * 128 + (((cq >> 2) ^ (rr & 7)) << 4))
+                         : "memory");
+            if (row_o >= args.M || col >= args.N) continue;
+            TC* crow = cbase + (long long)row_o * args.ldc;
+            const float* irow = ibase ? ibase + (long long)row_o * args.ldi : nullptr;
+            if (vec && col + 4 <= args.N) {
+              if (irow) {
+                const float4 ci = *reinterpret_cast<const float4*>(irow + col);
+                x[0] = fmaf(args.beta, ci.x, x[0]);
+                x[1] = fmaf(args.beta, ci.y, x[1]);
+                x[2] = fmaf(args.beta, ci.z, x[2]);
+                x[3] = fmaf(args.beta, ci.w, x[3]);
+              }
+              store4(crow + col, x);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                if (col + j >= args.N) break;
+                float y = x[j];
+                if (irow) y = fmaf(args.beta, irow[col + j], y);
+                crow[col + j] = from_f32<TC>(y);
+              }
+            }
+          }
+        }
         }
       } else if (args.grad) {
         // Gradient pieces of the recurrent form. Each output is produced in two 32-column
@@ -662,7 +716,7 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
     }
   }
   auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC, BRES>;
-  constexpr int SMEM = Smem<BN, STAGES, BRES, MODE>::TOTAL;
+  constexpr int SMEM = Smem<BN, STAGES, BRES, MODE, sizeof(TC) == 4>::TOTAL;
   static_assert(SMEM <= 232448, "shared memory budget");
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
       cudaSuccess) {
@@ -699,7 +753,7 @@ bool use_bres(const GemmProblem& p, int BN) {
 
 template <int BN, int STAGES, int MODE, typename TC>
 ttt_status dispatch_major(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  constexpr int RES_STAGES = MODE == EPI_SWIGLU ? 4 : 6;
+  constexpr int RES_STAGES = 4;
   if (BN == 256 && use_bres(p, BN)) {
     if (p.A.mn_major) return launch_umma<BN, true, false, RES_STAGES, MODE, TC, true>(p, a, s);
     return launch_umma<BN, false, false, RES_STAGES, MODE, TC, true>(p, a, s);
