@@ -358,17 +358,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         // the global loads of Cin and the stores of C are coalesced. bf16 C: each lane
         // stores its row's values directly (half the bytes; fewer instructions win there).
         constexpr int HALF = BN / 2;
-        uint32_t r[HALF];
-#pragma unroll
-        for (int c0 = 0; c0 < HALF; c0 += 32)
-          tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0),
-                    *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < HALF; ++j) asm volatile("" : "+r"(r[j]));
-        tc_fence_before();
-        mbar_arrive(smem_u32(&acc_empty[buf]));
-        const uint32_t stg = smem_base + L::OUT_OFF + ew * 4096;
         const int rbase = tc.tm * BM + quarter * 32;
         TC* cbase = static_cast<TC*>(args.C) + tc.z0 * args.cs0 + tc.z1 * args.cs1;
         const float* ibase =
@@ -379,6 +368,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             (args.ldc * (long long)sizeof(TC)) % 16 == 0 && (!ibase || args.ldi % 4 == 0);
         const int rr0 = lane >> 3, cq = (lane & 7) * 4;
         if constexpr (sizeof(TC) == 2) {
+          uint32_t r[HALF];
+#pragma unroll
+          for (int c0 = 0; c0 < HALF; c0 += 32)
+            tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0),
+                      *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < HALF; ++j) asm volatile("" : "+r"(r[j]));
+          tc_fence_before();
+          mbar_arrive(smem_u32(&acc_empty[buf]));
           if (row < args.M) {
             TC* crow = cbase + (long long)row * args.ldc;
             const float* irow = ibase ? ibase + (long long)row * args.ldi : nullptr;
@@ -415,55 +414,72 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         } else {
+          // the accumulator is read 32 columns at a time and released after the last read
+          float4* sbuf = reinterpret_cast<float4*>(smem + L::OUT_OFF + ew * 4096);
 #pragma unroll
-        for (int c0 = 0; c0 < HALF; c0 += 32) {
-          const int col0 = tc.tn * BN + part * HALF + c0;
-          if (col0 >= args.N) break;
-          __syncwarp();   // the previous chunk's staged values have been read
+          for (int c0 = 0; c0 < HALF; c0 += 32) {
+            const int col0 = tc.tn * BN + part * HALF + c0;
+            uint32_t r[32];
+            tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0), r);
+            tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float x0 = args.alpha * __uint_as_float(r[c0 + 4 * q]);
-            const float x1 = args.alpha * __uint_as_float(r[c0 + 4 * q + 1]);
-            const float x2 = args.alpha * __uint_as_float(r[c0 + 4 * q + 2]);
-            const float x3 = args.alpha * __uint_as_float(r[c0 + 4 * q + 3]);
-            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             stg + lane * 128 + ((q ^ (lane & 7)) << 4)),
-                         "f"(x0), "f"(x1), "f"(x2), "f"(x3)
-                         : "memory");
-          }
-          __syncwarp();
-          const int col = col0 + cq;
+            for (int j = 0; j < 32; ++j) asm volatile("" : "+r"(r[j]));
+            // the last chunk with columns inside N releases the accumulator, exactly once
+            const bool last = c0 + 32 >= HALF || col0 + 32 >= args.N;
+            if (last) {
+              tc_fence_before();
+              mbar_arrive(smem_u32(&acc_empty[buf]));
+            }
+            if (col0 >= args.N) break;
+            const int col = col0 + cq;
+            const bool cfull = vec && col + 4 <= args.N;
+            // this chunk's Cin values first, all eight 16-byte loads in flight together
+            float4 cin[8];
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rr = it * 4 + rr0, row_o = rbase + rr;
-            float x[4];
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3])
-                         : "r"(stg + rr * 128 + (((cq >> 2) ^ (rr & 7)) << 4))
-                         : "memory");
-            if (row_o >= args.M || col >= args.N) continue;
-            TC* crow = cbase + (long long)row_o * args.ldc;
-            const float* irow = ibase ? ibase + (long long)row_o * args.ldi : nullptr;
-            if (vec && col + 4 <= args.N) {
-              if (irow) {
-                const float4 ci = *reinterpret_cast<const float4*>(irow + col);
-                x[0] = fmaf(args.beta, ci.x, x[0]);
-                x[1] = fmaf(args.beta, ci.y, x[1]);
-                x[2] = fmaf(args.beta, ci.z, x[2]);
-                x[3] = fmaf(args.beta, ci.w, x[3]);
-              }
-              store4(crow + col, x);
-            } else {
+            for (int it = 0; it < 8; ++it) {
+              const int row_o = rbase + it * 4 + rr0;
+              cin[it] = (ibase && cfull && row_o < args.M)
+                            ? *reinterpret_cast<const float4*>(
+                                  ibase + (long long)row_o * args.ldi + col)
+                            : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+            __syncwarp();   // the previous chunk's staged values have been read
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                if (col + j >= args.N) break;
-                float y = x[j];
-                if (irow) y = fmaf(args.beta, irow[col + j], y);
-                crow[col + j] = from_f32<TC>(y);
+            for (int q = 0; q < 8; ++q)
+              sbuf[lane * 8 + (q ^ (lane & 7))] =
+                  make_float4(args.alpha * __uint_as_float(r[4 * q]),
+                              args.alpha * __uint_as_float(r[4 * q + 1]),
+                              args.alpha * __uint_as_float(r[4 * q + 2]),
+                              args.alpha * __uint_as_float(r[4 * q + 3]));
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int rr = it * 4 + rr0, row_o = rbase + rr;
+              const float4 sv = sbuf[rr * 8 + ((cq >> 2) ^ (rr & 7))];
+              if (row_o >= args.M || col >= args.N) continue;
+              TC* crow = cbase + (long long)row_o * args.ldc;
+              float x[4] = {sv.x, sv.y, sv.z, sv.w};
+              if (cfull) {
+                if (ibase) {
+                  x[0] = fmaf(args.beta, cin[it].x, x[0]);
+                  x[1] = fmaf(args.beta, cin[it].y, x[1]);
+                  x[2] = fmaf(args.beta, cin[it].z, x[2]);
+                  x[3] = fmaf(args.beta, cin[it].w, x[3]);
+                }
+                store4(crow + col, x);
+              } else {
+                const float* irow = ibase ? ibase + (long long)row_o * args.ldi : nullptr;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  if (col + j >= args.N) break;
+                  float y = x[j];
+                  if (irow) y = fmaf(args.beta, irow[col + j], y);
+                  crow[col + j] = from_f32<TC>(y);
+                }
               }
             }
+            if (last) break;
           }
-        }
         }
       } else if (args.grad) {
         // Gradient pieces of the recurrent form. Each output is produced in two 32-column
