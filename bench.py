@@ -180,6 +180,10 @@ def kernel_work(name: str, wl, form: str):
         "gemm_state_delta": ("tensor", unfused_k * 2.0 * hm * T),
         "chunk_scan": ("hbm", fw * scan),
         "fused_apply": ("tensor", 6.0 * hm * T),   # phi(Q) (4hm) and phi(Q) S_c (2hm)
+        # sequential schedule (large states): per chunk the update phi(K)^T eta V into the
+        # fp32 state, and the state's set-up
+        "gemm_state_update": ("tensor", 2.0 * hm * T),
+        "seq_init": ("hbm", BH * hm * (4.0 + 4.0 + es)),
         "gemm_features_q": ("tensor", 4.0 * hm * T),
         "gemm_output": ("tensor", 2.0 * hm * T),
         "momentum_scan": ("hbm", 2 * 4.0 * BH * C * hm + 4.0 * BH * C),

@@ -32,6 +32,9 @@ struct GemmOut {
   void* ptr = nullptr;
   int dtype = DT_F32;
   long long ld = 0, s0 = 0, s1 = 0;
+  // fp32 C on the tensor-core engine only: a bf16 copy of the result with C's element
+  // strides (e.g. the operand copy of a state kept in fp32), or null
+  void* copy16 = nullptr;
 };
 
 struct GemmCin {

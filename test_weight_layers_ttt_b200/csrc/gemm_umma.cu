@@ -49,6 +49,7 @@ struct UArgs {
   int a_b0, a_b1, b_b0, b_b1;  // 1 = operand uses that batch coordinate
   int a_hilo, a_k0, b_hilo, b_k0;  // split-precision operands (GemmOperand::hilo)
   void* C; long long ldc, cs0, cs1;
+  __nv_bfloat16* C16;   // fp32 C: bf16 copy with C's strides, or null
   const float* Cin; long long ldi, is0, is1;
   float alpha, beta;
   // SWIGLU: phi columns < n_valid are written; row factor rs[z0*rs0 + z1*rs1 + row]
@@ -467,6 +468,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                   x[3] = fmaf(args.beta, cin[it].w, x[3]);
                 }
                 store4(crow + col, x);
+                if (args.C16) {
+                  __nv_bfloat16* c16 = args.C16 + tc.z0 * args.cs0 + tc.z1 * args.cs1 +
+                                       (long long)row_o * args.ldc + col;
+                  *reinterpret_cast<uint2*>(c16) =
+                      make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+                }
               } else {
                 const float* irow = ibase ? ibase + (long long)row_o * args.ldi : nullptr;
 #pragma unroll
@@ -475,6 +482,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                   float y = x[j];
                   if (irow) y = fmaf(args.beta, irow[col + j], y);
                   crow[col + j] = from_f32<TC>(y);
+                  if (args.C16)
+                    args.C16[tc.z0 * args.cs0 + tc.z1 * args.cs1 + (long long)row_o * args.ldc +
+                             col + j] = __float2bfloat16_rn(y);
                 }
               }
             }
@@ -798,6 +808,7 @@ UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait
   a.a_b0 = p.A.s0 != 0; a.a_b1 = p.A.s1 != 0; a.b_b0 = p.B.s0 != 0; a.b_b1 = p.B.s1 != 0;
   a.a_hilo = p.A.hilo; a.a_k0 = (int)p.A.k0; a.b_hilo = p.B.hilo; a.b_k0 = (int)p.B.k0;
   a.C = p.C.ptr; a.ldc = p.C.ld; a.cs0 = p.C.s0; a.cs1 = p.C.s1;
+  a.C16 = static_cast<__nv_bfloat16*>(p.C.copy16);
   a.Cin = p.beta != 0.0f ? p.Cin.ptr : nullptr;
   a.ldi = p.Cin.ld; a.is0 = p.Cin.s0; a.is1 = p.Cin.s1;
   a.alpha = p.alpha; a.beta = p.beta;
@@ -823,6 +834,9 @@ const char* umma_unsupported_reason(const GemmProblem& p) {
   if ((long long)p.Z0 * p.Z1 * ((p.M + BM - 1) / BM) * ((p.N + 63) / 64) > (1LL << 31))
     return "too many output tiles";
   if (p.beta != 0.0f && !p.Cin.ptr) return "beta != 0 needs an addend";
+  if (p.C.copy16 && (p.C.dtype != DT_F32 || !aligned16(p.C.copy16) || !aligned16(p.C.ptr) ||
+                     p.C.ld % 4 != 0 || p.C.s0 % 4 != 0 || p.C.s1 % 4 != 0))
+    return "a bf16 copy needs an fp32 result with 16-byte aligned bases, strides multiples of 4";
   if (encode_fn() == nullptr) return "cuTensorMapEncodeTiled is unavailable";
   return nullptr;
 }

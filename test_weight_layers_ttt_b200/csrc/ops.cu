@@ -175,6 +175,20 @@ __global__ void chunk_scan4_kernel(const float4* __restrict__ dS, const float4* 
   }
 }
 
+// ------------------------------------------------------------------ sequential schedule
+// Per (b, head) entry bh: master = W1[bh % H] (zero when W1 is null) + sum of the n_prior
+// states prior[i, bh], and shadow = its bf16 copy; n elements per entry, any layout.
+__global__ void seq_init_kernel(const float* W1, const float* prior, int n_prior, int BH, int H,
+                                long long n, float* master, __nv_bfloat16* shadow) {
+  TTT_GRID_LOOP(idx, (long long)BH * n) {
+    const long long bh = idx / n, e = idx - bh * n;
+    float v = W1 ? W1[(bh % H) * n + e] : 0.0f;
+    for (int i = 0; i < n_prior; ++i) v += prior[((long long)i * BH + bh) * n + e];
+    master[idx] = v;
+    shadow[idx] = __float2bfloat16_rn(v);
+  }
+}
+
 // ------------------------------------------------------------------ recurrent state
 // Offset, in units of h*m, of part p of a (b, head) block of the split-K gradient partials,
 // stored [W0^T | W2^T | W1^T] so the W0 and W2 gradients are one GEMM's contiguous output.
@@ -1072,6 +1086,14 @@ cudaError_t wait_timeout_probe(unsigned* err, unsigned long long limit_ns, cudaS
 
 cudaError_t fill_f32(float* p, long long n, float v, cudaStream_t s) {
   fill_kernel<<<grid_for(n, 256), 256, 0, s>>>(p, n, v);
+  return cudaGetLastError();
+}
+
+cudaError_t seq_init(const float* W1, const float* prior, int n_prior, int BH, int H, long long n,
+                     float* master, void* shadow, cudaStream_t s) {
+  if (BH <= 0 || n <= 0) return cudaSuccess;
+  seq_init_kernel<<<grid_for((long long)BH * n, 256), 256, 0, s>>>(
+      W1, prior, n_prior, BH, H, n, master, static_cast<__nv_bfloat16*>(shadow));
   return cudaGetLastError();
 }
 

@@ -147,6 +147,11 @@ cudaError_t wait_timeout_probe(unsigned* err, unsigned long long limit_ns, cudaS
 
 cudaError_t fill_f32(float* p, long long n, float v, cudaStream_t s);
 
+// Start of the parallel form's sequential schedule: master[bh] = W1[bh % H] (zero when null)
+// + sum_i prior[i, bh] (fp32) and shadow = its bf16 copy; n elements per (b, head) entry.
+cudaError_t seq_init(const float* W1, const float* prior, int n_prior, int BH, int H, long long n,
+                     float* master, void* shadow, cudaStream_t s);
+
 // Debug checks (checks.cu). Guards: kGuardBytes-long words written before a call's first
 // kernel and compared after its last one (a change records DEVERR_BOUNDS); at most
 // kMaxGuards per launch. finite_scan records DEVERR_NONFINITE when any of the n elements

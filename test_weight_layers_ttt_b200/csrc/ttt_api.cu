@@ -308,11 +308,29 @@ struct ParBufs {
   float* dS;   // [BH, C, m, h]
   void* Sc;    // [BH, C, m, h] state read by each chunk
   float* scan_tmp;   // w1_layout 1: transposed W1 and final state ((H + BH) m h), else null
+  float* master;     // sequential schedule: fp32 state per (b, head) (S_final's layout)
+  void* shadow;      // sequential schedule: its bf16 copy, the apply GEMMs' operand
 };
 
 long long padded_m(int m) { return (m + 127LL) / 128 * 128; }
 
-size_t plan_parallel(const ttt_desc& d, void* base, ParBufs& b) {
+// The parallel form has two schedules for the same states. The prefix schedule forms every
+// chunk's delta at once and scans them, materialising an fp32 delta and a bf16 copy of every
+// chunk's state (B H C m h 6 bytes). The sequential schedule keeps one fp32 state per
+// (b, head) and, chunk by chunk, applies its bf16 copy and adds the chunk's delta in place
+// (an update GEMM with the state as its addend, whose epilogue also refreshes the copy).
+// bf16 mode takes the sequential schedule when the materialised states would exceed 2 GiB
+// (the In-Place workload's 32 states of 11008 x 4096), where their HBM round trips cost
+// more than per-chunk GEMM launches. TTT_SEQUENTIAL=1 or 0 overrides the choice (tests).
+bool sequential_schedule(const ttt_desc& d) {
+  if (d.dtype != TTT_DTYPE_BF16 || d.N <= 0) return false;
+  const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
+  const char* e = getenv("TTT_SEQUENTIAL");
+  if (e && *e) return e[0] == '1';
+  return C > 1 && BH * C * (long long)d.h * d.m * 6 > (2LL << 30);
+}
+
+size_t plan_parallel(const ttt_desc& d, void* base, ParBufs& b, bool seq = false) {
   Carve cv(base);
   const size_t os = d.dtype == TTT_DTYPE_BF16 ? 2 : 4;
   const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
@@ -320,6 +338,16 @@ size_t plan_parallel(const ttt_desc& d, void* base, ParBufs& b) {
   b.Wk = cv.take(os * 2 * padded_m(d.m) * d.h * d.H);
   b.phiA = cv.take(os * rows * d.m);
   b.phiB = cv.take(os * rows * d.m);
+  b.master = nullptr;
+  b.shadow = nullptr;
+  if (seq) {   // sequential schedule: one state per (b, head), no per-chunk states
+    b.dS = nullptr;
+    b.Sc = nullptr;
+    b.scan_tmp = nullptr;
+    b.master = cv.take_n<float>(BH * hm);
+    b.shadow = cv.take(2 * BH * hm);
+    return cv.off;
+  }
   b.dS = cv.take_n<float>(BH * C * hm);
   b.Sc = cv.take(os * BH * C * hm);
   b.scan_tmp = d.w1_layout == 1 ? cv.take_n<float>((d.H + BH) * hm) : nullptr;
@@ -443,6 +471,68 @@ ttt_status key_side(const ttt_desc& d, const void* k, const void* v, const float
   return state_deltas(d, b.phiA, v, b.dS, s);
 }
 
+// The sequential schedule of the parallel form (see sequential_schedule): features of the
+// keys (phi eta) and the queries (phi), the state set to W1 (+ priors), then per chunk the
+// apply GEMM O_c = phi(Q_c) S (bf16 copy of S) before or after the update GEMM
+// S <- S + sign phi(K_c)^T diag(eta_c) V_c (fp32 S as addend and output, copy refreshed).
+ttt_status sequential_impl(const ttt_desc& d, const void* q, const void* k, const void* v,
+                           const float* eta, const float* W0, const float* W2, const float* W1,
+                           void* out, float* S_final, const ParBufs& b, cudaStream_t s,
+                           const float* prior, int n_prior) {
+  const int ot = DT_BF16;
+  const size_t es = 2;
+  const bool shared_qk = (q == k) && out != nullptr;
+  const long long BH = (long long)d.B * d.H, N = d.N, h = d.h, m = d.m, L = d.chunk;
+  const long long hm = h * m;
+  TTT_OP("prep_weights",
+         prep_wk_blocked(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
+  TTT_TRY(run_swiglu("gemm_features_k",
+                     features_problem(d, k, b.Wk, b.phiA, shared_qk ? b.phiB : nullptr, eta),
+                     s));
+  if (out && !shared_qk)
+    TTT_TRY(run_swiglu("gemm_features_q",
+                       features_problem(d, q, b.Wk, b.phiB, nullptr, nullptr), s));
+  float* S = S_final ? S_final : b.master;
+  TTT_OP("seq_init", seq_init(W1, prior, n_prior, (int)BH, d.H, hm, S, b.shadow, s));
+  const bool t1 = d.w1_layout == 1;   // the state as [h, m] (else [m, h])
+  auto apply = [&](long long t0, long long Lc) -> ttt_status {
+    GemmProblem p;
+    p.M = (int)Lc; p.N = d.h; p.K = d.m; p.Z0 = (int)BH;
+    p.A = {static_cast<const char*>(b.phiB) + t0 * m * es, ot, false, m, N * m, 0};
+    p.B = t1 ? GemmOperand{b.shadow, ot, false, m, hm, 0}
+             : GemmOperand{b.shadow, ot, true, h, hm, 0};
+    p.C = {static_cast<char*>(out) + t0 * h * es, ot, h, N * h, 0};
+    return run_gemm("gemm_output", p, s);
+  };
+  auto update = [&](long long t0, long long Lc) -> ttt_status {
+    const GemmOperand pe = {static_cast<const char*>(b.phiA) + t0 * m * es, ot, true, m, N * m,
+                            0};
+    const GemmOperand vv = {static_cast<const char*>(v) + t0 * h * es, ot, true, h, N * h, 0};
+    GemmProblem p;
+    p.K = (int)Lc; p.Z0 = (int)BH;
+    if (t1) {   // S [h, m] += sign V^T (phi eta)
+      p.M = d.h; p.N = d.m; p.A = vv; p.B = pe;
+      p.C = {S, DT_F32, m, hm, 0};
+      p.Cin = {S, m, hm, 0};
+    } else {    // S [m, h] += sign (phi eta)^T V
+      p.M = d.m; p.N = d.h; p.A = pe; p.B = vv;
+      p.C = {S, DT_F32, h, hm, 0};
+      p.Cin = {S, h, hm, 0};
+    }
+    p.C.copy16 = b.shadow;
+    p.alpha = (float)d.sign;
+    p.beta = 1.0f;
+    return run_gemm("gemm_state_update", p, s);
+  };
+  for (long long t0 = 0; t0 < N; t0 += L) {
+    const long long Lc = t0 + L <= N ? L : N - t0;
+    if (out && d.order == TTT_ORDER_APPLY_UPDATE) TTT_TRY(apply(t0, Lc));
+    TTT_TRY(update(t0, Lc));
+    if (out && d.order == TTT_ORDER_UPDATE_APPLY) TTT_TRY(apply(t0, Lc));
+  }
+  return TTT_OK;
+}
+
 // The parallel form; the initial state of (b, head) is W1[head] (zero when W1 is null)
 // plus the n_prior states prior[i, b, head]. With out null only the final state is formed
 // (no query side, no per-chunk states).
@@ -450,6 +540,8 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
                          const float* eta, const float* W0, const float* W2, const float* W1,
                          void* out, float* S_final, const ParBufs& b, cudaStream_t s,
                          const float* prior = nullptr, int n_prior = 0) {
+  if (b.master)
+    return sequential_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s, prior, n_prior);
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const bool shared_qk = (q == k) && out != nullptr;
 
@@ -1103,7 +1195,7 @@ size_t ttt_workspace_bytes(const ttt_desc* desc, int32_t path) {
   if (check_desc(desc, path) != TTT_OK) return 0;
   if (path == TTT_PATH_PARALLEL) {
     ParBufs b;
-    return plan_parallel(*desc, nullptr, b);
+    return plan_parallel(*desc, nullptr, b, sequential_schedule(*desc));
   }
   if (path == TTT_PATH_LINEAR) {
     LinBufs b;
@@ -1137,10 +1229,11 @@ ttt_status ttt_la_parallel_fwd(const ttt_desc* desc, const void* q, const void* 
       return fail(TTT_ERR_INVALID_ARG, "q, k, v, out and the weights must be 16-byte aligned");
   }
   ParBufs b;
-  const size_t need = plan_parallel(d, nullptr, b);
+  const bool seq = sequential_schedule(d);
+  const size_t need = plan_parallel(d, nullptr, b, seq);
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
   t_guards.clear();
-  plan_parallel(d, workspace, b);
+  plan_parallel(d, workspace, b, seq);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const long long hm = (long long)d.h * d.m;
@@ -1179,10 +1272,11 @@ ttt_status ttt_la_parallel_fwd_shard(const ttt_desc* desc, const void* q, const 
       return fail(TTT_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
   }
   ParBufs b;
-  const size_t need = plan_parallel(d, nullptr, b);
+  const bool seq = sequential_schedule(d);
+  const size_t need = plan_parallel(d, nullptr, b, seq);
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
   t_guards.clear();
-  plan_parallel(d, workspace, b);
+  plan_parallel(d, workspace, b, seq);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   const long long hm = (long long)d.h * d.m;
@@ -1451,7 +1545,7 @@ ttt_status ttt_la_parallel_fwd_noalloc(const ttt_desc* desc, const void* q, cons
                                        float* S_final, ttt_stream_t stream) {
   TTT_TRY(check_desc(desc, TTT_PATH_PARALLEL));
   ParBufs b;
-  const size_t need = plan_parallel(*desc, nullptr, b);
+  const size_t need = plan_parallel(*desc, nullptr, b, sequential_schedule(*desc));
   if (need > TTT_STATIC_SCRATCH_BYTES)
     return fail(TTT_ERR_WORKSPACE,
                 "problem needs %zu bytes of scratch; the built-in scratch holds %llu bytes "
@@ -1536,7 +1630,11 @@ ttt_status ttt_debug_check_workspace(const ttt_desc* desc, int32_t path, void* w
   TTT_TRY(check_ws(workspace, workspace_bytes, need));
   t_guards.clear();
   switch (path) {
-    case TTT_PATH_PARALLEL: { ParBufs b; plan_parallel(*desc, workspace, b); break; }
+    case TTT_PATH_PARALLEL: {
+      ParBufs b;
+      plan_parallel(*desc, workspace, b, sequential_schedule(*desc));
+      break;
+    }
     case TTT_PATH_LINEAR: { LinBufs b; plan_linear(*desc, workspace, b); break; }
     case TTT_PATH_PARALLEL_MOMENTUM: { MomBufs b; plan_momentum(*desc, workspace, b); break; }
     case TTT_PATH_PARALLEL_BWD: { BwdBufs b; plan_backward(*desc, workspace, b); break; }

@@ -122,6 +122,43 @@ def test_fused_key_side_matches_oracle_and_unfused(case, monkeypatch):
     assert rel(host(fused), host(plain)) <= 1e-2
 
 
+@pytest.mark.parametrize("case", [
+    # B, H, N, h, m, chunk, order, sign, w1_layout: ragged last chunk, both state layouts
+    (2, 2, 1000, 128, 256, 256, "update_apply", 1, 0),
+    (1, 3, 700, 64, 192, 128, "apply_update", -1, 1),
+], ids=lambda c: "-".join(map(str, c)))
+def test_sequential_schedule_matches_oracle_and_prefix(case, monkeypatch):
+    """The parallel form's sequential schedule (one fp32 state per (b, head); per chunk an
+    apply GEMM on its bf16 copy and an update GEMM into it) against the oracle and against
+    the prefix schedule, with a zero initial state too (the state-driven part alone)."""
+    B, H, N, h, m, chunk, order, sign, lay = case
+    wl, inp = layer_inputs("lm", "bf16", B, H, N, h, m, chunk, seed=290 + N)
+    q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
+    W1d = W1.transpose(1, 2).contiguous() if lay else W1
+
+    def run(W):
+        return layer.la_parallel_fwd(q, k, v, eta, W0, W2, W, chunk, order=order, sign=sign,
+                                     w1_layout=lay)
+
+    def st(S):
+        return np.swapaxes(host(S), 2, 3) if lay else host(S)
+
+    monkeypatch.setenv("TTT_SEQUENTIAL", "1")
+    out, S = run(W1d)
+    out0, S0 = run(torch.zeros_like(W1d))
+    monkeypatch.setenv("TTT_SEQUENTIAL", "0")
+    pout, pS = run(W1d)
+    abi.ttt_last_device_status()
+    ref, Sref = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
+                                      inp["W2"], inp["W1"], chunk, order=ORD[order], sign=sign)
+    Z = np.zeros_like(inp["W1"])
+    ref0, Sref0 = O.la_parallel_batched(inp["q"], inp["k"], inp["v"], inp["eta"], inp["W0"],
+                                        inp["W2"], Z, chunk, order=ORD[order], sign=sign)
+    assert rel(host(out), ref) <= TOL["bf16"] and rel(st(S), Sref) <= TOL["bf16"]
+    assert rel(host(out0), ref0) <= TOL["bf16"] and rel(st(S0), Sref0) <= TOL["bf16"]
+    assert rel(host(out), host(pout)) <= 1e-2 and rel(st(S), st(pS)) <= 1e-3
+
+
 def test_parallel_ascent_equals_descent_with_negated_values():
     wl, inp = layer_inputs("lm", "bf16", 1, 2, 512, 64, 128, 128, seed=7)
     q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")

@@ -214,6 +214,23 @@ def test_inplace_reduced_width_all_chunks_match_the_oracle(inplace):
     assert rel(Oh[last], ref[last]) <= TOL["bf16"]
 
 
+def test_inplace_reduced_width_sequential_schedule_matches_the_oracle(inplace, monkeypatch):
+    """The same 32 chunks through the sequential schedule (one fp32 state, per chunk an
+    apply GEMM on its bf16 copy and an update GEMM into it), which the library takes for the
+    full-width In-Place workload, against the oracle's sequential route."""
+    monkeypatch.setenv("TTT_SEQUENTIAL", "1")
+    wl = WORKLOADS["inplace"].scaled(h=512, m=1408)
+    x = make_inplace_inputs(wl, seed=778)
+    vb, out, S = _inplace_gpu(x, wl.N, wl)
+    abi.ttt_last_device_status()
+    Vref = O.lm_target(x["X0"], x["conv_w"], x["W_target"])
+    ref, Wref = O.inplace_sequential(x["Hs"], x["Wg"], x["Wu"], x["W_down"], Vref, wl.chunk,
+                                     1e-3)
+    assert rel(host(out[0, 0]), ref) <= TOL["bf16"]
+    assert rel(host(S[0, 0]), Wref) <= TOL["bf16"]
+    assert rel(host(S[0, 0]) - x["W_down"], Wref - x["W_down"]) <= TOL["bf16"]
+
+
 def test_inplace_full_length_resume_is_bitwise(inplace):
     wl, x = inplace
     vb, out, S = _inplace_gpu(x, wl.N, wl)
