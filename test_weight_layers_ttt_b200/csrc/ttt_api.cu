@@ -319,15 +319,17 @@ long long padded_m(int m) { return (m + 127LL) / 128 * 128; }
 // chunk's state (B H C m h 6 bytes). The sequential schedule keeps one fp32 state per
 // (b, head) and, chunk by chunk, applies its bf16 copy and adds the chunk's delta in place
 // (an update GEMM with the state as its addend, whose epilogue also refreshes the copy).
-// bf16 mode takes the sequential schedule when the materialised states would exceed 2 GiB
-// (the In-Place workload's 32 states of 11008 x 4096), where their HBM round trips cost
-// more than per-chunk GEMM launches. TTT_SEQUENTIAL=1 or 0 overrides the choice (tests).
+// Measured on the In-Place workload (32 states of 11008 x 4096, 8.7 GB materialised): prefix
+// 13.3 ms, sequential 14.0 ms per call; the sequential schedule's per-chunk update GEMM is
+// bound by its fp32 state traffic. So bf16 mode takes the sequential schedule only when the
+// materialised states would exceed 32 GiB, where the prefix schedule's workspace would not
+// fit beside the inputs. TTT_SEQUENTIAL=1 or 0 overrides the choice (tests).
 bool sequential_schedule(const ttt_desc& d) {
   if (d.dtype != TTT_DTYPE_BF16 || d.N <= 0) return false;
   const long long BH = (long long)d.B * d.H, C = (d.N + d.chunk - 1) / d.chunk;
   const char* e = getenv("TTT_SEQUENTIAL");
   if (e && *e) return e[0] == '1';
-  return C > 1 && BH * C * (long long)d.h * d.m * 6 > (2LL << 30);
+  return C > 1 && BH * C * (long long)d.h * d.m * 6 > (32LL << 30);
 }
 
 size_t plan_parallel(const ttt_desc& d, void* base, ParBufs& b, bool seq = false) {

@@ -216,8 +216,8 @@ def test_inplace_reduced_width_all_chunks_match_the_oracle(inplace):
 
 def test_inplace_reduced_width_sequential_schedule_matches_the_oracle(inplace, monkeypatch):
     """The same 32 chunks through the sequential schedule (one fp32 state, per chunk an
-    apply GEMM on its bf16 copy and an update GEMM into it), which the library takes for the
-    full-width In-Place workload, against the oracle's sequential route."""
+    apply GEMM on its bf16 copy and an update GEMM into it), which the library takes for
+    states too large to materialise per chunk, against the oracle's sequential route."""
     monkeypatch.setenv("TTT_SEQUENTIAL", "1")
     wl = WORKLOADS["inplace"].scaled(h=512, m=1408)
     x = make_inplace_inputs(wl, seed=778)
