@@ -42,7 +42,10 @@ constexpr int BK = 64;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 
-enum EpiMode : int { EPI_STORE = 0, EPI_SWIGLU = 1 };
+// STORE: each lane stores its row directly (no addend, or bf16 C). STORE_STG: fp32 C with an
+// addend, staged per warp so Cin loads and C stores are row-contiguous. STORE_COPY: STORE_STG
+// plus a bf16 copy of the result. Separate instantiations, so no mode pays for another's code.
+enum EpiMode : int { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_STORE_STG = 2, EPI_STORE_COPY = 3 };
 
 struct UArgs {
   int M, N, K, Z0, Z1;
@@ -72,18 +75,36 @@ struct UArgs {
 // 128-byte-swizzled 64-column boxes) written by the epilogue and stored with TMA; STORE
 // mode uses the same 32 KB as one 32 x 32 fp32 staging block per epilogue warp, through
 // which each warp turns its row-per-lane values into row-contiguous global stores.
-template <int BN, int STAGES, bool BRES, int MODE, bool STG = true>
+template <int BN, int STAGES, bool BRES, int MODE>
 struct Smem {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;             // one k-block of B
   static constexpr int B_RES = BRES ? 4 * B_BYTES : 0;    // resident B, at most 4 k-blocks
   static constexpr int STAGE = BRES ? A_BYTES : A_BYTES + B_BYTES;
-  static constexpr int OUT_BYTES = (MODE == 1 || STG) ? BM * 128 * 2 : 0;
+  static constexpr int OUT_BYTES = MODE != EPI_STORE ? BM * 128 * 2 : 0;
   static constexpr int OUT_OFF = B_RES;
   static constexpr int RING_OFF = OUT_OFF + OUT_BYTES;
   static constexpr int BAR_OFF = RING_OFF + STAGES * STAGE;
   static constexpr int TOTAL = BAR_OFF + 256 + 1024;      // + barriers + alignment slack
 };
+
+// 32 consecutive values of a row to 16-byte-aligned memory.
+__device__ __forceinline__ void store32(float* dst, const float (&w)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4)
+    *reinterpret_cast<float4*>(dst + j) = make_float4(w[j], w[j + 1], w[j + 2], w[j + 3]);
+}
+__device__ __forceinline__ void store32(__nv_bfloat16* dst, const float (&w)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 8) {
+    uint4 pk;
+    pk.x = pack_bf16x2(w[j], w[j + 1]);
+    pk.y = pack_bf16x2(w[j + 2], w[j + 3]);
+    pk.z = pack_bf16x2(w[j + 4], w[j + 5]);
+    pk.w = pack_bf16x2(w[j + 6], w[j + 7]);
+    *reinterpret_cast<uint4*>(dst + j) = pk;
+  }
+}
 
 // Four consecutive values to 16-byte-aligned fp32 memory.
 __device__ __forceinline__ void store4(float* dst, const float (&x)[4]) {
@@ -169,7 +190,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ OutMaps om, const UArgs args) {
-  using L = Smem<BN, STAGES, BRES, MODE, sizeof(TC) == 4>;
+  using L = Smem<BN, STAGES, BRES, MODE>;
   constexpr uint32_t ACC_COLS = 2 * BN;  // two accumulators
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -352,12 +373,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      if constexpr (MODE == EPI_STORE) {
-        // alpha * acc (+ beta * Cin): each lane holds one row. fp32 C: per 32-column chunk
-        // the warp stages its 32 x 32 values in shared memory (128-byte rows, 16-byte chunks
-        // XOR-swizzled by row) and writes them back row-contiguous, eight lanes per row, so
-        // the global loads of Cin and the stores of C are coalesced. bf16 C: each lane
-        // stores its row's values directly (half the bytes; fewer instructions win there).
+      if constexpr (MODE != EPI_SWIGLU) {
+        // alpha * acc (+ beta * Cin): each lane holds one row. EPI_STORE: each lane stores its
+        // row's values directly (stores do not wait, so their scatter costs little).
+        // EPI_STORE_STG / COPY (fp32 C with an addend): per 32-column chunk the warp stages
+        // its 32 x 32 values in shared memory (128-byte rows, 16-byte chunks XOR-swizzled by
+        // row) and writes them back row-contiguous, eight lanes per row, so the loads of Cin,
+        // which the lanes wait for, are coalesced too.
         constexpr int HALF = BN / 2;
         const int rbase = tc.tm * BM + quarter * 32;
         TC* cbase = static_cast<TC*>(args.C) + tc.z0 * args.cs0 + tc.z1 * args.cs1;
@@ -368,7 +390,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 0 &&
             (args.ldc * (long long)sizeof(TC)) % 16 == 0 && (!ibase || args.ldi % 4 == 0);
         const int rr0 = lane >> 3, cq = (lane & 7) * 4;
-        if constexpr (sizeof(TC) == 2) {
+        if constexpr (MODE == EPI_STORE) {
           uint32_t r[HALF];
 #pragma unroll
           for (int c0 = 0; c0 < HALF; c0 += 32)
@@ -398,15 +420,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                   if (j < nv) w[j] += args.beta * irow[col0 + j];
               }
               if (vrow && nv == 32) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                  uint4 pk;
-                  pk.x = pack_bf16x2(w[j], w[j + 1]);
-                  pk.y = pack_bf16x2(w[j + 2], w[j + 3]);
-                  pk.z = pack_bf16x2(w[j + 4], w[j + 5]);
-                  pk.w = pack_bf16x2(w[j + 6], w[j + 7]);
-                  *reinterpret_cast<uint4*>(crow + col0 + j) = pk;
-                }
+                store32(crow + col0, w);
               } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
@@ -468,7 +482,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                   x[3] = fmaf(args.beta, cin[it].w, x[3]);
                 }
                 store4(crow + col, x);
-                if (args.C16) {
+                if constexpr (MODE == EPI_STORE_COPY) {
                   __nv_bfloat16* c16 = args.C16 + tc.z0 * args.cs0 + tc.z1 * args.cs1 +
                                        (long long)row_o * args.ldc + col;
                   *reinterpret_cast<uint2*>(c16) =
@@ -482,7 +496,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                   float y = x[j];
                   if (irow) y = fmaf(args.beta, irow[col + j], y);
                   crow[col + j] = from_f32<TC>(y);
-                  if (args.C16)
+                  if constexpr (MODE == EPI_STORE_COPY)
                     args.C16[tc.z0 * args.cs0 + tc.z1 * args.cs1 + (long long)row_o * args.ldc +
                              col + j] = __float2bfloat16_rn(y);
                 }
@@ -742,7 +756,7 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
     }
   }
   auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC, BRES>;
-  constexpr int SMEM = Smem<BN, STAGES, BRES, MODE, sizeof(TC) == 4>::TOTAL;
+  constexpr int SMEM = Smem<BN, STAGES, BRES, MODE>::TOTAL;
   static_assert(SMEM <= 232448, "shared memory budget");
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
       cudaSuccess) {
@@ -779,7 +793,7 @@ bool use_bres(const GemmProblem& p, int BN) {
 
 template <int BN, int STAGES, int MODE, typename TC>
 ttt_status dispatch_major(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  constexpr int RES_STAGES = 4;
+  constexpr int RES_STAGES = MODE == EPI_STORE ? 6 : 4;
   if (BN == 256 && use_bres(p, BN)) {
     if (p.A.mn_major) return launch_umma<BN, true, false, RES_STAGES, MODE, TC, true>(p, a, s);
     return launch_umma<BN, false, false, RES_STAGES, MODE, TC, true>(p, a, s);
@@ -793,11 +807,20 @@ ttt_status dispatch_major(const GemmProblem& p, const UArgs& a, cudaStream_t s) 
   }
 }
 
+template <typename TC, int MODE>
+ttt_status dispatch_bn_mode(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
+  if (p.N > 128) return dispatch_major<256, 4, MODE, TC>(p, a, s);
+  if (p.N > 64) return dispatch_major<128, 3, MODE, TC>(p, a, s);
+  return dispatch_major<64, 4, MODE, TC>(p, a, s);
+}
+
 template <typename TC>
 ttt_status dispatch_bn(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  if (p.N > 128) return dispatch_major<256, 4, EPI_STORE, TC>(p, a, s);
-  if (p.N > 64) return dispatch_major<128, 3, EPI_STORE, TC>(p, a, s);
-  return dispatch_major<64, 4, EPI_STORE, TC>(p, a, s);
+  if constexpr (sizeof(TC) == 4) {
+    if (a.C16) return dispatch_bn_mode<TC, EPI_STORE_COPY>(p, a, s);
+    if (a.Cin) return dispatch_bn_mode<TC, EPI_STORE_STG>(p, a, s);
+  }
+  return dispatch_bn_mode<TC, EPI_STORE>(p, a, s);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
