@@ -817,8 +817,11 @@ ttt_status dispatch_bn_mode(const GemmProblem& p, const UArgs& a, cudaStream_t s
 template <typename TC>
 ttt_status dispatch_bn(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   if constexpr (sizeof(TC) == 4) {
+    // staged fp32 stores where the lanes wait for an addend, or where the output leaves L2
+    // and HBM write efficiency decides (more than 64 MB)
     if (a.C16) return dispatch_bn_mode<TC, EPI_STORE_COPY>(p, a, s);
-    if (a.Cin) return dispatch_bn_mode<TC, EPI_STORE_STG>(p, a, s);
+    if (a.Cin || (long long)p.M * p.N * p.Z0 * p.Z1 * 4 > (64LL << 20))
+      return dispatch_bn_mode<TC, EPI_STORE_STG>(p, a, s);
   }
   return dispatch_bn_mode<TC, EPI_STORE>(p, a, s);
 }
