@@ -7,7 +7,9 @@
 // computed into TMEM by one 128 x 256 MMA against the blocked [W0/2 ; W2] operand, turned
 // into bf16 phi by the epilogue warps straight into shared memory, and consumed there by
 // the next MMA as the A operand of phi_j S_c[j]. The output accumulates in TMEM and is
-// written once per tile.
+// written once per tile: each epilogue warp converts its 32 rows to bf16 in its own 4 KB box
+// of the phi tile (free once the tile's last MMA completed) and writes them with TMA tensor
+// stores, 64 columns at a time, so the rows leave as whole lines.
 //
 // Warp roles (320 threads): warp 0 one lane issues TMA loads (Q tile; then, in the order
 // the MMAs consume them, 64-deep k-blocks of the weights and of S_c through a 3-stage ring);
@@ -60,11 +62,27 @@ struct FaArgs {
   unsigned long long wait_ns;
 };
 
+// 64 fp32 values of this lane's row as bf16 into row `lane` of a 128-byte-swizzled
+// 32 x 64 staging box (the layout of a TMA box {64, 32} with 128-byte swizzle).
+__device__ __forceinline__ void stage_row_bf16(const uint32_t* r, uint32_t box, int lane) {
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) {
+    const uint32_t addr = box + lane * 128 + ((cc ^ (lane & 7)) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                 "r"(pack_bf16x2(__uint_as_float(r[8 * cc]), __uint_as_float(r[8 * cc + 1]))),
+                 "r"(pack_bf16x2(__uint_as_float(r[8 * cc + 2]), __uint_as_float(r[8 * cc + 3]))),
+                 "r"(pack_bf16x2(__uint_as_float(r[8 * cc + 4]), __uint_as_float(r[8 * cc + 5]))),
+                 "r"(pack_bf16x2(__uint_as_float(r[8 * cc + 6]), __uint_as_float(r[8 * cc + 7])))
+                 : "memory");
+  }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(FA_THREADS, 1)
     apply_fused_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmW,
-                       const __grid_constant__ CUtensorMap tmS, const FaArgs a) {
+                       const __grid_constant__ CUtensorMap tmS,
+                       const __grid_constant__ CUtensorMap tmO, const FaArgs a) {
   using L = FaSmem<HD>;
   constexpr int QKB = HD / 64;          // k-blocks of the Q tile
   constexpr int S_STAGE = 64 * HD * 2;  // bytes of one S_c k-block (64 state rows x h)
@@ -113,6 +131,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmS);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -301,6 +320,11 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
         ++p_n[b];
         const uint32_t box = sP + b * 2 * FA_PBLK + part * FA_PBLK + quarter * 4096;
+        // the previous tile's output stores from this box have read it
+        if (j == 0) {
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
+        }
         swiglu_piece(ra0, rb0, 1.0f, box, lane, 0);
         swiglu_piece(ra1, rb1, 1.0f, box, lane, 4);
         fence_async_smem();
@@ -320,21 +344,25 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(o_empty));
-      const int row = row0 + quarter * 32 + lane;
-      if (row < a.N) {
-        uint4* dst = reinterpret_cast<uint4*>(a.out + ((long long)bh * a.N + row) * HD +
-                                              part * HALF);
+      // rows quarter*32 .. +31 through this warp's phi box (the tile's MMAs have all
+      // completed): 64 columns per TMA store; rows past N are clipped by the store
+      const uint32_t box = sP + part * FA_PBLK + quarter * 4096;
 #pragma unroll
-        for (int c = 0; c < HALF; c += 8) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1]));
-          v.y = pack_bf16x2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
-          v.z = pack_bf16x2(__uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
-          v.w = pack_bf16x2(__uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
-          dst[c / 8] = v;
+      for (int c0 = 0; c0 < HALF; c0 += 64) {
+        if (c0 > 0) {
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
+        }
+        stage_row_bf16(&r[c0], box, lane);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_4d(&tmO, box, part * HALF + c0, row0 + quarter * 32, bh, 0);
+          tma_store_commit();
         }
       }
     }
+    if (lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -399,9 +427,9 @@ ttt_status launch_fa(const void* q, const void* Wk, const void* Sc, void* out, i
                      cudaStream_t s) {
   const long long BH = (long long)B * H, C = (N + chunk - 1) / chunk;
   const long long mpad = (m + 127LL) / 128 * 128;
-  CUtensorMap mq, mw, ms;
+  CUtensorMap mq, mw, ms, mo;
   if (!fa_map(&mq, q, HD, N, BH, 128) || !fa_map(&mw, Wk, HD, 2 * mpad, H, 256) ||
-      !fa_map(&ms, Sc, HD, m, BH * C, 64)) {
+      !fa_map(&ms, Sc, HD, m, BH * C, 64) || !fa_map(&mo, out, HD, N, BH, 32)) {
     set_error_message("fused apply: cuTensorMapEncodeTiled failed");
     return TTT_ERR_CUDA;
   }
@@ -424,7 +452,7 @@ ttt_status launch_fa(const void* q, const void* Wk, const void* Sc, void* out, i
   int grid = fa_sm_count();
   if (a.tiles < grid) grid = a.tiles;
   if (grid < 1) return TTT_OK;
-  kern<<<grid, FA_THREADS, SMEM, s>>>(mq, mw, ms, a);
+  kern<<<grid, FA_THREADS, SMEM, s>>>(mq, mw, ms, mo, a);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error_message("fused apply launch: %s", cudaGetErrorString(e));

@@ -473,6 +473,25 @@ ttt_status key_side(const ttt_desc& d, const void* k, const void* v, const float
   return state_deltas(d, b.phiA, v, b.dS, s);
 }
 
+// The chunks' outputs phi(Q_c) S_c: fused (phi kept on chip) when the problem allows it,
+// else (fp32, q == k, other widths, TTT_NO_FUSED_APPLY) the feature GEMM followed by the
+// output GEMM.
+ttt_status query_side(const ttt_desc& d, const void* q, const ParBufs& b, bool shared_qk,
+                      void* out, cudaStream_t s) {
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  if (!shared_qk && !getenv("TTT_NO_FUSED_APPLY") &&
+      fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
+    // phi(Q) S_c with phi kept on chip
+    TraceScope ts("fused_apply@tcgen05", s);
+    return fused_apply(q, b.Wk, b.Sc, out, d.B, d.H, d.N, d.h, d.m, d.chunk,
+                       device_error_word(), wait_limit_ns(), s);
+  }
+  if (!shared_qk)
+    TTT_TRY(run_swiglu("gemm_features_q",
+                       features_problem(d, q, b.Wk, b.phiB, nullptr, nullptr), s));
+  return chunk_outputs(d, b.phiB, b.Sc, out, s);
+}
+
 // The sequential schedule of the parallel form (see sequential_schedule): features of the
 // keys (phi eta) and the queries (phi), the state set to W1 (+ priors), then per chunk the
 // apply GEMM O_c = phi(Q_c) S (bf16 copy of S) before or after the update GEMM
@@ -553,17 +572,7 @@ ttt_status parallel_impl(const ttt_desc& d, const void* q, const void* k, const 
   TTT_TRY(chunk_states(d, b.dS, W1, S_final, out ? b.Sc : nullptr, b.scan_tmp, s, prior,
                        n_prior));
   if (!out) return TTT_OK;
-  if (!shared_qk && !getenv("TTT_NO_FUSED_APPLY") &&
-      fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
-    // phi(Q) S_c with phi kept on chip
-    TraceScope ts("fused_apply@tcgen05", s);
-    return fused_apply(q, b.Wk, b.Sc, out, d.B, d.H, d.N, d.h, d.m, d.chunk,
-                       device_error_word(), wait_limit_ns(), s);
-  }
-  if (!shared_qk)
-    TTT_TRY(run_swiglu("gemm_features_q",
-                       features_problem(d, q, b.Wk, b.phiB, nullptr, nullptr), s));
-  return chunk_outputs(d, b.phiB, b.Sc, out, s);
+  return query_side(d, q, b, shared_qk, out, s);
 }
 
 // ------------------------------------------------------------------ identity features
@@ -766,16 +775,7 @@ ttt_status momentum_impl(const ttt_desc& d, const void* q, const void* k, const 
   if (d.ns_steps > 0)
     TTT_TRY(run_ns(ot, b.dS, (int)(BH * C), ns_layout_single(d.m, d.h), d.ns_steps, mb.ns, s));
   TTT_TRY(chunk_states(d, b.dS, W1, S_final, b.Sc, nullptr, s));
-  if (!shared_qk && !getenv("TTT_NO_FUSED_APPLY") &&
-      fused_apply_supported(ot, d.h, d.m, d.chunk, q, b.Wk, b.Sc, out)) {
-    TraceScope ts("fused_apply@tcgen05", s);
-    return fused_apply(q, b.Wk, b.Sc, out, d.B, d.H, d.N, d.h, d.m, d.chunk,
-                       device_error_word(), wait_limit_ns(), s);
-  }
-  if (!shared_qk)
-    TTT_TRY(run_swiglu("gemm_features_q",
-                       features_problem(d, q, b.Wk, b.phiB, nullptr, nullptr), s));
-  return chunk_outputs(d, b.phiB, b.Sc, out, s);
+  return query_side(d, q, b, shared_qk, out, s);
 }
 
 // ------------------------------------------------------------------ backward

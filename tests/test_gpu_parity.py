@@ -66,9 +66,12 @@ def test_parallel_matches_oracle(case, order):
 
 @pytest.mark.parametrize("case", [
     # B, H, N, h, m, chunk: odd number of 128-column phi blocks and more tiles than SMs;
-    # ragged m (zero-padded phi block, state rows past m) and ragged N
+    # ragged m (zero-padded phi block, state rows past m) and ragged N (the last tile's
+    # rows partly, or a 32-row store box wholly, past N)
     (2, 4, 4096, 128, 384, 512),
     (1, 2, 1000, 256, 200, 256),
+    (1, 3, 1100, 256, 512, 512),
+    (2, 1, 700, 128, 256, 384),
 ], ids=lambda c: "-".join(map(str, c)))
 def test_fused_query_side_matches_oracle_and_unfused(case, monkeypatch):
     """phi(Q_c) S_c computed with phi kept in shared memory (h = 128 or 256, chunk a
@@ -79,7 +82,14 @@ def test_fused_query_side_matches_oracle_and_unfused(case, monkeypatch):
                                       inp["W2"], inp["W1"], chunk)
     q, k, v, eta, W0, W2, W1 = gpu_args(inp, "bf16")
     monkeypatch.delenv("TTT_NO_FUSED_APPLY", raising=False)
-    fused, Sf = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk)
+    abi.ttt_trace_enable(256)
+    try:
+        fused, Sf = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk)
+        torch.cuda.synchronize()
+        names = [abi.ttt_trace_get(i)[0] for i in range(abi.ttt_trace_count())]
+    finally:
+        abi.ttt_trace_disable()
+    assert "fused_apply@tcgen05" in names
     monkeypatch.setenv("TTT_NO_FUSED_APPLY", "1")
     plain, Sp = layer.la_parallel_fwd(q, k, v, eta, W0, W2, W1, chunk)
     abi.ttt_last_device_status()
