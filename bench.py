@@ -30,6 +30,9 @@ if ROOT not in sys.path:
 
 METRIC = "TTT-layer tokens/sec at 1 B200 (parallel vs recurrent) and % of roofline"
 L2_BYTES = 126 * 2 ** 20
+# dense tf32 over dense bf16 tensor throughput (nominal 1.1 against 2.25 PFLOP/s): the peak
+# of a tf32 product is the measured bf16 peak times this ratio
+TF32_RATIO = 1.1 / 2.25
 
 
 # ----------------------------------------------------------------------------- cost model
@@ -58,8 +61,34 @@ def layer_flops(wl, form: str) -> float:
     if wl.ns_steps:
         r, c = min(wl.h, wl.m), max(wl.h, wl.m)
         per = wl.ns_steps * (2 * r * r * c + 2 * r ** 3 + 2 * r * r * c)
-        flops += 3.0 * per * wl.B * wl.H * wl.C
+        # one CTA per matrix: three bf16 terms per product; larger matrices: tf32 products
+        flops += (3.0 if ns_one_cta(r, c) else 1.0) * per * wl.B * wl.H * wl.C
     return flops
+
+
+def ns_one_cta(r: int, c: int) -> bool:
+    """The library's Newton-Schulz on one CTA per matrix (split bf16 operands) fits."""
+    return r <= 128 and c <= 256
+
+
+def tf32_flops(wl, form: str) -> float:
+    """The part of layer_flops that runs as tf32 products: Newton-Schulz on matrices too
+    large for one CTA (bf16 mode)."""
+    r, c = min(wl.h, wl.m), max(wl.h, wl.m)
+    if wl.dtype != "bf16" or ns_one_cta(r, c):
+        return 0.0
+    if form == "parallel_momentum":
+        return 5 * (4.0 * r * r * c + 2.0 * r ** 3) * wl.B * wl.H * wl.C
+    if form == "recurrent" and wl.ns_steps:
+        return wl.ns_steps * (4.0 * r * r * c + 2.0 * r ** 3) * wl.B * wl.H * wl.C
+    return 0.0
+
+
+def tensor_seconds(wl, form: str, flops: float, peak_tflops: float) -> float:
+    """Tensor-core time bound of `flops` algorithmic FLOPs of which tf32_flops run at the
+    tf32 rate."""
+    f32 = tf32_flops(wl, form)
+    return (flops - f32) / (peak_tflops * 1e12) + f32 / (peak_tflops * TF32_RATIO * 1e12)
 
 
 def layer_bytes(wl, form: str) -> float:
@@ -79,19 +108,17 @@ def layer_bytes(wl, form: str) -> float:
 
 def _ns_work(wl, r, c, matrices):
     """Step-level work of the Newton-Schulz kernels on `matrices` [r, c] matrices (r <= c):
-    tensor FLOPs of the split-precision products (three bf16 terms hi*hi + hi*lo + lo*hi per
-    fp32 product) and the HBM bytes of the fp32 set-up, splits and write-back."""
+    tensor FLOPs of the one-CTA kernel (three bf16 terms hi*hi + hi*lo + lo*hi per fp32
+    product), of the tf32 GEMMs (one term, at the tf32 rate), and the HBM bytes of the fp32
+    set-up (read U, write X and its transpose) and write-back."""
     steps = wl.ns_steps if wl.ns_steps else 5
     Z = float(matrices)
     return {
         "ns_mma": ("tensor", 3.0 * steps * (4.0 * r * r * c + 2.0 * r ** 3) * Z),
-        "ns_gram": ("tensor", 3.0 * steps * 2.0 * r * r * c * Z),
-        "ns_poly": ("tensor", 3.0 * steps * 2.0 * r ** 3 * Z),
-        "ns_apply": ("tensor", 3.0 * steps * 2.0 * r * r * c * Z),
-        # per step: X read (4rc) -> [hi|lo] along rows and down rows (8rc); A and P read
-        # (4r^2 each) -> [hi|lo] (4r^2 each)
-        "ns_split": ("hbm", steps * (12.0 * r * c + 16.0 * r * r) * Z),
-        "ns_normalize": ("hbm", 8.0 * r * c * Z),
+        "ns_gram": ("tensor_tf32", steps * 2.0 * r * r * c * Z),
+        "ns_poly": ("tensor_tf32", steps * 2.0 * r ** 3 * Z),
+        "ns_apply": ("tensor_tf32", steps * 2.0 * r * r * c * Z),
+        "ns_normalize": ("hbm", 12.0 * r * c * Z),
         "ns_writeback": ("hbm", 8.0 * r * c * Z),
     }
 
@@ -483,16 +510,17 @@ def _roofline(table, wl, peaks, form, steps):
                 "share": round(e["share"], 4), "peak_source": peaks["source"]}
     work = step_work / (e["launches"] / steps)
     secs = e["ms_avg"] / 1e3
-    if bound == "tensor":
+    if bound in ("tensor", "tensor_tf32"):
         achieved = work / secs / 1e12
-        peak = peaks["bf16_tflops"]
+        peak = peaks["bf16_tflops"] * (TF32_RATIO if bound == "tensor_tf32" else 1.0)
         unit = "TFLOP/s"
     else:
         achieved = work / secs / 1e9
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
     return {"kernel": name, "bound": "hbm" if bound == "hbm" else "tensor",
-            "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "dtype": "tf32" if bound == "tensor_tf32" else ("bf16" if bound == "tensor" else None),
+            "achieved": round(achieved, 2), "peak": round(peak, 2), "unit": unit,
             "frac": round(achieved / peak, 4),
             "traffic": (_traffic(wl.name, name)
                         if form == "parallel" and wl == WORKLOADS_REF().get(wl.name) else None),
@@ -613,14 +641,15 @@ def run_gpu(args, rank, local, world):
             nbytes = 2.0 * (2 * wl.N * wl.h + wl.h * wl.h) + 16.0 * wl.h
         else:
             flops, nbytes = layer_flops(wl, form), layer_bytes(wl, form)
-        t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+        t_roof = max(tensor_seconds(wl, form, flops, peaks["bf16_tflops"]),
+                     nbytes / (peaks["hbm_gbs"] * 1e9))
         result["forms"][form] = {
             "tokens_per_s": job_throughput(tokens, world, per_step / 1e3),
             "ms_per_step": per_step, "steps": steps,
             "flop_per_step": flops, "bytes_per_step": nbytes,
             "roofline_frac": t_roof / (per_step / 1e3),
             "roofline_frac_sustained": max(
-                flops / (peaks["bf16_tflops_sustained"] * 1e12),
+                tensor_seconds(wl, form, flops, peaks["bf16_tflops_sustained"]),
                 nbytes / (peaks["hbm_gbs"] * 1e9)) / (per_step / 1e3),
             "gpu_launches": len(trace) * steps // tsteps,
             "launch_mode": mode,

@@ -20,12 +20,6 @@ struct GemmOperand {
   int dtype = DT_F32;
   bool mn_major = false;  // false: k contiguous ("K-major"); true: the row index contiguous
   long long ld = 0, s0 = 0, s1 = 0;
-  // Split-precision operand (tensor-core engine only): the logical K = 3 * k0 is three
-  // k0-wide thirds, [hi hi lo] (hilo 1) or [hi lo hi] (hilo 2), of a matrix stored once as
-  // [hi | lo] along K (2 * k0 wide); k0 a multiple of 64. The engine reads each k-block
-  // from its third's copy, so hi*hi + hi*lo + lo*hi needs no duplicated copies.
-  int hilo = 0;
-  long long k0 = 0;
 };
 
 struct GemmOut {
@@ -35,6 +29,11 @@ struct GemmOut {
   // fp32 C on the tensor-core engine only: a bf16 copy of the result with C's element
   // strides (e.g. the operand copy of a state kept in fp32), or null
   void* copy16 = nullptr;
+  // fp32 C on the tensor-core engine only: the result also written transposed,
+  // t32[z0 * ts0 + z1 * ts1 + j * ldt + i] = C[z](i, j) (the K-major copy of an operand
+  // that the next product reads the other way round), or null
+  float* t32 = nullptr;
+  long long ldt = 0, ts0 = 0, ts1 = 0;
 };
 
 struct GemmCin {
@@ -61,6 +60,12 @@ bool umma_supported(const GemmProblem& p);
 const char* umma_unsupported_reason(const GemmProblem& p);
 ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,
                      unsigned long long wait_ns);
+// The same engine with fp32 A and B consumed as tf32 (tcgen05.mma kind::tf32: operands
+// rounded toward zero to a 10-bit mantissa, fp32 accumulation); both operands K-major, fp32
+// C. For bf16-mode products that need more than bf16 operand precision.
+const char* umma_tf32_unsupported_reason(const GemmProblem& p);
+ttt_status gemm_umma_tf32(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,
+                          unsigned long long wait_ns);
 
 // Feature GEMM with the SwiGLU applied in the epilogue. gemm.B holds the input-side
 // weights as 128-row blocks [W0^T rows j..j+127 / 2 ; W2^T rows j..j+127] (256 rows per

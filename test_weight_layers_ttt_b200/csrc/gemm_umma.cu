@@ -15,9 +15,9 @@
 //           writes phi = silu(a) * b times a per-row factor (bf16), and optionally the
 //           unscaled phi to a second output; the gradient variant writes the recurrent
 //           form's pieces (phi * eta, D * silu(a), D * b * silu'(a)) instead.
-// Split-precision operands (GemmOperand::hilo): the producer reads the k-blocks of a
-// K-tripled operand [hi hi lo] / [hi lo hi] from one [hi | lo] copy by remapping the K
-// coordinate; nothing else changes.
+// tf32 operands (TF): fp32 A and B, K-major, through the same 128-byte-swizzled k-blocks
+// (32 fp32 per 128-byte row instead of 64 bf16) and tcgen05.mma kind::tf32; the shared-memory
+// layout, descriptors and byte offsets are those of the bf16 path.
 // Every mbarrier wait is bounded; a timeout records DEVERR_TIMEOUT in the device error
 // word, raises a CTA-wide abort flag, and the CTA drains its in-flight copies and MMAs
 // (again with bounded waits) and frees its TMEM before returning.
@@ -44,15 +44,19 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 
 // STORE: each lane stores its row directly (no addend, or bf16 C). STORE_STG: fp32 C with an
 // addend, staged per warp so Cin loads and C stores are row-contiguous. STORE_COPY: STORE_STG
-// plus a bf16 copy of the result. Separate instantiations, so no mode pays for another's code.
-enum EpiMode : int { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_STORE_STG = 2, EPI_STORE_COPY = 3 };
+// plus a bf16 copy of the result. STORE_T: STORE_STG plus the result written transposed
+// (fp32), 128 contiguous bytes per store. Separate instantiations, so no mode pays for
+// another's code.
+enum EpiMode : int {
+  EPI_STORE = 0, EPI_SWIGLU = 1, EPI_STORE_STG = 2, EPI_STORE_COPY = 3, EPI_STORE_T = 4
+};
 
 struct UArgs {
   int M, N, K, Z0, Z1;
   int a_b0, a_b1, b_b0, b_b1;  // 1 = operand uses that batch coordinate
-  int a_hilo, a_k0, b_hilo, b_k0;  // split-precision operands (GemmOperand::hilo)
   void* C; long long ldc, cs0, cs1;
   __nv_bfloat16* C16;   // fp32 C: bf16 copy with C's strides, or null
+  float* Ct; long long ldt, ts0, ts1;   // fp32 C: transposed copy (EPI_STORE_T)
   const float* Cin; long long ldi, is0, is1;
   float alpha, beta;
   // SWIGLU: phi columns < n_valid are written; row factor rs[z0*rs0 + z1*rs1 + row]
@@ -115,17 +119,6 @@ struct TileCoord {
   int tm, tn, z0, z1;
 };
 
-// K coordinate, in the operand's buffer, of k-block kb: kb * BK, or for a split-precision
-// operand (logical K = three k0-wide thirds, stored once as [hi | lo]) the block's offset
-// inside its third plus k0 when that third is the lo copy.
-__device__ __forceinline__ int kcoord(int kb, int hilo, int k0) {
-  const int k = kb * BK;
-  if (!hilo) return k;
-  const int third = k / k0, kk = k - third * k0;
-  const bool lo = hilo == 1 ? third == 2 : third == 1;
-  return kk + (lo ? k0 : 0);
-}
-
 __device__ __forceinline__ TileCoord decode_tile(int t, int tiles_n, int tiles_mn, int Z0) {
   TileCoord c;
   const int z = t / tiles_mn, rem = t - z * tiles_mn;
@@ -185,11 +178,14 @@ struct OutMaps {
   CUtensorMap m[3];
 };
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES>
+template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES, bool TF>
 __global__ void __launch_bounds__(THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ OutMaps om, const UArgs args) {
+  static_assert(!TF || (!A_MN && !B_MN && !BRES && MODE != EPI_SWIGLU),
+                "tf32 operands: K-major, streamed, plain epilogues");
+  constexpr int BKE = TF ? 32 : BK;      // K elements per 128-byte k-block row
   using L = Smem<BN, STAGES, BRES, MODE>;
   constexpr uint32_t ACC_COLS = 2 * BN;  // two accumulators
   extern __shared__ uint8_t smem_raw[];
@@ -205,7 +201,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KB = (args.K + BK - 1) / BK;
+  const int KB = (args.K + BKE - 1) / BKE;
   const TileWalker walk(args.M, args.N, args.Z0, args.Z1, BN, BRES);
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t ring_base = smem_base + L::RING_OFF;
@@ -255,7 +251,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_arrive_expect_tx(bb, KB * L::B_BYTES);
           for (int kb = 0; kb < KB; ++kb) {
             const uint32_t sB = smem_base + kb * L::B_BYTES;
-            const int kB = kcoord(kb, args.b_hilo, args.b_k0);
+            const int kB = kb * BKE;
             if (B_MN) {
 #pragma unroll
               for (int q = 0; q < BN / 64; ++q)
@@ -279,7 +275,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t fb = smem_u32(&full[s]);
           mbar_arrive_expect_tx(fb, L::STAGE);
           const uint32_t sA = ring_base + s * L::STAGE;
-          const int kA = kcoord(kb, args.a_hilo, args.a_k0);
+          const int kA = kb * BKE;
           if (A_MN) {
             tma_load_4d(sA, &tmA, fb, tc.tm * BM, kA, ac2, ac3);
             tma_load_4d(sA + 8192, &tmA, fb, tc.tm * BM + 64, kA, ac2, ac3);
@@ -288,7 +284,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           if (!BRES) {
             const uint32_t sB = sA + L::A_BYTES;
-            const int kB = kcoord(kb, args.b_hilo, args.b_k0);
+            const int kB = kb * BKE;
             if (B_MN) {
 #pragma unroll
               for (int q = 0; q < BN / 64; ++q)
@@ -304,7 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t IDESC = make_idesc_bf16(BM, BN, A_MN, B_MN);
+      constexpr uint32_t IDESC = TF ? make_idesc_tf32(BM, BN) : make_idesc_bf16(BM, BN, A_MN, B_MN);
       uint32_t it = 0;
       int bkey = -1, b_uses = 0;
       bool ok = true;
@@ -346,7 +342,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                                      : make_sw128_desc(sA + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? make_sw128_desc(sB + kk * 2048, 8192, 1024)
                                      : make_sw128_desc(sB + kk * 32, 16, 1024);
-            mma_f16(dt, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+            if constexpr (TF)
+              mma_tf32(dt, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+            else
+              mma_f16(dt, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(smem_u32(&empty[s]));
         }
@@ -482,6 +481,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                   x[3] = fmaf(args.beta, cin[it].w, x[3]);
                 }
                 store4(crow + col, x);
+                if constexpr (MODE == EPI_STORE_T)
+                  sbuf[rr * 8 + ((cq >> 2) ^ (rr & 7))] = make_float4(x[0], x[1], x[2], x[3]);
                 if constexpr (MODE == EPI_STORE_COPY) {
                   __nv_bfloat16* c16 = args.C16 + tc.z0 * args.cs0 + tc.z1 * args.cs1 +
                                        (long long)row_o * args.ldc + col;
@@ -496,9 +497,28 @@ __global__ void __launch_bounds__(THREADS, 1)
                   float y = x[j];
                   if (irow) y = fmaf(args.beta, irow[col + j], y);
                   crow[col + j] = from_f32<TC>(y);
+                  x[j] = y;
                   if constexpr (MODE == EPI_STORE_COPY)
                     args.C16[tc.z0 * args.cs0 + tc.z1 * args.cs1 + (long long)row_o * args.ldc +
                              col + j] = __float2bfloat16_rn(y);
+                }
+                if constexpr (MODE == EPI_STORE_T)
+                  sbuf[rr * 8 + ((cq >> 2) ^ (rr & 7))] = make_float4(x[0], x[1], x[2], x[3]);
+              }
+            }
+            if constexpr (MODE == EPI_STORE_T) {
+              // the chunk's final values, transposed: lane l holds row rbase + l, and each
+              // store writes one column's 32 rows (128 contiguous bytes)
+              __syncwarp();
+              const int row_t = rbase + lane;
+              if (args.Ct && row_t < args.M) {
+                float* tb = args.Ct + tc.z0 * args.ts0 + tc.z1 * args.ts1 + row_t;
+                const float* sv = reinterpret_cast<const float*>(sbuf);
+#pragma unroll 8
+                for (int c = 0; c < 32; ++c) {
+                  if (col0 + c >= args.N) break;
+                  tb[(long long)(col0 + c) * args.ldt] =
+                      sv[(lane * 8 + ((c >> 2) ^ (lane & 7))) * 4 + (c & 3)];
                 }
               }
             }
@@ -688,13 +708,13 @@ int sm_count() {
   return cache[dev];
 }
 
-// 4-D map {inner, outer, z0, z1} over one operand; box {64, box_outer, 1, 1}.
+// 4-D map {inner, outer, z0, z1} over one operand; box {64, box_outer, 1, 1} (bf16), or
+// {32, box_outer, 1, 1} over fp32 for tf32 operands (128-byte rows either way).
 bool make_map(CUtensorMap* map, const GemmOperand& op, int rows, int K, int Z0, int Z1,
-              int box_rows) {
+              int box_rows, bool tf32 = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   const bool mn = op.mn_major;
-  if (op.hilo) K = (int)(2 * op.k0);   // the buffer holds [hi | lo] along K
   cuuint64_t dims[4];
   cuuint64_t strides[3];
   cuuint32_t box[4];
@@ -703,16 +723,18 @@ bool make_map(CUtensorMap* map, const GemmOperand& op, int rows, int K, int Z0, 
   dims[1] = (cuuint64_t)(mn ? K : rows);
   dims[2] = (cuuint64_t)(op.s0 ? Z0 : 1);
   dims[3] = (cuuint64_t)(op.s1 ? Z1 : 1);
-  const cuuint64_t row_bytes = (cuuint64_t)op.ld * 2;
+  const cuuint64_t es = tf32 ? 4 : 2;
+  const cuuint64_t row_bytes = (cuuint64_t)op.ld * es;
   const cuuint64_t plane = ((row_bytes * dims[1]) + 15) & ~(cuuint64_t)15;
   strides[0] = row_bytes;
-  strides[1] = op.s0 ? (cuuint64_t)op.s0 * 2 : plane;
-  strides[2] = op.s1 ? (cuuint64_t)op.s1 * 2 : plane * dims[2];
-  box[0] = 64;
+  strides[1] = op.s0 ? (cuuint64_t)op.s0 * es : plane;
+  strides[2] = op.s1 ? (cuuint64_t)op.s1 * es : plane * dims[2];
+  box[0] = tf32 ? 32 : 64;
   box[1] = (cuuint32_t)(mn ? 64 : box_rows);
   box[2] = 1;
   box[3] = 1;
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(op.ptr), dims,
+  CUresult r = fn(map, tf32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  4, const_cast<void*>(op.ptr), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -736,12 +758,13 @@ bool make_out_map(CUtensorMap* map, void* ptr, int cols, int rows, long long ld,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES>
+template <int BN, bool A_MN, bool B_MN, int STAGES, int MODE, typename TC, bool BRES,
+          bool TF = false>
 ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   CUtensorMap ma, mb;
   OutMaps om;
-  if (!make_map(&ma, p.A, p.M, p.K, p.Z0, p.Z1, BM) ||
-      !make_map(&mb, p.B, p.N, p.K, p.Z0, p.Z1, BN)) {
+  if (!make_map(&ma, p.A, p.M, p.K, p.Z0, p.Z1, BM, TF) ||
+      !make_map(&mb, p.B, p.N, p.K, p.Z0, p.Z1, BN, TF)) {
     set_error_message("gemm_umma: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", p.M, p.N, p.K);
     return TTT_ERR_CUDA;
   }
@@ -755,7 +778,7 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
       return TTT_ERR_CUDA;
     }
   }
-  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC, BRES>;
+  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, STAGES, MODE, TC, BRES, TF>;
   constexpr int SMEM = Smem<BN, STAGES, BRES, MODE>::TOTAL;
   static_assert(SMEM <= 232448, "shared memory budget");
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
@@ -828,13 +851,28 @@ ttt_status dispatch_bn(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// tf32 operands: streamed K-major operands, fp32 C; the transposed-copy epilogue when asked
+// for, the staged one with an addend or a large output, else direct row stores.
+template <int MODE>
+ttt_status dispatch_tf32_mode(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
+  if (p.N > 128) return launch_umma<256, false, false, 4, MODE, float, false, true>(p, a, s);
+  if (p.N > 64) return launch_umma<128, false, false, 3, MODE, float, false, true>(p, a, s);
+  return launch_umma<64, false, false, 4, MODE, float, false, true>(p, a, s);
+}
+ttt_status dispatch_tf32(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
+  if (a.Ct) return dispatch_tf32_mode<EPI_STORE_T>(p, a, s);
+  if (a.Cin || (long long)p.M * p.N * p.Z0 * p.Z1 * 4 > (64LL << 20))
+    return dispatch_tf32_mode<EPI_STORE_STG>(p, a, s);
+  return dispatch_tf32_mode<EPI_STORE>(p, a, s);
+}
+
 UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait_ns) {
   UArgs a{};
   a.M = p.M; a.N = p.N; a.K = p.K; a.Z0 = p.Z0; a.Z1 = p.Z1;
   a.a_b0 = p.A.s0 != 0; a.a_b1 = p.A.s1 != 0; a.b_b0 = p.B.s0 != 0; a.b_b1 = p.B.s1 != 0;
-  a.a_hilo = p.A.hilo; a.a_k0 = (int)p.A.k0; a.b_hilo = p.B.hilo; a.b_k0 = (int)p.B.k0;
   a.C = p.C.ptr; a.ldc = p.C.ld; a.cs0 = p.C.s0; a.cs1 = p.C.s1;
   a.C16 = static_cast<__nv_bfloat16*>(p.C.copy16);
+  a.Ct = p.C.t32; a.ldt = p.C.ldt; a.ts0 = p.C.ts0; a.ts1 = p.C.ts1;
   a.Cin = p.beta != 0.0f ? p.Cin.ptr : nullptr;
   a.ldi = p.Cin.ld; a.is0 = p.Cin.s0; a.is1 = p.Cin.s1;
   a.alpha = p.alpha; a.beta = p.beta;
@@ -852,9 +890,6 @@ const char* umma_unsupported_reason(const GemmProblem& p) {
     if (o->ld <= 0 || o->ld % 8 != 0) return "operand row stride must be a multiple of 8";
     if (o->s0 < 0 || o->s1 < 0 || o->s0 % 8 != 0 || o->s1 % 8 != 0)
       return "operand batch strides must be non-negative multiples of 8";
-    if (o->hilo && (o->hilo > 2 || o->k0 <= 0 || o->k0 % BK != 0 || p.K != 3 * o->k0 ||
-                    o->k0 > (1LL << 30)))
-      return "split-precision operand needs K = 3 k0 with k0 a multiple of 64";
   }
   if (p.K <= 0 || p.M <= 0 || p.N <= 0) return "M, N and K must be positive";
   if ((long long)p.Z0 * p.Z1 * ((p.M + BM - 1) / BM) * ((p.N + 63) / 64) > (1LL << 31))
@@ -863,6 +898,28 @@ const char* umma_unsupported_reason(const GemmProblem& p) {
   if (p.C.copy16 && (p.C.dtype != DT_F32 || !aligned16(p.C.copy16) || !aligned16(p.C.ptr) ||
                      p.C.ld % 4 != 0 || p.C.s0 % 4 != 0 || p.C.s1 % 4 != 0))
     return "a bf16 copy needs an fp32 result with 16-byte aligned bases, strides multiples of 4";
+  if (p.C.t32) return "a transposed copy is written only with tf32 operands";
+  if (encode_fn() == nullptr) return "cuTensorMapEncodeTiled is unavailable";
+  return nullptr;
+}
+
+const char* umma_tf32_unsupported_reason(const GemmProblem& p) {
+  for (const GemmOperand* o : {&p.A, &p.B}) {
+    if (o->dtype != DT_F32) return "tf32 operands must be fp32";
+    if (o->mn_major) return "tf32 operands must be K-major";
+    if (!o->ptr || !aligned16(o->ptr)) return "operand base must be 16-byte aligned";
+    if (o->ld <= 0 || o->ld % 4 != 0) return "operand row stride must be a multiple of 4";
+    if (o->s0 < 0 || o->s1 < 0 || o->s0 % 4 != 0 || o->s1 % 4 != 0)
+      return "operand batch strides must be non-negative multiples of 4";
+  }
+  if (p.K <= 0 || p.M <= 0 || p.N <= 0) return "M, N and K must be positive";
+  if ((long long)p.Z0 * p.Z1 * ((p.M + BM - 1) / BM) * ((p.N + 63) / 64) > (1LL << 31))
+    return "too many output tiles";
+  if (p.C.dtype != DT_F32) return "tf32 products write fp32";
+  if (p.beta != 0.0f && !p.Cin.ptr) return "beta != 0 needs an addend";
+  if (p.C.copy16) return "no bf16 copy with tf32 operands";
+  if (p.C.t32 && (p.C.ldt < p.M || p.C.ts0 < 0 || p.C.ts1 < 0))
+    return "transposed copy needs a row stride of at least M";
   if (encode_fn() == nullptr) return "cuTensorMapEncodeTiled is unavailable";
   return nullptr;
 }
@@ -879,6 +936,16 @@ ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_er
   const UArgs a = base_args(p, dev_err, wait_ns);
   if (p.C.dtype == DT_BF16) return dispatch_bn<__nv_bfloat16>(p, a, stream);
   return dispatch_bn<float>(p, a, stream);
+}
+
+ttt_status gemm_umma_tf32(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,
+                          unsigned long long wait_ns) {
+  if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
+  if (const char* why = umma_tf32_unsupported_reason(p)) {
+    set_error_message("gemm_umma_tf32: %s", why);
+    return TTT_ERR_UNSUPPORTED;
+  }
+  return dispatch_tf32(p, base_args(p, dev_err, wait_ns), stream);
 }
 
 const char* umma_swiglu_unsupported_reason(const SwigluGemm& g) {

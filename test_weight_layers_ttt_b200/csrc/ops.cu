@@ -370,11 +370,11 @@ __global__ void ns_sumsq_kernel(const float* U, NsLayout L, float* nrm) {
   }
 }
 
-// X (wide orientation) = U * scale, or U <- X back (to_u): 32 x 32 tiles through shared
-// memory so both sides are read and written along rows. grid (tiles of the problem,
-// parts, Z), block (32, 8).
+// X (wide orientation) = U * scale, and optionally Xt = X^T, or U <- X back (to_u): 32 x 32
+// tiles through shared memory so every side is read and written along rows. grid (tiles of
+// the problem, parts, Z), block (32, 8).
 __global__ void ns_copy_kernel(const float* U_in, float* X, float* U_out, NsLayout L,
-                               const float* nrm, float eps, int to_u) {
+                               const float* nrm, float eps, int to_u, float* Xt) {
   const int p = blockIdx.y, z = blockIdx.z;
   if (!(L.mask & (1 << p))) return;
   const int R = L.R[p], Cc = L.C[p];
@@ -395,14 +395,15 @@ __global__ void ns_copy_kernel(const float* U_in, float* X, float* U_out, NsLayo
       t[k][tx] = (i < R && j < Cc) ? u[(long long)i * Cc + j] * scale : 0.0f;
     }
     __syncthreads();
+    float* xt = Xt ? Xt + ((long long)z * L.parts + p) * n : nullptr;
     for (int k = ty; k < 32; k += 8) {
-      if (!tr) {
-        const int i = i0 + k, j = j0 + tx;
-        if (i < R && j < Cc) x[(long long)i * Cc + j] = t[k][tx];
-      } else {   // x is [Cc, R]: x[j][i] = u[i][j]
-        const int j = j0 + k, i = i0 + tx;
-        if (i < R && j < Cc) x[(long long)j * R + i] = t[tx][k];
-      }
+      // U's own orientation [R, Cc] and the transposed one [Cc, R]
+      const int i = i0 + k, j = j0 + tx;
+      const int jt = j0 + k, it = i0 + tx;
+      float* same = tr ? xt : x;
+      float* other = tr ? x : xt;
+      if (same && i < R && j < Cc) same[(long long)i * Cc + j] = t[k][tx];
+      if (other && it < R && jt < Cc) other[(long long)jt * R + it] = t[tx][k];
     }
   } else {
     float* u = U_out + uoff;
@@ -423,50 +424,6 @@ __global__ void ns_copy_kernel(const float* U_in, float* X, float* U_out, NsLayo
   }
 }
 
-
-// P row-major [rows, cols] fp32 matrices -> bf16 hi = bf16(x), lo = bf16(x - hi), stored
-// once each for split-precision GEMM operands:
-//   kmaj [P][rows][2 cols_p]   row r: hi (cols) | zeros | lo (cols) | zeros   (K along a row)
-//   mmaj [P][2 rows_p][cols]   rows 0..rows-1 hi, zero rows, rows_p.. lo, zero rows (K down)
-// (either may be null). One thread per 8 columns of one row of the padded shape.
-__global__ void split_hilo2_kernel(const float* M, long long P, int rows, int cols, int rows_p,
-                                   int cols_p, uint4* kmaj, uint4* mmaj) {
-  const int c8 = cols / 8, c8p = cols_p / 8;
-  TTT_GRID_LOOP(idx, P * rows_p * c8p) {
-    const long long pr = idx / c8p;             // p * rows_p + row
-    const int q = (int)(idx - pr * c8p);
-    const long long p = pr / rows_p;
-    const int row = (int)(pr - p * rows_p);
-    uint4 H = make_uint4(0u, 0u, 0u, 0u), Lo = H;
-    if (row < rows && q < c8) {
-      const float* src = M + (p * rows + row) * cols + 8 * q;
-      const float4 a = *reinterpret_cast<const float4*>(src);
-      const float4 b = *reinterpret_cast<const float4*>(src + 4);
-      const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * t], x[2 * t + 1]);
-        const float2 hf = __bfloat1622float2(h2);
-        const __nv_bfloat162 l2 = __floats2bfloat162_rn(x[2 * t] - hf.x, x[2 * t + 1] - hf.y);
-        hi[t] = *reinterpret_cast<const uint32_t*>(&h2);
-        lo[t] = *reinterpret_cast<const uint32_t*>(&l2);
-      }
-      H = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      Lo = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
-    if (kmaj && row < rows) {
-      uint4* o = kmaj + (p * rows + row) * 2 * c8p + q;
-      o[0] = H;
-      o[c8p] = Lo;
-    }
-    if (mmaj && q < c8) {
-      uint4* o = mmaj + (p * 2 * rows_p + row) * c8 + q;
-      o[0] = H;
-      o[(long long)rows_p * c8] = Lo;
-    }
-  }
-}
 
 // out[z] = in[z]^T for Z row-major [rows, cols] fp32 matrices: 32 x 32 tiles through shared
 // memory, both sides along rows. grid (ceil(cols/32), ceil(rows/32), Z), block (32, 8).
@@ -930,7 +887,7 @@ cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all
 }
 
 cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
-                         float* nrm, cudaStream_t s) {
+                         float* nrm, cudaStream_t s, float* Xt) {
   if (Z <= 0) return cudaSuccess;
   cudaError_t e = fill_f32(nrm, (long long)Z * L.parts, 0.0f, s);
   if (e != cudaSuccess) return e;
@@ -938,7 +895,8 @@ cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, flo
   int tiles = 0;
   for (int p = 0; p < L.parts; ++p)
     tiles = max(tiles, ((L.R[p] + 31) / 32) * ((L.C[p] + 31) / 32));
-  ns_copy_kernel<<<dim3(tiles, L.parts, Z), dim3(32, 8), 0, s>>>(U, X, nullptr, L, nrm, eps, 0);
+  ns_copy_kernel<<<dim3(tiles, L.parts, Z), dim3(32, 8), 0, s>>>(U, X, nullptr, L, nrm, eps, 0,
+                                                                 Xt);
   return cudaGetLastError();
 }
 
@@ -948,22 +906,11 @@ cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cud
   for (int p = 0; p < L.parts; ++p)
     tiles = max(tiles, ((L.R[p] + 31) / 32) * ((L.C[p] + 31) / 32));
   ns_copy_kernel<<<dim3(tiles, L.parts, Z), dim3(32, 8), 0, s>>>(
-      nullptr, const_cast<float*>(X), U, L, nullptr, 0.0f, 1);
+      nullptr, const_cast<float*>(X), U, L, nullptr, 0.0f, 1, nullptr);
   return cudaGetLastError();
 }
 
 
-cudaError_t split_hilo2(const float* M, int P, int rows, int cols, int rows_p, int cols_p,
-                        void* kmaj, void* mmaj, cudaStream_t s) {
-  if (P <= 0 || rows <= 0 || cols <= 0) return cudaSuccess;
-  if (cols % 8 != 0 || cols_p % 8 != 0 || cols_p < cols || rows_p < rows)
-    return cudaErrorInvalidValue;
-  const long long n = (long long)P * rows_p * (cols_p / 8);
-  split_hilo2_kernel<<<grid_for(n, 256), 256, 0, s>>>(M, P, rows, cols, rows_p, cols_p,
-                                                      static_cast<uint4*>(kmaj),
-                                                      static_cast<uint4*>(mmaj));
-  return cudaGetLastError();
-}
 
 cudaError_t suffix_scan(int ot, const float* dSc, const float* dS_final, void* G, float* R0,
                         int BH, int C, long long n, int order, cudaStream_t s) {

@@ -72,12 +72,12 @@ inline NsLayout ns_layout_single(int R, int C) {
   return NsLayout{1, 1, (long long)R * C, 0, {R, R, R}, {C, C, C}};
 }
 
-// Newton-Schulz set-up / tear-down for the CUDA-core path: X = U / (||U||_F + eps) in the
+// Newton-Schulz set-up / tear-down for the batched paths: X = U / (||U||_F + eps) in the
 // wide orientation ([min(R,C), max(R,C)]) into the scratch X (problem (z, p) at
-// (z * parts + p) * R * C), and U <- X back in U's own orientation. Z entries. nrm: fp32
-// scratch of Z * parts sums of squares.
+// (z * parts + p) * R * C), with its transpose into Xt when Xt is not null, and U <- X back
+// in U's own orientation. Z entries. nrm: fp32 scratch of Z * parts sums of squares.
 cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
-                         float* nrm, cudaStream_t s);
+                         float* nrm, cudaStream_t s, float* Xt = nullptr);
 cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cudaStream_t s);
 
 // The whole Newton-Schulz orthogonalisation of the matrices of L on the tensor cores
@@ -89,12 +89,6 @@ bool ns_mma_supported(int R, int C);
 cudaError_t ns_mma(float* U, int Z, const NsLayout& L, int steps, float eps, float a, float b,
                    float c, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
 
-// Split fp32 matrices M [P, rows, cols] (cols % 8 == 0) into bf16 hi = bf16(x) and
-// lo = bf16(x - hi), each stored once for split-precision GEMM operands (GemmOperand::hilo):
-// kmaj [P][rows][2 cols_p] = [hi | lo] along each row, mmaj [P][2 rows_p][cols] = [hi ; lo]
-// down the rows, zero padded to cols_p / rows_p (multiples of 64); either may be null.
-cudaError_t split_hilo2(const float* M, int P, int rows, int cols, int rows_p, int cols_p,
-                        void* kmaj, void* mmaj, cudaStream_t s);
 
 // Backward of the prefix scan: R = dS_final[bh] (or 0 when null), then for c = C-1 .. 0:
 // R += dSc[bh, c] and the gradient of chunk c's delta G[bh, c] (OT) is R (order 0) or the

@@ -114,10 +114,19 @@ ttt_status run_gemm(const char* name, const GemmProblem& p, cudaStream_t s) {
     TraceScope ts(g_trace.on ? engine_name(name, "tcgen05") : name, s);
     return gemm_umma(p, s, device_error_word(), wait_limit_ns());
   }
-  if (p.A.hilo || p.B.hilo)
-    return fail(TTT_ERR_UNSUPPORTED, "%s: split-precision operands need bf16", name);
   TraceScope ts(g_trace.on ? engine_name(name, "simt") : name, s);
   return gemm_simt(p, s);
+}
+
+// A product of the bf16 mode that needs more than bf16 operands: fp32 operands read as tf32
+// by the tensor-core engine (never the CUDA cores).
+ttt_status run_tf32(const char* name, const GemmProblem& p, cudaStream_t s) {
+  if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
+  if (const char* why = umma_tf32_unsupported_reason(p))
+    return fail(TTT_ERR_UNSUPPORTED, "%s: tensor-core engine (tf32): %s (M=%d N=%d K=%d)", name,
+                why, p.M, p.N, p.K);
+  TraceScope ts(g_trace.on ? engine_name(name, "tcgen05") : name, s);
+  return gemm_umma_tf32(p, s, device_error_word(), wait_limit_ns());
 }
 
 ttt_status run_simt(const char* name, const GemmProblem& p, cudaStream_t s) {
@@ -607,19 +616,16 @@ ttt_status linear_impl(const ttt_desc& d, const void* q, const void* k, const vo
 }
 
 // ------------------------------------------------------------------ Newton-Schulz
-// bf16 mode runs Newton-Schulz on the tensor cores with split bf16 operands (close to
-// fp32): one CTA per matrix when it fits, else batched GEMMs; fp32 mode uses fp32
-// CUDA-core products.
+// bf16 mode runs Newton-Schulz on the tensor cores at more than bf16 precision: one CTA
+// per matrix with split bf16 operands when it fits, else batched GEMMs on tf32 operands;
+// fp32 mode uses fp32 CUDA-core products.
 
 // Newton-Schulz scratch. CUDA-core path: X, X2 [problems, r, c], Ag, Pm [problems, r, r]
-// fp32. Split-bf16 GEMM path: the same fp32 buffers (Ag holds A = X X^T, Pm the polynomial)
-// plus the bf16 hi/lo operands below (see run_ns). The one-CTA path needs none of them.
+// fp32. tf32 GEMM path: the same, plus the transposes Xt, X2t [problems, c, r] (the K-major
+// form of X as the right operand of P X). The one-CTA path needs none of them.
 struct NsScratch {
   float *X = nullptr, *X2 = nullptr, *Ag = nullptr, *Pm = nullptr, *nrm = nullptr;
-  // split-precision operands of the tensor-core GEMM path ([hi | lo] stored once; r, c
-  // padded to rp, cp, multiples of 64): X along rows [r][2cp] and down rows [2rp][c], A and
-  // P along rows [r][2rp]
-  void *Xk = nullptr, *Xm = nullptr, *Gk = nullptr, *Pk = nullptr;
+  float *Xt = nullptr, *X2t = nullptr;
 };
 
 enum NsPath { NS_TENSOR_CTA = 0, NS_TENSOR_GEMM = 1, NS_CUDA_CORES = 2 };
@@ -641,11 +647,8 @@ NsScratch plan_ns(Carve& cv, int ot, long long problems, int R, int C) {
   w.Pm = cv.take_n<float>(problems * r * r);
   w.nrm = cv.take_n<float>(problems);
   if (path == NS_TENSOR_GEMM) {
-    const long long rp = (r + 63) / 64 * 64, cp = (c + 63) / 64 * 64;
-    w.Xk = cv.take(2 * problems * r * 2 * cp);
-    w.Xm = cv.take(2 * problems * 2 * rp * c);
-    w.Gk = cv.take(2 * problems * r * 2 * rp);
-    w.Pk = cv.take(2 * problems * r * 2 * rp);
+    w.Xt = cv.take_n<float>(problems * r * c);
+    w.X2t = cv.take_n<float>(problems * r * c);
   }
   return w;
 }
@@ -664,48 +667,44 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
   }
   const long long r = R < Cc ? R : Cc, cc = R < Cc ? Cc : R;
   const int P = Z * L.parts;
-  TTT_OP("ns_normalize", ns_normalize(U, w.X, Z, L, 1e-7f, w.nrm, s));
-  if (ns_path(ot, (int)R, (int)Cc) == NS_TENSOR_GEMM) {
-    // Each product as one bf16 GEMM over K tripled: hi*hi + hi*lo + lo*hi of the split
-    // operands (x = hi + lo to about 2^-16), fp32 accumulation in TMEM. Each split matrix
-    // is stored once as [hi | lo]; the GEMM reads the thirds [hi hi lo] of the A operand
-    // and [hi lo hi] of the B operand from it (GemmOperand::hilo).
-    float* X = w.X;
-    float* X2 = w.X2;
-    const long long rp = (r + 63) / 64 * 64, cp = (cc + 63) / 64 * 64;
-    auto op = [](void* ptr, bool mn, long long ld, long long s0, int hilo, long long k0) {
+  const bool tf32 = ns_path(ot, (int)R, (int)Cc) == NS_TENSOR_GEMM;
+  TTT_OP("ns_normalize", ns_normalize(U, w.X, Z, L, 1e-7f, w.nrm, s, tf32 ? w.Xt : nullptr));
+  if (tf32) {
+    // Each product on the tensor cores with fp32 operands read as tf32 (10-bit mantissa,
+    // fp32 accumulation in TMEM), all operands K-major: A = X X^T from X [r, c]; P = c A A +
+    // b A from A (symmetric, so it serves as its own K-major right operand); X' = P X + a X
+    // with X's transpose [c, r] as the right operand, and X'^T written by the same epilogue
+    // for the next step.
+    float *X = w.X, *X2 = w.X2, *Xt = w.Xt, *X2t = w.X2t;
+    auto op = [](const float* ptr, long long ld, long long s0) {
       GemmOperand o;
-      o.ptr = ptr; o.dtype = DT_BF16; o.mn_major = mn; o.ld = ld; o.s0 = s0; o.s1 = 0;
-      o.hilo = hilo; o.k0 = k0;
+      o.ptr = ptr; o.dtype = DT_F32; o.mn_major = false; o.ld = ld; o.s0 = s0; o.s1 = 0;
       return o;
     };
     for (int it = 0; it < steps; ++it) {
-      TTT_OP("ns_split", split_hilo2(X, P, (int)r, (int)cc, (int)rp, (int)cp, w.Xk, w.Xm, s));
       GemmProblem g1;  // A = X X^T
-      g1.M = (int)r; g1.N = (int)r; g1.K = (int)(3 * cp); g1.Z0 = P;
-      g1.A = op(w.Xk, false, 2 * cp, r * 2 * cp, 1, cp);
-      g1.B = op(w.Xk, false, 2 * cp, r * 2 * cp, 2, cp);
+      g1.M = (int)r; g1.N = (int)r; g1.K = (int)cc; g1.Z0 = P;
+      g1.A = op(X, cc, r * cc);
+      g1.B = op(X, cc, r * cc);
       g1.C = {w.Ag, DT_F32, r, r * r, 0};
-      TTT_TRY(run_gemm("ns_gram", g1, s));
-      TTT_OP("ns_split", split_hilo2(w.Ag, P, (int)r, (int)r, (int)rp, (int)rp, w.Gk, nullptr,
-                                      s));
-      GemmProblem g2;  // P = c A A + b A (A symmetric: its B operand is read K-major)
-      g2.M = (int)r; g2.N = (int)r; g2.K = (int)(3 * rp); g2.Z0 = P;
-      g2.A = op(w.Gk, false, 2 * rp, r * 2 * rp, 1, rp);
-      g2.B = op(w.Gk, false, 2 * rp, r * 2 * rp, 2, rp);
+      TTT_TRY(run_tf32("ns_gram", g1, s));
+      GemmProblem g2;  // P = c A A + b A
+      g2.M = (int)r; g2.N = (int)r; g2.K = (int)r; g2.Z0 = P;
+      g2.A = op(w.Ag, r, r * r);
+      g2.B = op(w.Ag, r, r * r);
       g2.C = {w.Pm, DT_F32, r, r * r, 0};
       g2.alpha = c3; g2.beta = b3; g2.Cin = {w.Ag, r, r * r, 0};
-      TTT_TRY(run_gemm("ns_poly", g2, s));
-      TTT_OP("ns_split", split_hilo2(w.Pm, P, (int)r, (int)r, (int)rp, (int)rp, w.Pk, nullptr,
-                                      s));
-      GemmProblem g3;  // X' = P X + a X
-      g3.M = (int)r; g3.N = (int)cc; g3.K = (int)(3 * rp); g3.Z0 = P;
-      g3.A = op(w.Pk, false, 2 * rp, r * 2 * rp, 1, rp);
-      g3.B = op(w.Xm, true, cc, 2 * rp * cc, 2, rp);
+      TTT_TRY(run_tf32("ns_poly", g2, s));
+      GemmProblem g3;  // X' = P X + a X, and X'^T
+      g3.M = (int)r; g3.N = (int)cc; g3.K = (int)r; g3.Z0 = P;
+      g3.A = op(w.Pm, r, r * r);
+      g3.B = op(Xt, r, r * cc);
       g3.C = {X2, DT_F32, cc, r * cc, 0};
+      g3.C.t32 = X2t; g3.C.ldt = r; g3.C.ts0 = r * cc;
       g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, cc, r * cc, 0};
-      TTT_TRY(run_gemm("ns_apply", g3, s));
-      float* t = X; X = X2; X2 = t;
+      TTT_TRY(run_tf32("ns_apply", g3, s));
+      std::swap(X, X2);
+      std::swap(Xt, X2t);
     }
     TTT_OP("ns_writeback", ns_writeback(X, U, Z, L, s));
     return TTT_OK;

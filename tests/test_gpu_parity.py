@@ -301,9 +301,11 @@ MOM_CASES = [
     ("lm", "bf16", 2, 1, 1000, 128, 256, 256, True, 5),    # tensor-core Newton-Schulz
     ("lm", "bf16", 1, 2, 640, 64, 192, 128, False, 5),
     ("lm", "bf16", 1, 2, 640, 64, 192, 128, True, 0),
-    # bf16 with 136 x 256 matrices (over the one-CTA limit): three split-precision GEMMs per
-    # step, K padded from 136 to 192
+    # bf16 with 136 x 256 matrices (over the one-CTA limit): three tf32 GEMMs per step,
+    # K = 136 not a multiple of the 32-wide k-block (zero-filled tail)
     ("lm", "bf16", 1, 1, 512, 256, 136, 128, True, 3),
+    # the lm shape: 256 x 512 matrices, five steps
+    ("lm", "bf16", 1, 1, 1024, 256, 512, 256, True, 5),
 ]
 
 
@@ -430,8 +432,7 @@ REC_CASES = [
     ("lm", "bf16", 1, 1, 512, 128, 64, 256, dict(update_mask=5, ns_steps=5)),
     # ragged matrices for the tensor-core Newton-Schulz (zero padding inside the CTA)
     ("lm", "bf16", 1, 2, 320, 40, 200, 96, dict(renorm=True, momentum=True, ns_steps=5)),
-    # min(h, m) > 128: bf16 mode runs Newton-Schulz as three split-precision GEMMs per step
-    # (K padded to a multiple of 64); 3 steps
+    # min(h, m) > 128: bf16 mode runs Newton-Schulz as three tf32 GEMMs per step; 3 steps
     ("lm", "bf16", 1, 1, 256, 256, 136, 128, dict(ns_steps=3)),
 ]
 
