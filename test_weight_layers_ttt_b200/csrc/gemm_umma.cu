@@ -359,6 +359,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int ew = warp - 2;
     const int quarter = warp & 3;
     const int part = ew >> 2;  // 0: first half of the tile's columns, 1: second half
+    int grad_stores = 0;       // gradient epilogue: stores issued (sub-box = count % 2)
     for (int lt = 0; lt < walk.count; ++lt) {
       const int buf = lt & 1;
       const TileCoord tc = walk.at(lt);
@@ -526,9 +527,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       } else if (args.grad) {
-        // Gradient pieces of the recurrent form. Each output is produced in two 32-column
-        // halves straight from TMEM (re-read per output to keep registers low) into this
-        // warp's staging box, then stored with TMA; TMEM is released after the last read.
+        // Gradient pieces of the recurrent form in one pass: per 32-column half, A/2 and B
+        // are read from TMEM once, tanh(a/2) is evaluated once per element, and the (up to)
+        // three outputs are packed to bf16 together; each output half leaves through one of
+        // this warp's two 2 KB sub-boxes (64-byte swizzle) with a TMA store, a sub-box being
+        // refilled once the store before the last has read it. TMEM is released after the
+        // second half's loads.
         constexpr int PH = BN / 2;
         constexpr int QW = PH / 2;
         const bool live = row < args.M;
@@ -539,76 +543,71 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int oy = tc.tm * BM + quarter * 32;
         const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
         const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
-        // this row's 64 dv values of the tile (both 32-column halves), loaded once for the
-        // two outputs that use them, all eight 16-byte loads in flight together
-        uint4 dvq[8];
+        const bool want[3] = {!args.skip_out1, args.C2 != nullptr, args.C3 != nullptr};
+        const bool need_dv = want[1] || want[2];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = ox + (j >> 2) * 32 + (j & 3) * 8;
-          dvq[j] = (live && (args.C2 || args.C3) && col + 8 <= args.n_valid)
-                       ? *reinterpret_cast<const uint4*>(dvrow + col)
-                       : make_uint4(0u, 0u, 0u, 0u);
-        }
-        for (int o = 0; o < 3; ++o) {
-          if ((o == 0 && args.skip_out1) || (o == 1 && !args.C2) || (o == 2 && !args.C3))
-            continue;
-          if (lane == 0) tma_store_wait_read();
-          __syncwarp();
+        for (int hh = 0; hh < 2; ++hh) {
+          // this row's 32 dv values of the half, all four 16-byte loads in flight together
+          uint4 dvq[4];
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t ra[32], rb[32];
-            tmem_ld32(lane_addr + (uint32_t)(part * QW + hh * 32), ra);
-            tmem_ld32(lane_addr + (uint32_t)(PH + part * QW + hh * 32), rb);
-            tmem_ld_wait();
-            float dvv[32];
+          for (int j = 0; j < 4; ++j) {
+            const int col = ox + hh * 32 + j * 8;
+            dvq[j] = (live && need_dv && col + 8 <= args.n_valid)
+                         ? *reinterpret_cast<const uint4*>(dvrow + col)
+                         : make_uint4(0u, 0u, 0u, 0u);
+          }
+          uint32_t ra[32], rb[32];
+          tmem_ld32(lane_addr + (uint32_t)(part * QW + hh * 32), ra);
+          tmem_ld32(lane_addr + (uint32_t)(PH + part * QW + hh * 32), rb);
+          tmem_ld_wait_regs(ra, rb);
+          if (hh == 1) {
+            tc_fence_before();
+            mbar_arrive(smem_u32(&acc_empty[buf]));
+          }
+          uint32_t pk[3][16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              const uint4 u = dvq[hh * 4 + j / 8];
-              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+          for (int j = 0; j < 32; j += 2) {
+            const uint32_t dw = (&dvq[j >> 3].x)[(j & 7) >> 1];
+            const float2 dvf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dw));
+            float v[3][2];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const float2 f = __bfloat1622float2(h2[q]);
-                dvv[j + 2 * q] = f.x;
-                dvv[j + 2 * q + 1] = f.y;
-              }
+            for (int u = 0; u < 2; ++u) {
+              // accumulator half A holds a/2 (the operand carries W0 / 2)
+              const float hlf = __uint_as_float(ra[j + u]), bb = __uint_as_float(rb[j + u]);
+              const float t = tanh_fast(hlf);
+              const float sg = fmaf(0.5f, t, 0.5f);   // sigmoid(a)
+              const float sa = fmaf(hlf, t, hlf);     // silu(a) = (a/2)(1 + tanh(a/2))
+              const float d = -eta * (u ? dvf.y : dvf.x);
+              v[0][u] = sa * bb * eta;
+              v[1][u] = d * sa;
+              v[2][u] = d * bb * sg * fmaf(2.0f * hlf, 1.0f - sg, 1.0f);   // silu'(a)
             }
-            uint32_t pk[16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              float v[2];
+            for (int o = 0; o < 3; ++o) pk[o][j / 2] = pack_bf16x2(v[o][0], v[o][1]);
+          }
 #pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                // accumulator half A holds a/2 (the operand carries W0 / 2)
-                const float hlf = __uint_as_float(ra[j + u]), bb = __uint_as_float(rb[j + u]);
-                const float t = tanh_fast(hlf);
-                const float sg = fmaf(0.5f, t, 0.5f);   // sigmoid(a)
-                const float sa = fmaf(hlf, t, hlf);     // silu(a) = (a/2)(1 + tanh(a/2))
-                const float d = -eta * dvv[j + u];
-                if (o == 0) v[u] = sa * bb * eta;
-                else if (o == 1) v[u] = d * sa;
-                else v[u] = d * bb * sg * fmaf(2.0f * hlf, 1.0f - sg, 1.0f);   // silu'(a)
-              }
-              pk[j / 2] = pack_bf16x2(v[0], v[1]);
-            }
+          for (int o = 0; o < 3; ++o) {
+            if (!want[o] || ox + hh * 32 >= args.n_valid) continue;
+            const uint32_t sub = box + (uint32_t)((grad_stores & 1) * 2048);
+            if (lane == 0) tma_store_wait_read_1();
+            __syncwarp();
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-              const int c = hh * 4 + cc;
-              const uint32_t addr = box + lane * 128 + ((c ^ (lane & 7)) << 4);
+              const uint32_t addr = sub + lane * 64 + ((cc ^ ((lane >> 1) & 3)) << 4);
               asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                           "r"(pk[4 * cc]), "r"(pk[4 * cc + 1]), "r"(pk[4 * cc + 2]),
-                           "r"(pk[4 * cc + 3])
+                           "r"(pk[o][4 * cc]), "r"(pk[o][4 * cc + 1]), "r"(pk[o][4 * cc + 2]),
+                           "r"(pk[o][4 * cc + 3])
                            : "memory");
             }
-          }
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0 && ox < args.n_valid) {
-            tma_store_4d(&om.m[o], box, ox, oy, c2, c3);
-            tma_store_commit();
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_4d(&om.m[o], sub, ox + hh * 32, oy, c2, c3);
+              tma_store_commit();
+            }
+            ++grad_stores;
           }
         }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&acc_empty[buf]));
       } else {
         // SWIGLU: phi column p of this tile uses accumulator columns p (A/2) and BN/2 + p (B).
         // Each epilogue warp owns 32 rows x 64 phi columns: two 32-column pieces, the
@@ -740,9 +739,10 @@ bool make_map(CUtensorMap* map, const GemmOperand& op, int rows, int K, int Z0, 
   return r == CUDA_SUCCESS;
 }
 
-// Map of a bf16 [rows, cols] output with two batch strides; box {64, 32}.
+// Map of a bf16 [rows, cols] output with two batch strides; box {64, 32} with 128-byte
+// swizzle, or (half) {32, 32} with 64-byte swizzle.
 bool make_out_map(CUtensorMap* map, void* ptr, int cols, int rows, long long ld, long long s0,
-                  long long s1, int Z0, int Z1) {
+                  long long s1, int Z0, int Z1, bool half = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)(s0 ? Z0 : 1),
@@ -751,10 +751,12 @@ bool make_out_map(CUtensorMap* map, void* ptr, int cols, int rows, long long ld,
   const cuuint64_t plane = ((row_bytes * dims[1]) + 15) & ~(cuuint64_t)15;
   cuuint64_t strides[3] = {row_bytes, s0 ? (cuuint64_t)s0 * 2 : plane,
                            s1 ? (cuuint64_t)s1 * 2 : plane * dims[2]};
-  cuuint32_t box[4] = {64, 32, 1, 1};  // one epilogue warp's 32 rows x 64 columns
+  // one epilogue warp's 32 rows x 64 (or 32) columns
+  cuuint32_t box[4] = {half ? 32u : 64u, 32, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            half ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -771,9 +773,13 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   memset(&om, 0, sizeof(om));
   if (MODE == EPI_SWIGLU) {
     // out2 / out3 share gemm.C's strides except for their own row stride and base
-    if (!make_out_map(&om.m[0], a.C, a.n_valid, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1) ||
-        (a.C2 && !make_out_map(&om.m[1], a.C2, a.n_valid, p.M, a.ld2, a.c2s0, a.c2s1, p.Z0, p.Z1)) ||
-        (a.C3 && !make_out_map(&om.m[2], a.C3, a.n_valid, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1))) {
+    // the gradient epilogue stores 32-column halves
+    const bool h = a.grad != 0;
+    if (!make_out_map(&om.m[0], a.C, a.n_valid, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1, h) ||
+        (a.C2 &&
+         !make_out_map(&om.m[1], a.C2, a.n_valid, p.M, a.ld2, a.c2s0, a.c2s1, p.Z0, p.Z1, h)) ||
+        (a.C3 &&
+         !make_out_map(&om.m[2], a.C3, a.n_valid, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1, h))) {
       set_error_message("gemm_umma: output tensor map encoding failed");
       return TTT_ERR_CUDA;
     }
