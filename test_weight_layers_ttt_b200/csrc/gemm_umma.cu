@@ -45,10 +45,12 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 // STORE: each lane stores its row directly (no addend, or bf16 C). STORE_STG: fp32 C with an
 // addend, staged per warp so Cin loads and C stores are row-contiguous. STORE_COPY: STORE_STG
 // plus a bf16 copy of the result. STORE_T: STORE_STG plus the result written transposed
-// (fp32), 128 contiguous bytes per store. Separate instantiations, so no mode pays for
-// another's code.
+// (fp32), 128 contiguous bytes per store. STORE_TMA: bf16 C without an addend, each warp's
+// 32 rows staged 64 columns at a time in its 4 KB box and written with TMA tensor stores.
+// Separate instantiations, so no mode pays for another's code.
 enum EpiMode : int {
-  EPI_STORE = 0, EPI_SWIGLU = 1, EPI_STORE_STG = 2, EPI_STORE_COPY = 3, EPI_STORE_T = 4
+  EPI_STORE = 0, EPI_SWIGLU = 1, EPI_STORE_STG = 2, EPI_STORE_COPY = 3, EPI_STORE_T = 4,
+  EPI_STORE_TMA = 5
 };
 
 struct UArgs {
@@ -390,7 +392,50 @@ __global__ void __launch_bounds__(THREADS, 1)
                 0 &&
             (args.ldc * (long long)sizeof(TC)) % 16 == 0 && (!ibase || args.ldi % 4 == 0);
         const int rr0 = lane >> 3, cq = (lane & 7) * 4;
-        if constexpr (MODE == EPI_STORE) {
+        if constexpr (MODE == EPI_STORE_TMA) {
+          // alpha * acc as bf16, 64 columns per TMA store from this warp's box; the
+          // accumulator is released after the last TMEM read
+          static_assert(HALF % 64 == 0, "64-column store boxes");
+          const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
+          const int oy = tc.tm * BM + quarter * 32;
+          const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
+#pragma unroll
+          for (int c0 = 0; c0 < HALF; c0 += 64) {
+            const int ox = tc.tn * BN + part * HALF + c0;
+            uint32_t ra[32], rb[32];
+            tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0), ra);
+            tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0 + 32), rb);
+            tmem_ld_wait_regs(ra, rb);
+            if (c0 + 64 >= HALF) {
+              tc_fence_before();
+              mbar_arrive(smem_u32(&acc_empty[buf]));
+            }
+            if (ox >= args.N) continue;
+            if (lane == 0) tma_store_wait_read();
+            __syncwarp();
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+              const uint32_t* v = cc < 4 ? &ra[8 * cc] : &rb[8 * (cc - 4)];
+              const uint32_t addr = box + lane * 128 + ((cc ^ (lane & 7)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                           "r"(pack_bf16x2(args.alpha * __uint_as_float(v[0]),
+                                           args.alpha * __uint_as_float(v[1]))),
+                           "r"(pack_bf16x2(args.alpha * __uint_as_float(v[2]),
+                                           args.alpha * __uint_as_float(v[3]))),
+                           "r"(pack_bf16x2(args.alpha * __uint_as_float(v[4]),
+                                           args.alpha * __uint_as_float(v[5]))),
+                           "r"(pack_bf16x2(args.alpha * __uint_as_float(v[6]),
+                                           args.alpha * __uint_as_float(v[7])))
+                           : "memory");
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_4d(&om.m[0], box, ox, oy, c2, c3);
+              tma_store_commit();
+            }
+          }
+        } else if constexpr (MODE == EPI_STORE) {
           uint32_t r[HALF];
 #pragma unroll
           for (int c0 = 0; c0 < HALF; c0 += 32)
@@ -651,7 +696,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-    if (MODE == EPI_SWIGLU && lane == 0) tma_store_wait_all();
+    if ((MODE == EPI_SWIGLU || MODE == EPI_STORE_TMA) && lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -771,6 +816,11 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
     return TTT_ERR_CUDA;
   }
   memset(&om, 0, sizeof(om));
+  if (MODE == EPI_STORE_TMA &&
+      !make_out_map(&om.m[0], a.C, p.N, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1)) {
+    set_error_message("gemm_umma: output tensor map encoding failed");
+    return TTT_ERR_CUDA;
+  }
   if (MODE == EPI_SWIGLU) {
     // out2 / out3 share gemm.C's strides except for their own row stride and base
     // the gradient epilogue stores 32-column halves
@@ -845,6 +895,15 @@ ttt_status dispatch_bn_mode(const GemmProblem& p, const UArgs& a, cudaStream_t s
 
 template <typename TC>
 ttt_status dispatch_bn(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
+  if constexpr (sizeof(TC) == 2) {
+    // bf16 C without an addend leaves through TMA stores, except where the resident B
+    // tile leaves no room for the staging boxes
+    // (256-column tiles: narrower ones keep two CTAs per SM without the boxes)
+    const bool tma_ok = !a.Cin && p.N > 128 && (reinterpret_cast<uintptr_t>(a.C) & 15) == 0 &&
+                        a.ldc % 8 == 0 && a.cs0 % 8 == 0 && a.cs1 % 8 == 0 &&
+                        !use_bres(p, 256);
+    if (tma_ok) return dispatch_major<256, 4, EPI_STORE_TMA, TC>(p, a, s);
+  }
   if constexpr (sizeof(TC) == 4) {
     // staged fp32 stores where the lanes wait for an addend, or where the output leaves L2
     // and HBM write efficiency decides (more than 64 MB)
