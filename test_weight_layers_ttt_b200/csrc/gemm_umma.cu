@@ -393,20 +393,28 @@ __global__ void __launch_bounds__(THREADS, 1)
             (args.ldc * (long long)sizeof(TC)) % 16 == 0 && (!ibase || args.ldi % 4 == 0);
         const int rr0 = lane >> 3, cq = (lane & 7) * 4;
         if constexpr (MODE == EPI_STORE_TMA) {
-          // alpha * acc as bf16, 64 columns per TMA store from this warp's box; the
-          // accumulator is released after the last TMEM read
-          static_assert(HALF % 64 == 0, "64-column store boxes");
+          // alpha * acc (bf16: 64 columns, fp32: 32 columns per 128-byte box row) per TMA
+          // store from this warp's 4 KB box; the accumulator is released after the last
+          // TMEM read
+          constexpr int PC = sizeof(TC) == 2 ? 64 : 32;   // columns per store
+          static_assert(HALF % PC == 0, "whole store boxes");
           const uint32_t box = smem_base + L::OUT_OFF + ew * 4096;
           const int oy = tc.tm * BM + quarter * 32;
           const int c2 = args.cs0 ? tc.z0 : 0, c3 = args.cs1 ? tc.z1 : 0;
 #pragma unroll
-          for (int c0 = 0; c0 < HALF; c0 += 64) {
+          for (int c0 = 0; c0 < HALF; c0 += PC) {
             const int ox = tc.tn * BN + part * HALF + c0;
             uint32_t ra[32], rb[32];
             tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0), ra);
-            tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0 + 32), rb);
-            tmem_ld_wait_regs(ra, rb);
-            if (c0 + 64 >= HALF) {
+            if constexpr (PC == 64) {
+              tmem_ld32(lane_addr + (uint32_t)(part * HALF + c0 + 32), rb);
+              tmem_ld_wait_regs(ra, rb);
+            } else {
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) asm volatile("" : "+r"(ra[j]));
+            }
+            if (c0 + PC >= HALF) {
               tc_fence_before();
               mbar_arrive(smem_u32(&acc_empty[buf]));
             }
@@ -415,17 +423,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc) {
-              const uint32_t* v = cc < 4 ? &ra[8 * cc] : &rb[8 * (cc - 4)];
               const uint32_t addr = box + lane * 128 + ((cc ^ (lane & 7)) << 4);
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                           "r"(pack_bf16x2(args.alpha * __uint_as_float(v[0]),
-                                           args.alpha * __uint_as_float(v[1]))),
-                           "r"(pack_bf16x2(args.alpha * __uint_as_float(v[2]),
-                                           args.alpha * __uint_as_float(v[3]))),
-                           "r"(pack_bf16x2(args.alpha * __uint_as_float(v[4]),
-                                           args.alpha * __uint_as_float(v[5]))),
-                           "r"(pack_bf16x2(args.alpha * __uint_as_float(v[6]),
-                                           args.alpha * __uint_as_float(v[7])))
+              uint32_t w[4];
+              if constexpr (PC == 64) {
+                const uint32_t* v = cc < 4 ? &ra[8 * cc] : &rb[8 * (cc - 4)];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  w[q] = pack_bf16x2(args.alpha * __uint_as_float(v[2 * q]),
+                                     args.alpha * __uint_as_float(v[2 * q + 1]));
+              } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  w[q] = __float_as_uint(args.alpha * __uint_as_float(ra[4 * cc + q]));
+              }
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]),
+                           "r"(w[1]), "r"(w[2]), "r"(w[3])
                            : "memory");
             }
             fence_async_smem();
@@ -785,21 +797,24 @@ bool make_map(CUtensorMap* map, const GemmOperand& op, int rows, int K, int Z0, 
 }
 
 // Map of a bf16 [rows, cols] output with two batch strides; box {64, 32} with 128-byte
-// swizzle, or (half) {32, 32} with 64-byte swizzle.
+// swizzle, or (half) {32, 32} with 64-byte swizzle; or (f32) of an fp32 output, box
+// {32, 32} with 128-byte swizzle.
 bool make_out_map(CUtensorMap* map, void* ptr, int cols, int rows, long long ld, long long s0,
-                  long long s1, int Z0, int Z1, bool half = false) {
+                  long long s1, int Z0, int Z1, bool half = false, bool f32 = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)(s0 ? Z0 : 1),
                         (cuuint64_t)(s1 ? Z1 : 1)};
-  const cuuint64_t row_bytes = (cuuint64_t)ld * 2;
+  const cuuint64_t es = f32 ? 4 : 2;
+  const cuuint64_t row_bytes = (cuuint64_t)ld * es;
   const cuuint64_t plane = ((row_bytes * dims[1]) + 15) & ~(cuuint64_t)15;
-  cuuint64_t strides[3] = {row_bytes, s0 ? (cuuint64_t)s0 * 2 : plane,
-                           s1 ? (cuuint64_t)s1 * 2 : plane * dims[2]};
+  cuuint64_t strides[3] = {row_bytes, s0 ? (cuuint64_t)s0 * es : plane,
+                           s1 ? (cuuint64_t)s1 * es : plane * dims[2]};
   // one epilogue warp's 32 rows x 64 (or 32) columns
-  cuuint32_t box[4] = {half ? 32u : 64u, 32, 1, 1};
+  cuuint32_t box[4] = {(half || f32) ? 32u : 64u, 32, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box, estr,
+  return fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+            ptr, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE,
             half ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -816,8 +831,8 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
     return TTT_ERR_CUDA;
   }
   memset(&om, 0, sizeof(om));
-  if (MODE == EPI_STORE_TMA &&
-      !make_out_map(&om.m[0], a.C, p.N, p.M, a.ldc, a.cs0, a.cs1, p.Z0, p.Z1)) {
+  if (MODE == EPI_STORE_TMA && !make_out_map(&om.m[0], a.C, p.N, p.M, a.ldc, a.cs0, a.cs1, p.Z0,
+                                             p.Z1, false, sizeof(TC) == 4)) {
     set_error_message("gemm_umma: output tensor map encoding failed");
     return TTT_ERR_CUDA;
   }
@@ -895,13 +910,14 @@ ttt_status dispatch_bn_mode(const GemmProblem& p, const UArgs& a, cudaStream_t s
 
 template <typename TC>
 ttt_status dispatch_bn(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  if constexpr (sizeof(TC) == 2) {
-    // bf16 C without an addend leaves through TMA stores, except where the resident B
-    // tile leaves no room for the staging boxes
-    // (256-column tiles: narrower ones keep two CTAs per SM without the boxes)
-    const bool tma_ok = !a.Cin && p.N > 128 && (reinterpret_cast<uintptr_t>(a.C) & 15) == 0 &&
-                        a.ldc % 8 == 0 && a.cs0 % 8 == 0 && a.cs1 % 8 == 0 &&
-                        !use_bres(p, 256);
+  {
+    // C without an addend (and without a copy) leaves through TMA stores, except where the
+    // resident B tile leaves no room for the staging boxes (256-column tiles: narrower
+    // ones keep two CTAs per SM without the boxes)
+    constexpr long long q = 16 / sizeof(TC);   // elements per 16 bytes
+    const bool tma_ok = !a.Cin && !a.C16 && p.N > 128 &&
+                        (reinterpret_cast<uintptr_t>(a.C) & 15) == 0 && a.ldc % q == 0 &&
+                        a.cs0 % q == 0 && a.cs1 % q == 0 && !use_bres(p, 256);
     if (tma_ok) return dispatch_major<256, 4, EPI_STORE_TMA, TC>(p, a, s);
   }
   if constexpr (sizeof(TC) == 4) {
