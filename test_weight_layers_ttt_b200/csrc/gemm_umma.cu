@@ -942,6 +942,9 @@ ttt_status dispatch_tf32_mode(const GemmProblem& p, const UArgs& a, cudaStream_t
 }
 ttt_status dispatch_tf32(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   if (a.Ct) return dispatch_tf32_mode<EPI_STORE_T>(p, a, s);
+  if (!a.Cin && p.N > 128 && (reinterpret_cast<uintptr_t>(a.C) & 15) == 0 && a.ldc % 4 == 0 &&
+      a.cs0 % 4 == 0 && a.cs1 % 4 == 0)
+    return launch_umma<256, false, false, 4, EPI_STORE_TMA, float, false, true>(p, a, s);
   if (a.Cin || (long long)p.M * p.N * p.Z0 * p.Z1 * 4 > (64LL << 20))
     return dispatch_tf32_mode<EPI_STORE_STG>(p, a, s);
   return dispatch_tf32_mode<EPI_STORE>(p, a, s);
