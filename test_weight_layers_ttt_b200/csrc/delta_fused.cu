@@ -81,7 +81,8 @@ template <int HD>
 __global__ void __launch_bounds__(DF_THREADS, 1)
     delta_fused_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmW,
-                       const __grid_constant__ CUtensorMap tmV, const DfArgs a) {
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmD, const DfArgs a) {
   using L = DfSmem<HD>;
   constexpr int RING = L::RING;
   constexpr int VT = L::VT;
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -330,6 +332,11 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         }
         ++p_n;
         const uint32_t box = sP + part * DF_PBLK + quarter * 4096;
+        // the previous unit's Delta S stores from this box have read it
+        if (t == 0) {
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
+        }
         swiglu_piece(ra0, rb0, sc, box, lane, 0);
         swiglu_piece(ra1, rb1, sc, box, lane, 4);
         fence_async_smem();
@@ -349,16 +356,33 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(d_empty));
-      const int mrow = walk.j * 128 + quarter * 32 + lane;
-      if (mrow < a.m) {
-        float4* dst = reinterpret_cast<float4*>(a.dS + (((long long)bh * a.C + c) * a.m + mrow) *
-                                                           HD + part * HALF);
+      // rows quarter*32 .. +31 through this warp's phi box (the unit's MMAs have all
+      // completed), 32 fp32 columns per TMA store; rows past m are clipped by the store
+      const uint32_t box = sP + part * DF_PBLK + quarter * 4096;
 #pragma unroll
-        for (int q = 0; q < HALF; q += 4)
-          dst[q / 4] = make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
-                                   __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
+      for (int c0 = 0; c0 < HALF; c0 += 32) {
+        if (c0 > 0) {
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
+        }
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint32_t addr = box + lane * 128 + ((cc ^ (lane & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "r"(r[c0 + 4 * cc]), "r"(r[c0 + 4 * cc + 1]), "r"(r[c0 + 4 * cc + 2]),
+                       "r"(r[c0 + 4 * cc + 3])
+                       : "memory");
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_4d(&tmD, box, part * HALF + c0, walk.j * 128 + quarter * 32,
+                       bh * a.C + c, 0);
+          tma_store_commit();
+        }
       }
     }
+    if (lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -409,6 +433,21 @@ bool df_map(CUtensorMap* map, const void* ptr, long long inner, long long rows, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 map of Delta S [z][m][HD], box {32, 32}, 128-byte swizzle (one warp's 32 rows x 32
+// columns per store).
+bool df_map_out(CUtensorMap* map, float* ptr, long long inner, long long rows, long long z) {
+  auto fn = df_encode();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)z, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)inner * 4, (cuuint64_t)(inner * rows * 4),
+                           (cuuint64_t)(inner * rows * z * 4)};
+  cuuint32_t box[4] = {32, 32, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int df_sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -423,9 +462,9 @@ ttt_status launch_df(const void* k, const void* v, const float* eta, const void*
                      unsigned long long wait_ns, cudaStream_t s) {
   const long long BH = (long long)B * H, C = (N + chunk - 1) / chunk;
   const long long mpad = (m + 127LL) / 128 * 128;
-  CUtensorMap mk, mw, mv;
+  CUtensorMap mk, mw, mv, md;
   if (!df_map(&mk, k, HD, N, BH, 128) || !df_map(&mw, Wk, HD, 2 * mpad, H, 256) ||
-      !df_map(&mv, v, HD, N, BH, DfSmem<HD>::VT)) {
+      !df_map(&mv, v, HD, N, BH, DfSmem<HD>::VT) || !df_map_out(&md, dS, HD, m, BH * C)) {
     set_error_message("fused state delta: cuTensorMapEncodeTiled failed");
     return TTT_ERR_CUDA;
   }
@@ -452,7 +491,7 @@ ttt_status launch_df(const void* k, const void* v, const float* eta, const void*
     set_error_message("fused state delta: cannot set %d bytes of dynamic shared memory", SMEM);
     return TTT_ERR_CUDA;
   }
-  kern<<<(unsigned)grid, DF_THREADS, SMEM, s>>>(mk, mw, mv, a);
+  kern<<<(unsigned)grid, DF_THREADS, SMEM, s>>>(mk, mw, mv, md, a);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error_message("fused state delta launch: %s", cudaGetErrorString(e));
