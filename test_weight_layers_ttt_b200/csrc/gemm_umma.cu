@@ -87,7 +87,9 @@ struct Smem {
   static constexpr int B_BYTES = BN * BK * 2;             // one k-block of B
   static constexpr int B_RES = BRES ? 4 * B_BYTES : 0;    // resident B, at most 4 k-blocks
   static constexpr int STAGE = BRES ? A_BYTES : A_BYTES + B_BYTES;
-  static constexpr int OUT_BYTES = MODE != EPI_STORE ? BM * 128 * 2 : 0;
+  // one 4 KB box per epilogue warp; STORE_T a second one for the transposed copy
+  static constexpr int OUT_BYTES =
+      MODE == EPI_STORE ? 0 : (MODE == EPI_STORE_T ? 2 : 1) * BM * 128 * 2;
   static constexpr int OUT_OFF = B_RES;
   static constexpr int RING_OFF = OUT_OFF + OUT_BYTES;
   static constexpr int BAR_OFF = RING_OFF + STAGES * STAGE;
@@ -488,6 +490,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else {
           // the accumulator is read 32 columns at a time and released after the last read
           float4* sbuf = reinterpret_cast<float4*>(smem + L::OUT_OFF + ew * 4096);
+          // STORE_T: the transposed chunk, 32 rows (chunk columns) of 32 fp32 (chunk rows),
+          // 128-byte swizzle, the layout of a TMA box {32, 32}
+          const uint32_t tbox = smem_base + L::OUT_OFF + BM * 128 * 2 + ew * 4096;
+          auto tput = [&](int c, int r, float v) {
+            const uint32_t addr =
+                tbox + c * 128 + ((((r >> 2) ^ (c & 7)) << 4) | ((r & 3) << 2));
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+          };
 #pragma unroll
           for (int c0 = 0; c0 < HALF; c0 += 32) {
             const int col0 = tc.tn * BN + part * HALF + c0;
@@ -515,6 +525,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                                   ibase + (long long)row_o * args.ldi + col)
                             : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             }
+            if constexpr (MODE == EPI_STORE_T) {
+              if (lane == 0) tma_store_wait_read();   // the previous transposed store read tbox
+            }
             __syncwarp();   // the previous chunk's staged values have been read
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -539,8 +552,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                   x[3] = fmaf(args.beta, cin[it].w, x[3]);
                 }
                 store4(crow + col, x);
-                if constexpr (MODE == EPI_STORE_T)
-                  sbuf[rr * 8 + ((cq >> 2) ^ (rr & 7))] = make_float4(x[0], x[1], x[2], x[3]);
+                if constexpr (MODE == EPI_STORE_T) {
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) tput(cq + j, rr, x[j]);
+                }
                 if constexpr (MODE == EPI_STORE_COPY) {
                   __nv_bfloat16* c16 = args.C16 + tc.z0 * args.cs0 + tc.z1 * args.cs1 +
                                        (long long)row_o * args.ldc + col;
@@ -560,24 +575,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                     args.C16[tc.z0 * args.cs0 + tc.z1 * args.cs1 + (long long)row_o * args.ldc +
                              col + j] = __float2bfloat16_rn(y);
                 }
-                if constexpr (MODE == EPI_STORE_T)
-                  sbuf[rr * 8 + ((cq >> 2) ^ (rr & 7))] = make_float4(x[0], x[1], x[2], x[3]);
+                if constexpr (MODE == EPI_STORE_T) {
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) tput(cq + j, rr, x[j]);
+                }
               }
             }
             if constexpr (MODE == EPI_STORE_T) {
-              // the chunk's final values, transposed: lane l holds row rbase + l, and each
-              // store writes one column's 32 rows (128 contiguous bytes)
+              // the chunk's final values, transposed in this warp's second box (column c of
+              // the chunk is row c of the box), leave with one TMA store
+              fence_async_smem();
               __syncwarp();
-              const int row_t = rbase + lane;
-              if (args.Ct && row_t < args.M) {
-                float* tb = args.Ct + tc.z0 * args.ts0 + tc.z1 * args.ts1 + row_t;
-                const float* sv = reinterpret_cast<const float*>(sbuf);
-#pragma unroll 8
-                for (int c = 0; c < 32; ++c) {
-                  if (col0 + c >= args.N) break;
-                  tb[(long long)(col0 + c) * args.ldt] =
-                      sv[(lane * 8 + ((c >> 2) ^ (lane & 7))) * 4 + (c & 3)];
-                }
+              if (lane == 0) {
+                tma_store_4d(&om.m[1], tbox, rbase, col0, args.ts0 ? tc.z0 : 0,
+                             args.ts1 ? tc.z1 : 0);
+                tma_store_commit();
               }
             }
             if (last) break;
@@ -708,7 +720,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-    if ((MODE == EPI_SWIGLU || MODE == EPI_STORE_TMA) && lane == 0) tma_store_wait_all();
+    if ((MODE == EPI_SWIGLU || MODE == EPI_STORE_TMA || MODE == EPI_STORE_T) && lane == 0)
+      tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -831,6 +844,11 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
     return TTT_ERR_CUDA;
   }
   memset(&om, 0, sizeof(om));
+  if (MODE == EPI_STORE_T &&
+      !make_out_map(&om.m[1], a.Ct, p.M, p.N, a.ldt, a.ts0, a.ts1, p.Z0, p.Z1, false, true)) {
+    set_error_message("gemm_umma: transposed-output tensor map encoding failed");
+    return TTT_ERR_CUDA;
+  }
   if (MODE == EPI_STORE_TMA && !make_out_map(&om.m[0], a.C, p.N, p.M, a.ldc, a.cs0, a.cs1, p.Z0,
                                              p.Z1, false, sizeof(TC) == 4)) {
     set_error_message("gemm_umma: output tensor map encoding failed");
@@ -936,7 +954,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 // for, the staged one with an addend or a large output, else direct row stores.
 template <int MODE>
 ttt_status dispatch_tf32_mode(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  if (p.N > 128) return launch_umma<256, false, false, 4, MODE, float, false, true>(p, a, s);
+  // the transposed copy's second set of boxes takes a ring stage's shared memory
+  constexpr int S256 = MODE == EPI_STORE_T ? 3 : 4;
+  if (p.N > 128) return launch_umma<256, false, false, S256, MODE, float, false, true>(p, a, s);
   if (p.N > 64) return launch_umma<128, false, false, 3, MODE, float, false, true>(p, a, s);
   return launch_umma<64, false, false, 4, MODE, float, false, true>(p, a, s);
 }
@@ -1002,8 +1022,10 @@ const char* umma_tf32_unsupported_reason(const GemmProblem& p) {
   if (p.C.dtype != DT_F32) return "tf32 products write fp32";
   if (p.beta != 0.0f && !p.Cin.ptr) return "beta != 0 needs an addend";
   if (p.C.copy16) return "no bf16 copy with tf32 operands";
-  if (p.C.t32 && (p.C.ldt < p.M || p.C.ts0 < 0 || p.C.ts1 < 0))
-    return "transposed copy needs a row stride of at least M";
+  if (p.C.t32 && (p.C.ldt < p.M || p.C.ts0 < 0 || p.C.ts1 < 0 || !aligned16(p.C.t32) ||
+                  p.C.ldt % 4 != 0 || p.C.ts0 % 4 != 0 || p.C.ts1 % 4 != 0))
+    return "transposed copy needs a 16-byte aligned base, a row stride of at least M and "
+           "strides multiples of 4";
   if (encode_fn() == nullptr) return "cuTensorMapEncodeTiled is unavailable";
   return nullptr;
 }
