@@ -370,6 +370,44 @@ __global__ void ns_sumsq_kernel(const float* U, NsLayout L, float* nrm) {
   }
 }
 
+// X (wide orientation) = U * scale and optionally Xt = X^T, 16 bytes per access: one
+// 32 x 32 tile per block of 256 threads, each thread one float4 of a tile row (rows and
+// columns multiples of 4, 16-byte aligned matrices); the transposed side goes through
+// shared memory. grid (tiles of the problem, parts, Z).
+__global__ void ns_norm4_kernel(const float* U, float* X, float* Xt, NsLayout L,
+                                const float* nrm, float eps) {
+  const int p = blockIdx.y, z = blockIdx.z;
+  if (!(L.mask & (1 << p))) return;
+  const int R = L.R[p], Cc = L.C[p];
+  const int tc = (Cc + 31) / 32, tr_ = (R + 31) / 32;
+  if ((int)blockIdx.x >= tc * tr_) return;
+  const int i0 = (blockIdx.x / tc) * 32, j0 = (blockIdx.x % tc) * 32;   // tile of U [R, Cc]
+  const long long n = (long long)R * Cc;
+  const float* u = U + z * L.zstride + p * L.pstride;
+  float* x = X + ((long long)z * L.parts + p) * n;
+  float* xt = Xt ? Xt + ((long long)z * L.parts + p) * n : nullptr;
+  const bool tr = R > Cc;
+  float* same = tr ? xt : x;     // U's orientation [R, Cc]
+  float* other = tr ? x : xt;    // the transposed one [Cc, R]
+  const float scale = 1.0f / (sqrtf(nrm[(long long)z * L.parts + p]) + eps);
+  __shared__ float t[32][33];
+  const int r = threadIdx.x >> 3, q = (threadIdx.x & 7) * 4;
+  const int i = i0 + r, j = j0 + q;
+  float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (i < R && j < Cc) {
+    v = *reinterpret_cast<const float4*>(u + (long long)i * Cc + j);
+    v.x *= scale; v.y *= scale; v.z *= scale; v.w *= scale;
+  }
+  if (same && i < R && j < Cc) *reinterpret_cast<float4*>(same + (long long)i * Cc + j) = v;
+  if (!other) return;
+  t[r][q] = v.x; t[r][q + 1] = v.y; t[r][q + 2] = v.z; t[r][q + 3] = v.w;
+  __syncthreads();
+  const int jt = j0 + r, it = i0 + q;   // row jt of the transposed side, columns it .. it + 3
+  if (jt < Cc && it < R)
+    *reinterpret_cast<float4*>(other + (long long)jt * R + it) =
+        make_float4(t[q][r], t[q + 1][r], t[q + 2][r], t[q + 3][r]);
+}
+
 // X (wide orientation) = U * scale, and optionally Xt = X^T, or U <- X back (to_u): 32 x 32
 // tiles through shared memory so every side is read and written along rows. grid (tiles of
 // the problem, parts, Z), block (32, 8).
@@ -895,8 +933,15 @@ cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, flo
   int tiles = 0;
   for (int p = 0; p < L.parts; ++p)
     tiles = max(tiles, ((L.R[p] + 31) / 32) * ((L.C[p] + 31) / 32));
-  ns_copy_kernel<<<dim3(tiles, L.parts, Z), dim3(32, 8), 0, s>>>(U, X, nullptr, L, nrm, eps, 0,
-                                                                 Xt);
+  bool vec = ((reinterpret_cast<uintptr_t>(U) | reinterpret_cast<uintptr_t>(X) |
+               reinterpret_cast<uintptr_t>(Xt)) & 15) == 0 &&
+             L.zstride % 4 == 0 && L.pstride % 4 == 0;
+  for (int p = 0; p < L.parts; ++p) vec = vec && L.R[p] % 4 == 0 && L.C[p] % 4 == 0;
+  if (vec)
+    ns_norm4_kernel<<<dim3(tiles, L.parts, Z), 256, 0, s>>>(U, X, Xt, L, nrm, eps);
+  else
+    ns_copy_kernel<<<dim3(tiles, L.parts, Z), dim3(32, 8), 0, s>>>(U, X, nullptr, L, nrm, eps, 0,
+                                                                   Xt);
   return cudaGetLastError();
 }
 

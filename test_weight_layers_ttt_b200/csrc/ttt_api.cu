@@ -681,6 +681,8 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
       o.ptr = ptr; o.dtype = DT_F32; o.mn_major = false; o.ld = ld; o.s0 = s0; o.s1 = 0;
       return o;
     };
+    // one part per entry: the last step writes U itself (no write-back pass)
+    const bool direct = L.parts == 1 && (L.mask & 1);
     for (int it = 0; it < steps; ++it) {
       GemmProblem g1;  // A = X X^T
       g1.M = (int)r; g1.N = (int)r; g1.K = (int)cc; g1.Z0 = P;
@@ -695,6 +697,25 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
       g2.C = {w.Pm, DT_F32, r, r * r, 0};
       g2.alpha = c3; g2.beta = b3; g2.Cin = {w.Ag, r, r * r, 0};
       TTT_TRY(run_tf32("ns_poly", g2, s));
+      if (direct && it == steps - 1) {
+        GemmProblem g4;
+        if (R > Cc) {  // U is [c, r]: X'^T = X^T P + a X^T (P symmetric)
+          g4.M = (int)cc; g4.N = (int)r; g4.K = (int)r; g4.Z0 = P;
+          g4.A = op(Xt, r, r * cc);
+          g4.B = op(w.Pm, r, r * r);
+          g4.C = {U, DT_F32, r, L.zstride, 0};
+          g4.Cin = {Xt, r, r * cc, 0};
+        } else {       // U is [r, c]: X' = P X + a X
+          g4.M = (int)r; g4.N = (int)cc; g4.K = (int)r; g4.Z0 = P;
+          g4.A = op(w.Pm, r, r * r);
+          g4.B = op(Xt, r, r * cc);
+          g4.C = {U, DT_F32, cc, L.zstride, 0};
+          g4.Cin = {X, cc, r * cc, 0};
+        }
+        g4.alpha = 1.0f; g4.beta = a3;
+        TTT_TRY(run_tf32("ns_apply", g4, s));
+        return TTT_OK;
+      }
       GemmProblem g3;  // X' = P X + a X, and X'^T
       g3.M = (int)r; g3.N = (int)cc; g3.K = (int)r; g3.Z0 = P;
       g3.A = op(w.Pm, r, r * r);
