@@ -135,3 +135,29 @@ def test_traffic_only_while_the_captured_source_is_unchanged():
         have = hashlib.sha256(open(f, "rb").read()).hexdigest()[:len(want)]
         assert bench._traffic(wl, kernel) == (float(value) if have == want else None)
     assert bench._traffic("lm", "no_such_kernel") is None
+
+
+def test_tf32_products_are_measured_against_the_tf32_peak():
+    """The batched Newton-Schulz GEMMs run as tf32 products: their work is one product per
+    step (not three split-bf16 terms) and their peak is the bf16 peak times the nominal
+    tf32 / bf16 ratio; the step roofline charges the Newton-Schulz FLOPs at that rate."""
+    wl = WORKLOADS["lm"]
+    r, c = min(wl.h, wl.m), max(wl.h, wl.m)
+    Z = wl.B * wl.H * wl.C
+    bound, work = bench.kernel_work("ns_apply@tcgen05", wl, "parallel_momentum")
+    assert bound == "tensor_tf32" and work == 5 * 2.0 * r * r * c * Z
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0, "source": "test"}
+    t = bench._roofline({"ns_apply@tcgen05": {"launches": 5, "ms_avg": 0.05, "share": 0.3}},
+                        wl, peaks, "parallel_momentum", 1)
+    assert t["bound"] == "tensor" and t["dtype"] == "tf32"
+    assert abs(t["peak"] - 1000.0 * 1.1 / 2.25) < 0.01
+    assert abs(t["frac"] - t["achieved"] / t["peak"]) < 1e-3
+    # the one-CTA kernel (matrices up to 128 x 256) stays a bf16 (three-term) product
+    nvs = WORKLOADS["nvs"]
+    assert bench.kernel_work("ns_mma", nvs, "recurrent")[0] == "tensor"
+    assert bench.tf32_flops(nvs, "recurrent") == 0.0
+    f = bench.layer_flops(wl, "parallel_momentum")
+    nsf = bench.tf32_flops(wl, "parallel_momentum")
+    assert 0 < nsf < f
+    s = bench.tensor_seconds(wl, "parallel_momentum", f, 1000.0)
+    assert abs(s - ((f - nsf) / 1e15 + nsf / (1e15 * 1.1 / 2.25))) < 1e-12
