@@ -619,33 +619,61 @@ __global__ void __launch_bounds__(256) rec_step_rows_kernel(float* W_all, const 
   float v[VEC ? MAXV * 4 : MAXV];
   float ss = 0.0f;
   const int n = VEC ? len / 4 : len;
+  if constexpr (VEC) {
+    // every 16-byte load of the row first (predicated, no early exit), so all of a lane's
+    // loads are in flight together; then the update
+    float4 wv[MAXV], uv[MAXV];
+    const float4 z4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const float4* usrc = reinterpret_cast<const float4*>(U ? U + off : partials + poff);
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int q = lane + 32 * i;
+      wv[i] = q < n ? reinterpret_cast<const float4*>(W_all + off)[q] : z4;
+      uv[i] = q < n ? usrc[q] : z4;
+    }
+    if (!U) {
+      for (int s2 = 1; s2 < splits; ++s2) {
+        const float4* src = reinterpret_cast<const float4*>(partials + s2 * pstride + poff);
+        float4 xv[MAXV];
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) xv[i] = lane + 32 * i < n ? src[lane + 32 * i] : z4;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) {
+          uv[i].x += xv[i].x; uv[i].y += xv[i].y; uv[i].z += xv[i].z; uv[i].w += xv[i].w;
+        }
+      }
+      if (M_all) {
+        float4 mv[MAXV];
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i)
+          mv[i] = lane + 32 * i < n ? reinterpret_cast<float4*>(M_all + off)[lane + 32 * i] : z4;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) {
+          const int q = lane + 32 * i;
+          if (q >= n) break;
+          mv[i].x = fmaf(a, mv[i].x, uv[i].x); mv[i].y = fmaf(a, mv[i].y, uv[i].y);
+          mv[i].z = fmaf(a, mv[i].z, uv[i].z); mv[i].w = fmaf(a, mv[i].w, uv[i].w);
+          reinterpret_cast<float4*>(M_all + off)[q] = mv[i];
+          uv[i] = mv[i];
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      v[4 * i] = wv[i].x - sg * uv[i].x; v[4 * i + 1] = wv[i].y - sg * uv[i].y;
+      v[4 * i + 2] = wv[i].z - sg * uv[i].z; v[4 * i + 3] = wv[i].w - sg * uv[i].w;
+      if (lane + 32 * i < n) {
+        ss = fmaf(v[4 * i], v[4 * i], ss); ss = fmaf(v[4 * i + 1], v[4 * i + 1], ss);
+        ss = fmaf(v[4 * i + 2], v[4 * i + 2], ss); ss = fmaf(v[4 * i + 3], v[4 * i + 3], ss);
+      }
+    }
+  }
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int q = lane + 32 * i;
     if (q >= n) break;
     if constexpr (VEC) {
-      const float4 w = reinterpret_cast<const float4*>(W_all + off)[q];
-      float4 u;
-      if (U) {
-        u = reinterpret_cast<const float4*>(U + off)[q];
-      } else {
-        u = reinterpret_cast<const float4*>(partials + poff)[q];
-        for (int s2 = 1; s2 < splits; ++s2) {
-          const float4 x = reinterpret_cast<const float4*>(partials + s2 * pstride + poff)[q];
-          u.x += x.x; u.y += x.y; u.z += x.z; u.w += x.w;
-        }
-        if (M_all) {
-          float4 mv = reinterpret_cast<float4*>(M_all + off)[q];
-          mv.x = fmaf(a, mv.x, u.x); mv.y = fmaf(a, mv.y, u.y);
-          mv.z = fmaf(a, mv.z, u.z); mv.w = fmaf(a, mv.w, u.w);
-          reinterpret_cast<float4*>(M_all + off)[q] = mv;
-          u = mv;
-        }
-      }
-      v[4 * i] = w.x - sg * u.x; v[4 * i + 1] = w.y - sg * u.y;
-      v[4 * i + 2] = w.z - sg * u.z; v[4 * i + 3] = w.w - sg * u.w;
-      ss = fmaf(v[4 * i], v[4 * i], ss); ss = fmaf(v[4 * i + 1], v[4 * i + 1], ss);
-      ss = fmaf(v[4 * i + 2], v[4 * i + 2], ss); ss = fmaf(v[4 * i + 3], v[4 * i + 3], ss);
+      break;   // done above
     } else {
       float u;
       if (U) {
