@@ -573,6 +573,49 @@ __global__ void sum_split_cols_kernel(const float* X, int nb, long long rows, in
   }
 }
 
+// One thread per 4 elements, chunks in order; the loads of eight chunks are issued
+// together before their updates (the chunk axis is short, the values are independent).
+// With nrm, the sum of squares of every (b, head, chunk) matrix M_c is accumulated into
+// nrm[bh * C + c] (block sums, one atomic add per block and chunk; n4 a multiple of the
+// block size, so a block never spans two (b, head) entries).
+__global__ void momentum_scan4_kernel(float4* D, const float* alpha, int BH, int C,
+                                      long long n4, float* nrm) {
+  __shared__ float red[8];
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)BH * n4) return;
+  const long long bh = idx / n4, e = idx - bh * n4;
+  float4* d = D + bh * C * n4 + e;
+  auto block_sum = [&](float v, int c) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = 0.0f;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+      atomicAdd(&nrm[bh * C + c], t);
+    }
+    __syncthreads();
+  };
+  float4 mv = d[0];
+  if (nrm) block_sum(mv.x * mv.x + mv.y * mv.y + mv.z * mv.z + mv.w * mv.w, 0);
+  for (int c0 = 1; c0 < C; c0 += 8) {
+    float4 x[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (c0 + k < C) x[k] = d[(long long)(c0 + k) * n4];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (c0 + k >= C) break;
+      const float a = alpha[bh * C + c0 + k];
+      mv.x = fmaf(a, mv.x, x[k].x); mv.y = fmaf(a, mv.y, x[k].y);
+      mv.z = fmaf(a, mv.z, x[k].z); mv.w = fmaf(a, mv.w, x[k].w);
+      d[(long long)(c0 + k) * n4] = mv;
+      if (nrm) block_sum(mv.x * mv.x + mv.y * mv.y + mv.z * mv.z + mv.w * mv.w, c0 + k);
+    }
+  }
+}
+
 // One thread per element, chunks in order (the chunk axis is short).
 __global__ void momentum_scan_kernel(float* D, const float* alpha, int BH, int C, long long n) {
   TTT_GRID_LOOP(idx, (long long)BH * n) {
@@ -953,11 +996,13 @@ cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all
 }
 
 cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
-                         float* nrm, cudaStream_t s, float* Xt) {
+                         float* nrm, cudaStream_t s, float* Xt, bool nrm_ready) {
   if (Z <= 0) return cudaSuccess;
-  cudaError_t e = fill_f32(nrm, (long long)Z * L.parts, 0.0f, s);
-  if (e != cudaSuccess) return e;
-  ns_sumsq_kernel<<<dim3(L.parts, Z, NS_SLABS), 256, 0, s>>>(U, L, nrm);
+  if (!nrm_ready) {
+    cudaError_t e = fill_f32(nrm, (long long)Z * L.parts, 0.0f, s);
+    if (e != cudaSuccess) return e;
+    ns_sumsq_kernel<<<dim3(L.parts, Z, NS_SLABS), 256, 0, s>>>(U, L, nrm);
+  }
   int tiles = 0;
   for (int p = 0; p < L.parts; ++p)
     tiles = max(tiles, ((L.R[p] + 31) / 32) * ((L.C[p] + 31) / 32));
@@ -1042,10 +1087,23 @@ cudaError_t sum_split_cols(const float* X, int nb, long long rows, int w, float*
   return cudaGetLastError();
 }
 
+bool momentum_scan_norms(int C, long long n, const float* D) {
+  return C > 1 && n % 1024 == 0 && (reinterpret_cast<uintptr_t>(D) & 15) == 0;
+}
+
 cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long n,
-                          cudaStream_t s) {
+                          cudaStream_t s, float* nrm) {
   if (BH <= 0 || C <= 1 || n <= 0) return cudaSuccess;
-  momentum_scan_kernel<<<grid_for((long long)BH * n, 256), 256, 0, s>>>(D, alpha, BH, C, n);
+  if (nrm && !momentum_scan_norms(C, n, D)) return cudaErrorInvalidValue;
+  if (nrm) {
+    cudaError_t e = fill_f32(nrm, (long long)BH * C, 0.0f, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (n % 4 == 0 && (reinterpret_cast<uintptr_t>(D) & 15) == 0)
+    momentum_scan4_kernel<<<(unsigned)(((long long)BH * n / 4 + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<float4*>(D), alpha, BH, C, n / 4, nrm);
+  else
+    momentum_scan_kernel<<<grid_for((long long)BH * n, 256), 256, 0, s>>>(D, alpha, BH, C, n);
   return cudaGetLastError();
 }
 

@@ -75,9 +75,11 @@ inline NsLayout ns_layout_single(int R, int C) {
 // Newton-Schulz set-up / tear-down for the batched paths: X = U / (||U||_F + eps) in the
 // wide orientation ([min(R,C), max(R,C)]) into the scratch X (problem (z, p) at
 // (z * parts + p) * R * C), with its transpose into Xt when Xt is not null, and U <- X back
-// in U's own orientation. Z entries. nrm: fp32 scratch of Z * parts sums of squares.
+// in U's own orientation. Z entries. nrm: fp32 scratch of Z * parts sums of squares
+// (already holding them when nrm_ready).
 cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
-                         float* nrm, cudaStream_t s, float* Xt = nullptr);
+                         float* nrm, cudaStream_t s, float* Xt = nullptr,
+                         bool nrm_ready = false);
 cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cudaStream_t s);
 
 // The whole Newton-Schulz orthogonalisation of the matrices of L on the tensor cores
@@ -112,9 +114,12 @@ cudaError_t sum_split_cols(const float* X, int nb, long long rows, int w, float*
                            float* out1, cudaStream_t s);
 
 // Momentum over chunks, in place: D[bh, c] <- alpha[bh, c] * D[bh, c - 1] + D[bh, c] for
-// c = 1 .. C-1 (D [BH, C, n] fp32, alpha [BH, C]).
+// c = 1 .. C-1 (D [BH, C, n] fp32, alpha [BH, C]). With nrm (only where
+// momentum_scan_norms holds), also nrm[bh * C + c] = the sum of squares of the result
+// D[bh, c] (the Frobenius norms the Newton-Schulz set-up needs).
+bool momentum_scan_norms(int C, long long n, const float* D);
 cudaError_t momentum_scan(float* D, const float* alpha, int BH, int C, long long n,
-                          cudaStream_t s);
+                          cudaStream_t s, float* nrm = nullptr);
 
 // One step on the output-major state, one warp per row: the update is U when given, else
 // the sum of the `splits` partials (parts ordered as for rec_reduce) with the momentum

@@ -657,7 +657,7 @@ NsScratch plan_ns(Carve& cv, int ot, long long problems, int R, int C) {
 // L: tensor cores for bf16 mode when they fit one CTA, else fp32 CUDA-core products (the
 // problems of the masked-out parts are computed and not written back).
 ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const NsScratch& w,
-                  cudaStream_t s) {
+                  cudaStream_t s, bool nrm_ready = false) {
   const float a3 = 3.4445f, b3 = -4.7750f, c3 = 2.0315f;
   const long long R = L.R[0], Cc = L.C[0];
   if (ot == DT_BF16 && ns_mma_supported((int)R, (int)Cc)) {
@@ -668,7 +668,8 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
   const long long r = R < Cc ? R : Cc, cc = R < Cc ? Cc : R;
   const int P = Z * L.parts;
   const bool tf32 = ns_path(ot, (int)R, (int)Cc) == NS_TENSOR_GEMM;
-  TTT_OP("ns_normalize", ns_normalize(U, w.X, Z, L, 1e-7f, w.nrm, s, tf32 ? w.Xt : nullptr));
+  TTT_OP("ns_normalize",
+         ns_normalize(U, w.X, Z, L, 1e-7f, w.nrm, s, tf32 ? w.Xt : nullptr, nrm_ready));
   if (tf32) {
     // Each product on the tensor cores with fp32 operands read as tf32 (10-bit mantissa,
     // fp32 accumulation in TMEM), all operands K-major: A = X X^T from X [r, c]; P = c A A +
@@ -790,10 +791,17 @@ ttt_status momentum_impl(const ttt_desc& d, const void* q, const void* k, const 
   TTT_OP("prep_weights",
          prep_wk_blocked(ot, W0, W2, b.Wk, d.H, d.H, d.h, d.m, d.w_in_layout, s));
   TTT_TRY(key_side(d, k, v, eta, b, shared_qk, s));
+  const long long hm = (long long)d.h * d.m;
+  // the Frobenius norms of the Newton-Schulz set-up come out of the momentum scan where
+  // the batched Newton-Schulz path needs them
+  const bool fuse_norms = d.momentum && d.ns_steps > 0 && mb.ns.nrm &&
+                          momentum_scan_norms((int)C, hm, b.dS);
   if (d.momentum)
-    TTT_OP("momentum_scan", momentum_scan(b.dS, alpha, (int)BH, (int)C, (long long)d.h * d.m, s));
+    TTT_OP("momentum_scan", momentum_scan(b.dS, alpha, (int)BH, (int)C, hm, s,
+                                          fuse_norms ? mb.ns.nrm : nullptr));
   if (d.ns_steps > 0)
-    TTT_TRY(run_ns(ot, b.dS, (int)(BH * C), ns_layout_single(d.m, d.h), d.ns_steps, mb.ns, s));
+    TTT_TRY(run_ns(ot, b.dS, (int)(BH * C), ns_layout_single(d.m, d.h), d.ns_steps, mb.ns, s,
+                   fuse_norms));
   TTT_TRY(chunk_states(d, b.dS, W1, S_final, b.Sc, nullptr, s));
   return query_side(d, q, b, shared_qk, out, s);
 }
