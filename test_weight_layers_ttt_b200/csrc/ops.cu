@@ -518,6 +518,37 @@ __global__ void suffix_scan_kernel(const float* dSc, const float* dS_final, OT* 
   }
 }
 
+// The same with 4 elements per thread (16-byte loads of dSc, eight chunks' loads issued
+// together; n a multiple of 4, 16-byte aligned buffers).
+template <typename OT>
+__global__ void suffix_scan4_kernel(const float4* dSc, const float4* dS_final, OT* G, float4* R0,
+                                    int BH, int C, long long n4, int order) {
+  TTT_GRID_LOOP(idx, (long long)BH * n4) {
+    const long long bh = idx / n4, e = idx - bh * n4;
+    float4 r = dS_final ? dS_final[idx] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    auto put = [&](long long o, const float4& x) {
+      OT* g = G + o * 4;
+      g[0] = from_f32<OT>(x.x); g[1] = from_f32<OT>(x.y);
+      g[2] = from_f32<OT>(x.z); g[3] = from_f32<OT>(x.w);
+    };
+    for (int c0 = C - 1; c0 >= 0; c0 -= 8) {
+      float4 x[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (c0 - k >= 0) x[k] = dSc[(bh * C + c0 - k) * n4 + e];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (c0 - k < 0) break;
+        const long long o = (bh * C + c0 - k) * n4 + e;
+        if (order == 1) put(o, r);
+        r.x += x[k].x; r.y += x[k].y; r.z += x[k].z; r.w += x[k].w;
+        if (order != 1) put(o, r);
+      }
+    }
+    R0[idx] = r;
+  }
+}
+
 // one warp per row
 template <typename OT>
 __global__ void row_grads_kernel(const float* T, const OT* v, const float* eta, float sgn,
@@ -569,6 +600,18 @@ __global__ void row_grads8_kernel(const float4* T, const uint4* v, const float* 
     }
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) deta[r] = sgn * acc;
+  }
+}
+
+__global__ void sum_batches4_kernel(const float4* X, int B, long long stride4, long long n4,
+                                    float4* out) {
+  TTT_GRID_LOOP(i, n4) {
+    float4 acc = X[i];
+    for (int b = 1; b < B; ++b) {
+      const float4 x = X[b * stride4 + i];
+      acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+    }
+    out[i] = acc;
   }
 }
 
@@ -1067,10 +1110,18 @@ cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cud
 cudaError_t suffix_scan(int ot, const float* dSc, const float* dS_final, void* G, float* R0,
                         int BH, int C, long long n, int order, cudaStream_t s) {
   if (BH <= 0 || n <= 0) return cudaSuccess;
+  const bool vec = n % 4 == 0 &&
+                   ((reinterpret_cast<uintptr_t>(dSc) | reinterpret_cast<uintptr_t>(dS_final) |
+                     reinterpret_cast<uintptr_t>(R0)) & 15) == 0;
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
-    suffix_scan_kernel<OT><<<grid_for((long long)BH * n, 256), 256, 0, s>>>(
-        dSc, dS_final, static_cast<OT*>(G), R0, BH, C, n, order);
+    if (vec)
+      suffix_scan4_kernel<OT><<<grid_for((long long)BH * n / 4, 256), 256, 0, s>>>(
+          reinterpret_cast<const float4*>(dSc), reinterpret_cast<const float4*>(dS_final),
+          static_cast<OT*>(G), reinterpret_cast<float4*>(R0), BH, C, n / 4, order);
+    else
+      suffix_scan_kernel<OT><<<grid_for((long long)BH * n, 256), 256, 0, s>>>(
+          dSc, dS_final, static_cast<OT*>(G), R0, BH, C, n, order);
     return cudaGetLastError();
   });
 }
@@ -1099,7 +1150,12 @@ cudaError_t row_grads(int ot, const float* T, const void* v, const float* eta, i
 cudaError_t sum_batches(const float* X, int B, long long stride, long long n, float* out,
                         cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  sum_batches_kernel<<<grid_for(n, 256), 256, 0, s>>>(X, B, stride, n, out);
+  if (B >= 1 && n % 4 == 0 && stride % 4 == 0 &&
+      ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(out)) & 15) == 0)
+    sum_batches4_kernel<<<grid_for(n / 4, 256), 256, 0, s>>>(
+        reinterpret_cast<const float4*>(X), B, stride / 4, n / 4, reinterpret_cast<float4*>(out));
+  else
+    sum_batches_kernel<<<grid_for(n, 256), 256, 0, s>>>(X, B, stride, n, out);
   return cudaGetLastError();
 }
 
