@@ -982,11 +982,11 @@ struct RecBufs {
   float* M_all;   // momentum, same layout
   float* U;       // update, same layout
   float* tnorm;   // initial column norms per head
-  // Two copies of the bf16/fp32 operands, alternating by chunk: the weights after update c
-  // are in copy (c + 1) % 2 (the initial weights in copy 0), so the apply of one chunk can
-  // read its copy while the next update writes the other.
-  void* Wk[2];    // [BH, 2*mpad, h] blocked [W0^T ; W2^T] operand
-  void* W1t[2];   // [BH, h, m] W1^T operand
+  // Three copies of the bf16/fp32 operands, in turn by chunk: the weights after update c
+  // are in copy (c + 1) % 3 (the initial weights in copy 0), so the apply reading one copy
+  // holds back only the update two chunks later, not the next one.
+  void* Wk[3];    // [BH, 2*mpad, h] blocked [W0^T ; W2^T] operand
+  void* W1t[3];   // [BH, h, m] W1^T operand
   void* Dv;       // [BH, chunk, m] V W1^T
   void* PE;       // [BH, chunk, 3m]: per token row E0 = d * B * silu'(A) | E2 = d * silu(A) |
                   // P = phi * eta (E0 and E2 side by side: one GEMM gives both gradients)
@@ -1024,7 +1024,8 @@ int choose_splits(const ttt_desc& d, long long L) {
 // caller's stream.
 struct SideStream {
   cudaStream_t s = nullptr;
-  cudaEvent_t gate = nullptr, applied = nullptr, joined = nullptr, feat = nullptr, g1 = nullptr;
+  cudaEvent_t gate = nullptr, joined = nullptr, feat = nullptr, g1 = nullptr;
+  cudaEvent_t applied[3] = {nullptr, nullptr, nullptr};   // by iteration % 3
   bool ok = false;
 };
 SideStream* side_stream() {
@@ -1038,7 +1039,9 @@ SideStream* side_stream() {
     tried[dev] = true;
     r.ok = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking) == cudaSuccess &&
            cudaEventCreateWithFlags(&r.gate, cudaEventDisableTiming) == cudaSuccess &&
-           cudaEventCreateWithFlags(&r.applied, cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&r.applied[0], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&r.applied[1], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&r.applied[2], cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&r.joined, cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&r.feat, cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&r.g1, cudaEventDisableTiming) == cudaSuccess;
@@ -1057,7 +1060,7 @@ size_t plan_recurrent(const ttt_desc& d, void* base, RecBufs& b) {
   b.M_all = d.momentum ? cv.take_n<float>(BH * 3 * hm) : nullptr;
   b.U = cv.take_n<float>(BH * 3 * hm);
   b.tnorm = cv.take_n<float>((long long)d.H * (2 * d.m + d.h));
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < 3; ++i) {
     b.Wk[i] = cv.take(os * BH * 2 * padded_m(d.m) * d.h);
     b.W1t[i] = cv.take(os * BH * hm);
   }
@@ -1471,13 +1474,15 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1t[0],
                               d.momentum ? M_io : nullptr, b.M_all, d.momentum, s));
   TTT_OP("prep_weights", prep_wk_blocked(ot, W0, W2, b.Wk[0], (int)BH, d.H, d.h, d.m, 0, s));
-  {  // both operand copies start from the initial weights (a matrix outside the update mask
+  {  // every operand copy starts from the initial weights (a matrix outside the update mask
      // is never rewritten)
     const size_t os = ot == DT_BF16 ? 2 : 4;
-    TTT_CUDA(cudaMemcpyAsync(b.Wk[1], b.Wk[0], os * BH * 2 * padded_m(d.m) * d.h,
-                             cudaMemcpyDeviceToDevice, s));
-    TTT_CUDA(cudaMemcpyAsync(b.W1t[1], b.W1t[0], os * BH * d.h * d.m, cudaMemcpyDeviceToDevice,
-                             s));
+    for (int i = 1; i < 3; ++i) {
+      TTT_CUDA(cudaMemcpyAsync(b.Wk[i], b.Wk[0], os * BH * 2 * padded_m(d.m) * d.h,
+                               cudaMemcpyDeviceToDevice, s));
+      TTT_CUDA(cudaMemcpyAsync(b.W1t[i], b.W1t[0], os * BH * d.h * d.m,
+                               cudaMemcpyDeviceToDevice, s));
+    }
   }
   if (d.renorm) TTT_OP("col_norms", col_norms(W0, W2, W1, d.H, d.h, d.m, b.tnorm, s));
   const long long N = d.N, L = d.chunk;
@@ -1485,7 +1490,8 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   // and the update of chunk c read the same operand copy and write disjoint buffers, so the
   // applies run on a second stream, each released by the gate event of update c (at its
   // Newton-Schulz kernel, which leaves most SMs idle, or at its start); each update waits
-  // for the apply that last read the operand copy it is about to overwrite.
+  // for the apply that last read the operand copy it is about to overwrite: with three
+  // copies, the apply enqueued two iterations earlier.
   SideStream* side = side_stream();
   const bool fork = side != nullptr && N > L;
   const bool ua = d.order == TTT_ORDER_UPDATE_APPLY;
@@ -1494,9 +1500,10 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
     int c = 0;
     for (long long t0 = 0; t0 < N; t0 += L, ++c) {
       const long long Lc = (t0 + L <= N) ? L : N - t0;
-      const int bin = c & 1, bout = (c + 1) & 1;
-      // update c writes copy bout; the apply enqueued in the previous iteration read it
-      if (fork && (ua ? c >= 2 : c >= 1)) TTT_CUDA(cudaStreamWaitEvent(s, side->applied, 0));
+      const int bin = c % 3, bout = (c + 1) % 3;
+      // update c writes copy bout; the apply enqueued two iterations earlier read it
+      if (fork && (ua ? c >= 3 : c >= 2))
+        TTT_CUDA(cudaStreamWaitEvent(s, side->applied[(c - 2) % 3], 0));
       TTT_TRY(rec_update(d, k, v, eta, alpha, c, t0, Lc, b, bin, bout, fork ? side : nullptr,
                          s));
       // the apply that reads copy bin (the weights after update c - 1): of chunk c - 1 in
@@ -1505,7 +1512,7 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
       const long long ta = ua ? t0 - L : t0, La = ua ? L : Lc;
       if (fork) TTT_CUDA(cudaStreamWaitEvent(sa, side->gate, 0));
       TTT_TRY(rec_apply(d, q, out, ta, La, b, bin, sa));
-      if (fork) TTT_CUDA(cudaEventRecord(side->applied, sa));
+      if (fork) TTT_CUDA(cudaEventRecord(side->applied[c % 3], sa));
     }
     if (ua && c > 0) {   // the last chunk's apply, after the last update
       const long long ta = (long long)(c - 1) * L;
@@ -1513,7 +1520,7 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
         TTT_CUDA(cudaEventRecord(side->gate, s));
         TTT_CUDA(cudaStreamWaitEvent(sa, side->gate, 0));
       }
-      TTT_TRY(rec_apply(d, q, out, ta, N - ta, b, c & 1, sa));
+      TTT_TRY(rec_apply(d, q, out, ta, N - ta, b, c % 3, sa));
     }
     return TTT_OK;
   };
