@@ -43,7 +43,11 @@
  * Precision: in TTT_DTYPE_BF16 mode the dense contractions take bf16 operands (q, k, v,
  * the fp32 weights rounded to bf16, the features rounded to bf16) and accumulate in
  * fp32 on the tensor cores; states, weights, momentum and all elementwise math stay
- * fp32. In TTT_DTYPE_FP32 mode every step is fp32 on the CUDA cores.
+ * fp32. Newton-Schulz, which bf16 operands would not keep within the parity tolerance,
+ * runs its products on the tensor cores at more than bf16 operand precision: as three
+ * bf16 terms hi*hi + hi*lo + lo*hi of split operands for matrices up to 128 x 256, as tf32
+ * products of the fp32 matrices (10-bit mantissa) for larger ones. In TTT_DTYPE_FP32 mode
+ * every step is fp32 on the CUDA cores.
  */
 #ifndef TTT_B200_TTT_H_
 #define TTT_B200_TTT_H_
