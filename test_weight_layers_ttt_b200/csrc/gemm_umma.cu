@@ -10,11 +10,14 @@
 //   warps 2..9         epilogue; warp w reads TMEM lanes 32*(w%4) .. +31, and warps 2-5 /
 //                      6-9 take the first / second half of the tile's columns
 // Epilogue modes:
-//   STORE   C = alpha * acc + beta * Cin (fp32 or bf16 C)
+//   STORE*  C = alpha * acc + beta * Cin (fp32 or bf16 C): lane-per-row stores, TMA stores
+//           from per-warp staging boxes (no addend), row-contiguous stores through a staged
+//           chunk (fp32 with an addend; optionally a bf16 copy, or the result also written
+//           transposed through a second box)
 //   SWIGLU  the tile's columns are [A block | B block] of the fused SwiGLU input weights;
 //           writes phi = silu(a) * b times a per-row factor (bf16), and optionally the
 //           unscaled phi to a second output; the gradient variant writes the recurrent
-//           form's pieces (phi * eta, D * silu(a), D * b * silu'(a)) instead.
+//           form's pieces (phi * eta, D * silu(a), D * b * silu'(a)) instead, in one pass.
 // tf32 operands (TF): fp32 A and B, K-major, through the same 128-byte-swizzled k-blocks
 // (32 fp32 per 128-byte row instead of 64 bf16) and tcgen05.mma kind::tf32; the shared-memory
 // layout, descriptors and byte offsets are those of the bf16 path.
@@ -77,10 +80,10 @@ struct UArgs {
 // Shared-memory layout. Streaming mode: a ring of STAGES (A tile + B tile) stages.
 // B-resident mode (BRES): the CTA's whole B tile for K <= 256 (up to four 64-wide k-blocks)
 // stays in shared memory and the ring carries only A tiles.
-// SWIGLU mode adds a 32 KB staging tile (128 rows x 128 bf16 phi columns, as two
-// 128-byte-swizzled 64-column boxes) written by the epilogue and stored with TMA; STORE
-// mode uses the same 32 KB as one 32 x 32 fp32 staging block per epilogue warp, through
-// which each warp turns its row-per-lane values into row-contiguous global stores.
+// Every mode but the lane-per-row STORE adds 32 KB of staging, one 4 KB box per epilogue
+// warp (STORE_T 64 KB, two boxes per warp): SWIGLU and STORE_TMA stage 32 rows x 64 bf16 (or
+// 32 fp32) columns and store them with TMA; STORE_STG / COPY / T stage 32 x 32 fp32 values
+// and write them back row-contiguous (STORE_T also transposed, through its second box).
 template <int BN, int STAGES, bool BRES, int MODE>
 struct Smem {
   static constexpr int A_BYTES = BM * BK * 2;
