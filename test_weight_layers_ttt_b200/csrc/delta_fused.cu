@@ -38,6 +38,10 @@ using namespace umma;
 constexpr int DF_THREADS = 320;
 constexpr int DF_STAGE = 16384;   // one ring stage: a K k-block (128 x 64) or a V stage
 constexpr int DF_PBLK = 16384;    // one 64-column block of the 128-token phi eta tile
+// At h = 256 (a 4-stage ring, too few bytes in flight to cover HBM latency) the first CTA
+// of each group pulls the K and V tiles this many tiles ahead of its own into L2 with
+// prefetch instructions. At h = 128 the 8-stage ring covers it and prefetching costs time.
+constexpr int DF_PREFETCH = 2;
 
 template <int HD>
 struct DfSmem {
@@ -54,6 +58,8 @@ struct DfSmem {
 struct DfArgs {
   int BH, H, N, m, mblocks, chunk, C, groups;
   float sign;
+  const __nv_bfloat16* kp;   // K and V [BH, N, HD], for the L2 prefetch
+  const __nv_bfloat16* vp;
   const float* eta;   // [BH, N]
   float* dS;          // [BH, C, m, HD] fp32
   unsigned* err;
@@ -308,6 +314,33 @@ __global__ void __launch_bounds__(DF_THREADS, 1)
         // this thread's token row of the tile; rows past the chunk contribute nothing
         const int row = t * 128 + quarter * 32 + lane;
         const float sc = row < Lc ? a.sign * eta_c[row] : 0.0f;
+        if (HD == 256 && walk.j == 0) {
+          // the tile DF_PREFETCH ahead: in this unit, else in the range's next unit
+          int pt = t + DF_PREFETCH, pbh = bh, pt0 = t0, pL = Lc;
+          bool have = pt < T;
+          if (!have && i + 1 < walk.count) {
+            const int np = pair + 1, nbh = np / a.C, nc = np - nbh * a.C;
+            pt -= T;
+            pbh = nbh;
+            pt0 = nc * a.chunk;
+            pL = min(a.chunk, a.N - pt0);
+            have = pt * 128 < pL;
+          }
+          if (have) {
+            // whole 128-byte lines of the tile's rows that exist: HD / 128 per thread and tensor
+            const int rows_in = min(128, pL - pt * 128);
+            const long long base = ((long long)pbh * a.N + pt0 + pt * 128) * HD;
+            const int tid = threadIdx.x - 64;   // the 256 epilogue threads
+#pragma unroll
+            for (int q = 0; q < HD / 128; ++q) {
+              const int line = tid + 256 * q;   // 64 bf16 = 128 bytes per line
+              if (line / (HD / 64) < rows_in) {
+                asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(a.kp + base + line * 64));
+                asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(a.vp + base + line * 64));
+              }
+            }
+          }
+        }
         if (!mbar_wait(smem_u32(ab_full), ab_n & 1, abort_flag, a.err, a.wait_ns)) {
           ok = false;
           break;
@@ -474,6 +507,8 @@ ttt_status launch_df(const void* k, const void* v, const float* eta, const void*
   a.sign = sign;
   a.eta = eta;
   a.dS = dS;
+  a.kp = static_cast<const __nv_bfloat16*>(k);
+  a.vp = static_cast<const __nv_bfloat16*>(v);
   a.err = err;
   a.wait_ns = wait_ns;
   // groups of mblocks CTAs (one per phi block) share the (b, head, chunk) pairs
