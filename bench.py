@@ -692,16 +692,33 @@ def run_gpu(args, rank, local, world):
         dq = {n: torch.empty_like(g[n]) for n in ("q", "k", "v", "eta")}
         hout = torch.empty(g["q"].shape, dtype=g["q"].dtype).pin_memory()
         dout = torch.empty_like(g["q"])
-        ws = layer.workspace(abi.ttt_workspace_bytes(
-            layer.parallel_desc(g["q"], g["W1"], wl.chunk, wl.order), 0), "cuda")
+        # The step as one layer call per (batch element, head), alternating between two
+        # streams: the (batch, head) problems are independent, so the host-to-device copies
+        # of one overlap the kernels and the device-to-host copy of another (the copy
+        # engines of the two directions run at the same time).
+        streams = [torch.cuda.Stream() for _ in range(2)]
+        one = lambda t, b, hh: t[b:b + 1, hh:hh + 1]
+        ws1 = [layer.workspace(abi.ttt_workspace_bytes(layer.parallel_desc(
+            one(g["q"], 0, 0), g["W1"][:1], wl.chunk, wl.order), 0), "cuda") for _ in streams]
 
         def e2e_step():
-            for n in dq:
-                dq[n].copy_(hq[n], non_blocking=True)
-            layer.la_parallel_fwd(dq["q"], dq["k"], dq["v"], dq["eta"], g["W0"], g["W2"],
-                                  g["W1"], wl.chunk, order=wl.order, return_state=False,
-                                  out=dout, ws=ws)
-            hout.copy_(dout, non_blocking=True)
+            cur = torch.cuda.current_stream()
+            for st in streams:
+                st.wait_stream(cur)
+            for i in range(wl.B * wl.H):
+                b, hh = divmod(i, wl.H)
+                st = streams[i % 2]
+                with torch.cuda.stream(st):
+                    for n in dq:
+                        one(dq[n], b, hh).copy_(one(hq[n], b, hh), non_blocking=True)
+                    layer.la_parallel_fwd(
+                        one(dq["q"], b, hh), one(dq["k"], b, hh), one(dq["v"], b, hh),
+                        one(dq["eta"], b, hh), g["W0"][hh:hh + 1], g["W2"][hh:hh + 1],
+                        g["W1"][hh:hh + 1], wl.chunk, order=wl.order, return_state=False,
+                        out=one(dout, b, hh), ws=ws1[i % 2])
+                    one(hout, b, hh).copy_(one(dout, b, hh), non_blocking=True)
+            for st in streams:
+                cur.wait_stream(st)
 
         steps = max(3, args.steps // 2)
         ms, _ = _timed(e2e_step, steps, args.warmup, world, torch)
