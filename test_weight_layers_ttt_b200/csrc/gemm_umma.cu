@@ -957,10 +957,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 // for, the staged one with an addend or a large output, else direct row stores.
 template <int MODE>
 ttt_status dispatch_tf32_mode(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  // the transposed copy's second set of boxes takes a ring stage's shared memory
-  constexpr int S256 = MODE == EPI_STORE_T ? 3 : 4;
-  if (p.N > 128) return launch_umma<256, false, false, S256, MODE, float, false, true>(p, a, s);
-  if (p.N > 64) return launch_umma<128, false, false, 3, MODE, float, false, true>(p, a, s);
+  // 128-column tiles with four ring stages: these epilogues, not the MMAs, set the pace,
+  // and the narrower tile halves each tile's epilogue and doubles the tile count (a fuller
+  // last wave). Faster than 256 columns (three or four stages) and than five or six stages.
+  if (p.N > 64) return launch_umma<128, false, false, 4, MODE, float, false, true>(p, a, s);
   return launch_umma<64, false, false, 4, MODE, float, false, true>(p, a, s);
 }
 ttt_status dispatch_tf32(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
