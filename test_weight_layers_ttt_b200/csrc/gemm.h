@@ -29,11 +29,6 @@ struct GemmOut {
   // fp32 C on the tensor-core engine only: a bf16 copy of the result with C's element
   // strides (e.g. the operand copy of a state kept in fp32), or null
   void* copy16 = nullptr;
-  // fp32 C on the tensor-core engine only: the result also written transposed,
-  // t32[z0 * ts0 + z1 * ts1 + j * ldt + i] = C[z](i, j) (the K-major copy of an operand
-  // that the next product reads the other way round), or null
-  float* t32 = nullptr;
-  long long ldt = 0, ts0 = 0, ts1 = 0;
 };
 
 struct GemmCin {
@@ -61,7 +56,7 @@ const char* umma_unsupported_reason(const GemmProblem& p);
 ttt_status gemm_umma(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,
                      unsigned long long wait_ns);
 // The same engine with fp32 A and B consumed as tf32 (tcgen05.mma kind::tf32: operands
-// rounded toward zero to a 10-bit mantissa, fp32 accumulation); both operands K-major, fp32
+// rounded toward zero to a 10-bit mantissa, fp32 accumulation); either major, fp32
 // C. For bf16-mode products that need more than bf16 operand precision.
 const char* umma_tf32_unsupported_reason(const GemmProblem& p);
 ttt_status gemm_umma_tf32(const GemmProblem& p, cudaStream_t stream, unsigned* dev_err,

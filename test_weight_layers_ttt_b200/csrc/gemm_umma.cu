@@ -12,15 +12,14 @@
 // Epilogue modes:
 //   STORE*  C = alpha * acc + beta * Cin (fp32 or bf16 C): lane-per-row stores, TMA stores
 //           from per-warp staging boxes (no addend), row-contiguous stores through a staged
-//           chunk (fp32 with an addend; optionally a bf16 copy, or the result also written
-//           transposed through a second box)
+//           chunk (fp32 with an addend; optionally a bf16 copy)
 //   SWIGLU  the tile's columns are [A block | B block] of the fused SwiGLU input weights;
 //           writes phi = silu(a) * b times a per-row factor (bf16), and optionally the
 //           unscaled phi to a second output; the gradient variant writes the recurrent
 //           form's pieces (phi * eta, D * silu(a), D * b * silu'(a)) instead, in one pass.
-// tf32 operands (TF): fp32 A and B, K-major, through the same 128-byte-swizzled k-blocks
-// (32 fp32 per 128-byte row instead of 64 bf16) and tcgen05.mma kind::tf32; the shared-memory
-// layout, descriptors and byte offsets are those of the bf16 path.
+// tf32 operands (TF): fp32 A and B through the same 128-byte-swizzled k-blocks (K-major: 32
+// fp32 of K per 128-byte row instead of 64 bf16; MN-major: 32-element MN blocks of 32 k rows,
+// 4 KB apart, in the 128-byte swizzle on 32-byte chunks) and tcgen05.mma kind::tf32.
 // Every mbarrier wait is bounded; a timeout records DEVERR_TIMEOUT in the device error
 // word, raises a CTA-wide abort flag, and the CTA drains its in-flight copies and MMAs
 // (again with bounded waits) and frees its TMEM before returning.
@@ -52,8 +51,7 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 // 32 rows staged 64 columns at a time in its 4 KB box and written with TMA tensor stores.
 // Separate instantiations, so no mode pays for another's code.
 enum EpiMode : int {
-  EPI_STORE = 0, EPI_SWIGLU = 1, EPI_STORE_STG = 2, EPI_STORE_COPY = 3, EPI_STORE_T = 4,
-  EPI_STORE_TMA = 5
+  EPI_STORE = 0, EPI_SWIGLU = 1, EPI_STORE_STG = 2, EPI_STORE_COPY = 3, EPI_STORE_TMA = 5
 };
 
 struct UArgs {
@@ -61,7 +59,6 @@ struct UArgs {
   int a_b0, a_b1, b_b0, b_b1;  // 1 = operand uses that batch coordinate
   void* C; long long ldc, cs0, cs1;
   __nv_bfloat16* C16;   // fp32 C: bf16 copy with C's strides, or null
-  float* Ct; long long ldt, ts0, ts1;   // fp32 C: transposed copy (EPI_STORE_T)
   const float* Cin; long long ldi, is0, is1;
   float alpha, beta;
   // SWIGLU: phi columns < n_valid are written; row factor rs[z0*rs0 + z1*rs1 + row]
@@ -81,9 +78,8 @@ struct UArgs {
 // B-resident mode (BRES): the CTA's whole B tile for K <= 256 (up to four 64-wide k-blocks)
 // stays in shared memory and the ring carries only A tiles.
 // Every mode but the lane-per-row STORE adds 32 KB of staging, one 4 KB box per epilogue
-// warp (STORE_T 64 KB, two boxes per warp): SWIGLU and STORE_TMA stage 32 rows x 64 bf16 (or
-// 32 fp32) columns and store them with TMA; STORE_STG / COPY / T stage 32 x 32 fp32 values
-// and write them back row-contiguous (STORE_T also transposed, through its second box).
+// warp: SWIGLU and STORE_TMA stage 32 rows x 64 bf16 (or 32 fp32) columns and store them
+// with TMA; STORE_STG / COPY stage 32 x 32 fp32 values and write them back row-contiguous.
 template <int BN, int STAGES, bool BRES, int MODE>
 struct Smem {
   static constexpr int A_BYTES = BM * BK * 2;
@@ -92,7 +88,7 @@ struct Smem {
   static constexpr int STAGE = BRES ? A_BYTES : A_BYTES + B_BYTES;
   // one 4 KB box per epilogue warp; STORE_T a second one for the transposed copy
   static constexpr int OUT_BYTES =
-      MODE == EPI_STORE ? 0 : (MODE == EPI_STORE_T ? 2 : 1) * BM * 128 * 2;
+      MODE == EPI_STORE ? 0 : BM * 128 * 2;
   static constexpr int OUT_OFF = B_RES;
   static constexpr int RING_OFF = OUT_OFF + OUT_BYTES;
   static constexpr int BAR_OFF = RING_OFF + STAGES * STAGE;
@@ -190,8 +186,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ OutMaps om, const UArgs args) {
-  static_assert(!TF || (!A_MN && !B_MN && !BRES && MODE != EPI_SWIGLU),
-                "tf32 operands: K-major, streamed, plain epilogues");
+  static_assert(!TF || (!BRES && MODE != EPI_SWIGLU),
+                "tf32 operands: streamed operands, plain epilogues");
   constexpr int BKE = TF ? 32 : BK;      // K elements per 128-byte k-block row
   using L = Smem<BN, STAGES, BRES, MODE>;
   constexpr uint32_t ACC_COLS = 2 * BN;  // two accumulators
@@ -261,8 +257,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int kB = kb * BKE;
             if (B_MN) {
 #pragma unroll
-              for (int q = 0; q < BN / 64; ++q)
-                tma_load_4d(sB + q * 8192, &tmB, bb, tc.tn * BN + 64 * q, kB, bc2, bc3);
+              for (int q = 0; q < BN / BKE; ++q)
+                tma_load_4d(sB + q * BKE * 128, &tmB, bb, tc.tn * BN + BKE * q, kB, bc2, bc3);
             } else {
               tma_load_4d(sB, &tmB, bb, kB, tc.tn * BN, bc2, bc3);
             }
@@ -284,8 +280,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t sA = ring_base + s * L::STAGE;
           const int kA = kb * BKE;
           if (A_MN) {
-            tma_load_4d(sA, &tmA, fb, tc.tm * BM, kA, ac2, ac3);
-            tma_load_4d(sA + 8192, &tmA, fb, tc.tm * BM + 64, kA, ac2, ac3);
+            // MN-major: BM / BKE blocks of BKE MN elements (128 bytes) x BKE k rows
+#pragma unroll
+            for (int q = 0; q < BM / BKE; ++q)
+              tma_load_4d(sA + q * BKE * 128, &tmA, fb, tc.tm * BM + BKE * q, kA, ac2, ac3);
           } else {
             tma_load_4d(sA, &tmA, fb, kA, tc.tm * BM, ac2, ac3);
           }
@@ -294,8 +292,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int kB = kb * BKE;
             if (B_MN) {
 #pragma unroll
-              for (int q = 0; q < BN / 64; ++q)
-                tma_load_4d(sB + q * 8192, &tmB, fb, tc.tn * BN + 64 * q, kB, bc2, bc3);
+              for (int q = 0; q < BN / BKE; ++q)
+                tma_load_4d(sB + q * BKE * 128, &tmB, fb, tc.tn * BN + BKE * q, kB, bc2, bc3);
             } else {
               tma_load_4d(sB, &tmB, fb, kB, tc.tn * BN, bc2, bc3);
             }
@@ -307,7 +305,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t IDESC = TF ? make_idesc_tf32(BM, BN) : make_idesc_bf16(BM, BN, A_MN, B_MN);
+      constexpr uint32_t IDESC =
+          TF ? make_idesc_tf32(BM, BN, A_MN, B_MN) : make_idesc_bf16(BM, BN, A_MN, B_MN);
       uint32_t it = 0;
       int bkey = -1, b_uses = 0;
       bool ok = true;
@@ -345,10 +344,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t sB = BRES ? smem_base + kb * L::B_BYTES : sA + L::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = A_MN ? make_sw128_desc(sA + kk * 2048, 8192, 1024)
-                                     : make_sw128_desc(sA + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? make_sw128_desc(sB + kk * 2048, 8192, 1024)
-                                     : make_sw128_desc(sB + kk * 32, 16, 1024);
+            // one instruction covers 32 bytes of K: K-major, 32 bytes along the row; MN-major,
+            // 16 (bf16) or 8 (tf32) k rows of 128 bytes, MN blocks BKE * 128 bytes apart
+            // (tf32: the 32-byte-base swizzle, 4-row groups 512 bytes apart)
+            auto mn_desc = [&](uint32_t base) {
+              return TF ? make_sw128b32_desc(base + kk * 1024, BKE * 128, 512)
+                        : make_sw128_desc(base + kk * 2048, BKE * 128, 1024);
+            };
+            const uint64_t ad = A_MN ? mn_desc(sA) : make_sw128_desc(sA + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? mn_desc(sB) : make_sw128_desc(sB + kk * 32, 16, 1024);
             if constexpr (TF)
               mma_tf32(dt, ad, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
             else
@@ -493,14 +497,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else {
           // the accumulator is read 32 columns at a time and released after the last read
           float4* sbuf = reinterpret_cast<float4*>(smem + L::OUT_OFF + ew * 4096);
-          // STORE_T: the transposed chunk, 32 rows (chunk columns) of 32 fp32 (chunk rows),
-          // 128-byte swizzle, the layout of a TMA box {32, 32}
-          const uint32_t tbox = smem_base + L::OUT_OFF + BM * 128 * 2 + ew * 4096;
-          auto tput = [&](int c, int r, float v) {
-            const uint32_t addr =
-                tbox + c * 128 + ((((r >> 2) ^ (c & 7)) << 4) | ((r & 3) << 2));
-            asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-          };
 #pragma unroll
           for (int c0 = 0; c0 < HALF; c0 += 32) {
             const int col0 = tc.tn * BN + part * HALF + c0;
@@ -528,9 +524,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                                   ibase + (long long)row_o * args.ldi + col)
                             : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             }
-            if constexpr (MODE == EPI_STORE_T) {
-              if (lane == 0) tma_store_wait_read();   // the previous transposed store read tbox
-            }
             __syncwarp();   // the previous chunk's staged values have been read
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -555,10 +548,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                   x[3] = fmaf(args.beta, cin[it].w, x[3]);
                 }
                 store4(crow + col, x);
-                if constexpr (MODE == EPI_STORE_T) {
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) tput(cq + j, rr, x[j]);
-                }
                 if constexpr (MODE == EPI_STORE_COPY) {
                   __nv_bfloat16* c16 = args.C16 + tc.z0 * args.cs0 + tc.z1 * args.cs1 +
                                        (long long)row_o * args.ldc + col;
@@ -578,21 +567,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     args.C16[tc.z0 * args.cs0 + tc.z1 * args.cs1 + (long long)row_o * args.ldc +
                              col + j] = __float2bfloat16_rn(y);
                 }
-                if constexpr (MODE == EPI_STORE_T) {
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) tput(cq + j, rr, x[j]);
-                }
-              }
-            }
-            if constexpr (MODE == EPI_STORE_T) {
-              // the chunk's final values, transposed in this warp's second box (column c of
-              // the chunk is row c of the box), leave with one TMA store
-              fence_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_4d(&om.m[1], tbox, rbase, col0, args.ts0 ? tc.z0 : 0,
-                             args.ts1 ? tc.z1 : 0);
-                tma_store_commit();
               }
             }
             if (last) break;
@@ -723,7 +697,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-    if ((MODE == EPI_SWIGLU || MODE == EPI_STORE_TMA || MODE == EPI_STORE_T) && lane == 0)
+    if ((MODE == EPI_SWIGLU || MODE == EPI_STORE_TMA) && lane == 0)
       tma_store_wait_all();
   }
 
@@ -802,12 +776,15 @@ bool make_map(CUtensorMap* map, const GemmOperand& op, int rows, int K, int Z0, 
   strides[1] = op.s0 ? (cuuint64_t)op.s0 * es : plane;
   strides[2] = op.s1 ? (cuuint64_t)op.s1 * es : plane * dims[2];
   box[0] = tf32 ? 32 : 64;
-  box[1] = (cuuint32_t)(mn ? 64 : box_rows);
+  box[1] = (cuuint32_t)(mn ? (tf32 ? 32 : 64) : box_rows);   // MN-major: one k-block of rows
   box[2] = 1;
   box[3] = 1;
+  // MN-major tf32 operands: the 128-byte swizzle on 32-byte chunks, their only UMMA layout
+  const CUtensorMapSwizzle sw =
+      (tf32 && mn) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = fn(map, tf32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                   4, const_cast<void*>(op.ptr), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -847,11 +824,6 @@ ttt_status launch_umma(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
     return TTT_ERR_CUDA;
   }
   memset(&om, 0, sizeof(om));
-  if (MODE == EPI_STORE_T &&
-      !make_out_map(&om.m[1], a.Ct, p.M, p.N, a.ldt, a.ts0, a.ts1, p.Z0, p.Z1, false, true)) {
-    set_error_message("gemm_umma: transposed-output tensor map encoding failed");
-    return TTT_ERR_CUDA;
-  }
   if (MODE == EPI_STORE_TMA && !make_out_map(&om.m[0], a.C, p.N, p.M, a.ldc, a.cs0, a.cs1, p.Z0,
                                              p.Z1, false, sizeof(TC) == 4)) {
     set_error_message("gemm_umma: output tensor map encoding failed");
@@ -953,21 +925,29 @@ ttt_status dispatch_bn(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// tf32 operands: streamed K-major operands, fp32 C; the transposed-copy epilogue when asked
-// for, the staged one with an addend or a large output, else direct row stores.
+// tf32 operands: streamed operands of either major, fp32 C; TMA stores without an addend,
+// the staged epilogue with an addend or a large output, else direct row stores.
+template <int BN, int STAGES, int MODE>
+ttt_status launch_tf32(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
+  switch ((p.A.mn_major ? 2 : 0) | (p.B.mn_major ? 1 : 0)) {
+    case 0: return launch_umma<BN, false, false, STAGES, MODE, float, false, true>(p, a, s);
+    case 1: return launch_umma<BN, false, true, STAGES, MODE, float, false, true>(p, a, s);
+    case 2: return launch_umma<BN, true, false, STAGES, MODE, float, false, true>(p, a, s);
+    default: return launch_umma<BN, true, true, STAGES, MODE, float, false, true>(p, a, s);
+  }
+}
 template <int MODE>
 ttt_status dispatch_tf32_mode(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
   // 128-column tiles with four ring stages: these epilogues, not the MMAs, set the pace,
   // and the narrower tile halves each tile's epilogue and doubles the tile count (a fuller
   // last wave). Faster than 256 columns (three or four stages) and than five or six stages.
-  if (p.N > 64) return launch_umma<128, false, false, 4, MODE, float, false, true>(p, a, s);
-  return launch_umma<64, false, false, 4, MODE, float, false, true>(p, a, s);
+  if (p.N > 64) return launch_tf32<128, 4, MODE>(p, a, s);
+  return launch_tf32<64, 4, MODE>(p, a, s);
 }
 ttt_status dispatch_tf32(const GemmProblem& p, const UArgs& a, cudaStream_t s) {
-  if (a.Ct) return dispatch_tf32_mode<EPI_STORE_T>(p, a, s);
   if (!a.Cin && p.N > 128 && (reinterpret_cast<uintptr_t>(a.C) & 15) == 0 && a.ldc % 4 == 0 &&
       a.cs0 % 4 == 0 && a.cs1 % 4 == 0)
-    return launch_umma<256, false, false, 4, EPI_STORE_TMA, float, false, true>(p, a, s);
+    return launch_tf32<256, 4, EPI_STORE_TMA>(p, a, s);
   if (a.Cin || (long long)p.M * p.N * p.Z0 * p.Z1 * 4 > (64LL << 20))
     return dispatch_tf32_mode<EPI_STORE_STG>(p, a, s);
   return dispatch_tf32_mode<EPI_STORE>(p, a, s);
@@ -979,7 +959,6 @@ UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait
   a.a_b0 = p.A.s0 != 0; a.a_b1 = p.A.s1 != 0; a.b_b0 = p.B.s0 != 0; a.b_b1 = p.B.s1 != 0;
   a.C = p.C.ptr; a.ldc = p.C.ld; a.cs0 = p.C.s0; a.cs1 = p.C.s1;
   a.C16 = static_cast<__nv_bfloat16*>(p.C.copy16);
-  a.Ct = p.C.t32; a.ldt = p.C.ldt; a.ts0 = p.C.ts0; a.ts1 = p.C.ts1;
   a.Cin = p.beta != 0.0f ? p.Cin.ptr : nullptr;
   a.ldi = p.Cin.ld; a.is0 = p.Cin.s0; a.is1 = p.Cin.s1;
   a.alpha = p.alpha; a.beta = p.beta;
@@ -1005,7 +984,6 @@ const char* umma_unsupported_reason(const GemmProblem& p) {
   if (p.C.copy16 && (p.C.dtype != DT_F32 || !aligned16(p.C.copy16) || !aligned16(p.C.ptr) ||
                      p.C.ld % 4 != 0 || p.C.s0 % 4 != 0 || p.C.s1 % 4 != 0))
     return "a bf16 copy needs an fp32 result with 16-byte aligned bases, strides multiples of 4";
-  if (p.C.t32) return "a transposed copy is written only with tf32 operands";
   if (encode_fn() == nullptr) return "cuTensorMapEncodeTiled is unavailable";
   return nullptr;
 }
@@ -1013,7 +991,6 @@ const char* umma_unsupported_reason(const GemmProblem& p) {
 const char* umma_tf32_unsupported_reason(const GemmProblem& p) {
   for (const GemmOperand* o : {&p.A, &p.B}) {
     if (o->dtype != DT_F32) return "tf32 operands must be fp32";
-    if (o->mn_major) return "tf32 operands must be K-major";
     if (!o->ptr || !aligned16(o->ptr)) return "operand base must be 16-byte aligned";
     if (o->ld <= 0 || o->ld % 4 != 0) return "operand row stride must be a multiple of 4";
     if (o->s0 < 0 || o->s1 < 0 || o->s0 % 4 != 0 || o->s1 % 4 != 0)
@@ -1025,10 +1002,6 @@ const char* umma_tf32_unsupported_reason(const GemmProblem& p) {
   if (p.C.dtype != DT_F32) return "tf32 products write fp32";
   if (p.beta != 0.0f && !p.Cin.ptr) return "beta != 0 needs an addend";
   if (p.C.copy16) return "no bf16 copy with tf32 operands";
-  if (p.C.t32 && (p.C.ldt < p.M || p.C.ts0 < 0 || p.C.ts1 < 0 || !aligned16(p.C.t32) ||
-                  p.C.ldt % 4 != 0 || p.C.ts0 % 4 != 0 || p.C.ts1 % 4 != 0))
-    return "transposed copy needs a 16-byte aligned base, a row stride of at least M and "
-           "strides multiples of 4";
   if (encode_fn() == nullptr) return "cuTensorMapEncodeTiled is unavailable";
   return nullptr;
 }

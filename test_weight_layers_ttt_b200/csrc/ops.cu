@@ -370,10 +370,10 @@ __global__ void ns_sumsq_kernel(const float* U, NsLayout L, float* nrm) {
   }
 }
 
-// X (wide orientation) = U * scale and optionally Xt = X^T, 16 bytes per access: one
-// 32 x 32 tile per block of 256 threads, each thread one float4 of a tile row (rows and
-// columns multiples of 4, 16-byte aligned matrices); the transposed side goes through
-// shared memory. grid (tiles of the problem, parts, Z).
+// X (wide orientation) = U * scale and / or Xt = X^T (either may be null), 16 bytes per
+// access: one 32 x 32 tile per block of 256 threads, each thread one float4 of a tile row
+// (rows and columns multiples of 4, 16-byte aligned matrices); the transposed side goes
+// through shared memory. grid (tiles of the problem, parts, Z).
 __global__ void ns_norm4_kernel(const float* U, float* X, float* Xt, NsLayout L,
                                 const float* nrm, float eps) {
   const int p = blockIdx.y, z = blockIdx.z;
@@ -384,7 +384,7 @@ __global__ void ns_norm4_kernel(const float* U, float* X, float* Xt, NsLayout L,
   const int i0 = (blockIdx.x / tc) * 32, j0 = (blockIdx.x % tc) * 32;   // tile of U [R, Cc]
   const long long n = (long long)R * Cc;
   const float* u = U + z * L.zstride + p * L.pstride;
-  float* x = X + ((long long)z * L.parts + p) * n;
+  float* x = X ? X + ((long long)z * L.parts + p) * n : nullptr;
   float* xt = Xt ? Xt + ((long long)z * L.parts + p) * n : nullptr;
   const bool tr = R > Cc;
   float* same = tr ? xt : x;     // U's orientation [R, Cc]
@@ -408,9 +408,9 @@ __global__ void ns_norm4_kernel(const float* U, float* X, float* Xt, NsLayout L,
         make_float4(t[q][r], t[q + 1][r], t[q + 2][r], t[q + 3][r]);
 }
 
-// X (wide orientation) = U * scale, and optionally Xt = X^T, or U <- X back (to_u): 32 x 32
-// tiles through shared memory so every side is read and written along rows. grid (tiles of
-// the problem, parts, Z), block (32, 8).
+// X (wide orientation) = U * scale and / or Xt = X^T (either may be null), or U <- X back
+// (to_u): 32 x 32 tiles through shared memory so every side is read and written along rows.
+// grid (tiles of the problem, parts, Z), block (32, 8).
 __global__ void ns_copy_kernel(const float* U_in, float* X, float* U_out, NsLayout L,
                                const float* nrm, float eps, int to_u, float* Xt) {
   const int p = blockIdx.y, z = blockIdx.z;
@@ -421,7 +421,7 @@ __global__ void ns_copy_kernel(const float* U_in, float* X, float* U_out, NsLayo
   const int i0 = (blockIdx.x / tc) * 32, j0 = (blockIdx.x % tc) * 32;   // tile of U [R, Cc]
   const long long n = (long long)R * Cc;
   const long long uoff = z * L.zstride + p * L.pstride;
-  float* x = X + ((long long)z * L.parts + p) * n;
+  float* x = X ? X + ((long long)z * L.parts + p) * n : nullptr;
   const bool tr = R > Cc;
   __shared__ float t[32][33];
   const int tx = threadIdx.x, ty = threadIdx.y;

@@ -74,7 +74,8 @@ inline NsLayout ns_layout_single(int R, int C) {
 
 // Newton-Schulz set-up / tear-down for the batched paths: X = U / (||U||_F + eps) in the
 // wide orientation ([min(R,C), max(R,C)]) into the scratch X (problem (z, p) at
-// (z * parts + p) * R * C), with its transpose into Xt when Xt is not null, and U <- X back
+// (z * parts + p) * R * C), with its transpose into Xt; either may be null (X null and Xt
+// set: the scaled matrix in U's own orientation when R > C), and U <- X back
 // in U's own orientation. Z entries. nrm: fp32 scratch of Z * parts sums of squares
 // (already holding them when nrm_ready).
 cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,

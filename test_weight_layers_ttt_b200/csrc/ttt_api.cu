@@ -620,12 +620,11 @@ ttt_status linear_impl(const ttt_desc& d, const void* q, const void* k, const vo
 // per matrix with split bf16 operands when it fits, else batched GEMMs on tf32 operands;
 // fp32 mode uses fp32 CUDA-core products.
 
-// Newton-Schulz scratch. CUDA-core path: X, X2 [problems, r, c], Ag, Pm [problems, r, r]
-// fp32. tf32 GEMM path: the same, plus the transposes Xt, X2t [problems, c, r] (the K-major
-// form of X as the right operand of P X). The one-CTA path needs none of them.
+// Newton-Schulz scratch of the batched paths (CUDA cores, tf32 GEMMs): X, X2 [problems,
+// r, c] (or [c, r]), Ag, Pm [problems, r, r] fp32 and the squared norms. The one-CTA path
+// needs none of them.
 struct NsScratch {
   float *X = nullptr, *X2 = nullptr, *Ag = nullptr, *Pm = nullptr, *nrm = nullptr;
-  float *Xt = nullptr, *X2t = nullptr;
 };
 
 enum NsPath { NS_TENSOR_CTA = 0, NS_TENSOR_GEMM = 1, NS_CUDA_CORES = 2 };
@@ -646,10 +645,6 @@ NsScratch plan_ns(Carve& cv, int ot, long long problems, int R, int C) {
   w.Ag = cv.take_n<float>(problems * r * r);
   w.Pm = cv.take_n<float>(problems * r * r);
   w.nrm = cv.take_n<float>(problems);
-  if (path == NS_TENSOR_GEMM) {
-    w.Xt = cv.take_n<float>(problems * r * c);
-    w.X2t = cv.take_n<float>(problems * r * c);
-  }
   return w;
 }
 
@@ -668,69 +663,62 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
   const long long r = R < Cc ? R : Cc, cc = R < Cc ? Cc : R;
   const int P = Z * L.parts;
   const bool tf32 = ns_path(ot, (int)R, (int)Cc) == NS_TENSOR_GEMM;
-  TTT_OP("ns_normalize",
-         ns_normalize(U, w.X, Z, L, 1e-7f, w.nrm, s, tf32 ? w.Xt : nullptr, nrm_ready));
   if (tf32) {
     // Each product on the tensor cores with fp32 operands read as tf32 (10-bit mantissa,
-    // fp32 accumulation in TMEM), all operands K-major: A = X X^T from X [r, c]; P = c A A +
-    // b A from A (symmetric, so it serves as its own K-major right operand); X' = P X + a X
-    // with X's transpose [c, r] as the right operand, and X'^T written by the same epilogue
-    // for the next step.
-    float *X = w.X, *X2 = w.X2, *Xt = w.Xt, *X2t = w.X2t;
-    auto op = [](const float* ptr, long long ld, long long s0) {
+    // fp32 accumulation in TMEM). One matrix per entry with R > C ("tall"): the iteration
+    // runs on Y = X^T in U's own orientation [c, r], A = Y^T Y (both operands MN-major),
+    // Y' = Y P + a Y (P symmetric, so it serves as its own K-major right operand), and the
+    // last step writes U. Otherwise on X [r, c] in the wide orientation: A = X X^T (both
+    // K-major), X' = P X + a X with X as an MN-major right operand, and the last step writes
+    // U when it has that orientation, else a write-back pass transposes the parts back.
+    // Either way P = c A A + b A from A (symmetric, K-major both sides).
+    const bool tall = L.parts == 1 && R > Cc;
+    TTT_OP("ns_normalize", ns_normalize(U, tall ? nullptr : w.X, Z, L, 1e-7f, w.nrm, s,
+                                        tall ? w.X : nullptr, nrm_ready));
+    float *X = w.X, *X2 = w.X2;
+    auto op = [](const float* ptr, bool mn, long long ld, long long s0) {
       GemmOperand o;
-      o.ptr = ptr; o.dtype = DT_F32; o.mn_major = false; o.ld = ld; o.s0 = s0; o.s1 = 0;
+      o.ptr = ptr; o.dtype = DT_F32; o.mn_major = mn; o.ld = ld; o.s0 = s0; o.s1 = 0;
       return o;
     };
-    // one part per entry: the last step writes U itself (no write-back pass)
+    const long long ldx = tall ? r : cc;   // row stride of X (or Y)
     const bool direct = L.parts == 1 && (L.mask & 1);
     for (int it = 0; it < steps; ++it) {
-      GemmProblem g1;  // A = X X^T
+      GemmProblem g1;  // A = X X^T (= Y^T Y)
       g1.M = (int)r; g1.N = (int)r; g1.K = (int)cc; g1.Z0 = P;
-      g1.A = op(X, cc, r * cc);
-      g1.B = op(X, cc, r * cc);
+      g1.A = op(X, tall, ldx, r * cc);
+      g1.B = op(X, tall, ldx, r * cc);
       g1.C = {w.Ag, DT_F32, r, r * r, 0};
       TTT_TRY(run_tf32("ns_gram", g1, s));
       GemmProblem g2;  // P = c A A + b A
       g2.M = (int)r; g2.N = (int)r; g2.K = (int)r; g2.Z0 = P;
-      g2.A = op(w.Ag, r, r * r);
-      g2.B = op(w.Ag, r, r * r);
+      g2.A = op(w.Ag, false, r, r * r);
+      g2.B = op(w.Ag, false, r, r * r);
       g2.C = {w.Pm, DT_F32, r, r * r, 0};
       g2.alpha = c3; g2.beta = b3; g2.Cin = {w.Ag, r, r * r, 0};
       TTT_TRY(run_tf32("ns_poly", g2, s));
-      if (direct && it == steps - 1) {
-        GemmProblem g4;
-        if (R > Cc) {  // U is [c, r]: X'^T = X^T P + a X^T (P symmetric)
-          g4.M = (int)cc; g4.N = (int)r; g4.K = (int)r; g4.Z0 = P;
-          g4.A = op(Xt, r, r * cc);
-          g4.B = op(w.Pm, r, r * r);
-          g4.C = {U, DT_F32, r, L.zstride, 0};
-          g4.Cin = {Xt, r, r * cc, 0};
-        } else {       // U is [r, c]: X' = P X + a X
-          g4.M = (int)r; g4.N = (int)cc; g4.K = (int)r; g4.Z0 = P;
-          g4.A = op(w.Pm, r, r * r);
-          g4.B = op(Xt, r, r * cc);
-          g4.C = {U, DT_F32, cc, L.zstride, 0};
-          g4.Cin = {X, cc, r * cc, 0};
-        }
-        g4.alpha = 1.0f; g4.beta = a3;
-        TTT_TRY(run_tf32("ns_apply", g4, s));
-        return TTT_OK;
+      const bool last = direct && it == steps - 1;
+      GemmProblem g3;  // X' = P X + a X (Y' = Y P + a Y)
+      g3.K = (int)r; g3.Z0 = P;
+      if (tall) {
+        g3.M = (int)cc; g3.N = (int)r;
+        g3.A = op(X, false, r, r * cc);
+        g3.B = op(w.Pm, false, r, r * r);
+      } else {
+        g3.M = (int)r; g3.N = (int)cc;
+        g3.A = op(w.Pm, false, r, r * r);
+        g3.B = op(X, true, cc, r * cc);
       }
-      GemmProblem g3;  // X' = P X + a X, and X'^T
-      g3.M = (int)r; g3.N = (int)cc; g3.K = (int)r; g3.Z0 = P;
-      g3.A = op(w.Pm, r, r * r);
-      g3.B = op(Xt, r, r * cc);
-      g3.C = {X2, DT_F32, cc, r * cc, 0};
-      g3.C.t32 = X2t; g3.C.ldt = r; g3.C.ts0 = r * cc;
-      g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, cc, r * cc, 0};
+      g3.C = last ? GemmOut{U, DT_F32, ldx, L.zstride, 0} : GemmOut{X2, DT_F32, ldx, r * cc, 0};
+      g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, ldx, r * cc, 0};
       TTT_TRY(run_tf32("ns_apply", g3, s));
+      if (last) return TTT_OK;
       std::swap(X, X2);
-      std::swap(Xt, X2t);
     }
     TTT_OP("ns_writeback", ns_writeback(X, U, Z, L, s));
     return TTT_OK;
   }
+  TTT_OP("ns_normalize", ns_normalize(U, w.X, Z, L, 1e-7f, w.nrm, s, nullptr, nrm_ready));
   float* X = w.X;
   float* X2 = w.X2;
   for (int it = 0; it < steps; ++it) {

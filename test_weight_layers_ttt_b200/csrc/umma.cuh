@@ -209,6 +209,16 @@ __host__ __device__ constexpr uint64_t make_sw128_desc(uint32_t saddr, uint32_t 
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same for the 128-byte swizzle on a 32-byte base (layout type 1), the one layout that
+// MN-major tf32 operands take: 32-byte chunks of each 128-byte row XOR-swizzled by the row
+// index mod 4 (what a TMA load with CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B writes); k rows of
+// 128 bytes, 4-row groups SBO bytes apart, 32-element MN blocks LBO bytes apart.
+__host__ __device__ constexpr uint64_t make_sw128b32_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                                          uint32_t sbo_bytes) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (1ull << 61);
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulation.
 //   bits [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),
 //   bit 15 A major (1 = MN), bit 16 B major, [17,23) N >> 3, [24,29) M >> 4.
@@ -216,10 +226,11 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn, 
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
          ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-// Instruction descriptor of kind::tf32 (A / B format 2 = tf32), both operands K-major.
-__host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N) {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
+// Instruction descriptor of kind::tf32 (A / B format 2 = tf32; either operand K- or
+// MN-major, same bits as above).
+__host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace umma
