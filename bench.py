@@ -110,7 +110,8 @@ def _ns_work(wl, r, c, matrices):
     """Step-level work of the Newton-Schulz kernels on `matrices` [r, c] matrices (r <= c):
     tensor FLOPs of the one-CTA kernel (three bf16 terms hi*hi + hi*lo + lo*hi per fp32
     product), of the tf32 GEMMs (one term, at the tf32 rate), and the HBM bytes of the fp32
-    set-up (read U, write the scaled X) and write-back."""
+    set-up (read U, write the scaled X; or only its norms, the scaling then riding on the
+    first step's epilogues) and write-back."""
     steps = wl.ns_steps if wl.ns_steps else 5
     Z = float(matrices)
     return {
@@ -119,6 +120,7 @@ def _ns_work(wl, r, c, matrices):
         "ns_poly": ("tensor_tf32", steps * 2.0 * r ** 3 * Z),
         "ns_apply": ("tensor_tf32", steps * 2.0 * r * r * c * Z),
         "ns_normalize": ("hbm", 8.0 * r * c * Z),
+        "ns_sumsq": ("hbm", 4.0 * r * c * Z),
         "ns_writeback": ("hbm", 8.0 * r * c * Z),
     }
 

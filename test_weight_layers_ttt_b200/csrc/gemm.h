@@ -43,6 +43,12 @@ struct GemmProblem {
   float alpha = 1.0f;
   float beta = 0.0f;
   GemmCin Cin;
+  // tf32 engine only: per batch entry z0, alpha and beta further scaled by s^zpa and s^zpb
+  // with s = 1 / (sqrt(zss[z0]) + zeps) (zss: sums of squares, e.g. of a Frobenius norm),
+  // or null
+  const float* zss = nullptr;
+  float zeps = 0.0f;
+  int zpa = 0, zpb = 0;
 };
 
 // CUDA-core engine: any strides, fp32 or bf16 operands, fp32 accumulation.

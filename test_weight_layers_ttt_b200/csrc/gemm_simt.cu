@@ -242,6 +242,10 @@ ttt_status gemm_simt_swiglu(const SwigluGemm& g, cudaStream_t stream) {
 
 ttt_status gemm_simt(const GemmProblem& p, cudaStream_t stream) {
   if (p.M <= 0 || p.N <= 0 || p.Z0 <= 0 || p.Z1 <= 0) return TTT_OK;
+  if (p.zss) {
+    set_error_message("gemm_simt: per-entry scales are taken only by the tf32 engine");
+    return TTT_ERR_UNSUPPORTED;
+  }
   const long long gy = (p.M + TM - 1) / TM, gz = (long long)p.Z0 * p.Z1;
   if (gy > 65535 || gz > 65535) {
     set_error_message("gemm_simt: grid too large (M=%d, Z=%lld)", p.M, gz);

@@ -61,6 +61,7 @@ struct UArgs {
   __nv_bfloat16* C16;   // fp32 C: bf16 copy with C's strides, or null
   const float* Cin; long long ldi, is0, is1;
   float alpha, beta;
+  const float* zss; float zeps; int zpa, zpb;   // per-z0 scale of alpha / beta, or null
   // SWIGLU: phi columns < n_valid are written; row factor rs[z0*rs0 + z1*rs1 + row]
   void* C2; long long ld2, c2s0, c2s1;
   const float* rs; long long rs0, rs1;
@@ -385,6 +386,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
       if constexpr (MODE != EPI_SWIGLU) {
+        float alpha = args.alpha, beta = args.beta;
+        if (args.zss) {
+          const float sc = 1.0f / (sqrtf(args.zss[tc.z0]) + args.zeps);
+          if (args.zpa) alpha *= args.zpa == 2 ? sc * sc : sc;
+          if (args.zpb) beta *= sc;
+        }
         // alpha * acc (+ beta * Cin): each lane holds one row. EPI_STORE: each lane stores its
         // row's values directly (stores do not wait, so their scatter costs little).
         // EPI_STORE_STG / COPY (fp32 C with an addend): per 32-column chunk the warp stages
@@ -438,12 +445,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t* v = cc < 4 ? &ra[8 * cc] : &rb[8 * (cc - 4)];
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                  w[q] = pack_bf16x2(args.alpha * __uint_as_float(v[2 * q]),
-                                     args.alpha * __uint_as_float(v[2 * q + 1]));
+                  w[q] = pack_bf16x2(alpha * __uint_as_float(v[2 * q]),
+                                     alpha * __uint_as_float(v[2 * q + 1]));
               } else {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                  w[q] = __float_as_uint(args.alpha * __uint_as_float(ra[4 * cc + q]));
+                  w[q] = __float_as_uint(alpha * __uint_as_float(ra[4 * cc + q]));
               }
               asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]),
                            "r"(w[1]), "r"(w[2]), "r"(w[3])
@@ -479,11 +486,11 @@ __global__ void __launch_bounds__(THREADS, 1)
               if (nv <= 0) break;
               float w[32];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) w[j] = args.alpha * __uint_as_float(r[c0 + j]);
+              for (int j = 0; j < 32; ++j) w[j] = alpha * __uint_as_float(r[c0 + j]);
               if (irow) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                  if (j < nv) w[j] += args.beta * irow[col0 + j];
+                  if (j < nv) w[j] += beta * irow[col0 + j];
               }
               if (vrow && nv == 32) {
                 store32(crow + col0, w);
@@ -528,10 +535,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               sbuf[lane * 8 + (q ^ (lane & 7))] =
-                  make_float4(args.alpha * __uint_as_float(r[4 * q]),
-                              args.alpha * __uint_as_float(r[4 * q + 1]),
-                              args.alpha * __uint_as_float(r[4 * q + 2]),
-                              args.alpha * __uint_as_float(r[4 * q + 3]));
+                  make_float4(alpha * __uint_as_float(r[4 * q]),
+                              alpha * __uint_as_float(r[4 * q + 1]),
+                              alpha * __uint_as_float(r[4 * q + 2]),
+                              alpha * __uint_as_float(r[4 * q + 3]));
             __syncwarp();
 #pragma unroll
             for (int it = 0; it < 8; ++it) {
@@ -542,10 +549,10 @@ __global__ void __launch_bounds__(THREADS, 1)
               float x[4] = {sv.x, sv.y, sv.z, sv.w};
               if (cfull) {
                 if (ibase) {
-                  x[0] = fmaf(args.beta, cin[it].x, x[0]);
-                  x[1] = fmaf(args.beta, cin[it].y, x[1]);
-                  x[2] = fmaf(args.beta, cin[it].z, x[2]);
-                  x[3] = fmaf(args.beta, cin[it].w, x[3]);
+                  x[0] = fmaf(beta, cin[it].x, x[0]);
+                  x[1] = fmaf(beta, cin[it].y, x[1]);
+                  x[2] = fmaf(beta, cin[it].z, x[2]);
+                  x[3] = fmaf(beta, cin[it].w, x[3]);
                 }
                 store4(crow + col, x);
                 if constexpr (MODE == EPI_STORE_COPY) {
@@ -560,7 +567,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int j = 0; j < 4; ++j) {
                   if (col + j >= args.N) break;
                   float y = x[j];
-                  if (irow) y = fmaf(args.beta, irow[col + j], y);
+                  if (irow) y = fmaf(beta, irow[col + j], y);
                   crow[col + j] = from_f32<TC>(y);
                   x[j] = y;
                   if constexpr (MODE == EPI_STORE_COPY)
@@ -962,6 +969,7 @@ UArgs base_args(const GemmProblem& p, unsigned* dev_err, unsigned long long wait
   a.Cin = p.beta != 0.0f ? p.Cin.ptr : nullptr;
   a.ldi = p.Cin.ld; a.is0 = p.Cin.s0; a.is1 = p.Cin.s1;
   a.alpha = p.alpha; a.beta = p.beta;
+  a.zss = p.zss; a.zeps = p.zeps; a.zpa = p.zpa; a.zpb = p.zpb;
   a.err = dev_err;
   a.wait_ns = wait_ns;
   return a;
@@ -981,6 +989,7 @@ const char* umma_unsupported_reason(const GemmProblem& p) {
   if ((long long)p.Z0 * p.Z1 * ((p.M + BM - 1) / BM) * ((p.N + 63) / 64) > (1LL << 31))
     return "too many output tiles";
   if (p.beta != 0.0f && !p.Cin.ptr) return "beta != 0 needs an addend";
+  if (p.zss) return "per-entry scales are taken only with tf32 operands";
   if (p.C.copy16 && (p.C.dtype != DT_F32 || !aligned16(p.C.copy16) || !aligned16(p.C.ptr) ||
                      p.C.ld % 4 != 0 || p.C.s0 % 4 != 0 || p.C.s1 % 4 != 0))
     return "a bf16 copy needs an fp32 result with 16-byte aligned bases, strides multiples of 4";

@@ -1072,13 +1072,20 @@ cudaError_t rec_reduce(const float* partials, int splits, float* U, float* M_all
   return cudaGetLastError();
 }
 
+cudaError_t ns_sumsq(const float* U, int Z, const NsLayout& L, float* nrm, cudaStream_t s) {
+  if (Z <= 0) return cudaSuccess;
+  cudaError_t e = fill_f32(nrm, (long long)Z * L.parts, 0.0f, s);
+  if (e != cudaSuccess) return e;
+  ns_sumsq_kernel<<<dim3(L.parts, Z, NS_SLABS), 256, 0, s>>>(U, L, nrm);
+  return cudaGetLastError();
+}
+
 cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, float eps,
                          float* nrm, cudaStream_t s, float* Xt, bool nrm_ready) {
   if (Z <= 0) return cudaSuccess;
   if (!nrm_ready) {
-    cudaError_t e = fill_f32(nrm, (long long)Z * L.parts, 0.0f, s);
+    cudaError_t e = ns_sumsq(U, Z, L, nrm, s);
     if (e != cudaSuccess) return e;
-    ns_sumsq_kernel<<<dim3(L.parts, Z, NS_SLABS), 256, 0, s>>>(U, L, nrm);
   }
   int tiles = 0;
   for (int p = 0; p < L.parts; ++p)

@@ -82,6 +82,8 @@ cudaError_t ns_normalize(const float* U, float* X, int Z, const NsLayout& L, flo
                          float* nrm, cudaStream_t s, float* Xt = nullptr,
                          bool nrm_ready = false);
 cudaError_t ns_writeback(const float* X, float* U, int Z, const NsLayout& L, cudaStream_t s);
+// The sums of squares alone (nrm[z * parts + p] = ||U_(z,p)||_F^2).
+cudaError_t ns_sumsq(const float* U, int Z, const NsLayout& L, float* nrm, cudaStream_t s);
 
 // The whole Newton-Schulz orthogonalisation of the matrices of L on the tensor cores
 // (ns_mma.cu; operands split into bf16 hi + lo pairs, fp32 accumulation): normalise,

@@ -673,22 +673,33 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
     // U when it has that orientation, else a write-back pass transposes the parts back.
     // Either way P = c A A + b A from A (symmetric, K-major both sides).
     const bool tall = L.parts == 1 && R > Cc;
-    TTT_OP("ns_normalize", ns_normalize(U, tall ? nullptr : w.X, Z, L, 1e-7f, w.nrm, s,
-                                        tall ? w.X : nullptr, nrm_ready));
-    float *X = w.X, *X2 = w.X2;
+    const bool direct = L.parts == 1 && (L.mask & 1);
+    // With one matrix per entry and at least two steps, the first step reads U itself and
+    // the normalisation rides on its epilogues: A = s^2 (U^T U) (or U U^T) and the apply
+    // s (U P) + a s U, s = 1 / (||U||_F + eps) per entry; no scaled copy is written.
+    const bool fold = direct && steps >= 2;
+    if (fold) {
+      if (!nrm_ready) TTT_OP("ns_sumsq", ns_sumsq(U, Z, L, w.nrm, s));
+    } else {
+      TTT_OP("ns_normalize", ns_normalize(U, tall ? nullptr : w.X, Z, L, 1e-7f, w.nrm, s,
+                                          tall ? w.X : nullptr, nrm_ready));
+    }
     auto op = [](const float* ptr, bool mn, long long ld, long long s0) {
       GemmOperand o;
       o.ptr = ptr; o.dtype = DT_F32; o.mn_major = mn; o.ld = ld; o.s0 = s0; o.s1 = 0;
       return o;
     };
     const long long ldx = tall ? r : cc;   // row stride of X (or Y)
-    const bool direct = L.parts == 1 && (L.mask & 1);
+    const float* X = fold ? U : w.X;       // this step's input and its entry stride
+    long long xs = fold ? L.zstride : r * cc;
     for (int it = 0; it < steps; ++it) {
+      const bool scaled = fold && it == 0;
       GemmProblem g1;  // A = X X^T (= Y^T Y)
       g1.M = (int)r; g1.N = (int)r; g1.K = (int)cc; g1.Z0 = P;
-      g1.A = op(X, tall, ldx, r * cc);
-      g1.B = op(X, tall, ldx, r * cc);
+      g1.A = op(X, tall, ldx, xs);
+      g1.B = op(X, tall, ldx, xs);
       g1.C = {w.Ag, DT_F32, r, r * r, 0};
+      if (scaled) { g1.zss = w.nrm; g1.zeps = 1e-7f; g1.zpa = 2; }
       TTT_TRY(run_tf32("ns_gram", g1, s));
       GemmProblem g2;  // P = c A A + b A
       g2.M = (int)r; g2.N = (int)r; g2.K = (int)r; g2.Z0 = P;
@@ -698,22 +709,25 @@ ttt_status run_ns(int ot, float* U, int Z, const NsLayout& L, int steps, const N
       g2.alpha = c3; g2.beta = b3; g2.Cin = {w.Ag, r, r * r, 0};
       TTT_TRY(run_tf32("ns_poly", g2, s));
       const bool last = direct && it == steps - 1;
+      float* out = last ? U : (X == w.X ? w.X2 : w.X);
       GemmProblem g3;  // X' = P X + a X (Y' = Y P + a Y)
       g3.K = (int)r; g3.Z0 = P;
       if (tall) {
         g3.M = (int)cc; g3.N = (int)r;
-        g3.A = op(X, false, r, r * cc);
+        g3.A = op(X, false, r, xs);
         g3.B = op(w.Pm, false, r, r * r);
       } else {
         g3.M = (int)r; g3.N = (int)cc;
         g3.A = op(w.Pm, false, r, r * r);
-        g3.B = op(X, true, cc, r * cc);
+        g3.B = op(X, true, cc, xs);
       }
-      g3.C = last ? GemmOut{U, DT_F32, ldx, L.zstride, 0} : GemmOut{X2, DT_F32, ldx, r * cc, 0};
-      g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, ldx, r * cc, 0};
+      g3.C = {out, DT_F32, ldx, last ? L.zstride : r * cc, 0};
+      g3.alpha = 1.0f; g3.beta = a3; g3.Cin = {X, ldx, xs, 0};
+      if (scaled) { g3.zss = w.nrm; g3.zeps = 1e-7f; g3.zpa = 1; g3.zpb = 1; }
       TTT_TRY(run_tf32("ns_apply", g3, s));
       if (last) return TTT_OK;
-      std::swap(X, X2);
+      X = out;
+      xs = r * cc;
     }
     TTT_OP("ns_writeback", ns_writeback(X, U, Z, L, s));
     return TTT_OK;
