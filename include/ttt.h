@@ -165,6 +165,31 @@ ttt_status ttt_la_parallel_fwd_shard(const ttt_desc* desc, const void* q, const 
                                      size_t workspace_bytes, ttt_stream_t stream);
 
 /*
+ * The outputs pass of a shard that reuses the key side of the state-only pass before it.
+ * A state-only call of ttt_la_parallel_fwd_shard (out = NULL) leaves in its workspace the
+ * blocked input weights and every chunk's delta; this call then forms the chunk states from
+ * W1 + sum_{i < n_prior} prior[i] and those deltas, and the outputs, without recomputing
+ * phi(K) (same section as above: the deltas do not depend on the initial state). So a
+ * shard's two passes cost one key side, one scan each and one query side.
+ *
+ *   desc       identical to the state-only call's
+ *   q          [B,H,N,h] dtype (the same tokens as the state-only call's k when q == k)
+ *   W1, prior, n_prior, S_final   as for ttt_la_parallel_fwd_shard
+ *   out        [B,H,N,h] dtype, not NULL
+ *   workspace  the state-only call's workspace and size, untouched since
+ * TTT_ERR_UNSUPPORTED when the problem takes the sequential schedule (its state-only pass
+ * keeps no chunk deltas: call ttt_la_parallel_fwd_shard again with out instead);
+ * TTT_ERR_INVALID_ARG unless the last ttt_la_parallel_fwd_shard call on this host thread
+ * was a successful state-only call with the same descriptor, workspace and size (each
+ * outputs pass consumes it). Streams as for ttt_la_parallel_fwd.
+ */
+ttt_status ttt_la_parallel_fwd_shard_outputs(const ttt_desc* desc, const void* q,
+                                             const float* W1, const float* prior,
+                                             int32_t n_prior, void* out, float* S_final,
+                                             void* workspace, size_t workspace_bytes,
+                                             ttt_stream_t stream);
+
+/*
  * Parallel last-layer-only form with momentum and orthogonalisation of the W1 update
  * ("Test-Time Training with KV Binding Is Secretly Linear Attention", section 方法步骤详情:
  * simplification variant 2 keeps momentum and Newton-Schulz; the pages' recurrent -> parallel

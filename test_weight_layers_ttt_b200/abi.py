@@ -44,7 +44,7 @@ TTT_CHECK_FINITE = 2
 # Every symbol include/ttt.h declares.
 EXPORTED = (
     "ttt_workspace_bytes", "ttt_la_parallel_fwd", "ttt_la_parallel_fwd_noalloc",
-    "ttt_la_parallel_fwd_shard",
+    "ttt_la_parallel_fwd_shard", "ttt_la_parallel_fwd_shard_outputs",
     "ttt_linear_attn_fwd", "ttt_la_parallel_momentum_fwd", "ttt_la_parallel_bwd",
     "ttt_lact_recurrent_fwd",
     "ttt_lm_target_workspace_bytes", "ttt_lm_target", "ttt_last_device_status",
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.ttt_la_parallel_fwd.restype = I32
         L.ttt_la_parallel_fwd_shard.argtypes = [D] + [P] * 8 + [I32, P, P, P, S, P]
         L.ttt_la_parallel_fwd_shard.restype = I32
+        L.ttt_la_parallel_fwd_shard_outputs.argtypes = [D] + [P] * 3 + [I32, P, P, P, S, P]
+        L.ttt_la_parallel_fwd_shard_outputs.restype = I32
         L.ttt_la_parallel_fwd_noalloc.argtypes = [D] + [P] * 10
         L.ttt_la_parallel_fwd_noalloc.restype = I32
         L.ttt_linear_attn_fwd.argtypes = [D] + [P] * 8 + [S, P]
@@ -193,6 +195,14 @@ def ttt_la_parallel_fwd_shard(desc, q, k, v, eta, W0, W2, W1, prior, n_prior, ou
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(W0), _ptr(W2), _ptr(W1),
         _ptr(prior), int(n_prior), _ptr(out), _ptr(S_final), _ptr(workspace), wb,
         _stream(stream)))
+
+
+def ttt_la_parallel_fwd_shard_outputs(desc, q, W1, prior, n_prior, out, S_final, workspace,
+                                      workspace_bytes=None, stream=None):
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    _check(lib().ttt_la_parallel_fwd_shard_outputs(
+        ctypes.byref(desc), _ptr(q), _ptr(W1), _ptr(prior), int(n_prior), _ptr(out),
+        _ptr(S_final), _ptr(workspace), wb, _stream(stream)))
 
 
 def ttt_la_parallel_momentum_fwd(desc, q, k, v, eta, alpha, W0, W2, W1, out, S_final,

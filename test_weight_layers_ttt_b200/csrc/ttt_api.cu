@@ -1222,6 +1222,20 @@ ttt_status check_ws(void* ws, size_t have, size_t need) {
 }  // namespace
 }  // namespace ttt
 
+namespace ttt {
+namespace {
+// The last successful state-only shard call on this thread, whose workspace still holds the
+// blocked weights and the chunk deltas for ttt_la_parallel_fwd_shard_outputs.
+struct ShardMark {
+  bool valid = false;
+  ttt_desc d{};
+  void* ws = nullptr;
+  size_t bytes = 0;
+};
+thread_local ShardMark t_shard_mark;
+}  // namespace
+}  // namespace ttt
+
 using namespace ttt;
 
 extern "C" {
@@ -1289,6 +1303,7 @@ ttt_status ttt_la_parallel_fwd_shard(const ttt_desc* desc, const void* q, const 
                                      const float* W2, const float* W1, const float* prior,
                                      int32_t n_prior, void* out, float* S_final, void* workspace,
                                      size_t workspace_bytes, ttt_stream_t stream) {
+  t_shard_mark.valid = false;
   TTT_TRY(check_desc(desc, TTT_PATH_PARALLEL));
   const ttt_desc& d = *desc;
   const long long BH = (long long)d.B * d.H;
@@ -1324,7 +1339,53 @@ ttt_status ttt_la_parallel_fwd_shard(const ttt_desc* desc, const void* q, const 
                                         b.scan_tmp, s));
       return TTT_OK;
     }
-    return parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s, prior, n_prior);
+    const ttt_status st =
+        parallel_impl(d, q, k, v, eta, W0, W2, W1, out, S_final, b, s, prior, n_prior);
+    if (st == TTT_OK && !out && !seq) {
+      // the blocked weights and every chunk's delta stay in the workspace for an outputs pass
+      t_shard_mark.valid = true;
+      t_shard_mark.d = d;
+      t_shard_mark.ws = workspace;
+      t_shard_mark.bytes = workspace_bytes;
+    }
+    return st;
+  });
+}
+
+ttt_status ttt_la_parallel_fwd_shard_outputs(const ttt_desc* desc, const void* q,
+                                             const float* W1, const float* prior,
+                                             int32_t n_prior, void* out, float* S_final,
+                                             void* workspace, size_t workspace_bytes,
+                                             ttt_stream_t stream) {
+  TTT_TRY(check_desc(desc, TTT_PATH_PARALLEL));
+  const ttt_desc& d = *desc;
+  const ShardMark mk = t_shard_mark;
+  t_shard_mark.valid = false;
+  if (sequential_schedule(d))
+    return fail(TTT_ERR_UNSUPPORTED, "the sequential schedule keeps no chunk deltas: run the "
+                                     "shard call again with out");
+  if (!mk.valid || mk.ws != workspace || mk.bytes != workspace_bytes ||
+      std::memcmp(&mk.d, &d, sizeof(ttt_desc)) != 0)
+    return fail(TTT_ERR_INVALID_ARG, "an outputs pass must follow, on this thread, a state-only "
+                                     "shard call with the same descriptor and workspace");
+  const long long BH = (long long)d.B * d.H;
+  if (BH == 0 || d.N == 0) return TTT_OK;
+  if (!q || !out) return fail(TTT_ERR_INVALID_ARG, "q and out must not be NULL");
+  if (!al16(q) || !al16(out) || (W1 && !al16(W1)))
+    return fail(TTT_ERR_INVALID_ARG, "q, out and W1 must be 16-byte aligned");
+  if (n_prior < 0 || n_prior > 4096) return fail(TTT_ERR_INVALID_ARG, "n_prior must be in 0..4096");
+  if (n_prior > 0 && (!prior || !al16(prior)))
+    return fail(TTT_ERR_INVALID_ARG, "prior must be a 16-byte aligned pointer when n_prior > 0");
+  ParBufs b;
+  plan_parallel(d, workspace, b, false);
+  t_guards.clear();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
+  const long long hm = (long long)d.h * d.m;
+  return with_checks(s, {{out, BH * d.N * d.h, ot}, {S_final, BH * hm, DT_F32}},
+                     [&]() -> ttt_status {
+    TTT_TRY(chunk_states(d, b.dS, W1, S_final, b.Sc, b.scan_tmp, s, prior, n_prior));
+    return query_side(d, q, b, false, out, s);
   });
 }
 

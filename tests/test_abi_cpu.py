@@ -113,6 +113,25 @@ def test_parallel_rejects_pointers_and_workspace():
     assert "256-byte" in abi.ttt_last_error_message()
 
 
+def test_shard_outputs_pass_needs_a_state_only_call_first():
+    """The outputs pass reuses what a state-only shard call left in the workspace: without
+    one just before on this thread (or after a failed one) it is refused."""
+    d = lm_desc()
+    need = abi.ttt_workspace_bytes(d, abi.TTT_PATH_PARALLEL)
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_la_parallel_fwd_shard_outputs(d, 256, 256, None, 0, 256, None, 256, need,
+                                              stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+    assert "state-only" in abi.ttt_last_error_message()
+    with pytest.raises(abi.TTTError):   # a state-only call that fails (NULL q) marks nothing
+        abi.ttt_la_parallel_fwd_shard(d, None, 256, 256, 256, 256, 256, None, None, 0, None,
+                                      256, 256, need, stream=0)
+    with pytest.raises(abi.TTTError) as ei:
+        abi.ttt_la_parallel_fwd_shard_outputs(d, 256, 256, None, 0, 256, None, 256, need,
+                                              stream=0)
+    assert ei.value.status == abi.TTT_ERR_INVALID_ARG
+
+
 def test_linear_attention_workspace_and_checks():
     d = lm_desc(m=256)   # identity features: the state is [h, h]
     BH, N, h, C = 8, 32768, 256, 16

@@ -398,6 +398,31 @@ def test_sequence_shards_through_the_library_match_the_oracle(case):
         assert rel(host(Sonly), host(Sfull)) <= 1e-3
     else:
         assert torch.equal(Sfull, Sonly)
+    # each shard's outputs pass reusing the chunk deltas its state-only pass left in the
+    # workspace: against the oracle, and (without q == k, where the full call forms phi once
+    # for both sides) bit for bit the second full pass's outputs
+    outs2 = []
+    for r, sl in enumerate(shards):
+        args = [t[:, :, sl].contiguous() for t in (q, k, v, eta)]
+        if qk:
+            args[1] = args[0]
+        desc = layer.parallel_desc(args[0], W1, chunk, order=order,
+                                   w_in_layout=lay.get("w_in_layout", 0),
+                                   w1_layout=lay.get("w1_layout", 0))
+        ws = layer.workspace(abi.ttt_workspace_bytes(desc, abi.TTT_PATH_PARALLEL), q.device)
+        layer.la_parallel_fwd_shard(*args, W0, W2, None, chunk, state_only=True, m=m, ws=ws,
+                                    **lay)
+        prior = torch.stack(totals[:r]) if r else None
+        o2, S2 = layer.la_parallel_fwd_shard_outputs(args[0], W1, chunk, ws, prior=prior, **lay)
+        outs2.append(o2)
+        if not qk:
+            assert torch.equal(o2, outs[r])
+    abi.ttt_last_device_status()
+    assert rel(host(torch.cat(outs2, 2)), ref) <= TOL["bf16"]
+    S2h = np.swapaxes(host(S2), 2, 3) if qk else host(S2)
+    assert rel(S2h, Sref) <= TOL["bf16"]
+    with pytest.raises(abi.TTTError):   # the outputs pass consumed the state-only record
+        layer.la_parallel_fwd_shard_outputs(args[0], W1, chunk, ws, prior=prior, **lay)
 
 
 def test_context_parallel_single_rank_nccl_matches_the_oracle():
