@@ -15,8 +15,8 @@ using bf16 = __nv_bfloat16;
 // of the blocked operand are coalesced. grid (mpad/32, ceil(h/32), 2 * n_entries),
 // block (32, 8); blockIdx.z = 2 * entry + which (0: W0, 1: W2).
 template <typename OT>
-__global__ void prep_wk_blocked_kernel(const float* W0, const float* W2, OT* Wk, int src_heads,
-                                       int h, int m, int layout) {
+__global__ void prep_wk_blocked_kernel(const float* W0, const float* W2, OT* Wk, OT* Wk1, OT* Wk2,
+                                       int src_heads, int h, int m, int layout) {
   __shared__ float tile[32][33];
   const int mpad = (m + 127) / 128 * 128;
   const int j0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
@@ -36,13 +36,16 @@ __global__ void prep_wk_blocked_kernel(const float* W0, const float* W2, OT* Wk,
     }
   }
   __syncthreads();
-  OT* dst = Wk + (long long)e * 2 * mpad * h;
+  const long long eo = (long long)e * 2 * mpad * h;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int jj = ty + 8 * k, j = j0 + jj, i = i0 + tx;
     if (j >= mpad || i >= h) continue;
     const long long row = (long long)(j >> 7) * 256 + (which ? 128 : 0) + (j & 127);
-    dst[row * h + i] = from_f32<OT>(which ? tile[jj][tx] : 0.5f * tile[jj][tx]);
+    const OT x = from_f32<OT>(which ? tile[jj][tx] : 0.5f * tile[jj][tx]);
+    Wk[eo + row * h + i] = x;
+    if (Wk1) Wk1[eo + row * h + i] = x;   // further copies of the same operand
+    if (Wk2) Wk2[eo + row * h + i] = x;
   }
 }
 
@@ -208,8 +211,8 @@ __device__ __forceinline__ void part_dims(int p, int h, int m, int& R, int& Cc) 
 // M_out = M_all^T).
 template <typename OT>
 __global__ void rec_transpose_kernel(int dir, const float* W0, const float* W2, const float* W1,
-                                     int H, int h, int m, float* W_all, OT* W1t,
-                                     const float* M_in, float* M_all, int momentum,
+                                     int H, int h, int m, float* W_all, OT* W1t, OT* W1t1,
+                                     OT* W1t2, const float* M_in, float* M_all, int momentum,
                                      float* W0_out, float* W2_out, float* W1_out, float* M_out) {
   __shared__ float t[2][32][33];
   const int p = blockIdx.y, bh = blockIdx.z, head = bh % H;
@@ -237,7 +240,12 @@ __global__ void rec_transpose_kernel(int dir, const float* W0, const float* W2, 
       if (r < R && c < Cc) {
         const long long o = (long long)c * R + r;
         W_all[st + o] = t[0][tx][k];
-        if (p == 1) W1t[(long long)bh * hm + o] = from_f32<OT>(t[0][tx][k]);
+        if (p == 1) {
+          const OT x = from_f32<OT>(t[0][tx][k]);
+          W1t[(long long)bh * hm + o] = x;
+          if (W1t1) W1t1[(long long)bh * hm + o] = x;   // further operand copies
+          if (W1t2) W1t2[(long long)bh * hm + o] = x;
+        }
         if (momentum) M_all[st + o] = t[1][tx][k];
       }
     }
@@ -961,13 +969,15 @@ cudaError_t by_ot(int ot, F&& f) {
 }  // namespace
 
 cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
-                            int src_heads, int h, int m, int src_layout, cudaStream_t s) {
+                            int src_heads, int h, int m, int src_layout, cudaStream_t s,
+                            void* Wk1, void* Wk2) {
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
     const int mpad = (m + 127) / 128 * 128;
     dim3 grid(mpad / 32, (h + 31) / 32, 2 * n_entries);
     prep_wk_blocked_kernel<OT><<<grid, dim3(32, 8), 0, s>>>(
-        W0, W2, static_cast<OT*>(Wk), src_heads, h, m, src_layout);
+        W0, W2, static_cast<OT*>(Wk), static_cast<OT*>(Wk1), static_cast<OT*>(Wk2), src_heads,
+        h, m, src_layout);
     return cudaGetLastError();
   });
 }
@@ -1035,13 +1045,13 @@ cudaError_t chunk_scan(int ot, const float* dS, const float* W1, const float* pr
 
 cudaError_t rec_init(int ot, const float* W0, const float* W2, const float* W1, int BH, int H,
                      int h, int m, float* W_all, void* W1t, const float* M_in, float* M_all,
-                     int momentum, cudaStream_t s) {
+                     int momentum, cudaStream_t s, void* W1t1, void* W1t2) {
   return by_ot(ot, [&](auto tag) {
     using OT = decltype(tag);
     const int tiles = ((h + 31) / 32) * ((m + 31) / 32);
     rec_transpose_kernel<OT><<<dim3(tiles, 3, BH), dim3(32, 8), 0, s>>>(
-        0, W0, W2, W1, H, h, m, W_all, static_cast<OT*>(W1t), M_in, M_all, momentum, nullptr,
-        nullptr, nullptr, nullptr);
+        0, W0, W2, W1, H, h, m, W_all, static_cast<OT*>(W1t), static_cast<OT*>(W1t1),
+        static_cast<OT*>(W1t2), M_in, M_all, momentum, nullptr, nullptr, nullptr, nullptr);
     return cudaGetLastError();
   });
 }
@@ -1243,7 +1253,7 @@ cudaError_t rec_finish(const float* W_all, int BH, int H, int h, int m, float* W
   const int tiles = ((h + 31) / 32) * ((m + 31) / 32);
   rec_transpose_kernel<float><<<dim3(tiles, 3, BH), dim3(32, 8), 0, s>>>(
       1, nullptr, nullptr, nullptr, H, h, m, const_cast<float*>(W_all), nullptr, nullptr,
-      const_cast<float*>(M_all), 0, W0_out, W2_out, W1_out, M_out);
+      nullptr, nullptr, const_cast<float*>(M_all), 0, W0_out, W2_out, W1_out, M_out);
   return cudaGetLastError();
 }
 

@@ -15,8 +15,10 @@ namespace ttt {
 // rows past m). W0 enters halved (exact in binary floating point), so the GEMM's first
 // half yields a/2 = (x W0)/2, the argument silu takes through tanh:
 // silu(a) = (a/2) (1 + tanh(a/2)).
+// Wk1, Wk2: further copies of the same operand, or null.
 cudaError_t prep_wk_blocked(int ot, const float* W0, const float* W2, void* Wk, int n_entries,
-                            int src_heads, int h, int m, int src_layout, cudaStream_t s);
+                            int src_heads, int h, int m, int src_layout, cudaStream_t s,
+                            void* Wk1 = nullptr, void* Wk2 = nullptr);
 
 // Xs[r, :] = X[r, :] * eta[r] for `rows` rows of width w (OT in and out; eta fp32).
 cudaError_t scale_rows(int ot, const void* X, const float* eta, void* Xs, long long rows, int w,
@@ -38,11 +40,12 @@ cudaError_t chunk_scan(int ot, const float* dS, const float* W1, const float* pr
 // row one output unit over the input dimension (so the renormalisation is a row norm);
 // momentum, the update buffer U and the split-K gradient partials use the same layout.
 // rec_init transposes the per-head initial weights (original layouts W0, W2 [h, m], W1
-// [m, h]) into W_all, writes W1t = the OT copy of W1^T [BH, h, m] and, with momentum, M_all
-// = M_in^T (M_in in the original part layouts) or 0.
+// [m, h]) into W_all, writes W1t = the OT copy of W1^T [BH, h, m] (and the same into W1t1,
+// W1t2 when not null) and, with momentum, M_all = M_in^T (M_in in the original part
+// layouts) or 0.
 cudaError_t rec_init(int ot, const float* W0, const float* W2, const float* W1, int BH, int H,
                      int h, int m, float* W_all, void* W1t, const float* M_in, float* M_all,
-                     int momentum, cudaStream_t s);
+                     int momentum, cudaStream_t s, void* W1t1 = nullptr, void* W1t2 = nullptr);
 // Column norms over the input dimension of the initial weights, per head:
 // tnorm[head] = [W0 columns (m) | W1 columns (h) | W2 columns (m)].
 cudaError_t col_norms(const float* W0, const float* W2, const float* W1, int H, int h, int m,

@@ -1534,19 +1534,13 @@ ttt_status ttt_lact_recurrent_fwd(const ttt_desc* desc, const void* q, const voi
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int ot = d.dtype == TTT_DTYPE_BF16 ? DT_BF16 : DT_F32;
   TTT_TRY(checks_begin(s));
+  // every operand copy starts from the initial weights (a matrix outside the update mask is
+  // never rewritten): the set-up kernels write all three copies
   TTT_OP("rec_init", rec_init(ot, W0, W2, W1, (int)BH, d.H, d.h, d.m, b.W_all, b.W1t[0],
-                              d.momentum ? M_io : nullptr, b.M_all, d.momentum, s));
-  TTT_OP("prep_weights", prep_wk_blocked(ot, W0, W2, b.Wk[0], (int)BH, d.H, d.h, d.m, 0, s));
-  {  // every operand copy starts from the initial weights (a matrix outside the update mask
-     // is never rewritten)
-    const size_t os = ot == DT_BF16 ? 2 : 4;
-    for (int i = 1; i < 3; ++i) {
-      TTT_CUDA(cudaMemcpyAsync(b.Wk[i], b.Wk[0], os * BH * 2 * padded_m(d.m) * d.h,
-                               cudaMemcpyDeviceToDevice, s));
-      TTT_CUDA(cudaMemcpyAsync(b.W1t[i], b.W1t[0], os * BH * d.h * d.m,
-                               cudaMemcpyDeviceToDevice, s));
-    }
-  }
+                              d.momentum ? M_io : nullptr, b.M_all, d.momentum, s, b.W1t[1],
+                              b.W1t[2]));
+  TTT_OP("prep_weights", prep_wk_blocked(ot, W0, W2, b.Wk[0], (int)BH, d.H, d.h, d.m, 0, s,
+                                         b.Wk[1], b.Wk[2]));
   if (d.renorm) TTT_OP("col_norms", col_norms(W0, W2, W1, d.H, d.h, d.m, b.tnorm, s));
   const long long N = d.N, L = d.chunk;
   // The apply of chunk c - 1 (update -> apply order; of chunk c in apply -> update order)
