@@ -304,8 +304,10 @@ MOM_CASES = [
     # bf16 with 136 x 256 matrices (over the one-CTA limit): three tf32 GEMMs per step,
     # K = 136 not a multiple of the 32-wide k-block (zero-filled tail)
     ("lm", "bf16", 1, 1, 512, 256, 136, 128, True, 3),
-    # the lm shape: 256 x 512 matrices, five steps
+    # the lm shape: 256 x 512 matrices, five steps (the first reads the momentum itself,
+    # normalised through per-matrix GEMM scales); one step (a scaled copy first)
     ("lm", "bf16", 1, 1, 1024, 256, 512, 256, True, 5),
+    ("lm", "bf16", 1, 2, 512, 256, 512, 256, True, 1),
 ]
 
 
