@@ -524,8 +524,11 @@ def _roofline(table, wl, peaks, form, steps):
             "dtype": "tf32" if bound == "tensor_tf32" else ("bf16" if bound == "tensor" else None),
             "achieved": round(achieved, 2), "peak": round(peak, 2), "unit": unit,
             "frac": round(achieved / peak, 4),
+            # captures exist for the parallel form's kernels and the momentum form's
+            # Newton-Schulz GEMMs (names that no other form launches)
             "traffic": (_traffic(wl.name, name)
-                        if form == "parallel" and wl == WORKLOADS_REF().get(wl.name) else None),
+                        if (form == "parallel" or name.startswith("ns_"))
+                        and wl == WORKLOADS_REF().get(wl.name) else None),
             "work_per_launch": work, "share": round(e["share"], 4),
             "peak_source": peaks["source"] + " (burst)"}
 
