@@ -308,6 +308,8 @@ MOM_CASES = [
     # normalised through per-matrix GEMM scales); one step (a scaled copy first)
     ("lm", "bf16", 1, 1, 1024, 256, 512, 256, True, 5),
     ("lm", "bf16", 1, 2, 512, 256, 512, 256, True, 1),
+    # no momentum: the norms come from their own pass, not from the momentum scan
+    ("lm", "bf16", 1, 1, 512, 256, 512, 256, False, 5),
 ]
 
 
