@@ -46,9 +46,9 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 
 // STORE: each lane stores its row directly (no addend, or bf16 C). STORE_STG: fp32 C with an
 // addend, staged per warp so Cin loads and C stores are row-contiguous. STORE_COPY: STORE_STG
-// plus a bf16 copy of the result. STORE_T: STORE_STG plus the result written transposed
-// (fp32), 128 contiguous bytes per store. STORE_TMA: bf16 C without an addend, each warp's
-// 32 rows staged 64 columns at a time in its 4 KB box and written with TMA tensor stores.
+// plus a bf16 copy of the result. STORE_TMA: C without an addend, each warp's 32 rows
+// staged 64 bf16 (or 32 fp32) columns at a time in its 4 KB box and written with TMA tensor
+// stores.
 // Separate instantiations, so no mode pays for another's code.
 enum EpiMode : int {
   EPI_STORE = 0, EPI_SWIGLU = 1, EPI_STORE_STG = 2, EPI_STORE_COPY = 3, EPI_STORE_TMA = 5
@@ -87,7 +87,7 @@ struct Smem {
   static constexpr int B_BYTES = BN * BK * 2;             // one k-block of B
   static constexpr int B_RES = BRES ? 4 * B_BYTES : 0;    // resident B, at most 4 k-blocks
   static constexpr int STAGE = BRES ? A_BYTES : A_BYTES + B_BYTES;
-  // one 4 KB box per epilogue warp; STORE_T a second one for the transposed copy
+  // one 4 KB box per epilogue warp
   static constexpr int OUT_BYTES =
       MODE == EPI_STORE ? 0 : BM * 128 * 2;
   static constexpr int OUT_OFF = B_RES;
