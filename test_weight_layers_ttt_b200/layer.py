@@ -101,16 +101,18 @@ def la_parallel_fwd_shard(q, k, v, eta, W0, W2, W1, chunk, *, prior=None, state_
 
 
 def la_parallel_fwd_shard_outputs(q, W1, chunk, ws, *, prior=None, order="update_apply",
-                                  sign=1, w_in_layout=0, w1_layout=0, out=None, stream=None):
+                                  sign=1, w_in_layout=0, w1_layout=0, m=None, out=None,
+                                  stream=None):
     """The outputs pass of a shard after its state-only pass ``la_parallel_fwd_shard(...,
     state_only=True, ws=ws)`` on this thread: reuses that call's chunk deltas (left in
-    ``ws``) and forms the states from W1 plus the sum of ``prior``, then the outputs.
-    Returns (out, final state)."""
+    ``ws``) and forms the states from W1 (zeros when None) plus the sum of ``prior``, then
+    the outputs. Returns (out, final state). ``m`` is needed when W1 is None."""
     _need(q, "q", q.dtype)
     for t, n in ((W1, "W1"), (prior, "prior")):
         _need(t, n, torch.float32)
     B, H, N, h = q.shape
-    m = W1.shape[1] if w1_layout == 0 else W1.shape[2]
+    if m is None:
+        m = W1.shape[1] if w1_layout == 0 else W1.shape[2]
     desc = abi.ttt_desc(B=B, H=H, N=N, h=h, m=m, chunk=chunk, dtype=_dtype_code(q),
                         order=ORDERS[order], sign=sign, w_in_layout=w_in_layout,
                         w1_layout=w1_layout)
